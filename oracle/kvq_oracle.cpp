@@ -1,0 +1,558 @@
+// kvq_oracle.cpp — plain, slow CPU oracle for the asymmetric low-bit KV cache and decode attention.
+//
+// TEST INFRASTRUCTURE ONLY. Nothing in the product path may link, load or call this file; only the
+// tests, the smoke check and the CPU-baseline leg of the benchmark do. It shares no code, header,
+// table or helper with the CUDA library: every step below is written out again from its definition.
+//
+// What it computes, and the passages it follows:
+//  * Keys are quantized per channel and values per token (The Asymmetric Key-Value Cache Compression
+//    framework page, Method; KVQuant review, Method and Key idea; KV cache quantization wiki page,
+//    verification notes on the KIVI full text: key outliers sit in a few fixed channels, and per-token
+//    value quantization keeps each token's error to itself).
+//  * Keys are grouped every G tokens along the sequence; the grouped part and a full-precision
+//    residual part both enter the attention score; freshly quantized groups are appended along the
+//    token axis (KV cache quantization wiki page, verification notes, KIVI grouped/residual split).
+//  * The newest tokens stay in FP16 (framework page, In practice: a window of 32 to 128 tokens).
+//  * Optional Walsh-Hadamard rotation of keys, with the same orthogonal transform applied to the
+//    query so q.k is unchanged (framework page, Method and In practice; Dual-QK abstract on the
+//    thelatestinai listing).
+//  * Min/max scale and zero-point, round to nearest, 2 or 4 bits (KVQuant review, Problem: 2 bits
+//    give 4 levels; uniform INT4/INT3/INT2 grids in Comparison).
+//  * Decode attention is one query against every cached token (NOVA-KV abstract on the
+//    thelatestinai listing: each decoding step reads the whole cache).
+//
+// Readings where the pages are silent (each also listed in the design notes):
+//  R1  quantized length Q = G * floor(max(T - R, 0) / G); tokens [Q, T) are the FP16 residual,
+//      kept in a ring of R + G slots at slot t mod (R + G).
+//  R2  Hadamard: Sylvester order H[i][j] = (-1)^popcount(i & j), fp32 butterfly with strides
+//      1, 2, ..., 64 (pair (i, i+h) -> (a+b, a-b)), then multiply by fp32(1/sqrt(128)), then round
+//      to fp16 (keys). The query gets the same rotation in fp64 here.
+//  R3  group min/max under the IEEE total order with -0 < +0.
+//  R4  s32 = (f32(mx) - f32(mn)) / f32(2^b - 1); s16 = fp16_rn(s32); zero = mn (fp16).
+//  R5  s16 == 0 -> all codes 0; else inv = 1 / f32(s16),
+//      code = clamp(rint_half_even((f32(x) - f32(mn)) * inv), 0, 2^b - 1), each op one IEEE fp32
+//      rounding, never fused.
+//  R6  dequant x^ = code * s16 + zero, evaluated here in fp64.
+//  R7  attention in fp64: no causal mask, no sink token, no RoPE; softmax over all T tokens.
+//  R8  packed layout "tile v1" (see key_word_bit / value_word_bit / key_param_pos below).
+//
+// Build: g++ -O2 -std=c++17 -ffp-contract=off -fno-fast-math -fPIC -shared (x86-64 SSE scalar fp32).
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+#include <algorithm>
+
+namespace {
+
+// ------------------------------------------------------------------------------------------------
+// IEEE 754 binary16 <-> binary32, written from the format definition (1 sign, 5 exponent bits with
+// bias 15, 10 fraction bits; subnormals have value fraction * 2^-24).
+// ------------------------------------------------------------------------------------------------
+float half_to_float(uint16_t h) {
+  const uint32_t sign = h >> 15, expo = (h >> 10) & 0x1fu, frac = h & 0x3ffu;
+  float mag;
+  if (expo == 0) {
+    mag = std::ldexp(static_cast<float>(frac), -24);  // exact: frac < 2^10
+  } else if (expo == 31) {
+    mag = frac ? std::nanf("") : INFINITY;
+  } else {
+    mag = std::ldexp(static_cast<float>(frac | 0x400u), static_cast<int>(expo) - 25);  // exact
+  }
+  return sign ? -mag : mag;
+}
+
+// Round-to-nearest-even conversion of a binary32 to binary16, done on the integer significand.
+uint16_t float_to_half(float f) {
+  uint32_t x;
+  std::memcpy(&x, &f, 4);
+  const uint16_t sign = static_cast<uint16_t>((x >> 16) & 0x8000u);
+  const uint32_t ax = x & 0x7fffffffu;
+  if (ax > 0x7f800000u) return sign | 0x7e00u;  // NaN
+  if (ax == 0x7f800000u) return sign | 0x7c00u;  // infinity
+  const int e = static_cast<int>(ax >> 23) - 127;  // unbiased exponent (normal binary32)
+  uint32_t sig = (ax & 0x7fffffu) | (ax >= 0x00800000u ? 0x800000u : 0u);  // 24-bit significand
+  int e_eff = (ax >= 0x00800000u) ? e : -126;  // binary32 subnormals: value = sig * 2^-149
+  // value = sig * 2^(e_eff - 23). Target unit: fp16 normal with exponent E has ulp 2^(E-10);
+  // subnormal ulp 2^-24. Choose the ulp of the result, shift the significand to it, round.
+  int target_exp = std::max(e_eff, -14);  // exponent whose ulp we round to
+  int shift = target_exp - 10 - (e_eff - 23);  // bits to drop from sig
+  // shift >= 32 means the magnitude is below 2^-32, far under half the smallest subnormal: zero.
+  if (shift >= 32) return sign;
+  uint32_t q = sig >> shift;
+  const uint32_t rem = sig & ((1u << shift) - 1u);
+  const uint32_t half = 1u << (shift - 1);
+  if (rem > half || (rem == half && (q & 1u))) q += 1;
+  // q is the significand in units of the result ulp. Rebuild the binary16 bit pattern.
+  uint32_t out;
+  if (target_exp == -14 && q < 0x400u) {
+    out = q;  // subnormal (or zero)
+  } else {
+    // q in [2^10, 2^11] for a normal; a carry to 2^11 bumps the exponent.
+    int E = target_exp;
+    if (q >= 0x800u) { q >>= 1; E += 1; }
+    if (E > 15) return sign | 0x7c00u;  // overflow -> infinity
+    out = (static_cast<uint32_t>(E + 15) << 10) | (q & 0x3ffu);
+  }
+  return static_cast<uint16_t>(sign | out);
+}
+
+// IEEE 754-2019 minimum / maximum on non-NaN binary16, with -0 ordered below +0 (reading R3).
+inline uint32_t order_key(uint16_t h) { return (h & 0x8000u) ? (~h & 0xffffu) : (h | 0x8000u); }
+inline uint16_t hmin(uint16_t a, uint16_t b) { return order_key(b) < order_key(a) ? b : a; }
+inline uint16_t hmax(uint16_t a, uint16_t b) { return order_key(b) > order_key(a) ? b : a; }
+
+// fp32 value of 1/sqrt(128) rounded to nearest (bit pattern 0x3DB504F3).
+float inv_sqrt128_f32() {
+  const uint32_t bits = 0x3DB504F3u;
+  float f;
+  std::memcpy(&f, &bits, 4);
+  return f;
+}
+
+// Walsh-Hadamard rotation of one 128-vector in fp32 (reading R2). Stride-h butterflies in the order
+// h = 1, 2, 4, ..., 64; each pair (i, i+h) with (i & h) == 0 becomes (a + b, a - b); then every
+// entry is multiplied by fp32(1/sqrt(128)).
+void wht128_f32(float* x) {
+  for (int h = 1; h < 128; h <<= 1)
+    for (int i = 0; i < 128; ++i)
+      if ((i & h) == 0) {
+        const float a = x[i], b = x[i + h];
+        x[i] = a + b;
+        x[i + h] = a - b;
+      }
+  const float s = inv_sqrt128_f32();
+  for (int i = 0; i < 128; ++i) x[i] = x[i] * s;
+}
+
+// The same rotation in fp64 with the exact scale 1/sqrt(128) (used for the query, reading R2).
+void wht128_f64(double* x) {
+  for (int h = 1; h < 128; h <<= 1)
+    for (int i = 0; i < 128; ++i)
+      if ((i & h) == 0) {
+        const double a = x[i], b = x[i + h];
+        x[i] = a + b;
+        x[i + h] = a - b;
+      }
+  const double s = 1.0 / std::sqrt(128.0);
+  for (int i = 0; i < 128; ++i) x[i] *= s;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Asymmetric min/max quantizer of one group (readings R3-R5).
+// ------------------------------------------------------------------------------------------------
+struct GroupQ {
+  uint16_t scale, zero;
+};
+
+GroupQ quantize_group(const uint16_t* x, int n, int stride, int bits, uint8_t* codes, int code_stride) {
+  uint16_t mn = x[0], mx = x[0];
+  for (int i = 1; i < n; ++i) {
+    mn = hmin(mn, x[i * stride]);
+    mx = hmax(mx, x[i * stride]);
+  }
+  const float levels = static_cast<float>((1 << bits) - 1);
+  const float range = half_to_float(mx) - half_to_float(mn);
+  const float s32 = range / levels;
+  const uint16_t s16 = float_to_half(s32);
+  GroupQ g{s16, mn};
+  if ((s16 & 0x7fffu) == 0) {
+    for (int i = 0; i < n; ++i) codes[i * code_stride] = 0;
+    return g;
+  }
+  const float inv = 1.0f / half_to_float(s16);
+  const float zf = half_to_float(mn);
+  const int top = (1 << bits) - 1;
+  for (int i = 0; i < n; ++i) {
+    const float d = half_to_float(x[i * stride]) - zf;
+    const float v = d * inv;
+    float r = std::nearbyint(v);  // default rounding mode: nearest, ties to even
+    int c = static_cast<int>(r);
+    if (c < 0) c = 0;
+    if (c > top) c = top;
+    codes[i * code_stride] = static_cast<uint8_t>(c);
+  }
+  return g;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Packed layout "tile v1" (reading R8). The cache of one (sequence, KV head) is cut into tiles of 16
+// tokens x 128 channels. A tile holds 32 "lanes" of W = 2*bits u32 words (4 words at 2 bits, 8 at
+// 4 bits); lane L's word w sits at word (w / 4) * 128 + 4 * L + (w % 4) of the tile. Each word holds
+// P = 16 / bits code pairs: pair k has element e = 0 at bits [bits*k, bits*k + bits) and e = 1 at
+// bits [16 + bits*k, ...). Pair slot p = w * P + k names (m = p / 4, reg = p % 4, u = reg % 2,
+// h = reg / 2), and with L = 4 r + qd:
+//   keys:   token i = r + 8u,          channel c = 16m + 2qd + 8h + e
+//   values: token i = 2qd + 8h + e,    channel c = 16m + r + 8u
+// Per-group key scale and zero store channel c = 16m + 2qd + 8h + e at position 32qd + 4m + 2h + e.
+// Value scale and zero are [token][channel group] in natural order.
+// ------------------------------------------------------------------------------------------------
+inline void slot_to_word_bit(int lane, int p, int bits, int e, int* word, int* bit) {
+  const int P = 16 / bits;
+  const int w = p / P, k = p % P;
+  *word = (w / 4) * 128 + 4 * lane + (w % 4);
+  *bit = bits * k + 16 * e;
+}
+
+void key_word_bit(int i, int c, int bits, int* word, int* bit) {
+  const int r = i % 8, u = i / 8;
+  const int m = c / 16, within = c % 16;
+  const int h = within / 8, qd = (within % 8) / 2, e = within % 2;
+  const int lane = 4 * r + qd;
+  const int p = 4 * m + (u + 2 * h);
+  slot_to_word_bit(lane, p, bits, e, word, bit);
+}
+
+void value_word_bit(int i, int c, int bits, int* word, int* bit) {
+  const int m = c / 16, within = c % 16;
+  const int r = within % 8, u = within / 8;
+  const int h = i / 8, qd = (i % 8) / 2, e = i % 2;
+  const int lane = 4 * r + qd;
+  const int p = 4 * m + (u + 2 * h);
+  slot_to_word_bit(lane, p, bits, e, word, bit);
+}
+
+int key_param_pos(int c) {
+  const int m = c / 16, within = c % 16;
+  const int h = within / 8, qd = (within % 8) / 2, e = within % 2;
+  return 32 * qd + 4 * m + 2 * h + e;
+}
+
+}  // namespace
+
+// ================================================================================================
+// C interface (host pointers only).
+// ================================================================================================
+extern "C" {
+
+typedef struct {
+  int32_t batch, num_q_heads, num_kv_heads, head_dim;
+  int32_t key_bits, value_bits, group_size, residual, hadamard;
+  int64_t capacity;
+} kvq_ref_config;
+
+typedef struct {
+  uint32_t* k_codes;  // [B][Hkv][Cap/16][64*key_bits]
+  uint32_t* v_codes;  // [B][Hkv][Cap/16][64*value_bits]
+  uint16_t* k_scale;  // [B][Hkv][Cap/G][128] (permuted channel order)
+  uint16_t* k_zero;   // same
+  uint16_t* v_scale;  // [B][Hkv][Cap][128/G]
+  uint16_t* v_zero;   // same
+  uint16_t* k_res;    // [B][Hkv][R+G][128] ring, fp16
+  uint16_t* v_res;    // same
+  int64_t* seq_len;   // [B]
+} kvq_ref_cache;
+
+enum { REF_OK = 0, REF_ERR_ARG = -1, REF_ERR_CAPACITY = -3 };
+
+static int check_config(const kvq_ref_config* c) {
+  if (!c) return REF_ERR_ARG;
+  if (c->head_dim != 128) return REF_ERR_ARG;
+  if (c->batch < 0 || c->num_kv_heads <= 0 || c->num_q_heads <= 0) return REF_ERR_ARG;
+  if (c->num_q_heads % c->num_kv_heads) return REF_ERR_ARG;
+  if ((c->key_bits != 2 && c->key_bits != 4) || (c->value_bits != 2 && c->value_bits != 4)) return REF_ERR_ARG;
+  const int G = c->group_size;
+  if (G <= 0 || G % 16 || 128 % G) return REF_ERR_ARG;
+  if (c->residual < 0 || c->capacity < 0 || c->capacity % G) return REF_ERR_ARG;
+  return REF_OK;
+}
+
+static int64_t quantized_len(int64_t T, int R, int G) {
+  const int64_t over = T - R;
+  return over > 0 ? (over / G) * G : 0;
+}
+
+struct Dims {
+  int64_t kw_tile, vw_tile, tiles, groups, ring, vpt;  // words per tile, tiles/unit, groups/unit, ring slots, value groups per token
+};
+static Dims dims(const kvq_ref_config* c) {
+  Dims d;
+  d.kw_tile = 64 * c->key_bits;
+  d.vw_tile = 64 * c->value_bits;
+  d.tiles = c->capacity / 16;
+  d.groups = c->capacity / c->group_size;
+  d.ring = c->residual + c->group_size;
+  d.vpt = 128 / c->group_size;
+  return d;
+}
+
+// Quantize tokens [t0, t0 + G) of key unit `kt` (fp16 [T][128], already rotated if enabled) into key
+// group t0 / G, and the same tokens of value unit `vt` per token.
+static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t unit, int64_t t0,
+                          const uint16_t* kt, int64_t k_ld, const uint16_t* vt, int64_t v_ld) {
+  const Dims d = dims(c);
+  const int G = c->group_size;
+  // Keys: per channel over the G tokens of the group.
+  std::vector<uint8_t> kc(static_cast<size_t>(G) * 128);
+  const int64_t g = t0 / G;
+  for (int ch = 0; ch < 128; ++ch) {
+    GroupQ q = quantize_group(kt + ch, G, static_cast<int>(k_ld), c->key_bits, kc.data() + ch, 128);
+    const int pos = key_param_pos(ch);
+    cache->k_scale[(unit * d.groups + g) * 128 + pos] = q.scale;
+    cache->k_zero[(unit * d.groups + g) * 128 + pos] = q.zero;
+  }
+  for (int i = 0; i < G; ++i) {
+    const int64_t t = t0 + i;
+    uint32_t* tile = cache->k_codes + (unit * d.tiles + t / 16) * d.kw_tile;
+    for (int ch = 0; ch < 128; ++ch) {
+      int word, bit;
+      key_word_bit(static_cast<int>(t % 16), ch, c->key_bits, &word, &bit);
+      const uint32_t mask = ((1u << c->key_bits) - 1u) << bit;
+      tile[word] = (tile[word] & ~mask) | (static_cast<uint32_t>(kc[i * 128 + ch]) << bit);
+    }
+  }
+  // Values: per token over channel groups of G.
+  std::vector<uint8_t> vc(128);
+  for (int i = 0; i < G; ++i) {
+    const int64_t t = t0 + i;
+    for (int j = 0; j < d.vpt; ++j) {
+      GroupQ q = quantize_group(vt + i * v_ld + j * G, G, 1, c->value_bits, vc.data() + j * G, 1);
+      cache->v_scale[(unit * c->capacity + t) * d.vpt + j] = q.scale;
+      cache->v_zero[(unit * c->capacity + t) * d.vpt + j] = q.zero;
+    }
+    uint32_t* tile = cache->v_codes + (unit * d.tiles + t / 16) * d.vw_tile;
+    for (int ch = 0; ch < 128; ++ch) {
+      int word, bit;
+      value_word_bit(static_cast<int>(t % 16), ch, c->value_bits, &word, &bit);
+      const uint32_t mask = ((1u << c->value_bits) - 1u) << bit;
+      tile[word] = (tile[word] & ~mask) | (static_cast<uint32_t>(vc[ch]) << bit);
+    }
+  }
+}
+
+static void rotate_key_f16(const uint16_t* in, uint16_t* out) {
+  float x[128];
+  for (int i = 0; i < 128; ++i) x[i] = half_to_float(in[i]);
+  wht128_f32(x);
+  for (int i = 0; i < 128; ++i) out[i] = float_to_half(x[i]);
+}
+
+static void prefill_unit(const kvq_ref_config* c, kvq_ref_cache* cache, const uint16_t* k, const uint16_t* v,
+                         int64_t sb, int64_t st, int64_t sh, int64_t b, int64_t kvh, int64_t T) {
+  const Dims d = dims(c);
+  const int G = c->group_size;
+  const int64_t unit = b * c->num_kv_heads + kvh;
+  const int64_t Q = quantized_len(T, c->residual, G);
+  // Gather this unit's tokens into contiguous [T][128] (keys rotated when enabled).
+  std::vector<uint16_t> kt(static_cast<size_t>(T) * 128), vt(static_cast<size_t>(T) * 128);
+  for (int64_t t = 0; t < T; ++t) {
+    const uint16_t* ks = k + b * sb + t * st + kvh * sh;
+    const uint16_t* vs = v + b * sb + t * st + kvh * sh;
+    if (c->hadamard)
+      rotate_key_f16(ks, &kt[t * 128]);
+    else
+      std::memcpy(&kt[t * 128], ks, 256);
+    std::memcpy(&vt[t * 128], vs, 256);
+  }
+  for (int64_t t0 = 0; t0 < Q; t0 += G) quantize_span(c, cache, unit, t0, &kt[t0 * 128], 128, &vt[t0 * 128], 128);
+  for (int64_t t = Q; t < T; ++t) {
+    const int64_t slot = t % d.ring;
+    std::memcpy(cache->k_res + (unit * d.ring + slot) * 128, &kt[t * 128], 256);
+    std::memcpy(cache->v_res + (unit * d.ring + slot) * 128, &vt[t * 128], 256);
+  }
+}
+
+// Prefill: quantize the first Q_b tokens of every (sequence, KV head) and keep [Q_b, T_b) in FP16.
+// k, v: fp16 [b][t][h][d] with element strides (sb, st, sh); d contiguous.
+int kvq_ref_quantize_prefill(const kvq_ref_config* c, kvq_ref_cache* cache, const uint16_t* k, const uint16_t* v,
+                             int64_t sb, int64_t st, int64_t sh, const int64_t* seq_lens, int nthreads) {
+  int rc = check_config(c);
+  if (rc) return rc;
+  for (int b = 0; b < c->batch; ++b)
+    if (seq_lens[b] < 0 || seq_lens[b] > c->capacity) return REF_ERR_CAPACITY;
+  const int64_t units = static_cast<int64_t>(c->batch) * c->num_kv_heads;
+  auto work = [&](int64_t u0, int64_t step) {
+    for (int64_t u = u0; u < units; u += step) {
+      const int64_t b = u / c->num_kv_heads, h = u % c->num_kv_heads;
+      prefill_unit(c, cache, k, v, sb, st, sh, b, h, seq_lens[b]);
+    }
+  };
+  if (nthreads <= 1) {
+    work(0, 1);
+  } else {
+    std::vector<std::thread> pool;
+    for (int i = 0; i < nthreads; ++i) pool.emplace_back(work, i, nthreads);
+    for (auto& t : pool) t.join();
+  }
+  for (int b = 0; b < c->batch; ++b) cache->seq_len[b] = seq_lens[b];
+  return REF_OK;
+}
+
+// Append one token to every sequence; flush a key/value group when the residual window has grown
+// past R by a whole group. k_new, v_new: fp16 [B][Hkv][128].
+int kvq_ref_append_token(const kvq_ref_config* c, kvq_ref_cache* cache, const uint16_t* k_new, const uint16_t* v_new) {
+  int rc = check_config(c);
+  if (rc) return rc;
+  const Dims d = dims(c);
+  const int G = c->group_size;
+  for (int b = 0; b < c->batch; ++b)
+    if (cache->seq_len[b] + 1 > c->capacity) return REF_ERR_CAPACITY;
+  for (int b = 0; b < c->batch; ++b) {
+    const int64_t t = cache->seq_len[b];
+    const int64_t Q_old = quantized_len(t, c->residual, G);
+    const int64_t Q_new = quantized_len(t + 1, c->residual, G);
+    for (int h = 0; h < c->num_kv_heads; ++h) {
+      const int64_t unit = static_cast<int64_t>(b) * c->num_kv_heads + h;
+      const uint16_t* ks = k_new + unit * 128;
+      const uint16_t* vs = v_new + unit * 128;
+      const int64_t slot = t % d.ring;
+      if (c->hadamard)
+        rotate_key_f16(ks, cache->k_res + (unit * d.ring + slot) * 128);
+      else
+        std::memcpy(cache->k_res + (unit * d.ring + slot) * 128, ks, 256);
+      std::memcpy(cache->v_res + (unit * d.ring + slot) * 128, vs, 256);
+      if (Q_new > Q_old) {
+        // Tokens [Q_old, Q_old + G) leave the window: gather them from the ring and quantize.
+        std::vector<uint16_t> kt(static_cast<size_t>(G) * 128), vt(static_cast<size_t>(G) * 128);
+        for (int i = 0; i < G; ++i) {
+          const int64_t s = (Q_old + i) % d.ring;
+          std::memcpy(&kt[i * 128], cache->k_res + (unit * d.ring + s) * 128, 256);
+          std::memcpy(&vt[i * 128], cache->v_res + (unit * d.ring + s) * 128, 256);
+        }
+        quantize_span(c, cache, unit, Q_old, kt.data(), 128, vt.data(), 128);
+      }
+    }
+    cache->seq_len[b] = t + 1;
+  }
+  return REF_OK;
+}
+
+// Dequantized key / value of token t (fp64, reading R6) or the FP16 residual copy.
+static void key_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t unit, int64_t t, int64_t Q, double* out) {
+  const Dims d = dims(c);
+  if (t >= Q) {
+    const uint16_t* r = cache->k_res + (unit * d.ring + t % d.ring) * 128;
+    for (int ch = 0; ch < 128; ++ch) out[ch] = half_to_float(r[ch]);
+    return;
+  }
+  const uint32_t* tile = cache->k_codes + (unit * d.tiles + t / 16) * d.kw_tile;
+  const int64_t g = t / c->group_size;
+  for (int ch = 0; ch < 128; ++ch) {
+    int word, bit;
+    key_word_bit(static_cast<int>(t % 16), ch, c->key_bits, &word, &bit);
+    const uint32_t code = (tile[word] >> bit) & ((1u << c->key_bits) - 1u);
+    const int pos = key_param_pos(ch);
+    const double s = half_to_float(cache->k_scale[(unit * d.groups + g) * 128 + pos]);
+    const double z = half_to_float(cache->k_zero[(unit * d.groups + g) * 128 + pos]);
+    out[ch] = static_cast<double>(code) * s + z;
+  }
+}
+
+static void value_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t unit, int64_t t, int64_t Q, double* out) {
+  const Dims d = dims(c);
+  if (t >= Q) {
+    const uint16_t* r = cache->v_res + (unit * d.ring + t % d.ring) * 128;
+    for (int ch = 0; ch < 128; ++ch) out[ch] = half_to_float(r[ch]);
+    return;
+  }
+  const uint32_t* tile = cache->v_codes + (unit * d.tiles + t / 16) * d.vw_tile;
+  for (int ch = 0; ch < 128; ++ch) {
+    int word, bit;
+    value_word_bit(static_cast<int>(t % 16), ch, c->value_bits, &word, &bit);
+    const uint32_t code = (tile[word] >> bit) & ((1u << c->value_bits) - 1u);
+    const int j = ch / c->group_size;
+    const double s = half_to_float(cache->v_scale[(unit * c->capacity + t) * d.vpt + j]);
+    const double z = half_to_float(cache->v_zero[(unit * c->capacity + t) * d.vpt + j]);
+    out[ch] = static_cast<double>(code) * s + z;
+  }
+}
+
+// Exact attention of query head h of sequence b over the dequantized cache (reading R7).
+static void decode_head(const kvq_ref_config* c, const kvq_ref_cache* cache, const uint16_t* q, double sm_scale,
+                        int64_t b, int64_t h, double* out) {
+  const int64_t gq = c->num_q_heads / c->num_kv_heads;
+  const int64_t kvh = h / gq;
+  const int64_t unit = b * c->num_kv_heads + kvh;
+  const int64_t T = cache->seq_len[b];
+  const int64_t Q = quantized_len(T, c->residual, c->group_size);
+  double qv[128];
+  const uint16_t* qs = q + (b * c->num_q_heads + h) * 128;
+  for (int i = 0; i < 128; ++i) qv[i] = half_to_float(qs[i]);
+  if (c->hadamard) wht128_f64(qv);
+  std::vector<double> s(static_cast<size_t>(T));
+  double row[128];
+  double mx = -INFINITY;
+  for (int64_t t = 0; t < T; ++t) {
+    key_row(c, cache, unit, t, Q, row);
+    double acc = 0.0;
+    for (int i = 0; i < 128; ++i) acc += qv[i] * row[i];
+    s[t] = sm_scale * acc;
+    mx = std::max(mx, s[t]);
+  }
+  double o[128] = {0};
+  double l = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    const double p = std::exp(s[t] - mx);
+    l += p;
+    value_row(c, cache, unit, t, Q, row);
+    for (int i = 0; i < 128; ++i) o[i] += p * row[i];
+  }
+  for (int i = 0; i < 128; ++i) out[i] = T > 0 ? o[i] / l : 0.0;
+}
+
+// Decode attention for every (sequence, query head). q: fp16 [B][Hq][128]; out: fp64 [B][Hq][128].
+int kvq_ref_decode(const kvq_ref_config* c, const kvq_ref_cache* cache, const uint16_t* q, double sm_scale,
+                   double* out, int nthreads) {
+  int rc = check_config(c);
+  if (rc) return rc;
+  const int64_t rows = static_cast<int64_t>(c->batch) * c->num_q_heads;
+  auto work = [&](int64_t r0, int64_t step) {
+    for (int64_t r = r0; r < rows; r += step)
+      decode_head(c, cache, q, sm_scale, r / c->num_q_heads, r % c->num_q_heads, out + r * 128);
+  };
+  if (nthreads <= 1) {
+    work(0, 1);
+  } else {
+    std::vector<std::thread> pool;
+    for (int i = 0; i < nthreads; ++i) pool.emplace_back(work, i, nthreads);
+    for (auto& t : pool) t.join();
+  }
+  return REF_OK;
+}
+
+// ---- single-step helpers exposed for the oracle's own pins --------------------------------------
+void kvq_ref_f16_to_f32(const uint16_t* in, float* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = half_to_float(in[i]);
+}
+void kvq_ref_f32_to_f16(const float* in, uint16_t* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = float_to_half(in[i]);
+}
+void kvq_ref_wht128_f32(float* x) { wht128_f32(x); }
+void kvq_ref_wht128_f64(double* x) { wht128_f64(x); }
+void kvq_ref_quantize_group(const uint16_t* x, int n, int bits, uint8_t* codes, uint16_t* scale, uint16_t* zero) {
+  GroupQ g = quantize_group(x, n, 1, bits, codes, 1);
+  *scale = g.scale;
+  *zero = g.zero;
+}
+void kvq_ref_key_word_bit(int i, int c, int bits, int* word, int* bit) { key_word_bit(i, c, bits, word, bit); }
+void kvq_ref_value_word_bit(int i, int c, int bits, int* word, int* bit) { value_word_bit(i, c, bits, word, bit); }
+int kvq_ref_key_param_pos(int c) { return key_param_pos(c); }
+int64_t kvq_ref_quantized_len(int64_t T, int R, int G) { return quantized_len(T, R, G); }
+
+// Exhaustive check of the binary32 -> binary16 converter against the compiler's _Float16 conversion
+// (round to nearest even) over every bit pattern in [lo, hi). Returns the number of mismatches
+// (NaNs compare as "both NaN").
+int64_t kvq_ref_check_f32_to_f16_range(uint64_t lo, uint64_t hi) {
+  int64_t bad = 0;
+  for (uint64_t u = lo; u < hi; ++u) {
+    const uint32_t bits = static_cast<uint32_t>(u);
+    float f;
+    std::memcpy(&f, &bits, 4);
+    const uint16_t mine = float_to_half(f);
+    const _Float16 ref = static_cast<_Float16>(f);
+    uint16_t rb;
+    std::memcpy(&rb, &ref, 2);
+    const bool mine_nan = (mine & 0x7c00u) == 0x7c00u && (mine & 0x3ffu);
+    const bool ref_nan = (rb & 0x7c00u) == 0x7c00u && (rb & 0x3ffu);
+    if (mine_nan || ref_nan) {
+      bad += (mine_nan != ref_nan);
+    } else {
+      bad += (mine != rb);
+    }
+  }
+  return bad;
+}
+
+}  // extern "C"

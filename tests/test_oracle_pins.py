@@ -1,0 +1,445 @@
+"""Pins for the CPU oracle: every check here compares the oracle with something other than itself —
+library routines (numpy's IEEE half conversion, scipy's Sylvester Hadamard matrix, torch's
+scaled-dot-product attention), closed forms, hand-worked fixtures under ``tests/golden``, invariants
+the method fixes (codes in range, error within half a step, streaming == bulk) and brute force.
+
+Passages: per-channel keys / per-token values and the min/max grid (KVQuant review, Method and
+Problem; KV cache quantization wiki page, KIVI notes), FP16 recent window (Asymmetric KV Cache
+Compression framework page, In practice), grouped/residual split and token-axis append (wiki page,
+KIVI notes), Hadamard rotation shared by keys and query (framework page, Method; Dual-QK abstract).
+"""
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------------------------------------
+# fp16 conversion
+# --------------------------------------------------------------------------------------------------
+def test_f16_to_f32_exhaustive(oracle_mod):
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mine = oracle_mod.f16_to_f32(h)
+    ref = h.view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan)
+    assert np.array_equal(mine[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_f32_to_f16_exhaustive_vs_compiler(oracle_mod):
+    # Every binary32 bit pattern against the compiler's _Float16 conversion (round to nearest even).
+    n = 1 << 32
+    chunks = 64
+    step = n // chunks
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+        bad = sum(ex.map(lambda i: oracle_mod.check_f32_to_f16_range(i * step, (i + 1) * step), range(chunks)))
+    assert bad == 0
+
+
+def test_f32_to_f16_sample_vs_numpy(oracle_mod):
+    rng = np.random.default_rng(0)
+    bits = rng.integers(0, 1 << 32, size=1 << 20, dtype=np.uint64).astype(np.uint32)
+    f = bits.view(np.float32)
+    f = f[~np.isnan(f)]
+    # ties and the subnormal / overflow edges explicitly
+    edges = np.array([65504, 65519.996, 65520, 2.0 ** -24, 2.0 ** -25, 1.5 * 2.0 ** -25, 2.0 ** -14,
+                      (1 - 2.0 ** -11) * 2.0 ** -14, 1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, -0.0, 0.0],
+                     np.float32)
+    f = np.concatenate([f, edges, -edges])
+    with np.errstate(over="ignore"):
+        ref = f.astype(np.float16).view(np.uint16)
+    assert np.array_equal(oracle_mod.f32_to_f16(f), ref)
+
+
+# --------------------------------------------------------------------------------------------------
+# Walsh-Hadamard rotation (framework page, Method / In practice; Dual-QK abstract)
+# --------------------------------------------------------------------------------------------------
+def test_wht_f64_columns_match_sylvester_hadamard(oracle_mod):
+    H = scipy.linalg.hadamard(128).astype(np.float64) / math.sqrt(128.0)
+    for i in range(128):
+        e = np.zeros(128)
+        e[i] = 1.0
+        np.testing.assert_allclose(oracle_mod.wht128_f64(e), H[:, i], rtol=0, atol=1e-15)
+
+
+def test_wht_is_orthogonal_and_preserves_dot(oracle_mod):
+    rng = np.random.default_rng(1)
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+    Hq, Hk = oracle_mod.wht128_f64(q), oracle_mod.wht128_f64(k)
+    assert abs(Hq @ Hk - q @ k) < 1e-12 * (np.abs(q) @ np.abs(k))
+    # applying it twice gives the identity (H symmetric and orthonormal after scaling)
+    np.testing.assert_allclose(oracle_mod.wht128_f64(Hq), q, atol=1e-13)
+
+
+def test_wht_f32_scale_constant_and_accuracy(oracle_mod):
+    e0 = np.zeros(128, np.float32)
+    e0[0] = 1.0
+    y = oracle_mod.wht128_f32(e0)
+    want = np.float32(1.0 / math.sqrt(128.0))
+    assert want.view(np.uint32) == 0x3DB504F3
+    assert np.all(y.view(np.uint32) == 0x3DB504F3)
+    H = scipy.linalg.hadamard(128).astype(np.float64) / math.sqrt(128.0)
+    rng = np.random.default_rng(2)
+    for _ in range(50):
+        x = (rng.standard_normal(128) * rng.choice([1, 20], 128)).astype(np.float16).astype(np.float32)
+        exact = H @ x.astype(np.float64)
+        got = oracle_mod.wht128_f32(x).astype(np.float64)
+        # 7 rounded adds on partial sums bounded by sum|x|, then one rounded multiply
+        bound = 8 * 2.0 ** -24 * np.abs(x).sum() / math.sqrt(128.0) + 1e-30
+        assert np.max(np.abs(got - exact)) <= bound
+
+
+# --------------------------------------------------------------------------------------------------
+# min/max quantizer of one group (KVQuant review, Problem; wiki page, KIVI notes)
+# --------------------------------------------------------------------------------------------------
+def _random_groups(rng, n_groups, G):
+    out = []
+    for i in range(n_groups):
+        kind = i % 5
+        if kind == 0:
+            x = rng.standard_normal(G)
+        elif kind == 1:
+            x = rng.standard_normal(G) * 20
+        elif kind == 2:
+            x = rng.standard_normal(G) * 1e-3 + 3.0
+        elif kind == 3:
+            x = rng.uniform(-60000, 60000, G)
+        else:
+            x = rng.standard_normal(G) * 1e-6  # subnormal-scale ranges
+        out.append(x.astype(np.float16))
+    return out
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("G", [16, 32, 64, 128])
+def test_quantizer_invariants(oracle_mod, bits, G):
+    rng = np.random.default_rng(bits * 1000 + G)
+    top = (1 << bits) - 1
+    for x in _random_groups(rng, 200, G):
+        codes, s16, z16 = oracle_mod.quantize_group(x, bits)
+        xf = x.astype(np.float64)
+        # the zero point is the group minimum, the scale is the step of a uniform grid over [min, max]
+        assert np.float16(np.uint16(z16).view(np.float16)) == x.min()
+        s = float(np.uint16(s16).view(np.float16))
+        z = float(np.uint16(z16).view(np.float16))
+        exact_step = (float(x.max()) - float(x.min())) / top
+        # fp32 subtraction + division (2 roundings) then fp16 rounding (half an fp16 ulp, 2^-25 abs floor)
+        assert abs(s - exact_step) <= 2.0 ** -11 * exact_step + 2.0 ** -25 + 4 * 2.0 ** -24 * exact_step
+        assert codes.min() >= 0 and codes.max() <= top
+        xh = codes.astype(np.float64) * s + z
+        err = np.abs(xf - xh)
+        if s == 0.0:
+            assert np.all(codes == 0)
+            assert np.all(err <= float(x.max()) - float(x.min()))
+            continue
+        bound = s / 2 + top * abs(exact_step - s) + 2.0 ** -20 * np.abs(xf) + 2.0 ** -20 * s
+        assert np.all(err <= bound)
+        # brute force: the chosen level is the nearest one (up to fp32 rounding of (x - z) / s)
+        levels = np.arange(top + 1)[None, :] * s + z
+        d = np.abs(xf[:, None] - levels)
+        best = d.min(axis=1)
+        chosen = d[np.arange(G), codes]
+        assert np.all(chosen <= best + 2.0 ** -20 * (np.abs(xf) + s))
+
+
+def test_quantizer_constant_group(oracle_mod):
+    for val in [0.0, 1.5, -3.25, 65504.0, 2.0 ** -24]:
+        x = np.full(32, val, np.float16)
+        codes, s16, z16 = oracle_mod.quantize_group(x, 2)
+        assert s16 == 0 and np.all(codes == 0)
+        assert np.uint16(z16).view(np.float16) == np.float16(val)
+
+
+def test_quantizer_signed_zero_minimum(oracle_mod):
+    # IEEE minimum/maximum order -0 below +0: a group of +0 and -0 has zero = -0 and max = +0.
+    x = np.array([0.0, -0.0] * 16, np.float16)
+    codes, s16, z16 = oracle_mod.quantize_group(x, 2)
+    assert z16 == 0x8000 and s16 == 0 and np.all(codes == 0)
+    x = np.array([0.0, 1.5, -0.0] + [0.5] * 29, np.float16)
+    codes, s16, z16 = oracle_mod.quantize_group(x, 2)
+    assert z16 == 0x8000 and np.uint16(s16).view(np.float16) == np.float16(0.5)
+    assert list(codes[:3]) == [0, 3, 0]
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_quantizer_two_valued_and_grid_round_trip(oracle_mod, bits):
+    top = (1 << bits) - 1
+    rng = np.random.default_rng(3)
+    # {min, max} only, with a step that fp16 represents exactly: codes are 0 and top, exact recon
+    x = np.where(rng.random(32) < 0.5, -1.0, -1.0 + top * 0.25).astype(np.float16)
+    x[0], x[1] = -1.0, -1.0 + top * 0.25
+    codes, s16, z16 = oracle_mod.quantize_group(x, bits)
+    assert set(codes.tolist()) == {0, top}
+    s, z = float(np.uint16(s16).view(np.float16)), float(np.uint16(z16).view(np.float16))
+    np.testing.assert_array_equal(codes * s + z, x.astype(np.float64))
+    # inputs on a power-of-two grid round-trip exactly
+    c = rng.integers(0, top + 1, 64)
+    c[0], c[1] = 0, top
+    x = (c * 0.125 - 1.5).astype(np.float16)
+    codes, s16, z16 = oracle_mod.quantize_group(x, bits)
+    np.testing.assert_array_equal(codes, c)
+
+
+def test_quantizer_half_way_ties_go_to_even(oracle_mod):
+    # min 0, max 3 -> step 1; x = 0.5, 1.5, 2.5 sit exactly half-way and round to the even level.
+    x = np.array([0.0, 3.0, 0.5, 1.5, 2.5] + [1.0] * 27, np.float16)
+    codes, s16, z16 = oracle_mod.quantize_group(x, 2)
+    assert np.uint16(s16).view(np.float16) == np.float16(1.0)
+    assert list(codes[:5]) == [0, 3, 0, 2, 2]
+
+
+# --------------------------------------------------------------------------------------------------
+# packed layout (hand-worked fixture)
+# --------------------------------------------------------------------------------------------------
+def _golden_layout():
+    rows = []
+    with open(os.path.join(GOLDEN, "layout_examples.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def test_layout_matches_hand_worked_examples(oracle_mod):
+    rows = _golden_layout()
+    assert len(rows) > 20
+    for r in rows:
+        if r[0] == "kparam":
+            assert oracle_mod.key_param_pos(int(r[1])) == int(r[2]), r
+            continue
+        kind, bits, i, c, word, bit = r[0], int(r[1]), int(r[2]), int(r[3]), int(r[4]), int(r[5])
+        fn = oracle_mod.key_word_bit if kind == "key" else oracle_mod.value_word_bit
+        assert fn(i, c, bits) == (word, bit), r
+
+
+@pytest.mark.parametrize("kind", ["key", "value"])
+@pytest.mark.parametrize("bits", [2, 4])
+def test_layout_is_a_bijection_onto_the_tile(oracle_mod, kind, bits):
+    fn = oracle_mod.key_word_bit if kind == "key" else oracle_mod.value_word_bit
+    used = np.zeros(64 * bits * 32, np.int32)  # one counter per bit of the tile
+    for i in range(16):
+        for c in range(128):
+            w, b = fn(i, c, bits)
+            assert 0 <= w < 64 * bits and b % bits == 0 and b + bits <= 32
+            used[w * 32 + b: w * 32 + b + bits] += 1
+    assert np.all(used == 1)
+    pos = sorted(oracle_mod.key_param_pos(c) for c in range(128))
+    assert pos == list(range(128))
+
+
+# --------------------------------------------------------------------------------------------------
+# whole-cache behaviour
+# --------------------------------------------------------------------------------------------------
+def _cfg(oracle_mod, B=2, Hq=4, Hkv=2, kb=2, vb=2, G=32, R=32, had=0, cap=512):
+    return oracle_mod.Config(B, Hq, Hkv, kb, vb, G, R, had, cap)
+
+
+def _inputs(B, T, Hkv, Hq, seed, outliers=True):
+    g = torch.Generator().manual_seed(seed)
+    k = torch.randn(B, T, Hkv, 128, generator=g)
+    if outliers:
+        k[..., 5] *= 20
+        k[..., 77] *= 15
+    v = torch.randn(B, T, Hkv, 128, generator=g)
+    q = torch.randn(B, Hq, 128, generator=g)
+    return k.half().numpy(), v.half().numpy(), q.half().numpy()
+
+
+def _unpack_key(oracle_mod, cfg, cache, b, h, t):
+    """Dequantize key (b, h, t) from the cache by reading the layout positions the fixture pins."""
+    G = cfg.group_size
+    tile = cache.k_codes[b, h, t // 16]
+    s = cache.k_scale[b, h, t // G].view(np.float16).astype(np.float64)
+    z = cache.k_zero[b, h, t // G].view(np.float16).astype(np.float64)
+    out = np.empty(128)
+    for c in range(128):
+        w, bit = oracle_mod.key_word_bit(t % 16, c, cfg.key_bits)
+        code = (int(tile[w]) >> bit) & ((1 << cfg.key_bits) - 1)
+        p = oracle_mod.key_param_pos(c)
+        out[c] = code * s[p] + z[p]
+    return out
+
+
+def _unpack_value(oracle_mod, cfg, cache, b, h, t):
+    G = cfg.group_size
+    tile = cache.v_codes[b, h, t // 16]
+    s = cache.v_scale[b, h, t].view(np.float16).astype(np.float64)
+    z = cache.v_zero[b, h, t].view(np.float16).astype(np.float64)
+    out = np.empty(128)
+    for c in range(128):
+        w, bit = oracle_mod.value_word_bit(t % 16, c, cfg.value_bits)
+        code = (int(tile[w]) >> bit) & ((1 << cfg.value_bits) - 1)
+        out[c] = code * s[c // G] + z[c // G]
+    return out
+
+
+def _sdpa(q, k, v, scale):
+    """torch's scaled-dot-product attention in fp64. q [B][Hq][D], k/v [B][Hkv][T][D] -> [B][Hq][D]."""
+    Hq, Hkv = q.shape[1], k.shape[1]
+    kk = torch.from_numpy(k).repeat_interleave(Hq // Hkv, dim=1)
+    vv = torch.from_numpy(v).repeat_interleave(Hq // Hkv, dim=1)
+    qq = torch.from_numpy(q)[:, :, None, :]
+    o = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=scale)
+    return o[:, :, 0, :].numpy()
+
+
+def test_no_quantization_equals_library_attention(oracle_mod):
+    # With R >= T nothing is quantized: the oracle must equal plain softmax attention (GQA 2:1).
+    B, T, Hkv, Hq = 2, 200, 2, 4
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, R=256, cap=512)
+    k, v, q = _inputs(B, T, Hkv, Hq, 11)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [T, T - 57])
+    out = oracle_mod.decode(cfg, cache, q, 1 / math.sqrt(128))
+    for b, Tb in enumerate([T, T - 57]):
+        kb = k[b, :Tb].astype(np.float64).transpose(1, 0, 2)[None]
+        vb = v[b, :Tb].astype(np.float64).transpose(1, 0, 2)[None]
+        ref = _sdpa(q[b:b + 1].astype(np.float64), kb, vb, 1 / math.sqrt(128))
+        np.testing.assert_allclose(out[b], ref[0], rtol=1e-12, atol=1e-13)
+
+
+def test_hadamard_no_quantization_equals_rotated_attention(oracle_mod):
+    # Keys are stored rotated (and rounded to fp16); the query is rotated by the same orthonormal H.
+    B, T, Hkv, Hq = 1, 96, 1, 2
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, R=128, had=1, cap=256)
+    k, v, q = _inputs(B, T, Hkv, Hq, 12)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [T])
+    out = oracle_mod.decode(cfg, cache, q, 0.1)
+    H = scipy.linalg.hadamard(128).astype(np.float64) / math.sqrt(128.0)
+    ring = cfg.residual + cfg.group_size
+    krot = np.stack([cache.k_res[0, 0, t % ring].view(np.float16).astype(np.float64) for t in range(T)])
+    # the stored keys are the fp16 rounding of H k (within one fp16 rounding of the exact rotation)
+    exact = k[0, :, 0].astype(np.float64) @ H.T
+    assert np.all(np.abs(krot - exact) <= np.abs(exact) * 2.0 ** -10 + 2.0 ** -23)
+    qrot = q.astype(np.float64) @ H.T
+    ref = _sdpa(qrot, krot[None, None], v[0, :, 0].astype(np.float64)[None, None], 0.1)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-13)
+    # and q.k is preserved by the rotation: attention on unrotated keys differs only by fp16 rounding
+    ref_unrot = _sdpa(q.astype(np.float64), k[0, :, 0].astype(np.float64)[None, None],
+                      v[0, :, 0].astype(np.float64)[None, None], 0.1)
+    np.testing.assert_allclose(out, ref_unrot, atol=2e-3)
+
+
+@pytest.mark.parametrize("kb,vb,G,R,had", [(2, 2, 32, 32, 0), (4, 2, 32, 0, 1), (2, 4, 64, 100, 0), (4, 4, 16, 16, 1)])
+def test_quantized_attention_equals_library_attention_on_dequantized_cache(oracle_mod, kb, vb, G, R, had):
+    B, Hkv, Hq = 2, 2, 4
+    lens = [301, 160]
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, kb, vb, G, R, had, cap=320)
+    k, v, q = _inputs(B, max(lens), Hkv, Hq, 13 + kb + G)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, lens)
+    out = oracle_mod.decode(cfg, cache, q, 1 / math.sqrt(128))
+    H = scipy.linalg.hadamard(128).astype(np.float64) / math.sqrt(128.0)
+    ring = R + G
+    for b, T in enumerate(lens):
+        Q = max(T - R, 0) // G * G
+        assert oracle_mod.quantized_len(T, R, G) == Q
+        assert T - Q <= R + G - 1 and (T < R or T - Q >= R)
+        K = np.zeros((Hkv, T, 128))
+        V = np.zeros((Hkv, T, 128))
+        for h in range(Hkv):
+            for t in range(T):
+                if t < Q:
+                    K[h, t] = _unpack_key(oracle_mod, cfg, cache, b, h, t)
+                    V[h, t] = _unpack_value(oracle_mod, cfg, cache, b, h, t)
+                else:
+                    K[h, t] = cache.k_res[b, h, t % ring].view(np.float16)
+                    V[h, t] = cache.v_res[b, h, t % ring].view(np.float16)
+        # dequantized keys stay close to the (rotated) inputs: error bounded by the group's step
+        kin = k[b, :T].astype(np.float64).transpose(1, 0, 2)
+        if had:
+            kin = kin @ H.T
+        # (per channel over each key group: at most half a step of that group's grid, plus roundings)
+        for g0 in range(0, Q, G):
+            blk = kin[:, g0:g0 + G]
+            step = (blk.max(axis=1) - blk.min(axis=1)) / ((1 << kb) - 1)
+            err = np.abs(K[:, g0:g0 + G] - blk).max(axis=1)
+            assert np.all(err <= step * (0.5 + 2.0 ** -9) + 2.0 ** -9 * np.abs(blk).max(axis=1))
+        qq = q[b:b + 1].astype(np.float64)
+        if had:
+            qq = qq @ H.T
+        ref = _sdpa(qq, K[None], V[None], 1 / math.sqrt(128))
+        np.testing.assert_allclose(out[b], ref[0], rtol=1e-11, atol=1e-12)
+
+
+def test_single_token_returns_its_value(oracle_mod):
+    cfg = _cfg(oracle_mod, 1, 2, 1, R=4, cap=64)
+    k, v, q = _inputs(1, 1, 1, 2, 14)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [1])
+    out = oracle_mod.decode(cfg, cache, q, 0.3)
+    for h in range(2):
+        np.testing.assert_array_equal(out[0, h], v[0, 0, 0].astype(np.float64))
+
+
+def test_tiny_case_against_long_double_brute_force(oracle_mod):
+    # T = 8 tokens, all quantized (R = 0, G = 16 over a 16-token capacity is not reached: use T=16).
+    cfg = _cfg(oracle_mod, 1, 1, 1, 2, 2, 16, 0, 0, cap=16)
+    k, v, q = _inputs(1, 16, 1, 1, 15)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [16])
+    out = oracle_mod.decode(cfg, cache, q, 1 / math.sqrt(128))
+    K = np.array([_unpack_key(oracle_mod, cfg, cache, 0, 0, t) for t in range(16)], np.longdouble)
+    V = np.array([_unpack_value(oracle_mod, cfg, cache, 0, 0, t) for t in range(16)], np.longdouble)
+    qq = q[0, 0].astype(np.longdouble)
+    s = (K @ qq) / np.sqrt(np.longdouble(128))
+    p = np.exp(s - s.max())
+    ref = (p[:, None] * V).sum(0) / p.sum()
+    np.testing.assert_allclose(out[0, 0], ref.astype(np.float64), rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("kb,vb,G,R,had", [(2, 2, 32, 32, 0), (4, 2, 32, 0, 1), (2, 2, 64, 128, 0), (4, 4, 16, 5, 0)])
+def test_streaming_append_equals_bulk_prefill(oracle_mod, kb, vb, G, R, had):
+    B, Hkv, Hq = 2, 2, 2
+    T0, n = 150, 3 * G + 7
+    cap = ((T0 + n + G - 1) // G) * G
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, kb, vb, G, R, had, cap=cap)
+    k, v, _ = _inputs(B, T0 + n, Hkv, Hq, 16 + G)
+    stream = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, stream, k[:, :T0], v[:, :T0], [T0, T0])
+    for t in range(T0, T0 + n):
+        oracle_mod.append_token(cfg, stream, k[:, t], v[:, t])
+    bulk = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, bulk, k, v, [T0 + n, T0 + n])
+    T = T0 + n
+    Q = max(T - R, 0) // G * G
+    assert np.array_equal(stream.seq_len, bulk.seq_len)
+    np.testing.assert_array_equal(stream.k_codes[:, :, : Q // 16], bulk.k_codes[:, :, : Q // 16])
+    np.testing.assert_array_equal(stream.v_codes[:, :, : Q // 16], bulk.v_codes[:, :, : Q // 16])
+    np.testing.assert_array_equal(stream.k_scale[:, :, : Q // G], bulk.k_scale[:, :, : Q // G])
+    np.testing.assert_array_equal(stream.k_zero[:, :, : Q // G], bulk.k_zero[:, :, : Q // G])
+    np.testing.assert_array_equal(stream.v_scale[:, :, :Q], bulk.v_scale[:, :, :Q])
+    np.testing.assert_array_equal(stream.v_zero[:, :, :Q], bulk.v_zero[:, :, :Q])
+    ring = R + G
+    live = [t % ring for t in range(Q, T)]
+    np.testing.assert_array_equal(stream.k_res[:, :, live], bulk.k_res[:, :, live])
+    np.testing.assert_array_equal(stream.v_res[:, :, live], bulk.v_res[:, :, live])
+
+
+def test_append_rejects_capacity_overflow(oracle_mod):
+    cfg = _cfg(oracle_mod, 1, 1, 1, G=16, R=0, cap=16)
+    k, v, _ = _inputs(1, 17, 1, 1, 17)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k[:, :16], v[:, :16], [16])
+    with pytest.raises(ValueError):
+        oracle_mod.append_token(cfg, cache, k[:, 16], v[:, 16])
+
+
+@pytest.mark.parametrize("bits,G", [(2, 32), (2, 64), (2, 128), (4, 32)])
+def test_average_bits_closed_form(oracle_mod, bits, G):
+    # Buffer sizes give b + 32/G bits per cached element (fp16 scale + zero shared by G elements);
+    # 2 bits at G = 32 is 3.0 bits, the size class of the KIVI-2 setting the KVQuant review quotes.
+    cfg = _cfg(oracle_mod, 1, 1, 1, bits, bits, G, 0, 0, cap=1024)
+    c = oracle_mod.Cache(cfg)
+    total_bits = 8 * (c.k_codes.nbytes + c.v_codes.nbytes + c.k_scale.nbytes + c.k_zero.nbytes
+                      + c.v_scale.nbytes + c.v_zero.nbytes)
+    per_elem = total_bits / (2 * 1024 * 128)
+    assert per_elem == bits + 32 / G
