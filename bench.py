@@ -1,0 +1,434 @@
+#!/usr/bin/env python3
+"""Benchmark: decode steps on the packed low-bit KV cache, B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl kvq|reference]
+
+One step is one serving decode step of the whole batch on the resident cache: append the new token of
+every sequence (Hadamard rotation of the key when enabled, group flush every G steps) and decode
+attention of one query per sequence over the packed cache plus the FP16 window (query prep, split-K
+attention, split combine). Prefill quantization of the full prompt (fp16 K/V -> codes, scales, window)
+is timed separately in the same run. The headline value is effective decode bandwidth: the bytes the
+method must read per step (packed codes, scales, zero-points, FP16 window, query and output) divided
+by the device time per step; inputs (> L2) are resident in HBM when timing starts.
+
+With --gpus N > 1 (torchrun) every rank runs its own replica of the workload (the path has no
+exchange step): weak scaling, value = bytes of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_kv_cache_prefill_b200 import inputs  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+L2_BYTES = 126 * 2**20
+METRIC = "decode-attn effective KV HBM GB/s (fraction of B200 peak); tokens/s"
+
+
+# ---------------------------------------------------------------------------------------------------
+# algorithmic bytes (what the method must move), per unit of work
+# ---------------------------------------------------------------------------------------------------
+def decode_bytes(w: inputs.Workload, lens: np.ndarray) -> int:
+    """Bytes one decode call must read/write: packed codes + key group scale/zero + value token
+    scale/zero for the quantized tokens, fp16 K/V for the window, q in and out."""
+    G, R = w.group_size, w.residual
+    total = 0
+    for T in lens:
+        T = int(T)
+        Q = max(T - R, 0) // G * G
+        per_unit = Q * 128 * (w.key_bits + w.value_bits) // 8 + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4
+        total += w.num_kv_heads * per_unit
+    return total + 2 * w.batch * w.num_q_heads * 128 * 2
+
+
+def prefill_bytes(w: inputs.Workload, lens: np.ndarray) -> int:
+    """fp16 K and V read + codes, scales, zero-points and window written."""
+    G, R = w.group_size, w.residual
+    total = 0
+    for T in lens:
+        T = int(T)
+        Q = max(T - R, 0) // G * G
+        total += w.num_kv_heads * (T * 128 * 4 + Q * 128 * (w.key_bits + w.value_bits) // 8
+                                   + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4)
+    return total
+
+
+def append_bytes(w: inputs.Workload) -> int:
+    return 2 * w.batch * w.num_kv_heads * 128 * 2
+
+
+# ---------------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------------------------------
+def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0):
+    """Time the oracle's decode on a bounded sample of the workload: whole (sequence, KV head) units
+    batched into one oracle problem (enough units to give every host core a query head), decoded
+    repeatedly until about budget_s seconds have passed. Returns (GB/s of algorithmic decode bytes,
+    threads used, description of the sample)."""
+    import oracle as ref
+
+    cores = len(os.sched_getaffinity(0))
+    g = w.gqa
+    lens_all = w.seq_lens() + w.appends
+    units = [(b, h) for b in range(w.batch) for h in range(w.num_kv_heads)]
+    n = max(1, min(len(units), -(-cores // g)))
+    while n > 1 and n * int(lens_all.max()) > (4 << 20):  # keep the sample's host memory bounded
+        n -= 1
+    stride = max(1, len(units) // n)
+    picked = units[::stride][:n]
+    lens = np.array([int(lens_all[b]) for b, _ in picked], np.int64)
+    Tmax = int(lens.max())
+    cap = int(math.ceil(Tmax / w.group_size) * w.group_size)
+    ocfg = ref.Config(n, g, 1, w.key_bits, w.value_bits, w.group_size, w.residual, w.hadamard, cap)
+    k = np.zeros((n, Tmax, 1, 128), np.float16)
+    v = np.zeros_like(k)
+    qs = np.zeros((n, g, 128), np.float16)
+    q = inputs.query(w).numpy()
+    for i, (b, h) in enumerate(picked):
+        ku, vu = inputs.unit_kv(w, b, h, int(lens[i]))
+        k[i, : lens[i], 0] = ku.numpy()
+        v[i, : lens[i], 0] = vu.numpy()
+        qs[i] = q[b, h * g:(h + 1) * g]
+    oc = ref.Cache(ocfg)
+    ref.quantize_prefill(ocfg, oc, k, v, lens, threads=cores)
+    threads = min(cores, n * g)
+    calls, spent = 0, 0.0
+    while spent < budget_s or calls == 0:
+        t0 = time.perf_counter()
+        ref.decode(ocfg, oc, qs, 1 / math.sqrt(128), threads=threads)
+        spent += time.perf_counter() - t0
+        calls += 1
+    per_call = decode_bytes(w.scaled(batch=n, num_q_heads=g, num_kv_heads=1), lens)
+    desc = f"{n} (sequence, KV head) units of {w.name} ({int(lens.sum())} tokens), decode x{calls}"
+    return per_call * calls / spent / 1e9, threads, desc
+
+
+def run_reference(args, w):
+    """--impl reference: the CPU oracle as it stands, timed on the host cores."""
+    import oracle as ref
+
+    ref.build()
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    lens = w.seq_lens() + w.appends
+    per_step = []
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        gbs, cores, sample = oracle_decode_sample(w, budget_s=budget)
+        if i >= args.warmup:
+            per_step.append(gbs)
+    value = statistics.mean(per_step)
+    step_bytes = decode_bytes(w, lens)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_bytes / (value * 1e9) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "num_q_heads": w.num_q_heads,
+                   "num_kv_heads": w.num_kv_heads, "key_bits": w.key_bits, "value_bits": w.value_bits,
+                   "group_size": w.group_size, "residual": w.residual, "hadamard": w.hadamard},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama2_7b_mha", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--prefill-iters", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling captures)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w0 = inputs.WORKLOADS[args.workload]
+    if args.batch > 0:
+        w0 = w0.scaled(batch=args.batch)
+
+    if args.impl == "reference":
+        return run_reference(args, w0)
+
+    import bit_kv_cache_prefill_b200 as kvq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # capacity for the prefill plus every appended token of this run
+    n_app = w0.appends + args.warmup + args.steps + (1 if not args.no_e2e else 0) * (args.steps + args.warmup)
+    w = w0.scaled(appends=n_app)
+    lens0 = w0.seq_lens()
+    k, v, _ = inputs.full_kv(w0)  # CPU, seeded
+    kd, vd = k.cuda(), v.cuda()
+    del k, v
+    cfg = kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size, w.residual,
+                          w.hadamard, w.capacity())
+    cache = kvq.Cache(cfg)
+    stream = torch.cuda.current_stream()
+
+    # ---- prefill quantization, timed separately (same input each iteration)
+    pre_ms = []
+    for i in range(args.prefill_iters + 1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kvq.kvq_quantize_prefill(cfg, cache, kd, vd, lens0)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i > 0:
+            pre_ms.append(e0.elapsed_time(e1))
+    pre_bytes = prefill_bytes(w0, lens0)
+    del kd, vd
+    torch.cuda.empty_cache()
+
+    # the workload's own streaming appends (e.g. 256 new tokens per sequence) before decode
+    for s in range(w0.appends):
+        kn, vn = inputs.append_tokens(w0, s)
+        kvq.kvq_append_token(cfg, cache, kn.cuda(), vn.cuda())
+    torch.cuda.synchronize()
+
+    q = inputs.query(w0).cuda()
+    out = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float16, device="cuda")
+    ws = torch.empty(kvq.kvq_decode_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+    sm_scale = 1 / math.sqrt(128)
+    steps_tok = [inputs.append_tokens(w0, w0.appends + s) for s in range(args.warmup + args.steps)]
+    app_k = [t[0].cuda() for t in steps_tok]
+    app_v = [t[1].cuda() for t in steps_tok]
+
+    def step(i, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kvq.kvq_append_token(cfg, cache, app_k[i], app_v[i])
+        if ev is not None:
+            ev[1].record(stream)
+        kvq.kvq_decode_attention(cfg, cache, q, out, sm_scale, ws)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+    lens_before = cache.seq_len_host.copy()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_id = visible.split(",")[local] if visible else str(local)
+    with ClockSampler(gpu_id) as clocks:
+        time.sleep(0.25)
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, evs[i])
+        t_end.record(stream)
+        barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    append_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    # bytes per step from the lengths each decode actually saw (append happens first)
+    step_bytes = [decode_bytes(w0, lens_before + i + 1) for i in range(args.steps)]
+    total_bytes = float(sum(step_bytes))
+    tokens = w.batch * args.steps
+
+    # max over ranks
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        tb = torch.tensor([total_bytes, float(tokens)], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tb)
+        total_bytes, tokens = float(tb[0].item()), int(tb[1].item())
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        q_host = inputs.query(w0).pin_memory()
+        out_host = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float16).pin_memory()
+        kn_host = [t[0].pin_memory() for t in steps_tok]
+        vn_host = [t[1].pin_memory() for t in steps_tok]
+        q_dev = torch.empty_like(q)
+        kn_dev = torch.empty_like(app_k[0])
+        vn_dev = torch.empty_like(app_v[0])
+        lens_e = cache.seq_len_host.copy()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            j = (args.warmup + i) % len(kn_host)
+            kn_dev.copy_(kn_host[j], non_blocking=True)
+            vn_dev.copy_(vn_host[j], non_blocking=True)
+            q_dev.copy_(q_host, non_blocking=True)
+            kvq.kvq_append_token(cfg, cache, kn_dev, vn_dev)
+            kvq.kvq_decode_attention(cfg, cache, q_dev, out, sm_scale, ws)
+            out_host.copy_(out, non_blocking=True)
+            stream.synchronize()  # the step's result is on the host
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        e2e_bytes = float(sum(decode_bytes(w0, lens_e + i + 1) for i in range(args.steps)))
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+            e2e_bytes *= world
+        h2d = q_host.numel() * 2 + kn_host[0].numel() * 2 * 2
+        d2h = out_host.numel() * 2
+        e2e = {"value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h),
+               "tokens_per_s": round(w.batch * world * args.steps / (e2e_ms * 1e-3), 1)}
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
+    peak, peak_kind = measured_hbm_peak()
+    value = total_bytes / (total_ms * 1e-3) / 1e9
+    mean_decode_ms = statistics.mean(decode_ms)
+    achieved = statistics.mean(step_bytes) / (mean_decode_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u2/u4 codes, fp16 in/out, fp32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": w0.name, "batch": w0.batch, "seq_len": w0.seq_len, "num_q_heads": w0.num_q_heads,
+                   "num_kv_heads": w0.num_kv_heads, "key_bits": w0.key_bits, "value_bits": w0.value_bits,
+                   "group_size": w0.group_size, "residual": w0.residual, "hadamard": w0.hadamard,
+                   "ragged": bool(w0.ragged_min), "parallelism": f"replicas{args.gpus}",
+                   "l2": f"inputs larger than L2 ({step_bytes[0] / 2**20:.0f} MiB read per decode > 126 MiB)"},
+        "tokens_per_s": round(tokens / (total_ms * 1e-3), 1),
+        "frac_of_nominal_8tbs": round(value / NOMINAL_HBM_GBS, 4),
+        "decode_ms": round(mean_decode_ms, 4),
+        "append_us": round(statistics.mean(append_ms) * 1e3, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "decode_split_kernel + decode_combine_kernel (one kvq_decode_attention call)"},
+        "prefill": {"gbs": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9, 1),
+                    "ms": round(statistics.mean(pre_ms), 3), "bytes": pre_bytes},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if args.gpus == 1 and not args.no_cpu_baseline:
+        import oracle as ref
+
+        ref.build()
+        gbs, cores, sample = oracle_decode_sample(w0)
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,267 @@
+// kvq_api.cu — host side of the libkvq C ABI: argument validation, split planning and launches.
+// The entry points, their arguments and error behaviour are documented in include/kvq.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "kvq.h"
+#include "kvq_common.cuh"
+#include "kvq_internal.h"
+
+using kvq::DecodeArgs;
+using kvq::QuantizeArgs;
+
+namespace {
+
+constexpr int kMaxResidual = 4096;
+constexpr int64_t kTargetCtas = 2048;  // split budget used to bound the decode workspace
+constexpr int kSplitQuantum = 64;      // split lengths are multiples of 4 warps x 16-token tiles
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+kvq_status check_config(const kvq_config* c) {
+  if (c == nullptr) return KVQ_ERR_INVALID_ARG;
+  if (c->layout != KVQ_LAYOUT_TILE_V1) return KVQ_ERR_UNSUPPORTED;
+  if (c->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+  if (c->batch < 1 || c->num_kv_heads < 1 || c->num_q_heads < 1) return KVQ_ERR_INVALID_ARG;
+  if (c->num_q_heads % c->num_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+  if (c->num_q_heads / c->num_kv_heads > 4) return KVQ_ERR_UNSUPPORTED;
+  if ((c->key_bits != 2 && c->key_bits != 4) || (c->value_bits != 2 && c->value_bits != 4)) return KVQ_ERR_INVALID_ARG;
+  const int G = c->group_size;
+  if (G != 16 && G != 32 && G != 64 && G != 128) return KVQ_ERR_INVALID_ARG;
+  if (c->residual < 0 || c->residual > kMaxResidual) return KVQ_ERR_INVALID_ARG;
+  if (c->hadamard != 0 && c->hadamard != 1) return KVQ_ERR_INVALID_ARG;
+  if (c->capacity < 0 || c->capacity % G != 0) return KVQ_ERR_INVALID_ARG;
+  if (c->capacity > (int64_t(1) << 40)) return KVQ_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(c->batch) * c->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;  // grid.y
+  return KVQ_OK;
+}
+
+void buffer_bytes(const kvq_config* c, size_t out[KVQ_NUM_BUFFERS]) {
+  const size_t units = static_cast<size_t>(c->batch) * c->num_kv_heads;
+  const size_t cap = static_cast<size_t>(c->capacity);
+  const size_t G = static_cast<size_t>(c->group_size);
+  out[KVQ_BUF_K_CODES] = units * (cap / 16) * 64 * c->key_bits * 4;
+  out[KVQ_BUF_V_CODES] = units * (cap / 16) * 64 * c->value_bits * 4;
+  out[KVQ_BUF_K_SCALE] = units * (cap / G) * 128 * 2;
+  out[KVQ_BUF_K_ZERO] = out[KVQ_BUF_K_SCALE];
+  out[KVQ_BUF_V_SCALE] = units * cap * (128 / G) * 2;
+  out[KVQ_BUF_V_ZERO] = out[KVQ_BUF_V_SCALE];
+  out[KVQ_BUF_K_RES] = units * (static_cast<size_t>(c->residual) + G) * 128 * 2;
+  out[KVQ_BUF_V_RES] = out[KVQ_BUF_K_RES];
+}
+
+kvq_status check_cache(const kvq_config* c, const kvq_cache* k) {
+  if (k == nullptr || k->seq_len_host == nullptr || k->seq_len_dev == nullptr) return KVQ_ERR_INVALID_ARG;
+  size_t sz[KVQ_NUM_BUFFERS];
+  buffer_bytes(c, sz);
+  const void* p[KVQ_NUM_BUFFERS] = {k->k_codes, k->v_codes, k->k_scale, k->k_zero, k->v_scale, k->v_zero, k->k_res, k->v_res};
+  for (int i = 0; i < KVQ_NUM_BUFFERS; ++i) {
+    if (sz[i] == 0) continue;
+    if (p[i] == nullptr || !aligned(p[i], 16)) return KVQ_ERR_INVALID_ARG;
+  }
+  if (!aligned(k->seq_len_dev, 8)) return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
+QuantizeArgs quantize_args(const kvq_config* c, kvq_cache* k) {
+  QuantizeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.seq_len = k->seq_len_dev;
+  a.k_codes = static_cast<uint32_t*>(k->k_codes);
+  a.v_codes = static_cast<uint32_t*>(k->v_codes);
+  a.k_scale = static_cast<uint16_t*>(k->k_scale);
+  a.k_zero = static_cast<uint16_t*>(k->k_zero);
+  a.v_scale = static_cast<uint16_t*>(k->v_scale);
+  a.v_zero = static_cast<uint16_t*>(k->v_zero);
+  a.k_res = static_cast<uint16_t*>(k->k_res);
+  a.v_res = static_cast<uint16_t*>(k->v_res);
+  a.batch = c->batch;
+  a.num_kv_heads = c->num_kv_heads;
+  a.G = c->group_size;
+  a.R = c->residual;
+  a.key_bits = c->key_bits;
+  a.value_bits = c->value_bits;
+  a.hadamard = c->hadamard;
+  a.capacity = c->capacity;
+  a.tiles = c->capacity / kvq::kTile;
+  a.groups = c->capacity / c->group_size;
+  a.ring = static_cast<int64_t>(c->residual) + c->group_size;
+  return a;
+}
+
+int64_t max_splits(const kvq_config* c) {
+  const int64_t units = static_cast<int64_t>(c->batch) * c->num_kv_heads;
+  return std::max<int64_t>(1, (2 * kTargetCtas + units - 1) / units);
+}
+
+// Choose the split length: among n = 1 .. max_splits splits of the longest sequence, minimise
+// (waves of CTAs) x (tokens per CTA + a fixed per-CTA overhead), counting only CTAs that hold
+// tokens. Returns the split length; *nsplit = ceil(Tmax / L).
+int plan_splits(const kvq_config* c, const int64_t* lens, int slots, int* nsplit) {
+  int64_t tmax = 0;
+  for (int b = 0; b < c->batch; ++b) tmax = std::max(tmax, lens[b]);
+  if (tmax <= 0) {
+    *nsplit = 1;
+    return kSplitQuantum;
+  }
+  const int64_t smax = max_splits(c);
+  const double overhead = 256.0;  // tokens' worth of per-CTA fixed cost (query prep, partial write)
+  double best = 1e300;
+  int64_t best_L = 0;
+  for (int64_t n = 1; n <= smax; ++n) {
+    int64_t L = (tmax + n - 1) / n;
+    L = (L + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
+    if (n > 1 && L == best_L) continue;
+    int64_t ctas = 0;
+    for (int b = 0; b < c->batch; ++b) ctas += (lens[b] + L - 1) / L;
+    ctas *= c->num_kv_heads;
+    const double waves = std::ceil(static_cast<double>(ctas) / slots);
+    const double cost = waves * (static_cast<double>(L) + overhead);
+    if (cost < best) {
+      best = cost;
+      best_L = L;
+    }
+  }
+  *nsplit = static_cast<int>((tmax + best_L - 1) / best_L);
+  return static_cast<int>(best_L);
+}
+
+kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_cache_buffer_bytes(const kvq_config* cfg, size_t out_bytes[KVQ_NUM_BUFFERS]) {
+  const kvq_status s = check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (out_bytes == nullptr) return KVQ_ERR_INVALID_ARG;
+  buffer_bytes(cfg, out_bytes);
+  return KVQ_OK;
+}
+
+kvq_status kvq_quantize_prefill(const kvq_config* cfg, kvq_cache* cache, const void* k, const void* v, int64_t stride_b,
+                                int64_t stride_t, int64_t stride_h, const int64_t* seq_lens, void* cuda_stream) {
+  kvq_status s = check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if ((s = check_cache(cfg, cache)) != KVQ_OK) return s;
+  if (seq_lens == nullptr) return KVQ_ERR_INVALID_ARG;
+  int64_t tmax = 0;
+  for (int b = 0; b < cfg->batch; ++b) {
+    if (seq_lens[b] < 0 || seq_lens[b] > cfg->capacity) return KVQ_ERR_CAPACITY;
+    tmax = std::max(tmax, seq_lens[b]);
+  }
+  if (tmax > 0) {
+    if (k == nullptr || v == nullptr || !aligned(k, 16) || !aligned(v, 16)) return KVQ_ERR_INVALID_ARG;
+    if (stride_b < 0 || stride_t < 0 || stride_h < 0 || stride_b % 8 || stride_t % 8 || stride_h % 8) return KVQ_ERR_INVALID_ARG;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  std::memcpy(cache->seq_len_host, seq_lens, sizeof(int64_t) * cfg->batch);
+  cudaError_t e = cudaMemcpyAsync(cache->seq_len_dev, cache->seq_len_host, sizeof(int64_t) * cfg->batch,
+                                  cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  QuantizeArgs a = quantize_args(cfg, cache);
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.stride_b = stride_b;
+  a.stride_t = stride_t;
+  a.stride_h = stride_h;
+  return cuda_status(kvq::launch_prefill(a, tmax, stream));
+}
+
+kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache, const void* k_new, const void* v_new,
+                            void* cuda_stream) {
+  kvq_status s = check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if ((s = check_cache(cfg, cache)) != KVQ_OK) return s;
+  if (k_new == nullptr || v_new == nullptr || !aligned(k_new, 16) || !aligned(v_new, 16)) return KVQ_ERR_INVALID_ARG;
+  for (int b = 0; b < cfg->batch; ++b)
+    if (cache->seq_len_host[b] < 0 || cache->seq_len_host[b] + 1 > cfg->capacity) return KVQ_ERR_CAPACITY;
+  QuantizeArgs a = quantize_args(cfg, cache);
+  const kvq_status r = cuda_status(kvq::launch_append(a, static_cast<const uint16_t*>(k_new),
+                                                      static_cast<const uint16_t*>(v_new),
+                                                      static_cast<cudaStream_t>(cuda_stream)));
+  if (r == KVQ_OK)
+    for (int b = 0; b < cfg->batch; ++b) cache->seq_len_host[b] += 1;
+  return r;
+}
+
+kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, size_t* bytes) {
+  const kvq_status s = check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (bytes == nullptr) return KVQ_ERR_INVALID_ARG;
+  const int64_t units = static_cast<int64_t>(cfg->batch) * cfg->num_kv_heads;
+  const int64_t g = cfg->num_q_heads / cfg->num_kv_heads;
+  *bytes = static_cast<size_t>(units * max_splits(cfg) * g * kvq::kPartFloats) * sizeof(float);
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, const void* q, void* out, float sm_scale,
+                                void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  kvq_status s = check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if ((s = check_cache(cfg, cache)) != KVQ_OK) return s;
+  if (q == nullptr || out == nullptr || !aligned(q, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return KVQ_ERR_INVALID_ARG;
+  size_t need = 0;
+  kvq_decode_workspace_bytes(cfg, &need);
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return KVQ_ERR_WORKSPACE;
+  for (int b = 0; b < cfg->batch; ++b)
+    if (cache->seq_len_host[b] < 0 || cache->seq_len_host[b] > cfg->capacity) return KVQ_ERR_INVALID_ARG;
+
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVQ_ERR_CUDA;
+  const int occ = kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size);
+  int nsplit = 1;
+  const int L = plan_splits(cfg, cache->seq_len_host, sms * occ, &nsplit);
+
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.k_codes = static_cast<const uint32_t*>(cache->k_codes);
+  a.v_codes = static_cast<const uint32_t*>(cache->v_codes);
+  a.k_scale = static_cast<const uint16_t*>(cache->k_scale);
+  a.k_zero = static_cast<const uint16_t*>(cache->k_zero);
+  a.v_scale = static_cast<const uint16_t*>(cache->v_scale);
+  a.v_zero = static_cast<const uint16_t*>(cache->v_zero);
+  a.k_res = static_cast<const uint16_t*>(cache->k_res);
+  a.v_res = static_cast<const uint16_t*>(cache->v_res);
+  a.seq_len = cache->seq_len_dev;
+  a.q = static_cast<const uint16_t*>(q);
+  a.out = static_cast<uint16_t*>(out);
+  a.part = static_cast<float*>(workspace);
+  a.batch = cfg->batch;
+  a.num_q_heads = cfg->num_q_heads;
+  a.num_kv_heads = cfg->num_kv_heads;
+  a.gqa = cfg->num_q_heads / cfg->num_kv_heads;
+  a.G = cfg->group_size;
+  a.R = cfg->residual;
+  a.key_bits = cfg->key_bits;
+  a.value_bits = cfg->value_bits;
+  a.hadamard = cfg->hadamard;
+  a.capacity = cfg->capacity;
+  a.tiles = cfg->capacity / kvq::kTile;
+  a.groups = cfg->capacity / cfg->group_size;
+  a.ring = static_cast<int64_t>(cfg->residual) + cfg->group_size;
+  a.split_len = L;
+  a.nsplit = nsplit;
+  a.qscale = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  return cuda_status(kvq::launch_decode(a, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+const char* kvq_status_string(kvq_status status) {
+  switch (status) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "sequence would exceed the cache capacity";
+    case KVQ_ERR_WORKSPACE: return "decode workspace missing, misaligned or too small";
+    case KVQ_ERR_CUDA: return "CUDA launch or copy failed";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

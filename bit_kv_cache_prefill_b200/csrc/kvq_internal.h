@@ -1,0 +1,54 @@
+// kvq_internal.h — argument blocks passed from the C-ABI host code to the kernels (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvq {
+
+struct QuantizeArgs {
+  const uint16_t* k;  // prefill input fp16 [b][t][h][d] (strided); unused by append
+  const uint16_t* v;
+  int64_t stride_b, stride_t, stride_h;
+  int64_t* seq_len;  // device mirror [batch]
+  uint32_t* k_codes;
+  uint32_t* v_codes;
+  uint16_t* k_scale;
+  uint16_t* k_zero;
+  uint16_t* v_scale;
+  uint16_t* v_zero;
+  uint16_t* k_res;
+  uint16_t* v_res;
+  int batch, num_kv_heads, G, R, key_bits, value_bits, hadamard;
+  int64_t capacity, tiles, groups, ring;  // per unit: capacity tokens, capacity/16 tiles, capacity/G groups, R+G slots
+};
+
+struct DecodeArgs {
+  const uint32_t* k_codes;
+  const uint32_t* v_codes;
+  const uint16_t* k_scale;
+  const uint16_t* k_zero;
+  const uint16_t* v_scale;
+  const uint16_t* v_zero;
+  const uint16_t* k_res;
+  const uint16_t* v_res;
+  const int64_t* seq_len;  // device mirror [batch]
+  const uint16_t* q;       // fp16 [batch][Hq][128]
+  uint16_t* out;           // fp16 [batch][Hq][128]
+  float* part;             // split partials [units][nsplit][g][2 + 128]
+  int batch, num_q_heads, num_kv_heads, gqa, G, R, key_bits, value_bits, hadamard;
+  int64_t capacity, tiles, groups, ring;
+  int split_len;  // tokens per split (multiple of 64)
+  int nsplit;     // splits per unit in the grid
+  float qscale;   // sm_scale * log2(e): scores are kept in base-2 units
+};
+
+cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream);
+cudaError_t launch_append(const QuantizeArgs& a, const uint16_t* k_new, const uint16_t* v_new, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+int decode_ctas_per_sm(int key_bits, int value_bits, int G);
+
+constexpr int kDecodeWarps = 4;
+constexpr int kPartFloats = 2 + 128;  // m, l, o[128]
+
+}  // namespace kvq

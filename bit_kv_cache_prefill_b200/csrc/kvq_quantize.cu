@@ -1,0 +1,247 @@
+// kvq_quantize.cu — prefill quantize/pack and streaming append/flush kernels.
+//
+// Prefill (KVQuant review, Limitations and Sparks: compress many keys and values in one pass) turns
+// fp16 K/V into 2- or 4-bit codes with fp16 scale/zero per group: keys per channel over G tokens,
+// values per token over G channels (KVQuant review, Method; KV cache quantization wiki page, KIVI
+// notes). Tokens of the FP16 window (framework page, In practice) go to a ring of R + G slots.
+// Append writes one token per sequence into the ring and, once the window holds a whole group
+// beyond R, quantizes that group and appends it along the token axis (wiki page, KIVI notes).
+//
+// One CTA quantizes one G-token chunk of one (sequence, KV head) for keys (blockIdx.z == 0) or
+// values (blockIdx.z == 1). The chunk is staged in shared memory (16-byte loads, a token row is 256
+// contiguous bytes), rotated in place when the Hadamard option is on (keys), reduced to per-group
+// min/max, coded, and packed word by word in the tile v1 order so that every warp store is a
+// contiguous 512-byte run.
+#include <cuda_runtime.h>
+
+#include "kvq_common.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+
+// Shared-memory footprint of one chunk: fp16 rows [G][128] plus one code byte per element.
+static size_t chunk_smem_bytes(int G) { return static_cast<size_t>(G) * kHeadDim * 3; }
+
+// Rotate (keys, optional) the G staged rows in place: two rows per warp per step.
+__device__ void rotate_rows(uint16_t* rows, int nrows) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  for (int r0 = warp * 2; r0 < nrows; r0 += nwarps * 2) {  // r0 is warp-uniform
+    const int row = r0 + (lane >> 4);
+    const bool valid = row < nrows;
+    float x[8];
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    uint4* p = reinterpret_cast<uint4*>(rows + static_cast<size_t>(valid ? row : 0) * kHeadDim) + (lane & 15);
+    if (valid) raw = *p;
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = h2f(h[i]);
+    wht128_16lanes(x);  // all 32 lanes take part; the half-warp past the last row works on zeros
+    uint16_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = __half_as_ushort(__float2half_rn(x[i]));
+    if (valid) *p = *reinterpret_cast<const uint4*>(o);
+  }
+}
+
+// Quantize G staged key rows (tokens t0 .. t0+G-1 of `unit`) and write group t0/G.
+__device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t t0, const uint16_t* rows,
+                                    uint8_t* codes) {
+  const int G = a.G, bits = a.key_bits;
+  const int64_t g = t0 / G;
+  for (int c = threadIdx.x; c < kHeadDim; c += blockDim.x) {
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int i = 0; i < G; ++i) {
+      const uint32_t k = order_key(rows[i * kHeadDim + c]);
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+    }
+    const QuantParams p = make_params(kmin, kmax, bits);
+    const int64_t pidx = (unit * a.groups + g) * kHeadDim + key_param_pos(c);
+    a.k_scale[pidx] = p.s16;
+    a.k_zero[pidx] = p.z16;
+    for (int i = 0; i < G; ++i) codes[i * kHeadDim + c] = static_cast<uint8_t>(code_of(rows[i * kHeadDim + c], p, bits));
+  }
+  __syncthreads();
+  const int words = 64 * bits;
+  const int P = 16 / bits;
+  uint32_t* dst = a.k_codes + (unit * a.tiles + t0 / kTile) * words;
+  for (int idx = threadIdx.x; idx < (G / kTile) * words; idx += blockDim.x) {
+    const int tile = idx / words, widx = idx % words;
+    int lane, w;
+    widx_to_lane_word(widx, &lane, &w);
+    uint32_t word = 0;
+    for (int j = 0; j < P; ++j) {
+      int i, c;
+      key_slot(lane, w * P + j, &i, &c);
+      const uint8_t* cr = codes + (tile * kTile + i) * kHeadDim + c;
+      word |= static_cast<uint32_t>(cr[0]) << (bits * j);
+      word |= static_cast<uint32_t>(cr[1]) << (16 + bits * j);
+    }
+    dst[static_cast<int64_t>(tile) * words + widx] = word;
+  }
+}
+
+// Quantize G staged value rows (per token, channel groups of G) and write their codes.
+__device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64_t t0, const uint16_t* rows,
+                                      uint8_t* codes) {
+  const int G = a.G, bits = a.value_bits;
+  const int vpt = kHeadDim / G;
+  for (int item = threadIdx.x; item < G * vpt; item += blockDim.x) {
+    const int i = item / vpt, j = item % vpt;
+    const uint16_t* x = rows + i * kHeadDim + j * G;
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int c = 0; c < G; ++c) {
+      const uint32_t k = order_key(x[c]);
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+    }
+    const QuantParams p = make_params(kmin, kmax, bits);
+    const int64_t pidx = (unit * a.capacity + t0 + i) * vpt + j;
+    a.v_scale[pidx] = p.s16;
+    a.v_zero[pidx] = p.z16;
+    for (int c = 0; c < G; ++c) codes[i * kHeadDim + j * G + c] = static_cast<uint8_t>(code_of(x[c], p, bits));
+  }
+  __syncthreads();
+  const int words = 64 * bits;
+  const int P = 16 / bits;
+  uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words;
+  for (int idx = threadIdx.x; idx < (G / kTile) * words; idx += blockDim.x) {
+    const int tile = idx / words, widx = idx % words;
+    int lane, w;
+    widx_to_lane_word(widx, &lane, &w);
+    uint32_t word = 0;
+    for (int j = 0; j < P; ++j) {
+      int i, c;
+      value_slot(lane, w * P + j, &i, &c);
+      const uint8_t* cr = codes + (tile * kTile + i) * kHeadDim + c;
+      word |= static_cast<uint32_t>(cr[0]) << (bits * j);
+      word |= static_cast<uint32_t>(cr[kHeadDim]) << (16 + bits * j);
+    }
+    dst[static_cast<int64_t>(tile) * words + widx] = word;
+  }
+}
+
+__global__ void __launch_bounds__(256) prefill_kernel(QuantizeArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int64_t chunk = blockIdx.x;
+  const int64_t unit = blockIdx.y;
+  const bool is_key = blockIdx.z == 0;
+  const int64_t b = unit / a.num_kv_heads, h = unit % a.num_kv_heads;
+  const int G = a.G;
+  const int64_t T = a.seq_len[b];
+  const int64_t Q = quantized_len(T, a.R, G);
+  const int64_t t0 = chunk * G;
+  if (t0 >= T) return;
+  const int64_t n = min(static_cast<int64_t>(G), T - t0);
+  uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
+  uint8_t* codes = smem + static_cast<size_t>(G) * kHeadDim * 2;
+  const uint16_t* src = is_key ? a.k : a.v;
+  // Stage the chunk: 16 lanes per 256-byte token row.
+  for (int idx = threadIdx.x; idx < n * 16; idx += blockDim.x) {
+    const int64_t i = idx >> 4;
+    const int part = idx & 15;
+    const uint4* gp = reinterpret_cast<const uint4*>(src + b * a.stride_b + (t0 + i) * a.stride_t + h * a.stride_h) + part;
+    reinterpret_cast<uint4*>(rows + i * kHeadDim)[part] = __ldg(gp);
+  }
+  __syncthreads();
+  if (is_key && a.hadamard) {
+    rotate_rows(rows, static_cast<int>(n));
+    __syncthreads();
+  }
+  if (t0 + G <= Q) {
+    if (is_key)
+      quantize_keys_chunk(a, unit, t0, rows, codes);
+    else
+      quantize_values_chunk(a, unit, t0, rows, codes);
+    return;
+  }
+  // FP16 window: tokens [t0, t0 + n) (all >= Q because Q is a multiple of G).
+  uint16_t* ring = (is_key ? a.k_res : a.v_res) + unit * a.ring * kHeadDim;
+  for (int idx = threadIdx.x; idx < n * 16; idx += blockDim.x) {
+    const int64_t i = idx >> 4;
+    const int part = idx & 15;
+    const int64_t slot = (t0 + i) % a.ring;
+    reinterpret_cast<uint4*>(ring + slot * kHeadDim)[part] = reinterpret_cast<const uint4*>(rows + i * kHeadDim)[part];
+  }
+}
+
+// Append one token to every (sequence, KV head) and flush a full group out of the window.
+// Lengths are read from the device mirror and not modified here (bump_lengths_kernel follows).
+__global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint16_t* __restrict__ k_new,
+                                                     const uint16_t* __restrict__ v_new) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int64_t unit = blockIdx.x;
+  const bool is_key = blockIdx.y == 0;
+  const int64_t b = unit / a.num_kv_heads;
+  const int G = a.G;
+  const int64_t t = a.seq_len[b];
+  const int64_t Q_old = quantized_len(t, a.R, G);
+  const int64_t Q_new = quantized_len(t + 1, a.R, G);
+  uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
+  uint8_t* codes = smem + static_cast<size_t>(G) * kHeadDim * 2;
+  uint16_t* ring = (is_key ? a.k_res : a.v_res) + unit * a.ring * kHeadDim;
+  const uint16_t* src = (is_key ? k_new : v_new) + unit * kHeadDim;
+  // New token -> ring slot t mod (R + G), rotated first for keys when enabled (warp 0, 16 lanes).
+  if (threadIdx.x < 32) {
+    float x[8];
+    const uint4 raw = (threadIdx.x < 16) ? __ldg(reinterpret_cast<const uint4*>(src) + threadIdx.x) : make_uint4(0, 0, 0, 0);
+    const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = h2f(hv[i]);
+    if (is_key && a.hadamard) wht128_16lanes(x);
+    uint16_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = __half_as_ushort(__float2half_rn(x[i]));
+    if (threadIdx.x < 16)
+      reinterpret_cast<uint4*>(ring + (t % a.ring) * kHeadDim)[threadIdx.x] =
+          (is_key && a.hadamard) ? *reinterpret_cast<const uint4*>(o) : raw;
+  }
+  if (Q_new == Q_old) return;
+  __syncthreads();  // the new token is in the ring (it is not part of the flushed group, but keep order simple)
+  // Flush tokens [Q_old, Q_old + G): gather from the ring, quantize as one group.
+  for (int idx = threadIdx.x; idx < G * 16; idx += blockDim.x) {
+    const int i = idx >> 4, part = idx & 15;
+    const int64_t slot = (Q_old + i) % a.ring;
+    reinterpret_cast<uint4*>(rows + i * kHeadDim)[part] = reinterpret_cast<const uint4*>(ring + slot * kHeadDim)[part];
+  }
+  __syncthreads();
+  if (is_key)
+    quantize_keys_chunk(a, unit, Q_old, rows, codes);
+  else
+    quantize_values_chunk(a, unit, Q_old, rows, codes);
+}
+
+__global__ void bump_lengths_kernel(int64_t* seq_len, int batch) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < batch) seq_len[b] += 1;
+}
+
+// ---- host launchers ---------------------------------------------------------------------------------
+cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
+  if (max_len <= 0 || a.batch == 0) return cudaSuccess;
+  const size_t smem = chunk_smem_bytes(a.G);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(static_cast<unsigned>((max_len + a.G - 1) / a.G), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads), 2);
+  prefill_kernel<<<grid, 256, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const QuantizeArgs& a, const uint16_t* k_new, const uint16_t* v_new, cudaStream_t stream) {
+  const size_t smem = chunk_smem_bytes(a.G);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads), 2);
+  append_kernel<<<grid, 256, smem, stream>>>(a, k_new, v_new);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bump_lengths_kernel<<<(a.batch + 255) / 256, 256, 0, stream>>>(a.seq_len, a.batch);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -1,0 +1,181 @@
+/* kvq.h — C ABI of libkvq: asymmetric low-bit KV cache quantization and decode attention that
+ * reads the packed cache directly, for NVIDIA B200 (sm_100a).
+ *
+ * The method (passages on the source pages):
+ *   - keys are quantized per channel, values per token ("KIVI partitioning": The Asymmetric
+ *     Key-Value Cache Compression framework page, Method; KVQuant review, Method and Key idea;
+ *     KV cache quantization wiki page, verification notes on the KIVI full text);
+ *   - keys form groups of G tokens along the sequence and values groups of G channels within a
+ *     token; each group has its own min/max scale and zero-point, codes are 2 or 4 bits,
+ *     round to nearest (KVQuant review, Problem and Comparison: uniform INT grids);
+ *   - the newest tokens stay in FP16 (framework page, In practice) and a full group leaves that
+ *     window and is appended to the quantized part along the token axis (wiki page, KIVI
+ *     grouped/residual split);
+ *   - an optional 128-point Walsh-Hadamard rotation is applied to keys and, identically, to the
+ *     query (framework page, Method and In practice; Dual-QK abstract on the thelatestinai listing);
+ *   - decode attention is bandwidth-bound because every step reads the whole cache (NOVA-KV
+ *     abstract on the thelatestinai listing), so it reads the packed codes without expanding them
+ *     in memory (KVQuant review, Method: custom kernels on the compressed cache).
+ *
+ * Conventions shared by every entry point:
+ *   - Ownership: the caller allocates and frees every buffer; the library allocates nothing on the
+ *     device or host and keeps no global mutable state. All device work is enqueued on the caller's
+ *     stream (`cuda_stream` is a cudaStream_t; NULL means the legacy default stream) and runs
+ *     asynchronously; the host-side length mirror is updated before the call returns.
+ *   - Errors: every entry point returns a kvq_status and never aborts. Arguments are validated on
+ *     the host before anything is launched; on an error nothing is enqueued and the cache is left
+ *     unchanged. A failed launch is reported as KVQ_ERR_CUDA (the CUDA error is left for the caller
+ *     to inspect with cudaGetLastError).
+ *   - Inputs must be finite fp16 values (NaN / Inf are not checked on the device).
+ *   - Only head_dim == 128 is supported.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned pointer, inconsistent config */
+  KVQ_ERR_UNSUPPORTED = -2, /* a configuration this build does not implement (e.g. head_dim != 128) */
+  KVQ_ERR_CAPACITY = -3,    /* a sequence would exceed config.capacity tokens */
+  KVQ_ERR_WORKSPACE = -4,   /* workspace missing or smaller than kvq_decode_workspace_bytes */
+  KVQ_ERR_CUDA = -5         /* a kernel launch or copy failed */
+} kvq_status;
+
+/* The only packed layout of this version ("tile v1"): see kvq_cache below. */
+#define KVQ_LAYOUT_TILE_V1 1
+
+/* Problem definition. Requirements checked by every entry point:
+ *   batch >= 1; num_kv_heads >= 1; num_q_heads a multiple of num_kv_heads with
+ *   num_q_heads / num_kv_heads in {1, 2, 4}; head_dim == 128;
+ *   key_bits, value_bits in {2, 4};
+ *   group_size G in {16, 32, 64, 128} (a multiple of the 16-token tile and a divisor of 128);
+ *   residual R >= 0 (tokens kept in FP16 beyond the last full group; 0 <= R <= 4096);
+ *   hadamard in {0, 1}; layout == KVQ_LAYOUT_TILE_V1;
+ *   capacity >= 0, a multiple of G (maximum tokens per sequence). */
+typedef struct {
+  int32_t batch;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t key_bits;
+  int32_t value_bits;
+  int32_t group_size;
+  int32_t residual;
+  int32_t hadamard;
+  int32_t layout;
+  int64_t capacity;
+} kvq_config;
+
+/* The packed cache: eight caller-owned device buffers plus the sequence lengths.
+ * A "unit" is one (sequence b, KV head h); unit index u = b * num_kv_heads + h. Sizes per unit:
+ *   k_codes  u32 [capacity/16][64*key_bits]     key codes, one 16-token tile per row
+ *   v_codes  u32 [capacity/16][64*value_bits]   value codes, same tiling
+ *   k_scale  fp16 [capacity/G][128]             per key group and channel (permuted channel order)
+ *   k_zero   fp16 [capacity/G][128]             same; the zero-point is the group minimum
+ *   v_scale  fp16 [capacity][128/G]             per token and channel group
+ *   v_zero   fp16 [capacity][128/G]             same
+ *   k_res    fp16 [R+G][128]                    FP16 ring of the newest keys (rotated if hadamard)
+ *   v_res    fp16 [R+G][128]                    FP16 ring of the newest values
+ * Every buffer must be 16-byte aligned. kvq_cache_buffer_bytes gives the total sizes.
+ *
+ * Quantized length of a sequence of T tokens: Q = G * floor(max(T - R, 0) / G). Tokens [0, Q) are
+ * quantized, tokens [Q, T) live in the ring at slot t mod (R + G).
+ *
+ * Tile v1: tile row k of a unit holds tokens 16k..16k+15. Within a tile, "lane" L (0..31) owns
+ * words (w / 4) * 128 + 4L + (w % 4) for w in [0, 2*bits). Word w holds 16/bits code pairs; pair j
+ * has its first code at bits [bits*j, bits*j + bits) and its second at bits [16 + bits*j, ...).
+ * With pair slot p = w * (16/bits) + j, m = p / 4, u = p % 2, hh = (p / 2) % 2, L = 4r + qd and
+ * e in {0, 1} naming the first / second code of the pair:
+ *   keys:   token 16k + r + 8u,          channel 16m + 2qd + 8hh + e
+ *   values: token 16k + 2qd + 8hh + e,   channel 16m + r + 8u
+ * Key scale/zero entry of channel c = 16m + 2qd + 8hh + e sits at index 32qd + 4m + 2hh + e.
+ * (This order lets the decode kernel feed 16-byte loads straight into tensor-core fragments.)
+ *
+ * seq_len_host: int64 [batch] in host memory, read and updated by the library.
+ * seq_len_dev:  int64 [batch] in device memory, the device mirror, updated on the stream.
+ */
+typedef struct {
+  void* k_codes;
+  void* v_codes;
+  void* k_scale;
+  void* k_zero;
+  void* v_scale;
+  void* v_zero;
+  void* k_res;
+  void* v_res;
+  int64_t* seq_len_host;
+  int64_t* seq_len_dev;
+} kvq_cache;
+
+enum {
+  KVQ_BUF_K_CODES = 0,
+  KVQ_BUF_V_CODES = 1,
+  KVQ_BUF_K_SCALE = 2,
+  KVQ_BUF_K_ZERO = 3,
+  KVQ_BUF_V_SCALE = 4,
+  KVQ_BUF_V_ZERO = 5,
+  KVQ_BUF_K_RES = 6,
+  KVQ_BUF_V_RES = 7,
+  KVQ_NUM_BUFFERS = 8
+};
+
+/* Byte size of each of the eight cache buffers for `cfg` (all units), in kvq_cache field order.
+ * Returns KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED for a bad config or null pointers. */
+kvq_status kvq_cache_buffer_bytes(const kvq_config* cfg, size_t out_bytes[KVQ_NUM_BUFFERS]);
+
+/* Prefill: quantize whole prompts at once (KVQuant review, Limitations and Sparks: a prefill-side
+ * kernel that compresses many keys and values in one pass).
+ * k, v: device fp16, element (b, t, h, d) at b*stride_b + t*stride_t + h*stride_h + d (strides in
+ * elements, d contiguous, the same strides for k and v; rows must be 16-byte aligned, i.e. the
+ * pointers 16-byte aligned and every stride a multiple of 8). seq_lens: host int64 [batch], each in
+ * [0, capacity]. Replaces the state of every sequence: T_b := seq_lens[b]; tokens [0, Q_b) are
+ * quantized (keys rotated first when hadamard is set) and [Q_b, T_b) copied to the ring.
+ * Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY (a length above capacity),
+ * KVQ_ERR_CUDA. */
+kvq_status kvq_quantize_prefill(const kvq_config* cfg, kvq_cache* cache, const void* k, const void* v,
+                                int64_t stride_b, int64_t stride_t, int64_t stride_h, const int64_t* seq_lens,
+                                void* cuda_stream);
+
+/* Streaming append (wiki page, KIVI notes: new tokens join the FP16 window, and a window that has
+ * grown a whole group past R is quantized and appended along the token axis).
+ * k_new, v_new: device fp16 [batch][num_kv_heads][128], 16-byte aligned. Appends exactly one token
+ * to every sequence (T_b += 1) and flushes group Q_b / G of every sequence whose T_b - R reached
+ * Q_b + G. Errors: KVQ_ERR_CAPACITY if any T_b + 1 > capacity (nothing is changed), plus the
+ * generic ones. */
+kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache, const void* k_new, const void* v_new,
+                            void* cuda_stream);
+
+/* Bytes of device workspace kvq_decode_attention needs for `cfg` (an upper bound that holds for
+ * every set of sequence lengths up to capacity). */
+kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, size_t* bytes);
+
+/* Decode attention of one query token per sequence over everything cached (NOVA-KV abstract:
+ * decoding reads the whole cache each step; wiki page, KIVI notes: the grouped and the FP16
+ * residual parts both enter the scores).
+ * q: device fp16 [batch][num_q_heads][128]; out: device fp16 [batch][num_q_heads][128]
+ * (16-byte aligned). Query head h attends to KV head h / (num_q_heads / num_kv_heads) over all
+ * T_b tokens: out = softmax(sm_scale * q~ . K^) V^ with K^, V^ the dequantized cache
+ * (code * scale + zero; FP16 residual as stored) and q~ = H q / sqrt(128) when hadamard is set.
+ * A sequence with T_b == 0 gets a zero output. The caller appends the current token first.
+ * workspace: device, 256-byte aligned, at least kvq_decode_workspace_bytes(cfg) bytes; it is
+ * scratch for split partials and may be reused after the stream passes this call.
+ * Errors: KVQ_ERR_WORKSPACE, KVQ_ERR_INVALID_ARG (non-finite or non-positive sm_scale, nulls,
+ * misalignment), KVQ_ERR_CUDA. */
+kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, const void* q, void* out, float sm_scale,
+                                void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* Static description of a status code. */
+const char* kvq_status_string(kvq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

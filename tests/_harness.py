@@ -1,0 +1,125 @@
+"""Shared helpers for the tests: run one workload through the CUDA library (C ABI) and through the
+CPU oracle on the same seeded inputs, and compare."""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from bit_kv_cache_prefill_b200 import inputs
+
+MAX_ABS_TOL = 2e-3  # decode attention output, absolute
+REL_L2_TOL = 1e-3   # decode attention output, relative L2 over all compared outputs
+
+
+def oracle_config(oracle, w: inputs.Workload, batch=None, hq=None, hkv=None):
+    return oracle.Config(batch or w.batch, hq or w.num_q_heads, hkv or w.num_kv_heads, w.key_bits, w.value_bits,
+                         w.group_size, w.residual, w.hadamard, w.capacity())
+
+
+def gpu_config(w: inputs.Workload):
+    import bit_kv_cache_prefill_b200 as kvq
+
+    return kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size,
+                           w.residual, w.hadamard, w.capacity())
+
+
+@dataclass
+class GpuRun:
+    cfg: object
+    cache: object
+    out: torch.Tensor  # fp16 [B][Hq][128] on the device
+    lens: np.ndarray
+
+
+def run_gpu(w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
+            appends: int = 0, sm_scale: Optional[float] = None) -> GpuRun:
+    """Prefill (k, v on the device), `appends` streaming appends, one decode."""
+    import bit_kv_cache_prefill_b200 as kvq
+
+    cfg = gpu_config(w)
+    cache = kvq.Cache(cfg)
+    kvq.kvq_quantize_prefill(cfg, cache, k, v, lens)
+    for step in range(appends):
+        kn, vn = inputs.append_tokens(w, step)
+        kvq.kvq_append_token(cfg, cache, kn.cuda(), vn.cuda())
+    ws = torch.empty(kvq.kvq_decode_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+    out = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float16, device="cuda")
+    kvq.kvq_decode_attention(cfg, cache, q.cuda(), out, sm_scale or 1 / math.sqrt(128), ws)
+    torch.cuda.synchronize()
+    return GpuRun(cfg, cache, out, lens + appends)
+
+
+def gpu_views(w: inputs.Workload, run: GpuRun) -> Dict[str, np.ndarray]:
+    """GPU cache buffers as numpy arrays with the oracle's shapes."""
+    B, H, cap, G = w.batch, w.num_kv_heads, w.capacity(), w.group_size
+    ring = w.residual + G
+    c = run.cache
+    return {
+        "k_codes": c.view("k_codes", torch.int32).cpu().numpy().view(np.uint32).reshape(B, H, cap // 16, 64 * w.key_bits),
+        "v_codes": c.view("v_codes", torch.int32).cpu().numpy().view(np.uint32).reshape(B, H, cap // 16, 64 * w.value_bits),
+        "k_scale": c.view("k_scale", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, cap // G, 128),
+        "k_zero": c.view("k_zero", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, cap // G, 128),
+        "v_scale": c.view("v_scale", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, cap, 128 // G),
+        "v_zero": c.view("v_zero", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, cap, 128 // G),
+        "k_res": c.view("k_res", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, ring, 128),
+        "v_res": c.view("v_res", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, ring, 128),
+    }
+
+
+def compare_unit_cache(w: inputs.Workload, gv: Dict[str, np.ndarray], b: int, h: int, oc, ob: int, oh: int, T: int) -> None:
+    """Bit-exact comparison of everything that is defined for one unit of length T."""
+    G, R = w.group_size, w.residual
+    Q = max(T - R, 0) // G * G
+    ring = R + G
+    np.testing.assert_array_equal(gv["k_codes"][b, h, : Q // 16], oc.k_codes[ob, oh, : Q // 16], err_msg=f"k_codes unit {b},{h}")
+    np.testing.assert_array_equal(gv["v_codes"][b, h, : Q // 16], oc.v_codes[ob, oh, : Q // 16], err_msg=f"v_codes unit {b},{h}")
+    np.testing.assert_array_equal(gv["k_scale"][b, h, : Q // G], oc.k_scale[ob, oh, : Q // G], err_msg=f"k_scale unit {b},{h}")
+    np.testing.assert_array_equal(gv["k_zero"][b, h, : Q // G], oc.k_zero[ob, oh, : Q // G], err_msg=f"k_zero unit {b},{h}")
+    np.testing.assert_array_equal(gv["v_scale"][b, h, :Q], oc.v_scale[ob, oh, :Q], err_msg=f"v_scale unit {b},{h}")
+    np.testing.assert_array_equal(gv["v_zero"][b, h, :Q], oc.v_zero[ob, oh, :Q], err_msg=f"v_zero unit {b},{h}")
+    live = [t % ring for t in range(Q, T)]
+    np.testing.assert_array_equal(gv["k_res"][b, h, live], oc.k_res[ob, oh, live], err_msg=f"k_res unit {b},{h}")
+    np.testing.assert_array_equal(gv["v_res"][b, h, live], oc.v_res[ob, oh, live], err_msg=f"v_res unit {b},{h}")
+
+
+def check_attention(gpu_out: np.ndarray, ref: np.ndarray, what: str) -> Tuple[float, float]:
+    gpu = gpu_out.astype(np.float64)
+    err = np.abs(gpu - ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    denom = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(gpu - ref) / denom) if denom > 0 else float(np.linalg.norm(gpu))
+    assert max_abs <= MAX_ABS_TOL, f"{what}: max abs error {max_abs:.3e} > {MAX_ABS_TOL}"
+    assert rel <= REL_L2_TOL, f"{what}: relative L2 error {rel:.3e} > {REL_L2_TOL}"
+    return max_abs, rel
+
+
+def oracle_full(oracle, w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
+                appends: int = 0, sm_scale: Optional[float] = None, threads: int = 8):
+    ocfg = oracle_config(oracle, w)
+    oc = oracle.Cache(ocfg)
+    oracle.quantize_prefill(ocfg, oc, k.numpy(), v.numpy(), lens, threads=threads)
+    for step in range(appends):
+        kn, vn = inputs.append_tokens(w, step)
+        oracle.append_token(ocfg, oc, kn.numpy(), vn.numpy())
+    out = oracle.decode(ocfg, oc, q.numpy(), sm_scale or 1 / math.sqrt(128), threads=threads)
+    return oc, out
+
+
+def oracle_unit(oracle, w: inputs.Workload, b: int, h: int, T0: int, q: torch.Tensor, appends: int = 0,
+                sm_scale: Optional[float] = None, threads: int = 4):
+    """Oracle on the (sequence b, KV head h) sub-problem only (batch 1, one KV head, its g query heads)."""
+    g = w.gqa
+    ocfg = oracle_config(oracle, w, batch=1, hq=g, hkv=1)
+    oc = oracle.Cache(ocfg)
+    ku, vu = inputs.unit_kv(w, b, h, T0)
+    oracle.quantize_prefill(ocfg, oc, ku.numpy()[None, :, None, :], vu.numpy()[None, :, None, :], [T0])
+    for step in range(appends):
+        kn, vn = inputs.append_tokens(w, step)
+        oracle.append_token(ocfg, oc, kn[b:b + 1, h:h + 1].numpy(), vn[b:b + 1, h:h + 1].numpy())
+    qq = q[b:b + 1, h * g:(h + 1) * g].contiguous().numpy()
+    out = oracle.decode(ocfg, oc, qq, sm_scale or 1 / math.sqrt(128), threads=threads)
+    return oc, out[0]

@@ -1,0 +1,129 @@
+"""CPU checks of the C ABI: the library loads without a GPU, exports every entry point that
+include/kvq.h declares, reports buffer sizes from the layout's closed form, and rejects bad arguments
+on the host before anything is launched (no device memory is touched by these calls)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_kv_cache_prefill_b200 as kvq
+from bit_kv_cache_prefill_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_entry_point():
+    names = _declared_symbols()
+    assert names == ["kvq_append_token", "kvq_cache_buffer_bytes", "kvq_decode_attention",
+                     "kvq_decode_workspace_bytes", "kvq_quantize_prefill", "kvq_status_string"]
+    lib = ctypes.CDLL(kvq.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert hasattr(kvq, n), n  # the Python binding uses the same names
+
+
+def test_status_strings():
+    for s in (0, -1, -2, -3, -4, -5):
+        assert kvq.kvq_status_string(s) and kvq.kvq_status_string(s) != "unknown status"
+    assert kvq.kvq_status_string(7) == "unknown status"
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,kb,vb,G,R,cap", [(8, 32, 32, 2, 2, 32, 128, 32768), (16, 32, 8, 2, 2, 64, 128, 131328),
+                                                      (64, 32, 8, 4, 2, 32, 32, 16384), (1, 32, 8, 2, 2, 128, 128, 1 << 20)])
+def test_buffer_bytes_closed_form(B, Hq, Hkv, kb, vb, G, R, cap):
+    cfg = kvq.make_config(B, Hq, Hkv, kb, vb, G, R, 0, cap)
+    got = kvq.kvq_cache_buffer_bytes(cfg)
+    u = B * Hkv
+    # codes: bits per element; key scale/zero: fp16 per (group, channel); value: fp16 per (token, group)
+    want = [u * cap * 128 * kb // 8, u * cap * 128 * vb // 8, u * (cap // G) * 128 * 2, u * (cap // G) * 128 * 2,
+            u * cap * (128 // G) * 2, u * cap * (128 // G) * 2, u * (R + G) * 128 * 2, u * (R + G) * 128 * 2]
+    assert got == want
+    assert kvq.kvq_decode_workspace_bytes(cfg) > 0
+
+
+def _status(fn, *args):
+    return getattr(_lib.lib, fn)(*args)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 64, kvq.KVQ_ERR_UNSUPPORTED), ("key_bits", 3, kvq.KVQ_ERR_INVALID_ARG),
+    ("value_bits", 8, kvq.KVQ_ERR_INVALID_ARG), ("group_size", 48, kvq.KVQ_ERR_INVALID_ARG),
+    ("group_size", 256, kvq.KVQ_ERR_INVALID_ARG), ("num_q_heads", 33, kvq.KVQ_ERR_INVALID_ARG),
+    ("num_q_heads", 64, kvq.KVQ_ERR_UNSUPPORTED), ("residual", -1, kvq.KVQ_ERR_INVALID_ARG),
+    ("hadamard", 2, kvq.KVQ_ERR_INVALID_ARG), ("capacity", 100, kvq.KVQ_ERR_INVALID_ARG),
+    ("layout", 2, kvq.KVQ_ERR_UNSUPPORTED), ("batch", 0, kvq.KVQ_ERR_INVALID_ARG),
+])
+def test_config_validation(field, value, status):
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024)
+    setattr(cfg, field, value)
+    sizes = (ctypes.c_size_t * 8)()
+    assert _status("kvq_cache_buffer_bytes", ctypes.byref(cfg), sizes) == status
+    n = ctypes.c_size_t()
+    assert _status("kvq_decode_workspace_bytes", ctypes.byref(cfg), ctypes.byref(n)) == status
+    assert _status("kvq_cache_buffer_bytes", None, sizes) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def _fake_cache(cfg, lens):
+    # Non-null, 16-byte aligned placeholder addresses: every call below is rejected on the host before
+    # any of them could be used.
+    host = np.asarray(lens, np.int64).copy()
+    c = _lib.kvq_cache(*([0x10000 * (i + 1) for i in range(8)]),
+                       host.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), 0x90000)
+    return c, host
+
+
+def test_prefill_rejects_lengths_beyond_capacity_and_bad_strides():
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024)
+    c, host = _fake_cache(cfg, [0, 0])
+    lens = np.array([1025, 5], np.int64)
+    P = ctypes.POINTER(ctypes.c_int64)
+    assert _status("kvq_quantize_prefill", ctypes.byref(cfg), ctypes.byref(c), 0x100000, 0x200000, 0, 0, 0,
+                   lens.ctypes.data_as(P), None) == kvq.KVQ_ERR_CAPACITY
+    lens = np.array([10, -1], np.int64)
+    assert _status("kvq_quantize_prefill", ctypes.byref(cfg), ctypes.byref(c), 0x100000, 0x200000, 0, 0, 0,
+                   lens.ctypes.data_as(P), None) == kvq.KVQ_ERR_CAPACITY
+    lens = np.array([10, 5], np.int64)
+    # misaligned input pointer, odd stride, null input, null lengths
+    assert _status("kvq_quantize_prefill", ctypes.byref(cfg), ctypes.byref(c), 0x100002, 0x200000, 2048, 256, 128,
+                   lens.ctypes.data_as(P), None) == kvq.KVQ_ERR_INVALID_ARG
+    assert _status("kvq_quantize_prefill", ctypes.byref(cfg), ctypes.byref(c), 0x100000, 0x200000, 2048, 256, 129,
+                   lens.ctypes.data_as(P), None) == kvq.KVQ_ERR_INVALID_ARG
+    assert _status("kvq_quantize_prefill", ctypes.byref(cfg), ctypes.byref(c), None, 0x200000, 2048, 256, 128,
+                   lens.ctypes.data_as(P), None) == kvq.KVQ_ERR_INVALID_ARG
+    assert _status("kvq_quantize_prefill", ctypes.byref(cfg), ctypes.byref(c), 0x100000, 0x200000, 2048, 256, 128,
+                   None, None) == kvq.KVQ_ERR_INVALID_ARG
+    # a misaligned cache buffer
+    c.k_scale = 0x30008
+    assert _status("kvq_quantize_prefill", ctypes.byref(cfg), ctypes.byref(c), 0x100000, 0x200000, 2048, 256, 128,
+                   lens.ctypes.data_as(P), None) == kvq.KVQ_ERR_INVALID_ARG
+    assert list(host) == [0, 0]  # nothing changed on rejection
+
+
+def test_append_rejects_capacity_overflow_without_side_effects():
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024)
+    c, host = _fake_cache(cfg, [1024, 3])
+    assert _status("kvq_append_token", ctypes.byref(cfg), ctypes.byref(c), 0x100000, 0x200000, None) == kvq.KVQ_ERR_CAPACITY
+    assert list(host) == [1024, 3]
+    assert _status("kvq_append_token", ctypes.byref(cfg), ctypes.byref(c), 0x100008, 0x200000, None) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_decode_rejects_small_workspace_and_bad_scale():
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024)
+    c, _ = _fake_cache(cfg, [100, 3])
+    need = kvq.kvq_decode_workspace_bytes(cfg)
+    args = (ctypes.byref(cfg), ctypes.byref(c), 0x100000, 0x200000)
+    assert _status("kvq_decode_attention", *args, ctypes.c_float(0.1), 0x300000, need - 1, None) == kvq.KVQ_ERR_WORKSPACE
+    assert _status("kvq_decode_attention", *args, ctypes.c_float(0.1), None, need, None) == kvq.KVQ_ERR_WORKSPACE
+    assert _status("kvq_decode_attention", *args, ctypes.c_float(0.1), 0x300010, need, None) == kvq.KVQ_ERR_WORKSPACE
+    assert _status("kvq_decode_attention", *args, ctypes.c_float(0.0), 0x300000, need, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert _status("kvq_decode_attention", *args, ctypes.c_float(float("nan")), 0x300000, need, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert _status("kvq_decode_attention", ctypes.byref(cfg), ctypes.byref(c), None, 0x200000, ctypes.c_float(0.1),
+                   0x300000, need, None) == kvq.KVQ_ERR_INVALID_ARG

@@ -1,0 +1,171 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on the same seeded inputs.
+
+Codes, scales, zero-points and the FP16 ring must match bit for bit; decode attention must be within
+max-abs 2e-3 and relative L2 1e-3 of the oracle's fp64 result. Small cases span several 16-token
+tiles, several key groups, ragged tails and the edge cases (empty sequence, one token, everything in
+the FP16 window, R = 0, flush boundaries); the model-shaped workloads run at full size with the
+oracle checking sampled (sequence, KV head) units.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from bit_kv_cache_prefill_b200 import inputs
+
+import _harness as H
+
+pytestmark = pytest.mark.gpu
+
+W = inputs.Workload
+
+SMALL = [
+    # name, workload, lengths
+    ("k2v2_g32_r32_mha", W("t1", 2, 2, 2, 2, 2, 32, 32, 0, 1000, seed=11, outlier_channels=4,
+                           outlier_per_head=True, outlier_scale=20.0), [1000, 517]),
+    ("k2v2_g64_r128_gqa4", W("t2", 2, 8, 2, 2, 2, 64, 128, 0, 2125, seed=12), [2125, 300]),
+    ("k4v2_g32_r32_wht_gqa4", W("t3", 3, 8, 2, 4, 2, 32, 32, 1, 1500, seed=13, outlier_channels=8,
+                                outlier_per_head=False, outlier_scale=15.0), [1500, 33, 0]),
+    ("k2v2_g128_r128_gqa4", W("t4", 1, 4, 1, 2, 2, 128, 128, 0, 3000, seed=14), [3000]),
+    ("k4v4_g16_r0_gqa2", W("t5", 2, 4, 2, 4, 4, 16, 0, 0, 777, seed=15), [777, 16]),
+    ("k2v4_g16_r5_wht_gqa3", W("t6", 2, 6, 2, 2, 4, 16, 5, 1, 401, seed=16), [401, 1]),
+    ("all_in_window", W("t7", 2, 4, 1, 2, 2, 32, 256, 0, 200, seed=17), [200, 256]),
+]
+
+
+def _lens_workload(w, lens):
+    # capacity from the given lengths (round up to G)
+    return w.scaled(seq_len=max(lens) if max(lens) > 0 else w.group_size)
+
+
+def _inputs_for(w, lens):
+    B = w.batch
+    Tmax = max(max(lens), 1)
+    k = torch.zeros(B, Tmax, w.num_kv_heads, 128, dtype=torch.float16)
+    v = torch.zeros_like(k)
+    mask = inputs.outlier_mask(w)
+    for b in range(B):
+        for h in range(w.num_kv_heads):
+            if lens[b] > 0:
+                ku, vu = inputs.unit_kv(w, b, h, lens[b], mask)
+                k[b, : lens[b], h] = ku
+                v[b, : lens[b], h] = vu
+    return k, v
+
+
+@pytest.mark.parametrize("name,w,lens", SMALL, ids=[s[0] for s in SMALL])
+def test_small_prefill_bit_exact_and_decode(oracle_mod, name, w, lens):
+    w = _lens_workload(w, lens)
+    lens = np.array(lens, np.int64)
+    k, v = _inputs_for(w, lens)
+    q = inputs.query(w)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q)
+    oc, ref = H.oracle_full(oracle_mod, w, k, v, lens, q)
+    gv = H.gpu_views(w, run)
+    for b in range(w.batch):
+        for h in range(w.num_kv_heads):
+            H.compare_unit_cache(w, gv, b, h, oc, b, h, int(lens[b]))
+    H.check_attention(run.out.cpu().numpy(), ref, name)
+    # empty sequences decode to exact zeros
+    for b in range(w.batch):
+        if lens[b] == 0:
+            assert np.all(run.out[b].cpu().numpy() == 0)
+
+
+@pytest.mark.parametrize("case", [
+    dict(w=W("s1", 2, 8, 2, 2, 2, 32, 32, 0, 300, seed=21), T0=300, n=3 * 32 + 7),
+    dict(w=W("s2", 2, 2, 2, 4, 2, 16, 0, 1, 100, seed=22), T0=100, n=40),
+    dict(w=W("s3", 1, 4, 1, 2, 2, 64, 128, 0, 10, seed=23), T0=10, n=200),
+], ids=["g32_r32_gqa4", "g16_r0_wht", "g64_r128_from_window"])
+def test_streaming_append_matches_oracle_and_bulk_prefill(oracle_mod, case):
+    w, T0, n = case["w"], case["T0"], case["n"]
+    w = w.scaled(seq_len=T0, appends=n)
+    lens = np.full(w.batch, T0, np.int64)
+    k, v = _inputs_for(w, list(lens))
+    q = inputs.query(w)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, appends=n)
+    oc, ref = H.oracle_full(oracle_mod, w, k, v, lens, q, appends=n)
+    gv = H.gpu_views(w, run)
+    assert np.array_equal(run.cache.seq_len_host, lens + n)
+    assert np.array_equal(run.cache.seq_len_dev.cpu().numpy(), lens + n)
+    for b in range(w.batch):
+        for h in range(w.num_kv_heads):
+            H.compare_unit_cache(w, gv, b, h, oc, b, h, T0 + n)
+    H.check_attention(run.out.cpu().numpy(), ref, "streaming")
+    # the GPU's own bulk prefill of all T0 + n tokens gives the same defined bits
+    kk = torch.zeros(w.batch, T0 + n, w.num_kv_heads, 128, dtype=torch.float16)
+    vv = torch.zeros_like(kk)
+    kk[:, :T0], vv[:, :T0] = k, v
+    for s in range(n):
+        kn, vn = inputs.append_tokens(w, s)
+        kk[:, T0 + s], vv[:, T0 + s] = kn, vn
+    bulk = H.run_gpu(w, kk.cuda(), vv.cuda(), np.full(w.batch, T0 + n, np.int64), q)
+    gb = H.gpu_views(w, bulk)
+    G, R = w.group_size, w.residual
+    T = T0 + n
+    Q = max(T - R, 0) // G * G
+    live = [t % (R + G) for t in range(Q, T)]
+    for key in ("k_codes", "v_codes"):
+        np.testing.assert_array_equal(gv[key][:, :, : Q // 16], gb[key][:, :, : Q // 16])
+    for key in ("k_scale", "k_zero"):
+        np.testing.assert_array_equal(gv[key][:, :, : Q // G], gb[key][:, :, : Q // G])
+    for key in ("v_scale", "v_zero"):
+        np.testing.assert_array_equal(gv[key][:, :, :Q], gb[key][:, :, :Q])
+    for key in ("k_res", "v_res"):
+        np.testing.assert_array_equal(gv[key][:, :, live], gb[key][:, :, live])
+    np.testing.assert_array_equal(run.out.cpu().numpy(), bulk.out.cpu().numpy())
+
+
+def test_sm_scale_and_single_token(oracle_mod):
+    w = W("one", 1, 4, 1, 2, 2, 32, 4, 0, 1, seed=31)
+    lens = np.array([1], np.int64)
+    k, v = _inputs_for(w, [1])
+    q = inputs.query(w)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, sm_scale=0.37)
+    # one token: every head returns that token's value exactly (as fp16)
+    for h in range(4):
+        np.testing.assert_array_equal(run.out[0, h].cpu().numpy(), v[0, 0, 0].numpy())
+    w2 = W("scl", 1, 4, 1, 2, 2, 32, 32, 0, 700, seed=32)
+    k2, v2 = _inputs_for(w2, [700])
+    q2 = inputs.query(w2)
+    run2 = H.run_gpu(w2, k2.cuda(), v2.cuda(), np.array([700]), q2, sm_scale=0.02)
+    _, ref2 = H.oracle_full(oracle_mod, w2, k2, v2, np.array([700]), q2, sm_scale=0.02)
+    H.check_attention(run2.out.cpu().numpy(), ref2, "sm_scale 0.02")
+
+
+# ---- model-shaped workloads at full size; the oracle checks sampled units -------------------------
+FULL = ["tiny", "llama2_7b_mha", "llama3_8b_gqa", "mistral_7b_ragged", "million_token"]
+
+
+def _sample_units(w, lens):
+    B, Hkv = w.batch, w.num_kv_heads
+    picks = {(0, 0), (B - 1, Hkv - 1), (B // 2, Hkv // 2)}
+    if w.ragged_min:
+        picks |= {(int(np.argmax(lens)), 0), (int(np.argmin(lens)), Hkv - 1)}
+    if w.seq_len >= 1 << 20:
+        picks = {(0, Hkv - 1)}
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload_sampled(oracle_mod, name):
+    w = inputs.WORKLOADS[name]
+    k, v, lens = inputs.full_kv(w)
+    q = inputs.query(w)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, appends=w.appends)
+    del k, v
+    gv = H.gpu_views(w, run)
+    out = run.out.cpu().numpy()
+    refs, gots = [], []
+    for b, h in _sample_units(w, lens):
+        oc, ref = H.oracle_unit(oracle_mod, w, b, h, int(lens[b]), q, appends=w.appends)
+        H.compare_unit_cache(w, gv, b, h, oc, 0, 0, int(lens[b]) + w.appends)
+        got = out[b, h * w.gqa:(h + 1) * w.gqa]
+        H.check_attention(got, ref, f"{name} unit ({b},{h})")
+        refs.append(ref)
+        gots.append(got)
+    H.check_attention(np.concatenate(gots), np.concatenate(refs), f"{name} sampled units")
+    # every output is finite and the lengths advanced by the appends
+    assert np.isfinite(out.astype(np.float32)).all()
+    assert np.array_equal(run.cache.seq_len_host, lens + w.appends)
