@@ -9,7 +9,8 @@ _BINDING_NAMES = {
     "BUFFER_NAMES", "Cache", "KvqError", "KVQ_ERR_CAPACITY", "KVQ_ERR_CUDA", "KVQ_ERR_INVALID_ARG",
     "KVQ_ERR_UNSUPPORTED", "KVQ_ERR_WORKSPACE", "KVQ_OK", "LIB_PATH", "kvq_append_token", "kvq_cache",
     "kvq_cache_buffer_bytes", "kvq_config", "kvq_decode_attention", "kvq_decode_workspace_bytes",
-    "kvq_quantize_prefill", "kvq_status_string", "make_config",
+    "kvq_quantize_prefill", "kvq_status_string", "make_config", "kvq_decode_attention_noalloc",
+    "STATIC_SCRATCH_BYTES",
 }
 
 

@@ -62,6 +62,8 @@ def _load() -> ctypes.CDLL:
     L.kvq_decode_workspace_bytes.restype = S
     L.kvq_decode_attention.argtypes = [C, K, P, P, ctypes.c_float, P, ctypes.c_size_t, P]
     L.kvq_decode_attention.restype = S
+    L.kvq_decode_attention_noalloc.argtypes = [C, K, P, P, ctypes.c_float, P]
+    L.kvq_decode_attention_noalloc.restype = S
     L.kvq_status_string.argtypes = [S]
     L.kvq_status_string.restype = ctypes.c_char_p
     return L
@@ -146,3 +148,16 @@ def kvq_decode_attention(cfg: kvq_config, cache: Cache, q: torch.Tensor, out: to
     _check(lib.kvq_decode_attention(ctypes.byref(cfg), ctypes.byref(cache.c), q.data_ptr(), out.data_ptr(),
                                     float(sm_scale), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream_ptr(stream)), "kvq_decode_attention")
+
+
+STATIC_SCRATCH_BYTES = 16 << 20
+
+
+def kvq_decode_attention_noalloc(cfg: kvq_config, cache: Cache, q: torch.Tensor, out: torch.Tensor, sm_scale: float,
+                                 stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Decode attention for callers that cannot allocate device memory: the split partials live in
+    the library's fixed 16 MiB per-GPU scratch array (see include/kvq.h). Calls that overlap on the
+    GPU race on that array."""
+    assert q.is_contiguous() and out.is_contiguous()
+    _check(lib.kvq_decode_attention_noalloc(ctypes.byref(cfg), ctypes.byref(cache.c), q.data_ptr(), out.data_ptr(),
+                                            float(sm_scale), _stream_ptr(stream)), "kvq_decode_attention_noalloc")

@@ -171,6 +171,24 @@ kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, size_t* bytes);
 kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, const void* q, void* out, float sm_scale,
                                 void* workspace, size_t workspace_bytes, void* cuda_stream);
 
+/* Decode attention without a caller-provided workspace. The source pages have no counterpart to
+ * this entry point; it serves callers that cannot allocate device memory, such as a plugin inside a
+ * host framework that owns every device allocation through its own pool, or a serving loop whose
+ * policy forbids allocation after start-up.
+ * Same arguments, results and errors as kvq_decode_attention, except that the split partials live
+ * in a fixed device array inside the library: KVQ_STATIC_SCRATCH_BYTES (16 MiB) per GPU that loads
+ * the library, held until the process exits. It allocates nothing (no cudaMalloc, no allocating
+ * library routine).
+ *   - Returns KVQ_ERR_WORKSPACE if kvq_decode_workspace_bytes(cfg) exceeds KVQ_STATIC_SCRATCH_BYTES.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call shares the one array per device: calls whose GPU work overlaps (e.g. on two
+ *     streams) race on it; the caller must serialise them. No scratch content needs to start at
+ *     zero. */
+#define KVQ_STATIC_SCRATCH_BYTES (16u << 20)
+kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache* cache, const void* q, void* out,
+                                        float sm_scale, void* cuda_stream);
+
 /* Static description of a status code. */
 const char* kvq_status_string(kvq_status status);
 

@@ -23,7 +23,8 @@ def _declared_symbols():
 def test_library_exports_every_declared_entry_point():
     names = _declared_symbols()
     assert names == ["kvq_append_token", "kvq_cache_buffer_bytes", "kvq_decode_attention",
-                     "kvq_decode_workspace_bytes", "kvq_quantize_prefill", "kvq_status_string"]
+                     "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes", "kvq_quantize_prefill",
+                     "kvq_status_string"]
     lib = ctypes.CDLL(kvq.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
