@@ -215,7 +215,7 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVQ_ERR_CUDA;
-  const int occ = kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size);
+  const int occ = kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size, cfg->num_q_heads / cfg->num_kv_heads);
   int nsplit = 1;
   const int L = plan_splits(cfg, cache->seq_len_host, sms * occ, &nsplit);
 

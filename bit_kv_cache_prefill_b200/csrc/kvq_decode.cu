@@ -40,7 +40,7 @@
 namespace kvq {
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kStages = 3;  // pipeline stages per warp (each one step of 1 or 2 tiles)
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
@@ -153,44 +153,123 @@ __device__ __forceinline__ void load_halves(const uint8_t* p, float (&out)[2 * V
   }
 }
 
-template <int KB, int VB, int VPT>
+// Per-warp pipeline: a ring of kStages stages, each holding one step of TS 16-token tiles (codes
+// and value scale/zero), plus a ring of KP slots holding the key scale and zero of the KGB key groups
+// of one key block. A key block spans kBlockSteps steps; its parameters are read only when the
+// block's first step is consumed. Step j is issued at the top of iteration j - (kStages - 1) = j - 2,
+// so a new block's parameters may land in the slot of the block two back only once that block's
+// first step has been consumed: with kBlockSteps >= 2 this holds for two slots (a partial first
+// block plus a full block lie in between); one-step blocks use four slots (three blocks lie in
+// between).
+template <int KB, int VB, int VPT, int KGB, int TS>
 struct Stage {
-  static constexpr int kKC = 256 * KB;  // key codes of one tile
-  static constexpr int kVC = 256 * VB;  // value codes of one tile
-  static constexpr int kVS = 32 * VPT;  // value scale (or zero) of 16 tokens
-  static constexpr int kKP = 512;       // key scale[128] + zero[128] of one group
+  static constexpr int kKC = 256 * KB * TS;  // key codes of the step's tiles
+  static constexpr int kVC = 256 * VB * TS;  // value codes
+  static constexpr int kVS = 32 * VPT * TS;  // value scale (or zero) of the step's tokens
   static constexpr int oKC = 0;
   static constexpr int oVC = oKC + kKC;
   static constexpr int oVS = oVC + kVC;
   static constexpr int oVZ = oVS + kVS;
-  static constexpr int oKP = oVZ + kVS;
-  static constexpr int kBytes = oKP + kKP;
+  static constexpr int kBytes = oVZ + kVS;
+  static constexpr int kKP = 512 * KGB;  // key scale[128] + zero[128] per group of the block
+  static constexpr int kBlockSteps = (128 / VPT) * KGB / (16 * TS);
+  static constexpr int kKPSlots = kBlockSteps >= 2 ? 2 : 4;
+  static constexpr int kWarpBytes = kStages * kBytes + kKPSlots * kKP;
 };
 
-// Shared memory: query [4][128] f32, exponents [4] i32 (16 B), warp partials [W][4][130] f32,
-// zero sums [W][4][8] f32, then the per-warp stage rings.
-constexpr int kSmemQ = 4 * 128 * 4;
+// Shared memory: q~ [4][128] f32 (base-2 logit units), q^ = q~ * 2^-e [4][128] f32, exponents [4]
+// i32 (16 B), then the per-warp rings. After the main loops the ring area holds the warp partials
+// [W][4][130] f32 and the zero-point sums [W][4][8] f32.
+constexpr int kSmemQ = 2 * 4 * 128 * 4;
 constexpr int kSmemE = 16;
-constexpr int kSmemCM = kDecodeWarps * 4 * kPartFloats * 4;
-constexpr int kSmemZB = kDecodeWarps * 4 * 8 * 4;
-constexpr int kSmemFixed = kSmemQ + kSmemE + kSmemCM + kSmemZB;
+constexpr int kSmemFixed = kSmemQ + kSmemE;
+constexpr int kCm = 132;   // shared-memory partial stride (floats): m, l, 2 pad, o[128] 16-byte aligned
+constexpr int kCmO = 4;    // offset of o[] within a shared-memory partial
+constexpr int kSmemEpilogue = kDecodeWarps * 4 * kCm * 4 + kDecodeWarps * 4 * 8 * 4;
 static_assert(kSmemFixed % 16 == 0, "stage ring must start 16-byte aligned");
 
-template <int KB, int VB, int VPT>
+template <int KB, int VB, int VPT, int GQ>
+struct Shape {
+  static constexpr int KGB = 4 / GQ;                     // key groups per QK B block
+  static constexpr int VGB = 4 / GQ;                     // value groups per PV n-block
+  static constexpr int NBV = (VPT + VGB - 1) / VGB;      // PV n-blocks
+  static constexpr int G = 128 / VPT;
+  static constexpr int TS = G >= 32 ? 2 : 1;             // tiles per step
+  using S = Stage<KB, VB, VPT, KGB, TS>;
+};
+
+template <int KB, int VB, int VPT, int GQ>
 constexpr int decode_smem_bytes() {
-  return kSmemFixed + kDecodeWarps * kStages * Stage<KB, VB, VPT>::kBytes;
+  using S = typename Shape<KB, VB, VPT, GQ>::S;
+  constexpr int ring = kDecodeWarps * S::kWarpBytes;
+  return kSmemFixed + (ring > kSmemEpilogue ? ring : kSmemEpilogue);
 }
 
-template <int KB, int VB, int VPT>
-__global__ void __launch_bounds__(128, 3) decode_split_kernel(const DecodeArgs a) {
-  using S = Stage<KB, VB, VPT>;
-  constexpr int G = 128 / VPT;
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// cp.async of 16 bytes that writes zeros (and reads nothing) when `valid` is false.
+__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool valid) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
+}
+
+// QK of one 16-token tile: scores (base-2 units) of tokens r and r + 8 for this lane's column pair
+// (2 independent accumulator chains over the 8 channel blocks).
+template <int KB>
+__device__ __forceinline__ void tile_scores(const uint8_t* kc, int lane, const uint32_t (&bq)[8][2], float bias,
+                                            float p2e, float& s_lo, float& s_hi) {
+  float acc[2][4];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
+  if constexpr (KB == 2) {
+    const uint4 kw = *reinterpret_cast<const uint4*>(kc + 16 * lane);
+    const uint32_t w4[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t h[8];
+      unpack_word2(w4[w], h);
+      mma16816(acc[0], h[0], h[1], h[2], h[3], bq[2 * w][0], bq[2 * w][1]);
+      mma16816(acc[1], h[4], h[5], h[6], h[7], bq[2 * w + 1][0], bq[2 * w + 1][1]);
+    }
+  } else {
+    const uint4 k0 = *reinterpret_cast<const uint4*>(kc + 16 * lane);
+    const uint4 k1 = *reinterpret_cast<const uint4*>(kc + 512 + 16 * lane);
+    const uint32_t w8[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      uint32_t h[4];
+      unpack_word4(w8[w], h);
+      mma16816(acc[w & 1], h[0], h[1], h[2], h[3], bq[w][0], bq[w][1]);
+    }
+  }
+  s_lo = ((acc[0][0] + acc[1][0]) + (acc[0][1] + acc[1][1]) + bias) * p2e;  // hi + lo columns, token r
+  s_hi = ((acc[0][2] + acc[1][2]) + (acc[0][3] + acc[1][3]) + bias) * p2e;  // token r + 8
+}
+
+// N columns of the tensor-core tiles. GQ (1, 2 or 4) query heads share one KV head; the 8 columns of
+// an m16n8k16 B operand hold (group offset, head, hi/lo) for 4/GQ key (or value) groups:
+//   column n -> group offset n / (2 GQ), head (n / 2) % GQ, part n % 2 (0 = hi, 1 = lo).
+// With GQ = 4 every column is a (head, part) of one group; with GQ = 1 one B fragment covers 4 key
+// groups (QK) or 4 value groups (PV), so the per-group B rebuild is shared by 4 groups.
+// A lane (r, qd) of a D fragment holds columns 2qd, 2qd + 1, i.e. (group offset qd / GQ, head qd % GQ).
+template <int KB, int VB, int VPT, int GQ>
+__global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a) {
+  using SH = Shape<KB, VB, VPT, GQ>;
+  using S = typename SH::S;
+  constexpr int KGB = SH::KGB, VGB = SH::VGB, NBV = SH::NBV, G = SH::G, TS = SH::TS;
+  constexpr int kBlockTokens = G * KGB;
+  constexpr int kStepTokens = 16 * TS;
   extern __shared__ __align__(16) uint8_t smem[];
   float* sq = reinterpret_cast<float*>(smem);
   int* se = reinterpret_cast<int*>(smem + kSmemQ);
-  float* cm = reinterpret_cast<float*>(smem + kSmemQ + kSmemE);
-  float* zb = reinterpret_cast<float*>(smem + kSmemQ + kSmemE + kSmemCM);
   uint8_t* rings = smem + kSmemFixed;
+  float* cm = reinterpret_cast<float*>(rings);        // epilogue: [W][4][kCm] (m, l, -, -, o[128])
+  float* zb = cm + kDecodeWarps * 4 * kCm;            // epilogue: [W][4][8]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x;
@@ -198,12 +277,13 @@ __global__ void __launch_bounds__(128, 3) decode_split_kernel(const DecodeArgs a
   const int64_t b = unit / a.num_kv_heads;
   const int kvh = static_cast<int>(unit % a.num_kv_heads);
   const int gq = a.gqa;
-  const int64_t T = a.seq_len[b];
-  const int64_t start = static_cast<int64_t>(split) * a.split_len;
+  const int T = static_cast<int>(a.seq_len[b]);
+  const int L = a.split_len;
+  const int start = split * L;
   if (start >= T) return;
-  const int64_t end = min(start + static_cast<int64_t>(a.split_len), T);
-  const int64_t Q = quantized_len(T, a.R, G);
-  const int64_t qend = min(end, Q);
+  const int end = min(start + L, T);
+  const int Q = static_cast<int>(quantized_len(T, a.R, G));
+  const int qend = min(end, Q);
 
   // ---- query: optional Hadamard rotation, scale to base-2 logits, per-head power-of-two exponent.
   {
@@ -241,87 +321,101 @@ __global__ void __launch_bounds__(128, 3) decode_split_kernel(const DecodeArgs a
     for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, d));
     const int e = mx > 0.f ? ((__float_as_int(mx) >> 23) & 0xff) - 126 : 0;
     *reinterpret_cast<float4*>(sq + warp * kHeadDim + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
+    const float inv = pow2i(-e);
+    *reinterpret_cast<float4*>(sq + 4 * kHeadDim + warp * kHeadDim + 4 * lane) =
+        make_float4(x[0] * inv, x[1] * inv, x[2] * inv, x[3] * inv);
     if (lane == 0) se[warp] = e;
   }
   __syncthreads();
 
   const int qd = lane & 3, r = lane >> 2;
-  const int hb = r >> 1;              // head of this lane's B-fragment column (lane >> 2 = column n)
-  const bool lo_half = (r & 1) != 0;  // column n = 2*head + (0: hi, 1: lo)
-  float qn[32];                       // q^ of head hb at channel 16m + 2qd + 8hh + e, index 4m + 2hh + e
-  {
-    const float inv = pow2i(-se[hb]);
-#pragma unroll
-    for (int m = 0; m < 8; ++m)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) qn[4 * m + k] = sq[hb * kHeadDim + 16 * m + 2 * qd + 8 * (k >> 1) + (k & 1)] * inv;
-  }
-  const float p2e_d = pow2i(se[qd]);  // scale of this lane's D-fragment head (head qd)
+  // B-fragment role (column n = r): group offset, head, hi/lo part.
+  const int col_off = r / (2 * GQ);
+  const int col_head = (r >> 1) % GQ;
+  const bool lo_half = (r & 1) != 0;
+  // D-fragment role: this lane's head for the softmax.
+  const int h_d = qd % GQ;
+  const float* qn_row = sq + 4 * kHeadDim + col_head * kHeadDim + 2 * qd;  // q^ of head col_head
+  const float p2e_d = pow2i(se[h_d]);
 
-  // ---- this warp's quantized tiles
-  const int64_t ntiles = qend > start ? (qend - start) / kTile : 0;
-  const int64_t per = (ntiles + kDecodeWarps - 1) / kDecodeWarps;
-  const int64_t tb = min(ntiles, per * warp);
-  const int nt = static_cast<int>(min(ntiles, per * (warp + 1)) - tb);
-  uint8_t* ring = rings + warp * kStages * S::kBytes;
-  const int64_t first_token = start + tb * kTile;
+  // ---- this warp's quantized steps (contiguous)
+  const int nsteps = qend > start ? (qend - start) / kStepTokens : 0;
+  const int per = (nsteps + kDecodeWarps - 1) / kDecodeWarps;
+  const int sb = min(nsteps, per * warp);
+  const int nst = min(nsteps, per * (warp + 1)) - sb;
+  uint8_t* ring = rings + warp * S::kWarpBytes;
+  uint8_t* kp_ring = ring + kStages * S::kBytes;
+  const int first_token = start + sb * kStepTokens;
+  const int q_groups = Q / G;
 
   float m_run = -CUDART_INF_F, l_run = 0.f;
   float O[8][4];
 #pragma unroll
   for (int m = 0; m < 8; ++m) O[m][0] = O[m][1] = O[m][2] = O[m][3] = 0.f;
-  float zacc[VPT];
+  float zacc[NBV];
 #pragma unroll
-  for (int j = 0; j < VPT; ++j) zacc[j] = 0.f;
+  for (int j = 0; j < NBV; ++j) zacc[j] = 0.f;
   uint32_t bq[8][2];
 #pragma unroll
   for (int m = 0; m < 8; ++m) bq[m][0] = bq[m][1] = 0u;
-  float bias_d = 0.f;
+  float bias_col = 0.f;
 
-  const uint8_t* kc_base = reinterpret_cast<const uint8_t*>(a.k_codes + unit * a.tiles * (64 * KB));
-  const uint8_t* vc_base = reinterpret_cast<const uint8_t*>(a.v_codes + unit * a.tiles * (64 * VB));
-  const uint8_t* vs_base = reinterpret_cast<const uint8_t*>(a.v_scale + unit * a.capacity * VPT);
-  const uint8_t* vz_base = reinterpret_cast<const uint8_t*>(a.v_zero + unit * a.capacity * VPT);
-  const uint16_t* ks_base = a.k_scale + unit * a.groups * kHeadDim;
-  const uint16_t* kz_base = a.k_zero + unit * a.groups * kHeadDim;
+  const uint8_t* kc_ptr = reinterpret_cast<const uint8_t*>(a.k_codes + unit * a.tiles * (64 * KB)) +
+                          static_cast<int64_t>(first_token / kTile) * (256 * KB) + 16 * lane;
+  const uint8_t* vc_ptr = reinterpret_cast<const uint8_t*>(a.v_codes + unit * a.tiles * (64 * VB)) +
+                          static_cast<int64_t>(first_token / kTile) * (256 * VB) + 16 * lane;
+  const uint8_t* vs_ptr = reinterpret_cast<const uint8_t*>(a.v_scale + (unit * a.capacity + first_token) * VPT) + 16 * lane;
+  const uint8_t* vz_ptr = reinterpret_cast<const uint8_t*>(a.v_zero + (unit * a.capacity + first_token) * VPT) + 16 * lane;
+  const uint16_t* kp_src = (lane < 16 ? a.k_scale : a.k_zero) + unit * a.groups * kHeadDim + 8 * (lane & 15);
 
+  // issue(i): step i of this warp into stage i % kStages; the lane pointers advance one step per call
   auto issue = [&](int i) {
-    uint8_t* st = ring + (i % kStages) * S::kBytes;
-    const int64_t t = first_token + static_cast<int64_t>(i) * kTile;
-    const int64_t tile = t / kTile;
+    uint8_t* st = ring + (i % kStages) * S::kBytes + 16 * lane;
 #pragma unroll
-    for (int c = lane; c < S::kKC / 16; c += 32) cp_async16(st + S::oKC + 16 * c, kc_base + tile * S::kKC + 16 * c);
+    for (int c = 0; c < S::kKC / 512; ++c) cp_async16(st + S::oKC + 512 * c, kc_ptr + 512 * c);
 #pragma unroll
-    for (int c = lane; c < S::kVC / 16; c += 32) cp_async16(st + S::oVC + 16 * c, vc_base + tile * S::kVC + 16 * c);
+    for (int c = 0; c < S::kVC / 512; ++c) cp_async16(st + S::oVC + 512 * c, vc_ptr + 512 * c);
     if (lane < S::kVS / 16) {
-      cp_async16(st + S::oVS + 16 * lane, vs_base + t * (2 * VPT) + 16 * lane);
-      cp_async16(st + S::oVZ + 16 * lane, vz_base + t * (2 * VPT) + 16 * lane);
+      cp_async16(st + S::oVS, vs_ptr);
+      cp_async16(st + S::oVZ, vz_ptr);
     }
-    if (i == 0 || (t % G) == 0) {
-      const int64_t g = t / G;
-      const uint16_t* src = lane < 16 ? ks_base + g * kHeadDim + 8 * lane : kz_base + g * kHeadDim + 8 * (lane - 16);
-      cp_async16(st + S::oKP + 16 * lane, src);
+    const int t = first_token + i * kStepTokens;
+    if (i == 0 || (t % kBlockTokens) == 0) {
+      const int blk = t / kBlockTokens;
+      uint8_t* kp = kp_ring + (blk % S::kKPSlots) * S::kKP + 16 * lane;
+#pragma unroll
+      for (int kg = 0; kg < KGB; ++kg) {
+        const int g = blk * KGB + kg;
+        const bool valid = g < q_groups;
+        cp_async16_zfill(kp + 512 * kg, kp_src + static_cast<int64_t>(valid ? g : 0) * kHeadDim, valid);
+      }
     }
+    kc_ptr += S::kKC;
+    vc_ptr += S::kVC;
+    vs_ptr += S::kVS;
+    vz_ptr += S::kVS;
   };
 
 #pragma unroll
   for (int i = 0; i < kStages - 1; ++i) {
-    if (i < nt) issue(i);
+    if (i < nst) issue(i);
     cp_async_commit();
   }
 
-  for (int i = 0; i < nt; ++i) {
-    if (i + kStages - 1 < nt) issue(i + kStages - 1);
+  for (int i = 0; i < nst; ++i) {
+    if (i + kStages - 1 < nst) issue(i + kStages - 1);
     cp_async_commit();
     cp_async_wait<kStages - 1>();
     __syncwarp();
     const uint8_t* st = ring + (i % kStages) * S::kBytes;
-    const int64_t t = first_token + static_cast<int64_t>(i) * kTile;
+    const int t = first_token + i * kStepTokens;
 
-    // -- new key group: fold its scale into the query (hi/lo fp16) and its zero into a bias
-    if (i == 0 || (t % G) == 0) {
-      const uint4* sp = reinterpret_cast<const uint4*>(st + S::oKP + 64 * qd);
-      const uint4* zp = reinterpret_cast<const uint4*>(st + S::oKP + 256 + 64 * qd);
+    // -- new key block: fold the scales of its KGB groups into the query (hi/lo fp16) and the
+    //    zero-points into per-column biases
+    if (i == 0 || (t % kBlockTokens) == 0) {
+      const uint8_t* kp = kp_ring + ((t / kBlockTokens) % S::kKPSlots) * S::kKP + 512 * col_off;
+      const uint4* sp = reinterpret_cast<const uint4*>(kp + 64 * qd);
+      const uint4* zp = reinterpret_cast<const uint4*>(kp + 256 + 64 * qd);
       float bias = 0.f;
 #pragma unroll
       for (int v4 = 0; v4 < 4; ++v4) {
@@ -331,54 +425,51 @@ __global__ void __launch_bounds__(128, 3) decode_split_kernel(const DecodeArgs a
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int idx = 8 * v4 + 2 * k;  // = 4m + 2hh
+          const float2 qq = *reinterpret_cast<const float2*>(qn_row + 16 * (idx >> 2) + 8 * ((idx >> 1) & 1));
           const float s0 = h2f(static_cast<uint16_t>(sw[k] & 0xffffu)), s1 = h2f(static_cast<uint16_t>(sw[k] >> 16));
           const float z0 = h2f(static_cast<uint16_t>(zw[k] & 0xffffu)), z1 = h2f(static_cast<uint16_t>(zw[k] >> 16));
-          const float x0 = qn[idx] * s0, x1 = qn[idx + 1] * s1;
-          bq[idx >> 2][(idx >> 1) & 1] = pack_h2(split_part(x0, lo_half), split_part(x1, lo_half));
-          bias = fmaf(qn[idx], z0, bias);
-          bias = fmaf(qn[idx + 1], z1, bias);
+          bq[idx >> 2][(idx >> 1) & 1] = pack_h2(split_part(qq.x * s0, lo_half), split_part(qq.y * s1, lo_half));
+          bias = fmaf(qq.x, z0, bias);
+          bias = fmaf(qq.y, z1, bias);
         }
       }
       bias += __shfl_xor_sync(kFull, bias, 1);
       bias += __shfl_xor_sync(kFull, bias, 2);
-      bias_d = __shfl_sync(kFull, bias, 8 * qd);  // lanes with column n = 2qd hold head qd
+      bias_col = __shfl_sync(kFull, bias, 8 * qd);  // lanes of column 2qd hold its bias
     }
 
-    // -- scores of the 16 tokens: rows r, r+8; columns (head qd hi, head qd lo)
-    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-    if constexpr (KB == 2) {
-      const uint4 kw = *reinterpret_cast<const uint4*>(st + S::oKC + 16 * lane);
-      const uint32_t w4[4] = {kw.x, kw.y, kw.z, kw.w};
+    // -- scores of the step's tokens (TS tiles). With GQ < 4 the tile's key group offset selects the
+    //    lane whose column pair holds its score.
+    float s[TS][2];
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t h[8];
-        unpack_word2(w4[w], h);
-        mma16816(sacc, h[0], h[1], h[2], h[3], bq[2 * w][0], bq[2 * w][1]);
-        mma16816(sacc, h[4], h[5], h[6], h[7], bq[2 * w + 1][0], bq[2 * w + 1][1]);
-      }
-    } else {
-      const uint4 k0 = *reinterpret_cast<const uint4*>(st + S::oKC + 16 * lane);
-      const uint4 k1 = *reinterpret_cast<const uint4*>(st + S::oKC + 512 + 16 * lane);
-      const uint32_t w8[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+    for (int u = 0; u < TS; ++u) tile_scores<KB>(st + S::oKC + u * 256 * KB, lane, bq, bias_col, p2e_d, s[u][0], s[u][1]);
+    if constexpr (GQ < 4) {
+      const int src = 4 * r + ((t / G) % KGB) * GQ + h_d;  // one key group per step (G >= step)
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        uint32_t h[4];
-        unpack_word4(w8[w], h);
-        mma16816(sacc, h[0], h[1], h[2], h[3], bq[w][0], bq[w][1]);
+      for (int u = 0; u < TS; ++u) {
+        s[u][0] = __shfl_sync(kFull, s[u][0], src);
+        s[u][1] = __shfl_sync(kFull, s[u][1], src);
       }
     }
-    const float s_lo = (sacc[0] + sacc[1] + bias_d) * p2e_d;  // token r
-    const float s_hi = (sacc[2] + sacc[3] + bias_d) * p2e_d;  // token r + 8
 
-    // -- online softmax for head qd over this tile
-    float tmax = fmaxf(s_lo, s_hi);
+    // -- online softmax for head h_d over the step
+    float tmax = fmaxf(s[0][0], s[0][1]);
+#pragma unroll
+    for (int u = 1; u < TS; ++u) tmax = fmaxf(tmax, fmaxf(s[u][0], s[u][1]));
     tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 4));
     tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 8));
     tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 16));
     const float m_new = fmaxf(m_run, tmax);
-    const float alpha = exp2f(m_run - m_new);
-    const float p_lo = exp2f(s_lo - m_new), p_hi = exp2f(s_hi - m_new);
-    l_run = l_run * alpha + p_lo + p_hi;
+    const float alpha = fast_exp2(m_run - m_new);
+    float p[TS][2];
+    float lsum = 0.f;
+#pragma unroll
+    for (int u = 0; u < TS; ++u) {
+      p[u][0] = fast_exp2(s[u][0] - m_new);
+      p[u][1] = fast_exp2(s[u][1] - m_new);
+      lsum += p[u][0] + p[u][1];
+    }
+    l_run = fmaf(l_run, alpha, lsum);
     if (__any_sync(kFull, alpha != 1.f)) {
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
@@ -387,144 +478,187 @@ __global__ void __launch_bounds__(128, 3) decode_split_kernel(const DecodeArgs a
         O[m][2] *= alpha;
         O[m][3] *= alpha;
       }
-      const float az = __shfl_sync(kFull, alpha, hb);  // lane hb holds head hb's factor
+      const float az = __shfl_sync(kFull, alpha, col_head);  // lane col_head has h_d == col_head
 #pragma unroll
-      for (int j = 0; j < VPT; ++j) zacc[j] *= az;
+      for (int j = 0; j < NBV; ++j) zacc[j] *= az;
     }
     m_run = m_new;
 
-    // -- P.V: B = p * sv (hi/lo) for tokens 2qd, 2qd+1, 2qd+8, 2qd+9 of head hb
-    const int la = 8 * qd + hb;
-    const float pa = __shfl_sync(kFull, p_lo, la), pb = __shfl_sync(kFull, p_lo, la + 4);
-    const float pc = __shfl_sync(kFull, p_hi, la), pd = __shfl_sync(kFull, p_hi, la + 4);
-    float sv01[2 * VPT], sv89[2 * VPT], zv01[2 * VPT], zv89[2 * VPT];
-    load_halves<VPT>(st + S::oVS + 4 * VPT * qd, sv01);
-    load_halves<VPT>(st + S::oVS + 4 * VPT * qd + 16 * VPT, sv89);
-    load_halves<VPT>(st + S::oVZ + 4 * VPT * qd, zv01);
-    load_halves<VPT>(st + S::oVZ + 4 * VPT * qd + 16 * VPT, zv89);
-    // v^ = code * sv + zv = (code - cbar) * sv + mid with mid = zv + cbar * sv, the group midpoint
+    // -- P.V per tile: B = p * sv (hi/lo) of head col_head for tokens 2qd, 2qd+1, 2qd+8, 2qd+9 and
+    //    the value group of this lane's column in each n-block; A = centered value codes
+    const int la = 8 * qd + col_head;
     constexpr float kCbar = VB == 2 ? 1.5f : 7.5f;
-    uint32_t bp[VPT][2];
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      bp[j][0] = pack_h2(split_part(pa * sv01[j], lo_half), split_part(pb * sv01[VPT + j], lo_half));
-      bp[j][1] = pack_h2(split_part(pc * sv89[j], lo_half), split_part(pd * sv89[VPT + j], lo_half));
-      float z = zacc[j];
-      z = fmaf(pa, fmaf(kCbar, sv01[j], zv01[j]), z);
-      z = fmaf(pb, fmaf(kCbar, sv01[VPT + j], zv01[VPT + j]), z);
-      z = fmaf(pc, fmaf(kCbar, sv89[j], zv89[j]), z);
-      z = fmaf(pd, fmaf(kCbar, sv89[VPT + j], zv89[VPT + j]), z);
-      zacc[j] = z;
-    }
-    if constexpr (VB == 2) {
-      const uint4 vw = *reinterpret_cast<const uint4*>(st + S::oVC + 16 * lane);
-      const uint32_t w4[4] = {vw.x, vw.y, vw.z, vw.w};
+    for (int u = 0; u < TS; ++u) {
+      const float pa = __shfl_sync(kFull, p[u][0], la), pb = __shfl_sync(kFull, p[u][0], la + 4);
+      const float pc = __shfl_sync(kFull, p[u][1], la), pd = __shfl_sync(kFull, p[u][1], la + 4);
+      const uint16_t* vsh = reinterpret_cast<const uint16_t*>(st + S::oVS) + u * 16 * VPT;
+      const uint16_t* vzh = reinterpret_cast<const uint16_t*>(st + S::oVZ) + u * 16 * VPT;
+      uint32_t bp[NBV][2];
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t h[8];
-        unpack_word2_centered(w4[w], h);
-        constexpr int kMPerJ = 8 / VPT;  // 16-channel blocks per value group
-        mma16816(O[2 * w], h[0], h[1], h[2], h[3], bp[(2 * w) / kMPerJ][0], bp[(2 * w) / kMPerJ][1]);
-        mma16816(O[2 * w + 1], h[4], h[5], h[6], h[7], bp[(2 * w + 1) / kMPerJ][0], bp[(2 * w + 1) / kMPerJ][1]);
+      for (int nb = 0; nb < NBV; ++nb) {
+        const int j = nb * VGB + col_off;
+        if (VPT % VGB == 0 || j < VPT) {
+          const int t0 = 2 * qd * VPT + j;
+          const float s0 = h2f(vsh[t0]), s1 = h2f(vsh[t0 + VPT]), s2 = h2f(vsh[t0 + 8 * VPT]), s3 = h2f(vsh[t0 + 9 * VPT]);
+          const float z0 = h2f(vzh[t0]), z1 = h2f(vzh[t0 + VPT]), z2 = h2f(vzh[t0 + 8 * VPT]), z3 = h2f(vzh[t0 + 9 * VPT]);
+          bp[nb][0] = pack_h2(split_part(pa * s0, lo_half), split_part(pb * s1, lo_half));
+          bp[nb][1] = pack_h2(split_part(pc * s2, lo_half), split_part(pd * s3, lo_half));
+          float z = zacc[nb];
+          z = fmaf(pa, fmaf(kCbar, s0, z0), z);
+          z = fmaf(pb, fmaf(kCbar, s1, z1), z);
+          z = fmaf(pc, fmaf(kCbar, s2, z2), z);
+          z = fmaf(pd, fmaf(kCbar, s3, z3), z);
+          zacc[nb] = z;
+        } else {
+          bp[nb][0] = bp[nb][1] = 0u;
+        }
       }
-    } else {
-      const uint4 v0 = *reinterpret_cast<const uint4*>(st + S::oVC + 16 * lane);
-      const uint4 v1 = *reinterpret_cast<const uint4*>(st + S::oVC + 512 + 16 * lane);
-      const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      // m-block m (channels 16m .. 16m+15) lies in value group (16m) / G, held by n-block group / VGB
+      const uint8_t* vc = st + S::oVC + u * 256 * VB;
+      if constexpr (VB == 2) {
+        const uint4 vw = *reinterpret_cast<const uint4*>(vc + 16 * lane);
+        const uint32_t w4[4] = {vw.x, vw.y, vw.z, vw.w};
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        uint32_t h[4];
-        unpack_word4_centered(w8[w], h);
-        constexpr int kMPerJ = 8 / VPT;
-        mma16816(O[w], h[0], h[1], h[2], h[3], bp[w / kMPerJ][0], bp[w / kMPerJ][1]);
+        for (int w = 0; w < 4; ++w) {
+          uint32_t h[8];
+          unpack_word2_centered(w4[w], h);
+          const int nb0 = (2 * w * VPT / 8) / VGB;
+          const int nb1 = ((2 * w + 1) * VPT / 8) / VGB;
+          mma16816(O[2 * w], h[0], h[1], h[2], h[3], bp[nb0][0], bp[nb0][1]);
+          mma16816(O[2 * w + 1], h[4], h[5], h[6], h[7], bp[nb1][0], bp[nb1][1]);
+        }
+      } else {
+        const uint4 v0 = *reinterpret_cast<const uint4*>(vc + 16 * lane);
+        const uint4 v1 = *reinterpret_cast<const uint4*>(vc + 512 + 16 * lane);
+        const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          uint32_t h[4];
+          unpack_word4_centered(w8[w], h);
+          const int nb = (w * VPT / 8) / VGB;
+          mma16816(O[w], h[0], h[1], h[2], h[3], bp[nb][0], bp[nb][1]);
+        }
       }
     }
     __syncwarp();  // every lane is done with this stage before it is refilled
   }
   cp_async_wait<0>();
-  __syncwarp();
+  __syncthreads();  // the ring area becomes the epilogue area below
 
-  // ---- FP16 residual tokens (CUDA cores): lane (r, qd) covers channels 16m + r, 16m + r + 8 of head qd
-  const int64_t rbeg = max(start, Q);
-  if (rbeg + warp < end) {
-    float qr[16];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      qr[2 * m] = sq[qd * kHeadDim + 16 * m + r];
-      qr[2 * m + 1] = sq[qd * kHeadDim + 16 * m + r + 8];
-    }
-    uint16_t* kbuf = reinterpret_cast<uint16_t*>(ring);
-    uint16_t* vbuf = kbuf + kHeadDim;
-    for (int64_t t = rbeg + warp; t < end; t += kDecodeWarps) {
-      const int64_t slot = (unit * a.ring + t % a.ring) * kHeadDim;
-      reinterpret_cast<uint2*>(kbuf)[lane] = reinterpret_cast<const uint2*>(a.k_res + slot)[lane];
-      reinterpret_cast<uint2*>(vbuf)[lane] = reinterpret_cast<const uint2*>(a.v_res + slot)[lane];
-      __syncwarp();
-      float dot = 0.f;
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        dot = fmaf(qr[2 * m], h2f(kbuf[16 * m + r]), dot);
-        dot = fmaf(qr[2 * m + 1], h2f(kbuf[16 * m + r + 8]), dot);
-      }
-      dot += __shfl_xor_sync(kFull, dot, 4);
-      dot += __shfl_xor_sync(kFull, dot, 8);
-      dot += __shfl_xor_sync(kFull, dot, 16);
-      const float m_new = fmaxf(m_run, dot);
-      const float alpha = exp2f(m_run - m_new);
-      const float p = exp2f(dot - m_new);
-      l_run = l_run * alpha + (r == 0 ? p : 0.f);
-      if (__any_sync(kFull, alpha != 1.f)) {
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          O[m][0] *= alpha;
-          O[m][1] *= alpha;
-          O[m][2] *= alpha;
-          O[m][3] *= alpha;
-        }
-        const float az = __shfl_sync(kFull, alpha, hb);
-#pragma unroll
-        for (int j = 0; j < VPT; ++j) zacc[j] *= az;
-      }
-      m_run = m_new;
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        O[m][0] = fmaf(p, h2f(vbuf[16 * m + r]), O[m][0]);
-        O[m][2] = fmaf(p, h2f(vbuf[16 * m + r + 8]), O[m][2]);
-      }
-      __syncwarp();
-    }
-  }
-
-  // ---- warp partial -> shared memory
+  // ---- warp partial of the quantized tokens -> shared memory
   l_run += __shfl_xor_sync(kFull, l_run, 4);
   l_run += __shfl_xor_sync(kFull, l_run, 8);
   l_run += __shfl_xor_sync(kFull, l_run, 16);
 #pragma unroll
-  for (int j = 0; j < VPT; ++j) {
+  for (int j = 0; j < NBV; ++j) {
     zacc[j] += __shfl_xor_sync(kFull, zacc[j], 1);
     zacc[j] += __shfl_xor_sync(kFull, zacc[j], 2);
   }
-  float* cw = cm + warp * 4 * kPartFloats;
-  if (qd < gq) {
-    float* o = cw + qd * kPartFloats + 2;
+  float* cw = cm + warp * 4 * kCm;
+  if (h_d < gq) {
+    float* o = cw + h_d * kCm + kCmO;
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
-      o[16 * m + r] = O[m][0] + O[m][1];
-      o[16 * m + r + 8] = O[m][2] + O[m][3];
+      const int jm = (16 * m) / G;
+      if (qd / GQ == jm % VGB) {  // this lane owns the columns of m-block m's value group
+        o[16 * m + r] = O[m][0] + O[m][1];
+        o[16 * m + r + 8] = O[m][2] + O[m][3];
+      }
     }
-    if (r == 0) {
-      cw[qd * kPartFloats] = m_run;
-      cw[qd * kPartFloats + 1] = l_run;
+    if (r == 0 && qd < GQ) {
+      cw[h_d * kCm] = m_run;
+      cw[h_d * kCm + 1] = l_run;
     }
   }
-  if (qd == 0 && !lo_half && hb < gq) {
+  if (qd == 0 && !lo_half && col_head < gq) {
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) zb[(warp * 4 + hb) * 8 + j] = zacc[j];
+    for (int nb = 0; nb < NBV; ++nb) {
+      const int j = nb * VGB + col_off;
+      if (j < VPT) zb[(warp * 4 + col_head) * 8 + j] = zacc[nb];
+    }
   }
   __syncwarp();
   for (int idx = lane; idx < gq * kHeadDim; idx += 32) {
     const int h = idx >> 7, c = idx & 127;
-    cw[h * kPartFloats + 2 + c] += zb[(warp * 4 + h) * 8 + c / G];
+    cw[h * kCm + kCmO + c] += zb[(warp * 4 + h) * 8 + c / G];
+  }
+  __syncwarp();
+
+  // ---- FP16 window tokens [Q, T), spread over all splits of the unit: this CTA takes tokens
+  //      Q + split + k * ns (ns = splits holding tokens), warp w the k = w (mod 4); batches of 8 with
+  //      all loads issued first. Lane l holds channels 4l .. 4l + 3; the batch's partial is merged
+  //      into the warp partial in shared memory.
+  {
+    const int ns = (T + L - 1) / L;
+    float qr[GQ][4];
+#pragma unroll
+    for (int h = 0; h < GQ; ++h) {
+      const float4 v = *reinterpret_cast<const float4*>(sq + h * kHeadDim + 4 * lane);
+      qr[h][0] = v.x;
+      qr[h][1] = v.y;
+      qr[h][2] = v.z;
+      qr[h][3] = v.w;
+    }
+    const uint2* kres = reinterpret_cast<const uint2*>(a.k_res + unit * a.ring * kHeadDim) + lane;
+    const uint2* vres = reinterpret_cast<const uint2*>(a.v_res + unit * a.ring * kHeadDim) + lane;
+    for (int k0 = warp; Q + split + k0 * ns < T; k0 += 4 * 8) {
+      uint2 kk[8], vv[8];
+      bool valid[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int tt = Q + split + (k0 + 4 * j) * ns;
+        valid[j] = tt < T;
+        const int slot = valid[j] ? static_cast<int>(tt % a.ring) : 0;
+        kk[j] = kres[slot * (kHeadDim / 4)];
+        vv[j] = vres[slot * (kHeadDim / 4)];
+      }
+#pragma unroll
+      for (int h = 0; h < GQ; ++h) {
+        if (h >= gq) break;
+        float sc[8];
+        float mb = -CUDART_INF_F;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float d = qr[h][0] * h2f(static_cast<uint16_t>(kk[j].x & 0xffffu));
+          d = fmaf(qr[h][1], h2f(static_cast<uint16_t>(kk[j].x >> 16)), d);
+          d = fmaf(qr[h][2], h2f(static_cast<uint16_t>(kk[j].y & 0xffffu)), d);
+          d = fmaf(qr[h][3], h2f(static_cast<uint16_t>(kk[j].y >> 16)), d);
+#pragma unroll
+          for (int x = 16; x > 0; x >>= 1) d += __shfl_xor_sync(kFull, d, x);
+          sc[j] = valid[j] ? d : -CUDART_INF_F;
+          mb = fmaxf(mb, sc[j]);
+        }
+        // merge this batch into the warp partial of head h (channels 4 lane .. 4 lane + 3)
+        float* ph = cw + h * kCm;
+        const float m_old = ph[0];
+        const float m_new = fmaxf(m_old, mb);
+        const float f_old = fast_exp2(m_old - m_new);
+        float o4[4] = {0.f, 0.f, 0.f, 0.f};
+        float lb = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float pj = fast_exp2(sc[j] - m_new);
+          lb += pj;
+          o4[0] = fmaf(pj, h2f(static_cast<uint16_t>(vv[j].x & 0xffffu)), o4[0]);
+          o4[1] = fmaf(pj, h2f(static_cast<uint16_t>(vv[j].x >> 16)), o4[1]);
+          o4[2] = fmaf(pj, h2f(static_cast<uint16_t>(vv[j].y & 0xffffu)), o4[2]);
+          o4[3] = fmaf(pj, h2f(static_cast<uint16_t>(vv[j].y >> 16)), o4[3]);
+        }
+        float4 cur = *reinterpret_cast<float4*>(ph + kCmO + 4 * lane);
+        cur.x = fmaf(cur.x, f_old, o4[0]);
+        cur.y = fmaf(cur.y, f_old, o4[1]);
+        cur.z = fmaf(cur.z, f_old, o4[2]);
+        cur.w = fmaf(cur.w, f_old, o4[3]);
+        *reinterpret_cast<float4*>(ph + kCmO + 4 * lane) = cur;
+        __syncwarp();
+        if (lane == 0) {
+          ph[0] = m_new;
+          ph[1] = fmaf(ph[1], f_old, lb);
+        }
+        __syncwarp();
+      }
+    }
   }
   __syncthreads();
 
@@ -534,13 +668,16 @@ __global__ void __launch_bounds__(128, 3) decode_split_kernel(const DecodeArgs a
     const int h = idx >> 7, c = idx & 127;
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, cm[(w * 4 + h) * kPartFloats]);
+    for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, cm[(w * 4 + h) * kCm]);
+    // A split can hold no token at all (its range lies in the FP16 window and the window tokens went
+    // to other splits): its partial is (m = -inf, l = 0, o = 0), which the combine weighs by 0.
+    const bool empty = M == -CUDART_INF_F;
     float o = 0.f, l = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecodeWarps; ++w) {
-      const float* pw = cm + (w * 4 + h) * kPartFloats;
-      const float f = exp2f(pw[0] - M);
-      o = fmaf(f, pw[2 + c], o);
+      const float* pw = cm + (w * 4 + h) * kCm;
+      const float f = empty ? 0.f : fast_exp2(pw[0] - M);
+      o = fmaf(f, pw[kCmO + c], o);
       l = fmaf(f, pw[1], l);
     }
     part[h * kPartFloats + 2 + c] = o;
@@ -573,51 +710,72 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a)
   float l = 0.f, acc = 0.f;
   for (int s = 0; s < ns; ++s) {
     const float* p = base + s * stride;
-    const float f = exp2f(p[0] - M);
+    const float f = fast_exp2(p[0] - M);
     l = fmaf(f, p[1], l);
     acc = fmaf(f, p[2 + c], acc);
   }
   out[c] = __half_as_ushort(__float2half_rn(acc / l));
 }
 
-template <int KB, int VB, int VPT>
+template <int KB, int VB, int VPT, int GQ>
 cudaError_t launch_split(const DecodeArgs& a, cudaStream_t stream) {
-  constexpr int smem = decode_smem_bytes<KB, VB, VPT>();
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  constexpr int smem = decode_smem_bytes<KB, VB, VPT, GQ>();
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads));
-  decode_split_kernel<KB, VB, VPT><<<grid, 32 * kDecodeWarps, smem, stream>>>(a);
+  decode_split_kernel<KB, VB, VPT, GQ><<<grid, 32 * kDecodeWarps, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <int KB, int VB, int VPT>
+template <int KB, int VB, int VPT, int GQ>
 int occupancy() {
-  constexpr int smem = decode_smem_bytes<KB, VB, VPT>();
-  if (cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  constexpr int smem = decode_smem_bytes<KB, VB, VPT, GQ>();
+  if (cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<KB, VB, VPT>, 32 * kDecodeWarps, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<KB, VB, VPT, GQ>, 32 * kDecodeWarps, smem) != cudaSuccess)
     return 1;
   return n > 0 ? n : 1;
+}
+
+// GQ template: the smallest of 1, 2, 4 that holds the query heads of one KV head.
+inline int gq_class(int gqa) { return gqa <= 1 ? 1 : (gqa <= 2 ? 2 : 4); }
+
+template <int KB, int VB, int VPT>
+cudaError_t dispatch_gq(const DecodeArgs& a, cudaStream_t s) {
+  switch (gq_class(a.gqa)) {
+    case 1: return launch_split<KB, VB, VPT, 1>(a, s);
+    case 2: return launch_split<KB, VB, VPT, 2>(a, s);
+    default: return launch_split<KB, VB, VPT, 4>(a, s);
+  }
+}
+
+template <int KB, int VB, int VPT>
+int occupancy_gq(int gqa) {
+  switch (gq_class(gqa)) {
+    case 1: return occupancy<KB, VB, VPT, 1>();
+    case 2: return occupancy<KB, VB, VPT, 2>();
+    default: return occupancy<KB, VB, VPT, 4>();
+  }
 }
 
 template <int KB, int VB>
 cudaError_t dispatch_vpt(const DecodeArgs& a, cudaStream_t s) {
   switch (a.G) {
-    case 128: return launch_split<KB, VB, 1>(a, s);
-    case 64: return launch_split<KB, VB, 2>(a, s);
-    case 32: return launch_split<KB, VB, 4>(a, s);
-    default: return launch_split<KB, VB, 8>(a, s);
+    case 128: return dispatch_gq<KB, VB, 1>(a, s);
+    case 64: return dispatch_gq<KB, VB, 2>(a, s);
+    case 32: return dispatch_gq<KB, VB, 4>(a, s);
+    default: return dispatch_gq<KB, VB, 8>(a, s);
   }
 }
 
 template <int KB, int VB>
-int occupancy_vpt(int G) {
+int occupancy_vpt(int G, int gqa) {
   switch (G) {
-    case 128: return occupancy<KB, VB, 1>();
-    case 64: return occupancy<KB, VB, 2>();
-    case 32: return occupancy<KB, VB, 4>();
-    default: return occupancy<KB, VB, 8>();
+    case 128: return occupancy_gq<KB, VB, 1>(gqa);
+    case 64: return occupancy_gq<KB, VB, 2>(gqa);
+    case 32: return occupancy_gq<KB, VB, 4>(gqa);
+    default: return occupancy_gq<KB, VB, 8>(gqa);
   }
 }
 
@@ -634,9 +792,9 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-int decode_ctas_per_sm(int key_bits, int value_bits, int G) {
-  if (key_bits == 2) return value_bits == 2 ? occupancy_vpt<2, 2>(G) : occupancy_vpt<2, 4>(G);
-  return value_bits == 2 ? occupancy_vpt<4, 2>(G) : occupancy_vpt<4, 4>(G);
+int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa) {
+  if (key_bits == 2) return value_bits == 2 ? occupancy_vpt<2, 2>(G, gqa) : occupancy_vpt<2, 4>(G, gqa);
+  return value_bits == 2 ? occupancy_vpt<4, 2>(G, gqa) : occupancy_vpt<4, 4>(G, gqa);
 }
 
 }  // namespace kvq

@@ -46,7 +46,7 @@ struct DecodeArgs {
 cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream);
 cudaError_t launch_append(const QuantizeArgs& a, const uint16_t* k_new, const uint16_t* v_new, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
-int decode_ctas_per_sm(int key_bits, int value_bits, int G);
+int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);
 
 constexpr int kDecodeWarps = 4;
 constexpr int kPartFloats = 2 + 128;  // m, l, o[128]

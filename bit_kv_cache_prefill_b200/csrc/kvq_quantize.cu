@@ -19,8 +19,10 @@
 
 namespace kvq {
 
-// Shared-memory footprint of one chunk: fp16 rows [G][128] plus one code byte per element.
-static size_t chunk_smem_bytes(int G) { return static_cast<size_t>(G) * kHeadDim * 3; }
+// Shared memory of one chunk: fp16 rows [G][128], then per-chunk parameters: keys use (f32(zero),
+// 1/f32(scale)) per channel [128] plus per-quarter min/max keys [4][128] x 2; values use
+// (f32(zero), 1/f32(scale)) per (token, channel group) [G][128/G] = 128 entries.
+static size_t chunk_smem_bytes(int G) { return static_cast<size_t>(G) * kHeadDim * 2 + 128 * 8 + 2 * 4 * 128 * 4; }
 
 // Rotate (keys, optional) the G staged rows in place: two rows per warp per step.
 __device__ void rotate_rows(uint16_t* rows, int nrows) {
@@ -44,23 +46,51 @@ __device__ void rotate_rows(uint16_t* rows, int nrows) {
   }
 }
 
-// Quantize G staged key rows (tokens t0 .. t0+G-1 of `unit`) and write group t0/G.
+// Code of x on the grid (zf, inv): rint_even((f32(x) - zf) * inv) clamped to [0, 2^bits - 1].
+// inv == 0 encodes a zero scale and yields code 0 (x - zf is finite).
+__device__ __forceinline__ uint32_t code_with(uint16_t x, float zf, float inv, int top) {
+  int c = __float2int_rn(__fmul_rn(__fsub_rn(h2f(x), zf), inv));
+  c = c < 0 ? 0 : (c > top ? top : c);
+  return static_cast<uint32_t>(c);
+}
+
+// Quantize G staged key rows (tokens t0 .. t0+G-1 of `unit`) and write key group t0/G.
+// All 256 threads work in every phase: min/max over token quarters for channel pairs, parameters per
+// channel, then one packed word per thread-iteration built straight from the fp16 rows.
 __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t t0, const uint16_t* rows,
-                                    uint8_t* codes) {
-  const int G = a.G, bits = a.key_bits;
+                                    uint8_t* pbuf) {
+  const int G = a.G, bits = a.key_bits, top = (1 << bits) - 1;
+  float2* prm = reinterpret_cast<float2*>(pbuf);                  // [128] (zf, inv)
+  uint32_t* pmin = reinterpret_cast<uint32_t*>(pbuf + 128 * 8);   // [4][128]
+  uint32_t* pmax = pmin + 4 * 128;                                // [4][128]
   const int64_t g = t0 / G;
-  for (int c = threadIdx.x; c < kHeadDim; c += blockDim.x) {
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int i = 0; i < G; ++i) {
-      const uint32_t k = order_key(rows[i * kHeadDim + c]);
-      kmin = min(kmin, k);
-      kmax = max(kmax, k);
+  {
+    const int cp = threadIdx.x & 63, tq = threadIdx.x >> 6;
+    const int n = G / 4;
+    uint32_t mn0 = 0xffffffffu, mx0 = 0u, mn1 = 0xffffffffu, mx1 = 0u;
+    for (int i = tq * n; i < (tq + 1) * n; ++i) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(rows + i * kHeadDim + 2 * cp);
+      const uint32_t k0 = order_key(w & 0xffffu), k1 = order_key(w >> 16);
+      mn0 = min(mn0, k0);
+      mx0 = max(mx0, k0);
+      mn1 = min(mn1, k1);
+      mx1 = max(mx1, k1);
     }
+    pmin[tq * 128 + 2 * cp] = mn0;
+    pmin[tq * 128 + 2 * cp + 1] = mn1;
+    pmax[tq * 128 + 2 * cp] = mx0;
+    pmax[tq * 128 + 2 * cp + 1] = mx1;
+  }
+  __syncthreads();
+  if (threadIdx.x < kHeadDim) {
+    const int c = threadIdx.x;
+    const uint32_t kmin = min(min(pmin[c], pmin[128 + c]), min(pmin[256 + c], pmin[384 + c]));
+    const uint32_t kmax = max(max(pmax[c], pmax[128 + c]), max(pmax[256 + c], pmax[384 + c]));
     const QuantParams p = make_params(kmin, kmax, bits);
     const int64_t pidx = (unit * a.groups + g) * kHeadDim + key_param_pos(c);
     a.k_scale[pidx] = p.s16;
     a.k_zero[pidx] = p.z16;
-    for (int i = 0; i < G; ++i) codes[i * kHeadDim + c] = static_cast<uint8_t>(code_of(rows[i * kHeadDim + c], p, bits));
+    prm[c] = make_float2(p.zf, p.inv);
   }
   __syncthreads();
   const int words = 64 * bits;
@@ -73,10 +103,11 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
     uint32_t word = 0;
     for (int j = 0; j < P; ++j) {
       int i, c;
-      key_slot(lane, w * P + j, &i, &c);
-      const uint8_t* cr = codes + (tile * kTile + i) * kHeadDim + c;
-      word |= static_cast<uint32_t>(cr[0]) << (bits * j);
-      word |= static_cast<uint32_t>(cr[1]) << (16 + bits * j);
+      key_slot(lane, w * P + j, &i, &c);  // c is even: the pair is channels c, c + 1 of token i
+      const uint32_t x = *reinterpret_cast<const uint32_t*>(rows + (tile * kTile + i) * kHeadDim + c);
+      const float4 pp = *reinterpret_cast<const float4*>(prm + c);  // (zf, inv) of c and c + 1
+      word |= code_with(static_cast<uint16_t>(x & 0xffffu), pp.x, pp.y, top) << (bits * j);
+      word |= code_with(static_cast<uint16_t>(x >> 16), pp.z, pp.w, top) << (16 + bits * j);
     }
     dst[static_cast<int64_t>(tile) * words + widx] = word;
   }
@@ -84,23 +115,35 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
 
 // Quantize G staged value rows (per token, channel groups of G) and write their codes.
 __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64_t t0, const uint16_t* rows,
-                                      uint8_t* codes) {
-  const int G = a.G, bits = a.value_bits;
+                                      uint8_t* pbuf) {
+  const int G = a.G, bits = a.value_bits, top = (1 << bits) - 1;
   const int vpt = kHeadDim / G;
-  for (int item = threadIdx.x; item < G * vpt; item += blockDim.x) {
+  float2* prm = reinterpret_cast<float2*>(pbuf);  // [G][vpt] (zf, inv)
+  {
+    // item (token i, group j) = threadIdx.x / 2; each of the two threads scans half of the G channels
+    const int item = threadIdx.x >> 1, half = threadIdx.x & 1;
     const int i = item / vpt, j = item % vpt;
-    const uint16_t* x = rows + i * kHeadDim + j * G;
+    const uint16_t* x = rows + i * kHeadDim + j * G + half * (G / 2);
     uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int c = 0; c < G; ++c) {
-      const uint32_t k = order_key(x[c]);
-      kmin = min(kmin, k);
-      kmax = max(kmax, k);
+    for (int c8 = 0; c8 < G / 2; c8 += 8) {
+      const uint4 v = *reinterpret_cast<const uint4*>(x + c8);
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t k0 = order_key(wv[q] & 0xffffu), k1 = order_key(wv[q] >> 16);
+        kmin = min(kmin, min(k0, k1));
+        kmax = max(kmax, max(k0, k1));
+      }
     }
-    const QuantParams p = make_params(kmin, kmax, bits);
-    const int64_t pidx = (unit * a.capacity + t0 + i) * vpt + j;
-    a.v_scale[pidx] = p.s16;
-    a.v_zero[pidx] = p.z16;
-    for (int c = 0; c < G; ++c) codes[i * kHeadDim + j * G + c] = static_cast<uint8_t>(code_of(x[c], p, bits));
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, 1));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 1));
+    if (half == 0) {
+      const QuantParams p = make_params(kmin, kmax, bits);
+      const int64_t pidx = (unit * a.capacity + t0 + i) * vpt + j;
+      a.v_scale[pidx] = p.s16;
+      a.v_zero[pidx] = p.z16;
+      prm[i * vpt + j] = make_float2(p.zf, p.inv);
+    }
   }
   __syncthreads();
   const int words = 64 * bits;
@@ -113,10 +156,11 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
     uint32_t word = 0;
     for (int j = 0; j < P; ++j) {
       int i, c;
-      value_slot(lane, w * P + j, &i, &c);
-      const uint8_t* cr = codes + (tile * kTile + i) * kHeadDim + c;
-      word |= static_cast<uint32_t>(cr[0]) << (bits * j);
-      word |= static_cast<uint32_t>(cr[kHeadDim]) << (16 + bits * j);
+      value_slot(lane, w * P + j, &i, &c);  // the pair is tokens i, i + 1 of channel c
+      const int ti = tile * kTile + i;
+      const float2 p0 = prm[ti * vpt + c / G], p1 = prm[(ti + 1) * vpt + c / G];
+      word |= code_with(rows[ti * kHeadDim + c], p0.x, p0.y, top) << (bits * j);
+      word |= code_with(rows[(ti + 1) * kHeadDim + c], p1.x, p1.y, top) << (16 + bits * j);
     }
     dst[static_cast<int64_t>(tile) * words + widx] = word;
   }
@@ -135,7 +179,7 @@ __global__ void __launch_bounds__(256) prefill_kernel(QuantizeArgs a) {
   if (t0 >= T) return;
   const int64_t n = min(static_cast<int64_t>(G), T - t0);
   uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
-  uint8_t* codes = smem + static_cast<size_t>(G) * kHeadDim * 2;
+  uint8_t* pbuf = smem + static_cast<size_t>(G) * kHeadDim * 2;
   const uint16_t* src = is_key ? a.k : a.v;
   // Stage the chunk: 16 lanes per 256-byte token row.
   for (int idx = threadIdx.x; idx < n * 16; idx += blockDim.x) {
@@ -151,9 +195,9 @@ __global__ void __launch_bounds__(256) prefill_kernel(QuantizeArgs a) {
   }
   if (t0 + G <= Q) {
     if (is_key)
-      quantize_keys_chunk(a, unit, t0, rows, codes);
+      quantize_keys_chunk(a, unit, t0, rows, pbuf);
     else
-      quantize_values_chunk(a, unit, t0, rows, codes);
+      quantize_values_chunk(a, unit, t0, rows, pbuf);
     return;
   }
   // FP16 window: tokens [t0, t0 + n) (all >= Q because Q is a multiple of G).
@@ -179,7 +223,7 @@ __global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint1
   const int64_t Q_old = quantized_len(t, a.R, G);
   const int64_t Q_new = quantized_len(t + 1, a.R, G);
   uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
-  uint8_t* codes = smem + static_cast<size_t>(G) * kHeadDim * 2;
+  uint8_t* pbuf = smem + static_cast<size_t>(G) * kHeadDim * 2;
   uint16_t* ring = (is_key ? a.k_res : a.v_res) + unit * a.ring * kHeadDim;
   const uint16_t* src = (is_key ? k_new : v_new) + unit * kHeadDim;
   // New token -> ring slot t mod (R + G), rotated first for keys when enabled (warp 0, 16 lanes).
@@ -207,9 +251,9 @@ __global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint1
   }
   __syncthreads();
   if (is_key)
-    quantize_keys_chunk(a, unit, Q_old, rows, codes);
+    quantize_keys_chunk(a, unit, Q_old, rows, pbuf);
   else
-    quantize_values_chunk(a, unit, Q_old, rows, codes);
+    quantize_values_chunk(a, unit, Q_old, rows, pbuf);
 }
 
 __global__ void bump_lengths_kernel(int64_t* seq_len, int batch) {

@@ -31,6 +31,9 @@ SMALL = [
     ("k4v4_g16_r0_gqa2", W("t5", 2, 4, 2, 4, 4, 16, 0, 0, 777, seed=15), [777, 16]),
     ("k2v4_g16_r5_wht_gqa3", W("t6", 2, 6, 2, 2, 4, 16, 5, 1, 401, seed=16), [401, 1]),
     ("all_in_window", W("t7", 2, 4, 1, 2, 2, 32, 256, 0, 200, seed=17), [200, 256]),
+    # R = 0 with a partial group in the window: splits whose range is all window can get no token
+    ("r0_window_tail_mha", W("t8", 2, 2, 2, 2, 2, 32, 0, 0, 777, seed=18), [777, 40]),
+    ("r0_window_tail_gqa4_g16", W("t9", 1, 8, 2, 4, 2, 16, 0, 1, 1000, seed=19), [1000]),
 ]
 
 
