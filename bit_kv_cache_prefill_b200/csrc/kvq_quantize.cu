@@ -47,11 +47,13 @@ __device__ void rotate_rows(uint16_t* rows, int nrows) {
 }
 
 // Code of x on the grid (zf, inv): rint_even((f32(x) - zf) * inv) clamped to [0, 2^bits - 1].
-// inv == 0 encodes a zero scale and yields code 0 (x - zf is finite).
+// inv == 0 encodes a zero scale and yields code 0 (x - zf is finite). v = (x - zf) * inv is >= 0
+// because x >= zf; clamping before rounding gives the same code as rounding then clamping. The
+// round-half-even to an integer is an IEEE add of 1.5 * 2^23 (exact for 0 <= v < 2^22): the sum's low
+// mantissa bits are the rounded integer.
 __device__ __forceinline__ uint32_t code_with(uint16_t x, float zf, float inv, int top) {
-  int c = __float2int_rn(__fmul_rn(__fsub_rn(h2f(x), zf), inv));
-  c = c < 0 ? 0 : (c > top ? top : c);
-  return static_cast<uint32_t>(c);
+  const float v = fminf(__fmul_rn(__fsub_rn(h2f(x), zf), inv), static_cast<float>(top));
+  return __float_as_uint(__fadd_rn(v, 12582912.0f)) & 0xffu;
 }
 
 // Quantize G staged key rows (tokens t0 .. t0+G-1 of `unit`) and write key group t0/G.
