@@ -227,6 +227,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling captures)")
+    ap.add_argument("--layout", type=int, default=1, choices=[1, 2],
+                    help="packed layout: 1 = tile v1 (mma.sync decode), 2 = rows v2 (tcgen05 decode)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w0 = inputs.WORKLOADS[args.workload]
@@ -262,8 +264,11 @@ def main():
     k, v, _ = inputs.full_kv(w0)  # CPU, seeded
     kd, vd = k.cuda(), v.cuda()
     del k, v
+    cap = w.capacity()
+    if args.layout == 2:
+        cap = -(-cap // 128) * 128  # rows v2 stores values in whole 128-token blocks
     cfg = kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size, w.residual,
-                          w.hadamard, w.capacity())
+                          w.hadamard, cap, layout=args.layout)
     cache = kvq.Cache(cfg)
     stream = torch.cuda.current_stream()
 
@@ -401,7 +406,7 @@ def main():
         "config": {"workload": w0.name, "batch": w0.batch, "seq_len": w0.seq_len, "num_q_heads": w0.num_q_heads,
                    "num_kv_heads": w0.num_kv_heads, "key_bits": w0.key_bits, "value_bits": w0.value_bits,
                    "group_size": w0.group_size, "residual": w0.residual, "hadamard": w0.hadamard,
-                   "ragged": bool(w0.ragged_min), "parallelism": f"replicas{args.gpus}",
+                   "ragged": bool(w0.ragged_min), "parallelism": f"replicas{args.gpus}", "layout": args.layout,
                    "l2": f"inputs larger than L2 ({step_bytes[0] / 2**20:.0f} MiB read per decode > 126 MiB)"},
         "tokens_per_s": round(tokens / (total_ms * 1e-3), 1),
         "frac_of_nominal_8tbs": round(value / NOMINAL_HBM_GBS, 4),
@@ -409,7 +414,8 @@ def main():
         "append_us": round(statistics.mean(append_ms) * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
-                     "kernel": "decode_split_kernel + decode_combine_kernel (one kvq_decode_attention call)"},
+                     "kernel": ("decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
+                     + " + decode_combine_kernel (one kvq_decode_attention call)"},
         "prefill": {"gbs": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9, 1),
                     "ms": round(statistics.mean(pre_ms), 3), "bytes": pre_bytes},
         "gpu_launches": 4 * args.steps,

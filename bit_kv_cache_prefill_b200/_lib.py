@@ -23,6 +23,7 @@ KVQ_ERR_CAPACITY = -3
 KVQ_ERR_WORKSPACE = -4
 KVQ_ERR_CUDA = -5
 KVQ_LAYOUT_TILE_V1 = 1
+KVQ_LAYOUT_ROWS_V2 = 2
 BUFFER_NAMES = ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero", "k_res", "v_res")
 
 
@@ -77,9 +78,10 @@ def kvq_status_string(status: int) -> str:
 
 
 def make_config(batch: int, num_q_heads: int, num_kv_heads: int, key_bits: int, value_bits: int, group_size: int,
-                residual: int, hadamard: int, capacity: int, head_dim: int = 128) -> kvq_config:
+                residual: int, hadamard: int, capacity: int, head_dim: int = 128,
+                layout: int = KVQ_LAYOUT_TILE_V1) -> kvq_config:
     return kvq_config(batch, num_q_heads, num_kv_heads, head_dim, key_bits, value_bits, group_size, residual,
-                      hadamard, KVQ_LAYOUT_TILE_V1, capacity)
+                      hadamard, layout, capacity)
 
 
 def _check(status: int, where: str) -> None:

@@ -17,13 +17,14 @@ namespace {
 
 constexpr int kMaxResidual = 4096;
 constexpr int64_t kTargetCtas = 2048;  // split budget used to bound the decode workspace
-constexpr int kSplitQuantum = 64;      // split lengths are multiples of 4 warps x 16-token tiles
+constexpr int kSplitQuantum = 64;      // tile v1: split lengths are multiples of 4 warps x 16-token tiles
+constexpr int kSplitQuantumTc = 128;   // rows v2: whole 128-token steps
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 kvq_status check_config(const kvq_config* c) {
   if (c == nullptr) return KVQ_ERR_INVALID_ARG;
-  if (c->layout != KVQ_LAYOUT_TILE_V1) return KVQ_ERR_UNSUPPORTED;
+  if (c->layout != KVQ_LAYOUT_TILE_V1 && c->layout != KVQ_LAYOUT_ROWS_V2) return KVQ_ERR_UNSUPPORTED;
   if (c->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
   if (c->batch < 1 || c->num_kv_heads < 1 || c->num_q_heads < 1) return KVQ_ERR_INVALID_ARG;
   if (c->num_q_heads % c->num_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
@@ -34,7 +35,8 @@ kvq_status check_config(const kvq_config* c) {
   if (c->residual < 0 || c->residual > kMaxResidual) return KVQ_ERR_INVALID_ARG;
   if (c->hadamard != 0 && c->hadamard != 1) return KVQ_ERR_INVALID_ARG;
   if (c->capacity < 0 || c->capacity % G != 0) return KVQ_ERR_INVALID_ARG;
-  if (c->capacity > (int64_t(1) << 40)) return KVQ_ERR_INVALID_ARG;
+  if (c->capacity >= (int64_t(1) << 31)) return KVQ_ERR_INVALID_ARG;  // token indices are 32-bit on the device
+  if (c->layout == KVQ_LAYOUT_ROWS_V2 && c->capacity % 128 != 0) return KVQ_ERR_INVALID_ARG;  // whole value blocks
   if (static_cast<int64_t>(c->batch) * c->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;  // grid.y
   return KVQ_OK;
 }
@@ -44,7 +46,8 @@ void buffer_bytes(const kvq_config* c, size_t out[KVQ_NUM_BUFFERS]) {
   const size_t cap = static_cast<size_t>(c->capacity);
   const size_t G = static_cast<size_t>(c->group_size);
   out[KVQ_BUF_K_CODES] = units * (cap / 16) * 64 * c->key_bits * 4;
-  out[KVQ_BUF_V_CODES] = units * (cap / 16) * 64 * c->value_bits * 4;
+  const size_t vcap = c->layout == KVQ_LAYOUT_ROWS_V2 ? (cap + 127) / 128 * 128 : cap;
+  out[KVQ_BUF_V_CODES] = units * (vcap / 16) * 64 * c->value_bits * 4;
   out[KVQ_BUF_K_SCALE] = units * (cap / G) * 128 * 2;
   out[KVQ_BUF_K_ZERO] = out[KVQ_BUF_K_SCALE];
   out[KVQ_BUF_V_SCALE] = units * cap * (128 / G) * 2;
@@ -89,6 +92,8 @@ QuantizeArgs quantize_args(const kvq_config* c, kvq_cache* k) {
   a.tiles = c->capacity / kvq::kTile;
   a.groups = c->capacity / c->group_size;
   a.ring = static_cast<int64_t>(c->residual) + c->group_size;
+  a.layout = c->layout;
+  a.vwords = (c->layout == KVQ_LAYOUT_ROWS_V2 ? (c->capacity + 127) / 128 * 128 : c->capacity) * 4 * c->value_bits;
   return a;
 }
 
@@ -103,18 +108,21 @@ int64_t max_splits(const kvq_config* c) {
 int plan_splits(const kvq_config* c, const int64_t* lens, int slots, int* nsplit) {
   int64_t tmax = 0;
   for (int b = 0; b < c->batch; ++b) tmax = std::max(tmax, lens[b]);
+  const bool tc = c->layout == KVQ_LAYOUT_ROWS_V2;
+  const int64_t quantum = tc ? kSplitQuantumTc : kSplitQuantum;
   if (tmax <= 0) {
     *nsplit = 1;
-    return kSplitQuantum;
+    return static_cast<int>(quantum);
   }
   const int64_t smax = max_splits(c);
+  const int64_t nmin = 1;
   const double overhead = 256.0;  // tokens' worth of per-CTA fixed cost (query prep, partial write)
   double best = 1e300;
   int64_t best_L = 0;
-  for (int64_t n = 1; n <= smax; ++n) {
+  for (int64_t n = nmin; n <= smax; ++n) {
     int64_t L = (tmax + n - 1) / n;
-    L = (L + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
-    if (n > 1 && L == best_L) continue;
+    L = (L + quantum - 1) / quantum * quantum;
+    if (n > nmin && L == best_L) continue;
     int64_t ctas = 0;
     for (int b = 0; b < c->batch; ++b) ctas += (lens[b] + L - 1) / L;
     ctas *= c->num_kv_heads;
@@ -215,7 +223,10 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVQ_ERR_CUDA;
-  const int occ = kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size, cfg->num_q_heads / cfg->num_kv_heads);
+  const int occ = cfg->layout == KVQ_LAYOUT_ROWS_V2
+                      ? kvq::kTcCtasPerSm
+                      : kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size,
+                                                cfg->num_q_heads / cfg->num_kv_heads);
   int nsplit = 1;
   const int L = plan_splits(cfg, cache->seq_len_host, sms * occ, &nsplit);
 
@@ -246,6 +257,7 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   a.tiles = cfg->capacity / kvq::kTile;
   a.groups = cfg->capacity / cfg->group_size;
   a.ring = static_cast<int64_t>(cfg->residual) + cfg->group_size;
+  a.layout = cfg->layout;
   a.split_len = L;
   a.nsplit = nsplit;
   a.qscale = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);

@@ -35,6 +35,7 @@
 #include <math_constants.h>
 
 #include "kvq_common.cuh"
+#include "kvq_decode_common.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -42,59 +43,6 @@ namespace {
 
 constexpr int kStages = 3;  // pipeline stages per warp (each one step of 1 or 2 tiles)
 constexpr unsigned kFull = 0xffffffffu;
-
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-// Eight exact fp16x2 code pairs from a 2-bit word, pair k of the word in element k.
-__device__ __forceinline__ void unpack_word2(uint32_t x, uint32_t (&h)[8]) {
-  const uint32_t y = x >> 10;
-  h[0] = hsub2((x & 0x00030003u) | 0x64006400u, 0x64006400u);  // 1024 + c
-  h[1] = hsub2((x & 0x000C000Cu) | 0x5C005C00u, 0x5C005C00u);  // 256 + c
-  h[2] = hsub2((x & 0x00300030u) | 0x54005400u, 0x54005400u);  // 64 + c
-  h[3] = hsub2((x & 0x00C000C0u) | 0x4C004C00u, 0x4C004C00u);  // 16 + c
-  h[4] = hsub2((x & 0x03000300u) | 0x44004400u, 0x44004400u);  // 4 + c
-  h[5] = hsub2((y & 0x00030003u) | 0x64006400u, 0x64006400u);
-  h[6] = hsub2((y & 0x000C000Cu) | 0x5C005C00u, 0x5C005C00u);
-  h[7] = hsub2((y & 0x00300030u) | 0x54005400u, 0x54005400u);
-}
-
-// Four exact fp16x2 code pairs from a 4-bit word.
-__device__ __forceinline__ void unpack_word4(uint32_t x, uint32_t (&h)[4]) {
-  const uint32_t y = x >> 8;
-  h[0] = hsub2((x & 0x000F000Fu) | 0x64006400u, 0x64006400u);  // 1024 + c
-  h[1] = hsub2((x & 0x00F000F0u) | 0x54005400u, 0x54005400u);  // 64 + c
-  h[2] = hsub2((y & 0x000F000Fu) | 0x64006400u, 0x64006400u);
-  h[3] = hsub2((y & 0x00F000F0u) | 0x54005400u, 0x54005400u);
-}
-
-// Value codes are used centered, c - (2^b - 1)/2, so that sum_t p_t * sv * code does not carry the
-// group minimum's large offset (the offset moves into the group midpoint, see below). With 2-bit
-// codes the centered value is exact in fp16 after one subtraction of (2^(10-2k) + 1.5), except at
-// the pair positions whose constant is 1024 (spacing 1), which subtract 1024 and then 1.5.
-__device__ __forceinline__ void unpack_word2_centered(uint32_t x, uint32_t (&h)[8]) {
-  const uint32_t y = x >> 10;
-  h[0] = hsub2(hsub2((x & 0x00030003u) | 0x64006400u, 0x64006400u), 0x3E003E00u);  // c - 1.5
-  h[1] = hsub2((x & 0x000C000Cu) | 0x5C005C00u, 0x5C065C06u);                      // 256 + c - 257.5
-  h[2] = hsub2((x & 0x00300030u) | 0x54005400u, 0x54185418u);                      // 64 + c - 65.5
-  h[3] = hsub2((x & 0x00C000C0u) | 0x4C004C00u, 0x4C604C60u);                      // 16 + c - 17.5
-  h[4] = hsub2((x & 0x03000300u) | 0x44004400u, 0x45804580u);                      // 4 + c - 5.5
-  h[5] = hsub2(hsub2((y & 0x00030003u) | 0x64006400u, 0x64006400u), 0x3E003E00u);
-  h[6] = hsub2((y & 0x000C000Cu) | 0x5C005C00u, 0x5C065C06u);
-  h[7] = hsub2((y & 0x00300030u) | 0x54005400u, 0x54185418u);
-}
-
-// 4-bit codes centered at 7.5.
-__device__ __forceinline__ void unpack_word4_centered(uint32_t x, uint32_t (&h)[4]) {
-  const uint32_t y = x >> 8;
-  h[0] = hsub2(hsub2((x & 0x000F000Fu) | 0x64006400u, 0x64006400u), 0x47804780u);  // c - 7.5
-  h[1] = hsub2((x & 0x00F000F0u) | 0x54005400u, 0x54785478u);                      // 64 + c - 71.5
-  h[2] = hsub2(hsub2((y & 0x000F000Fu) | 0x64006400u, 0x64006400u), 0x47804780u);
-  h[3] = hsub2((y & 0x00F000F0u) | 0x54005400u, 0x54785478u);
-}
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                          uint32_t b1) {
@@ -113,18 +61,6 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
 }
-
-// hi keeps the leading 11 significant bits of x (exact in fp16 when x is in fp16's normal range),
-// lo = x - hi exactly; each fp16 column gets one of them.
-__device__ __forceinline__ float split_part(float x, bool lo) {
-  const float hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
-  return lo ? __fsub_rn(x, hi) : hi;
-}
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-  const __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 
 // Load 2*VPT consecutive fp16 (aligned to 4*VPT bytes) as floats.
 template <int VPT>
@@ -203,12 +139,6 @@ constexpr int decode_smem_bytes() {
   using S = typename Shape<KB, VB, VPT, GQ>::S;
   constexpr int ring = kDecodeWarps * S::kWarpBytes;
   return kSmemFixed + (ring > kSmemEpilogue ? ring : kSmemEpilogue);
-}
-
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
 }
 
 // cp.async of 16 bytes that writes zeros (and reads nothing) when `valid` is false.
@@ -783,7 +713,9 @@ int occupancy_vpt(int G, int gqa) {
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e;
-  if (a.key_bits == 2)
+  if (a.layout == KVQ_LAYOUT_ROWS_V2)
+    e = launch_decode_tc(a, stream);
+  else if (a.key_bits == 2)
     e = a.value_bits == 2 ? dispatch_vpt<2, 2>(a, stream) : dispatch_vpt<2, 4>(a, stream);
   else
     e = a.value_bits == 2 ? dispatch_vpt<4, 2>(a, stream) : dispatch_vpt<4, 4>(a, stream);

@@ -21,6 +21,8 @@ struct QuantizeArgs {
   uint16_t* v_res;
   int batch, num_kv_heads, G, R, key_bits, value_bits, hadamard;
   int64_t capacity, tiles, groups, ring;  // per unit: capacity tokens, capacity/16 tiles, capacity/G groups, R+G slots
+  int layout;                             // KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2
+  int64_t vwords;                         // value code words per unit
 };
 
 struct DecodeArgs {
@@ -38,17 +40,20 @@ struct DecodeArgs {
   float* part;             // split partials [units][nsplit][g][2 + 128]
   int batch, num_q_heads, num_kv_heads, gqa, G, R, key_bits, value_bits, hadamard;
   int64_t capacity, tiles, groups, ring;
-  int split_len;  // tokens per split (multiple of 64)
+  int layout;     // KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2
+  int split_len;  // tokens per split (multiple of 64; rows v2: multiple of 128)
   int nsplit;     // splits per unit in the grid
   float qscale;   // sm_scale * log2(e): scores are kept in base-2 units
 };
 
 cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream);
 cudaError_t launch_append(const QuantizeArgs& a, const uint16_t* k_new, const uint16_t* v_new, cudaStream_t stream);
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);     // split + combine, either layout
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // rows-v2 split kernel only
 int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);
 
 constexpr int kDecodeWarps = 4;
+constexpr int kTcCtasPerSm = 2;    // rows-v2 kernel: 256 TMEM columns per CTA
 constexpr int kPartFloats = 2 + 128;  // m, l, o[128]
 
 }  // namespace kvq

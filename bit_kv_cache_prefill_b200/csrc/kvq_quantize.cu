@@ -89,7 +89,8 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
     const uint32_t kmin = min(min(pmin[c], pmin[128 + c]), min(pmin[256 + c], pmin[384 + c]));
     const uint32_t kmax = max(max(pmax[c], pmax[128 + c]), max(pmax[256 + c], pmax[384 + c]));
     const QuantParams p = make_params(kmin, kmax, bits);
-    const int64_t pidx = (unit * a.groups + g) * kHeadDim + key_param_pos(c);
+    const int pos = a.layout == KVQ_LAYOUT_ROWS_V2 ? c : key_param_pos(c);  // rows v2: natural channel order
+    const int64_t pidx = (unit * a.groups + g) * kHeadDim + pos;
     a.k_scale[pidx] = p.s16;
     a.k_zero[pidx] = p.z16;
     prm[c] = make_float2(p.zf, p.inv);
@@ -97,6 +98,24 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
   __syncthreads();
   const int words = 64 * bits;
   const int P = 16 / bits;
+  if (a.layout == KVQ_LAYOUT_ROWS_V2) {
+    // one row of 4*bits words per token: pair j = P*w + k holds channels 2j, 2j + 1
+    const int wpt = 4 * bits;
+    uint32_t* dst2 = a.k_codes + (unit * a.capacity + t0) * wpt;
+    for (int idx = threadIdx.x; idx < G * wpt; idx += blockDim.x) {
+      const int i = idx / wpt, w = idx % wpt;
+      uint32_t word = 0;
+      for (int k = 0; k < P; ++k) {
+        const int c = 2 * (P * w + k);
+        const uint32_t x = *reinterpret_cast<const uint32_t*>(rows + i * kHeadDim + c);
+        const float4 pp = *reinterpret_cast<const float4*>(prm + c);
+        word |= code_with(static_cast<uint16_t>(x & 0xffffu), pp.x, pp.y, top) << (bits * k);
+        word |= code_with(static_cast<uint16_t>(x >> 16), pp.z, pp.w, top) << (16 + bits * k);
+      }
+      dst2[idx] = word;
+    }
+    return;
+  }
   uint32_t* dst = a.k_codes + (unit * a.tiles + t0 / kTile) * words;
   for (int idx = threadIdx.x; idx < (G / kTile) * words; idx += blockDim.x) {
     const int tile = idx / words, widx = idx % words;
@@ -150,6 +169,25 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
   __syncthreads();
   const int words = 64 * bits;
   const int P = 16 / bits;
+  if (a.layout == KVQ_LAYOUT_ROWS_V2) {
+    // the chunk lies inside one 128-token block; channel c's row of that block gets G / (2P) words
+    const int wpr = 4 * bits, wpc = G / (2 * P);
+    const int64_t block = t0 / 128;
+    const int ib = static_cast<int>(t0 % 128);
+    uint32_t* dst2 = a.v_codes + unit * a.vwords + block * 128 * wpr + (ib / 2) / P;
+    for (int idx = threadIdx.x; idx < kHeadDim * wpc; idx += blockDim.x) {
+      const int c = idx / wpc, w = idx % wpc;
+      uint32_t word = 0;
+      for (int k = 0; k < P; ++k) {
+        const int i0 = 2 * (P * w + k);  // chunk-relative token pair i0, i0 + 1
+        const float2 p0 = prm[i0 * vpt + c / G], p1 = prm[(i0 + 1) * vpt + c / G];
+        word |= code_with(rows[i0 * kHeadDim + c], p0.x, p0.y, top) << (bits * k);
+        word |= code_with(rows[(i0 + 1) * kHeadDim + c], p1.x, p1.y, top) << (16 + bits * k);
+      }
+      dst2[c * wpr + w] = word;
+    }
+    return;
+  }
   uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words;
   for (int idx = threadIdx.x; idx < (G / kTile) * words; idx += blockDim.x) {
     const int tile = idx / words, widx = idx % words;

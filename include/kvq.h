@@ -48,8 +48,10 @@ typedef enum {
   KVQ_ERR_CUDA = -5         /* a kernel launch or copy failed */
 } kvq_status;
 
-/* The only packed layout of this version ("tile v1"): see kvq_cache below. */
+/* Packed layouts (see kvq_cache below): "tile v1" feeds warp-level mma fragments, "rows v2" feeds
+ * the tcgen05 tensor cores (one token's key codes / one channel's value codes per row). */
 #define KVQ_LAYOUT_TILE_V1 1
+#define KVQ_LAYOUT_ROWS_V2 2
 
 /* Problem definition. Requirements checked by every entry point:
  *   batch >= 1; num_kv_heads >= 1; num_q_heads a multiple of num_kv_heads with
@@ -57,8 +59,9 @@ typedef enum {
  *   key_bits, value_bits in {2, 4};
  *   group_size G in {16, 32, 64, 128} (a multiple of the 16-token tile and a divisor of 128);
  *   residual R >= 0 (tokens kept in FP16 beyond the last full group; 0 <= R <= 4096);
- *   hadamard in {0, 1}; layout == KVQ_LAYOUT_TILE_V1;
- *   capacity >= 0, a multiple of G (maximum tokens per sequence). */
+ *   hadamard in {0, 1}; layout KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2;
+ *   capacity >= 0, a multiple of G (maximum tokens per sequence); with layout ROWS_V2 also a
+ *   multiple of 128 (value rows come in whole 128-token blocks). */
 typedef struct {
   int32_t batch;
   int32_t num_q_heads;
@@ -75,9 +78,12 @@ typedef struct {
 
 /* The packed cache: eight caller-owned device buffers plus the sequence lengths.
  * A "unit" is one (sequence b, KV head h); unit index u = b * num_kv_heads + h. Sizes per unit:
- *   k_codes  u32 [capacity/16][64*key_bits]     key codes, one 16-token tile per row
- *   v_codes  u32 [capacity/16][64*value_bits]   value codes, same tiling
- *   k_scale  fp16 [capacity/G][128]             per key group and channel (permuted channel order)
+ *   k_codes  u32 [capacity/16][64*key_bits]     tile v1: key codes, one 16-token tile per row
+ *            u32 [capacity][4*key_bits]         rows v2: one row of codes per token
+ *   v_codes  u32 [capacity/16][64*value_bits]   tile v1: value codes, same tiling
+ *            u32 [ceil(capacity/128)][128][4*value_bits]  rows v2: per 128-token block, one row per channel
+ *   k_scale  fp16 [capacity/G][128]             per key group and channel (tile v1: permuted channel
+ *                                               order as below; rows v2: natural order)
  *   k_zero   fp16 [capacity/G][128]             same; the zero-point is the group minimum
  *   v_scale  fp16 [capacity][128/G]             per token and channel group
  *   v_zero   fp16 [capacity][128/G]             same
@@ -97,6 +103,12 @@ typedef struct {
  *   values: token 16k + 2qd + 8hh + e,   channel 16m + r + 8u
  * Key scale/zero entry of channel c = 16m + 2qd + 8hh + e sits at index 32qd + 4m + 2hh + e.
  * (This order lets the decode kernel feed 16-byte loads straight into tensor-core fragments.)
+ *
+ * Rows v2 (P = 16/bits code pairs per u32 word; pair k of a word has its first code at bits
+ * [bits*k, bits*k + bits) and its second at bits [16 + bits*k, ...)):
+ *   keys:   token t's row holds channel pair j = c/2 in word j/P as pair j%P (channel 2j first);
+ *   values: token t lies in block t/128 at i = t%128; channel c's row of that block holds token
+ *           pair j = i/2 in word j/P as pair j%P (token 2j first).
  *
  * seq_len_host: int64 [batch] in host memory, read and updated by the library.
  * seq_len_dev:  int64 [batch] in device memory, the device mirror, updated on the stream.

@@ -52,7 +52,7 @@ class _CConfig(ctypes.Structure):
         ("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32), ("value_bits", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("residual", ctypes.c_int32), ("hadamard", ctypes.c_int32),
-        ("capacity", ctypes.c_int64),
+        ("layout", ctypes.c_int32), ("capacity", ctypes.c_int64),
     ]
 
 
@@ -77,6 +77,8 @@ def _declare(L: ctypes.CDLL) -> None:
     L.kvq_ref_quantize_group.argtypes = [P, I, I, P, P, P]
     L.kvq_ref_key_word_bit.argtypes = [I, I, I, P, P]
     L.kvq_ref_value_word_bit.argtypes = [I, I, I, P, P]
+    L.kvq_ref_key_word_bit_v2.argtypes = [I64, I, I, P, P]
+    L.kvq_ref_value_word_bit_v2.argtypes = [I64, I, I, P, P]
     L.kvq_ref_key_param_pos.argtypes = [I]
     L.kvq_ref_key_param_pos.restype = I
     L.kvq_ref_quantized_len.argtypes = [I64, I, I]
@@ -97,10 +99,11 @@ class Config:
     hadamard: int
     capacity: int
     head_dim: int = 128
+    layout: int = 1  # 1 = tile v1 (mma fragment order), 2 = rows v2 (token rows of keys, channel rows of values)
 
     def c(self) -> _CConfig:
         return _CConfig(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.key_bits,
-                        self.value_bits, self.group_size, self.residual, self.hadamard, self.capacity)
+                        self.value_bits, self.group_size, self.residual, self.hadamard, self.layout, self.capacity)
 
 
 class Cache:
@@ -109,8 +112,12 @@ class Cache:
     def __init__(self, cfg: Config):
         B, H, cap, G = cfg.batch, cfg.num_kv_heads, cfg.capacity, cfg.group_size
         ring = cfg.residual + G
-        self.k_codes = np.zeros((B, H, cap // 16, 64 * cfg.key_bits), np.uint32)
-        self.v_codes = np.zeros((B, H, cap // 16, 64 * cfg.value_bits), np.uint32)
+        if cfg.layout == 2:
+            self.k_codes = np.zeros((B, H, cap, 4 * cfg.key_bits), np.uint32)
+            self.v_codes = np.zeros((B, H, (cap + 127) // 128, 128, 4 * cfg.value_bits), np.uint32)
+        else:
+            self.k_codes = np.zeros((B, H, cap // 16, 64 * cfg.key_bits), np.uint32)
+            self.v_codes = np.zeros((B, H, cap // 16, 64 * cfg.value_bits), np.uint32)
         self.k_scale = np.zeros((B, H, cap // G, 128), np.uint16)
         self.k_zero = np.zeros((B, H, cap // G, 128), np.uint16)
         self.v_scale = np.zeros((B, H, cap, 128 // G), np.uint16)
@@ -216,6 +223,18 @@ def key_word_bit(i: int, c: int, bits: int):
 def value_word_bit(i: int, c: int, bits: int):
     w, b = ctypes.c_int(), ctypes.c_int()
     lib().kvq_ref_value_word_bit(i, c, bits, ctypes.byref(w), ctypes.byref(b))
+    return w.value, b.value
+
+
+def key_word_bit_v2(t: int, c: int, bits: int):
+    w, b = ctypes.c_int64(), ctypes.c_int()
+    lib().kvq_ref_key_word_bit_v2(t, c, bits, ctypes.byref(w), ctypes.byref(b))
+    return w.value, b.value
+
+
+def value_word_bit_v2(t: int, c: int, bits: int):
+    w, b = ctypes.c_int64(), ctypes.c_int()
+    lib().kvq_ref_value_word_bit_v2(t, c, bits, ctypes.byref(w), ctypes.byref(b))
     return w.value, b.value
 
 

@@ -34,7 +34,9 @@
 //      rounding, never fused.
 //  R6  dequant x^ = code * s16 + zero, evaluated here in fp64.
 //  R7  attention in fp64: no causal mask, no sink token, no RoPE; softmax over all T tokens.
-//  R8  packed layout "tile v1" (see key_word_bit / value_word_bit / key_param_pos below).
+//  R8  packed layouts "tile v1" (mma fragment order) and "rows v2" (one token's key codes, one
+//      channel's value codes per row); see key_word_bit / value_word_bit / key_param_pos and the
+//      v2 functions below.
 //
 // Build: g++ -O2 -std=c++17 -ffp-contract=off -fno-fast-math -fPIC -shared (x86-64 SSE scalar fp32).
 
@@ -220,6 +222,28 @@ int key_param_pos(int c) {
   return 32 * qd + 4 * m + 2 * h + e;
 }
 
+// Layout "rows v2". Keys: token t's codes form a row of 4*bits u32 words; channel pair j = c / 2
+// sits in word j / P (P = 16 / bits pairs per word) as pair k = j % P: channel 2j at bits
+// [bits*k, bits*k + bits), channel 2j + 1 at bits [16 + bits*k, ...). Values: tokens are cut into
+// blocks of 128; within a block, channel c's codes form a row of 4*bits words and token pair
+// j = i / 2 (i = t % 128) sits in word j / P as pair k = j % P (token 2j low, 2j + 1 high).
+// Key scale / zero keep the natural channel order.
+void key_word_bit_v2(int64_t t, int c, int bits, int64_t* word, int* bit) {
+  const int P = 16 / bits;
+  const int j = c / 2, e = c % 2;
+  *word = t * (4 * bits) + j / P;
+  *bit = bits * (j % P) + 16 * e;
+}
+
+void value_word_bit_v2(int64_t t, int c, int bits, int64_t* word, int* bit) {
+  const int P = 16 / bits;
+  const int64_t block = t / 128;
+  const int i = static_cast<int>(t % 128);
+  const int j = i / 2, e = i % 2;
+  *word = (block * 128 + c) * (4 * bits) + j / P;
+  *bit = bits * (j % P) + 16 * e;
+}
+
 }  // namespace
 
 // ================================================================================================
@@ -229,7 +253,7 @@ extern "C" {
 
 typedef struct {
   int32_t batch, num_q_heads, num_kv_heads, head_dim;
-  int32_t key_bits, value_bits, group_size, residual, hadamard;
+  int32_t key_bits, value_bits, group_size, residual, hadamard, layout;  // layout: 1 = tile v1, 2 = rows v2
   int64_t capacity;
 } kvq_ref_config;
 
@@ -256,6 +280,7 @@ static int check_config(const kvq_ref_config* c) {
   const int G = c->group_size;
   if (G <= 0 || G % 16 || 128 % G) return REF_ERR_ARG;
   if (c->residual < 0 || c->capacity < 0 || c->capacity % G) return REF_ERR_ARG;
+  if (c->layout != 1 && c->layout != 2) return REF_ERR_ARG;
   return REF_OK;
 }
 
@@ -264,14 +289,38 @@ static int64_t quantized_len(int64_t T, int R, int G) {
   return over > 0 ? (over / G) * G : 0;
 }
 
+// Word (within the unit's code buffer) and bit of the code of token t, channel ch, per layout.
+static void key_pos(const kvq_ref_config* c, int64_t t, int ch, int64_t* word, int* bit) {
+  if (c->layout == 2) {
+    key_word_bit_v2(t, ch, c->key_bits, word, bit);
+  } else {
+    int w;
+    key_word_bit(static_cast<int>(t % 16), ch, c->key_bits, &w, bit);
+    *word = (t / 16) * (64 * c->key_bits) + w;
+  }
+}
+static void value_pos(const kvq_ref_config* c, int64_t t, int ch, int64_t* word, int* bit) {
+  if (c->layout == 2) {
+    value_word_bit_v2(t, ch, c->value_bits, word, bit);
+  } else {
+    int w;
+    value_word_bit(static_cast<int>(t % 16), ch, c->value_bits, &w, bit);
+    *word = (t / 16) * (64 * c->value_bits) + w;
+  }
+}
+static int key_param_index(const kvq_ref_config* c, int ch) { return c->layout == 2 ? ch : key_param_pos(ch); }
+
 struct Dims {
   int64_t kw_tile, vw_tile, tiles, groups, ring, vpt;  // words per tile, tiles/unit, groups/unit, ring slots, value groups per token
+  int64_t kwords, vwords;                              // code words per unit
 };
 static Dims dims(const kvq_ref_config* c) {
   Dims d;
   d.kw_tile = 64 * c->key_bits;
   d.vw_tile = 64 * c->value_bits;
   d.tiles = c->capacity / 16;
+  d.kwords = c->capacity * 4 * c->key_bits;
+  d.vwords = (c->layout == 2 ? (c->capacity + 127) / 128 * 128 : c->capacity) * 4 * c->value_bits;
   d.groups = c->capacity / c->group_size;
   d.ring = c->residual + c->group_size;
   d.vpt = 128 / c->group_size;
@@ -289,18 +338,19 @@ static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, i
   const int64_t g = t0 / G;
   for (int ch = 0; ch < 128; ++ch) {
     GroupQ q = quantize_group(kt + ch, G, static_cast<int>(k_ld), c->key_bits, kc.data() + ch, 128);
-    const int pos = key_param_pos(ch);
+    const int pos = key_param_index(c, ch);
     cache->k_scale[(unit * d.groups + g) * 128 + pos] = q.scale;
     cache->k_zero[(unit * d.groups + g) * 128 + pos] = q.zero;
   }
+  uint32_t* kbuf = cache->k_codes + unit * d.kwords;
   for (int i = 0; i < G; ++i) {
     const int64_t t = t0 + i;
-    uint32_t* tile = cache->k_codes + (unit * d.tiles + t / 16) * d.kw_tile;
     for (int ch = 0; ch < 128; ++ch) {
-      int word, bit;
-      key_word_bit(static_cast<int>(t % 16), ch, c->key_bits, &word, &bit);
+      int64_t word;
+      int bit;
+      key_pos(c, t, ch, &word, &bit);
       const uint32_t mask = ((1u << c->key_bits) - 1u) << bit;
-      tile[word] = (tile[word] & ~mask) | (static_cast<uint32_t>(kc[i * 128 + ch]) << bit);
+      kbuf[word] = (kbuf[word] & ~mask) | (static_cast<uint32_t>(kc[i * 128 + ch]) << bit);
     }
   }
   // Values: per token over channel groups of G.
@@ -312,12 +362,13 @@ static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, i
       cache->v_scale[(unit * c->capacity + t) * d.vpt + j] = q.scale;
       cache->v_zero[(unit * c->capacity + t) * d.vpt + j] = q.zero;
     }
-    uint32_t* tile = cache->v_codes + (unit * d.tiles + t / 16) * d.vw_tile;
+    uint32_t* vbuf = cache->v_codes + unit * d.vwords;
     for (int ch = 0; ch < 128; ++ch) {
-      int word, bit;
-      value_word_bit(static_cast<int>(t % 16), ch, c->value_bits, &word, &bit);
+      int64_t word;
+      int bit;
+      value_pos(c, t, ch, &word, &bit);
       const uint32_t mask = ((1u << c->value_bits) - 1u) << bit;
-      tile[word] = (tile[word] & ~mask) | (static_cast<uint32_t>(vc[ch]) << bit);
+      vbuf[word] = (vbuf[word] & ~mask) | (static_cast<uint32_t>(vc[ch]) << bit);
     }
   }
 }
@@ -427,13 +478,14 @@ static void key_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t
     for (int ch = 0; ch < 128; ++ch) out[ch] = half_to_float(r[ch]);
     return;
   }
-  const uint32_t* tile = cache->k_codes + (unit * d.tiles + t / 16) * d.kw_tile;
+  const uint32_t* kbuf = cache->k_codes + unit * d.kwords;
   const int64_t g = t / c->group_size;
   for (int ch = 0; ch < 128; ++ch) {
-    int word, bit;
-    key_word_bit(static_cast<int>(t % 16), ch, c->key_bits, &word, &bit);
-    const uint32_t code = (tile[word] >> bit) & ((1u << c->key_bits) - 1u);
-    const int pos = key_param_pos(ch);
+    int64_t word;
+    int bit;
+    key_pos(c, t, ch, &word, &bit);
+    const uint32_t code = (kbuf[word] >> bit) & ((1u << c->key_bits) - 1u);
+    const int pos = key_param_index(c, ch);
     const double s = half_to_float(cache->k_scale[(unit * d.groups + g) * 128 + pos]);
     const double z = half_to_float(cache->k_zero[(unit * d.groups + g) * 128 + pos]);
     out[ch] = static_cast<double>(code) * s + z;
@@ -447,11 +499,12 @@ static void value_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64
     for (int ch = 0; ch < 128; ++ch) out[ch] = half_to_float(r[ch]);
     return;
   }
-  const uint32_t* tile = cache->v_codes + (unit * d.tiles + t / 16) * d.vw_tile;
+  const uint32_t* vbuf = cache->v_codes + unit * d.vwords;
   for (int ch = 0; ch < 128; ++ch) {
-    int word, bit;
-    value_word_bit(static_cast<int>(t % 16), ch, c->value_bits, &word, &bit);
-    const uint32_t code = (tile[word] >> bit) & ((1u << c->value_bits) - 1u);
+    int64_t word;
+    int bit;
+    value_pos(c, t, ch, &word, &bit);
+    const uint32_t code = (vbuf[word] >> bit) & ((1u << c->value_bits) - 1u);
     const int j = ch / c->group_size;
     const double s = half_to_float(cache->v_scale[(unit * c->capacity + t) * d.vpt + j]);
     const double z = half_to_float(cache->v_zero[(unit * c->capacity + t) * d.vpt + j]);
@@ -529,6 +582,8 @@ void kvq_ref_quantize_group(const uint16_t* x, int n, int bits, uint8_t* codes, 
 void kvq_ref_key_word_bit(int i, int c, int bits, int* word, int* bit) { key_word_bit(i, c, bits, word, bit); }
 void kvq_ref_value_word_bit(int i, int c, int bits, int* word, int* bit) { value_word_bit(i, c, bits, word, bit); }
 int kvq_ref_key_param_pos(int c) { return key_param_pos(c); }
+void kvq_ref_key_word_bit_v2(int64_t t, int c, int bits, int64_t* word, int* bit) { key_word_bit_v2(t, c, bits, word, bit); }
+void kvq_ref_value_word_bit_v2(int64_t t, int c, int bits, int64_t* word, int* bit) { value_word_bit_v2(t, c, bits, word, bit); }
 int64_t kvq_ref_quantized_len(int64_t T, int R, int G) { return quantized_len(T, R, G); }
 
 // Exhaustive check of the binary32 -> binary16 converter against the compiler's _Float16 conversion

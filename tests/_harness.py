@@ -15,16 +15,22 @@ MAX_ABS_TOL = 2e-3  # decode attention output, absolute
 REL_L2_TOL = 1e-3   # decode attention output, relative L2 over all compared outputs
 
 
-def oracle_config(oracle, w: inputs.Workload, batch=None, hq=None, hkv=None):
+def capacity(w: inputs.Workload, layout: int) -> int:
+    """Workload capacity, rounded up to whole 128-token blocks for the rows-v2 layout."""
+    cap = w.capacity()
+    return -(-cap // 128) * 128 if layout == 2 else cap
+
+
+def oracle_config(oracle, w: inputs.Workload, batch=None, hq=None, hkv=None, layout: int = 1):
     return oracle.Config(batch or w.batch, hq or w.num_q_heads, hkv or w.num_kv_heads, w.key_bits, w.value_bits,
-                         w.group_size, w.residual, w.hadamard, w.capacity())
+                         w.group_size, w.residual, w.hadamard, capacity(w, layout), layout=layout)
 
 
-def gpu_config(w: inputs.Workload):
+def gpu_config(w: inputs.Workload, layout: int = 1):
     import bit_kv_cache_prefill_b200 as kvq
 
     return kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size,
-                           w.residual, w.hadamard, w.capacity())
+                           w.residual, w.hadamard, capacity(w, layout), layout=layout)
 
 
 @dataclass
@@ -33,34 +39,44 @@ class GpuRun:
     cache: object
     out: torch.Tensor  # fp16 [B][Hq][128] on the device
     lens: np.ndarray
+    layout: int = 1
 
 
 def run_gpu(w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
-            appends: int = 0, sm_scale: Optional[float] = None) -> GpuRun:
-    """Prefill (k, v on the device), `appends` streaming appends, one decode."""
+            appends: int = 0, sm_scale: Optional[float] = None, layout: int = 1, decode: bool = True) -> GpuRun:
+    """Prefill (k, v on the device), `appends` streaming appends, one decode (unless decode=False)."""
     import bit_kv_cache_prefill_b200 as kvq
 
-    cfg = gpu_config(w)
+    cfg = gpu_config(w, layout)
     cache = kvq.Cache(cfg)
     kvq.kvq_quantize_prefill(cfg, cache, k, v, lens)
     for step in range(appends):
         kn, vn = inputs.append_tokens(w, step)
         kvq.kvq_append_token(cfg, cache, kn.cuda(), vn.cuda())
-    ws = torch.empty(kvq.kvq_decode_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
     out = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float16, device="cuda")
-    kvq.kvq_decode_attention(cfg, cache, q.cuda(), out, sm_scale or 1 / math.sqrt(128), ws)
+    if decode:
+        ws = torch.empty(kvq.kvq_decode_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+        kvq.kvq_decode_attention(cfg, cache, q.cuda(), out, sm_scale or 1 / math.sqrt(128), ws)
     torch.cuda.synchronize()
-    return GpuRun(cfg, cache, out, lens + appends)
+    return GpuRun(cfg, cache, out, lens + appends, layout)
+
+
+def code_shapes(w: inputs.Workload, layout: int):
+    B, H, cap = w.batch, w.num_kv_heads, capacity(w, layout)
+    if layout == 2:
+        return (B, H, cap, 4 * w.key_bits), (B, H, cap // 128, 128, 4 * w.value_bits)
+    return (B, H, cap // 16, 64 * w.key_bits), (B, H, cap // 16, 64 * w.value_bits)
 
 
 def gpu_views(w: inputs.Workload, run: GpuRun) -> Dict[str, np.ndarray]:
     """GPU cache buffers as numpy arrays with the oracle's shapes."""
-    B, H, cap, G = w.batch, w.num_kv_heads, w.capacity(), w.group_size
+    B, H, cap, G = w.batch, w.num_kv_heads, capacity(w, run.layout), w.group_size
     ring = w.residual + G
     c = run.cache
+    ks, vs = code_shapes(w, run.layout)
     return {
-        "k_codes": c.view("k_codes", torch.int32).cpu().numpy().view(np.uint32).reshape(B, H, cap // 16, 64 * w.key_bits),
-        "v_codes": c.view("v_codes", torch.int32).cpu().numpy().view(np.uint32).reshape(B, H, cap // 16, 64 * w.value_bits),
+        "k_codes": c.view("k_codes", torch.int32).cpu().numpy().view(np.uint32).reshape(ks),
+        "v_codes": c.view("v_codes", torch.int32).cpu().numpy().view(np.uint32).reshape(vs),
         "k_scale": c.view("k_scale", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, cap // G, 128),
         "k_zero": c.view("k_zero", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, cap // G, 128),
         "v_scale": c.view("v_scale", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, cap, 128 // G),
@@ -70,13 +86,23 @@ def gpu_views(w: inputs.Workload, run: GpuRun) -> Dict[str, np.ndarray]:
     }
 
 
-def compare_unit_cache(w: inputs.Workload, gv: Dict[str, np.ndarray], b: int, h: int, oc, ob: int, oh: int, T: int) -> None:
+def compare_unit_cache(w: inputs.Workload, gv: Dict[str, np.ndarray], b: int, h: int, oc, ob: int, oh: int, T: int,
+                       layout: int = 1) -> None:
     """Bit-exact comparison of everything that is defined for one unit of length T."""
     G, R = w.group_size, w.residual
     Q = max(T - R, 0) // G * G
     ring = R + G
-    np.testing.assert_array_equal(gv["k_codes"][b, h, : Q // 16], oc.k_codes[ob, oh, : Q // 16], err_msg=f"k_codes unit {b},{h}")
-    np.testing.assert_array_equal(gv["v_codes"][b, h, : Q // 16], oc.v_codes[ob, oh, : Q // 16], err_msg=f"v_codes unit {b},{h}")
+    if layout == 2:
+        np.testing.assert_array_equal(gv["k_codes"][b, h, :Q], oc.k_codes[ob, oh, :Q], err_msg=f"k_codes unit {b},{h}")
+        nb, rem = divmod(Q, 128)
+        np.testing.assert_array_equal(gv["v_codes"][b, h, :nb], oc.v_codes[ob, oh, :nb], err_msg=f"v_codes unit {b},{h}")
+        if rem:  # a partial block: only the words of the quantized token pairs are defined
+            words = rem * w.value_bits // 32
+            np.testing.assert_array_equal(gv["v_codes"][b, h, nb, :, :words], oc.v_codes[ob, oh, nb, :, :words],
+                                          err_msg=f"v_codes unit {b},{h} partial block")
+    else:
+        np.testing.assert_array_equal(gv["k_codes"][b, h, : Q // 16], oc.k_codes[ob, oh, : Q // 16], err_msg=f"k_codes unit {b},{h}")
+        np.testing.assert_array_equal(gv["v_codes"][b, h, : Q // 16], oc.v_codes[ob, oh, : Q // 16], err_msg=f"v_codes unit {b},{h}")
     np.testing.assert_array_equal(gv["k_scale"][b, h, : Q // G], oc.k_scale[ob, oh, : Q // G], err_msg=f"k_scale unit {b},{h}")
     np.testing.assert_array_equal(gv["k_zero"][b, h, : Q // G], oc.k_zero[ob, oh, : Q // G], err_msg=f"k_zero unit {b},{h}")
     np.testing.assert_array_equal(gv["v_scale"][b, h, :Q], oc.v_scale[ob, oh, :Q], err_msg=f"v_scale unit {b},{h}")
@@ -98,8 +124,8 @@ def check_attention(gpu_out: np.ndarray, ref: np.ndarray, what: str) -> Tuple[fl
 
 
 def oracle_full(oracle, w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
-                appends: int = 0, sm_scale: Optional[float] = None, threads: int = 8):
-    ocfg = oracle_config(oracle, w)
+                appends: int = 0, sm_scale: Optional[float] = None, threads: int = 8, layout: int = 1):
+    ocfg = oracle_config(oracle, w, layout=layout)
     oc = oracle.Cache(ocfg)
     oracle.quantize_prefill(ocfg, oc, k.numpy(), v.numpy(), lens, threads=threads)
     for step in range(appends):
@@ -110,10 +136,10 @@ def oracle_full(oracle, w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, le
 
 
 def oracle_unit(oracle, w: inputs.Workload, b: int, h: int, T0: int, q: torch.Tensor, appends: int = 0,
-                sm_scale: Optional[float] = None, threads: int = 4):
+                sm_scale: Optional[float] = None, threads: int = 4, layout: int = 1):
     """Oracle on the (sequence b, KV head h) sub-problem only (batch 1, one KV head, its g query heads)."""
     g = w.gqa
-    ocfg = oracle_config(oracle, w, batch=1, hq=g, hkv=1)
+    ocfg = oracle_config(oracle, w, batch=1, hq=g, hkv=1, layout=layout)
     oc = oracle.Cache(ocfg)
     ku, vu = inputs.unit_kv(w, b, h, T0)
     oracle.quantize_prefill(ocfg, oc, ku.numpy()[None, :, None, :], vu.numpy()[None, :, None, :], [T0])

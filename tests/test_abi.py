@@ -50,6 +50,24 @@ def test_buffer_bytes_closed_form(B, Hq, Hkv, kb, vb, G, R, cap):
     assert kvq.kvq_decode_workspace_bytes(cfg) > 0
 
 
+@pytest.mark.parametrize("cap", [4096, 4224, 1 << 20])
+def test_buffer_bytes_rows_v2(cap):
+    cfg = kvq.make_config(3, 8, 2, 4, 2, 32, 64, 0, cap, layout=kvq.KVQ_LAYOUT_ROWS_V2)
+    got = kvq.kvq_cache_buffer_bytes(cfg)
+    u = 3 * 2
+    vcap = -(-cap // 128) * 128  # value rows come in whole 128-token blocks
+    assert got[0] == u * cap * 4 * 4 * 4 and got[1] == u * vcap * 4 * 2 * 4
+    assert got[2:] == kvq.kvq_cache_buffer_bytes(kvq.make_config(3, 8, 2, 4, 2, 32, 64, 0, cap))[2:]
+
+
+def test_rows_v2_needs_whole_128_token_blocks():
+    sizes = (ctypes.c_size_t * 8)()
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1056, layout=kvq.KVQ_LAYOUT_ROWS_V2)
+    assert _status("kvq_cache_buffer_bytes", ctypes.byref(cfg), sizes) == kvq.KVQ_ERR_INVALID_ARG
+    cfg.layout = kvq.KVQ_LAYOUT_TILE_V1
+    assert _status("kvq_cache_buffer_bytes", ctypes.byref(cfg), sizes) == kvq.KVQ_OK
+
+
 def _status(fn, *args):
     return getattr(_lib.lib, fn)(*args)
 
@@ -60,7 +78,8 @@ def _status(fn, *args):
     ("group_size", 256, kvq.KVQ_ERR_INVALID_ARG), ("num_q_heads", 33, kvq.KVQ_ERR_INVALID_ARG),
     ("num_q_heads", 64, kvq.KVQ_ERR_UNSUPPORTED), ("residual", -1, kvq.KVQ_ERR_INVALID_ARG),
     ("hadamard", 2, kvq.KVQ_ERR_INVALID_ARG), ("capacity", 100, kvq.KVQ_ERR_INVALID_ARG),
-    ("layout", 2, kvq.KVQ_ERR_UNSUPPORTED), ("batch", 0, kvq.KVQ_ERR_INVALID_ARG),
+    ("layout", 3, kvq.KVQ_ERR_UNSUPPORTED), ("layout", 0, kvq.KVQ_ERR_UNSUPPORTED),
+    ("batch", 0, kvq.KVQ_ERR_INVALID_ARG),
 ])
 def test_config_validation(field, value, status):
     cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024)

@@ -57,18 +57,22 @@ def _inputs_for(w, lens):
     return k, v
 
 
+LAYOUTS = [1, 2]  # tile v1 (mma.sync kernel), rows v2 (tcgen05 kernel)
+
+
+@pytest.mark.parametrize("layout", LAYOUTS, ids=["tile_v1", "rows_v2"])
 @pytest.mark.parametrize("name,w,lens", SMALL, ids=[s[0] for s in SMALL])
-def test_small_prefill_bit_exact_and_decode(oracle_mod, name, w, lens):
+def test_small_prefill_bit_exact_and_decode(oracle_mod, name, w, lens, layout):
     w = _lens_workload(w, lens)
     lens = np.array(lens, np.int64)
     k, v = _inputs_for(w, lens)
     q = inputs.query(w)
-    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q)
-    oc, ref = H.oracle_full(oracle_mod, w, k, v, lens, q)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, layout=layout)
+    oc, ref = H.oracle_full(oracle_mod, w, k, v, lens, q, layout=layout)
     gv = H.gpu_views(w, run)
     for b in range(w.batch):
         for h in range(w.num_kv_heads):
-            H.compare_unit_cache(w, gv, b, h, oc, b, h, int(lens[b]))
+            H.compare_unit_cache(w, gv, b, h, oc, b, h, int(lens[b]), layout=layout)
     H.check_attention(run.out.cpu().numpy(), ref, name)
     # empty sequences decode to exact zeros
     for b in range(w.batch):
@@ -81,20 +85,21 @@ def test_small_prefill_bit_exact_and_decode(oracle_mod, name, w, lens):
     dict(w=W("s2", 2, 2, 2, 4, 2, 16, 0, 1, 100, seed=22), T0=100, n=40),
     dict(w=W("s3", 1, 4, 1, 2, 2, 64, 128, 0, 10, seed=23), T0=10, n=200),
 ], ids=["g32_r32_gqa4", "g16_r0_wht", "g64_r128_from_window"])
-def test_streaming_append_matches_oracle_and_bulk_prefill(oracle_mod, case):
+@pytest.mark.parametrize("layout", LAYOUTS, ids=["tile_v1", "rows_v2"])
+def test_streaming_append_matches_oracle_and_bulk_prefill(oracle_mod, case, layout):
     w, T0, n = case["w"], case["T0"], case["n"]
     w = w.scaled(seq_len=T0, appends=n)
     lens = np.full(w.batch, T0, np.int64)
     k, v = _inputs_for(w, list(lens))
     q = inputs.query(w)
-    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, appends=n)
-    oc, ref = H.oracle_full(oracle_mod, w, k, v, lens, q, appends=n)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, appends=n, layout=layout)
+    oc, ref = H.oracle_full(oracle_mod, w, k, v, lens, q, appends=n, layout=layout)
     gv = H.gpu_views(w, run)
     assert np.array_equal(run.cache.seq_len_host, lens + n)
     assert np.array_equal(run.cache.seq_len_dev.cpu().numpy(), lens + n)
     for b in range(w.batch):
         for h in range(w.num_kv_heads):
-            H.compare_unit_cache(w, gv, b, h, oc, b, h, T0 + n)
+            H.compare_unit_cache(w, gv, b, h, oc, b, h, T0 + n, layout=layout)
     H.check_attention(run.out.cpu().numpy(), ref, "streaming")
     # the GPU's own bulk prefill of all T0 + n tokens gives the same defined bits
     kk = torch.zeros(w.batch, T0 + n, w.num_kv_heads, 128, dtype=torch.float16)
@@ -103,14 +108,21 @@ def test_streaming_append_matches_oracle_and_bulk_prefill(oracle_mod, case):
     for s in range(n):
         kn, vn = inputs.append_tokens(w, s)
         kk[:, T0 + s], vv[:, T0 + s] = kn, vn
-    bulk = H.run_gpu(w, kk.cuda(), vv.cuda(), np.full(w.batch, T0 + n, np.int64), q)
+    bulk = H.run_gpu(w, kk.cuda(), vv.cuda(), np.full(w.batch, T0 + n, np.int64), q, layout=layout)
     gb = H.gpu_views(w, bulk)
     G, R = w.group_size, w.residual
     T = T0 + n
     Q = max(T - R, 0) // G * G
     live = [t % (R + G) for t in range(Q, T)]
-    for key in ("k_codes", "v_codes"):
-        np.testing.assert_array_equal(gv[key][:, :, : Q // 16], gb[key][:, :, : Q // 16])
+    if layout == 2:
+        np.testing.assert_array_equal(gv["k_codes"][:, :, :Q], gb["k_codes"][:, :, :Q])
+        nb, rem = divmod(Q, 128)
+        np.testing.assert_array_equal(gv["v_codes"][:, :, :nb], gb["v_codes"][:, :, :nb])
+        words = rem * w.value_bits // 32
+        np.testing.assert_array_equal(gv["v_codes"][:, :, nb:nb + 1, :, :words], gb["v_codes"][:, :, nb:nb + 1, :, :words])
+    else:
+        for key in ("k_codes", "v_codes"):
+            np.testing.assert_array_equal(gv[key][:, :, : Q // 16], gb[key][:, :, : Q // 16])
     for key in ("k_scale", "k_zero"):
         np.testing.assert_array_equal(gv[key][:, :, : Q // G], gb[key][:, :, : Q // G])
     for key in ("v_scale", "v_zero"):
@@ -120,19 +132,20 @@ def test_streaming_append_matches_oracle_and_bulk_prefill(oracle_mod, case):
     np.testing.assert_array_equal(run.out.cpu().numpy(), bulk.out.cpu().numpy())
 
 
-def test_sm_scale_and_single_token(oracle_mod):
+@pytest.mark.parametrize("layout", LAYOUTS, ids=["tile_v1", "rows_v2"])
+def test_sm_scale_and_single_token(oracle_mod, layout):
     w = W("one", 1, 4, 1, 2, 2, 32, 4, 0, 1, seed=31)
     lens = np.array([1], np.int64)
     k, v = _inputs_for(w, [1])
     q = inputs.query(w)
-    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, sm_scale=0.37)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, sm_scale=0.37, layout=layout)
     # one token: every head returns that token's value exactly (as fp16)
     for h in range(4):
         np.testing.assert_array_equal(run.out[0, h].cpu().numpy(), v[0, 0, 0].numpy())
     w2 = W("scl", 1, 4, 1, 2, 2, 32, 32, 0, 700, seed=32)
     k2, v2 = _inputs_for(w2, [700])
     q2 = inputs.query(w2)
-    run2 = H.run_gpu(w2, k2.cuda(), v2.cuda(), np.array([700]), q2, sm_scale=0.02)
+    run2 = H.run_gpu(w2, k2.cuda(), v2.cuda(), np.array([700]), q2, sm_scale=0.02, layout=layout)
     _, ref2 = H.oracle_full(oracle_mod, w2, k2, v2, np.array([700]), q2, sm_scale=0.02)
     H.check_attention(run2.out.cpu().numpy(), ref2, "sm_scale 0.02")
 
@@ -151,19 +164,20 @@ def _sample_units(w, lens):
     return sorted(picks)
 
 
+@pytest.mark.parametrize("layout", LAYOUTS, ids=["tile_v1", "rows_v2"])
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_workload_sampled(oracle_mod, name):
+def test_full_size_workload_sampled(oracle_mod, name, layout):
     w = inputs.WORKLOADS[name]
     k, v, lens = inputs.full_kv(w)
     q = inputs.query(w)
-    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, appends=w.appends)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, appends=w.appends, layout=layout)
     del k, v
     gv = H.gpu_views(w, run)
     out = run.out.cpu().numpy()
     refs, gots = [], []
     for b, h in _sample_units(w, lens):
-        oc, ref = H.oracle_unit(oracle_mod, w, b, h, int(lens[b]), q, appends=w.appends)
-        H.compare_unit_cache(w, gv, b, h, oc, 0, 0, int(lens[b]) + w.appends)
+        oc, ref = H.oracle_unit(oracle_mod, w, b, h, int(lens[b]), q, appends=w.appends, layout=layout)
+        H.compare_unit_cache(w, gv, b, h, oc, 0, 0, int(lens[b]) + w.appends, layout=layout)
         got = out[b, h * w.gqa:(h + 1) * w.gqa]
         H.check_attention(got, ref, f"{name} unit ({b},{h})")
         refs.append(ref)

@@ -47,6 +47,10 @@ MUTANTS = [
     ("residual_window_rounded_up",
      "return over > 0 ? (over / G) * G : 0;", "return over > 0 ? ((over + G - 1) / G) * G : 0;",
      ["test_quantized_attention_equals_library_attention_on_dequantized_cache"]),
+    ("rows_v2_value_words_swapped",
+     "  *word = (block * 128 + c) * (4 * bits) + j / P;",
+     "  *word = (block * 128 + c) * (4 * bits) + ((j / P) ^ 1);",
+     ["test_layout_matches_hand_worked_examples"]),
     ("value_group_index_off",
      "    const int j = ch / c->group_size;", "    const int j = (ch / c->group_size + 1) % d.vpt;",
      ["test_quantized_attention_equals_library_attention_on_dequantized_cache"]),
@@ -74,7 +78,7 @@ def _run_pin(fn_name, mod):
         "test_quantizer_invariants": [dict(bits=2, G=32), dict(bits=4, G=16)],
         "test_quantizer_two_valued_and_grid_round_trip": [dict(bits=2), dict(bits=4)],
         "test_quantized_attention_equals_library_attention_on_dequantized_cache":
-            [dict(kb=2, vb=2, G=32, R=32, had=0)],
+            [dict(kb=2, vb=2, G=32, R=32, had=0, layout=1), dict(kb=2, vb=2, G=32, R=32, had=0, layout=2)],
     }.get(fn_name, [dict()])
     for kw in params:
         fn(mod, **kw)

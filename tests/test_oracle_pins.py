@@ -210,13 +210,17 @@ def _golden_layout():
 def test_layout_matches_hand_worked_examples(oracle_mod):
     rows = _golden_layout()
     assert len(rows) > 20
+    kinds = set()
     for r in rows:
+        kinds.add(r[0])
         if r[0] == "kparam":
             assert oracle_mod.key_param_pos(int(r[1])) == int(r[2]), r
             continue
         kind, bits, i, c, word, bit = r[0], int(r[1]), int(r[2]), int(r[3]), int(r[4]), int(r[5])
-        fn = oracle_mod.key_word_bit if kind == "key" else oracle_mod.value_word_bit
+        fn = {"key": oracle_mod.key_word_bit, "value": oracle_mod.value_word_bit,
+              "key_v2": oracle_mod.key_word_bit_v2, "value_v2": oracle_mod.value_word_bit_v2}[kind]
         assert fn(i, c, bits) == (word, bit), r
+    assert kinds == {"key", "value", "kparam", "key_v2", "value_v2"}
 
 
 @pytest.mark.parametrize("kind", ["key", "value"])
@@ -234,11 +238,25 @@ def test_layout_is_a_bijection_onto_the_tile(oracle_mod, kind, bits):
     assert pos == list(range(128))
 
 
+@pytest.mark.parametrize("kind", ["key", "value"])
+@pytest.mark.parametrize("bits", [2, 4])
+def test_layout_v2_is_a_bijection_onto_rows(oracle_mod, kind, bits):
+    # one 128-token block of one unit: every code bit is used exactly once
+    fn = oracle_mod.key_word_bit_v2 if kind == "key" else oracle_mod.value_word_bit_v2
+    used = np.zeros(128 * 4 * bits * 32, np.int32)
+    for t in range(128):
+        for c in range(128):
+            w, b = fn(t, c, bits)
+            assert 0 <= w < 128 * 4 * bits and b % bits == 0 and b + bits <= 32
+            used[w * 32 + b: w * 32 + b + bits] += 1
+    assert np.all(used == 1)
+
+
 # --------------------------------------------------------------------------------------------------
 # whole-cache behaviour
 # --------------------------------------------------------------------------------------------------
-def _cfg(oracle_mod, B=2, Hq=4, Hkv=2, kb=2, vb=2, G=32, R=32, had=0, cap=512):
-    return oracle_mod.Config(B, Hq, Hkv, kb, vb, G, R, had, cap)
+def _cfg(oracle_mod, B=2, Hq=4, Hkv=2, kb=2, vb=2, G=32, R=32, had=0, cap=512, layout=1):
+    return oracle_mod.Config(B, Hq, Hkv, kb, vb, G, R, had, cap, layout=layout)
 
 
 def _inputs(B, T, Hkv, Hq, seed, outliers=True):
@@ -252,31 +270,45 @@ def _inputs(B, T, Hkv, Hq, seed, outliers=True):
     return k.half().numpy(), v.half().numpy(), q.half().numpy()
 
 
+def _key_code(oracle_mod, cfg, cache, b, h, t, c):
+    if cfg.layout == 2:
+        w, bit = oracle_mod.key_word_bit_v2(t, c, cfg.key_bits)
+        word = cache.k_codes[b, h].reshape(-1)[w]
+    else:
+        w, bit = oracle_mod.key_word_bit(t % 16, c, cfg.key_bits)
+        word = cache.k_codes[b, h, t // 16][w]
+    return (int(word) >> bit) & ((1 << cfg.key_bits) - 1)
+
+
+def _value_code(oracle_mod, cfg, cache, b, h, t, c):
+    if cfg.layout == 2:
+        w, bit = oracle_mod.value_word_bit_v2(t, c, cfg.value_bits)
+        word = cache.v_codes[b, h].reshape(-1)[w]
+    else:
+        w, bit = oracle_mod.value_word_bit(t % 16, c, cfg.value_bits)
+        word = cache.v_codes[b, h, t // 16][w]
+    return (int(word) >> bit) & ((1 << cfg.value_bits) - 1)
+
+
 def _unpack_key(oracle_mod, cfg, cache, b, h, t):
     """Dequantize key (b, h, t) from the cache by reading the layout positions the fixture pins."""
     G = cfg.group_size
-    tile = cache.k_codes[b, h, t // 16]
     s = cache.k_scale[b, h, t // G].view(np.float16).astype(np.float64)
     z = cache.k_zero[b, h, t // G].view(np.float16).astype(np.float64)
     out = np.empty(128)
     for c in range(128):
-        w, bit = oracle_mod.key_word_bit(t % 16, c, cfg.key_bits)
-        code = (int(tile[w]) >> bit) & ((1 << cfg.key_bits) - 1)
-        p = oracle_mod.key_param_pos(c)
-        out[c] = code * s[p] + z[p]
+        p = oracle_mod.key_param_pos(c) if cfg.layout == 1 else c
+        out[c] = _key_code(oracle_mod, cfg, cache, b, h, t, c) * s[p] + z[p]
     return out
 
 
 def _unpack_value(oracle_mod, cfg, cache, b, h, t):
     G = cfg.group_size
-    tile = cache.v_codes[b, h, t // 16]
     s = cache.v_scale[b, h, t].view(np.float16).astype(np.float64)
     z = cache.v_zero[b, h, t].view(np.float16).astype(np.float64)
     out = np.empty(128)
     for c in range(128):
-        w, bit = oracle_mod.value_word_bit(t % 16, c, cfg.value_bits)
-        code = (int(tile[w]) >> bit) & ((1 << cfg.value_bits) - 1)
-        out[c] = code * s[c // G] + z[c // G]
+        out[c] = _value_code(oracle_mod, cfg, cache, b, h, t, c) * s[c // G] + z[c // G]
     return out
 
 
@@ -328,11 +360,12 @@ def test_hadamard_no_quantization_equals_rotated_attention(oracle_mod):
     np.testing.assert_allclose(out, ref_unrot, atol=2e-3)
 
 
+@pytest.mark.parametrize("layout", [1, 2])
 @pytest.mark.parametrize("kb,vb,G,R,had", [(2, 2, 32, 32, 0), (4, 2, 32, 0, 1), (2, 4, 64, 100, 0), (4, 4, 16, 16, 1)])
-def test_quantized_attention_equals_library_attention_on_dequantized_cache(oracle_mod, kb, vb, G, R, had):
+def test_quantized_attention_equals_library_attention_on_dequantized_cache(oracle_mod, kb, vb, G, R, had, layout):
     B, Hkv, Hq = 2, 2, 4
     lens = [301, 160]
-    cfg = _cfg(oracle_mod, B, Hq, Hkv, kb, vb, G, R, had, cap=320)
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, kb, vb, G, R, had, cap=320, layout=layout)
     k, v, q = _inputs(B, max(lens), Hkv, Hq, 13 + kb + G)
     cache = oracle_mod.Cache(cfg)
     oracle_mod.quantize_prefill(cfg, cache, k, v, lens)
@@ -396,12 +429,13 @@ def test_tiny_case_against_long_double_brute_force(oracle_mod):
     np.testing.assert_allclose(out[0, 0], ref.astype(np.float64), rtol=1e-13, atol=1e-14)
 
 
+@pytest.mark.parametrize("layout", [1, 2])
 @pytest.mark.parametrize("kb,vb,G,R,had", [(2, 2, 32, 32, 0), (4, 2, 32, 0, 1), (2, 2, 64, 128, 0), (4, 4, 16, 5, 0)])
-def test_streaming_append_equals_bulk_prefill(oracle_mod, kb, vb, G, R, had):
+def test_streaming_append_equals_bulk_prefill(oracle_mod, kb, vb, G, R, had, layout):
     B, Hkv, Hq = 2, 2, 2
     T0, n = 150, 3 * G + 7
     cap = ((T0 + n + G - 1) // G) * G
-    cfg = _cfg(oracle_mod, B, Hq, Hkv, kb, vb, G, R, had, cap=cap)
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, kb, vb, G, R, had, cap=cap, layout=layout)
     k, v, _ = _inputs(B, T0 + n, Hkv, Hq, 16 + G)
     stream = oracle_mod.Cache(cfg)
     oracle_mod.quantize_prefill(cfg, stream, k[:, :T0], v[:, :T0], [T0, T0])
@@ -412,8 +446,15 @@ def test_streaming_append_equals_bulk_prefill(oracle_mod, kb, vb, G, R, had):
     T = T0 + n
     Q = max(T - R, 0) // G * G
     assert np.array_equal(stream.seq_len, bulk.seq_len)
-    np.testing.assert_array_equal(stream.k_codes[:, :, : Q // 16], bulk.k_codes[:, :, : Q // 16])
-    np.testing.assert_array_equal(stream.v_codes[:, :, : Q // 16], bulk.v_codes[:, :, : Q // 16])
+    if layout == 1:
+        np.testing.assert_array_equal(stream.k_codes[:, :, : Q // 16], bulk.k_codes[:, :, : Q // 16])
+        np.testing.assert_array_equal(stream.v_codes[:, :, : Q // 16], bulk.v_codes[:, :, : Q // 16])
+    else:
+        np.testing.assert_array_equal(stream.k_codes[:, :, :Q], bulk.k_codes[:, :, :Q])
+        per_word = 32 // vb  # tokens covered by one value word
+        for t0 in range(0, Q, 128):
+            nw = (min(Q, t0 + 128) - t0) // per_word
+            np.testing.assert_array_equal(stream.v_codes[:, :, t0 // 128, :, :nw], bulk.v_codes[:, :, t0 // 128, :, :nw])
     np.testing.assert_array_equal(stream.k_scale[:, :, : Q // G], bulk.k_scale[:, :, : Q // G])
     np.testing.assert_array_equal(stream.k_zero[:, :, : Q // G], bulk.k_zero[:, :, : Q // G])
     np.testing.assert_array_equal(stream.v_scale[:, :, :Q], bulk.v_scale[:, :, :Q])
