@@ -24,10 +24,13 @@
 //   Online softmax: one running max per head for the CTA; O, l and the midpoint sums are rescaled
 //   only in a step where some score exceeds it (a CTA vote), so p <= 1 always.
 // Pipeline: one elected thread streams each step's key rows, value block, value scale / zero and
-// key scale / zero with bulk async copies into a 3-4 stage ring (one mbarrier per stage) and issues
-// QK(i+1) and PV(i) after the step's barrier; each MMA batch signals its own mbarrier through
-// tcgen05.commit. While the tensor cores run, the token warps do the softmax of step i and unpack
-// keys of step i+1, the channel warps build B_QK of step i+1 and unpack values of step i.
+// key scale / zero with bulk async copies into a 4-8 stage ring (one mbarrier per stage) and issues
+// the MMAs; each MMA batch signals an mbarrier through tcgen05.commit. The key side runs two steps
+// ahead: A_K, B_QK and S are double-buffered, so in iteration i the token warps read S(i) (issued two
+// iterations earlier), write B_PV(i) and unpack the keys of step i + 2, while the channel warps build
+// B_QK(i + 2) and unpack the values of step i. One CTA barrier per step carries the vote on a new
+// maximum; only a step that raises it takes a second barrier (rescale and redo its probabilities).
+// Configs whose columns fit 256 TMEM columns run two CTAs per SM, the others one CTA with 512.
 // Every wait is bounded; a CTA that gives up on a wait marks its partial (l = NaN), so the affected
 // outputs read NaN instead of the kernel hanging.
 #include <cuda_runtime.h>
@@ -42,9 +45,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kStep = 128;  // tokens per step
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColAK = 0, kColAV = 64, kColS = 128, kColO = 192;
-constexpr int kWaitIters = 1 << 22;
+constexpr uint32_t kWaitSliceNs = 1000000;  // 1 ms
+constexpr int kWaitSlices = 2000;
 constexpr int kPartStride = 132;  // shared-memory partial: m, l, 2 pad, o[128] (16-byte aligned)
 constexpr int kPartO = 4;
 constexpr unsigned kAll = 0xffffffffu;
@@ -55,19 +57,22 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
+// try_wait with a suspend-time hint: the thread sleeps until the phase completes or about
+// kWaitSliceNs elapse, instead of spinning on the barrier.
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\nselp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitSliceNs)
       : "memory");
   return ok != 0;
 }
-// Bounded wait on an mbarrier phase. Gives up (and raises the CTA's abort flag) after kWaitIters
-// polls, or at once when another thread of the CTA has already given up.
+// Bounded wait on an mbarrier phase: at most kWaitSlices sleeps of up to kWaitSliceNs each (about 2 s
+// in all). Gives up (and raises the CTA's abort flag) after that, or at once when another thread of
+// the CTA has already given up.
 __device__ __forceinline__ void mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  for (int it = 0; it < kWaitIters; ++it) {
+  for (int it = 0; it < kWaitSlices; ++it) {
     if (mbar_try(bar, parity)) return;
     if (*abort_flag) return;
   }
@@ -177,13 +182,17 @@ __device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t (&r)[16]) {
       : "memory");
 }
 
-// ---- shared-memory plan ------------------------------------------------------------------------------
+// ---- shared-memory and TMEM plan -----------------------------------------------------------------------
 template <int KB, int VB, int VPT, int GQ>
 struct TcPlan {
   static constexpr int G = 128 / VPT;
   static constexpr int kUsedCols = VPT * GQ * 2;  // B columns in use, QK and PV alike (128/G = VPT groups per step)
   static constexpr int kN = kUsedCols < 16 ? 16 : kUsedCols;
   static constexpr int kChunks = (kUsedCols + 7) / 8;  // 16-byte chunks per B row written
+  // TMEM columns: A_K double-buffered (steps of even / odd index), A_V, S double-buffered, O.
+  static constexpr uint32_t kColAK = 0, kColAV = 128, kColS = 192, kColO = 192 + 2 * kN;
+  static constexpr uint32_t kTmemCols = kColO + kN <= 256 ? 256 : 512;
+  static constexpr int kCtasPerSm = 512 / kTmemCols;
   // One stage: everything a step reads from the cache.
   static constexpr int kKC = kStep * 16 * KB;  // key rows of 128 tokens
   static constexpr int kVC = 128 * 16 * VB;    // value rows of 128 channels (one 128-token block)
@@ -191,26 +200,32 @@ struct TcPlan {
   static constexpr int kKS = VPT * 256;        // key scale of the step's groups (key zero: same)
   static constexpr int oKC = 0, oVC = oKC + kKC, oVS = oVC + kVC, oVZ = oVS + kVS, oKS = oVZ + kVS, oKZ = oKS + kKS;
   static constexpr int kStageBytes = oKZ + kKS;
-  static constexpr int kStages = kStageBytes <= 16384 ? 4 : 3;
+  static constexpr int kStageBudget = kCtasPerSm == 2 ? 64 * 1024 : 144 * 1024;
+  static constexpr int kStagesRaw = kStageBudget / kStageBytes;
+  static constexpr int kStages = kStagesRaw < 4 ? 4 : (kStagesRaw > 8 ? 8 : kStagesRaw);
   static constexpr int kB = 128 * kN * 2;  // one B operand
-  static constexpr int oBQK = kStages * kStageBytes;
-  static constexpr int oBPV = oBQK + kB;
-  static constexpr int oQ = oBPV + kB;                 // q~ [GQ][128] f32
-  static constexpr int oQH = oQ + GQ * 512;            // q^ [GQ][128] f32
-  static constexpr int oBias = oQH + GQ * 512;         // [2][VPT * GQ] f32, by step parity
-  static constexpr int oRed = oBias + 2 * VPT * GQ * 4;  // [4][GQ] f32 warp maxima
-  static constexpr int oE = oRed + 4 * GQ * 4;         // [4] i32 per-head exponents
-  static constexpr int oBar = oE + 16;                 // mbarriers: qk, pv, stage[kStages]
-  static constexpr int oTmem = oBar + 8 * (2 + kStages);
+  static constexpr int oBQK = kStages * kStageBytes;  // [2] (by step parity)
+  static constexpr int oBPV = oBQK + 2 * kB;
+  static constexpr int oQ = oBPV + kB;                   // q~ [GQ][128] f32
+  static constexpr int oQH = oQ + GQ * 512;              // q^ [GQ][128] f32
+  static constexpr int oBias = oQH + GQ * 512;           // [4][VPT * GQ] f32, by step index mod 4
+  static constexpr int oRed = oBias + 4 * VPT * GQ * 4;  // [4][GQ] f32 warp maxima
+  static constexpr int oE = oRed + 4 * GQ * 4;           // [4] i32 per-head exponents
+  static constexpr int oBar = oE + 16;                   // mbarriers: QK[2], PV, stage[kStages]
+  static constexpr int kBarQK = 0, kBarPV = 2, kBarStage = 3;
+  static constexpr int oTmem = oBar + 8 * (3 + kStages);
   static constexpr int oFlag = oTmem + 4;
   static constexpr int kUsed = oFlag + 4;
-  // At least 78 KB per CTA: two CTAs fit on an SM, a third never does (each holds 256 TMEM columns).
-  static constexpr int kSmem = kUsed > 78 * 1024 ? kUsed : 78 * 1024;
+  // Two CTAs per SM (256 TMEM columns each) need at least 78 KB each so that a third never fits;
+  // one CTA per SM (512 columns) needs more than half of the SM's shared memory.
+  static constexpr int kFloor = kCtasPerSm == 2 ? 78 * 1024 : 116 * 1024;
+  static constexpr int kSmem = kUsed > kFloor ? kUsed : kFloor;
   // Epilogue (in the stage area): quantized partial [GQ], window partials [8][GQ], sums [4][GQ*(1+VPT)].
   static constexpr int kEpiFloats = 9 * GQ * kPartStride + 4 * GQ * (1 + VPT);
   static_assert(kEpiFloats * 4 <= kStages * kStageBytes, "epilogue does not fit the stage area");
   static_assert(oBar % 8 == 0 && oBQK % 16 == 0 && oBPV % 16 == 0, "alignment");
-  static_assert(kUsed <= 200 * 1024, "shared memory");
+  static_assert(kColO + kN <= kTmemCols, "TMEM plan");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
 template <int N>
@@ -270,7 +285,7 @@ __device__ __forceinline__ void unpack_row_half(const uint8_t* src, uint32_t tad
 }
 
 template <int KB, int VB, int VPT, int GQ>
-__global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, TcPlan<KB, VB, VPT, GQ>::kCtasPerSm) decode_tc_kernel(const DecodeArgs a) {
   using P = TcPlan<KB, VB, VPT, GQ>;
   constexpr int G = P::G, S = P::kStages, NC = P::kUsedCols;
   constexpr float kCbar = VB == 2 ? 1.5f : 7.5f;
@@ -280,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
   float* sbias = reinterpret_cast<float*>(smem + P::oBias);
   float* sred = reinterpret_cast<float*>(smem + P::oRed);
   int* se = reinterpret_cast<int*>(smem + P::oE);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::oBar);  // [0] QK done, [1] PV done, [2 + s] stage s
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::oBar);
   uint32_t* stmem = reinterpret_cast<uint32_t*>(smem + P::oTmem);
   volatile int* sflag = reinterpret_cast<volatile int*>(smem + P::oFlag);
 
@@ -310,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
   const uint8_t* kz_base = reinterpret_cast<const uint8_t*>(a.k_zero) + (unit * a.groups + start / G) * 256;
   auto issue = [&](int j) {
     uint8_t* st = smem + (j % S) * P::kStageBytes;
-    uint64_t* bar = &bars[2 + j % S];
+    uint64_t* bar = &bars[P::kBarStage + j % S];
     const int64_t t0 = static_cast<int64_t>(j) * kStep;
     mbar_expect_tx(bar, P::kStageBytes);
     bulk_g2s(st + P::oKC, kc_base + t0 * (16 * KB), P::kKC, bar);
@@ -320,10 +335,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
     bulk_g2s(st + P::oKS, ks_base + (t0 / G) * 256, P::kKS, bar);
     bulk_g2s(st + P::oKZ, kz_base + (t0 / G) * 256, P::kKS, bar);
   };
+  auto wait_stage = [&](int j) { mbar_wait(&bars[P::kBarStage + j % S], (j / S) & 1, sflag); };
 
-  if (warp == 0) tmem_alloc(stmem, kTmemCols);
+  if (warp == 0) tmem_alloc(stmem, P::kTmemCols);
   if (tid == 32) {
-    for (int i = 0; i < 2 + S; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 3 + S; ++i) mbar_init(&bars[i], 1);
     *sflag = 0;
     fence_mbar_init();
     fence_proxy_async();
@@ -379,9 +395,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
   const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
 
   // per-role constants
-  float qh[GQ];       // channel warps: q^[h][row]
-  float qz[4];        // channel warps: q~[h_w][4 lane .. 4 lane + 3], h_w = wq % GQ (bias dots)
-  float p2e[GQ];      // token warps: 2^e per head
+  float qh[GQ];   // channel warps: q^[h][row]
+  float qz[4];    // channel warps: q~[h_w][4 lane .. 4 lane + 3], h_w = wq % GQ (bias dots)
+  float p2e[GQ];  // token warps: 2^e per head
 #pragma unroll
   for (int h = 0; h < GQ; ++h) {
     qh[h] = sqh[h * kHeadDim + row];
@@ -395,8 +411,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
     qz[3] = v.w;
   }
 
-  // Channel warps: B_QK of step j (row = channel) and the step's zero-point biases (one warp-wide dot
-  // per (group, head); warp wq takes the pairs d = wq (mod 4), whose head is wq % GQ).
+  // Channel warps: B_QK of step j (row = channel) into buffer j % 2, and the step's zero-point biases
+  // into slot j % 4 (one warp-wide dot per (group, head); warp wq takes the pairs d = wq (mod 4), whose
+  // head is wq % GQ).
   auto build_qk = [&](int j) {
     const uint8_t* st = smem + (j % S) * P::kStageBytes;
     const uint16_t* ks = reinterpret_cast<const uint16_t*>(st + P::oKS);
@@ -412,12 +429,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
         w[gl * GQ + h] = pack_h2(split_part(x, false), split_part(x, true));
       }
     }
-    uint8_t* dst = smem + P::oBQK + row * 16;
+    uint8_t* dst = smem + P::oBQK + (j & 1) * P::kB + row * 16;
 #pragma unroll
     for (int c = 0; c < P::kChunks; ++c)
       *reinterpret_cast<uint4*>(dst + c * 2048) = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
     const uint16_t* kz = reinterpret_cast<const uint16_t*>(st + P::oKZ);
-    float* bias = sbias + (j & 1) * (VPT * GQ);
+    float* bias = sbias + (j & 3) * (VPT * GQ);
 #pragma unroll
     for (int d0 = 0; d0 < VPT * GQ; d0 += 4) {
       const int d = d0 + wq;
@@ -433,17 +450,29 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
       }
     }
   };
-  // Token warps: key rows of step j -> A_K (row = token).
+  // Token warps: key rows of step j -> A_K buffer j % 2 (row = token).
   auto unpack_keys = [&](int j) {
     const uint8_t* src = smem + (j % S) * P::kStageBytes + P::oKC + row * (16 * KB);
-    unpack_row_half<KB, false>(src, tmem + lane_base + kColAK);
-    unpack_row_half<KB, false>(src + 8 * KB, tmem + lane_base + kColAK + 32);
+    const uint32_t col = P::kColAK + 64 * (j & 1);
+    unpack_row_half<KB, false>(src, tmem + lane_base + col);
+    unpack_row_half<KB, false>(src + 8 * KB, tmem + lane_base + col + 32);
   };
   // Channel warps: value rows of step j -> A_V (row = channel), centered.
   auto unpack_values = [&](int j) {
     const uint8_t* src = smem + (j % S) * P::kStageBytes + P::oVC + row * (16 * VB);
-    unpack_row_half<VB, true>(src, tmem + lane_base + kColAV);
-    unpack_row_half<VB, true>(src + 8 * VB, tmem + lane_base + kColAV + 32);
+    unpack_row_half<VB, true>(src, tmem + lane_base + P::kColAV);
+    unpack_row_half<VB, true>(src + 8 * VB, tmem + lane_base + P::kColAV + 32);
+  };
+
+  constexpr uint32_t kIdesc = idesc_f16(P::kN);
+  const uint32_t bqk_addr = smem_u32(smem + P::oBQK), bpv_addr = smem_u32(smem + P::oBPV);
+  // One thread: QK(j) = S[j % 2] from A_K[j % 2] and B_QK[j % 2], signalled on the QK barrier j % 2.
+  auto issue_qk = [&](int j) {
+    const uint32_t d = tmem + P::kColS + P::kN * (j & 1), acol = tmem + P::kColAK + 64 * (j & 1);
+    const uint32_t baddr = bqk_addr + (j & 1) * P::kB;
+#pragma unroll
+    for (int s2 = 0; s2 < 8; ++s2) mma_f16_ts(d, acol + 8 * s2, b_desc(baddr + 256 * s2), kIdesc, s2 > 0);
+    mma_commit(&bars[P::kBarQK + (j & 1)]);
   };
 
   // token-warp softmax state (m_ref is CTA-uniform and kept by every thread)
@@ -456,47 +485,64 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
     for (int j = 0; j < VPT; ++j) zacc[h][j] = 0.f;
   }
 
-  constexpr uint32_t kIdesc = idesc_f16(P::kN);
-  const uint32_t bqk_addr = smem_u32(smem + P::oBQK), bpv_addr = smem_u32(smem + P::oBPV);
-
-  // ---- prologue: step 0's key operands, then QK(0)
-  if (nsteps > 0) {
-    mbar_wait(&bars[2], 0, sflag);
+  // ---- prologue: key operands of steps 0 and 1, then QK(0) and QK(1)
+  const int npro = nsteps < 2 ? nsteps : 2;
+  for (int j = 0; j < npro; ++j) {
+    wait_stage(j);
     if (token_warp)
-      unpack_keys(0);
+      unpack_keys(j);
     else
-      build_qk(0);
-    fence_proxy_async();
-    tc_wait_st();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int s = 0; s < 8; ++s) mma_f16_ts(tmem + kColS, tmem + kColAK + 8 * s, b_desc(bqk_addr + 256 * s), kIdesc, s > 0);
-      mma_commit(&bars[0]);
-    }
+      build_qk(j);
+  }
+  fence_proxy_async();
+  tc_wait_st();
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && npro > 0) {
+    tc_fence_after();
+    for (int j = 0; j < npro; ++j) issue_qk(j);
   }
 
+  // ---- main loop. Iteration i: softmax and PV operands of step i, key operands of step i + 2; one
+  //      barrier (with the new-maximum vote) in the common case; then PV(i) and QK(i + 2) are issued.
   for (int i = 0; i < nsteps; ++i) {
     const int t_step = start + i * kStep;
-    const bool more = i + 1 < nsteps;
+    const bool ahead = i + 2 < nsteps;
     const uint8_t* st = smem + (i % S) * P::kStageBytes;
-    mbar_wait(&bars[0], i & 1, sflag);  // QK(i) done: S(i) readable, A_K and B_QK free
+    mbar_wait(&bars[P::kBarQK + (i & 1)], (i >> 1) & 1, sflag);  // QK(i): S(i) readable; A_K, B_QK buffer i % 2 free
     tc_fence_after();
 
-    float s[GQ];
+    float s[GQ], p[GQ], sv[VPT], zv[VPT];
     bool exceed = false;
+    const bool valid = t_step + row < qend;
+#pragma unroll
+    for (int h = 0; h < GQ; ++h) s[h] = p[h] = 0.f;
+    // B_PV row of this token from p: hi/lo of p * sv per (value group, head); zero for masked tokens.
+    auto write_bpv = [&]() {
+      uint32_t w[P::kChunks * 4];
+#pragma unroll
+      for (int k = 0; k < P::kChunks * 4; ++k) w[k] = 0u;
+#pragma unroll
+      for (int j = 0; j < VPT; ++j)
+#pragma unroll
+        for (int h = 0; h < GQ; ++h) {
+          const float x = valid ? p[h] * sv[j] : 0.f;
+          w[j * GQ + h] = pack_h2(split_part(x, false), split_part(x, true));
+        }
+      uint8_t* dst = smem + P::oBPV + row * 16;
+#pragma unroll
+      for (int c = 0; c < P::kChunks; ++c)
+        *reinterpret_cast<uint4*>(dst + c * 2048) = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+    };
     if (token_warp) {
       constexpr int kGpw = G >= 32 ? 1 : 32 / G;  // groups per warp
       constexpr int kCols = kGpw * 2 * GQ;
       uint32_t d[kCols];
       const int gl0 = (32 * wq) / G;
-      tmem_ld<kCols>(tmem + lane_base + kColS + gl0 * 2 * GQ, d);
+      tmem_ld<kCols>(tmem + lane_base + P::kColS + P::kN * (i & 1) + gl0 * 2 * GQ, d);
       tc_wait_ld();
       const int gsel = kGpw > 1 ? (lane * kGpw) / 32 : 0;  // this token's group within the warp's columns
-      const bool valid = t_step + row < qend;
-      const float* bias = sbias + (i & 1) * (VPT * GQ) + (row / G) * GQ;
+      const float* bias = sbias + (i & 3) * (VPT * GQ) + (row / G) * GQ;
 #pragma unroll
       for (int h = 0; h < GQ; ++h) {
         float hi = __uint_as_float(d[2 * h]), lo = __uint_as_float(d[2 * h + 1]);
@@ -510,27 +556,38 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
         }
         s[h] = valid ? fmaf(hi + lo, p2e[h], bias[h]) : -CUDART_INF_F;
         exceed |= (h < gq) && (s[h] > m_ref[h]);
+        float mx = s[h];
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kAll, mx, x));
+        if (lane == 0) sred[wq * GQ + h] = mx;
+      }
+      load_u16s<VPT>(reinterpret_cast<const uint16_t*>(st + P::oVS) + row * VPT, sv);
+      load_u16s<VPT>(reinterpret_cast<const uint16_t*>(st + P::oVZ) + row * VPT, zv);
+#pragma unroll
+      for (int h = 0; h < GQ; ++h) p[h] = valid ? fast_exp2(s[h] - m_ref[h]) : 0.f;
+      if (i > 0) mbar_wait(&bars[P::kBarPV], (i - 1) & 1, sflag);  // PV(i-1): B_PV and O free
+      tc_fence_after();
+      write_bpv();  // rewritten below if the vote finds a new maximum
+      if (ahead) {
+        wait_stage(i + 2);
+        unpack_keys(i + 2);
       }
     } else {
-      // channel warps: B_QK and the biases of step i+1 (A_K / B_QK are free once QK(i) is done)
-      if (more) {
-        mbar_wait(&bars[2 + (i + 1) % S], ((i + 1) / S) & 1, sflag);
-        build_qk(i + 1);
+      if (ahead) {
+        wait_stage(i + 2);
+        build_qk(i + 2);
       }
+      if (i > 0) mbar_wait(&bars[P::kBarPV], (i - 1) & 1, sflag);  // PV(i-1): A_V free
+      tc_fence_after();
+      unpack_values(i);
     }
-
-    // ---- online softmax: a new maximum anywhere in the CTA rescales O, l and the midpoint sums
+    fence_proxy_async();
+    tc_wait_st();
+    tc_fence_before();
     if (__syncthreads_or(exceed)) {
-      if (token_warp) {
-#pragma unroll
-        for (int h = 0; h < GQ; ++h) {
-          float mx = s[h];
-#pragma unroll
-          for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kAll, mx, x));
-          if (lane == 0) sred[wq * GQ + h] = mx;
-        }
-      }
-      __syncthreads();
+      // A score above the running maximum: move the maximum to the step's, rescale l, the midpoint
+      // sums and O (held in TMEM), and redo this step's probabilities.
+      tc_fence_after();
       float alpha[GQ];
 #pragma unroll
       for (int h = 0; h < GQ; ++h) {
@@ -546,83 +603,50 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
           l_run[h] *= alpha[h];
 #pragma unroll
           for (int j = 0; j < VPT; ++j) zacc[h][j] *= alpha[h];
+          p[h] = valid ? fast_exp2(s[h] - m_ref[h]) : 0.f;
         }
-        if (i > 0) {  // O holds steps 0 .. i-1: rescale it in TMEM once PV(i-1) is done
-          mbar_wait(&bars[1], (i - 1) & 1, sflag);
-          tc_fence_after();
+        if (i > 0) {
 #pragma unroll
           for (int c0 = 0; c0 < P::kN; c0 += 16) {
             uint32_t o[16];
-            tmem_ld<16>(tmem + lane_base + kColO + c0, o);
+            tmem_ld<16>(tmem + lane_base + P::kColO + c0, o);
             tc_wait_ld();
 #pragma unroll
             for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha[((c0 + c) >> 1) % GQ]);
-            tmem_st16(tmem + lane_base + kColO + c0, o);
+            tmem_st16(tmem + lane_base + P::kColO + c0, o);
           }
-          tc_wait_st();
         }
+        write_bpv();
       }
+      fence_proxy_async();
+      tc_wait_st();
+      tc_fence_before();
+      __syncthreads();
     }
-
-    if (i > 0) mbar_wait(&bars[1], (i - 1) & 1, sflag);  // PV(i-1) done: A_V, B_PV free
-    tc_fence_after();
     if (token_warp) {
-      // p, l, midpoint sums and this token's B_PV row
-      const bool valid = t_step + row < qend;
-      float sv[VPT], zv[VPT];
-      load_u16s<VPT>(reinterpret_cast<const uint16_t*>(st + P::oVS) + row * VPT, sv);
-      load_u16s<VPT>(reinterpret_cast<const uint16_t*>(st + P::oVZ) + row * VPT, zv);
-      float p[GQ];
 #pragma unroll
-      for (int h = 0; h < GQ; ++h) {
-        p[h] = valid ? fast_exp2(s[h] - m_ref[h]) : 0.f;
-        l_run[h] += p[h];
-      }
-      uint32_t w[P::kChunks * 4];
+      for (int h = 0; h < GQ; ++h) l_run[h] += p[h];
+      if (valid) {
 #pragma unroll
-      for (int k = 0; k < P::kChunks * 4; ++k) w[k] = 0u;
+        for (int j = 0; j < VPT; ++j) {
+          const float mid = fmaf(kCbar, sv[j], zv[j]);
 #pragma unroll
-      for (int j = 0; j < VPT; ++j) {
-        const float mid = fmaf(kCbar, sv[j], zv[j]);
-#pragma unroll
-        for (int h = 0; h < GQ; ++h) {
-          const float x = valid ? p[h] * sv[j] : 0.f;
-          w[j * GQ + h] = pack_h2(split_part(x, false), split_part(x, true));
-          if (valid) zacc[h][j] = fmaf(p[h], mid, zacc[h][j]);
+          for (int h = 0; h < GQ; ++h) zacc[h][j] = fmaf(p[h], mid, zacc[h][j]);
         }
       }
-      uint8_t* dst = smem + P::oBPV + row * 16;
-#pragma unroll
-      for (int c = 0; c < P::kChunks; ++c)
-        *reinterpret_cast<uint4*>(dst + c * 2048) = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-      // keys of step i+1
-      if (more) {
-        mbar_wait(&bars[2 + (i + 1) % S], ((i + 1) / S) & 1, sflag);
-        unpack_keys(i + 1);
-      }
-    } else {
-      unpack_values(i);
     }
-    fence_proxy_async();
-    tc_wait_st();
-    tc_fence_before();
-    __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      if (more) {
-#pragma unroll
-        for (int s2 = 0; s2 < 8; ++s2)
-          mma_f16_ts(tmem + kColS, tmem + kColAK + 8 * s2, b_desc(bqk_addr + 256 * s2), kIdesc, s2 > 0);
-        mma_commit(&bars[0]);
-      }
 #pragma unroll
       for (int s2 = 0; s2 < 8; ++s2)
-        mma_f16_ts(tmem + kColO, tmem + kColAV + 8 * s2, b_desc(bpv_addr + 256 * s2), kIdesc, (i > 0 || s2 > 0) ? 1u : 0u);
-      mma_commit(&bars[1]);
+        mma_f16_ts(tmem + P::kColO, tmem + P::kColAV + 8 * s2, b_desc(bpv_addr + 256 * s2), kIdesc,
+                   (i > 0 || s2 > 0) ? 1u : 0u);
+      mma_commit(&bars[P::kBarPV]);
+      if (ahead) issue_qk(i + 2);
       if (i + S < nsteps) issue(i + S);  // stage i % S is consumed
     }
   }
-  if (nsteps > 0) mbar_wait(&bars[1], (nsteps - 1) & 1, sflag);
+  if (nsteps > 0) mbar_wait(&bars[P::kBarPV], (nsteps - 1) & 1, sflag);
   tc_fence_after();
 
   // ---- epilogue: quantized partial of the CTA -> shared memory (stage area)
@@ -652,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
 #pragma unroll
       for (int c0 = 0; c0 < NC; c0 += 16) {
         uint32_t d[16];
-        tmem_ld<16>(tmem + lane_base + kColO + c0, d);
+        tmem_ld<16>(tmem + lane_base + P::kColO + c0, d);
         tc_wait_ld();
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -689,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const DecodeArgs
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, P::kTmemCols);
   }
 
   // ---- FP16 window tokens [Q, T), spread over all splits of the unit: this CTA takes tokens
@@ -826,7 +850,26 @@ cudaError_t dispatch_tc_vpt(const DecodeArgs& a, cudaStream_t s) {
   }
 }
 
+template <int KB, int VB, int VPT>
+int ctas_tc_gq(int gqa) {
+  switch (gq_class_tc(gqa)) {
+    case 1: return TcPlan<KB, VB, VPT, 1>::kCtasPerSm;
+    case 2: return TcPlan<KB, VB, VPT, 2>::kCtasPerSm;
+    default: return TcPlan<KB, VB, VPT, 4>::kCtasPerSm;
+  }
+}
+
 }  // namespace
+
+int decode_tc_ctas_per_sm(int G, int gqa) {
+  // TMEM columns depend on G and gqa only (bits do not enter the plan's column count)
+  switch (G) {
+    case 128: return ctas_tc_gq<2, 2, 1>(gqa);
+    case 64: return ctas_tc_gq<2, 2, 2>(gqa);
+    case 32: return ctas_tc_gq<2, 2, 4>(gqa);
+    default: return ctas_tc_gq<2, 2, 8>(gqa);
+  }
+}
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   if (a.key_bits == 2) return a.value_bits == 2 ? dispatch_tc_vpt<2, 2>(a, stream) : dispatch_tc_vpt<2, 4>(a, stream);

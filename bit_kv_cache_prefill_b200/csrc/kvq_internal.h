@@ -50,10 +50,10 @@ cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t 
 cudaError_t launch_append(const QuantizeArgs& a, const uint16_t* k_new, const uint16_t* v_new, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);     // split + combine, either layout
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // rows-v2 split kernel only
-int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);
+int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);  // tile-v1 kernel
+int decode_tc_ctas_per_sm(int G, int gqa);                              // rows-v2 kernel (1 or 2)
 
 constexpr int kDecodeWarps = 4;
-constexpr int kTcCtasPerSm = 2;    // rows-v2 kernel: 256 TMEM columns per CTA
 constexpr int kPartFloats = 2 + 128;  // m, l, o[128]
 
 }  // namespace kvq
