@@ -1,0 +1,458 @@
+// kvq_prefill.cu — bulk prefill: quantize and pack many tokens at once (KVQuant review, Limitations and
+// Sparks: the prefill compresses all keys and values of the prompt in one pass).
+//
+// One CTA takes one 128-token block of one (sequence, KV head) unit, keys (blockIdx.z == 0) or values
+// (blockIdx.z == 1). The block's fp16 rows are staged in shared memory with cp.async (row stride 272
+// bytes, so that column reads by consecutive rows spread over the banks), rotated in place for keys when
+// the Hadamard option is on, and then
+//   keys:   min/max per (key group, channel) over G tokens, parameters per (group, channel);
+//   values: min/max per (token, value group) over G channels, parameters per (token, group);
+// (KVQuant review, Method; KV cache quantization wiki page, KIVI notes), and finally every packed word
+// is built by one thread that holds the parameters of its channels (keys) or reads them per token
+// (values). Tokens of the block at or beyond the quantized length go to the FP16 ring (framework page,
+// In practice). The codec arithmetic is the one fixed in kvq_common.cuh: min/max in the IEEE total
+// order, s32 = (mx - mn) / (2^b - 1) rounded to fp16, zero = mn, code = rint_even((x - mn) * (1 / s16))
+// clamped to [0, 2^b - 1], every step an explicit round-to-nearest operation.
+//
+// Throughput notes: the order keys of two halves are formed and compared as u16x2 (min/max.u16x2); two
+// codes share packed fp32x2 subtract and multiply instructions; the round-half-even to an integer is a
+// scalar IEEE add of 1.5 * 2^23, exact for 0 <= v < 2^22. The clamp to 2^b - 1 only matters for groups whose fp16
+// scale rounded down far enough (subnormal scales); such groups are flagged when their parameters are
+// made and take a scalar path with the explicit clamp.
+#include <cuda_runtime.h>
+
+#include "kvq_common.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+constexpr int kPB = 128;      // tokens per block
+constexpr int kRS = 136;      // staged row stride in halves (272 bytes)
+constexpr int kPThreads = 256;
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint32_t order_key2(uint32_t x) {
+  const uint32_t s = (x >> 15) & 0x00010001u;  // each half's sign bit at its bit 0
+  return x ^ ((s * 0xFFFFu) | 0x80008000u);      // negative half: flip all 16 bits; else flip the sign bit
+}
+__device__ __forceinline__ uint32_t vmin2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t vmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+// Codes of the two fp16 halves of x: rint_even((x_i - zf_i) * inv_i) on exact IEEE fp32 steps, for
+// groups that need no clamp (returned in bits [0, 8) of each 32-bit half of the result). The rounding
+// add is scalar: a packed multiply followed by a packed add was executed as one fused multiply-add
+// (a single rounding of the exact product), which moves values that round to a tie (v = k + 0.5 in
+// fp32) to the wrong code.
+__device__ __forceinline__ uint64_t codes2(uint32_t x, uint64_t zf2, uint64_t inv2) {
+  const uint64_t f = pk2(h2f(static_cast<uint16_t>(x & 0xffffu)), h2f(static_cast<uint16_t>(x >> 16)));
+  uint64_t d, v;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f), "l"(zf2));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(v) : "l"(d), "l"(inv2));
+  const float r0 = __fadd_rn(__uint_as_float(static_cast<uint32_t>(v)), kMagic);
+  const float r1 = __fadd_rn(__uint_as_float(static_cast<uint32_t>(v >> 32)), kMagic);
+  return static_cast<uint64_t>(__float_as_uint(r0)) | (static_cast<uint64_t>(__float_as_uint(r1)) << 32);
+}
+// The same for one value with the explicit clamp (flagged groups).
+__device__ __forceinline__ uint32_t code_clamped(uint16_t x, float zf, float inv, int top) {
+  const float v = fminf(__fmul_rn(__fsub_rn(h2f(x), zf), inv), static_cast<float>(top));
+  return __float_as_uint(__fadd_rn(v, kMagic)) & 0xffu;
+}
+// Whether any element of a group can reach a code above 2^b - 1: v is monotone in x, so the group's
+// maximum decides.
+__device__ __forceinline__ bool needs_clamp(const QuantParams& p, uint32_t kmax, int top) {
+  if (p.zero_scale) return false;
+  const float vmax = __fmul_rn(__fsub_rn(h2f(key_to_half(kmax)), p.zf), p.inv);
+  return vmax >= static_cast<float>(top) + 0.5f;
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+
+// Hadamard rotation of the staged key rows, in place: two rows per warp per step (16 lanes per row).
+__device__ void rotate_block(uint16_t* rows, int nrows) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r0 = warp * 2; r0 < nrows; r0 += (kPThreads / 32) * 2) {  // r0 is warp-uniform
+    const int row = r0 + (lane >> 4);
+    const bool valid = row < nrows;
+    uint4* p = reinterpret_cast<uint4*>(rows + static_cast<size_t>(valid ? row : 0) * kRS) + (lane & 15);
+    uint4 raw = valid ? *p : make_uint4(0, 0, 0, 0);
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(&raw);
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = h2f(h[i]);
+    wht128_16lanes(x);  // all 32 lanes take part; the half-warp past the last row works on zeros
+    uint16_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = __half_as_ushort(__float2half_rn(x[i]));
+    if (valid) *p = *reinterpret_cast<const uint4*>(o);
+  }
+}
+
+// ---- keys ---------------------------------------------------------------------------------------------
+// Shared memory after the rows: per (group, quarter, channel pair) min / max keys [8][4][64] u32 x 2,
+// then per (group, channel) zf and inv [8][128] f32 x 2 and clamp flags [8][128] u8.
+constexpr int kKeyScratch = 2 * 8 * 4 * 64 * 4 + 2 * 8 * 128 * 4 + 8 * 128;
+
+template <int BITS, int LAYOUT>
+__device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int nq, const uint16_t* rows, uint8_t* scratch) {
+  constexpr int top = (1 << BITS) - 1;
+  constexpr int P = 16 / BITS;  // code pairs per word
+  const int G = a.G, NG = nq / G;
+  uint32_t* pmn = reinterpret_cast<uint32_t*>(scratch);  // [8][4][64]
+  uint32_t* pmx = pmn + 8 * 4 * 64;
+  float* pz = reinterpret_cast<float*>(pmx + 8 * 4 * 64);  // [8][128]
+  float* pinv = pz + 8 * 128;
+  uint8_t* pcl = reinterpret_cast<uint8_t*>(pinv + 8 * 128);  // [8][128]
+  const int tid = threadIdx.x;
+
+  // min / max: thread (channel pair cp, quarter q) scans quarter q of every group
+  {
+    const int cp = tid & 63, q = tid >> 6, ql = G / 4;
+    for (int g = 0; g < NG; ++g) {
+      uint32_t mn = 0xffffffffu, mx = 0u;
+      const uint16_t* src = rows + (g * G + q * ql) * kRS + 2 * cp;
+      for (int i = 0; i < ql; ++i) {
+        const uint32_t k = order_key2(*reinterpret_cast<const uint32_t*>(src + i * kRS));
+        mn = vmin2(mn, k);
+        mx = vmax2(mx, k);
+      }
+      pmn[(g * 4 + q) * 64 + cp] = mn;
+      pmx[(g * 4 + q) * 64 + cp] = mx;
+    }
+  }
+  __syncthreads();
+  // parameters per (group, channel)
+  {
+    const int c = tid & 127, sh = 16 * (c & 1);
+    for (int g = tid >> 7; g < NG; g += 2) {
+      uint32_t kmin = 0xffffu, kmax = 0u;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        kmin = min(kmin, (pmn[(g * 4 + q) * 64 + (c >> 1)] >> sh) & 0xffffu);
+        kmax = max(kmax, (pmx[(g * 4 + q) * 64 + (c >> 1)] >> sh) & 0xffffu);
+      }
+      const QuantParams p = make_params(kmin, kmax, BITS);
+      const int pos = LAYOUT == KVQ_LAYOUT_ROWS_V2 ? c : key_param_pos(c);
+      const int64_t pidx = (unit * a.groups + t0 / G + g) * kHeadDim + pos;
+      a.k_scale[pidx] = p.s16;
+      a.k_zero[pidx] = p.z16;
+      pz[g * 128 + c] = p.zf;
+      pinv[g * 128 + c] = p.inv;
+      pcl[g * 128 + c] = needs_clamp(p, kmax, top) ? 1 : 0;
+    }
+  }
+  __syncthreads();
+
+  if constexpr (LAYOUT == KVQ_LAYOUT_ROWS_V2) {
+    // word w of token t holds channels [2P w, 2P w + 2P): pair k -> channels 2(Pw + k), +1 at bits
+    // BITS k and 16 + BITS k. Thread (w, lane-group) takes TPT tokens of one 16-token window (so of one
+    // group), consecutive threads consecutive words of nearby rows.
+    constexpr int W = 4 * BITS, R = kPThreads / W, TPT = kPB / R, STRIDE = 16 / TPT;
+    const int w = tid % W, rr = tid / W;
+    const int tbase = 16 * (rr / STRIDE) + (rr % STRIDE);
+    if (tbase >= nq) return;
+    const int g = tbase / G;
+    const int c0 = 2 * P * w;
+    float zf[2 * P], iv[2 * P];
+    bool slow = false;
+#pragma unroll
+    for (int i = 0; i < 2 * P; ++i) {
+      zf[i] = pz[g * 128 + c0 + i];
+      iv[i] = pinv[g * 128 + c0 + i];
+      slow |= pcl[g * 128 + c0 + i] != 0;
+    }
+    uint32_t* dst = a.k_codes + (unit * a.capacity + t0) * W + w;
+#pragma unroll 2
+    for (int it = 0; it < TPT; ++it) {
+      const int t = tbase + STRIDE * it;
+      const uint16_t* src = rows + t * kRS + c0;
+      uint32_t x[P];
+#pragma unroll
+      for (int v = 0; v < P / 4; ++v) {
+        const uint4 q4 = reinterpret_cast<const uint4*>(src)[v];
+        x[4 * v] = q4.x;
+        x[4 * v + 1] = q4.y;
+        x[4 * v + 2] = q4.z;
+        x[4 * v + 3] = q4.w;
+      }
+      uint32_t word = 0;
+      if (!slow) {
+#pragma unroll
+        for (int k = 0; k < P; ++k) {
+          const uint64_t r = codes2(x[k], pk2(zf[2 * k], zf[2 * k + 1]), pk2(iv[2 * k], iv[2 * k + 1]));
+          word |= ((static_cast<uint32_t>(r) & top) << (BITS * k)) | ((static_cast<uint32_t>(r >> 32) & top) << (16 + BITS * k));
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < P; ++k) {
+          word |= code_clamped(static_cast<uint16_t>(x[k] & 0xffffu), zf[2 * k], iv[2 * k], top) << (BITS * k);
+          word |= code_clamped(static_cast<uint16_t>(x[k] >> 16), zf[2 * k + 1], iv[2 * k + 1], top) << (16 + BITS * k);
+        }
+      }
+      dst[static_cast<int64_t>(t) * W] = word;
+    }
+  } else {
+    // Tile v1: word w of lane L = 4r + qd in tile tl; pair j -> token r + 8u, channels 16m + 2qd + 8hh
+    // (+1), with (m, hh, u) from the pair slot p = P w + j. Thread (w % 4, L, half) keeps the parameters
+    // of the word's channels for the tiles of one group.
+    constexpr int NCP = P / 2;  // channel pairs per word (each at two token rows)
+    const int wl = tid & 3, L = (tid >> 2) & 31, hi = tid >> 7;
+    const int w = BITS == 2 ? wl : 4 * hi + wl;
+    const int tl0 = BITS == 2 ? 4 * hi : 0, ntl = BITS == 2 ? 4 : 8;
+    const int r = L >> 2, qd = L & 3;
+    const int words = 64 * BITS;
+    const int widx = (w >> 2) * 128 + 4 * L + (w & 3);
+    int cpair[NCP];  // first channel of each channel pair of the word
+    int jbase[NCP];  // pair slot j of the pair at u = 0 (u = 1 is j + 1)
+#pragma unroll
+    for (int i = 0; i < NCP; ++i) {
+      const int j = 2 * i;  // u = 0
+      const int p = P * w + j;
+      const int m = p >> 2, hh = (p >> 1) & 1;
+      cpair[i] = 16 * m + 2 * qd + 8 * hh;
+      jbase[i] = j;
+    }
+    float zf[2 * NCP], iv[2 * NCP];
+    bool slow = false;
+    int gcur = -1;
+    uint32_t* dst = a.k_codes + (unit * a.tiles + t0 / kTile) * words + widx;
+    for (int tl = tl0; tl < tl0 + ntl && tl * kTile < nq; ++tl) {
+      const int g = (tl * kTile) / G;
+      if (g != gcur) {
+        gcur = g;
+        slow = false;
+#pragma unroll
+        for (int i = 0; i < NCP; ++i) {
+          zf[2 * i] = pz[g * 128 + cpair[i]];
+          zf[2 * i + 1] = pz[g * 128 + cpair[i] + 1];
+          iv[2 * i] = pinv[g * 128 + cpair[i]];
+          iv[2 * i + 1] = pinv[g * 128 + cpair[i] + 1];
+          slow |= (pcl[g * 128 + cpair[i]] | pcl[g * 128 + cpair[i] + 1]) != 0;
+        }
+      }
+      uint32_t word = 0;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint16_t* src = rows + (tl * kTile + r + 8 * u) * kRS;
+#pragma unroll
+        for (int i = 0; i < NCP; ++i) {
+          const uint32_t x = *reinterpret_cast<const uint32_t*>(src + cpair[i]);
+          const int j = jbase[i] + u;
+          if (!slow) {
+            const uint64_t rr = codes2(x, pk2(zf[2 * i], zf[2 * i + 1]), pk2(iv[2 * i], iv[2 * i + 1]));
+            word |= ((static_cast<uint32_t>(rr) & top) << (BITS * j)) | ((static_cast<uint32_t>(rr >> 32) & top) << (16 + BITS * j));
+          } else {
+            word |= code_clamped(static_cast<uint16_t>(x & 0xffffu), zf[2 * i], iv[2 * i], top) << (BITS * j);
+            word |= code_clamped(static_cast<uint16_t>(x >> 16), zf[2 * i + 1], iv[2 * i + 1], top) << (16 + BITS * j);
+          }
+        }
+      }
+      dst[static_cast<int64_t>(tl) * words] = word;
+    }
+  }
+}
+
+// ---- values -------------------------------------------------------------------------------------------
+// Shared memory after the rows: per (token, group) zf and inv as float2 [128][8], clamp flags [128][8]
+// u8, and (rows v2) the packed output words [128][4 * BITS] u32.
+constexpr int kValScratch = 128 * 8 * 8 + 128 * 8 + 128 * 16 * 4;
+
+template <int BITS, int LAYOUT>
+__device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int nq, const uint16_t* rows, uint8_t* scratch) {
+  constexpr int top = (1 << BITS) - 1;
+  constexpr int P = 16 / BITS;
+  const int G = a.G, VPT = kHeadDim / G;
+  float2* prm = reinterpret_cast<float2*>(scratch);              // [128][8]
+  uint8_t* pcl = scratch + 128 * 8 * 8;                          // [128][8]
+  uint32_t* outw = reinterpret_cast<uint32_t*>(pcl + 128 * 8);   // [128][4 * BITS] (rows v2)
+  const int tid = threadIdx.x;
+
+  // parameters per (token, group): item (t, j) scans G channels of row t
+  for (int idx = tid; idx < nq * VPT; idx += kPThreads) {
+    const int t = idx / VPT, j = idx % VPT;
+    const uint16_t* src = rows + t * kRS + j * G;
+    uint32_t mn = 0xffffffffu, mx = 0u;
+    for (int c8 = 0; c8 < G; c8 += 8) {
+      const uint4 q4 = *reinterpret_cast<const uint4*>(src + c8);
+      const uint32_t k0 = order_key2(q4.x), k1 = order_key2(q4.y), k2 = order_key2(q4.z), k3 = order_key2(q4.w);
+      mn = vmin2(mn, vmin2(vmin2(k0, k1), vmin2(k2, k3)));
+      mx = vmax2(mx, vmax2(vmax2(k0, k1), vmax2(k2, k3)));
+    }
+    const uint32_t kmin = min(mn & 0xffffu, mn >> 16), kmax = max(mx & 0xffffu, mx >> 16);
+    const QuantParams p = make_params(kmin, kmax, BITS);
+    const int64_t pidx = (unit * a.capacity + t0 + t) * VPT + j;
+    a.v_scale[pidx] = p.s16;
+    a.v_zero[pidx] = p.z16;
+    prm[t * 8 + j] = make_float2(p.zf, p.inv);
+    pcl[t * 8 + j] = needs_clamp(p, kmax, top) ? 1 : 0;
+  }
+  __syncthreads();
+
+  if constexpr (LAYOUT == KVQ_LAYOUT_ROWS_V2) {
+    // Channel c's row of the 128-token block: word wv holds token pairs k -> tokens 2(P wv + k), +1 at
+    // bits BITS k and 16 + BITS k. Lane = channel quad (4 channels, one 8-byte load per token), warp =
+    // word(s); words go to shared memory first and leave as coalesced 16-byte stores.
+    constexpr int W = 4 * BITS;
+    const int cq = tid & 31, wv0 = tid >> 5;
+    const int c = 4 * cq, j = c / G;
+    const int nw = nq * BITS / 32;  // complete words (nq is a multiple of 16)
+    for (int wv = wv0; wv < nw; wv += kPThreads / 32) {
+      uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int k = 0; k < P; ++k) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * (P * wv + k) + e;
+          const uint2 x = *reinterpret_cast<const uint2*>(rows + t * kRS + c);
+          const float2 pp = prm[t * 8 + j];
+          const int sh = BITS * k + 16 * e;
+          if (!pcl[t * 8 + j]) {
+            const uint64_t z2 = pk2(pp.x, pp.x), i2 = pk2(pp.y, pp.y);
+            const uint64_t r0 = codes2(x.x, z2, i2), r1 = codes2(x.y, z2, i2);
+            wd[0] |= (static_cast<uint32_t>(r0) & top) << sh;
+            wd[1] |= (static_cast<uint32_t>(r0 >> 32) & top) << sh;
+            wd[2] |= (static_cast<uint32_t>(r1) & top) << sh;
+            wd[3] |= (static_cast<uint32_t>(r1 >> 32) & top) << sh;
+          } else {
+            wd[0] |= code_clamped(static_cast<uint16_t>(x.x & 0xffffu), pp.x, pp.y, top) << sh;
+            wd[1] |= code_clamped(static_cast<uint16_t>(x.x >> 16), pp.x, pp.y, top) << sh;
+            wd[2] |= code_clamped(static_cast<uint16_t>(x.y & 0xffffu), pp.x, pp.y, top) << sh;
+            wd[3] |= code_clamped(static_cast<uint16_t>(x.y >> 16), pp.x, pp.y, top) << sh;
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) outw[(c + i) * W + wv] = wd[i];
+    }
+    __syncthreads();
+    // 128 channel rows x nw words -> the block's rows (W words each), 16 bytes per thread-store
+    uint32_t* dst = a.v_codes + unit * a.vwords + (t0 / 128) * 128 * W;
+    const int q4 = nw / 4;  // nw is a multiple of 4 when nq is a multiple of 16 * 4 / BITS ...
+    if (q4 * 4 == nw) {
+      for (int idx = tid; idx < 128 * q4; idx += kPThreads) {
+        const int ch = idx / q4, v = idx % q4;
+        reinterpret_cast<uint4*>(dst + ch * W)[v] = reinterpret_cast<const uint4*>(outw + ch * W)[v];
+      }
+    } else {
+      for (int idx = tid; idx < 128 * nw; idx += kPThreads) {
+        const int ch = idx / nw, v = idx % nw;
+        dst[ch * W + v] = outw[ch * W + v];
+      }
+    }
+  } else {
+    // Tile v1: word w of lane L = 4r + qd in tile tl; pair j -> tokens 2qd + 8hh (+1), channel
+    // 16m + r + 8u, with (m, hh, u) from p = P w + j. The two codes of a pair are consecutive tokens
+    // of one channel and share packed fp32x2 arithmetic.
+    const int wl = tid & 3, L = (tid >> 2) & 31, hi = tid >> 7;
+    const int w = BITS == 2 ? wl : 4 * hi + wl;
+    const int tl0 = BITS == 2 ? 4 * hi : 0, ntl = BITS == 2 ? 4 : 8;
+    const int r = L >> 2, qd = L & 3;
+    const int words = 64 * BITS;
+    const int widx = (w >> 2) * 128 + 4 * L + (w & 3);
+    uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words + widx;
+    for (int tl = tl0; tl < tl0 + ntl && tl * kTile < nq; ++tl) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < P; ++j) {
+        const int p = P * w + j;
+        const int m = p >> 2, u = p & 1, hh = (p >> 1) & 1;
+        const int ch = 16 * m + r + 8 * u, gj = ch / G;
+        const int t = tl * kTile + 2 * qd + 8 * hh;
+        const uint16_t x0 = rows[t * kRS + ch], x1 = rows[(t + 1) * kRS + ch];
+        const float2 p0 = prm[t * 8 + gj], p1 = prm[(t + 1) * 8 + gj];
+        if (!(pcl[t * 8 + gj] | pcl[(t + 1) * 8 + gj])) {
+          const uint64_t rr = codes2(static_cast<uint32_t>(x0) | (static_cast<uint32_t>(x1) << 16), pk2(p0.x, p1.x), pk2(p0.y, p1.y));
+          word |= ((static_cast<uint32_t>(rr) & top) << (BITS * j)) | ((static_cast<uint32_t>(rr >> 32) & top) << (16 + BITS * j));
+        } else {
+          word |= code_clamped(x0, p0.x, p0.y, top) << (BITS * j);
+          word |= code_clamped(x1, p1.x, p1.y, top) << (16 + BITS * j);
+        }
+      }
+      dst[static_cast<int64_t>(tl) * words] = word;
+    }
+  }
+}
+
+template <int BITS_K, int BITS_V, int LAYOUT>
+__global__ void __launch_bounds__(kPThreads) prefill_block_kernel(QuantizeArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
+  uint8_t* scratch = smem + kPB * kRS * 2;
+  const int64_t unit = blockIdx.y;
+  const bool is_key = blockIdx.z == 0;
+  const int64_t b = unit / a.num_kv_heads, h = unit % a.num_kv_heads;
+  const int64_t T = a.seq_len[b];
+  const int64_t Q = quantized_len(T, a.R, a.G);
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kPB;
+  if (t0 >= T) return;
+  const int n = static_cast<int>(min(static_cast<int64_t>(kPB), T - t0));
+  const int nq = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(n), Q - t0)));
+  const uint16_t* src = (is_key ? a.k : a.v) + b * a.stride_b + t0 * a.stride_t + h * a.stride_h;
+  for (int idx = threadIdx.x; idx < n * 16; idx += kPThreads) {
+    const int i = idx >> 4, part = idx & 15;
+    cp_async16(rows + i * kRS + 8 * part, src + i * a.stride_t + 8 * part);
+  }
+  asm volatile("cp.async.commit_group;\n" ::);
+  asm volatile("cp.async.wait_group 0;\n" ::);
+  __syncthreads();
+  if (is_key && a.hadamard) {
+    rotate_block(rows, n);
+    __syncthreads();
+  }
+  // FP16 window: tokens [t0 + nq, t0 + n) of the block (all at or beyond Q)
+  if (nq < n) {
+    uint16_t* ring = (is_key ? a.k_res : a.v_res) + unit * a.ring * kHeadDim;
+    for (int idx = threadIdx.x; idx < (n - nq) * 16; idx += kPThreads) {
+      const int i = nq + (idx >> 4), part = idx & 15;
+      const int64_t slot = (t0 + i) % a.ring;
+      reinterpret_cast<uint4*>(ring + slot * kHeadDim)[part] = reinterpret_cast<const uint4*>(rows + i * kRS)[part];
+    }
+  }
+  if (nq == 0) return;
+  if (is_key)
+    key_block<BITS_K, LAYOUT>(a, unit, t0, nq, rows, scratch);
+  else
+    value_block<BITS_V, LAYOUT>(a, unit, t0, nq, rows, scratch);
+}
+
+constexpr int kPrefillSmem = kPB * kRS * 2 + (kKeyScratch > kValScratch ? kKeyScratch : kValScratch);
+
+template <int BK, int BV, int LAYOUT>
+cudaError_t launch_block(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(prefill_block_kernel<BK, BV, LAYOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>((max_len + kPB - 1) / kPB), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads), 2);
+  prefill_block_kernel<BK, BV, LAYOUT><<<grid, kPThreads, kPrefillSmem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int LAYOUT>
+cudaError_t launch_bits(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
+  if (a.key_bits == 2) return a.value_bits == 2 ? launch_block<2, 2, LAYOUT>(a, max_len, stream) : launch_block<2, 4, LAYOUT>(a, max_len, stream);
+  return a.value_bits == 2 ? launch_block<4, 2, LAYOUT>(a, max_len, stream) : launch_block<4, 4, LAYOUT>(a, max_len, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
+  if (max_len <= 0 || a.batch == 0) return cudaSuccess;
+  return a.layout == KVQ_LAYOUT_ROWS_V2 ? launch_bits<KVQ_LAYOUT_ROWS_V2>(a, max_len, stream)
+                                        : launch_bits<KVQ_LAYOUT_TILE_V1>(a, max_len, stream);
+}
+
+}  // namespace kvq

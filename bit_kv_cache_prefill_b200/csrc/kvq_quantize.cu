@@ -1,17 +1,14 @@
-// kvq_quantize.cu — prefill quantize/pack and streaming append/flush kernels.
+// kvq_quantize.cu — streaming append and group flush.
 //
-// Prefill (KVQuant review, Limitations and Sparks: compress many keys and values in one pass) turns
-// fp16 K/V into 2- or 4-bit codes with fp16 scale/zero per group: keys per channel over G tokens,
-// values per token over G channels (KVQuant review, Method; KV cache quantization wiki page, KIVI
-// notes). Tokens of the FP16 window (framework page, In practice) go to a ring of R + G slots.
-// Append writes one token per sequence into the ring and, once the window holds a whole group
-// beyond R, quantizes that group and appends it along the token axis (wiki page, KIVI notes).
+// Append writes one token per sequence into the FP16 ring of R + G slots (framework page, In practice)
+// and, once the window holds a whole group beyond R, quantizes that group and appends it along the
+// token axis (KV cache quantization wiki page, KIVI notes): keys per channel over the G tokens, values
+// per token over G channels (KVQuant review, Method), 2- or 4-bit codes with fp16 scale / zero. The
+// bulk prefill lives in kvq_prefill.cu.
 //
-// One CTA quantizes one G-token chunk of one (sequence, KV head) for keys (blockIdx.z == 0) or
-// values (blockIdx.z == 1). The chunk is staged in shared memory (16-byte loads, a token row is 256
-// contiguous bytes), rotated in place when the Hadamard option is on (keys), reduced to per-group
-// min/max, coded, and packed word by word in the tile v1 order so that every warp store is a
-// contiguous 512-byte run.
+// One CTA flushes one (sequence, KV head) for keys (blockIdx.y == 0) or values (blockIdx.y == 1): the
+// group is gathered from the ring into shared memory, reduced to min/max, coded and packed word by word
+// in the cache layout.
 #include <cuda_runtime.h>
 
 #include "kvq_common.cuh"
@@ -23,28 +20,6 @@ namespace kvq {
 // 1/f32(scale)) per channel [128] plus per-quarter min/max keys [4][128] x 2; values use
 // (f32(zero), 1/f32(scale)) per (token, channel group) [G][128/G] = 128 entries.
 static size_t chunk_smem_bytes(int G) { return static_cast<size_t>(G) * kHeadDim * 2 + 128 * 8 + 2 * 4 * 128 * 4; }
-
-// Rotate (keys, optional) the G staged rows in place: two rows per warp per step.
-__device__ void rotate_rows(uint16_t* rows, int nrows) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
-  for (int r0 = warp * 2; r0 < nrows; r0 += nwarps * 2) {  // r0 is warp-uniform
-    const int row = r0 + (lane >> 4);
-    const bool valid = row < nrows;
-    float x[8];
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    uint4* p = reinterpret_cast<uint4*>(rows + static_cast<size_t>(valid ? row : 0) * kHeadDim) + (lane & 15);
-    if (valid) raw = *p;
-    const uint16_t* h = reinterpret_cast<const uint16_t*>(&raw);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = h2f(h[i]);
-    wht128_16lanes(x);  // all 32 lanes take part; the half-warp past the last row works on zeros
-    uint16_t o[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) o[i] = __half_as_ushort(__float2half_rn(x[i]));
-    if (valid) *p = *reinterpret_cast<const uint4*>(o);
-  }
-}
 
 // Code of x on the grid (zf, inv): rint_even((f32(x) - zf) * inv) clamped to [0, 2^bits - 1].
 // inv == 0 encodes a zero scale and yields code 0 (x - zf is finite). v = (x - zf) * inv is >= 0
@@ -206,50 +181,6 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
   }
 }
 
-__global__ void __launch_bounds__(256) prefill_kernel(QuantizeArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int64_t chunk = blockIdx.x;
-  const int64_t unit = blockIdx.y;
-  const bool is_key = blockIdx.z == 0;
-  const int64_t b = unit / a.num_kv_heads, h = unit % a.num_kv_heads;
-  const int G = a.G;
-  const int64_t T = a.seq_len[b];
-  const int64_t Q = quantized_len(T, a.R, G);
-  const int64_t t0 = chunk * G;
-  if (t0 >= T) return;
-  const int64_t n = min(static_cast<int64_t>(G), T - t0);
-  uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
-  uint8_t* pbuf = smem + static_cast<size_t>(G) * kHeadDim * 2;
-  const uint16_t* src = is_key ? a.k : a.v;
-  // Stage the chunk: 16 lanes per 256-byte token row.
-  for (int idx = threadIdx.x; idx < n * 16; idx += blockDim.x) {
-    const int64_t i = idx >> 4;
-    const int part = idx & 15;
-    const uint4* gp = reinterpret_cast<const uint4*>(src + b * a.stride_b + (t0 + i) * a.stride_t + h * a.stride_h) + part;
-    reinterpret_cast<uint4*>(rows + i * kHeadDim)[part] = __ldg(gp);
-  }
-  __syncthreads();
-  if (is_key && a.hadamard) {
-    rotate_rows(rows, static_cast<int>(n));
-    __syncthreads();
-  }
-  if (t0 + G <= Q) {
-    if (is_key)
-      quantize_keys_chunk(a, unit, t0, rows, pbuf);
-    else
-      quantize_values_chunk(a, unit, t0, rows, pbuf);
-    return;
-  }
-  // FP16 window: tokens [t0, t0 + n) (all >= Q because Q is a multiple of G).
-  uint16_t* ring = (is_key ? a.k_res : a.v_res) + unit * a.ring * kHeadDim;
-  for (int idx = threadIdx.x; idx < n * 16; idx += blockDim.x) {
-    const int64_t i = idx >> 4;
-    const int part = idx & 15;
-    const int64_t slot = (t0 + i) % a.ring;
-    reinterpret_cast<uint4*>(ring + slot * kHeadDim)[part] = reinterpret_cast<const uint4*>(rows + i * kHeadDim)[part];
-  }
-}
-
 // Append one token to every (sequence, KV head) and flush a full group out of the window.
 // Lengths are read from the device mirror and not modified here (bump_lengths_kernel follows).
 __global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint16_t* __restrict__ k_new,
@@ -302,18 +233,6 @@ __global__ void bump_lengths_kernel(int64_t* seq_len, int batch) {
 }
 
 // ---- host launchers ---------------------------------------------------------------------------------
-cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
-  if (max_len <= 0 || a.batch == 0) return cudaSuccess;
-  const size_t smem = chunk_smem_bytes(a.G);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
-  dim3 grid(static_cast<unsigned>((max_len + a.G - 1) / a.G), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads), 2);
-  prefill_kernel<<<grid, 256, smem, stream>>>(a);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_append(const QuantizeArgs& a, const uint16_t* k_new, const uint16_t* v_new, cudaStream_t stream) {
   const size_t smem = chunk_smem_bytes(a.G);
   if (smem > 48 * 1024) {
