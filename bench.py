@@ -127,6 +127,30 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def measured_traffic(w: inputs.Workload, layout: int):
+    """DRAM bytes per decode-split launch from the committed ncu counters (profiles/decode_traffic_counters.txt, JSON), scaled
+    from the captured batch to this one by the units processed; None if there is no capture for this
+    workload and layout or the kernel sources changed since it was taken."""
+    import hashlib
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "decode_traffic_counters.txt")
+    try:
+        entries = json.load(open(path))
+    except (OSError, ValueError):
+        return None
+    root = os.path.dirname(os.path.abspath(__file__))
+    for e in entries.values():
+        if e.get("workload") != w.name or e.get("layout") != layout:
+            continue
+        h = hashlib.sha256()
+        for f in e["kernel_sources"]:
+            h.update(open(os.path.join(root, f), "rb").read())
+        if h.hexdigest() != e["sources_sha256"]:
+            return None
+        units = w.batch * w.num_kv_heads
+        return int(round((e["dram_read_bytes"] + e["dram_write_bytes"]) * units / e["capture_units"]))
+    return None
+
+
 def measured_hbm_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -413,7 +437,7 @@ def main():
         "decode_ms": round(mean_decode_ms, 4),
         "append_us": round(statistics.mean(append_ms) * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout), "peak_kind": peak_kind,
                      "kernel": ("decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
                      + " + decode_combine_kernel (one kvq_decode_attention call)"},
         "prefill": {"gbs": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9, 1),

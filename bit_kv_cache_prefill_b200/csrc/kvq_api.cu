@@ -220,9 +220,14 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   for (int b = 0; b < cfg->batch; ++b)
     if (cache->seq_len_host[b] < 0 || cache->seq_len_host[b] > cfg->capacity) return KVQ_ERR_INVALID_ARG;
 
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVQ_ERR_CUDA;
+  static kvq::DeviceMemo sm_count;
+  const int sms = sm_count.get([] {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    return n;
+  });
+  if (sms <= 0) return KVQ_ERR_CUDA;
   const int occ = cfg->layout == KVQ_LAYOUT_ROWS_V2
                       ? kvq::decode_tc_ctas_per_sm(cfg->group_size, cfg->num_q_heads / cfg->num_kv_heads)
                       : kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size,

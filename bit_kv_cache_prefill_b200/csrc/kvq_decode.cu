@@ -650,8 +650,11 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a)
 template <int KB, int VB, int VPT, int GQ>
 cudaError_t launch_split(const DecodeArgs& a, cudaStream_t stream) {
   constexpr int smem = decode_smem_bytes<KB, VB, VPT, GQ>();
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
+  static DeviceMemo attr;
+  const int ok = attr.get([] {
+    return cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1 : -1;
+  });
+  if (ok < 0) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads));
   decode_split_kernel<KB, VB, VPT, GQ><<<grid, 32 * kDecodeWarps, smem, stream>>>(a);
   return cudaGetLastError();
@@ -659,13 +662,16 @@ cudaError_t launch_split(const DecodeArgs& a, cudaStream_t stream) {
 
 template <int KB, int VB, int VPT, int GQ>
 int occupancy() {
-  constexpr int smem = decode_smem_bytes<KB, VB, VPT, GQ>();
-  if (cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<KB, VB, VPT, GQ>, 32 * kDecodeWarps, smem) != cudaSuccess)
-    return 1;
-  return n > 0 ? n : 1;
+  static DeviceMemo memo;
+  return memo.get([] {
+    constexpr int smem = decode_smem_bytes<KB, VB, VPT, GQ>();
+    if (cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<KB, VB, VPT, GQ>, 32 * kDecodeWarps, smem) != cudaSuccess)
+      return 1;
+    return n > 0 ? n : 1;
+  });
 }
 
 // GQ template: the smallest of 1, 2, 4 that holds the query heads of one KV head.

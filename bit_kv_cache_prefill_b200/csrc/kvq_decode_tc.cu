@@ -822,8 +822,11 @@ __global__ void __launch_bounds__(kThreads, TcPlan<KB, VB, VPT, GQ>::kCtasPerSm)
 template <int KB, int VB, int VPT, int GQ>
 cudaError_t launch_tc(const DecodeArgs& a, cudaStream_t stream) {
   constexpr int smem = TcPlan<KB, VB, VPT, GQ>::kSmem;
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
+  static DeviceMemo attr;
+  const int ok = attr.get([] {
+    return cudaFuncSetAttribute(decode_tc_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1 : -1;
+  });
+  if (ok < 0) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads));
   decode_tc_kernel<KB, VB, VPT, GQ><<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace kvq {
 
 struct QuantizeArgs {
@@ -52,6 +54,28 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);     // spli
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // rows-v2 split kernel only
 int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);  // tile-v1 kernel
 int decode_tc_ctas_per_sm(int G, int gqa);                              // rows-v2 kernel (1 or 2)
+
+// Per-device memo of a small non-negative value (a function attribute already set, an occupancy, an
+// SM count), so that the launch path does not repeat runtime queries on every call. Concurrent first
+// calls may both compute the value; they store the same result.
+constexpr int kMaxDevices = 64;
+struct DeviceMemo {
+  std::atomic<int> v[kMaxDevices];
+  DeviceMemo() {
+    for (auto& x : v) x.store(-1, std::memory_order_relaxed);
+  }
+  // Value for the current device, computing it with fn() (returning < 0 on failure) the first time.
+  template <typename F>
+  int get(F&& fn) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return fn();
+    int x = v[dev].load(std::memory_order_acquire);
+    if (x >= 0) return x;
+    x = fn();
+    if (x >= 0) v[dev].store(x, std::memory_order_release);
+    return x;
+  }
+};
 
 constexpr int kDecodeWarps = 4;
 constexpr int kPartFloats = 2 + 128;  // m, l, o[128]

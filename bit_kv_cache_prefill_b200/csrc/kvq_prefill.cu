@@ -65,10 +65,21 @@ __device__ __forceinline__ uint64_t codes2(uint32_t x, uint64_t zf2, uint64_t in
   const float r1 = __fadd_rn(__uint_as_float(static_cast<uint32_t>(v >> 32)), kMagic);
   return static_cast<uint64_t>(__float_as_uint(r0)) | (static_cast<uint64_t>(__float_as_uint(r1)) << 32);
 }
-// The same for one value with the explicit clamp (flagged groups).
+// The same for one value with the explicit clamp (flagged groups); also returns the rounded bits.
 __device__ __forceinline__ uint32_t code_clamped(uint16_t x, float zf, float inv, int top) {
   const float v = fminf(__fmul_rn(__fsub_rn(h2f(x), zf), inv), static_cast<float>(top));
-  return __float_as_uint(__fadd_rn(v, kMagic)) & 0xffu;
+  return __float_as_uint(__fadd_rn(v, kMagic));
+}
+// The rounded bits of a code are r = 0x4B400000 + code (the add of 1.5 * 2^23 leaves the integer in
+// the low mantissa bits). A packed word is built as the sum of r << shift over its 2 * (16 / BITS)
+// codes plus kWordBias, which cancels the constant part modulo 2^32: the code fields do not overlap,
+// so the sum carries nothing between them, and each code costs one shift-add.
+constexpr uint32_t kMagicBits = 0x4B400000u;
+template <int BITS>
+__host__ __device__ constexpr uint32_t word_bias() {
+  uint32_t b = 0;
+  for (int k = 0; k < 16 / BITS; ++k) b += (kMagicBits << (BITS * k)) + (kMagicBits << (16 + BITS * k));
+  return 0u - b;
 }
 // Whether any element of a group can reach a code above 2^b - 1: v is monotone in x, so the group's
 // maximum decides.
@@ -190,18 +201,18 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
         x[4 * v + 2] = q4.z;
         x[4 * v + 3] = q4.w;
       }
-      uint32_t word = 0;
+      uint32_t word = word_bias<BITS>();
       if (!slow) {
 #pragma unroll
         for (int k = 0; k < P; ++k) {
           const uint64_t r = codes2(x[k], pk2(zf[2 * k], zf[2 * k + 1]), pk2(iv[2 * k], iv[2 * k + 1]));
-          word |= ((static_cast<uint32_t>(r) & top) << (BITS * k)) | ((static_cast<uint32_t>(r >> 32) & top) << (16 + BITS * k));
+          word += (static_cast<uint32_t>(r) << (BITS * k)) + (static_cast<uint32_t>(r >> 32) << (16 + BITS * k));
         }
       } else {
 #pragma unroll
         for (int k = 0; k < P; ++k) {
-          word |= code_clamped(static_cast<uint16_t>(x[k] & 0xffffu), zf[2 * k], iv[2 * k], top) << (BITS * k);
-          word |= code_clamped(static_cast<uint16_t>(x[k] >> 16), zf[2 * k + 1], iv[2 * k + 1], top) << (16 + BITS * k);
+          word += code_clamped(static_cast<uint16_t>(x[k] & 0xffffu), zf[2 * k], iv[2 * k], top) << (BITS * k);
+          word += code_clamped(static_cast<uint16_t>(x[k] >> 16), zf[2 * k + 1], iv[2 * k + 1], top) << (16 + BITS * k);
         }
       }
       dst[static_cast<int64_t>(t) * W] = word;
@@ -245,7 +256,7 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
           slow |= (pcl[g * 128 + cpair[i]] | pcl[g * 128 + cpair[i] + 1]) != 0;
         }
       }
-      uint32_t word = 0;
+      uint32_t word = word_bias<BITS>();
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const uint16_t* src = rows + (tl * kTile + r + 8 * u) * kRS;
@@ -255,10 +266,10 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
           const int j = jbase[i] + u;
           if (!slow) {
             const uint64_t rr = codes2(x, pk2(zf[2 * i], zf[2 * i + 1]), pk2(iv[2 * i], iv[2 * i + 1]));
-            word |= ((static_cast<uint32_t>(rr) & top) << (BITS * j)) | ((static_cast<uint32_t>(rr >> 32) & top) << (16 + BITS * j));
+            word += (static_cast<uint32_t>(rr) << (BITS * j)) + (static_cast<uint32_t>(rr >> 32) << (16 + BITS * j));
           } else {
-            word |= code_clamped(static_cast<uint16_t>(x & 0xffffu), zf[2 * i], iv[2 * i], top) << (BITS * j);
-            word |= code_clamped(static_cast<uint16_t>(x >> 16), zf[2 * i + 1], iv[2 * i + 1], top) << (16 + BITS * j);
+            word += code_clamped(static_cast<uint16_t>(x & 0xffffu), zf[2 * i], iv[2 * i], top) << (BITS * j);
+            word += code_clamped(static_cast<uint16_t>(x >> 16), zf[2 * i + 1], iv[2 * i + 1], top) << (16 + BITS * j);
           }
         }
       }
@@ -312,7 +323,7 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     const int c = 4 * cq, j = c / G;
     const int nw = nq * BITS / 32;  // complete words (nq is a multiple of 16)
     for (int wv = wv0; wv < nw; wv += kPThreads / 32) {
-      uint32_t wd[4] = {0u, 0u, 0u, 0u};
+      uint32_t wd[4] = {word_bias<BITS>(), word_bias<BITS>(), word_bias<BITS>(), word_bias<BITS>()};
 #pragma unroll
       for (int k = 0; k < P; ++k) {
 #pragma unroll
@@ -324,15 +335,15 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
           if (!pcl[t * 8 + j]) {
             const uint64_t z2 = pk2(pp.x, pp.x), i2 = pk2(pp.y, pp.y);
             const uint64_t r0 = codes2(x.x, z2, i2), r1 = codes2(x.y, z2, i2);
-            wd[0] |= (static_cast<uint32_t>(r0) & top) << sh;
-            wd[1] |= (static_cast<uint32_t>(r0 >> 32) & top) << sh;
-            wd[2] |= (static_cast<uint32_t>(r1) & top) << sh;
-            wd[3] |= (static_cast<uint32_t>(r1 >> 32) & top) << sh;
+            wd[0] += static_cast<uint32_t>(r0) << sh;
+            wd[1] += static_cast<uint32_t>(r0 >> 32) << sh;
+            wd[2] += static_cast<uint32_t>(r1) << sh;
+            wd[3] += static_cast<uint32_t>(r1 >> 32) << sh;
           } else {
-            wd[0] |= code_clamped(static_cast<uint16_t>(x.x & 0xffffu), pp.x, pp.y, top) << sh;
-            wd[1] |= code_clamped(static_cast<uint16_t>(x.x >> 16), pp.x, pp.y, top) << sh;
-            wd[2] |= code_clamped(static_cast<uint16_t>(x.y & 0xffffu), pp.x, pp.y, top) << sh;
-            wd[3] |= code_clamped(static_cast<uint16_t>(x.y >> 16), pp.x, pp.y, top) << sh;
+            wd[0] += code_clamped(static_cast<uint16_t>(x.x & 0xffffu), pp.x, pp.y, top) << sh;
+            wd[1] += code_clamped(static_cast<uint16_t>(x.x >> 16), pp.x, pp.y, top) << sh;
+            wd[2] += code_clamped(static_cast<uint16_t>(x.y & 0xffffu), pp.x, pp.y, top) << sh;
+            wd[3] += code_clamped(static_cast<uint16_t>(x.y >> 16), pp.x, pp.y, top) << sh;
           }
         }
       }
@@ -356,34 +367,49 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     }
   } else {
     // Tile v1: word w of lane L = 4r + qd in tile tl; pair j -> tokens 2qd + 8hh (+1), channel
-    // 16m + r + 8u, with (m, hh, u) from p = P w + j. The two codes of a pair are consecutive tokens
-    // of one channel and share packed fp32x2 arithmetic.
-    const int wl = tid & 3, L = (tid >> 2) & 31, hi = tid >> 7;
-    const int w = BITS == 2 ? wl : 4 * hi + wl;
-    const int tl0 = BITS == 2 ? 4 * hi : 0, ntl = BITS == 2 ? 4 : 8;
-    const int r = L >> 2, qd = L & 3;
+    // 16m + r + 8u, with (m, hh, u) from p = P w + j (so hh and u depend on j only). Thread (w, lane
+    // pair, tile part) builds the words of lanes L0 = 4 r0 + qd and L1 = L0 + 4 (r0 even): they hold the
+    // same tokens and the adjacent channels r0, r0 + 1, so one 4-byte load feeds both, and a token's two
+    // channels share packed fp32x2 arithmetic.
+    constexpr int NW = 2 * BITS;                    // words per lane per tile
+    constexpr int TPARTS = kPThreads / (NW * 16);   // 4 (2-bit) or 2 (4-bit)
+    constexpr int TPT = 8 / TPARTS;                 // tiles per thread
+    const int w = tid % NW, lp = (tid / NW) % 16, part = tid / (NW * 16);
+    const int qd = lp & 3, r0 = 2 * (lp >> 2);
+    const int L0 = 4 * r0 + qd;
     const int words = 64 * BITS;
-    const int widx = (w >> 2) * 128 + 4 * L + (w & 3);
-    uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words + widx;
-    for (int tl = tl0; tl < tl0 + ntl && tl * kTile < nq; ++tl) {
-      uint32_t word = 0;
+    const int widx0 = (w >> 2) * 128 + 4 * L0 + (w & 3);  // lane L1 = L0 + 4: widx0 + 16
+    const int ch0 = 16 * ((P * w) >> 2) + r0;              // channel of pair j: ch0 + 16 (j >> 2) + 8 (j & 1)
+    uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words + widx0;
+    for (int tl = part * TPT; tl < (part + 1) * TPT && tl * kTile < nq; ++tl) {
+      const int tb = tl * kTile + 2 * qd;  // token of pair j: tb + 8 ((j >> 1) & 1) (+1)
+      uint32_t acc0 = word_bias<BITS>(), acc1 = word_bias<BITS>();
 #pragma unroll
       for (int j = 0; j < P; ++j) {
-        const int p = P * w + j;
-        const int m = p >> 2, u = p & 1, hh = (p >> 1) & 1;
-        const int ch = 16 * m + r + 8 * u, gj = ch / G;
-        const int t = tl * kTile + 2 * qd + 8 * hh;
-        const uint16_t x0 = rows[t * kRS + ch], x1 = rows[(t + 1) * kRS + ch];
-        const float2 p0 = prm[t * 8 + gj], p1 = prm[(t + 1) * 8 + gj];
+        const int ch = ch0 + 16 * (j >> 2) + 8 * (j & 1), gj = ch / G;
+        const int t = tb + 8 * ((j >> 1) & 1);
+        const uint32_t xa = *reinterpret_cast<const uint32_t*>(rows + t * kRS + ch);        // token t, channels ch, ch + 1
+        const uint32_t xb = *reinterpret_cast<const uint32_t*>(rows + (t + 1) * kRS + ch);  // token t + 1
+        const float2 pa = prm[t * 8 + gj], pb = prm[(t + 1) * 8 + gj];
+        uint32_t ra0, ra1, rb0, rb1;
         if (!(pcl[t * 8 + gj] | pcl[(t + 1) * 8 + gj])) {
-          const uint64_t rr = codes2(static_cast<uint32_t>(x0) | (static_cast<uint32_t>(x1) << 16), pk2(p0.x, p1.x), pk2(p0.y, p1.y));
-          word |= ((static_cast<uint32_t>(rr) & top) << (BITS * j)) | ((static_cast<uint32_t>(rr >> 32) & top) << (16 + BITS * j));
+          const uint64_t ra = codes2(xa, pk2(pa.x, pa.x), pk2(pa.y, pa.y));
+          const uint64_t rb = codes2(xb, pk2(pb.x, pb.x), pk2(pb.y, pb.y));
+          ra0 = static_cast<uint32_t>(ra);
+          ra1 = static_cast<uint32_t>(ra >> 32);
+          rb0 = static_cast<uint32_t>(rb);
+          rb1 = static_cast<uint32_t>(rb >> 32);
         } else {
-          word |= code_clamped(x0, p0.x, p0.y, top) << (BITS * j);
-          word |= code_clamped(x1, p1.x, p1.y, top) << (16 + BITS * j);
+          ra0 = code_clamped(static_cast<uint16_t>(xa & 0xffffu), pa.x, pa.y, top);
+          ra1 = code_clamped(static_cast<uint16_t>(xa >> 16), pa.x, pa.y, top);
+          rb0 = code_clamped(static_cast<uint16_t>(xb & 0xffffu), pb.x, pb.y, top);
+          rb1 = code_clamped(static_cast<uint16_t>(xb >> 16), pb.x, pb.y, top);
         }
+        acc0 += (ra0 << (BITS * j)) + (rb0 << (16 + BITS * j));  // lane L0: channel ch
+        acc1 += (ra1 << (BITS * j)) + (rb1 << (16 + BITS * j));  // lane L1: channel ch + 1
       }
-      dst[static_cast<int64_t>(tl) * words] = word;
+      dst[static_cast<int64_t>(tl) * words] = acc0;
+      dst[static_cast<int64_t>(tl) * words + 16] = acc1;
     }
   }
 }
@@ -434,8 +460,11 @@ constexpr int kPrefillSmem = kPB * kRS * 2 + (kKeyScratch > kValScratch ? kKeySc
 
 template <int BK, int BV, int LAYOUT>
 cudaError_t launch_block(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(prefill_block_kernel<BK, BV, LAYOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
-  if (e != cudaSuccess) return e;
+  static DeviceMemo attr;
+  const int ok = attr.get([] {
+    return cudaFuncSetAttribute(prefill_block_kernel<BK, BV, LAYOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem) == cudaSuccess ? 1 : -1;
+  });
+  if (ok < 0) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>((max_len + kPB - 1) / kPB), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads), 2);
   prefill_block_kernel<BK, BV, LAYOUT><<<grid, kPThreads, kPrefillSmem, stream>>>(a);
   return cudaGetLastError();
