@@ -127,6 +127,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def reduce_over_ranks(dist, device, ms: float, *sums: float):
+    """Whole-job aggregates of a replicated run: the max of the per-rank times `ms` (the job ends with its
+    slowest rank) and the sums of `sums` (bytes, tokens) over the ranks. Without a process group the
+    values are returned unchanged."""
+    if dist is None:
+        return (float(ms),) + tuple(float(x) for x in sums)
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    out = (float(t.item()),)
+    if sums:
+        s = torch.tensor(list(sums), device=device, dtype=torch.float64)
+        dist.all_reduce(s)
+        out += tuple(float(x) for x in s.tolist())
+    return out
+
+
 def measured_traffic(w: inputs.Workload, layout: int):
     """DRAM bytes per decode-split launch from the committed ncu counters (profiles/decode_traffic_counters.txt, JSON), scaled
     from the captured batch to this one by the units processed; None if there is no capture for this
@@ -358,14 +374,9 @@ def main():
     total_bytes = float(sum(step_bytes))
     tokens = w.batch * args.steps
 
-    # max over ranks
-    if dist is not None:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        tb = torch.tensor([total_bytes, float(tokens)], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tb)
-        total_bytes, tokens = float(tb[0].item()), int(tb[1].item())
+    # max over ranks of the time, sums of the work
+    total_ms, total_bytes, tokens = reduce_over_ranks(dist, "cuda", total_ms, total_bytes, float(tokens))
+    tokens = int(tokens)
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -394,11 +405,7 @@ def main():
         barrier()
         e2e_ms = e0.elapsed_time(e1)
         e2e_bytes = float(sum(decode_bytes(w0, lens_e + i + 1) for i in range(args.steps)))
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-            e2e_bytes *= world
+        e2e_ms, e2e_bytes = reduce_over_ranks(dist, "cuda", e2e_ms, e2e_bytes)
         h2d = q_host.numel() * 2 + kn_host[0].numel() * 2 * 2
         d2h = out_host.numel() * 2
         e2e = {"value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),

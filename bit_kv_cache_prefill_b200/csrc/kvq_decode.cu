@@ -52,6 +52,12 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// cp.async of 16 bytes to a shared-space address with compile-time offsets folded into the
+// instruction's address operands (no per-copy address arithmetic).
+template <int SOFF, int GOFF>
+__device__ __forceinline__ void cp_async16_at(uint32_t saddr, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0+%2], [%1+%3], 16;\n" ::"r"(saddr), "l"(gmem), "n"(SOFF), "n"(GOFF));
+}
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
@@ -298,16 +304,25 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   const uint8_t* vz_ptr = reinterpret_cast<const uint8_t*>(a.v_zero + (unit * a.capacity + first_token) * VPT) + 16 * lane;
   const uint16_t* kp_src = (lane < 16 ? a.k_scale : a.k_zero) + unit * a.groups * kHeadDim + 8 * (lane & 15);
 
-  // issue(i): step i of this warp into stage i % kStages; the lane pointers advance one step per call
+  // issue(i): step i of this warp into stage i % kStages (tracked by stage_in); the lane pointers
+  // advance one step per call
+  static_assert(S::kKC % 512 == 0 && S::kKC / 512 <= 4 && S::kVC % 512 == 0 && S::kVC / 512 <= 4, "stage copies");
+  const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(ring)) + 16 * lane;
+  int stage_in = 0;
   auto issue = [&](int i) {
-    uint8_t* st = ring + (i % kStages) * S::kBytes + 16 * lane;
-#pragma unroll
-    for (int c = 0; c < S::kKC / 512; ++c) cp_async16(st + S::oKC + 512 * c, kc_ptr + 512 * c);
-#pragma unroll
-    for (int c = 0; c < S::kVC / 512; ++c) cp_async16(st + S::oVC + 512 * c, vc_ptr + 512 * c);
+    const uint32_t st = ring_s + stage_in * S::kBytes;
+    stage_in = stage_in == kStages - 1 ? 0 : stage_in + 1;
+    cp_async16_at<S::oKC, 0>(st, kc_ptr);
+    if constexpr (S::kKC / 512 > 1) cp_async16_at<S::oKC + 512, 512>(st, kc_ptr);
+    if constexpr (S::kKC / 512 > 2) cp_async16_at<S::oKC + 1024, 1024>(st, kc_ptr);
+    if constexpr (S::kKC / 512 > 3) cp_async16_at<S::oKC + 1536, 1536>(st, kc_ptr);
+    cp_async16_at<S::oVC, 0>(st, vc_ptr);
+    if constexpr (S::kVC / 512 > 1) cp_async16_at<S::oVC + 512, 512>(st, vc_ptr);
+    if constexpr (S::kVC / 512 > 2) cp_async16_at<S::oVC + 1024, 1024>(st, vc_ptr);
+    if constexpr (S::kVC / 512 > 3) cp_async16_at<S::oVC + 1536, 1536>(st, vc_ptr);
     if (lane < S::kVS / 16) {
-      cp_async16(st + S::oVS, vs_ptr);
-      cp_async16(st + S::oVZ, vz_ptr);
+      cp_async16_at<S::oVS, 0>(st, vs_ptr);
+      cp_async16_at<S::oVZ, 0>(st, vz_ptr);
     }
     const int t = first_token + i * kStepTokens;
     if (i == 0 || (t % kBlockTokens) == 0) {
@@ -332,12 +347,14 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
     cp_async_commit();
   }
 
+  int stage_out = 0;  // i % kStages for the consumed step
   for (int i = 0; i < nst; ++i) {
     if (i + kStages - 1 < nst) issue(i + kStages - 1);
     cp_async_commit();
     cp_async_wait<kStages - 1>();
     __syncwarp();
-    const uint8_t* st = ring + (i % kStages) * S::kBytes;
+    const uint8_t* st = ring + stage_out * S::kBytes;
+    stage_out = stage_out == kStages - 1 ? 0 : stage_out + 1;
     const int t = first_token + i * kStepTokens;
 
     // -- new key block: fold the scales of its KGB groups into the query (hi/lo fp16) and the
