@@ -52,7 +52,7 @@ class _CConfig(ctypes.Structure):
         ("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32), ("value_bits", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("residual", ctypes.c_int32), ("hadamard", ctypes.c_int32),
-        ("layout", ctypes.c_int32), ("capacity", ctypes.c_int64),
+        ("layout", ctypes.c_int32), ("sink", ctypes.c_int32), ("capacity", ctypes.c_int64),
     ]
 
 
@@ -100,10 +100,12 @@ class Config:
     capacity: int
     head_dim: int = 128
     layout: int = 1  # 1 = tile v1 (mma fragment order), 2 = rows v2 (token rows of keys, channel rows of values)
+    sink: int = 0    # 1: the first token stays in fp16 (an extra row after the ring)
 
     def c(self) -> _CConfig:
         return _CConfig(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.key_bits,
-                        self.value_bits, self.group_size, self.residual, self.hadamard, self.layout, self.capacity)
+                        self.value_bits, self.group_size, self.residual, self.hadamard, self.layout, self.sink,
+                        self.capacity)
 
 
 class Cache:
@@ -111,7 +113,7 @@ class Cache:
 
     def __init__(self, cfg: Config):
         B, H, cap, G = cfg.batch, cfg.num_kv_heads, cfg.capacity, cfg.group_size
-        ring = cfg.residual + G
+        ring = cfg.residual + G + cfg.sink  # ring slots, then the first token's row when the sink is on
         if cfg.layout == 2:
             self.k_codes = np.zeros((B, H, cap, 4 * cfg.key_bits), np.uint32)
             self.v_codes = np.zeros((B, H, (cap + 127) // 128, 128, 4 * cfg.value_bits), np.uint32)

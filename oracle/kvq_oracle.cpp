@@ -254,6 +254,7 @@ extern "C" {
 typedef struct {
   int32_t batch, num_q_heads, num_kv_heads, head_dim;
   int32_t key_bits, value_bits, group_size, residual, hadamard, layout;  // layout: 1 = tile v1, 2 = rows v2
+  int32_t sink;  // 1: the first token stays in fp16 (reading R10)
   int64_t capacity;
 } kvq_ref_config;
 
@@ -264,7 +265,7 @@ typedef struct {
   uint16_t* k_zero;   // same
   uint16_t* v_scale;  // [B][Hkv][Cap][128/G]
   uint16_t* v_zero;   // same
-  uint16_t* k_res;    // [B][Hkv][R+G][128] ring, fp16
+  uint16_t* k_res;    // [B][Hkv][R+G+sink][128] ring, fp16 (row R+G: the first token when sink is on)
   uint16_t* v_res;    // same
   int64_t* seq_len;   // [B]
 } kvq_ref_cache;
@@ -281,6 +282,7 @@ static int check_config(const kvq_ref_config* c) {
   if (G <= 0 || G % 16 || 128 % G) return REF_ERR_ARG;
   if (c->residual < 0 || c->capacity < 0 || c->capacity % G) return REF_ERR_ARG;
   if (c->layout != 1 && c->layout != 2) return REF_ERR_ARG;
+  if (c->sink != 0 && c->sink != 1) return REF_ERR_ARG;
   return REF_OK;
 }
 
@@ -313,6 +315,7 @@ static int key_param_index(const kvq_ref_config* c, int ch) { return c->layout =
 struct Dims {
   int64_t kw_tile, vw_tile, tiles, groups, ring, vpt;  // words per tile, tiles/unit, groups/unit, ring slots, value groups per token
   int64_t kwords, vwords;                              // code words per unit
+  int64_t res_rows;                                    // rows of k_res / v_res per unit: ring slots + the sink row
 };
 static Dims dims(const kvq_ref_config* c) {
   Dims d;
@@ -323,21 +326,27 @@ static Dims dims(const kvq_ref_config* c) {
   d.vwords = (c->layout == 2 ? (c->capacity + 127) / 128 * 128 : c->capacity) * 4 * c->value_bits;
   d.groups = c->capacity / c->group_size;
   d.ring = c->residual + c->group_size;
+  d.res_rows = d.ring + c->sink;
   d.vpt = 128 / c->group_size;
   return d;
 }
 
 // Quantize tokens [t0, t0 + G) of key unit `kt` (fp16 [T][128], already rotated if enabled) into key
 // group t0 / G, and the same tokens of value unit `vt` per token.
+// With the sink on (reading R10) the first token of the sequence stays out of the quantizer: key group
+// 0's min/max run over its other G - 1 tokens, and the first token's key codes, value codes, value
+// scale and value zero are 0 (it is read from its fp16 row instead).
 static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t unit, int64_t t0,
                           const uint16_t* kt, int64_t k_ld, const uint16_t* vt, int64_t v_ld) {
   const Dims d = dims(c);
   const int G = c->group_size;
-  // Keys: per channel over the G tokens of the group.
-  std::vector<uint8_t> kc(static_cast<size_t>(G) * 128);
+  const int skip = (c->sink && t0 == 0) ? 1 : 0;  // tokens at the start of the span kept out
+  // Keys: per channel over the G (or G - 1) tokens of the group.
+  std::vector<uint8_t> kc(static_cast<size_t>(G) * 128, 0);
   const int64_t g = t0 / G;
   for (int ch = 0; ch < 128; ++ch) {
-    GroupQ q = quantize_group(kt + ch, G, static_cast<int>(k_ld), c->key_bits, kc.data() + ch, 128);
+    GroupQ q = quantize_group(kt + skip * k_ld + ch, G - skip, static_cast<int>(k_ld), c->key_bits,
+                              kc.data() + skip * 128 + ch, 128);
     const int pos = key_param_index(c, ch);
     cache->k_scale[(unit * d.groups + g) * 128 + pos] = q.scale;
     cache->k_zero[(unit * d.groups + g) * 128 + pos] = q.zero;
@@ -358,7 +367,11 @@ static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, i
   for (int i = 0; i < G; ++i) {
     const int64_t t = t0 + i;
     for (int j = 0; j < d.vpt; ++j) {
-      GroupQ q = quantize_group(vt + i * v_ld + j * G, G, 1, c->value_bits, vc.data() + j * G, 1);
+      GroupQ q{0, 0};
+      if (i < skip)
+        std::memset(vc.data() + j * G, 0, G);
+      else
+        q = quantize_group(vt + i * v_ld + j * G, G, 1, c->value_bits, vc.data() + j * G, 1);
       cache->v_scale[(unit * c->capacity + t) * d.vpt + j] = q.scale;
       cache->v_zero[(unit * c->capacity + t) * d.vpt + j] = q.zero;
     }
@@ -400,8 +413,12 @@ static void prefill_unit(const kvq_ref_config* c, kvq_ref_cache* cache, const ui
   for (int64_t t0 = 0; t0 < Q; t0 += G) quantize_span(c, cache, unit, t0, &kt[t0 * 128], 128, &vt[t0 * 128], 128);
   for (int64_t t = Q; t < T; ++t) {
     const int64_t slot = t % d.ring;
-    std::memcpy(cache->k_res + (unit * d.ring + slot) * 128, &kt[t * 128], 256);
-    std::memcpy(cache->v_res + (unit * d.ring + slot) * 128, &vt[t * 128], 256);
+    std::memcpy(cache->k_res + (unit * d.res_rows + slot) * 128, &kt[t * 128], 256);
+    std::memcpy(cache->v_res + (unit * d.res_rows + slot) * 128, &vt[t * 128], 256);
+  }
+  if (c->sink && T > 0) {  // the first token's fp16 row (reading R10)
+    std::memcpy(cache->k_res + (unit * d.res_rows + d.ring) * 128, &kt[0], 256);
+    std::memcpy(cache->v_res + (unit * d.res_rows + d.ring) * 128, &vt[0], 256);
   }
 }
 
@@ -449,18 +466,24 @@ int kvq_ref_append_token(const kvq_ref_config* c, kvq_ref_cache* cache, const ui
       const uint16_t* ks = k_new + unit * 128;
       const uint16_t* vs = v_new + unit * 128;
       const int64_t slot = t % d.ring;
+      uint16_t* kslot = cache->k_res + (unit * d.res_rows + slot) * 128;
+      uint16_t* vslot = cache->v_res + (unit * d.res_rows + slot) * 128;
       if (c->hadamard)
-        rotate_key_f16(ks, cache->k_res + (unit * d.ring + slot) * 128);
+        rotate_key_f16(ks, kslot);
       else
-        std::memcpy(cache->k_res + (unit * d.ring + slot) * 128, ks, 256);
-      std::memcpy(cache->v_res + (unit * d.ring + slot) * 128, vs, 256);
+        std::memcpy(kslot, ks, 256);
+      std::memcpy(vslot, vs, 256);
+      if (c->sink && t == 0) {  // the first token's fp16 row (reading R10)
+        std::memcpy(cache->k_res + (unit * d.res_rows + d.ring) * 128, kslot, 256);
+        std::memcpy(cache->v_res + (unit * d.res_rows + d.ring) * 128, vslot, 256);
+      }
       if (Q_new > Q_old) {
         // Tokens [Q_old, Q_old + G) leave the window: gather them from the ring and quantize.
         std::vector<uint16_t> kt(static_cast<size_t>(G) * 128), vt(static_cast<size_t>(G) * 128);
         for (int i = 0; i < G; ++i) {
           const int64_t s = (Q_old + i) % d.ring;
-          std::memcpy(&kt[i * 128], cache->k_res + (unit * d.ring + s) * 128, 256);
-          std::memcpy(&vt[i * 128], cache->v_res + (unit * d.ring + s) * 128, 256);
+          std::memcpy(&kt[i * 128], cache->k_res + (unit * d.res_rows + s) * 128, 256);
+          std::memcpy(&vt[i * 128], cache->v_res + (unit * d.res_rows + s) * 128, 256);
         }
         quantize_span(c, cache, unit, Q_old, kt.data(), 128, vt.data(), 128);
       }
@@ -473,8 +496,9 @@ int kvq_ref_append_token(const kvq_ref_config* c, kvq_ref_cache* cache, const ui
 // Dequantized key / value of token t (fp64, reading R6) or the FP16 residual copy.
 static void key_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t unit, int64_t t, int64_t Q, double* out) {
   const Dims d = dims(c);
-  if (t >= Q) {
-    const uint16_t* r = cache->k_res + (unit * d.ring + t % d.ring) * 128;
+  if (t >= Q || (c->sink && t == 0)) {
+    const int64_t row = (c->sink && t == 0) ? d.ring : t % d.ring;
+    const uint16_t* r = cache->k_res + (unit * d.res_rows + row) * 128;
     for (int ch = 0; ch < 128; ++ch) out[ch] = half_to_float(r[ch]);
     return;
   }
@@ -494,8 +518,9 @@ static void key_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t
 
 static void value_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t unit, int64_t t, int64_t Q, double* out) {
   const Dims d = dims(c);
-  if (t >= Q) {
-    const uint16_t* r = cache->v_res + (unit * d.ring + t % d.ring) * 128;
+  if (t >= Q || (c->sink && t == 0)) {
+    const int64_t row = (c->sink && t == 0) ? d.ring : t % d.ring;
+    const uint16_t* r = cache->v_res + (unit * d.res_rows + row) * 128;
     for (int ch = 0; ch < 128; ++ch) out[ch] = half_to_float(r[ch]);
     return;
   }

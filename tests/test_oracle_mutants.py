@@ -51,6 +51,13 @@ MUTANTS = [
      "  *word = (block * 128 + c) * (4 * bits) + j / P;",
      "  *word = (block * 128 + c) * (4 * bits) + ((j / P) ^ 1);",
      ["test_layout_matches_hand_worked_examples"]),
+    ("sink_first_token_in_group_zero_stats",
+     "  const int skip = (c->sink && t0 == 0) ? 1 : 0;", "  const int skip = 0;",
+     ["test_sink_first_token_left_out_of_group_zero"]),
+    ("sink_row_ignored_by_decode",
+     "  if (t >= Q || (c->sink && t == 0)) {\n    const int64_t row = (c->sink && t == 0) ? d.ring : t % d.ring;\n    const uint16_t* r = cache->k_res",
+     "  if (t >= Q) {\n    const int64_t row = (c->sink && t == 0) ? d.ring : t % d.ring;\n    const uint16_t* r = cache->k_res",
+     ["test_sink_dominant_first_token_returns_its_fp16_value"]),
     ("value_group_index_off",
      "    const int j = ch / c->group_size;", "    const int j = (ch / c->group_size + 1) % d.vpt;",
      ["test_quantized_attention_equals_library_attention_on_dequantized_cache"]),
@@ -79,6 +86,8 @@ def _run_pin(fn_name, mod):
         "test_quantizer_two_valued_and_grid_round_trip": [dict(bits=2), dict(bits=4)],
         "test_quantized_attention_equals_library_attention_on_dequantized_cache":
             [dict(kb=2, vb=2, G=32, R=32, had=0, layout=1), dict(kb=2, vb=2, G=32, R=32, had=0, layout=2)],
+        "test_sink_first_token_left_out_of_group_zero": [dict(layout=1), dict(layout=2)],
+        "test_sink_dominant_first_token_returns_its_fp16_value": [dict(layout=1), dict(layout=2)],
     }.get(fn_name, [dict()])
     for kw in params:
         fn(mod, **kw)

@@ -255,8 +255,8 @@ def test_layout_v2_is_a_bijection_onto_rows(oracle_mod, kind, bits):
 # --------------------------------------------------------------------------------------------------
 # whole-cache behaviour
 # --------------------------------------------------------------------------------------------------
-def _cfg(oracle_mod, B=2, Hq=4, Hkv=2, kb=2, vb=2, G=32, R=32, had=0, cap=512, layout=1):
-    return oracle_mod.Config(B, Hq, Hkv, kb, vb, G, R, had, cap, layout=layout)
+def _cfg(oracle_mod, B=2, Hq=4, Hkv=2, kb=2, vb=2, G=32, R=32, had=0, cap=512, layout=1, sink=0):
+    return oracle_mod.Config(B, Hq, Hkv, kb, vb, G, R, had, cap, layout=layout, sink=sink)
 
 
 def _inputs(B, T, Hkv, Hq, seed, outliers=True):
@@ -484,3 +484,101 @@ def test_average_bits_closed_form(oracle_mod, bits, G):
                       + c.v_scale.nbytes + c.v_zero.nbytes)
     per_elem = total_bits / (2 * 1024 * 128)
     assert per_elem == bits + 32 / G
+
+
+# ---- fp16 first token (attention sink): KVQuant review, Method; wiki page, verification notes ------
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_sink_first_token_left_out_of_group_zero(oracle_mod, layout):
+    # Token 0 is made the unique minimum of every channel of key group 0: with the sink on, group 0's
+    # zero-point must be the minimum over tokens 1..G-1 (brute force here), not token 0's value, and
+    # token 0's own codes and value scale / zero must be 0.
+    B, Hkv, Hq, G, T = 1, 1, 1, 32, 160
+    k, v, _ = _inputs(B, T, Hkv, Hq, 41)
+    k[0, 0, 0, :] = np.float16(-1000.0)
+    v[0, 0, 0, :] = np.float16(-1000.0)
+    for sink in (0, 1):
+        cfg = _cfg(oracle_mod, B, Hq, Hkv, G=G, R=0, cap=T, layout=layout, sink=sink)
+        cache = oracle_mod.Cache(cfg)
+        oracle_mod.quantize_prefill(cfg, cache, k, v, [T])
+        zero = cache.k_zero[0, 0, 0].view(np.float16).astype(np.float64)
+        want = k[0, 1:G, 0, :].astype(np.float64).min(axis=0) if sink else np.full(128, -1000.0)
+        for c in range(128):
+            pos = oracle_mod.key_param_pos(c) if layout == 1 else c
+            assert zero[pos] == want[c], (sink, c)
+        if sink:
+            assert all(_key_code(oracle_mod, cfg, cache, 0, 0, 0, c) == 0 for c in range(128))
+            assert all(_value_code(oracle_mod, cfg, cache, 0, 0, 0, c) == 0 for c in range(128))
+            assert not cache.v_scale[0, 0, 0].any() and not cache.v_zero[0, 0, 0].any()
+            np.testing.assert_array_equal(cache.k_res[0, 0, G], k[0, 0, 0].view(np.uint16))  # row R + G
+            np.testing.assert_array_equal(cache.v_res[0, 0, G], v[0, 0, 0].view(np.uint16))
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_sink_dominant_first_token_returns_its_fp16_value(oracle_mod, layout):
+    # The query points along token 0's key with a margin of e^-60 over every other token, so the
+    # softmax is token 0 to within 1e-20: with the sink on the output is token 0's fp16 value exactly
+    # (to fp64 rounding); without it, token 0 is read back through its 2-bit codes and misses by the
+    # quantization error.
+    B, Hkv, Hq, G, T = 1, 1, 1, 32, 300
+    k, v, _ = _inputs(B, T, Hkv, Hq, 43, outliers=False)
+    k[0, 0, 0, :] = np.float16(16.0)
+    q = np.full((1, 1, 128), np.float16(0.5), np.float16)
+    scale = 1.0 / math.sqrt(128)
+    base = (k[0, :, 0, :].astype(np.float64) @ q[0, 0].astype(np.float64)) * scale
+    assert base[0] - base[1:].max() > 60.0
+    outs = {}
+    for sink in (0, 1):
+        cfg = _cfg(oracle_mod, B, Hq, Hkv, G=G, R=32, cap=320, layout=layout, sink=sink)
+        cache = oracle_mod.Cache(cfg)
+        oracle_mod.quantize_prefill(cfg, cache, k, v, [T])
+        outs[sink] = oracle_mod.decode(cfg, cache, q, scale)[0, 0]
+    np.testing.assert_allclose(outs[1], v[0, 0, 0].astype(np.float64), rtol=0, atol=1e-13)
+    assert np.abs(outs[0] - v[0, 0, 0].astype(np.float64)).max() > 1e-2
+
+
+def test_sink_without_quantization_equals_library_attention(oracle_mod):
+    # R >= T: nothing is quantized, and the fp16 first-token row holds the same bits as the window did,
+    # so the result is plain softmax attention (GQA 2:1).
+    B, T, Hkv, Hq = 2, 200, 2, 4
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, R=256, cap=512, sink=1)
+    k, v, q = _inputs(B, T, Hkv, Hq, 47)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [T, T - 57])
+    out = oracle_mod.decode(cfg, cache, q, 1 / math.sqrt(128))
+    for b, Tb in enumerate([T, T - 57]):
+        kb = k[b, :Tb].astype(np.float64).transpose(1, 0, 2)[None]
+        vb = v[b, :Tb].astype(np.float64).transpose(1, 0, 2)[None]
+        ref = _sdpa(q[b:b + 1].astype(np.float64), kb, vb, 1 / math.sqrt(128))
+        np.testing.assert_allclose(out[b], ref[0], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+@pytest.mark.parametrize("had", [0, 1])
+def test_sink_streaming_from_empty_equals_bulk(oracle_mod, layout, had):
+    # Starting from an empty cache, the first append writes the fp16 first-token row and the first
+    # flush leaves token 0 out of group 0; the result must match a bulk prefill bit for bit.
+    B, Hkv, Hq, G, R = 2, 2, 2, 32, 16
+    n = 4 * G + 9
+    cap = ((n + G - 1) // G) * G
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, had, cap=cap, layout=layout, sink=1)
+    k, v, _ = _inputs(B, n, Hkv, Hq, 53)
+    stream = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, stream, k[:, :0], v[:, :0], [0, 0])
+    for t in range(n):
+        oracle_mod.append_token(cfg, stream, k[:, t], v[:, t])
+    bulk = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, bulk, k, v, [n, n])
+    Q = (n - R) // G * G
+    if layout == 1:
+        np.testing.assert_array_equal(stream.k_codes[:, :, : Q // 16], bulk.k_codes[:, :, : Q // 16])
+        np.testing.assert_array_equal(stream.v_codes[:, :, : Q // 16], bulk.v_codes[:, :, : Q // 16])
+    else:
+        np.testing.assert_array_equal(stream.k_codes[:, :, :Q], bulk.k_codes[:, :, :Q])
+        np.testing.assert_array_equal(stream.v_codes[:, :, 0, :, : Q * 2 // 32], bulk.v_codes[:, :, 0, :, : Q * 2 // 32])
+    for key in ("k_scale", "k_zero"):
+        np.testing.assert_array_equal(getattr(stream, key)[:, :, : Q // G], getattr(bulk, key)[:, :, : Q // G])
+    for key in ("v_scale", "v_zero"):
+        np.testing.assert_array_equal(getattr(stream, key)[:, :, :Q], getattr(bulk, key)[:, :, :Q])
+    np.testing.assert_array_equal(stream.k_res[:, :, R + G], bulk.k_res[:, :, R + G])
+    np.testing.assert_array_equal(stream.v_res[:, :, R + G], bulk.v_res[:, :, R + G])
