@@ -43,28 +43,32 @@ METRIC = "decode-attn effective KV HBM GB/s (fraction of B200 peak); tokens/s"
 # ---------------------------------------------------------------------------------------------------
 # algorithmic bytes (what the method must move), per unit of work
 # ---------------------------------------------------------------------------------------------------
-def decode_bytes(w: inputs.Workload, lens: np.ndarray) -> int:
+def decode_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
     """Bytes one decode call must read/write: packed codes + key group scale/zero + value token
-    scale/zero for the quantized tokens, fp16 K/V for the window, q in and out."""
+    scale/zero for the quantized tokens, fp16 K/V for the window (and for the first token when the
+    sink is on), q in and out."""
     G, R = w.group_size, w.residual
     total = 0
     for T in lens:
         T = int(T)
         Q = max(T - R, 0) // G * G
         per_unit = Q * 128 * (w.key_bits + w.value_bits) // 8 + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4
+        if sink and Q > 0:
+            per_unit += 128 * 4
         total += w.num_kv_heads * per_unit
     return total + 2 * w.batch * w.num_q_heads * 128 * 2
 
 
-def prefill_bytes(w: inputs.Workload, lens: np.ndarray) -> int:
-    """fp16 K and V read + codes, scales, zero-points and window written."""
+def prefill_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
+    """fp16 K and V read + codes, scales, zero-points and window (and the sink row) written."""
     G, R = w.group_size, w.residual
     total = 0
     for T in lens:
         T = int(T)
         Q = max(T - R, 0) // G * G
         total += w.num_kv_heads * (T * 128 * 4 + Q * 128 * (w.key_bits + w.value_bits) // 8
-                                   + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4)
+                                   + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4
+                                   + (128 * 4 if sink and T > 0 else 0))
     return total
 
 
@@ -179,7 +183,7 @@ def measured_hbm_peak():
 # ---------------------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------------------------------
-def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0):
+def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int = 1, sink: int = 0):
     """Time the oracle's decode on a bounded sample of the workload: whole (sequence, KV head) units
     batched into one oracle problem (enough units to give every host core a query head), decoded
     repeatedly until about budget_s seconds have passed. Returns (GB/s of algorithmic decode bytes,
@@ -198,7 +202,10 @@ def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0):
     lens = np.array([int(lens_all[b]) for b, _ in picked], np.int64)
     Tmax = int(lens.max())
     cap = int(math.ceil(Tmax / w.group_size) * w.group_size)
-    ocfg = ref.Config(n, g, 1, w.key_bits, w.value_bits, w.group_size, w.residual, w.hadamard, cap)
+    if layout == 2:
+        cap = -(-cap // 128) * 128
+    ocfg = ref.Config(n, g, 1, w.key_bits, w.value_bits, w.group_size, w.residual, w.hadamard, cap,
+                      layout=layout, sink=sink)
     k = np.zeros((n, Tmax, 1, 128), np.float16)
     v = np.zeros_like(k)
     qs = np.zeros((n, g, 128), np.float16)
@@ -217,9 +224,18 @@ def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0):
         ref.decode(ocfg, oc, qs, 1 / math.sqrt(128), threads=threads)
         spent += time.perf_counter() - t0
         calls += 1
-    per_call = decode_bytes(w.scaled(batch=n, num_q_heads=g, num_kv_heads=1), lens)
+    per_call = decode_bytes(w.scaled(batch=n, num_q_heads=g, num_kv_heads=1), lens, sink)
     desc = f"{n} (sequence, KV head) units of {w.name} ({int(lens.sum())} tokens), decode x{calls}"
     return per_call * calls / spent / 1e9, threads, desc
+
+
+def workload_config(w: inputs.Workload, args, step_bytes: int) -> dict:
+    """The JSON line's config, the same for both arms."""
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "key_bits": w.key_bits, "value_bits": w.value_bits,
+            "group_size": w.group_size, "residual": w.residual, "hadamard": w.hadamard,
+            "ragged": bool(w.ragged_min), "parallelism": f"replicas{args.gpus}", "layout": args.layout,
+            "sink": args.sink, "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
 
 
 def run_reference(args, w):
@@ -234,18 +250,16 @@ def run_reference(args, w):
     per_step = []
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
-        gbs, cores, sample = oracle_decode_sample(w, budget_s=budget)
+        gbs, cores, sample = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink)
         if i >= args.warmup:
             per_step.append(gbs)
     value = statistics.mean(per_step)
-    step_bytes = decode_bytes(w, lens)
+    step_bytes = decode_bytes(w, lens, args.sink)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_bytes / (value * 1e9) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "num_q_heads": w.num_q_heads,
-                   "num_kv_heads": w.num_kv_heads, "key_bits": w.key_bits, "value_bits": w.value_bits,
-                   "group_size": w.group_size, "residual": w.residual, "hadamard": w.hadamard},
+        "config": workload_config(w, args, step_bytes),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -269,6 +283,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling captures)")
     ap.add_argument("--layout", type=int, default=1, choices=[1, 2],
                     help="packed layout: 1 = tile v1 (mma.sync decode), 2 = rows v2 (tcgen05 decode)")
+    ap.add_argument("--sink", type=int, default=0, choices=[0, 1],
+                    help="1: keep every sequence's first token in fp16 (attention sink)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w0 = inputs.WORKLOADS[args.workload]
@@ -308,7 +324,7 @@ def main():
     if args.layout == 2:
         cap = -(-cap // 128) * 128  # rows v2 stores values in whole 128-token blocks
     cfg = kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size, w.residual,
-                          w.hadamard, cap, layout=args.layout)
+                          w.hadamard, cap, layout=args.layout, sink=args.sink)
     cache = kvq.Cache(cfg)
     stream = torch.cuda.current_stream()
 
@@ -322,7 +338,7 @@ def main():
         torch.cuda.synchronize()
         if i > 0:
             pre_ms.append(e0.elapsed_time(e1))
-    pre_bytes = prefill_bytes(w0, lens0)
+    pre_bytes = prefill_bytes(w0, lens0, args.sink)
     del kd, vd
     torch.cuda.empty_cache()
 
@@ -370,7 +386,7 @@ def main():
     decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
     append_ms = [e[0].elapsed_time(e[1]) for e in evs]
     # bytes per step from the lengths each decode actually saw (append happens first)
-    step_bytes = [decode_bytes(w0, lens_before + i + 1) for i in range(args.steps)]
+    step_bytes = [decode_bytes(w0, lens_before + i + 1, args.sink) for i in range(args.steps)]
     total_bytes = float(sum(step_bytes))
     tokens = w.batch * args.steps
 
@@ -404,7 +420,7 @@ def main():
         e1.record(stream)
         barrier()
         e2e_ms = e0.elapsed_time(e1)
-        e2e_bytes = float(sum(decode_bytes(w0, lens_e + i + 1) for i in range(args.steps)))
+        e2e_bytes = float(sum(decode_bytes(w0, lens_e + i + 1, args.sink) for i in range(args.steps)))
         e2e_ms, e2e_bytes = reduce_over_ranks(dist, "cuda", e2e_ms, e2e_bytes)
         h2d = q_host.numel() * 2 + kn_host[0].numel() * 2 * 2
         d2h = out_host.numel() * 2
@@ -434,11 +450,7 @@ def main():
         "vs_baseline": None,
         "dtype": "u2/u4 codes, fp16 in/out, fp32 accumulate",
         "data": "synthetic",
-        "config": {"workload": w0.name, "batch": w0.batch, "seq_len": w0.seq_len, "num_q_heads": w0.num_q_heads,
-                   "num_kv_heads": w0.num_kv_heads, "key_bits": w0.key_bits, "value_bits": w0.value_bits,
-                   "group_size": w0.group_size, "residual": w0.residual, "hadamard": w0.hadamard,
-                   "ragged": bool(w0.ragged_min), "parallelism": f"replicas{args.gpus}", "layout": args.layout,
-                   "l2": f"inputs larger than L2 ({step_bytes[0] / 2**20:.0f} MiB read per decode > 126 MiB)"},
+        "config": workload_config(w0, args, step_bytes[0]),
         "tokens_per_s": round(tokens / (total_ms * 1e-3), 1),
         "frac_of_nominal_8tbs": round(value / NOMINAL_HBM_GBS, 4),
         "decode_ms": round(mean_decode_ms, 4),
@@ -458,7 +470,7 @@ def main():
         import oracle as ref
 
         ref.build()
-        gbs, cores, sample = oracle_decode_sample(w0)
+        gbs, cores, sample = oracle_decode_sample(w0, layout=args.layout, sink=args.sink)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     print(json.dumps(line), flush=True)

@@ -34,6 +34,7 @@ kvq_status check_config(const kvq_config* c) {
   if (G != 16 && G != 32 && G != 64 && G != 128) return KVQ_ERR_INVALID_ARG;
   if (c->residual < 0 || c->residual > kMaxResidual) return KVQ_ERR_INVALID_ARG;
   if (c->hadamard != 0 && c->hadamard != 1) return KVQ_ERR_INVALID_ARG;
+  if (c->sink != 0 && c->sink != 1) return KVQ_ERR_INVALID_ARG;
   if (c->capacity < 0 || c->capacity % G != 0) return KVQ_ERR_INVALID_ARG;
   if (c->capacity >= (int64_t(1) << 31)) return KVQ_ERR_INVALID_ARG;  // token indices are 32-bit on the device
   if (c->layout == KVQ_LAYOUT_ROWS_V2 && c->capacity % 128 != 0) return KVQ_ERR_INVALID_ARG;  // whole value blocks
@@ -52,7 +53,7 @@ void buffer_bytes(const kvq_config* c, size_t out[KVQ_NUM_BUFFERS]) {
   out[KVQ_BUF_K_ZERO] = out[KVQ_BUF_K_SCALE];
   out[KVQ_BUF_V_SCALE] = units * cap * (128 / G) * 2;
   out[KVQ_BUF_V_ZERO] = out[KVQ_BUF_V_SCALE];
-  out[KVQ_BUF_K_RES] = units * (static_cast<size_t>(c->residual) + G) * 128 * 2;
+  out[KVQ_BUF_K_RES] = units * (static_cast<size_t>(c->residual) + G + c->sink) * 128 * 2;
   out[KVQ_BUF_V_RES] = out[KVQ_BUF_K_RES];
 }
 
@@ -93,6 +94,8 @@ QuantizeArgs quantize_args(const kvq_config* c, kvq_cache* k) {
   a.groups = c->capacity / c->group_size;
   a.ring = static_cast<int64_t>(c->residual) + c->group_size;
   a.layout = c->layout;
+  a.sink = c->sink;
+  a.res_rows = a.ring + c->sink;
   a.vwords = (c->layout == KVQ_LAYOUT_ROWS_V2 ? (c->capacity + 127) / 128 * 128 : c->capacity) * 4 * c->value_bits;
   return a;
 }
@@ -262,6 +265,8 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   a.tiles = cfg->capacity / kvq::kTile;
   a.groups = cfg->capacity / cfg->group_size;
   a.ring = static_cast<int64_t>(cfg->residual) + cfg->group_size;
+  a.sink = cfg->sink;
+  a.res_rows = a.ring + cfg->sink;
   a.layout = cfg->layout;
   a.split_len = L;
   a.nsplit = nsplit;

@@ -398,6 +398,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
         s[u][1] = __shfl_sync(kFull, s[u][1], src);
       }
     }
+    if (a.sink && t == 0 && r == 0) s[0][0] = -CUDART_INF_F;  // the sink token is read from its fp16 row
 
     // -- online softmax for head h_d over the step
     float tmax = fmaxf(s[0][0], s[0][1]);
@@ -535,8 +536,10 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   // ---- FP16 window tokens [Q, T), spread over all splits of the unit: this CTA takes tokens
   //      Q + split + k * ns (ns = splits holding tokens), warp w the k = w (mod 4); batches of 8 with
   //      all loads issued first. Lane l holds channels 4l .. 4l + 3; the batch's partial is merged
-  //      into the warp partial in shared memory.
+  //      into the warp partial in shared memory. With the sink on and Q > 0 the list starts one
+  //      earlier, at Q - 1, which stands for the sink token's row R + G.
   {
+    const int W0 = (a.sink && Q > 0) ? Q - 1 : Q;
     const int ns = (T + L - 1) / L;
     float qr[GQ][4];
 #pragma unroll
@@ -547,16 +550,16 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
       qr[h][2] = v.z;
       qr[h][3] = v.w;
     }
-    const uint2* kres = reinterpret_cast<const uint2*>(a.k_res + unit * a.ring * kHeadDim) + lane;
-    const uint2* vres = reinterpret_cast<const uint2*>(a.v_res + unit * a.ring * kHeadDim) + lane;
-    for (int k0 = warp; Q + split + k0 * ns < T; k0 += 4 * 8) {
+    const uint2* kres = reinterpret_cast<const uint2*>(a.k_res + unit * a.res_rows * kHeadDim) + lane;
+    const uint2* vres = reinterpret_cast<const uint2*>(a.v_res + unit * a.res_rows * kHeadDim) + lane;
+    for (int k0 = warp; W0 + split + k0 * ns < T; k0 += 4 * 8) {
       uint2 kk[8], vv[8];
       bool valid[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int tt = Q + split + (k0 + 4 * j) * ns;
+        const int tt = W0 + split + (k0 + 4 * j) * ns;
         valid[j] = tt < T;
-        const int slot = valid[j] ? static_cast<int>(tt % a.ring) : 0;
+        const int slot = !valid[j] ? 0 : tt < Q ? static_cast<int>(a.ring) : static_cast<int>(tt % a.ring);
         kk[j] = kres[slot * (kHeadDim / 4)];
         vv[j] = vres[slot * (kHeadDim / 4)];
       }

@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, TcPlan<KB, VB, VPT, GQ>::kCtasPerSm)
 
     float s[GQ], p[GQ], sv[VPT], zv[VPT];
     bool exceed = false;
-    const bool valid = t_step + row < qend;
+    const bool valid = t_step + row < qend && t_step + row >= a.sink;  // the sink token: fp16 row instead
 #pragma unroll
     for (int h = 0; h < GQ; ++h) s[h] = p[h] = 0.f;
     // B_PV row of this token from p: hi/lo of p * sv per (value group, head); zero for masked tokens.
@@ -718,8 +718,10 @@ __global__ void __launch_bounds__(kThreads, TcPlan<KB, VB, VPT, GQ>::kCtasPerSm)
 
   // ---- FP16 window tokens [Q, T), spread over all splits of the unit: this CTA takes tokens
   //      Q + split + k * ns (ns = splits holding tokens), warp w the k = w (mod 8), in batches of 8
-  //      with all loads issued first. Lane l holds channels 4l .. 4l + 3.
+  //      with all loads issued first. Lane l holds channels 4l .. 4l + 3. With the sink on and Q > 0
+  //      the list starts at Q - 1, which stands for the sink token's row R + G.
   {
+    const int W0 = (a.sink && Q > 0) ? Q - 1 : Q;
     const int ns = (T + L - 1) / L;
     float qr[GQ][4];
 #pragma unroll
@@ -731,16 +733,16 @@ __global__ void __launch_bounds__(kThreads, TcPlan<KB, VB, VPT, GQ>::kCtasPerSm)
       qr[h][3] = v.w;
     }
     float* cw = wp + warp * GQ * kPartStride;
-    const uint2* kres = reinterpret_cast<const uint2*>(a.k_res + unit * a.ring * kHeadDim) + lane;
-    const uint2* vres = reinterpret_cast<const uint2*>(a.v_res + unit * a.ring * kHeadDim) + lane;
-    for (int k0 = warp; Q + split + k0 * ns < T; k0 += 8 * 8) {
+    const uint2* kres = reinterpret_cast<const uint2*>(a.k_res + unit * a.res_rows * kHeadDim) + lane;
+    const uint2* vres = reinterpret_cast<const uint2*>(a.v_res + unit * a.res_rows * kHeadDim) + lane;
+    for (int k0 = warp; W0 + split + k0 * ns < T; k0 += 8 * 8) {
       uint2 kk[8], vv[8];
       bool valid[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int tt = Q + split + (k0 + 8 * j) * ns;
+        const int tt = W0 + split + (k0 + 8 * j) * ns;
         valid[j] = tt < T;
-        const int slot = valid[j] ? static_cast<int>(tt % a.ring) : 0;
+        const int slot = !valid[j] ? 0 : tt < Q ? static_cast<int>(a.ring) : static_cast<int>(tt % a.ring);
         kk[j] = kres[slot * (kHeadDim / 4)];
         vv[j] = vres[slot * (kHeadDim / 4)];
       }

@@ -25,6 +25,8 @@ struct QuantizeArgs {
   int64_t capacity, tiles, groups, ring;  // per unit: capacity tokens, capacity/16 tiles, capacity/G groups, R+G slots
   int layout;                             // KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2
   int64_t vwords;                         // value code words per unit
+  int sink;                               // 1: token 0 stays in fp16 in ring row R+G
+  int64_t res_rows;                       // rows of k_res / v_res per unit: R + G + sink
 };
 
 struct DecodeArgs {
@@ -42,6 +44,8 @@ struct DecodeArgs {
   float* part;             // split partials [units][nsplit][g][2 + 128]
   int batch, num_q_heads, num_kv_heads, gqa, G, R, key_bits, value_bits, hadamard;
   int64_t capacity, tiles, groups, ring;
+  int sink;          // 1: token 0 is read from ring row R+G (fp16) and masked in the quantized part
+  int64_t res_rows;  // rows of k_res / v_res per unit: R + G + sink
   int layout;     // KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2
   int split_len;  // tokens per split (multiple of 64; rows v2: multiple of 128)
   int nsplit;     // splits per unit in the grid

@@ -131,13 +131,15 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
   uint8_t* pcl = reinterpret_cast<uint8_t*>(pinv + 8 * 128);  // [8][128]
   const int tid = threadIdx.x;
 
+  // With the sink on, the block at t0 = 0 keeps token 0 out of group 0 (its min/max and its codes).
+  const bool sink0 = a.sink && t0 == 0;
   // min / max: thread (channel pair cp, quarter q) scans quarter q of every group
   {
     const int cp = tid & 63, q = tid >> 6, ql = G / 4;
     for (int g = 0; g < NG; ++g) {
       uint32_t mn = 0xffffffffu, mx = 0u;
       const uint16_t* src = rows + (g * G + q * ql) * kRS + 2 * cp;
-      for (int i = 0; i < ql; ++i) {
+      for (int i = (sink0 && g == 0 && q == 0) ? 1 : 0; i < ql; ++i) {
         const uint32_t k = order_key2(*reinterpret_cast<const uint32_t*>(src + i * kRS));
         mn = vmin2(mn, k);
         mx = vmax2(mx, k);
@@ -165,6 +167,8 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
       pz[g * 128 + c] = p.zf;
       pinv[g * 128 + c] = p.inv;
       pcl[g * 128 + c] = needs_clamp(p, kmax, top) ? 1 : 0;
+      // token 0 becomes the group's zero, which codes to 0 on every path (x - zf = 0)
+      if (sink0 && g == 0) const_cast<uint16_t*>(rows)[c] = p.z16;
     }
   }
   __syncthreads();
@@ -305,12 +309,14 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
       mx = vmax2(mx, vmax2(vmax2(k0, k1), vmax2(k2, k3)));
     }
     const uint32_t kmin = min(mn & 0xffffu, mn >> 16), kmax = max(mx & 0xffffu, mx >> 16);
-    const QuantParams p = make_params(kmin, kmax, BITS);
+    QuantParams p = make_params(kmin, kmax, BITS);
+    const bool sink_tok = a.sink && t0 + t == 0;  // the sink token: scale, zero and codes 0
+    if (sink_tok) p = QuantParams{0.f, 0.f, 0, 0, true};
     const int64_t pidx = (unit * a.capacity + t0 + t) * VPT + j;
     a.v_scale[pidx] = p.s16;
     a.v_zero[pidx] = p.z16;
     prm[t * 8 + j] = make_float2(p.zf, p.inv);
-    pcl[t * 8 + j] = needs_clamp(p, kmax, top) ? 1 : 0;
+    pcl[t * 8 + j] = !sink_tok && needs_clamp(p, kmax, top) ? 1 : 0;
   }
   __syncthreads();
 
@@ -440,9 +446,12 @@ __global__ void __launch_bounds__(kPThreads) prefill_block_kernel(QuantizeArgs a
     rotate_block(rows, n);
     __syncthreads();
   }
+  uint16_t* ring = (is_key ? a.k_res : a.v_res) + unit * a.res_rows * kHeadDim;
+  // The sink token's fp16 row (ring row R + G), copied before key_block overwrites row 0
+  if (a.sink && t0 == 0 && threadIdx.x < 16)
+    reinterpret_cast<uint4*>(ring + a.ring * kHeadDim)[threadIdx.x] = reinterpret_cast<const uint4*>(rows)[threadIdx.x];
   // FP16 window: tokens [t0 + nq, t0 + n) of the block (all at or beyond Q)
   if (nq < n) {
-    uint16_t* ring = (is_key ? a.k_res : a.v_res) + unit * a.ring * kHeadDim;
     for (int idx = threadIdx.x; idx < (n - nq) * 16; idx += kPThreads) {
       const int i = nq + (idx >> 4), part = idx & 15;
       const int64_t slot = (t0 + i) % a.ring;

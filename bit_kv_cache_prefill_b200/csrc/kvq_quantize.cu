@@ -41,11 +41,12 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
   uint32_t* pmin = reinterpret_cast<uint32_t*>(pbuf + 128 * 8);   // [4][128]
   uint32_t* pmax = pmin + 4 * 128;                                // [4][128]
   const int64_t g = t0 / G;
+  const bool sink0 = a.sink && t0 == 0;  // token 0 stays out of group 0 (min/max and codes)
   {
     const int cp = threadIdx.x & 63, tq = threadIdx.x >> 6;
     const int n = G / 4;
     uint32_t mn0 = 0xffffffffu, mx0 = 0u, mn1 = 0xffffffffu, mx1 = 0u;
-    for (int i = tq * n; i < (tq + 1) * n; ++i) {
+    for (int i = tq * n + ((sink0 && tq == 0) ? 1 : 0); i < (tq + 1) * n; ++i) {
       const uint32_t w = *reinterpret_cast<const uint32_t*>(rows + i * kHeadDim + 2 * cp);
       const uint32_t k0 = order_key(w & 0xffffu), k1 = order_key(w >> 16);
       mn0 = min(mn0, k0);
@@ -69,6 +70,7 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
     a.k_scale[pidx] = p.s16;
     a.k_zero[pidx] = p.z16;
     prm[c] = make_float2(p.zf, p.inv);
+    if (sink0) const_cast<uint16_t*>(rows)[c] = p.z16;  // codes to 0: x - zf = 0
   }
   __syncthreads();
   const int words = 64 * bits;
@@ -134,7 +136,8 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, 1));
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 1));
     if (half == 0) {
-      const QuantParams p = make_params(kmin, kmax, bits);
+      QuantParams p = make_params(kmin, kmax, bits);
+      if (a.sink && t0 + i == 0) p = QuantParams{0.f, 0.f, 0, 0, true};  // the sink token: all zero
       const int64_t pidx = (unit * a.capacity + t0 + i) * vpt + j;
       a.v_scale[pidx] = p.s16;
       a.v_zero[pidx] = p.z16;
@@ -195,7 +198,7 @@ __global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint1
   const int64_t Q_new = quantized_len(t + 1, a.R, G);
   uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
   uint8_t* pbuf = smem + static_cast<size_t>(G) * kHeadDim * 2;
-  uint16_t* ring = (is_key ? a.k_res : a.v_res) + unit * a.ring * kHeadDim;
+  uint16_t* ring = (is_key ? a.k_res : a.v_res) + unit * a.res_rows * kHeadDim;
   const uint16_t* src = (is_key ? k_new : v_new) + unit * kHeadDim;
   // New token -> ring slot t mod (R + G), rotated first for keys when enabled (warp 0, 16 lanes).
   if (threadIdx.x < 32) {
@@ -208,9 +211,11 @@ __global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint1
     uint16_t o[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i] = __half_as_ushort(__float2half_rn(x[i]));
-    if (threadIdx.x < 16)
-      reinterpret_cast<uint4*>(ring + (t % a.ring) * kHeadDim)[threadIdx.x] =
-          (is_key && a.hadamard) ? *reinterpret_cast<const uint4*>(o) : raw;
+    if (threadIdx.x < 16) {
+      const uint4 row = (is_key && a.hadamard) ? *reinterpret_cast<const uint4*>(o) : raw;
+      reinterpret_cast<uint4*>(ring + (t % a.ring) * kHeadDim)[threadIdx.x] = row;
+      if (a.sink && t == 0) reinterpret_cast<uint4*>(ring + a.ring * kHeadDim)[threadIdx.x] = row;  // sink row
+    }
   }
   if (Q_new == Q_old) return;
   __syncthreads();  // the new token is in the ring (it is not part of the flushed group, but keep order simple)

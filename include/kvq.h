@@ -59,7 +59,7 @@ typedef enum {
  *   key_bits, value_bits in {2, 4};
  *   group_size G in {16, 32, 64, 128} (a multiple of the 16-token tile and a divisor of 128);
  *   residual R >= 0 (tokens kept in FP16 beyond the last full group; 0 <= R <= 4096);
- *   hadamard in {0, 1}; layout KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2;
+ *   hadamard in {0, 1}; layout KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2; sink in {0, 1};
  *   capacity >= 0, a multiple of G (maximum tokens per sequence); with layout ROWS_V2 also a
  *   multiple of 128 (value rows come in whole 128-token blocks). */
 typedef struct {
@@ -73,6 +73,7 @@ typedef struct {
   int32_t residual;
   int32_t hadamard;
   int32_t layout;
+  int32_t sink;  /* 1: the first token of every sequence stays in fp16 (see below) */
   int64_t capacity;
 } kvq_config;
 
@@ -87,12 +88,18 @@ typedef struct {
  *   k_zero   fp16 [capacity/G][128]             same; the zero-point is the group minimum
  *   v_scale  fp16 [capacity][128/G]             per token and channel group
  *   v_zero   fp16 [capacity][128/G]             same
- *   k_res    fp16 [R+G][128]                    FP16 ring of the newest keys (rotated if hadamard)
- *   v_res    fp16 [R+G][128]                    FP16 ring of the newest values
+ *   k_res    fp16 [R+G+sink][128]               FP16 ring of the newest keys (rotated if hadamard);
+ *                                               with sink = 1, row R+G holds the first token's key
+ *   v_res    fp16 [R+G+sink][128]               same for values
  * Every buffer must be 16-byte aligned. kvq_cache_buffer_bytes gives the total sizes.
  *
  * Quantized length of a sequence of T tokens: Q = G * floor(max(T - R, 0) / G). Tokens [0, Q) are
  * quantized, tokens [Q, T) live in the ring at slot t mod (R + G).
+ *
+ * Attention sink (sink = 1; the KVQuant review, Method, keeps the first token in fp16): token 0's key
+ * and value are also kept in fp16 in ring row R+G, written by the prefill or by the append that adds
+ * token 0. Key group 0's min/max leave token 0 out, token 0's codes and value scale / zero are 0, and
+ * decode reads token 0 only from its fp16 row.
  *
  * Tile v1: tile row k of a unit holds tokens 16k..16k+15. Within a tile, "lane" L (0..31) owns
  * words (w / 4) * 128 + 4L + (w % 4) for w in [0, 2*bits). Word w holds 16/bits code pairs; pair j

@@ -21,16 +21,16 @@ def capacity(w: inputs.Workload, layout: int) -> int:
     return -(-cap // 128) * 128 if layout == 2 else cap
 
 
-def oracle_config(oracle, w: inputs.Workload, batch=None, hq=None, hkv=None, layout: int = 1):
+def oracle_config(oracle, w: inputs.Workload, batch=None, hq=None, hkv=None, layout: int = 1, sink: int = 0):
     return oracle.Config(batch or w.batch, hq or w.num_q_heads, hkv or w.num_kv_heads, w.key_bits, w.value_bits,
-                         w.group_size, w.residual, w.hadamard, capacity(w, layout), layout=layout)
+                         w.group_size, w.residual, w.hadamard, capacity(w, layout), layout=layout, sink=sink)
 
 
-def gpu_config(w: inputs.Workload, layout: int = 1):
+def gpu_config(w: inputs.Workload, layout: int = 1, sink: int = 0):
     import bit_kv_cache_prefill_b200 as kvq
 
     return kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size,
-                           w.residual, w.hadamard, capacity(w, layout), layout=layout)
+                           w.residual, w.hadamard, capacity(w, layout), layout=layout, sink=sink)
 
 
 @dataclass
@@ -40,14 +40,16 @@ class GpuRun:
     out: torch.Tensor  # fp16 [B][Hq][128] on the device
     lens: np.ndarray
     layout: int = 1
+    sink: int = 0
 
 
 def run_gpu(w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
-            appends: int = 0, sm_scale: Optional[float] = None, layout: int = 1, decode: bool = True) -> GpuRun:
+            appends: int = 0, sm_scale: Optional[float] = None, layout: int = 1, decode: bool = True,
+            sink: int = 0) -> GpuRun:
     """Prefill (k, v on the device), `appends` streaming appends, one decode (unless decode=False)."""
     import bit_kv_cache_prefill_b200 as kvq
 
-    cfg = gpu_config(w, layout)
+    cfg = gpu_config(w, layout, sink)
     cache = kvq.Cache(cfg)
     kvq.kvq_quantize_prefill(cfg, cache, k, v, lens)
     for step in range(appends):
@@ -58,7 +60,7 @@ def run_gpu(w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarr
         ws = torch.empty(kvq.kvq_decode_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
         kvq.kvq_decode_attention(cfg, cache, q.cuda(), out, sm_scale or 1 / math.sqrt(128), ws)
     torch.cuda.synchronize()
-    return GpuRun(cfg, cache, out, lens + appends, layout)
+    return GpuRun(cfg, cache, out, lens + appends, layout, sink)
 
 
 def code_shapes(w: inputs.Workload, layout: int):
@@ -71,7 +73,7 @@ def code_shapes(w: inputs.Workload, layout: int):
 def gpu_views(w: inputs.Workload, run: GpuRun) -> Dict[str, np.ndarray]:
     """GPU cache buffers as numpy arrays with the oracle's shapes."""
     B, H, cap, G = w.batch, w.num_kv_heads, capacity(w, run.layout), w.group_size
-    ring = w.residual + G
+    ring = w.residual + G + run.sink  # ring slots, then the sink row
     c = run.cache
     ks, vs = code_shapes(w, run.layout)
     return {
@@ -87,7 +89,7 @@ def gpu_views(w: inputs.Workload, run: GpuRun) -> Dict[str, np.ndarray]:
 
 
 def compare_unit_cache(w: inputs.Workload, gv: Dict[str, np.ndarray], b: int, h: int, oc, ob: int, oh: int, T: int,
-                       layout: int = 1) -> None:
+                       layout: int = 1, sink: int = 0) -> None:
     """Bit-exact comparison of everything that is defined for one unit of length T."""
     G, R = w.group_size, w.residual
     Q = max(T - R, 0) // G * G
@@ -110,6 +112,9 @@ def compare_unit_cache(w: inputs.Workload, gv: Dict[str, np.ndarray], b: int, h:
     live = [t % ring for t in range(Q, T)]
     np.testing.assert_array_equal(gv["k_res"][b, h, live], oc.k_res[ob, oh, live], err_msg=f"k_res unit {b},{h}")
     np.testing.assert_array_equal(gv["v_res"][b, h, live], oc.v_res[ob, oh, live], err_msg=f"v_res unit {b},{h}")
+    if sink and T > 0:  # the sink token's fp16 row
+        for key in ("k_res", "v_res"):
+            np.testing.assert_array_equal(gv[key][b, h, ring], getattr(oc, key)[ob, oh, ring], err_msg=f"{key} sink row {b},{h}")
 
 
 def check_attention(gpu_out: np.ndarray, ref: np.ndarray, what: str) -> Tuple[float, float]:
@@ -124,8 +129,8 @@ def check_attention(gpu_out: np.ndarray, ref: np.ndarray, what: str) -> Tuple[fl
 
 
 def oracle_full(oracle, w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
-                appends: int = 0, sm_scale: Optional[float] = None, threads: int = 8, layout: int = 1):
-    ocfg = oracle_config(oracle, w, layout=layout)
+                appends: int = 0, sm_scale: Optional[float] = None, threads: int = 8, layout: int = 1, sink: int = 0):
+    ocfg = oracle_config(oracle, w, layout=layout, sink=sink)
     oc = oracle.Cache(ocfg)
     oracle.quantize_prefill(ocfg, oc, k.numpy(), v.numpy(), lens, threads=threads)
     for step in range(appends):
