@@ -28,9 +28,14 @@
 //       accumulation error of a million-token sum would be amplified by that cancellation.
 //   Online softmax keeps a running max per head; accumulators are rescaled only when some head's
 //   max moves.
-// Codes -> fp16: a 2-bit code at bit 2k of a 16-bit half is OR-ed into the mantissa of the fp16
-// constant 2^(10-2k) (so the half reads 2^(10-2k) + code) and the constant is subtracted again: two
-// ALU instructions per pair of codes, exact. 4-bit codes use 2^(10-4k) the same way.
+// Codes -> fp16: a code AND-ed out in place at bit offset o of a 16-bit half is the fp16 subnormal
+// code * 2^(o - 24), exact, one AND per code pair (value codes are taken one bit higher and centered
+// with one exact subnormal subtraction). The m16n8k16 A fragment of one word holds element k at
+// 2^(2k - 24) (2-bit) or 2^(-24), 2^(-20), 2^(-24), 2^(-20) (4-bit). Elements 0 and 1 (2 and 3)
+// share the K columns 2qd, 2qd+1 (2qd+8, 2qd+9) and elements 0, 2 (1, 3) the M row r (r + 8), so
+// the scale factors into a per-K-half factor, put on the B operand (2-bit: 2^-4 on the upper
+// K half), and a per-row factor taken off the fp32 result (row r: 2^24, row r + 8: 2^22 for 2-bit,
+// 2^20 for 4-bit; value rows carry one more factor 1/2 from the doubled centered code).
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
@@ -168,7 +173,7 @@ __device__ __forceinline__ void tile_scores(const uint8_t* kc, int lane, const u
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       uint32_t h[8];
-      unpack_word2(w4[w], h);
+      unpack_word2_sub(w4[w], h);
       mma16816(acc[0], h[0], h[1], h[2], h[3], bq[2 * w][0], bq[2 * w][1]);
       mma16816(acc[1], h[4], h[5], h[6], h[7], bq[2 * w + 1][0], bq[2 * w + 1][1]);
     }
@@ -179,12 +184,14 @@ __device__ __forceinline__ void tile_scores(const uint8_t* kc, int lane, const u
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       uint32_t h[4];
-      unpack_word4(w8[w], h);
+      unpack_word4_sub(w8[w], h);
       mma16816(acc[w & 1], h[0], h[1], h[2], h[3], bq[w][0], bq[w][1]);
     }
   }
-  s_lo = ((acc[0][0] + acc[1][0]) + (acc[0][1] + acc[1][1]) + bias) * p2e;  // hi + lo columns, token r
-  s_hi = ((acc[0][2] + acc[1][2]) + (acc[0][3] + acc[1][3]) + bias) * p2e;  // token r + 8
+  // hi + lo columns; the subnormal row scales come off here
+  constexpr float kRowLo = 16777216.0f, kRowHi = KB == 2 ? 4194304.0f : 1048576.0f;  // 2^24, 2^22 / 2^20
+  s_lo = fmaf((acc[0][0] + acc[1][0]) + (acc[0][1] + acc[1][1]), kRowLo, bias) * p2e;  // token r
+  s_hi = fmaf((acc[0][2] + acc[1][2]) + (acc[0][3] + acc[1][3]), kRowHi, bias) * p2e;  // token r + 8
 }
 
 // N columns of the tensor-core tiles. GQ (1, 2 or 4) query heads share one KV head; the 8 columns of
@@ -375,7 +382,10 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
           const float2 qq = *reinterpret_cast<const float2*>(qn_row + 16 * (idx >> 2) + 8 * ((idx >> 1) & 1));
           const float s0 = h2f(static_cast<uint16_t>(sw[k] & 0xffffu)), s1 = h2f(static_cast<uint16_t>(sw[k] >> 16));
           const float z0 = h2f(static_cast<uint16_t>(zw[k] & 0xffffu)), z1 = h2f(static_cast<uint16_t>(zw[k] >> 16));
-          bq[idx >> 2][(idx >> 1) & 1] = pack_h2(split_part(qq.x * s0, lo_half), split_part(qq.y * s1, lo_half));
+          // 2-bit: the upper K half (channels 16m + 8 ..) carries 2^-4 against the subnormal codes
+          const float kf = (KB == 2 && (k & 1)) ? 0.0625f : 1.f;
+          bq[idx >> 2][(idx >> 1) & 1] =
+              pack_h2(split_part(qq.x * s0 * kf, lo_half), split_part(qq.y * s1 * kf, lo_half));
           bias = fmaf(qq.x, z0, bias);
           bias = fmaf(qq.y, z1, bias);
         }
@@ -440,6 +450,9 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
     for (int u = 0; u < TS; ++u) {
       const float pa = __shfl_sync(kFull, p[u][0], la), pb = __shfl_sync(kFull, p[u][0], la + 4);
       const float pc = __shfl_sync(kFull, p[u][1], la), pd = __shfl_sync(kFull, p[u][1], la + 4);
+      // 2-bit: tokens 2qd + 8, + 9 (the upper K half) carry 2^-4 against the subnormal codes
+      constexpr float kTf = VB == 2 ? 0.0625f : 1.f;
+      const float pcs = pc * kTf, pds = pd * kTf;
       const uint16_t* vsh = reinterpret_cast<const uint16_t*>(st + S::oVS) + u * 16 * VPT;
       const uint16_t* vzh = reinterpret_cast<const uint16_t*>(st + S::oVZ) + u * 16 * VPT;
       uint32_t bp[NBV][2];
@@ -451,7 +464,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
           const float s0 = h2f(vsh[t0]), s1 = h2f(vsh[t0 + VPT]), s2 = h2f(vsh[t0 + 8 * VPT]), s3 = h2f(vsh[t0 + 9 * VPT]);
           const float z0 = h2f(vzh[t0]), z1 = h2f(vzh[t0 + VPT]), z2 = h2f(vzh[t0 + 8 * VPT]), z3 = h2f(vzh[t0 + 9 * VPT]);
           bp[nb][0] = pack_h2(split_part(pa * s0, lo_half), split_part(pb * s1, lo_half));
-          bp[nb][1] = pack_h2(split_part(pc * s2, lo_half), split_part(pd * s3, lo_half));
+          bp[nb][1] = pack_h2(split_part(pcs * s2, lo_half), split_part(pds * s3, lo_half));
           float z = zacc[nb];
           z = fmaf(pa, fmaf(kCbar, s0, z0), z);
           z = fmaf(pb, fmaf(kCbar, s1, z1), z);
@@ -470,7 +483,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
           uint32_t h[8];
-          unpack_word2_centered(w4[w], h);
+          unpack_word2_centered_sub(w4[w], h);
           const int nb0 = (2 * w * VPT / 8) / VGB;
           const int nb1 = ((2 * w + 1) * VPT / 8) / VGB;
           mma16816(O[2 * w], h[0], h[1], h[2], h[3], bp[nb0][0], bp[nb0][1]);
@@ -483,7 +496,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
           uint32_t h[4];
-          unpack_word4_centered(w8[w], h);
+          unpack_word4_centered_sub(w8[w], h);
           const int nb = (w * VPT / 8) / VGB;
           mma16816(O[w], h[0], h[1], h[2], h[3], bp[nb][0], bp[nb][1]);
         }
@@ -510,8 +523,10 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
     for (int m = 0; m < 8; ++m) {
       const int jm = (16 * m) / G;
       if (qd / GQ == jm % VGB) {  // this lane owns the columns of m-block m's value group
-        o[16 * m + r] = O[m][0] + O[m][1];
-        o[16 * m + r + 8] = O[m][2] + O[m][3];
+        // row scales of the subnormal centered codes (2 (c - cbar) 2^-24 on row r)
+        constexpr float kORowLo = 8388608.0f, kORowHi = VB == 2 ? 2097152.0f : 524288.0f;  // 2^23, 2^21 / 2^19
+        o[16 * m + r] = (O[m][0] + O[m][1]) * kORowLo;
+        o[16 * m + r + 8] = (O[m][2] + O[m][3]) * kORowHi;
       }
     }
     if (r == 0 && qd < GQ) {

@@ -60,6 +60,57 @@ __device__ __forceinline__ void unpack_word4_centered(uint32_t x, uint32_t (&h)[
   h[3] = hsub2((y & 0x00F000F0u) | 0x54005400u, 0x54785478u);
 }
 
+// Subnormal unpacking (the mma.sync decode). A code AND-ed out in place at bit offset o of a 16-bit half
+// reads, as an fp16 with a zero exponent field, as the subnormal code * 2^(o - 24): exact, one AND with
+// an immediate per code pair, and no constant to OR in or subtract. Each position's power of two is
+// taken out again around the tensor-core product (on the other operand and on the result rows).
+//
+// 2-bit: pairs 0..3 of the word from bits 0, 2, 4, 6 and pairs 4..7 from bits 8 .. 14 shifted down to
+// the same offsets, so element k of each group of four carries 2^(2k - 24).
+__device__ __forceinline__ void unpack_word2_sub(uint32_t x, uint32_t (&h)[8]) {
+  const uint32_t y = x >> 8;
+  h[0] = x & 0x00030003u;
+  h[1] = x & 0x000C000Cu;
+  h[2] = x & 0x00300030u;
+  h[3] = x & 0x00C000C0u;
+  h[4] = y & 0x00030003u;
+  h[5] = y & 0x000C000Cu;
+  h[6] = y & 0x00300030u;
+  h[7] = y & 0x00C000C0u;
+}
+
+// 4-bit: elements 0, 2 carry 2^-24 and elements 1, 3 carry 2^-20.
+__device__ __forceinline__ void unpack_word4_sub(uint32_t x, uint32_t (&h)[4]) {
+  const uint32_t y = x >> 8;
+  h[0] = x & 0x000F000Fu;
+  h[1] = x & 0x00F000F0u;
+  h[2] = y & 0x000F000Fu;
+  h[3] = y & 0x00F000F0u;
+}
+
+// Centered value codes as subnormals: the code is taken one bit higher (2c), and the odd integer
+// 2c - (2^b - 1) = 2 (c - cbar) stays exact after one subnormal subtraction (fixed-point, no rounding).
+// Scales per element as in unpack_word2_sub / unpack_word4_sub.
+__device__ __forceinline__ void unpack_word2_centered_sub(uint32_t x, uint32_t (&h)[8]) {
+  const uint32_t z = x << 1, y = x >> 7;
+  h[0] = hsub2(z & 0x00060006u, 0x00030003u);  // (2c - 3) 2^-24
+  h[1] = hsub2(z & 0x00180018u, 0x000C000Cu);  // (2c - 3) 2^-22
+  h[2] = hsub2(z & 0x00600060u, 0x00300030u);  // (2c - 3) 2^-20
+  h[3] = hsub2(z & 0x01800180u, 0x00C000C0u);  // (2c - 3) 2^-18
+  h[4] = hsub2(y & 0x00060006u, 0x00030003u);
+  h[5] = hsub2(y & 0x00180018u, 0x000C000Cu);
+  h[6] = hsub2(y & 0x00600060u, 0x00300030u);
+  h[7] = hsub2(y & 0x01800180u, 0x00C000C0u);
+}
+
+__device__ __forceinline__ void unpack_word4_centered_sub(uint32_t x, uint32_t (&h)[4]) {
+  const uint32_t z = x << 1, y = x >> 7;
+  h[0] = hsub2(z & 0x001E001Eu, 0x000F000Fu);  // (2c - 15) 2^-24
+  h[1] = hsub2(z & 0x01E001E0u, 0x00F000F0u);  // (2c - 15) 2^-20
+  h[2] = hsub2(y & 0x001E001Eu, 0x000F000Fu);
+  h[3] = hsub2(y & 0x01E001E0u, 0x00F000F0u);
+}
+
 // hi keeps the leading 11 significant bits of x (exact in fp16 when x is in fp16's normal range),
 // lo = x - hi exactly; each fp16 column gets one of them.
 __device__ __forceinline__ float split_part(float x, bool lo) {
