@@ -115,20 +115,26 @@ __device__ void rotate_block(uint16_t* rows, int nrows) {
 }
 
 // ---- keys ---------------------------------------------------------------------------------------------
-// Shared memory after the rows: per (group, quarter, channel pair) min / max keys [8][4][64] u32 x 2,
-// then per (group, channel) zf and inv [8][128] f32 x 2 and clamp flags [8][128] u8.
-constexpr int kKeyScratch = 2 * 8 * 4 * 64 * 4 + 2 * 8 * 128 * 4 + 8 * 128;
+// Shared memory after the rows: per (group, quarter, channel pair) min / max keys [NGM][4][64] u32 x 2,
+// then per (group, channel) zf and inv [NGM][128] f32 x 2 and clamp flags [NGM][128] u8, with
+// NGM = 128 / G groups per block.
+template <int G>
+constexpr int key_scratch_bytes() {
+  constexpr int NGM = kPB / G;  // groups per block
+  return 2 * NGM * 4 * 64 * 4 + 2 * NGM * 128 * 4 + NGM * 128;
+}
 
-template <int BITS, int LAYOUT>
+template <int BITS, int LAYOUT, int G>
 __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int nq, const uint16_t* rows, uint8_t* scratch) {
   constexpr int top = (1 << BITS) - 1;
   constexpr int P = 16 / BITS;  // code pairs per word
-  const int G = a.G, NG = nq / G;
-  uint32_t* pmn = reinterpret_cast<uint32_t*>(scratch);  // [8][4][64]
-  uint32_t* pmx = pmn + 8 * 4 * 64;
-  float* pz = reinterpret_cast<float*>(pmx + 8 * 4 * 64);  // [8][128]
-  float* pinv = pz + 8 * 128;
-  uint8_t* pcl = reinterpret_cast<uint8_t*>(pinv + 8 * 128);  // [8][128]
+  const int NG = nq / G;
+  constexpr int NGM = kPB / G;
+  uint32_t* pmn = reinterpret_cast<uint32_t*>(scratch);  // [NGM][4][64]
+  uint32_t* pmx = pmn + NGM * 4 * 64;
+  float* pz = reinterpret_cast<float*>(pmx + NGM * 4 * 64);  // [NGM][128]
+  float* pinv = pz + NGM * 128;
+  uint8_t* pcl = reinterpret_cast<uint8_t*>(pinv + NGM * 128);  // [NGM][128]
   const int tid = threadIdx.x;
 
   // With the sink on, the block at t0 = 0 keeps token 0 out of group 0 (its min/max and its codes).
@@ -283,18 +289,22 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
 }
 
 // ---- values -------------------------------------------------------------------------------------------
-// Shared memory after the rows: per (token, group) zf and inv as float2 [128][8], clamp flags [128][8]
-// u8, and (rows v2) the packed output words [128][4 * BITS] u32.
-constexpr int kValScratch = 128 * 8 * 8 + 128 * 8 + 128 * 16 * 4;
+// Shared memory after the rows: per (token, group) zf and inv as float2 [128][VPT], clamp flags
+// [128][VPT] u8, and (rows v2) the packed output words [128][4 * BITS] u32.
+template <int G, int LAYOUT, int BITS>
+constexpr int val_scratch_bytes() {
+  constexpr int VPT = kHeadDim / G;
+  return kPB * VPT * 8 + kPB * VPT + (LAYOUT == KVQ_LAYOUT_ROWS_V2 ? kHeadDim * 4 * BITS * 4 : 0);
+}
 
-template <int BITS, int LAYOUT>
+template <int BITS, int LAYOUT, int G>
 __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int nq, const uint16_t* rows, uint8_t* scratch) {
   constexpr int top = (1 << BITS) - 1;
   constexpr int P = 16 / BITS;
-  const int G = a.G, VPT = kHeadDim / G;
-  float2* prm = reinterpret_cast<float2*>(scratch);              // [128][8]
-  uint8_t* pcl = scratch + 128 * 8 * 8;                          // [128][8]
-  uint32_t* outw = reinterpret_cast<uint32_t*>(pcl + 128 * 8);   // [128][4 * BITS] (rows v2)
+  constexpr int VPT = kHeadDim / G;
+  float2* prm = reinterpret_cast<float2*>(scratch);               // [128][VPT]
+  uint8_t* pcl = scratch + kPB * VPT * 8;                         // [128][VPT]
+  uint32_t* outw = reinterpret_cast<uint32_t*>(pcl + kPB * VPT);  // [128][4 * BITS] (rows v2)
   const int tid = threadIdx.x;
 
   // parameters per (token, group): item (t, j) scans G channels of row t
@@ -315,8 +325,8 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     const int64_t pidx = (unit * a.capacity + t0 + t) * VPT + j;
     a.v_scale[pidx] = p.s16;
     a.v_zero[pidx] = p.z16;
-    prm[t * 8 + j] = make_float2(p.zf, p.inv);
-    pcl[t * 8 + j] = !sink_tok && needs_clamp(p, kmax, top) ? 1 : 0;
+    prm[t * VPT + j] = make_float2(p.zf, p.inv);
+    pcl[t * VPT + j] = !sink_tok && needs_clamp(p, kmax, top) ? 1 : 0;
   }
   __syncthreads();
 
@@ -336,9 +346,9 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
         for (int e = 0; e < 2; ++e) {
           const int t = 2 * (P * wv + k) + e;
           const uint2 x = *reinterpret_cast<const uint2*>(rows + t * kRS + c);
-          const float2 pp = prm[t * 8 + j];
+          const float2 pp = prm[t * VPT + j];
           const int sh = BITS * k + 16 * e;
-          if (!pcl[t * 8 + j]) {
+          if (!pcl[t * VPT + j]) {
             const uint64_t z2 = pk2(pp.x, pp.x), i2 = pk2(pp.y, pp.y);
             const uint64_t r0 = codes2(x.x, z2, i2), r1 = codes2(x.y, z2, i2);
             wd[0] += static_cast<uint32_t>(r0) << sh;
@@ -396,9 +406,9 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
         const int t = tb + 8 * ((j >> 1) & 1);
         const uint32_t xa = *reinterpret_cast<const uint32_t*>(rows + t * kRS + ch);        // token t, channels ch, ch + 1
         const uint32_t xb = *reinterpret_cast<const uint32_t*>(rows + (t + 1) * kRS + ch);  // token t + 1
-        const float2 pa = prm[t * 8 + gj], pb = prm[(t + 1) * 8 + gj];
+        const float2 pa = prm[t * VPT + gj], pb = prm[(t + 1) * VPT + gj];
         uint32_t ra0, ra1, rb0, rb1;
-        if (!(pcl[t * 8 + gj] | pcl[(t + 1) * 8 + gj])) {
+        if (!(pcl[t * VPT + gj] | pcl[(t + 1) * VPT + gj])) {
           const uint64_t ra = codes2(xa, pk2(pa.x, pa.x), pk2(pa.y, pa.y));
           const uint64_t rb = codes2(xb, pk2(pb.x, pb.x), pk2(pb.y, pb.y));
           ra0 = static_cast<uint32_t>(ra);
@@ -420,16 +430,19 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
   }
 }
 
-template <int BITS_K, int BITS_V, int LAYOUT>
+// G (16, 32, 64 or 128) is a template parameter so that every division by it is a shift.
+template <int BITS_K, int BITS_V, int LAYOUT, int G>
 __global__ void __launch_bounds__(kPThreads) prefill_block_kernel(QuantizeArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
   uint8_t* scratch = smem + kPB * kRS * 2;
-  const int64_t unit = blockIdx.y;
+  const int unit32 = static_cast<int>(blockIdx.y);
+  const int64_t unit = unit32;
   const bool is_key = blockIdx.z == 0;
-  const int64_t b = unit / a.num_kv_heads, h = unit % a.num_kv_heads;
+  const int b32 = unit32 / a.num_kv_heads;
+  const int64_t b = b32, h = unit32 - b32 * a.num_kv_heads;
   const int64_t T = a.seq_len[b];
-  const int64_t Q = quantized_len(T, a.R, a.G);
+  const int64_t Q = quantized_len(T, a.R, G);
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kPB;
   if (t0 >= T) return;
   const int n = static_cast<int>(min(static_cast<int64_t>(kPB), T - t0));
@@ -454,35 +467,53 @@ __global__ void __launch_bounds__(kPThreads) prefill_block_kernel(QuantizeArgs a
   if (nq < n) {
     for (int idx = threadIdx.x; idx < (n - nq) * 16; idx += kPThreads) {
       const int i = nq + (idx >> 4), part = idx & 15;
-      const int64_t slot = (t0 + i) % a.ring;
+      const int64_t slot = static_cast<int>(t0 + i) % static_cast<int>(a.ring);  // 32-bit: capacity < 2^31
       reinterpret_cast<uint4*>(ring + slot * kHeadDim)[part] = reinterpret_cast<const uint4*>(rows + i * kRS)[part];
     }
   }
   if (nq == 0) return;
   if (is_key)
-    key_block<BITS_K, LAYOUT>(a, unit, t0, nq, rows, scratch);
+    key_block<BITS_K, LAYOUT, G>(a, unit, t0, nq, rows, scratch);
   else
-    value_block<BITS_V, LAYOUT>(a, unit, t0, nq, rows, scratch);
+    value_block<BITS_V, LAYOUT, G>(a, unit, t0, nq, rows, scratch);
 }
 
-constexpr int kPrefillSmem = kPB * kRS * 2 + (kKeyScratch > kValScratch ? kKeyScratch : kValScratch);
+// Shared memory of one CTA: the rows, then the larger of the key and value scratch. With G >= 32 it
+// fits four CTAs per SM.
+template <int BK, int BV, int LAYOUT, int G>
+constexpr int prefill_smem_bytes() {
+  constexpr int ks = key_scratch_bytes<G>(), vs = val_scratch_bytes<G, LAYOUT, BV>();
+  return kPB * kRS * 2 + (ks > vs ? ks : vs);
+}
 
-template <int BK, int BV, int LAYOUT>
+template <int BK, int BV, int LAYOUT, int G>
 cudaError_t launch_block(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
   static DeviceMemo attr;
   const int ok = attr.get([] {
-    return cudaFuncSetAttribute(prefill_block_kernel<BK, BV, LAYOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem) == cudaSuccess ? 1 : -1;
+    return cudaFuncSetAttribute(prefill_block_kernel<BK, BV, LAYOUT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                prefill_smem_bytes<BK, BV, LAYOUT, G>()) == cudaSuccess ? 1 : -1;
   });
   if (ok < 0) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>((max_len + kPB - 1) / kPB), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads), 2);
-  prefill_block_kernel<BK, BV, LAYOUT><<<grid, kPThreads, kPrefillSmem, stream>>>(a);
+  prefill_block_kernel<BK, BV, LAYOUT, G><<<grid, kPThreads, prefill_smem_bytes<BK, BV, LAYOUT, G>(), stream>>>(a);
   return cudaGetLastError();
+}
+
+template <int BK, int BV, int LAYOUT>
+cudaError_t launch_group(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
+  switch (a.G) {
+    case 16: return launch_block<BK, BV, LAYOUT, 16>(a, max_len, stream);
+    case 32: return launch_block<BK, BV, LAYOUT, 32>(a, max_len, stream);
+    case 64: return launch_block<BK, BV, LAYOUT, 64>(a, max_len, stream);
+    case 128: return launch_block<BK, BV, LAYOUT, 128>(a, max_len, stream);
+  }
+  return cudaErrorInvalidValue;
 }
 
 template <int LAYOUT>
 cudaError_t launch_bits(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
-  if (a.key_bits == 2) return a.value_bits == 2 ? launch_block<2, 2, LAYOUT>(a, max_len, stream) : launch_block<2, 4, LAYOUT>(a, max_len, stream);
-  return a.value_bits == 2 ? launch_block<4, 2, LAYOUT>(a, max_len, stream) : launch_block<4, 4, LAYOUT>(a, max_len, stream);
+  if (a.key_bits == 2) return a.value_bits == 2 ? launch_group<2, 2, LAYOUT>(a, max_len, stream) : launch_group<2, 4, LAYOUT>(a, max_len, stream);
+  return a.value_bits == 2 ? launch_group<4, 2, LAYOUT>(a, max_len, stream) : launch_group<4, 4, LAYOUT>(a, max_len, stream);
 }
 
 }  // namespace
