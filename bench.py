@@ -147,10 +147,11 @@ def reduce_over_ranks(dist, device, ms: float, *sums: float):
     return out
 
 
-def measured_traffic(w: inputs.Workload, layout: int):
-    """DRAM bytes per decode-split launch from the committed ncu counters (profiles/decode_traffic_counters.txt, JSON), scaled
-    from the captured batch to this one by the units processed; None if there is no capture for this
-    workload and layout or the kernel sources changed since it was taken."""
+def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode"):
+    """DRAM bytes per launch of the decode-split (kind "decode") or bulk-prefill (kind "prefill")
+    kernel from the committed ncu counters (profiles/decode_traffic_counters.txt, JSON), scaled from
+    the captured batch to this one by the units processed; None if there is no capture for this
+    workload, layout and kernel or the kernel sources changed since it was taken."""
     import hashlib
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "decode_traffic_counters.txt")
     try:
@@ -159,7 +160,7 @@ def measured_traffic(w: inputs.Workload, layout: int):
         return None
     root = os.path.dirname(os.path.abspath(__file__))
     for e in entries.values():
-        if e.get("workload") != w.name or e.get("layout") != layout:
+        if e.get("workload") != w.name or e.get("layout") != layout or e.get("kind", "decode") != kind:
             continue
         h = hashlib.sha256()
         for f in e["kernel_sources"]:
@@ -460,7 +461,10 @@ def main():
                      "kernel": ("decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
                      + " + decode_combine_kernel (one kvq_decode_attention call)"},
         "prefill": {"gbs": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9, 1),
-                    "ms": round(statistics.mean(pre_ms), 3), "bytes": pre_bytes},
+                    "ms": round(statistics.mean(pre_ms), 3), "bytes": pre_bytes, "bound": "hbm", "peak": peak,
+                    "frac": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9 / peak, 4),
+                    "traffic": measured_traffic(w0, args.layout, "prefill"),
+                    "kernel": "prefill_block_kernel (one kvq_quantize_prefill call)"},
         "gpu_launches": 4 * args.steps,
         "clocks": clocks.summary(),
     }

@@ -232,7 +232,9 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
     // (+1), with (m, hh, u) from the pair slot p = P w + j. Thread (w % 4, L, half) keeps the parameters
     // of the word's channels for the tiles of one group.
     constexpr int NCP = P / 2;  // channel pairs per word (each at two token rows)
-    const int wl = tid & 3, L = (tid >> 2) & 31, hi = tid >> 7;
+    // A warp holds the 32 lanes L of one word: its row reads (token r or r + 8, channels 2qd + ..)
+    // then fall in 32 distinct shared-memory banks.
+    const int L = tid & 31, wl = (tid >> 5) & 3, hi = tid >> 7;
     const int w = BITS == 2 ? wl : 4 * hi + wl;
     const int tl0 = BITS == 2 ? 4 * hi : 0, ntl = BITS == 2 ? 4 : 8;
     const int r = L >> 2, qd = L & 3;
@@ -383,25 +385,30 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     }
   } else {
     // Tile v1: word w of lane L = 4r + qd in tile tl; pair j -> tokens 2qd + 8hh (+1), channel
-    // 16m + r + 8u, with (m, hh, u) from p = P w + j (so hh and u depend on j only). Thread (w, lane
-    // pair, tile part) builds the words of lanes L0 = 4 r0 + qd and L1 = L0 + 4 (r0 even): they hold the
+    // 16m + r + 8u, with (m, hh, u) from p = P w + j (so hh and u depend on j only). Thread (lane pair,
+    // half, w, part) builds the words of lanes L0 = 4 r0 + qd and L1 = L0 + 4 (r0 even): they hold the
     // same tokens and the adjacent channels r0, r0 + 1, so one 4-byte load feeds both, and a token's two
-    // channels share packed fp32x2 arithmetic.
+    // channels share packed fp32x2 arithmetic. A warp is one w: its 16 lane pairs read banks
+    // 8 qd + r0 / 2 (+ const), and the two half-warps (tiles of either parity) visit the pair slots in the
+    // orders j and j ^ 1, i.e. channel offsets 8 apart, 4 banks further: 32 distinct banks.
     constexpr int NW = 2 * BITS;                    // words per lane per tile
-    constexpr int TPARTS = kPThreads / (NW * 16);   // 4 (2-bit) or 2 (4-bit)
-    constexpr int TPT = 8 / TPARTS;                 // tiles per thread
-    const int w = tid % NW, lp = (tid / NW) % 16, part = tid / (NW * 16);
+    constexpr int NPART = kPThreads / (32 * NW);    // 2 (2-bit) or 1 (4-bit)
+    constexpr int TPT = 8 / (2 * NPART);            // tiles per thread
+    const int lp = tid & 15, half = (tid >> 4) & 1, w = (tid >> 5) % NW, part = (tid >> 5) / NW;
     const int qd = lp & 3, r0 = 2 * (lp >> 2);
     const int L0 = 4 * r0 + qd;
     const int words = 64 * BITS;
     const int widx0 = (w >> 2) * 128 + 4 * L0 + (w & 3);  // lane L1 = L0 + 4: widx0 + 16
     const int ch0 = 16 * ((P * w) >> 2) + r0;              // channel of pair j: ch0 + 16 (j >> 2) + 8 (j & 1)
     uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words + widx0;
-    for (int tl = part * TPT; tl < (part + 1) * TPT && tl * kTile < nq; ++tl) {
+    for (int k = 0; k < TPT; ++k) {
+      const int tl = 2 * (part + NPART * k) + half;
+      if (tl * kTile >= nq) break;
       const int tb = tl * kTile + 2 * qd;  // token of pair j: tb + 8 ((j >> 1) & 1) (+1)
       uint32_t acc0 = word_bias<BITS>(), acc1 = word_bias<BITS>();
 #pragma unroll
-      for (int j = 0; j < P; ++j) {
+      for (int jo = 0; jo < P; ++jo) {
+        const int j = jo ^ half;  // this half-warp's slot order
         const int ch = ch0 + 16 * (j >> 2) + 8 * (j & 1), gj = ch / G;
         const int t = tb + 8 * ((j >> 1) & 1);
         const uint32_t xa = *reinterpret_cast<const uint32_t*>(rows + t * kRS + ch);        // token t, channels ch, ch + 1
