@@ -32,20 +32,21 @@ constexpr int kRS = 136;      // staged row stride in halves (272 bytes)
 constexpr int kPThreads = 256;
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
 
-__device__ __forceinline__ uint32_t order_key2(uint32_t x) {
-  const uint32_t s = (x >> 15) & 0x00010001u;  // each half's sign bit at its bit 0
-  return x ^ ((s * 0xFFFFu) | 0x80008000u);      // negative half: flip all 16 bits; else flip the sign bit
-}
-__device__ __forceinline__ uint32_t vmin2(uint32_t a, uint32_t b) {
+// fp16x2 min / max (native). For non-NaN inputs they select exactly; only which zero they return for
+// {-0, +0} is left open, so a group whose min or max is a zero is redone with the total-order keys.
+__device__ __forceinline__ uint32_t hmin2u(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("min.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
-__device__ __forceinline__ uint32_t vmax2(uint32_t a, uint32_t b) {
+__device__ __forceinline__ uint32_t hmax2u(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
+constexpr uint32_t kPosInf2 = 0x7C007C00u, kNegInf2 = 0xFC00FC00u;
+__device__ __forceinline__ bool is_zero_h(uint32_t h) { return (h & 0x7fffu) == 0; }
+
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
@@ -57,7 +58,8 @@ __device__ __forceinline__ uint64_t pk2(float a, float b) {
 // (a single rounding of the exact product), which moves values that round to a tie (v = k + 0.5 in
 // fp32) to the wrong code.
 __device__ __forceinline__ uint64_t codes2(uint32_t x, uint64_t zf2, uint64_t inv2) {
-  const uint64_t f = pk2(h2f(static_cast<uint16_t>(x & 0xffffu)), h2f(static_cast<uint16_t>(x >> 16)));
+  const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(&x));
+  const uint64_t f = pk2(xf.x, xf.y);
   uint64_t d, v;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f), "l"(zf2));
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(v) : "l"(d), "l"(inv2));
@@ -143,12 +145,12 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
   {
     const int cp = tid & 63, q = tid >> 6, ql = G / 4;
     for (int g = 0; g < NG; ++g) {
-      uint32_t mn = 0xffffffffu, mx = 0u;
+      uint32_t mn = kPosInf2, mx = kNegInf2;
       const uint16_t* src = rows + (g * G + q * ql) * kRS + 2 * cp;
       for (int i = (sink0 && g == 0 && q == 0) ? 1 : 0; i < ql; ++i) {
-        const uint32_t k = order_key2(*reinterpret_cast<const uint32_t*>(src + i * kRS));
-        mn = vmin2(mn, k);
-        mx = vmax2(mx, k);
+        const uint32_t x = *reinterpret_cast<const uint32_t*>(src + i * kRS);
+        mn = hmin2u(mn, x);
+        mx = hmax2u(mx, x);
       }
       pmn[(g * 4 + q) * 64 + cp] = mn;
       pmx[(g * 4 + q) * 64 + cp] = mx;
@@ -159,11 +161,22 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
   {
     const int c = tid & 127, sh = 16 * (c & 1);
     for (int g = tid >> 7; g < NG; g += 2) {
-      uint32_t kmin = 0xffffu, kmax = 0u;
+      uint32_t mn2 = kPosInf2, mx2 = kNegInf2;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        kmin = min(kmin, (pmn[(g * 4 + q) * 64 + (c >> 1)] >> sh) & 0xffffu);
-        kmax = max(kmax, (pmx[(g * 4 + q) * 64 + (c >> 1)] >> sh) & 0xffffu);
+        mn2 = hmin2u(mn2, pmn[(g * 4 + q) * 64 + (c >> 1)]);
+        mx2 = hmax2u(mx2, pmx[(g * 4 + q) * 64 + (c >> 1)]);
+      }
+      const uint32_t hmn = (mn2 >> sh) & 0xffffu, hmx = (mx2 >> sh) & 0xffffu;
+      uint32_t kmin = order_key(hmn), kmax = order_key(hmx);
+      if (is_zero_h(hmn) || is_zero_h(hmx)) {  // a signed zero: redo with the total order (-0 < +0)
+        kmin = 0xffffu;
+        kmax = 0u;
+        for (int t = g * G + ((sink0 && g == 0) ? 1 : 0); t < (g + 1) * G; ++t) {
+          const uint32_t k = order_key(rows[t * kRS + c]);
+          kmin = min(kmin, k);
+          kmax = max(kmax, k);
+        }
       }
       const QuantParams p = make_params(kmin, kmax, BITS);
       const int pos = LAYOUT == KVQ_LAYOUT_ROWS_V2 ? c : key_param_pos(c);
@@ -313,14 +326,23 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
   for (int idx = tid; idx < nq * VPT; idx += kPThreads) {
     const int t = idx / VPT, j = idx % VPT;
     const uint16_t* src = rows + t * kRS + j * G;
-    uint32_t mn = 0xffffffffu, mx = 0u;
+    uint32_t mn = kPosInf2, mx = kNegInf2;
     for (int c8 = 0; c8 < G; c8 += 8) {
       const uint4 q4 = *reinterpret_cast<const uint4*>(src + c8);
-      const uint32_t k0 = order_key2(q4.x), k1 = order_key2(q4.y), k2 = order_key2(q4.z), k3 = order_key2(q4.w);
-      mn = vmin2(mn, vmin2(vmin2(k0, k1), vmin2(k2, k3)));
-      mx = vmax2(mx, vmax2(vmax2(k0, k1), vmax2(k2, k3)));
+      mn = hmin2u(mn, hmin2u(hmin2u(q4.x, q4.y), hmin2u(q4.z, q4.w)));
+      mx = hmax2u(mx, hmax2u(hmax2u(q4.x, q4.y), hmax2u(q4.z, q4.w)));
     }
-    const uint32_t kmin = min(mn & 0xffffu, mn >> 16), kmax = max(mx & 0xffffu, mx >> 16);
+    const uint32_t hmn = hmin2u(mn, mn >> 16) & 0xffffu, hmx = hmax2u(mx, mx >> 16) & 0xffffu;
+    uint32_t kmin = order_key(hmn), kmax = order_key(hmx);
+    if (is_zero_h(hmn) || is_zero_h(hmx)) {  // a signed zero: redo with the total order (-0 < +0)
+      kmin = 0xffffu;
+      kmax = 0u;
+      for (int c = 0; c < G; ++c) {
+        const uint32_t k = order_key(src[c]);
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+      }
+    }
     QuantParams p = make_params(kmin, kmax, BITS);
     const bool sink_tok = a.sink && t0 + t == 0;  // the sink token: scale, zero and codes 0
     if (sink_tok) p = QuantParams{0.f, 0.f, 0, 0, true};

@@ -186,3 +186,59 @@ def test_full_size_workload_sampled(oracle_mod, name, layout):
     # every output is finite and the lengths advanced by the appends
     assert np.isfinite(out.astype(np.float32)).all()
     assert np.array_equal(run.cache.seq_len_host, lens + w.appends)
+
+
+def _signed_zero_kv(w, T, seed):
+    """K/V of one sequence where many groups have a signed zero as min or max (random zero signs)."""
+    rng = np.random.default_rng(seed)
+    H = w.num_kv_heads
+
+    def zeros(shape):
+        return rng.choice(np.array([0x0000, 0x8000], np.uint16), size=shape)
+
+    base = rng.standard_normal((T, H, 128)).astype(np.float16)
+    k = base.view(np.uint16).copy()
+    pos = np.abs(base).view(np.uint16)              # non-negative values
+    neg = (-np.abs(base)).view(np.uint16)           # non-positive values
+    zmask = rng.random((T, H, 128)) < 0.3
+    # keys (per channel over tokens): a zero mix; zeros + positives (min a zero); zeros + negatives
+    # (max a zero); only -0; only +0
+    k[:, :, 0:16] = zeros((T, H, 16))
+    k[:, :, 16:32] = np.where(zmask[:, :, 16:32], zeros((T, H, 16)), pos[:, :, 16:32])
+    k[:, :, 32:48] = np.where(zmask[:, :, 32:48], zeros((T, H, 16)), neg[:, :, 32:48])
+    k[:, :, 48:56] = 0x8000
+    k[:, :, 56:64] = 0x0000
+    # values (per token over channels): whole rows of zeros, zeros + positives, zeros + negatives
+    v = rng.standard_normal((T, H, 128)).astype(np.float16).view(np.uint16).copy()
+    vpos = np.abs(v.view(np.float16)).view(np.uint16)
+    vneg = (-np.abs(v.view(np.float16))).view(np.uint16)
+    sel = np.arange(T) % 4
+    v[sel == 0] = zeros(((sel == 0).sum(), H, 128))
+    v[sel == 1] = np.where(rng.random(((sel == 1).sum(), H, 128)) < 0.3, zeros(((sel == 1).sum(), H, 128)), vpos[sel == 1])
+    v[sel == 2] = np.where(rng.random(((sel == 2).sum(), H, 128)) < 0.3, zeros(((sel == 2).sum(), H, 128)), vneg[sel == 2])
+    kt = torch.from_numpy(k.view(np.float16)).unsqueeze(0).contiguous()
+    vt = torch.from_numpy(v.view(np.float16)).unsqueeze(0).contiguous()
+    return kt, vt
+
+
+@pytest.mark.parametrize("layout", LAYOUTS, ids=["tile_v1", "rows_v2"])
+@pytest.mark.parametrize("G", [16, 32, 128])
+def test_signed_zero_groups_bit_exact(oracle_mod, layout, G):
+    """Groups whose min or max is -0 or +0 (the total order puts -0 below +0) match the oracle bit for
+    bit, on every layout and with G = 16, 32 and 128."""
+    T = 300
+    w = W("z", 1, 4, 2, 2, 2, G, 8, 0, T, seed=51).scaled(seq_len=T)
+    lens = np.array([T], np.int64)
+    k, v = _signed_zero_kv(w, T, seed=G)
+    q = inputs.query(w)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, layout=layout)
+    oc, ref = H.oracle_full(oracle_mod, w, k, v, lens, q, layout=layout)
+    gv = H.gpu_views(w, run)
+    for h in range(w.num_kv_heads):
+        H.compare_unit_cache(w, gv, 0, h, oc, 0, h, T, layout=layout)
+    # rows v2 keeps key parameters in channel order: the all -0 channels have zero-point -0, the
+    # all +0 ones +0
+    if layout == 2:
+        kz = gv["k_zero"][0, :, : (T - w.residual) // G]
+        assert np.all(kz[:, :, 48:56] == 0x8000) and np.all(kz[:, :, 56:64] == 0x0000)
+    H.check_attention(run.out.cpu().numpy(), ref, f"signed zeros G={G}")
