@@ -52,7 +52,8 @@ class _CConfig(ctypes.Structure):
         ("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32), ("value_bits", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("residual", ctypes.c_int32), ("hadamard", ctypes.c_int32),
-        ("layout", ctypes.c_int32), ("sink", ctypes.c_int32), ("capacity", ctypes.c_int64),
+        ("layout", ctypes.c_int32), ("sink", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+        ("capacity", ctypes.c_int64),
     ]
 
 
@@ -101,11 +102,12 @@ class Config:
     head_dim: int = 128
     layout: int = 1  # 1 = tile v1 (mma fragment order), 2 = rows v2 (token rows of keys, channel rows of values)
     sink: int = 0    # 1: the first token stays in fp16 (an extra row after the ring)
+    rope_theta: float = 0.0  # > 0: keys are cached before RoPE and decode applies it (0: off)
 
     def c(self) -> _CConfig:
         return _CConfig(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.key_bits,
                         self.value_bits, self.group_size, self.residual, self.hadamard, self.layout, self.sink,
-                        self.capacity)
+                        self.rope_theta, self.capacity)
 
 
 class Cache:

@@ -33,10 +33,19 @@
 //      code = clamp(rint_half_even((f32(x) - f32(mn)) * inv), 0, 2^b - 1), each op one IEEE fp32
 //      rounding, never fused.
 //  R6  dequant x^ = code * s16 + zero, evaluated here in fp64.
-//  R7  attention in fp64: no causal mask, no sink token, no RoPE; softmax over all T tokens.
+//  R7  attention in fp64: no causal mask; softmax over all T tokens (the sink token, R10, and RoPE,
+//      R11, are options, off by default).
 //  R8  packed layouts "tile v1" (mma fragment order) and "rows v2" (one token's key codes, one
 //      channel's value codes per row); see key_word_bit / value_word_bit / key_param_pos and the
 //      v2 functions below.
+//  R10 optional attention sink: the first token stays in fp16 (see quantize_span and key_row).
+//  R11 optional pre-RoPE keys (rope_theta > 0; KVQuant review, Method and Key idea: keys are
+//      quantized before RoPE, and RoPE is applied after dequantization). The cache holds the keys as
+//      given, without RoPE; decode rotates every key at its absolute position t (0-based) after
+//      dequantization, or from its fp16 row: channel pairs (i, i + 64), i < 64, by the angle
+//      t * theta^(-i/64), k'[i] = k[i] cos - k[i+64] sin, k'[i+64] = k[i] sin + k[i+64] cos, in
+//      fp64. The query is taken as given (rotated at its own position by the caller). RoPE and the
+//      Hadamard option exclude each other.
 //
 // Build: g++ -O2 -std=c++17 -ffp-contract=off -fno-fast-math -fPIC -shared (x86-64 SSE scalar fp32).
 
@@ -254,7 +263,8 @@ extern "C" {
 typedef struct {
   int32_t batch, num_q_heads, num_kv_heads, head_dim;
   int32_t key_bits, value_bits, group_size, residual, hadamard, layout;  // layout: 1 = tile v1, 2 = rows v2
-  int32_t sink;  // 1: the first token stays in fp16 (reading R10)
+  int32_t sink;        // 1: the first token stays in fp16 (reading R10)
+  float rope_theta;    // > 0: keys are cached before RoPE, decode applies it (reading R11); 0: off
   int64_t capacity;
 } kvq_ref_config;
 
@@ -283,6 +293,8 @@ static int check_config(const kvq_ref_config* c) {
   if (c->residual < 0 || c->capacity < 0 || c->capacity % G) return REF_ERR_ARG;
   if (c->layout != 1 && c->layout != 2) return REF_ERR_ARG;
   if (c->sink != 0 && c->sink != 1) return REF_ERR_ARG;
+  if (!(c->rope_theta >= 0.0f) || !std::isfinite(c->rope_theta)) return REF_ERR_ARG;
+  if (c->rope_theta > 0.0f && c->hadamard) return REF_ERR_ARG;
   return REF_OK;
 }
 
@@ -537,6 +549,17 @@ static void value_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64
   }
 }
 
+// RoPE of one key at position t (reading R11): channel pairs (i, i + 64) rotated by t * omega[i].
+static void rope_rotate(double* k, int64_t t, const double* omega) {
+  for (int i = 0; i < 64; ++i) {
+    const double ang = static_cast<double>(t) * omega[i];
+    const double cs = std::cos(ang), sn = std::sin(ang);
+    const double a = k[i], b = k[i + 64];
+    k[i] = a * cs - b * sn;
+    k[i + 64] = a * sn + b * cs;
+  }
+}
+
 // Exact attention of query head h of sequence b over the dequantized cache (reading R7).
 static void decode_head(const kvq_ref_config* c, const kvq_ref_cache* cache, const uint16_t* q, double sm_scale,
                         int64_t b, int64_t h, double* out) {
@@ -551,9 +574,13 @@ static void decode_head(const kvq_ref_config* c, const kvq_ref_cache* cache, con
   if (c->hadamard) wht128_f64(qv);
   std::vector<double> s(static_cast<size_t>(T));
   double row[128];
+  double omega[64];  // RoPE frequencies theta^(-i/64)
+  const bool rope = c->rope_theta > 0.0f;
+  for (int i = 0; i < 64; ++i) omega[i] = rope ? std::pow(static_cast<double>(c->rope_theta), -i / 64.0) : 0.0;
   double mx = -INFINITY;
   for (int64_t t = 0; t < T; ++t) {
     key_row(c, cache, unit, t, Q, row);
+    if (rope) rope_rotate(row, t, omega);
     double acc = 0.0;
     for (int i = 0; i < 128; ++i) acc += qv[i] * row[i];
     s[t] = sm_scale * acc;

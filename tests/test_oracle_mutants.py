@@ -58,6 +58,16 @@ MUTANTS = [
      "  if (t >= Q || (c->sink && t == 0)) {\n    const int64_t row = (c->sink && t == 0) ? d.ring : t % d.ring;\n    const uint16_t* r = cache->k_res",
      "  if (t >= Q) {\n    const int64_t row = (c->sink && t == 0) ? d.ring : t % d.ring;\n    const uint16_t* r = cache->k_res",
      ["test_sink_dominant_first_token_returns_its_fp16_value"]),
+    ("rope_sin_sign_flipped",
+     "    k[i] = a * cs - b * sn;", "    k[i] = a * cs + b * sn;",
+     ["test_rope_without_quantization_equals_library_attention_on_rotated_keys"]),
+    ("rope_frequency_exponent_halved",
+     "std::pow(static_cast<double>(c->rope_theta), -i / 64.0)",
+     "std::pow(static_cast<double>(c->rope_theta), -i / 128.0)",
+     ["test_rope_without_quantization_equals_library_attention_on_rotated_keys"]),
+    ("rope_position_off_by_one",
+     "    if (rope) rope_rotate(row, t, omega);", "    if (rope) rope_rotate(row, t + 1, omega);",
+     ["test_rope_without_quantization_equals_library_attention_on_rotated_keys", "test_rope_relative_position"]),
     ("value_group_index_off",
      "    const int j = ch / c->group_size;", "    const int j = (ch / c->group_size + 1) % d.vpt;",
      ["test_quantized_attention_equals_library_attention_on_dequantized_cache"]),
@@ -88,6 +98,7 @@ def _run_pin(fn_name, mod):
             [dict(kb=2, vb=2, G=32, R=32, had=0, layout=1), dict(kb=2, vb=2, G=32, R=32, had=0, layout=2)],
         "test_sink_first_token_left_out_of_group_zero": [dict(layout=1), dict(layout=2)],
         "test_sink_dominant_first_token_returns_its_fp16_value": [dict(layout=1), dict(layout=2)],
+        "test_rope_without_quantization_equals_library_attention_on_rotated_keys": [dict(theta=10000.0)],
     }.get(fn_name, [dict()])
     for kw in params:
         fn(mod, **kw)

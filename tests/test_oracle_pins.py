@@ -255,8 +255,8 @@ def test_layout_v2_is_a_bijection_onto_rows(oracle_mod, kind, bits):
 # --------------------------------------------------------------------------------------------------
 # whole-cache behaviour
 # --------------------------------------------------------------------------------------------------
-def _cfg(oracle_mod, B=2, Hq=4, Hkv=2, kb=2, vb=2, G=32, R=32, had=0, cap=512, layout=1, sink=0):
-    return oracle_mod.Config(B, Hq, Hkv, kb, vb, G, R, had, cap, layout=layout, sink=sink)
+def _cfg(oracle_mod, B=2, Hq=4, Hkv=2, kb=2, vb=2, G=32, R=32, had=0, cap=512, layout=1, sink=0, rope=0.0):
+    return oracle_mod.Config(B, Hq, Hkv, kb, vb, G, R, had, cap, layout=layout, sink=sink, rope_theta=rope)
 
 
 def _inputs(B, T, Hkv, Hq, seed, outliers=True):
@@ -582,3 +582,102 @@ def test_sink_streaming_from_empty_equals_bulk(oracle_mod, layout, had):
         np.testing.assert_array_equal(getattr(stream, key)[:, :, :Q], getattr(bulk, key)[:, :, :Q])
     np.testing.assert_array_equal(stream.k_res[:, :, R + G], bulk.k_res[:, :, R + G])
     np.testing.assert_array_equal(stream.v_res[:, :, R + G], bulk.v_res[:, :, R + G])
+
+
+
+# ---- pre-RoPE keys (KVQuant review, Method and Key idea: quantize keys before RoPE, apply RoPE after
+# dequantization) ------------------------------------------------------------------------------------
+def _rope_complex(K, theta):
+    """RoPE written as complex multiplication: channel pair (i, i + 64) is the complex number
+    k[i] + j k[i + 64], turned by exp(j t theta^(-i/64)) at position t. K: [..., T, 128] float64."""
+    T = K.shape[-2]
+    z = K[..., :64] + 1j * K[..., 64:]
+    ang = np.arange(T, dtype=np.float64)[:, None] * theta ** (-np.arange(64, dtype=np.float64) / 64.0)[None, :]
+    z = z * np.exp(1j * ang)
+    return np.concatenate([z.real, z.imag], axis=-1)
+
+
+@pytest.mark.parametrize("theta", [10000.0, 500000.0])
+def test_rope_without_quantization_equals_library_attention_on_rotated_keys(oracle_mod, theta):
+    # R >= T: nothing is quantized; the cache keeps the keys without RoPE, and decode rotates each one
+    # at its own position, so the result is plain softmax attention over the rotated keys (GQA 2:1).
+    B, T, Hkv, Hq = 2, 300, 2, 4
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, R=512, cap=512, rope=theta)
+    k, v, q = _inputs(B, T, Hkv, Hq, 61)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [T, T - 99])
+    # the window holds the keys exactly as given (no RoPE in the cache)
+    ring = cfg.residual + cfg.group_size
+    assert np.array_equal(cache.k_res[0, 1, 7 % ring], k[0, 7, 1].view(np.uint16))
+    out = oracle_mod.decode(cfg, cache, q, 1 / math.sqrt(128))
+    for b, Tb in enumerate([T, T - 99]):
+        kb = _rope_complex(k[b, :Tb].astype(np.float64).transpose(1, 0, 2), theta)[None]
+        vb = v[b, :Tb].astype(np.float64).transpose(1, 0, 2)[None]
+        ref = _sdpa(q[b:b + 1].astype(np.float64), kb, vb, 1 / math.sqrt(128))
+        np.testing.assert_allclose(out[b], ref[0], rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_rope_quantized_equals_library_attention_on_dequantized_rotated_keys(oracle_mod, layout):
+    # Keys are quantized before RoPE: the dequantized cache rotated at each position, then plain
+    # attention, gives the oracle's output; and the stored codes equal those of the same cache
+    # without RoPE (quantization does not see the rotation).
+    B, Hkv, Hq, G, R = 1, 2, 4, 32, 32
+    lens = [301]
+    theta = 10000.0
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=384, layout=layout, rope=theta)
+    k, v, q = _inputs(B, max(lens), Hkv, Hq, 62)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, lens)
+    pcfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=384, layout=layout)
+    plain = oracle_mod.Cache(pcfg)
+    oracle_mod.quantize_prefill(pcfg, plain, k, v, lens)
+    for name in ("k_codes", "k_scale", "k_zero", "v_codes", "k_res"):
+        assert np.array_equal(getattr(cache, name), getattr(plain, name)), name
+    out = oracle_mod.decode(cfg, cache, q, 1 / math.sqrt(128))
+    T = lens[0]
+    Q = max(T - R, 0) // G * G
+    ring = R + G
+    K = np.zeros((Hkv, T, 128))
+    V = np.zeros((Hkv, T, 128))
+    for h in range(Hkv):
+        for t in range(T):
+            if t < Q:
+                K[h, t] = _unpack_key(oracle_mod, cfg, cache, 0, h, t)
+                V[h, t] = _unpack_value(oracle_mod, cfg, cache, 0, h, t)
+            else:
+                K[h, t] = cache.k_res[0, h, t % ring].view(np.float16)
+                V[h, t] = cache.v_res[0, h, t % ring].view(np.float16)
+    ref = _sdpa(q.astype(np.float64), _rope_complex(K, theta)[None], V[None], 1 / math.sqrt(128))
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_rope_relative_position(oracle_mod):
+    # RoPE makes q.k depend on positions only through their difference: a query turned by m positions
+    # against keys at positions t scores like the unturned query against keys at t - m. With a single
+    # key repeated at every position, turning the query by m therefore moves the attention pattern by m.
+    T, theta = 64, 10000.0
+    cfg = _cfg(oracle_mod, 1, 1, 1, R=128, cap=128, rope=theta)
+    rng = np.random.default_rng(63)
+    k1 = rng.standard_normal(128).astype(np.float16)
+    k = np.tile(k1, (1, T, 1, 1)).reshape(1, T, 1, 128)
+    v = np.zeros((1, T, 1, 128), np.float16)
+    v[0, :, 0, 0] = np.arange(T) / 8.0        # channel 0 of the output: the mean attended position / 8
+    v[0, :, 0, 1] = (np.arange(T) % 2) * 1.0
+    q0 = (2.0 * k1.astype(np.float64))
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k.astype(np.float16), v, [T])
+    m = 20
+    z = q0[:64] + 1j * q0[64:]
+    z = z * np.exp(1j * m * theta ** (-np.arange(64) / 64.0))
+    qm = np.concatenate([z.real, z.imag]).astype(np.float16)[None, None]
+    out_m = oracle_mod.decode(cfg, cache, qm, 0.5)
+    # reference: scores of the turned query equal those of q0 against keys rotated by (t - m)
+    qm64 = qm.astype(np.float64)[0, 0]
+    K = _rope_complex(np.tile(k1.astype(np.float64), (T, 1)), theta)
+    s = 0.5 * K @ qm64
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    assert abs(out_m[0, 0, 0] - p @ (np.arange(T) / 8.0)) < 1e-9
+    # the attention peaks at position m, where the key is turned exactly like the query
+    assert int(np.argmax(s)) == m
