@@ -184,7 +184,8 @@ def measured_hbm_peak():
 # ---------------------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------------------------------
-def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int = 1, sink: int = 0):
+def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int = 1, sink: int = 0,
+                         rope: float = 0.0):
     """Time the oracle's decode on a bounded sample of the workload: whole (sequence, KV head) units
     batched into one oracle problem (enough units to give every host core a query head), decoded
     repeatedly until about budget_s seconds have passed. Returns (GB/s of algorithmic decode bytes,
@@ -206,7 +207,7 @@ def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int
     if layout == 2:
         cap = -(-cap // 128) * 128
     ocfg = ref.Config(n, g, 1, w.key_bits, w.value_bits, w.group_size, w.residual, w.hadamard, cap,
-                      layout=layout, sink=sink)
+                      layout=layout, sink=sink, rope_theta=rope)
     k = np.zeros((n, Tmax, 1, 128), np.float16)
     v = np.zeros_like(k)
     qs = np.zeros((n, g, 128), np.float16)
@@ -236,7 +237,7 @@ def workload_config(w: inputs.Workload, args, step_bytes: int) -> dict:
             "num_kv_heads": w.num_kv_heads, "key_bits": w.key_bits, "value_bits": w.value_bits,
             "group_size": w.group_size, "residual": w.residual, "hadamard": w.hadamard,
             "ragged": bool(w.ragged_min), "parallelism": f"replicas{args.gpus}", "layout": args.layout,
-            "sink": args.sink, "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
+            "sink": args.sink, "rope_theta": args.rope, "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
 
 
 def run_reference(args, w):
@@ -251,7 +252,7 @@ def run_reference(args, w):
     per_step = []
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
-        gbs, cores, sample = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink)
+        gbs, cores, sample = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink, rope=args.rope)
         if i >= args.warmup:
             per_step.append(gbs)
     value = statistics.mean(per_step)
@@ -286,6 +287,8 @@ def main():
                     help="packed layout: 1 = tile v1 (mma.sync decode), 2 = rows v2 (tcgen05 decode)")
     ap.add_argument("--sink", type=int, default=0, choices=[0, 1],
                     help="1: keep every sequence's first token in fp16 (attention sink)")
+    ap.add_argument("--rope", type=float, default=0.0,
+                    help="> 0: cache keys before RoPE with this theta and rotate them in decode (needs --layout 2)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w0 = inputs.WORKLOADS[args.workload]
@@ -325,7 +328,7 @@ def main():
     if args.layout == 2:
         cap = -(-cap // 128) * 128  # rows v2 stores values in whole 128-token blocks
     cfg = kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size, w.residual,
-                          w.hadamard, cap, layout=args.layout, sink=args.sink)
+                          w.hadamard, cap, layout=args.layout, sink=args.sink, rope_theta=args.rope)
     cache = kvq.Cache(cfg)
     stream = torch.cuda.current_stream()
 
@@ -458,7 +461,8 @@ def main():
         "append_us": round(statistics.mean(append_ms) * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout), "peak_kind": peak_kind,
-                     "kernel": ("decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
+                     "kernel": ("decode_rope_kernel" if args.rope > 0 else
+                                "decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
                      + " + decode_combine_kernel (one kvq_decode_attention call)"},
         "prefill": {"gbs": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9, 1),
                     "ms": round(statistics.mean(pre_ms), 3), "bytes": pre_bytes, "bound": "hbm", "peak": peak,
@@ -474,7 +478,7 @@ def main():
         import oracle as ref
 
         ref.build()
-        gbs, cores, sample = oracle_decode_sample(w0, layout=args.layout, sink=args.sink)
+        gbs, cores, sample = oracle_decode_sample(w0, layout=args.layout, sink=args.sink, rope=args.rope)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     print(json.dumps(line), flush=True)

@@ -38,7 +38,8 @@ class kvq_config(ctypes.Structure):
         ("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32), ("value_bits", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("residual", ctypes.c_int32), ("hadamard", ctypes.c_int32),
-        ("layout", ctypes.c_int32), ("sink", ctypes.c_int32), ("capacity", ctypes.c_int64),
+        ("layout", ctypes.c_int32), ("sink", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+        ("capacity", ctypes.c_int64),
     ]
 
 
@@ -79,9 +80,9 @@ def kvq_status_string(status: int) -> str:
 
 def make_config(batch: int, num_q_heads: int, num_kv_heads: int, key_bits: int, value_bits: int, group_size: int,
                 residual: int, hadamard: int, capacity: int, head_dim: int = 128,
-                layout: int = KVQ_LAYOUT_TILE_V1, sink: int = 0) -> kvq_config:
+                layout: int = KVQ_LAYOUT_TILE_V1, sink: int = 0, rope_theta: float = 0.0) -> kvq_config:
     return kvq_config(batch, num_q_heads, num_kv_heads, head_dim, key_bits, value_bits, group_size, residual,
-                      hadamard, layout, sink, capacity)
+                      hadamard, layout, sink, rope_theta, capacity)
 
 
 def _check(status: int, where: str) -> None:

@@ -13,7 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libkvq.so")
-SOURCES = ["kvq_api.cu", "kvq_prefill.cu", "kvq_quantize.cu", "kvq_decode.cu", "kvq_decode_tc.cu", "kvq_static.cu"]
+SOURCES = ["kvq_api.cu", "kvq_prefill.cu", "kvq_quantize.cu", "kvq_decode.cu", "kvq_decode_tc.cu", "kvq_decode_rope.cu",
+           "kvq_static.cu"]
 HEADERS = ["kvq_common.cuh", "kvq_decode_common.cuh", "kvq_internal.h"]
 
 NVCC_FLAGS = [

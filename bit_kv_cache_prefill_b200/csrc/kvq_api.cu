@@ -35,6 +35,9 @@ kvq_status check_config(const kvq_config* c) {
   if (c->residual < 0 || c->residual > kMaxResidual) return KVQ_ERR_INVALID_ARG;
   if (c->hadamard != 0 && c->hadamard != 1) return KVQ_ERR_INVALID_ARG;
   if (c->sink != 0 && c->sink != 1) return KVQ_ERR_INVALID_ARG;
+  if (!(c->rope_theta >= 0.f) || !std::isfinite(c->rope_theta)) return KVQ_ERR_INVALID_ARG;
+  if (c->rope_theta > 0.f && c->hadamard) return KVQ_ERR_INVALID_ARG;                 // the two exclude each other
+  if (c->rope_theta > 0.f && c->layout != KVQ_LAYOUT_ROWS_V2) return KVQ_ERR_UNSUPPORTED;  // token-row keys only
   if (c->capacity < 0 || c->capacity % G != 0) return KVQ_ERR_INVALID_ARG;
   if (c->capacity >= (int64_t(1) << 31)) return KVQ_ERR_INVALID_ARG;  // token indices are 32-bit on the device
   if (c->layout == KVQ_LAYOUT_ROWS_V2 && c->capacity % 128 != 0) return KVQ_ERR_INVALID_ARG;  // whole value blocks
@@ -206,7 +209,9 @@ kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, size_t* bytes) {
   if (bytes == nullptr) return KVQ_ERR_INVALID_ARG;
   const int64_t units = static_cast<int64_t>(cfg->batch) * cfg->num_kv_heads;
   const int64_t g = cfg->num_q_heads / cfg->num_kv_heads;
-  *bytes = static_cast<size_t>(units * max_splits(cfg) * g * kvq::kPartFloats) * sizeof(float);
+  size_t part = static_cast<size_t>(units * max_splits(cfg) * g * kvq::kPartFloats) * sizeof(float);
+  if (cfg->rope_theta > 0.f) part = (part + 255) / 256 * 256 + static_cast<size_t>(kvq::rope_table_floats(cfg->capacity)) * 4;
+  *bytes = part;
   return KVQ_OK;
 }
 
@@ -231,7 +236,8 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
     return n;
   });
   if (sms <= 0) return KVQ_ERR_CUDA;
-  const int occ = cfg->layout == KVQ_LAYOUT_ROWS_V2
+  const int occ = cfg->rope_theta > 0.f ? kvq::decode_rope_ctas_per_sm()
+                  : cfg->layout == KVQ_LAYOUT_ROWS_V2
                       ? kvq::decode_tc_ctas_per_sm(cfg->group_size, cfg->num_q_heads / cfg->num_kv_heads)
                       : kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size,
                                                 cfg->num_q_heads / cfg->num_kv_heads);
@@ -271,6 +277,13 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   a.split_len = L;
   a.nsplit = nsplit;
   a.qscale = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  if (cfg->rope_theta > 0.f) {
+    const size_t part = static_cast<size_t>(static_cast<int64_t>(cfg->batch) * cfg->num_kv_heads * max_splits(cfg) *
+                                            a.gqa * kvq::kPartFloats) * sizeof(float);
+    a.rope_theta = cfg->rope_theta;
+    a.rope_base = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + (part + 255) / 256 * 256);
+    a.rope_off = a.rope_base + (cfg->capacity + 31) / 32 * 64;
+  }
   return cuda_status(kvq::launch_decode(a, static_cast<cudaStream_t>(cuda_stream)));
 }
 

@@ -754,7 +754,9 @@ int occupancy_vpt(int G, int gqa) {
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e;
-  if (a.layout == KVQ_LAYOUT_ROWS_V2)
+  if (a.rope_theta > 0.f)
+    e = launch_decode_rope(a, stream);
+  else if (a.layout == KVQ_LAYOUT_ROWS_V2)
     e = launch_decode_tc(a, stream);
   else if (a.key_bits == 2)
     e = a.value_bits == 2 ? dispatch_vpt<2, 2>(a, stream) : dispatch_vpt<2, 4>(a, stream);

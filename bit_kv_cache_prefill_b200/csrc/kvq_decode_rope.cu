@@ -1,0 +1,480 @@
+// kvq_decode_rope.cu — split-K decode attention over pre-RoPE keys (rows-v2 layout), on CUDA cores.
+//
+// Keys can be cached before RoPE and rotated only after dequantization (KVQuant review, Method and
+// Key idea: RoPE mixes channel pairs and smears the key outlier channels, so the quantizer runs
+// before the rotation and a fused kernel applies RoPE to the dequantized keys). Token t's key is
+// turned pair by pair, channels (i, i + 64), by the angle t * theta^(-i/64); the query arrives already
+// rotated at its own position.
+//
+// A rotation per token defeats the shared-B tensor-core formulation of the other decode kernels (the
+// effective query would change with every key row), so this path computes on CUDA cores:
+//   * QK, lane = token. <q, R_t k> = <R_-t0 q, R_j k> with t = t0 + j and t0 the warp step's first
+//     token (a multiple of 32): the query is turned once per step to R_-t0 q (cooperatively, into
+//     shared memory) and each lane turns its dequantized key by its in-step offset j only, from a
+//     padded shared table of cos / sin (j w_i).
+//   * PV, lane = 4 channels. o = sum_t (p_t sv_t) c_t + sum_t p_t zv_t per value group.
+//   * Codes are read as fp16 subnormals (one AND per code pair, the position's power of two folded
+//     into the staged scales), as in the tile-v1 kernel.
+// The angle tables are built once per call in fp64 (cos / sin of 32 s w_i and of j w_i) into the
+// decode workspace behind the split partials; partials have the layout the split-combine kernel
+// reads.
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "kvq_common.cuh"
+#include "kvq_decode_common.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+constexpr int kRW = 4;         // warps per CTA
+constexpr int kRStep = 32;     // tokens per warp step
+constexpr unsigned kAll = 0xffffffffu;
+constexpr int kOffStride = 65;  // padded row of the in-step cos / sin tables (conflict-free per lane)
+constexpr int kRPart = 132;    // shared partial stride (floats): m, l, 2 pad, o[128]
+
+// (cos, sin) of 32 s w_i for s < nbase and of j w_i for j < 32, w_i = theta^(-i/64), in fp64.
+__global__ void rope_table_kernel(float2* base, float2* off, int nbase, float theta) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const int i = idx & 63, s = idx >> 6;
+  const double w = pow(static_cast<double>(theta), -static_cast<double>(i) / 64.0);
+  double sn, cs;
+  if (s < nbase) {
+    sincos(static_cast<double>(kRStep) * static_cast<double>(s) * w, &sn, &cs);
+    base[idx] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  }
+  if (s < kRStep) {
+    sincos(static_cast<double>(s) * w, &sn, &cs);
+    off[idx] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  }
+}
+
+// Shared memory layout (bytes).
+template <int GQ>
+struct RopeSmem {
+  static constexpr int oQ = 0;                                  // q~ [GQ][128] f32 (base-2 logits)
+  static constexpr int oCos = oQ + GQ * 128 * 4;                // cos (j w_i) [32][65] f32
+  static constexpr int oSin = oCos + kRStep * kOffStride * 4;   // sin (j w_i) [32][65] f32
+  static constexpr int oWarp = oSin + kRStep * kOffStride * 4;  // per-warp areas
+  // per warp: turned query [GQ][64] float4 (q_i, q_{i+1}, q_{i+64}, q_{i+65}) for even i -> [GQ][32]
+  // float4; key scale / zero of up to two groups [2][32] float4 x 2 (low / high channel pairs);
+  // value scale (pre-scaled) / zero of the step's tokens [32][8] f32 x 2
+  static constexpr int wQ = 0;
+  static constexpr int wKP = wQ + GQ * 32 * 16;
+  static constexpr int wVS = wKP + 2 * 2 * 32 * 16;
+  static constexpr int wVZ = wVS + kRStep * 8 * 4;
+  static constexpr int kWarpBytes = wVZ + kRStep * 8 * 4;
+  static constexpr int kLoop = oWarp + kRW * kWarpBytes;
+  static constexpr int kEpi = oWarp + kRW * GQ * kRPart * 4;  // warp partials reuse the per-warp areas
+  static constexpr int kBytes = kLoop > kEpi ? kLoop : kEpi;
+};
+
+// Two codes of a word as the fp16 subnormals code * 2^(bit - 24), converted to fp32. Only bits 0..9
+// of a half are mantissa, so a code at bit offset o >= 8 of its half is first shifted down by 8:
+// codes are read at offset o & 7 and carry 2^((o & 7) - 24).
+__device__ __forceinline__ float2 sub2f(uint32_t x) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&x));
+}
+template <int BITS>
+__device__ __forceinline__ float2 code_pair(uint32_t word, int slot) {  // slot: compile-time after unrolling
+  const int o = BITS * slot;
+  const uint32_t m = ((1u << BITS) - 1u) << (o & 7);
+  return sub2f((o >= 8 ? word >> 8 : word) & (m | (m << 16)));
+}
+
+template <int KB, int VB, int G, int GQ>
+__global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs a, const float2* __restrict__ rbase,
+                                                               const float2* __restrict__ roff) {
+  using SM = RopeSmem<GQ>;
+  constexpr int VPT = kHeadDim / G;
+  constexpr int KW = 4 * KB;       // key words per token
+  constexpr int KP = 16 / KB;      // code pairs per key word
+  constexpr int VW = 4 * VB;       // value words per channel row of a 128-token block
+  constexpr int VP = 16 / VB;      // token pairs per value word
+  extern __shared__ __align__(16) uint8_t smem[];
+  float* sq = reinterpret_cast<float*>(smem + SM::oQ);
+  float* scos = reinterpret_cast<float*>(smem + SM::oCos);
+  float* ssin = reinterpret_cast<float*>(smem + SM::oSin);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* wsm = smem + SM::oWarp + warp * SM::kWarpBytes;
+  float4* wq = reinterpret_cast<float4*>(wsm + SM::wQ);    // [GQ][32]
+  float4* wkp = reinterpret_cast<float4*>(wsm + SM::wKP);  // [2 groups][2 halves][32]
+  float* wvs = reinterpret_cast<float*>(wsm + SM::wVS);    // [32][VPT]
+  float* wvz = reinterpret_cast<float*>(wsm + SM::wVZ);
+
+  const int split = blockIdx.x;
+  const int64_t unit = blockIdx.y;
+  const int64_t b = unit / a.num_kv_heads;
+  const int kvh = static_cast<int>(unit % a.num_kv_heads);
+  const int gq = a.gqa;
+  const int T = static_cast<int>(a.seq_len[b]);
+  const int L = a.split_len;
+  const int start = split * L;
+  if (start >= T) return;
+  const int end = min(start + L, T);
+  const int Q = static_cast<int>(quantized_len(T, a.R, G));
+  const int qend = min(end, Q);
+
+  // ---- query (scaled to base-2 logits) and the in-step angle tables
+  for (int idx = threadIdx.x; idx < GQ * kHeadDim; idx += kRW * 32) {
+    const int h = idx >> 7, c = idx & 127;
+    sq[idx] = h < gq ? h2f(a.q[(b * a.num_q_heads + static_cast<int64_t>(kvh) * gq + h) * kHeadDim + c]) * a.qscale : 0.f;
+  }
+  for (int idx = threadIdx.x; idx < kRStep * 64; idx += kRW * 32) {
+    const int j = idx >> 6, i = idx & 63;
+    const float2 cs = roff[idx];
+    scos[j * kOffStride + i] = cs.x;
+    ssin[j * kOffStride + i] = cs.y;
+  }
+  __syncthreads();
+
+  // ---- this warp's quantized steps (contiguous runs of 32 tokens)
+  const int nsteps = qend > start ? (qend - start + kRStep - 1) / kRStep : 0;
+  const int per = (nsteps + kRW - 1) / kRW;
+  const int sb = min(nsteps, per * warp);
+  const int nst = min(nsteps, per * (warp + 1)) - sb;
+
+  float m_run[GQ], l_run[GQ], o[GQ][4], zacc[GQ];
+#pragma unroll
+  for (int h = 0; h < GQ; ++h) {
+    m_run[h] = -CUDART_INF_F;
+    l_run[h] = 0.f;
+    zacc[h] = 0.f;
+    o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0.f;
+  }
+  const int c0 = 4 * lane;    // PV: this lane's channels c0 .. c0 + 3
+  const int jv = c0 / G;      // their value group
+  int kp_group = -1;          // first key group staged in wkp
+
+  for (int i = 0; i < nst; ++i) {
+    const int t0 = start + (sb + i) * kRStep;
+    const int t = t0 + lane;
+    const bool valid = t < qend && !(a.sink && t == 0);
+    // key scale / zero of the step's groups: wkp[g][half][p] = (s, z) of channels 2p, 2p + 1
+    // (half 0) or 64 + 2p, 65 + 2p (half 1), fp16 scales pre-multiplied by 2^(24 - bit) of their
+    // code position so that a subnormal code times the scale is code * s
+    const int g0 = t0 / G;
+    if (g0 != kp_group) {
+      kp_group = g0;
+      constexpr int NG = G >= kRStep ? 1 : kRStep / G;
+#pragma unroll
+      for (int gg = 0; gg < NG; ++gg) {
+        const int64_t gidx = (unit * a.groups + g0 + gg) * kHeadDim;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int c = 64 * hf + 2 * lane;
+          const uint32_t sv = *reinterpret_cast<const uint32_t*>(a.k_scale + gidx + c);
+          const uint32_t zv = *reinterpret_cast<const uint32_t*>(a.k_zero + gidx + c);
+          // channel c sits in key word c / (2 KP) at pair slot (c % (2 KP)) / 2, bit KB * slot
+          const int slot = (c % (2 * KP)) / 2;
+          const float sc = pow2i(24 - ((KB * slot) & 7));
+          wkp[(gg * 2 + hf) * 32 + lane] = make_float4(h2f(static_cast<uint16_t>(sv & 0xffffu)) * sc,
+                                                       h2f(static_cast<uint16_t>(zv & 0xffffu)),
+                                                       h2f(static_cast<uint16_t>(sv >> 16)) * sc,
+                                                       h2f(static_cast<uint16_t>(zv >> 16)));
+        }
+      }
+    }
+    // value scale / zero of the step's tokens: wvs pre-multiplied by 2^(24 - bit) of the token's
+    // position in its value word (token pair slot (t % 128 / 2) % VP, bit VB * slot)
+    for (int idx = lane; idx < kRStep * VPT; idx += 32) {
+      const int jj = idx / VPT, g = idx % VPT;
+      const int tt = t0 + jj;
+      const bool ok = tt < qend;
+      const int64_t pidx = (unit * a.capacity + (ok ? tt : 0)) * VPT + g;
+      const int slot = ((tt & 127) >> 1) % VP;
+      wvs[jj * VPT + g] = ok ? h2f(a.v_scale[pidx]) * pow2i(24 - ((VB * slot) & 7)) : 0.f;
+      wvz[jj * VPT + g] = ok ? h2f(a.v_zero[pidx]) : 0.f;
+    }
+    // the query turned back to the step start: R_-t0 q, pair (i, i + 64) by -t0 w_i
+    {
+      const float2* bt = rbase + static_cast<int64_t>(t0 / kRStep) * 64;
+      const float2 cs0 = bt[2 * lane], cs1 = bt[2 * lane + 1];  // pairs 2 lane, 2 lane + 1
+#pragma unroll
+      for (int h = 0; h < GQ; ++h) {
+        const float* qh = sq + h * kHeadDim;
+        const float a0 = qh[2 * lane], a1 = qh[2 * lane + 1], b0 = qh[64 + 2 * lane], b1 = qh[65 + 2 * lane];
+        // R_-x (a, b) = (a cos + b sin, b cos - a sin)
+        wq[h * 32 + lane] = make_float4(fmaf(a0, cs0.x, b0 * cs0.y), fmaf(a1, cs1.x, b1 * cs1.y),
+                                        fmaf(b0, cs0.x, -a0 * cs0.y), fmaf(b1, cs1.x, -a1 * cs1.y));
+      }
+    }
+    __syncwarp();
+
+    // -- QK: lane = token t, offset j = lane from the step start
+    float s[GQ];
+#pragma unroll
+    for (int h = 0; h < GQ; ++h) s[h] = 0.f;
+    {
+      uint32_t kw[KW];
+      const uint4* src = reinterpret_cast<const uint4*>(a.k_codes + (unit * a.capacity + (valid ? t : 0)) * KW);
+#pragma unroll
+      for (int v = 0; v < KW / 4; ++v) {
+        const uint4 x = src[v];
+        kw[4 * v] = x.x;
+        kw[4 * v + 1] = x.y;
+        kw[4 * v + 2] = x.z;
+        kw[4 * v + 3] = x.w;
+      }
+      const int gl = G >= kRStep ? 0 : lane / G;  // this token's group among the staged ones
+      const float* cj = scos + lane * kOffStride;
+      const float* sj = ssin + lane * kOffStride;
+#pragma unroll
+      for (int p = 0; p < 32; ++p) {  // channel pairs 2p, 2p + 1 (low) and 64 + 2p, 65 + 2p (high)
+        const int c = 2 * p, w = c / (2 * KP), slot = (c % (2 * KP)) / 2;
+        const float2 lo = code_pair<KB>(kw[w], slot);           // codes of c, c + 1
+        const float2 hi = code_pair<KB>(kw[w + KW / 2], slot);  // codes of c + 64, c + 65
+        const float4 kl = wkp[(gl * 2 + 0) * 32 + p];
+        const float4 kh = wkp[(gl * 2 + 1) * 32 + p];
+        const float x0 = fmaf(lo.x, kl.x, kl.y), x1 = fmaf(lo.y, kl.z, kl.w);
+        const float y0 = fmaf(hi.x, kh.x, kh.y), y1 = fmaf(hi.y, kh.z, kh.w);
+        // R_j on pairs (c, c + 64) and (c + 1, c + 65)
+        const float cs0 = cj[c], sn0 = sj[c], cs1 = cj[c + 1], sn1 = sj[c + 1];
+        const float r0 = fmaf(x0, cs0, -y0 * sn0), u0 = fmaf(x0, sn0, y0 * cs0);
+        const float r1 = fmaf(x1, cs1, -y1 * sn1), u1 = fmaf(x1, sn1, y1 * cs1);
+#pragma unroll
+        for (int h = 0; h < GQ; ++h) {
+          const float4 qv = wq[h * 32 + p];
+          s[h] = fmaf(qv.x, r0, s[h]);
+          s[h] = fmaf(qv.y, r1, s[h]);
+          s[h] = fmaf(qv.z, u0, s[h]);
+          s[h] = fmaf(qv.w, u1, s[h]);
+        }
+      }
+    }
+
+    // -- online softmax per head over the step
+    float p[GQ];
+#pragma unroll
+    for (int h = 0; h < GQ; ++h) {
+      const float sh = valid && h < gq ? s[h] : -CUDART_INF_F;
+      float mx = sh;
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kAll, mx, d));
+      const float m_new = fmaxf(m_run[h], mx);
+      const float alpha = m_new == -CUDART_INF_F ? 1.f : fast_exp2(m_run[h] - m_new);
+      p[h] = sh == -CUDART_INF_F ? 0.f : fast_exp2(sh - m_new);
+      l_run[h] = fmaf(l_run[h], alpha, p[h]);
+      zacc[h] *= alpha;
+      o[h][0] *= alpha;
+      o[h][1] *= alpha;
+      o[h][2] *= alpha;
+      o[h][3] *= alpha;
+      m_run[h] = m_new;
+    }
+
+    // -- PV: lane = channels c0 .. c0 + 3; token pairs of the channel rows of this 128-token block
+    {
+      const int64_t blk = t0 / 128;
+      const int wv0 = ((t0 & 127) >> 1) / VP;  // first value word of the step
+      constexpr int NWV = kRStep / (2 * VP);   // value words per step per channel
+      uint32_t vw[4][NWV];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t* row = a.v_codes + (unit * a.capacity + blk * 128 + c0 + e) * VW + wv0;
+#pragma unroll
+        for (int k = 0; k < NWV; ++k) vw[e][k] = row[k];
+      }
+#pragma unroll
+      for (int jp = 0; jp < kRStep / 2; ++jp) {  // token pair (2 jp, 2 jp + 1) of the step
+        const int k = jp / VP, slot = jp % VP;
+        float pe[GQ], po[GQ];
+#pragma unroll
+        for (int h = 0; h < GQ; ++h) {
+          pe[h] = __shfl_sync(kAll, p[h], 2 * jp);
+          po[h] = __shfl_sync(kAll, p[h], 2 * jp + 1);
+        }
+        const float se = wvs[(2 * jp) * VPT + jv], so = wvs[(2 * jp + 1) * VPT + jv];
+        const float ze = wvz[(2 * jp) * VPT + jv], zo = wvz[(2 * jp + 1) * VPT + jv];
+        float pse[GQ], pso[GQ];
+#pragma unroll
+        for (int h = 0; h < GQ; ++h) {
+          pse[h] = pe[h] * se;
+          pso[h] = po[h] * so;
+          zacc[h] = fmaf(pe[h], ze, fmaf(po[h], zo, zacc[h]));
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 cc = code_pair<VB>(vw[e][k], slot);  // codes of tokens 2 jp, 2 jp + 1
+#pragma unroll
+          for (int h = 0; h < GQ; ++h) o[h][e] = fmaf(pse[h], cc.x, fmaf(pso[h], cc.y, o[h][e]));
+        }
+      }
+    }
+    __syncwarp();  // the per-warp staging is rewritten by the next step
+  }
+
+  // ---- warp partials -> shared memory (l summed over lanes; the zero-point term per value group)
+  __syncthreads();  // the per-warp areas become the partials
+  float* cw = reinterpret_cast<float*>(smem + SM::oWarp) + warp * GQ * kRPart;
+#pragma unroll
+  for (int h = 0; h < GQ; ++h) {
+    float l = l_run[h];
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) l += __shfl_xor_sync(kAll, l, d);
+    float* ph = cw + h * kRPart;
+    if (lane == 0) {
+      ph[0] = m_run[h];
+      ph[1] = l;
+    }
+    *reinterpret_cast<float4*>(ph + 4 + c0) =
+        make_float4(o[h][0] + zacc[h], o[h][1] + zacc[h], o[h][2] + zacc[h], o[h][3] + zacc[h]);
+  }
+  __syncwarp();
+
+  // ---- FP16 window (and the sink row): tokens W0 + split + k ns, warp w the k = w (mod 4); RoPE at
+  //      each token's position. Lane l holds channels 2l, 2l + 1, 64 + 2l, 65 + 2l.
+  {
+    const int ns = (T + L - 1) / L;
+    const int W0 = (a.sink && Q > 0) ? Q - 1 : Q;
+    const uint16_t* kres = a.k_res + unit * a.res_rows * kHeadDim;
+    const uint16_t* vres = a.v_res + unit * a.res_rows * kHeadDim;
+    for (int k0 = warp; W0 + split + k0 * ns < T; k0 += kRW) {
+      const int tt = W0 + split + k0 * ns;
+      const int pos = tt < Q ? 0 : tt;  // the sink row is token 0
+      const int slot = tt < Q ? static_cast<int>(a.ring) : tt % static_cast<int>(a.ring);
+      const uint16_t* kr = kres + static_cast<int64_t>(slot) * kHeadDim;
+      const uint16_t* vr = vres + static_cast<int64_t>(slot) * kHeadDim;
+      const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(kr + 2 * lane));
+      const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(kr + 64 + 2 * lane));
+      const float2* bt = rbase + static_cast<int64_t>(pos / kRStep) * 64;
+      const int j = pos % kRStep;
+      float r[4];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = 2 * lane + e;
+        const float2 cb = bt[i];
+        const float cs = fmaf(cb.x, scos[j * kOffStride + i], -cb.y * ssin[j * kOffStride + i]);
+        const float sn = fmaf(cb.y, scos[j * kOffStride + i], cb.x * ssin[j * kOffStride + i]);
+        const float x = e ? lo.y : lo.x, y = e ? hi.y : hi.x;
+        r[e] = fmaf(x, cs, -y * sn);      // channel i
+        r[2 + e] = fmaf(x, sn, y * cs);   // channel i + 64
+      }
+      const float2 v_lo = __half22float2(*reinterpret_cast<const __half2*>(vr + 2 * lane));
+      const float2 v_hi = __half22float2(*reinterpret_cast<const __half2*>(vr + 64 + 2 * lane));
+#pragma unroll
+      for (int h = 0; h < GQ; ++h) {
+        if (h >= gq) break;
+        const float* qh = sq + h * kHeadDim;
+        float d = qh[2 * lane] * r[0];
+        d = fmaf(qh[2 * lane + 1], r[1], d);
+        d = fmaf(qh[64 + 2 * lane], r[2], d);
+        d = fmaf(qh[65 + 2 * lane], r[3], d);
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) d += __shfl_xor_sync(kAll, d, x);
+        float* ph = cw + h * kRPart;
+        const float m_old = ph[0];
+        const float m_new = fmaxf(m_old, d);
+        const float f_old = m_old == -CUDART_INF_F ? 0.f : fast_exp2(m_old - m_new);
+        const float pj = fast_exp2(d - m_new);
+        __syncwarp();
+        float* oo = ph + 4;
+        oo[2 * lane] = fmaf(oo[2 * lane], f_old, pj * v_lo.x);
+        oo[2 * lane + 1] = fmaf(oo[2 * lane + 1], f_old, pj * v_lo.y);
+        oo[64 + 2 * lane] = fmaf(oo[64 + 2 * lane], f_old, pj * v_hi.x);
+        oo[65 + 2 * lane] = fmaf(oo[65 + 2 * lane], f_old, pj * v_hi.y);
+        __syncwarp();
+        if (lane == 0) {
+          ph[0] = m_new;
+          ph[1] = fmaf(ph[1], f_old, pj);
+        }
+        __syncwarp();
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- CTA partial (merge the warps) -> workspace, the split-combine kernel's layout
+  float* part = a.part + ((unit * a.nsplit + split) * gq) * kPartFloats;
+  const float* allw = reinterpret_cast<const float*>(smem + SM::oWarp);
+  for (int idx = threadIdx.x; idx < gq * kHeadDim; idx += kRW * 32) {
+    const int h = idx >> 7, c = idx & 127;
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kRW; ++w) M = fmaxf(M, allw[(w * GQ + h) * kRPart]);
+    const bool empty = M == -CUDART_INF_F;
+    float ov = 0.f, l = 0.f;
+#pragma unroll
+    for (int w = 0; w < kRW; ++w) {
+      const float* pw = allw + (w * GQ + h) * kRPart;
+      const float f = empty || pw[0] == -CUDART_INF_F ? 0.f : fast_exp2(pw[0] - M);
+      ov = fmaf(f, pw[4 + c], ov);
+      l = fmaf(f, pw[1], l);
+    }
+    part[h * kPartFloats + 2 + c] = ov;
+    if (c == 0) {
+      part[h * kPartFloats] = M;
+      part[h * kPartFloats + 1] = l;
+    }
+  }
+}
+
+template <int KB, int VB, int G, int GQ>
+cudaError_t launch_rope_kernel(const DecodeArgs& a, cudaStream_t stream) {
+  using SM = RopeSmem<GQ>;
+  static DeviceMemo attr;
+  const int ok = attr.get([] {
+    return cudaFuncSetAttribute(decode_rope_kernel<KB, VB, G, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SM::kBytes) == cudaSuccess ? 1 : -1;
+  });
+  if (ok < 0) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads));
+  decode_rope_kernel<KB, VB, G, GQ><<<grid, kRW * 32, SM::kBytes, stream>>>(a, a.rope_base, a.rope_off);
+  return cudaGetLastError();
+}
+
+template <int KB, int VB, int G>
+cudaError_t rope_gq(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.gqa) {
+    case 1: return launch_rope_kernel<KB, VB, G, 1>(a, stream);
+    case 2: return launch_rope_kernel<KB, VB, G, 2>(a, stream);
+    case 3:
+    case 4: return launch_rope_kernel<KB, VB, G, 4>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int KB, int VB>
+cudaError_t rope_g(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.G) {
+    case 16: return rope_gq<KB, VB, 16>(a, stream);
+    case 32: return rope_gq<KB, VB, 32>(a, stream);
+    case 64: return rope_gq<KB, VB, 64>(a, stream);
+    case 128: return rope_gq<KB, VB, 128>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+int64_t rope_table_floats(int64_t capacity) {
+  return ((capacity + kRStep - 1) / kRStep) * 64 * 2 + kRStep * 64 * 2;
+}
+
+cudaError_t launch_decode_rope(const DecodeArgs& a, cudaStream_t stream) {
+  const int nbase = static_cast<int>((a.capacity + kRStep - 1) / kRStep);
+  const int n = (nbase > kRStep ? nbase : kRStep) * 64;
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(a.rope_base, a.rope_off, nbase, a.rope_theta);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.key_bits == 2) return a.value_bits == 2 ? rope_g<2, 2>(a, stream) : rope_g<2, 4>(a, stream);
+  return a.value_bits == 2 ? rope_g<4, 2>(a, stream) : rope_g<4, 4>(a, stream);
+}
+
+int decode_rope_ctas_per_sm() {
+  static DeviceMemo occ;
+  return occ.get([] {
+    using SM = RopeSmem<4>;
+    if (cudaFuncSetAttribute(decode_rope_kernel<2, 2, 32, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) !=
+        cudaSuccess)
+      return 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rope_kernel<2, 2, 32, 4>, kRW * 32, SM::kBytes) !=
+        cudaSuccess)
+      return 1;
+    return n > 0 ? n : 1;
+  });
+}
+
+}  // namespace kvq

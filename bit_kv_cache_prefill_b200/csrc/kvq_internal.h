@@ -50,12 +50,18 @@ struct DecodeArgs {
   int split_len;  // tokens per split (multiple of 64; rows v2: multiple of 128)
   int nsplit;     // splits per unit in the grid
   float qscale;   // sm_scale * log2(e): scores are kept in base-2 units
+  float rope_theta;  // > 0: keys are cached before RoPE; decode rotates them (rows v2 only)
+  float2* rope_base;  // workspace: (cos, sin)(32 s w_i), [ceil(capacity / 32)][64]
+  float2* rope_off;   // workspace: (cos, sin)(j w_i), [32][64]
 };
 
 cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream);
 cudaError_t launch_append(const QuantizeArgs& a, const uint16_t* k_new, const uint16_t* v_new, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);     // split + combine, either layout
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // rows-v2 split kernel only
+cudaError_t launch_decode_rope(const DecodeArgs& a, cudaStream_t stream);  // pre-RoPE keys: tables + split kernel
+int decode_rope_ctas_per_sm();
+int64_t rope_table_floats(int64_t capacity);  // floats of the two RoPE tables in the workspace
 int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);  // tile-v1 kernel
 int decode_tc_ctas_per_sm(int G, int gqa);                              // rows-v2 kernel (1 or 2)
 

@@ -60,6 +60,8 @@ typedef enum {
  *   group_size G in {16, 32, 64, 128} (a multiple of the 16-token tile and a divisor of 128);
  *   residual R >= 0 (tokens kept in FP16 beyond the last full group; 0 <= R <= 4096);
  *   hadamard in {0, 1}; layout KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2; sink in {0, 1};
+ *   rope_theta finite and >= 0; rope_theta > 0 needs hadamard = 0 (KVQ_ERR_INVALID_ARG) and layout
+ *   KVQ_LAYOUT_ROWS_V2 (KVQ_ERR_UNSUPPORTED);
  *   capacity >= 0, a multiple of G (maximum tokens per sequence); with layout ROWS_V2 also a
  *   multiple of 128 (value rows come in whole 128-token blocks). */
 typedef struct {
@@ -74,6 +76,7 @@ typedef struct {
   int32_t hadamard;
   int32_t layout;
   int32_t sink;  /* 1: the first token of every sequence stays in fp16 (see below) */
+  float rope_theta; /* > 0: keys are cached before RoPE and decode rotates them (see below); 0: off */
   int64_t capacity;
 } kvq_config;
 
@@ -100,6 +103,14 @@ typedef struct {
  * and value are also kept in fp16 in ring row R+G, written by the prefill or by the append that adds
  * token 0. Key group 0's min/max leave token 0 out, token 0's codes and value scale / zero are 0, and
  * decode reads token 0 only from its fp16 row.
+ *
+ * Pre-RoPE keys (rope_theta > 0; the KVQuant review, Method and Key idea, quantizes keys before RoPE
+ * and applies RoPE after dequantization): the cache holds the keys as passed to prefill and append,
+ * without RoPE. Decode rotates every key at its absolute position t (0-based) after dequantization,
+ * or from its fp16 row: channel pairs (i, i + 64), i < 64, by the angle t * rope_theta^(-i/64),
+ * k'[i] = k[i] cos - k[i+64] sin, k'[i+64] = k[i] sin + k[i+64] cos. The query is used as given
+ * (already rotated at its own position by the caller). The decode workspace then also holds the
+ * angle tables, built at the start of every call.
  *
  * Tile v1: tile row k of a unit holds tokens 16k..16k+15. Within a tile, "lane" L (0..31) owns
  * words (w / 4) * 128 + 4L + (w % 4) for w in [0, 2*bits). Word w holds 16/bits code pairs; pair j

@@ -21,16 +21,18 @@ def capacity(w: inputs.Workload, layout: int) -> int:
     return -(-cap // 128) * 128 if layout == 2 else cap
 
 
-def oracle_config(oracle, w: inputs.Workload, batch=None, hq=None, hkv=None, layout: int = 1, sink: int = 0):
+def oracle_config(oracle, w: inputs.Workload, batch=None, hq=None, hkv=None, layout: int = 1, sink: int = 0,
+                  rope: float = 0.0):
     return oracle.Config(batch or w.batch, hq or w.num_q_heads, hkv or w.num_kv_heads, w.key_bits, w.value_bits,
-                         w.group_size, w.residual, w.hadamard, capacity(w, layout), layout=layout, sink=sink)
+                         w.group_size, w.residual, w.hadamard, capacity(w, layout), layout=layout, sink=sink,
+                         rope_theta=rope)
 
 
-def gpu_config(w: inputs.Workload, layout: int = 1, sink: int = 0):
+def gpu_config(w: inputs.Workload, layout: int = 1, sink: int = 0, rope: float = 0.0):
     import bit_kv_cache_prefill_b200 as kvq
 
     return kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size,
-                           w.residual, w.hadamard, capacity(w, layout), layout=layout, sink=sink)
+                           w.residual, w.hadamard, capacity(w, layout), layout=layout, sink=sink, rope_theta=rope)
 
 
 @dataclass
@@ -45,11 +47,11 @@ class GpuRun:
 
 def run_gpu(w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
             appends: int = 0, sm_scale: Optional[float] = None, layout: int = 1, decode: bool = True,
-            sink: int = 0) -> GpuRun:
+            sink: int = 0, rope: float = 0.0) -> GpuRun:
     """Prefill (k, v on the device), `appends` streaming appends, one decode (unless decode=False)."""
     import bit_kv_cache_prefill_b200 as kvq
 
-    cfg = gpu_config(w, layout, sink)
+    cfg = gpu_config(w, layout, sink, rope)
     cache = kvq.Cache(cfg)
     kvq.kvq_quantize_prefill(cfg, cache, k, v, lens)
     for step in range(appends):
@@ -129,8 +131,9 @@ def check_attention(gpu_out: np.ndarray, ref: np.ndarray, what: str) -> Tuple[fl
 
 
 def oracle_full(oracle, w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
-                appends: int = 0, sm_scale: Optional[float] = None, threads: int = 8, layout: int = 1, sink: int = 0):
-    ocfg = oracle_config(oracle, w, layout=layout, sink=sink)
+                appends: int = 0, sm_scale: Optional[float] = None, threads: int = 8, layout: int = 1, sink: int = 0,
+                rope: float = 0.0):
+    ocfg = oracle_config(oracle, w, layout=layout, sink=sink, rope=rope)
     oc = oracle.Cache(ocfg)
     oracle.quantize_prefill(ocfg, oc, k.numpy(), v.numpy(), lens, threads=threads)
     for step in range(appends):

@@ -91,6 +91,33 @@ def test_config_validation(field, value, status):
     assert _status("kvq_cache_buffer_bytes", None, sizes) == kvq.KVQ_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("layout,had,theta,status", [
+    (2, 0, 10000.0, kvq.KVQ_OK), (2, 0, 0.0, kvq.KVQ_OK),
+    (1, 0, 10000.0, kvq.KVQ_ERR_UNSUPPORTED),      # pre-RoPE keys need token-row keys (rows v2)
+    (2, 1, 10000.0, kvq.KVQ_ERR_INVALID_ARG),      # RoPE and the Hadamard rotation exclude each other
+    (2, 0, -1.0, kvq.KVQ_ERR_INVALID_ARG), (2, 0, float("nan"), kvq.KVQ_ERR_INVALID_ARG),
+    (2, 0, float("inf"), kvq.KVQ_ERR_INVALID_ARG),
+])
+def test_rope_config_validation(layout, had, theta, status):
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, had, 1024, layout=layout, rope_theta=theta)
+    sizes = (ctypes.c_size_t * 8)()
+    assert _status("kvq_cache_buffer_bytes", ctypes.byref(cfg), sizes) == status
+    n = ctypes.c_size_t()
+    assert _status("kvq_decode_workspace_bytes", ctypes.byref(cfg), ctypes.byref(n)) == status
+
+
+@pytest.mark.parametrize("cap", [1024, 1 << 20])
+def test_rope_workspace_holds_the_angle_tables(cap):
+    # the cache buffers do not change; the decode workspace gains the two angle tables,
+    # (cos, sin) of every 32-token step start and of the 32 in-step offsets, after the partials
+    base = kvq.make_config(1, 32, 8, 2, 2, 128, 128, 0, cap, layout=kvq.KVQ_LAYOUT_ROWS_V2)
+    rope = kvq.make_config(1, 32, 8, 2, 2, 128, 128, 0, cap, layout=kvq.KVQ_LAYOUT_ROWS_V2, rope_theta=10000.0)
+    assert kvq.kvq_cache_buffer_bytes(rope) == kvq.kvq_cache_buffer_bytes(base)
+    part = kvq.kvq_decode_workspace_bytes(base)
+    tables = (-(-cap // 32) * 64 + 32 * 64) * 8
+    assert kvq.kvq_decode_workspace_bytes(rope) == -(-part // 256) * 256 + tables
+
+
 def _fake_cache(cfg, lens):
     # Non-null, 16-byte aligned placeholder addresses: every call below is rejected on the host before
     # any of them could be used.
