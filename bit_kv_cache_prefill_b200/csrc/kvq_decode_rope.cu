@@ -11,7 +11,7 @@
 //   * QK, lane = token. <q, R_t k> = <R_-t0 q, R_j k> with t = t0 + j and t0 the warp step's first
 //     token (a multiple of 32): the query is turned once per step to R_-t0 q (cooperatively, into
 //     shared memory) and each lane turns its dequantized key by its in-step offset j only, from a
-//     padded shared table of cos / sin (j w_i).
+//     padded shared table of (cos, sin) (j w_i) for two channel pairs per 16-byte entry.
 //   * PV, lane = 4 channels. o = sum_t (p_t sv_t) c_t + sum_t p_t zv_t per value group.
 //   * Codes are read as fp16 subnormals (one AND per code pair, the position's power of two folded
 //     into the staged scales), as in the tile-v1 kernel.
@@ -31,7 +31,7 @@ namespace {
 constexpr int kRW = 4;         // warps per CTA
 constexpr int kRStep = 32;     // tokens per warp step
 constexpr unsigned kAll = 0xffffffffu;
-constexpr int kOffStride = 65;  // padded row of the in-step cos / sin tables (conflict-free per lane)
+constexpr int kOffStride = 33;  // padded row (float4) of the in-step table: 8 lanes, 8 bank groups
 constexpr int kRPart = 132;    // shared partial stride (floats): m, l, 2 pad, o[128]
 
 // (cos, sin) of 32 s w_i for s < nbase and of j w_i for j < 32, w_i = theta^(-i/64), in fp64.
@@ -54,9 +54,8 @@ __global__ void rope_table_kernel(float2* base, float2* off, int nbase, float th
 template <int GQ>
 struct RopeSmem {
   static constexpr int oQ = 0;                                  // q~ [GQ][128] f32 (base-2 logits)
-  static constexpr int oCos = oQ + GQ * 128 * 4;                // cos (j w_i) [32][65] f32
-  static constexpr int oSin = oCos + kRStep * kOffStride * 4;   // sin (j w_i) [32][65] f32
-  static constexpr int oWarp = oSin + kRStep * kOffStride * 4;  // per-warp areas
+  static constexpr int oOff = oQ + GQ * 128 * 4;                // (cos, sin) (j w_i), pairs 2p, 2p + 1: [32][33] float4
+  static constexpr int oWarp = oOff + kRStep * kOffStride * 16;  // per-warp areas
   // per warp: turned query [GQ][64] float4 (q_i, q_{i+1}, q_{i+64}, q_{i+65}) for even i -> [GQ][32]
   // float4; key scale / zero of up to two groups [2][32] float4 x 2 (low / high channel pairs);
   // value scale (pre-scaled) / zero of the step's tokens [32][8] f32 x 2
@@ -94,8 +93,7 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
   constexpr int VP = 16 / VB;      // token pairs per value word
   extern __shared__ __align__(16) uint8_t smem[];
   float* sq = reinterpret_cast<float*>(smem + SM::oQ);
-  float* scos = reinterpret_cast<float*>(smem + SM::oCos);
-  float* ssin = reinterpret_cast<float*>(smem + SM::oSin);
+  float4* soff = reinterpret_cast<float4*>(smem + SM::oOff);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* wsm = smem + SM::oWarp + warp * SM::kWarpBytes;
   float4* wq = reinterpret_cast<float4*>(wsm + SM::wQ);    // [GQ][32]
@@ -121,11 +119,10 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
     const int h = idx >> 7, c = idx & 127;
     sq[idx] = h < gq ? h2f(a.q[(b * a.num_q_heads + static_cast<int64_t>(kvh) * gq + h) * kHeadDim + c]) * a.qscale : 0.f;
   }
-  for (int idx = threadIdx.x; idx < kRStep * 64; idx += kRW * 32) {
-    const int j = idx >> 6, i = idx & 63;
-    const float2 cs = roff[idx];
-    scos[j * kOffStride + i] = cs.x;
-    ssin[j * kOffStride + i] = cs.y;
+  for (int idx = threadIdx.x; idx < kRStep * 32; idx += kRW * 32) {
+    const int j = idx >> 5, p = idx & 31;
+    const float2 c0 = roff[j * 64 + 2 * p], c1 = roff[j * 64 + 2 * p + 1];
+    soff[j * kOffStride + p] = make_float4(c0.x, c0.y, c1.x, c1.y);
   }
   __syncthreads();
 
@@ -218,8 +215,7 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
         kw[4 * v + 3] = x.w;
       }
       const int gl = G >= kRStep ? 0 : lane / G;  // this token's group among the staged ones
-      const float* cj = scos + lane * kOffStride;
-      const float* sj = ssin + lane * kOffStride;
+      const float4* oj = soff + lane * kOffStride;
 #pragma unroll
       for (int p = 0; p < 32; ++p) {  // channel pairs 2p, 2p + 1 (low) and 64 + 2p, 65 + 2p (high)
         const int c = 2 * p, w = c / (2 * KP), slot = (c % (2 * KP)) / 2;
@@ -230,7 +226,8 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
         const float x0 = fmaf(lo.x, kl.x, kl.y), x1 = fmaf(lo.y, kl.z, kl.w);
         const float y0 = fmaf(hi.x, kh.x, kh.y), y1 = fmaf(hi.y, kh.z, kh.w);
         // R_j on pairs (c, c + 64) and (c + 1, c + 65)
-        const float cs0 = cj[c], sn0 = sj[c], cs1 = cj[c + 1], sn1 = sj[c + 1];
+        const float4 csn = oj[p];
+        const float cs0 = csn.x, sn0 = csn.y, cs1 = csn.z, sn1 = csn.w;
         const float r0 = fmaf(x0, cs0, -y0 * sn0), u0 = fmaf(x0, sn0, y0 * cs0);
         const float r1 = fmaf(x1, cs1, -y1 * sn1), u1 = fmaf(x1, sn1, y1 * cs1);
 #pragma unroll
@@ -341,12 +338,14 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       const float2* bt = rbase + static_cast<int64_t>(pos / kRStep) * 64;
       const int j = pos % kRStep;
       float r[4];
+      const float4 oj = soff[j * kOffStride + lane];  // in-step (cos, sin) of pairs 2 lane, 2 lane + 1
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int i = 2 * lane + e;
         const float2 cb = bt[i];
-        const float cs = fmaf(cb.x, scos[j * kOffStride + i], -cb.y * ssin[j * kOffStride + i]);
-        const float sn = fmaf(cb.y, scos[j * kOffStride + i], cb.x * ssin[j * kOffStride + i]);
+        const float co = e ? oj.z : oj.x, so = e ? oj.w : oj.y;
+        const float cs = fmaf(cb.x, co, -cb.y * so);
+        const float sn = fmaf(cb.y, co, cb.x * so);
         const float x = e ? lo.y : lo.x, y = e ? hi.y : hi.x;
         r[e] = fmaf(x, cs, -y * sn);      // channel i
         r[2 + e] = fmaf(x, sn, y * cs);   // channel i + 64
