@@ -370,26 +370,43 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
       const uint8_t* kp = kp_ring + ((t / kBlockTokens) % S::kKPSlots) * S::kKP + 512 * col_off;
       const uint4* sp = reinterpret_cast<const uint4*>(kp + 64 * qd);
       const uint4* zp = reinterpret_cast<const uint4*>(kp + 256 + 64 * qd);
+      // The hi and lo lanes of a column (r, r ^ 1: lanes L, L ^ 4) share the products q^ * sk: the hi
+      // lane makes both parts for m-blocks 0..3, the lo lane for 4..7, and each passes the other the
+      // parts it needs.
+      const int vb = lo_half ? 2 : 0;
       float bias = 0.f;
+      uint32_t hpk[4][2], lpk[4][2];  // hi / lo packs of this lane's m-blocks (local index mm)
 #pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4) {
+      for (int vv = 0; vv < 2; ++vv) {
+        const int v4 = vb + vv;
         const uint4 s4 = sp[v4], z4 = zp[v4];
         const uint32_t sw[4] = {s4.x, s4.y, s4.z, s4.w};
         const uint32_t zw[4] = {z4.x, z4.y, z4.z, z4.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int idx = 8 * v4 + 2 * k;  // = 4m + 2hh
-          const float2 qq = *reinterpret_cast<const float2*>(qn_row + 16 * (idx >> 2) + 8 * ((idx >> 1) & 1));
+          const int hh = k & 1, mm = 2 * vv + (k >> 1);  // m = 4 lo_half + mm
+          const float2 qq = *reinterpret_cast<const float2*>(qn_row + 16 * (2 * v4 + (k >> 1)) + 8 * hh);
           const float s0 = h2f(static_cast<uint16_t>(sw[k] & 0xffffu)), s1 = h2f(static_cast<uint16_t>(sw[k] >> 16));
           const float z0 = h2f(static_cast<uint16_t>(zw[k] & 0xffffu)), z1 = h2f(static_cast<uint16_t>(zw[k] >> 16));
           // 2-bit: the upper K half (channels 16m + 8 ..) carries 2^-4 against the subnormal codes
-          const float kf = (KB == 2 && (k & 1)) ? 0.0625f : 1.f;
-          bq[idx >> 2][(idx >> 1) & 1] =
-              pack_h2(split_part(qq.x * s0 * kf, lo_half), split_part(qq.y * s1 * kf, lo_half));
+          const float kf = (KB == 2 && hh) ? 0.0625f : 1.f;
+          const float x0 = qq.x * s0 * kf, x1 = qq.y * s1 * kf;
+          const float h0 = split_part(x0, false), h1 = split_part(x1, false);
+          hpk[mm][hh] = pack_h2(h0, h1);
+          lpk[mm][hh] = pack_h2(__fsub_rn(x0, h0), __fsub_rn(x1, h1));
           bias = fmaf(qq.x, z0, bias);
           bias = fmaf(qq.y, z1, bias);
         }
       }
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t recv = __shfl_xor_sync(kFull, lo_half ? hpk[mm][hh] : lpk[mm][hh], 4);
+          bq[mm][hh] = lo_half ? recv : hpk[mm][hh];
+          bq[4 + mm][hh] = lo_half ? lpk[mm][hh] : recv;
+        }
+      bias += __shfl_xor_sync(kFull, bias, 4);  // the two halves of the channels
       bias += __shfl_xor_sync(kFull, bias, 1);
       bias += __shfl_xor_sync(kFull, bias, 2);
       bias_col = __shfl_sync(kFull, bias, 8 * qd);  // lanes of column 2qd hold its bias
@@ -450,30 +467,36 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
     for (int u = 0; u < TS; ++u) {
       const float pa = __shfl_sync(kFull, p[u][0], la), pb = __shfl_sync(kFull, p[u][0], la + 4);
       const float pc = __shfl_sync(kFull, p[u][1], la), pd = __shfl_sync(kFull, p[u][1], la + 4);
+      // The hi lane of a column (r even) takes tokens 2qd, 2qd + 1 (the lower K half of the B
+      // fragment), the lo lane (r odd) tokens 2qd + 8, 2qd + 9; each makes both parts of its products
+      // and passes the partner lane (L ^ 4) the part that lane needs.
       // 2-bit: tokens 2qd + 8, + 9 (the upper K half) carry 2^-4 against the subnormal codes
       constexpr float kTf = VB == 2 ? 0.0625f : 1.f;
-      const float pcs = pc * kTf, pds = pd * kTf;
+      const float pe = lo_half ? pc : pa, po = lo_half ? pd : pb;  // probabilities of this lane's tokens
+      const float pes = lo_half ? pc * kTf : pa, pos = lo_half ? pd * kTf : pb;
       const uint16_t* vsh = reinterpret_cast<const uint16_t*>(st + S::oVS) + u * 16 * VPT;
       const uint16_t* vzh = reinterpret_cast<const uint16_t*>(st + S::oVZ) + u * 16 * VPT;
       uint32_t bp[NBV][2];
 #pragma unroll
       for (int nb = 0; nb < NBV; ++nb) {
         const int j = nb * VGB + col_off;
+        uint32_t hpk = 0u, lpk = 0u;  // both parts of this lane's two products (0 past the groups)
         if (VPT % VGB == 0 || j < VPT) {
-          const int t0 = 2 * qd * VPT + j;
-          const float s0 = h2f(vsh[t0]), s1 = h2f(vsh[t0 + VPT]), s2 = h2f(vsh[t0 + 8 * VPT]), s3 = h2f(vsh[t0 + 9 * VPT]);
-          const float z0 = h2f(vzh[t0]), z1 = h2f(vzh[t0 + VPT]), z2 = h2f(vzh[t0 + 8 * VPT]), z3 = h2f(vzh[t0 + 9 * VPT]);
-          bp[nb][0] = pack_h2(split_part(pa * s0, lo_half), split_part(pb * s1, lo_half));
-          bp[nb][1] = pack_h2(split_part(pcs * s2, lo_half), split_part(pds * s3, lo_half));
+          const int te = 2 * qd * VPT + j + (lo_half ? 8 * VPT : 0);  // this lane's first token
+          const float se = h2f(vsh[te]), so = h2f(vsh[te + VPT]);
+          const float ze = h2f(vzh[te]), zo = h2f(vzh[te + VPT]);
+          const float xe = pes * se, xo = pos * so;
+          const float he = split_part(xe, false), ho = split_part(xo, false);
+          hpk = pack_h2(he, ho);
+          lpk = pack_h2(__fsub_rn(xe, he), __fsub_rn(xo, ho));
           float z = zacc[nb];
-          z = fmaf(pa, fmaf(kCbar, s0, z0), z);
-          z = fmaf(pb, fmaf(kCbar, s1, z1), z);
-          z = fmaf(pc, fmaf(kCbar, s2, z2), z);
-          z = fmaf(pd, fmaf(kCbar, s3, z3), z);
+          z = fmaf(pe, fmaf(kCbar, se, ze), z);
+          z = fmaf(po, fmaf(kCbar, so, zo), z);
           zacc[nb] = z;
-        } else {
-          bp[nb][0] = bp[nb][1] = 0u;
         }
+        const uint32_t recv = __shfl_xor_sync(kFull, lo_half ? hpk : lpk, 4);
+        bp[nb][0] = lo_half ? recv : hpk;  // tokens 2qd, 2qd + 1: hi part here (hi lane), lo part from it
+        bp[nb][1] = lo_half ? lpk : recv;  // tokens 2qd + 8, + 9: lo part here (lo lane), hi part from it
       }
       // m-block m (channels 16m .. 16m+15) lies in value group (16m) / G, held by n-block group / VGB
       const uint8_t* vc = st + S::oVC + u * 256 * VB;
@@ -513,6 +536,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   l_run += __shfl_xor_sync(kFull, l_run, 16);
 #pragma unroll
   for (int j = 0; j < NBV; ++j) {
+    zacc[j] += __shfl_xor_sync(kFull, zacc[j], 4);  // the hi and lo lanes' tokens
     zacc[j] += __shfl_xor_sync(kFull, zacc[j], 1);
     zacc[j] += __shfl_xor_sync(kFull, zacc[j], 2);
   }
