@@ -1,0 +1,60 @@
+"""CPU checks of bench.py's accounting: the algorithmic byte counts behind every GB/s figure, the
+rank reduction's inputs, and the committed-counter lookup that fills roofline.traffic."""
+import json
+import os
+
+import numpy as np
+
+import bench
+from bit_kv_cache_prefill_b200 import inputs
+
+
+def test_decode_bytes_closed_form():
+    # llama2_7b_mha: 8 sequences x 32 heads x 32768 tokens, 2/2-bit, G = 32, R = 128
+    w = inputs.WORKLOADS["llama2_7b_mha"]
+    T, G, R = 32768, 32, 128
+    Q = (T - R) // G * G
+    per_unit = Q * 128 * 4 // 8 + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4
+    want = 8 * 32 * per_unit + 2 * 8 * 32 * 128 * 2
+    assert bench.decode_bytes(w, np.full(8, T)) == want
+    assert abs(want / 1e6 - 819) < 1  # 819 MB per call
+    # the sink adds the first token's fp16 key and value row once a group is quantized
+    assert bench.decode_bytes(w, np.full(8, T), sink=1) == want + 8 * 32 * 512
+    assert bench.decode_bytes(w, np.full(8, 100), sink=1) == bench.decode_bytes(w, np.full(8, 100))
+
+
+def test_prefill_bytes_closed_form():
+    w = inputs.WORKLOADS["million_token"]
+    T, G, R = 1 << 20, 128, 128
+    Q = (T - R) // G * G
+    per_unit = T * 128 * 4 + Q * 128 * 4 // 8 + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4
+    assert bench.prefill_bytes(w, np.array([T])) == 8 * per_unit
+    assert bench.prefill_bytes(w, np.array([T]), sink=1) == 8 * (per_unit + 512)
+
+
+def test_traffic_counters_match_their_sources():
+    # every committed counter names its kernel sources and their hash; a record is used only while
+    # the hash matches, and it scales to another batch by the units processed
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles",
+                        "decode_traffic_counters.txt")
+    entries = json.load(open(path))
+    kinds = {e.get("kind", "decode") for e in entries.values()}
+    assert {"decode", "prefill"} <= kinds
+    w = inputs.WORKLOADS["llama2_7b_mha"]
+    for e in entries.values():
+        kind = e.get("kind", "decode")
+        got = bench.measured_traffic(w, e["layout"], kind)
+        assert got is not None, f"{kind} counters are stale (sources changed since the capture)"
+        units = w.batch * w.num_kv_heads
+        assert got == round((e["dram_read_bytes"] + e["dram_write_bytes"]) * units / e["capture_units"])
+    # the DRAM bytes of the capture stay within a few percent of the algorithmic bytes
+    dec = bench.measured_traffic(w, 1, "decode")
+    assert 1.0 < dec / bench.decode_bytes(w, w.seq_lens()) < 1.06
+    pre = bench.measured_traffic(w, 1, "prefill")
+    assert 0.95 < pre / bench.prefill_bytes(w, w.seq_lens()) < 1.02
+
+
+def test_traffic_lookup_is_none_for_other_layouts_and_kernels():
+    w = inputs.WORKLOADS["llama2_7b_mha"]
+    assert bench.measured_traffic(w, 2, "decode") is None
+    assert bench.measured_traffic(inputs.WORKLOADS["llama3_8b_gqa"], 1, "decode") is None
