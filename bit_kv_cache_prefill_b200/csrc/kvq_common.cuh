@@ -119,12 +119,14 @@ __device__ __forceinline__ void wht128_16lanes(float x[8]) {
   const int sub = threadIdx.x & 15;
 #pragma unroll
   for (int d = 1; d < 16; d <<= 1) {  // element stride 8*d
-    const bool upper = (sub & d) != 0;
+    // lower lane holds a (first of the pair) and makes a + b; upper lane holds b and makes a - b.
+    // fma(+-1, x, other) rounds the exact sum once, the same as the IEEE add / subtract (signed
+    // zeros included), in one instruction.
+    const float sgn = (sub & d) != 0 ? -1.f : 1.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float other = __shfl_xor_sync(0xffffffffu, x[i], d);
-      // lower lane holds a (first of the pair), upper lane holds b
-      x[i] = upper ? __fsub_rn(other, x[i]) : __fadd_rn(x[i], other);
+      x[i] = __fmaf_rn(sgn, x[i], other);
     }
   }
   const float s = inv_sqrt128();
