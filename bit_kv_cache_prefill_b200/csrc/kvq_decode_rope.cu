@@ -149,8 +149,9 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
     const int t = t0 + lane;
     const bool valid = t < qend && !(a.sink && t == 0);
     // key scale / zero of the step's groups: wkp[g][half][p] = (s, z) of channels 2p, 2p + 1
-    // (half 0) or 64 + 2p, 65 + 2p (half 1), fp16 scales pre-multiplied by 2^(24 - bit) of their
-    // code position so that a subnormal code times the scale is code * s
+    // (half 0) or 64 + 2p, 65 + 2p (half 1), fp16 scales pre-multiplied by 2^(24 - (bit & 7)) of
+    // their code position (code_pair reads a code at bit & 7) so that the subnormal code times the
+    // scale is code * s
     const int g0 = t0 / G;
     if (g0 != kp_group) {
       kp_group = g0;
@@ -173,8 +174,8 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
         }
       }
     }
-    // value scale / zero of the step's tokens: wvs pre-multiplied by 2^(24 - bit) of the token's
-    // position in its value word (token pair slot (t % 128 / 2) % VP, bit VB * slot)
+    // value scale / zero of the step's tokens: wvs pre-multiplied by 2^(24 - (bit & 7)) of the
+    // token's position in its value word (token pair slot (t % 128 / 2) % VP, bit VB * slot)
     for (int idx = lane; idx < kRStep * VPT; idx += 32) {
       const int jj = idx / VPT, g = idx % VPT;
       const int tt = t0 + jj;
