@@ -60,15 +60,6 @@ __device__ __forceinline__ QuantParams make_params(uint32_t kmin, uint32_t kmax,
   return p;
 }
 
-__device__ __forceinline__ uint32_t code_of(uint16_t x, const QuantParams& p, int bits) {
-  if (p.zero_scale) return 0u;
-  const float v = __fmul_rn(__fsub_rn(h2f(x), p.zf), p.inv);
-  int c = __float2int_rn(v);  // round half to even
-  const int top = (1 << bits) - 1;
-  c = c < 0 ? 0 : (c > top ? top : c);
-  return static_cast<uint32_t>(c);
-}
-
 // --- tile v1 layout ----------------------------------------------------------------------------------
 // Word index `widx` of a tile (0 .. 64*bits-1) -> (lane, logical word w).
 __device__ __forceinline__ void widx_to_lane_word(int widx, int* lane, int* w) {

@@ -63,41 +63,10 @@ template <int SOFF, int GOFF>
 __device__ __forceinline__ void cp_async16_at(uint32_t saddr, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0+%2], [%1+%3], 16;\n" ::"r"(saddr), "l"(gmem), "n"(SOFF), "n"(GOFF));
 }
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
-}
-
-// Load 2*VPT consecutive fp16 (aligned to 4*VPT bytes) as floats.
-template <int VPT>
-__device__ __forceinline__ void load_halves(const uint8_t* p, float (&out)[2 * VPT]) {
-  uint32_t w[VPT];
-  if constexpr (VPT == 1) {
-    w[0] = *reinterpret_cast<const uint32_t*>(p);
-  } else if constexpr (VPT == 2) {
-    const uint2 v = *reinterpret_cast<const uint2*>(p);
-    w[0] = v.x;
-    w[1] = v.y;
-  } else {
-#pragma unroll
-    for (int i = 0; i < VPT / 4; ++i) {
-      const uint4 v = reinterpret_cast<const uint4*>(p)[i];
-      w[4 * i] = v.x;
-      w[4 * i + 1] = v.y;
-      w[4 * i + 2] = v.z;
-      w[4 * i + 3] = v.w;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    out[2 * i] = h2f(static_cast<uint16_t>(w[i] & 0xffffu));
-    out[2 * i + 1] = h2f(static_cast<uint16_t>(w[i] >> 16));
-  }
 }
 
 // Per-warp pipeline: a ring of kStages stages, each holding one step of TS 16-token tiles (codes
