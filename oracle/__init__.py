@@ -53,13 +53,14 @@ class _CConfig(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32), ("value_bits", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("residual", ctypes.c_int32), ("hadamard", ctypes.c_int32),
         ("layout", ctypes.c_int32), ("sink", ctypes.c_int32), ("rope_theta", ctypes.c_float),
-        ("capacity", ctypes.c_int64),
+        ("outliers", ctypes.c_int32), ("capacity", ctypes.c_int64),
     ]
 
 
 class _CCache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero", "k_res", "v_res", "seq_len")]
+                ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero", "k_res", "v_res", "seq_len",
+                 "k_out_ch", "k_out_val", "v_out_ch", "v_out_val")]
 
 
 def _declare(L: ctypes.CDLL) -> None:
@@ -103,11 +104,12 @@ class Config:
     layout: int = 1  # 1 = tile v1 (mma fragment order), 2 = rows v2 (token rows of keys, channel rows of values)
     sink: int = 0    # 1: the first token stays in fp16 (an extra row after the ring)
     rope_theta: float = 0.0  # > 0: keys are cached before RoPE and decode applies it (0: off)
+    outliers: int = 0  # 1: each quantized token's largest-magnitude key / value entry stays fp16
 
     def c(self) -> _CConfig:
         return _CConfig(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.key_bits,
                         self.value_bits, self.group_size, self.residual, self.hadamard, self.layout, self.sink,
-                        self.rope_theta, self.capacity)
+                        self.rope_theta, self.outliers, self.capacity)
 
 
 class Cache:
@@ -129,11 +131,17 @@ class Cache:
         self.k_res = np.zeros((B, H, ring, 128), np.uint16)
         self.v_res = np.zeros((B, H, ring, 128), np.uint16)
         self.seq_len = np.zeros((B,), np.int64)
+        # sparse outliers (one per quantized token and tensor): channel (0xffff: none) and fp16 value
+        self.k_out_ch = np.full((B, H, cap), 0xFFFF, np.uint16)
+        self.k_out_val = np.zeros((B, H, cap), np.uint16)
+        self.v_out_ch = np.full((B, H, cap), 0xFFFF, np.uint16)
+        self.v_out_val = np.zeros((B, H, cap), np.uint16)
 
     def c(self) -> _CCache:
         return _CCache(*(a.ctypes.data for a in (self.k_codes, self.v_codes, self.k_scale, self.k_zero,
                                                  self.v_scale, self.v_zero, self.k_res, self.v_res,
-                                                 self.seq_len)))
+                                                 self.seq_len, self.k_out_ch, self.k_out_val, self.v_out_ch,
+                                                 self.v_out_val)))
 
 
 def _u16(a: np.ndarray) -> np.ndarray:

@@ -46,6 +46,13 @@
 //      t * theta^(-i/64), k'[i] = k[i] cos - k[i+64] sin, k'[i+64] = k[i] sin + k[i+64] cos, in
 //      fp64. The query is taken as given (rotated at its own position by the caller). RoPE and the
 //      Hadamard option exclude each other.
+//  R12 optional dense-and-sparse outliers (outliers = 1; KVQuant review, Method: per-vector
+//      thresholds move about 1% of the entries into an fp16 sparse store). Per quantized token and
+//      tensor, the entry of largest magnitude (ties: the lowest channel) is that vector's outlier,
+//      1 of 128 entries. It is kept exactly in fp16 (channel and value per token), left out of the
+//      min/max of its key group (per channel) or value group (per token), and coded 0; dequantization
+//      puts the fp16 value back. A key channel whose entries in a group are all outliers gets scale
+//      and zero 0. The sink token (R10) has no outlier; the fp16 window needs none.
 //
 // Build: g++ -O2 -std=c++17 -ffp-contract=off -fno-fast-math -fPIC -shared (x86-64 SSE scalar fp32).
 
@@ -158,9 +165,19 @@ struct GroupQ {
   uint16_t scale, zero;
 };
 
-GroupQ quantize_group(const uint16_t* x, int n, int stride, int bits, uint8_t* codes, int code_stride) {
-  uint16_t mn = x[0], mx = x[0];
-  for (int i = 1; i < n; ++i) {
+// skip (optional): entries with skip[i * skip_stride] != 0 stay out of the min / max and get code 0
+// (reading R12); a group with every entry skipped gets scale and zero 0.
+GroupQ quantize_group(const uint16_t* x, int n, int stride, int bits, uint8_t* codes, int code_stride,
+                      const uint8_t* skip = nullptr, int skip_stride = 0) {
+  int first = 0;
+  while (skip && first < n && skip[first * skip_stride]) ++first;
+  if (first == n) {
+    for (int i = 0; i < n; ++i) codes[i * code_stride] = 0;
+    return GroupQ{0, 0};
+  }
+  uint16_t mn = x[first * stride], mx = x[first * stride];
+  for (int i = first + 1; i < n; ++i) {
+    if (skip && skip[i * skip_stride]) continue;
     mn = hmin(mn, x[i * stride]);
     mx = hmax(mx, x[i * stride]);
   }
@@ -177,6 +194,10 @@ GroupQ quantize_group(const uint16_t* x, int n, int stride, int bits, uint8_t* c
   const float zf = half_to_float(mn);
   const int top = (1 << bits) - 1;
   for (int i = 0; i < n; ++i) {
+    if (skip && skip[i * skip_stride]) {
+      codes[i * code_stride] = 0;
+      continue;
+    }
     const float d = half_to_float(x[i * stride]) - zf;
     const float v = d * inv;
     float r = std::nearbyint(v);  // default rounding mode: nearest, ties to even
@@ -265,6 +286,7 @@ typedef struct {
   int32_t key_bits, value_bits, group_size, residual, hadamard, layout;  // layout: 1 = tile v1, 2 = rows v2
   int32_t sink;        // 1: the first token stays in fp16 (reading R10)
   float rope_theta;    // > 0: keys are cached before RoPE, decode applies it (reading R11); 0: off
+  int32_t outliers;    // 1: each quantized token's largest-magnitude key and value entry stay fp16 (R12)
   int64_t capacity;
 } kvq_ref_config;
 
@@ -278,6 +300,10 @@ typedef struct {
   uint16_t* k_res;    // [B][Hkv][R+G+sink][128] ring, fp16 (row R+G: the first token when sink is on)
   uint16_t* v_res;    // same
   int64_t* seq_len;   // [B]
+  uint16_t* k_out_ch;   // [B][Hkv][Cap] channel of the token's key outlier (0xffff: none); reading R12
+  uint16_t* k_out_val;  // [B][Hkv][Cap] its fp16 value
+  uint16_t* v_out_ch;   // same for values
+  uint16_t* v_out_val;
 } kvq_ref_cache;
 
 enum { REF_OK = 0, REF_ERR_ARG = -1, REF_ERR_CAPACITY = -3 };
@@ -295,6 +321,7 @@ static int check_config(const kvq_ref_config* c) {
   if (c->sink != 0 && c->sink != 1) return REF_ERR_ARG;
   if (!(c->rope_theta >= 0.0f) || !std::isfinite(c->rope_theta)) return REF_ERR_ARG;
   if (c->rope_theta > 0.0f && c->hadamard) return REF_ERR_ARG;
+  if (c->outliers != 0 && c->outliers != 1) return REF_ERR_ARG;
   return REF_OK;
 }
 
@@ -343,6 +370,15 @@ static Dims dims(const kvq_ref_config* c) {
   return d;
 }
 
+// The channel of a token vector's largest-magnitude entry (reading R12): binary16 magnitudes order
+// like the integers of their low 15 bits (non-NaN); ties go to the lowest channel.
+static int largest_entry(const uint16_t* x) {
+  int best = 0;
+  for (int ch = 1; ch < 128; ++ch)
+    if ((x[ch] & 0x7fffu) > (x[best] & 0x7fffu)) best = ch;
+  return best;
+}
+
 // Quantize tokens [t0, t0 + G) of key unit `kt` (fp16 [T][128], already rotated if enabled) into key
 // group t0 / G, and the same tokens of value unit `vt` per token.
 // With the sink on (reading R10) the first token of the sequence stays out of the quantizer: key group
@@ -353,12 +389,31 @@ static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, i
   const Dims d = dims(c);
   const int G = c->group_size;
   const int skip = (c->sink && t0 == 0) ? 1 : 0;  // tokens at the start of the span kept out
-  // Keys: per channel over the G (or G - 1) tokens of the group.
+  // Outliers (reading R12): each token's largest-magnitude key entry and value entry.
+  std::vector<uint8_t> kout(static_cast<size_t>(G) * 128, 0), vout(static_cast<size_t>(G) * 128, 0);
+  if (c->outliers) {
+    for (int i = 0; i < G; ++i) {
+      const int64_t at = unit * c->capacity + t0 + i;
+      if (i < skip) {  // the sink token is fp16 as a whole
+        cache->k_out_ch[at] = cache->v_out_ch[at] = 0xffffu;
+        cache->k_out_val[at] = cache->v_out_val[at] = 0;
+        continue;
+      }
+      const int kch = largest_entry(kt + i * k_ld), vch = largest_entry(vt + i * v_ld);
+      kout[i * 128 + kch] = 1;
+      vout[i * 128 + vch] = 1;
+      cache->k_out_ch[at] = static_cast<uint16_t>(kch);
+      cache->k_out_val[at] = kt[i * k_ld + kch];
+      cache->v_out_ch[at] = static_cast<uint16_t>(vch);
+      cache->v_out_val[at] = vt[i * v_ld + vch];
+    }
+  }
+  // Keys: per channel over the G (or G - 1) tokens of the group, outliers left out.
   std::vector<uint8_t> kc(static_cast<size_t>(G) * 128, 0);
   const int64_t g = t0 / G;
   for (int ch = 0; ch < 128; ++ch) {
     GroupQ q = quantize_group(kt + skip * k_ld + ch, G - skip, static_cast<int>(k_ld), c->key_bits,
-                              kc.data() + skip * 128 + ch, 128);
+                              kc.data() + skip * 128 + ch, 128, kout.data() + skip * 128 + ch, 128);
     const int pos = key_param_index(c, ch);
     cache->k_scale[(unit * d.groups + g) * 128 + pos] = q.scale;
     cache->k_zero[(unit * d.groups + g) * 128 + pos] = q.zero;
@@ -383,7 +438,8 @@ static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, i
       if (i < skip)
         std::memset(vc.data() + j * G, 0, G);
       else
-        q = quantize_group(vt + i * v_ld + j * G, G, 1, c->value_bits, vc.data() + j * G, 1);
+        q = quantize_group(vt + i * v_ld + j * G, G, 1, c->value_bits, vc.data() + j * G, 1,
+                           vout.data() + i * 128 + j * G, 1);
       cache->v_scale[(unit * c->capacity + t) * d.vpt + j] = q.scale;
       cache->v_zero[(unit * c->capacity + t) * d.vpt + j] = q.zero;
     }
@@ -526,6 +582,10 @@ static void key_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t
     const double z = half_to_float(cache->k_zero[(unit * d.groups + g) * 128 + pos]);
     out[ch] = static_cast<double>(code) * s + z;
   }
+  if (c->outliers) {  // the token's fp16 outlier replaces its entry (reading R12)
+    const uint16_t ch = cache->k_out_ch[unit * c->capacity + t];
+    if (ch < 128) out[ch] = half_to_float(cache->k_out_val[unit * c->capacity + t]);
+  }
 }
 
 static void value_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t unit, int64_t t, int64_t Q, double* out) {
@@ -546,6 +606,10 @@ static void value_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64
     const double s = half_to_float(cache->v_scale[(unit * c->capacity + t) * d.vpt + j]);
     const double z = half_to_float(cache->v_zero[(unit * c->capacity + t) * d.vpt + j]);
     out[ch] = static_cast<double>(code) * s + z;
+  }
+  if (c->outliers) {  // the token's fp16 outlier replaces its entry (reading R12)
+    const uint16_t ch = cache->v_out_ch[unit * c->capacity + t];
+    if (ch < 128) out[ch] = half_to_float(cache->v_out_val[unit * c->capacity + t]);
   }
 }
 

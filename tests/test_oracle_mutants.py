@@ -16,8 +16,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 # (name, text to replace, replacement, pins expected to notice)
 MUTANTS = [
     ("dropped_key_zero_point",
-     "    out[ch] = static_cast<double>(code) * s + z;\n  }\n}\n\nstatic void value_row",
-     "    out[ch] = static_cast<double>(code) * s + 0.0 * z;\n  }\n}\n\nstatic void value_row",
+     "    out[ch] = static_cast<double>(code) * s + z;\n  }\n  if (c->outliers) {  // the token's fp16 outlier replaces its entry (reading R12)\n    const uint16_t ch = cache->k_out_ch",
+     "    out[ch] = static_cast<double>(code) * s + 0.0 * z;\n  }\n  if (c->outliers) {  // the token's fp16 outlier replaces its entry (reading R12)\n    const uint16_t ch = cache->k_out_ch",
      ["test_quantized_attention_equals_library_attention_on_dequantized_cache"]),
     ("hadamard_sign_flip",
      "        x[i] = a + b;\n        x[i + h] = a - b;\n      }\n  const float s",
@@ -68,6 +68,18 @@ MUTANTS = [
     ("rope_position_off_by_one",
      "    if (rope) rope_rotate(row, t, omega);", "    if (rope) rope_rotate(row, t + 1, omega);",
      ["test_rope_without_quantization_equals_library_attention_on_rotated_keys", "test_rope_relative_position"]),
+    ("outliers_kept_in_key_statistics",
+     "kc.data() + skip * 128 + ch, 128, kout.data() + skip * 128 + ch, 128);",
+     "kc.data() + skip * 128 + ch, 128);",
+     ["test_outliers_left_out_of_group_statistics"]),
+    ("value_outlier_not_restored_in_decode",
+     "    if (ch < 128) out[ch] = half_to_float(cache->v_out_val[unit * c->capacity + t]);",
+     "    (void)ch;",
+     ["test_outliers_dequantized_attention_equals_library_attention"]),
+    ("outlier_ties_to_the_highest_channel",
+     "    if ((x[ch] & 0x7fffu) > (x[best] & 0x7fffu)) best = ch;",
+     "    if ((x[ch] & 0x7fffu) >= (x[best] & 0x7fffu)) best = ch;",
+     ["test_outliers_are_each_tokens_largest_entry_kept_in_fp16"]),
     ("value_group_index_off",
      "    const int j = ch / c->group_size;", "    const int j = (ch / c->group_size + 1) % d.vpt;",
      ["test_quantized_attention_equals_library_attention_on_dequantized_cache"]),
@@ -99,6 +111,8 @@ def _run_pin(fn_name, mod):
         "test_sink_first_token_left_out_of_group_zero": [dict(layout=1), dict(layout=2)],
         "test_sink_dominant_first_token_returns_its_fp16_value": [dict(layout=1), dict(layout=2)],
         "test_rope_without_quantization_equals_library_attention_on_rotated_keys": [dict(theta=10000.0)],
+        "test_outliers_left_out_of_group_statistics": [dict(layout=1)],
+        "test_outliers_are_each_tokens_largest_entry_kept_in_fp16": [dict(layout=1)],
     }.get(fn_name, [dict()])
     for kw in params:
         fn(mod, **kw)

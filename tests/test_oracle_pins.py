@@ -681,3 +681,120 @@ def test_rope_relative_position(oracle_mod):
     assert abs(out_m[0, 0, 0] - p @ (np.arange(T) / 8.0)) < 1e-9
     # the attention peaks at position m, where the key is turned exactly like the query
     assert int(np.argmax(s)) == m
+
+
+# ---- dense-and-sparse outliers (KVQuant review, Method: per-vector thresholds keep about 1% of the
+# entries in an fp16 sparse store; reading R12) ----------------------------------------------------------
+def _total_order_key(h):
+    """IEEE total order of binary16 bit patterns (-0 < +0), as signed integers; numpy only."""
+    h = h.astype(np.int32)
+    return np.where(h & 0x8000, -(h & 0x7FFF) - 1, h)
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_outliers_are_each_tokens_largest_entry_kept_in_fp16(oracle_mod, layout):
+    B, T, Hkv, Hq, G, R = 1, 300, 2, 2, 32, 32
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=384, layout=layout)
+    cfg.outliers = 1
+    k, v, q = _inputs(B, T, Hkv, Hq, 81)
+    k[0, 17, 1, 40] = -k[0, 17, 1, 40:41].max() - 100.0   # a tie-free negative outlier
+    v[0, 20, 0, 3] = v[0, 20, 0, 9] = 50.0                 # a tie: the lower channel wins
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [T])
+    Q = (T - R) // G * G
+    for h in range(Hkv):
+        for name, x in (("k", k), ("v", v)):
+            mag = x[0, :Q, h].view(np.uint16) & 0x7FFF
+            want = mag.argmax(axis=1)  # numpy's argmax takes the first of equal maxima
+            ch = getattr(cache, f"{name}_out_ch")[0, h, :Q]
+            val = getattr(cache, f"{name}_out_val")[0, h, :Q]
+            assert np.array_equal(ch, want)
+            assert np.array_equal(val, x[0, np.arange(Q), h, want].view(np.uint16))
+            assert np.all(getattr(cache, f"{name}_out_ch")[0, h, Q:] == 0xFFFF)  # window tokens: none
+    assert cache.k_out_ch[0, 1, 17] == 40 and cache.v_out_ch[0, 0, 20] == 3
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_outliers_left_out_of_group_statistics(oracle_mod, layout):
+    # every key group's per-channel min / max and every value group's per-token min / max run over
+    # the non-outlier entries only; a key channel whose entries are all outliers has scale and zero 0
+    B, T, Hkv, Hq, G, R, kb, vb = 1, 200, 1, 1, 32, 8, 2, 4
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, kb, vb, G, R, 0, cap=256, layout=layout)
+    cfg.outliers = 1
+    k, v, q = _inputs(B, T, Hkv, Hq, 82)
+    k[0, :64, 0, 5] = 1000.0  # channel 5 is every token's outlier in the first two groups
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [T])
+    Q = (T - R) // G * G
+    kb16 = k[0, :Q, 0].view(np.uint16)
+    kout = np.zeros((Q, 128), bool)
+    kout[np.arange(Q), cache.k_out_ch[0, 0, :Q]] = True
+    for g in range(Q // G):
+        for c in range(128):
+            keep = ~kout[g * G:(g + 1) * G, c]
+            pos = oracle_mod.key_param_pos(c) if layout == 1 else c
+            s16, z16 = cache.k_scale[0, 0, g, pos], cache.k_zero[0, 0, g, pos]
+            if not keep.any():
+                assert s16 == 0 and z16 == 0
+                continue
+            col = kb16[g * G:(g + 1) * G, c][keep]
+            mn, mx = col[np.argmin(_total_order_key(col))], col[np.argmax(_total_order_key(col))]
+            assert z16 == mn
+            s32 = np.float32((np.float32(mx.view(np.float16)) - np.float32(mn.view(np.float16))) / np.float32(3))
+            assert s16 == np.float16(s32).view(np.uint16)
+    assert np.all(cache.k_scale[0, 0, :2, 5 if layout == 2 else oracle_mod.key_param_pos(5)] == 0)
+    vb16 = v[0, :Q, 0].view(np.uint16)
+    for t in range(Q):
+        for j in range(128 // G):
+            row = vb16[t, j * G:(j + 1) * G]
+            keep = np.arange(j * G, (j + 1) * G) != cache.v_out_ch[0, 0, t]
+            col = row[keep]
+            assert cache.v_zero[0, 0, t, j] == col[np.argmin(_total_order_key(col))]
+
+
+def test_outliers_dequantized_attention_equals_library_attention(oracle_mod):
+    # the dense codes dequantized, each token's outlier put back, then plain attention = the oracle
+    B, Hkv, Hq, G, R = 1, 2, 4, 32, 32
+    T = 301
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=320)
+    cfg.outliers = 1
+    k, v, q = _inputs(B, T, Hkv, Hq, 83)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [T])
+    out = oracle_mod.decode(cfg, cache, q, 1 / math.sqrt(128))
+    Q = (T - R) // G * G
+    ring = R + G
+    K = np.zeros((Hkv, T, 128))
+    V = np.zeros((Hkv, T, 128))
+    for h in range(Hkv):
+        for t in range(T):
+            if t < Q:
+                K[h, t] = _unpack_key(oracle_mod, cfg, cache, 0, h, t)
+                V[h, t] = _unpack_value(oracle_mod, cfg, cache, 0, h, t)
+                K[h, t, cache.k_out_ch[0, h, t]] = cache.k_out_val[0, h, t].view(np.float16)
+                V[h, t, cache.v_out_ch[0, h, t]] = cache.v_out_val[0, h, t].view(np.float16)
+            else:
+                K[h, t] = cache.k_res[0, h, t % ring].view(np.float16)
+                V[h, t] = cache.v_res[0, h, t % ring].view(np.float16)
+    ref = _sdpa(q.astype(np.float64), K[None], V[None], 1 / math.sqrt(128))
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+    # and the outliers are exact: the largest entries of the inputs come back bit for bit
+    assert np.array_equal(K[0, np.arange(Q), cache.k_out_ch[0, 0, :Q]].astype(np.float16),
+                          k[0, np.arange(Q), 0, cache.k_out_ch[0, 0, :Q]])
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_outliers_streaming_equals_bulk(oracle_mod, layout):
+    B, Hkv, Hq, G, R = 1, 1, 2, 32, 32
+    T0, n = 70, 3 * 32 + 5
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=256, layout=layout)
+    cfg.outliers = 1
+    k, v, q = _inputs(B, T0 + n, Hkv, Hq, 84)
+    bulk = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, bulk, k, v, [T0 + n])
+    stream = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, stream, k[:, :T0], v[:, :T0], [T0])
+    for s in range(n):
+        oracle_mod.append_token(cfg, stream, k[:, T0 + s], v[:, T0 + s])
+    for name in ("k_codes", "k_scale", "k_zero", "v_scale", "v_zero", "k_out_ch", "k_out_val", "v_out_ch", "v_out_val"):
+        assert np.array_equal(getattr(stream, name), getattr(bulk, name)), name
