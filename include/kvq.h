@@ -49,13 +49,14 @@ typedef enum {
 } kvq_status;
 
 /* Packed layouts (see kvq_cache below): "tile v1" feeds warp-level mma fragments, "rows v2" feeds
- * the tcgen05 tensor cores (one token's key codes / one channel's value codes per row). */
+ * the tcgen05 tensor cores and the pre-RoPE decode (one token's key codes / one channel's value codes
+ * per row). */
 #define KVQ_LAYOUT_TILE_V1 1
 #define KVQ_LAYOUT_ROWS_V2 2
 
 /* Problem definition. Requirements checked by every entry point:
  *   batch >= 1; num_kv_heads >= 1; num_q_heads a multiple of num_kv_heads with
- *   num_q_heads / num_kv_heads in {1, 2, 4}; head_dim == 128;
+ *   num_q_heads / num_kv_heads in {1, 2, 3, 4}; head_dim == 128;
  *   key_bits, value_bits in {2, 4};
  *   group_size G in {16, 32, 64, 128} (a multiple of the 16-token tile and a divisor of 128);
  *   residual R >= 0 (tokens kept in FP16 beyond the last full group; 0 <= R <= 4096);
@@ -192,8 +193,10 @@ kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, size_t* bytes);
  * q: device fp16 [batch][num_q_heads][128]; out: device fp16 [batch][num_q_heads][128]
  * (16-byte aligned). Query head h attends to KV head h / (num_q_heads / num_kv_heads) over all
  * T_b tokens: out = softmax(sm_scale * q~ . K^) V^ with K^, V^ the dequantized cache
- * (code * scale + zero; FP16 residual as stored) and q~ = H q / sqrt(128) when hadamard is set.
- * A sequence with T_b == 0 gets a zero output. The caller appends the current token first.
+ * (code * scale + zero; FP16 residual as stored; with sink = 1 token 0 from its fp16 row; with
+ * rope_theta > 0 every key turned at its position as described above) and q~ = H q / sqrt(128)
+ * when hadamard is set. A sequence with T_b == 0 gets a zero output. The caller appends the current
+ * token first.
  * workspace: device, 256-byte aligned, at least kvq_decode_workspace_bytes(cfg) bytes; it is
  * scratch for split partials and may be reused after the stream passes this call.
  * Errors: KVQ_ERR_WORKSPACE, KVQ_ERR_INVALID_ARG (non-finite or non-positive sm_scale, nulls,
