@@ -469,7 +469,8 @@ def main():
                     "frac": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9 / peak, 4),
                     "traffic": measured_traffic(w0, args.layout, "prefill"),
                     "kernel": "prefill_block_kernel (one kvq_quantize_prefill call)"},
-        "gpu_launches": 4 * args.steps,
+        # per step: append + length bump, then the decode split kernel + combine (+ the RoPE angle tables)
+        "gpu_launches": (5 if args.rope > 0 else 4) * args.steps,
         "clocks": clocks.summary(),
     }
     if e2e is not None:
