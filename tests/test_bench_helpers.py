@@ -85,4 +85,5 @@ def test_flush_steps_and_scanned_tokens():
 def test_oracle_sample_reports_one_thread_time():
     res = bench.oracle_decode_sample(inputs.WORKLOADS["tiny"], budget_s=0.05, single_thread_s=0.01)
     assert res.gbs > 0 and res.threads >= 1 and res.single_thread_gbs > 0 and "one thread" in res.sample
+    assert res.prefill_gbs > 0
     assert bench.oracle_decode_sample(inputs.WORKLOADS["tiny"], budget_s=0.01).single_thread_gbs is None
