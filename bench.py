@@ -302,7 +302,7 @@ def run_reference(args, w):
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
         res = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink, rope=args.rope)
-        cores, sample = res.threads, res.sample
+        cores, sample, pre_gbs = res.threads, res.sample, res.prefill_gbs
         if i >= args.warmup:
             per_step.append(res.gbs)
     value = statistics.mean(per_step)
@@ -313,7 +313,7 @@ def run_reference(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, args, step_bytes),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
-                         "cpu_model": cpu_model()},
+                         "prefill_value": round(pre_gbs, 4), "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
