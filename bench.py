@@ -90,6 +90,16 @@ def kv_tokens(w: inputs.Workload, lens: np.ndarray) -> int:
     return int(np.asarray(lens, np.int64).sum()) * w.num_kv_heads
 
 
+def input_digest(*arrays) -> str:
+    """SHA-256 of the arrays' bytes in order (C-contiguous numpy arrays): names the exact synthetic
+    inputs a run used."""
+    import hashlib
+    h = hashlib.sha256()
+    for a in arrays:
+        h.update(memoryview(np.ascontiguousarray(a)))
+    return h.hexdigest()
+
+
 def cpu_model() -> Optional[str]:
     try:
         with open("/proc/cpuinfo") as f:
@@ -373,6 +383,7 @@ def main():
     w = w0.scaled(appends=n_app)
     lens0 = w0.seq_lens()
     k, v, _ = inputs.full_kv(w0)  # CPU, seeded
+    digest = input_digest(k.numpy(), v.numpy(), inputs.query(w0).numpy())
     kd, vd = k.cuda(), v.cuda()
     del k, v
     cap = w.capacity()
@@ -532,6 +543,7 @@ def main():
         # per step: append + length bump, then the decode split kernel + combine (+ the RoPE angle tables)
         "gpu_launches": (5 if args.rope > 0 else 4) * args.steps,
         "clocks": clocks.summary(),
+        "input_sha256": digest,  # prefill K, V (fp16 [B][T][Hkv][128], zero past each length) and q
     }
     if e2e is not None:
         line["e2e"] = e2e
