@@ -115,3 +115,10 @@ def test_input_digest_names_the_inputs():
     assert bench.input_digest(k2.numpy(), v2.numpy(), inputs.query(w).numpy()) == d1
     v2[0, 0, 0, 0] += 1
     assert bench.input_digest(k2.numpy(), v2.numpy(), inputs.query(w).numpy()) != d1
+
+
+def test_append_summary():
+    assert bench.append_summary([], []) is None
+    got = bench.append_summary([0.004, 0.010, 0.006], [False, True, False])
+    assert got == {"n": 3, "mean_us": 6.67, "flush_us": 10.0, "n_flush": 1, "noflush_us": 5.0}
+    assert bench.append_summary([0.004], [False])["flush_us"] is None
