@@ -894,12 +894,15 @@ def test_paged_shuffled_pool_gathers_to_the_contiguous_cache(oracle_mod, layout,
     assert np.array_equal(out_c, out_p)
 
 
+@pytest.mark.parametrize("outliers,sink", [(0, 0), (1, 1)])
 @pytest.mark.parametrize("layout", [1, 2])
-def test_paged_streaming_with_pages_allocated_on_demand(oracle_mod, layout):
+def test_paged_streaming_with_pages_allocated_on_demand(oracle_mod, layout, outliers, sink):
     # the caller hands out a page only when the quantized part first reaches it; streaming then
-    # equals a bulk prefill into the same pages, and a missing page is an argument error
+    # equals a bulk prefill into the same pages (outlier words and the sink row included), and a
+    # missing page is an argument error
     B, Hkv, Hq, G, R, P, cap = 1, 2, 2, 32, 32, 128, 512
-    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=cap, layout=layout)
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=cap, layout=layout, sink=sink)
+    cfg.outliers = outliers
     cfg.page_tokens, cfg.num_pages = P, 16
     T0, n = 100, 300
     k, v, q = _inputs(B, T0 + n, Hkv, Hq, 92)
@@ -930,6 +933,8 @@ def test_paged_streaming_with_pages_allocated_on_demand(oracle_mod, layout):
         assert np.array_equal(getattr(stream, name), getattr(bulk, name)), name
     T, Q = T0 + n, oracle_mod.quantized_len(T0 + n, R, G)
     live = [t % (R + G) for t in range(Q, T)]  # ring slots that hold window tokens
+    if sink:
+        live.append(R + G)  # the first token's fp16 row
     for name in ("k_res", "v_res"):
         assert np.array_equal(getattr(stream, name)[:, :, live], getattr(bulk, name)[:, :, live]), name
     assert np.array_equal(oracle_mod.decode(cfg, stream, q, 0.1), oracle_mod.decode(cfg, bulk, q, 0.1))
