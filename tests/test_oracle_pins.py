@@ -714,6 +714,26 @@ def test_outliers_are_each_tokens_largest_entry_kept_in_fp16(oracle_mod, layout)
     assert cache.k_out_ch[0, 1, 17] == 40 and cache.v_out_ch[0, 0, 20] == 3
 
 
+def test_outliers_are_chosen_on_the_rotated_keys(oracle_mod):
+    # with the Hadamard option the cache holds rotated keys (reading R2), so a key's outlier is the
+    # largest entry of the rotated fp16 key: rotate each input key with the pinned fp32 transform,
+    # round to fp16, and take the first largest magnitude; values are not rotated
+    B, T, Hkv, Hq, G, R = 1, 200, 1, 2, 32, 32
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 1, cap=224)
+    cfg.outliers = 1
+    k, v, q = _inputs(B, T, Hkv, Hq, 85)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [T])
+    Q = (T - R) // G * G
+    rot = np.stack([oracle_mod.f32_to_f16(oracle_mod.wht128_f32(oracle_mod.f16_to_f32(k[0, t, 0]))) for t in range(Q)])
+    want = (rot & 0x7FFF).argmax(axis=1)
+    assert np.array_equal(cache.k_out_ch[0, 0, :Q], want)
+    assert np.array_equal(cache.k_out_val[0, 0, :Q], rot[np.arange(Q), want])
+    raw = (k[0, :Q, 0].view(np.uint16) & 0x7FFF).argmax(axis=1)
+    assert not np.array_equal(want, raw)  # the rotation moves the outliers (channels 5 and 77 are spread)
+    assert np.array_equal(cache.v_out_ch[0, 0, :Q], (v[0, :Q, 0].view(np.uint16) & 0x7FFF).argmax(axis=1))
+
+
 @pytest.mark.parametrize("layout", [1, 2])
 def test_outliers_left_out_of_group_statistics(oracle_mod, layout):
     # every key group's per-channel min / max and every value group's per-token min / max run over
