@@ -38,6 +38,8 @@ kvq_status check_config(const kvq_config* c) {
   if (!(c->rope_theta >= 0.f) || !std::isfinite(c->rope_theta)) return KVQ_ERR_INVALID_ARG;
   if (c->rope_theta > 0.f && c->hadamard) return KVQ_ERR_INVALID_ARG;                 // the two exclude each other
   if (c->rope_theta > 0.f && c->layout != KVQ_LAYOUT_ROWS_V2) return KVQ_ERR_UNSUPPORTED;  // token-row keys only
+  if (c->outliers != 0 && c->outliers != 1) return KVQ_ERR_INVALID_ARG;
+  if (c->outliers && (c->layout != KVQ_LAYOUT_TILE_V1 || c->rope_theta > 0.f)) return KVQ_ERR_UNSUPPORTED;
   if (c->capacity < 0 || c->capacity % G != 0) return KVQ_ERR_INVALID_ARG;
   if (c->capacity >= (int64_t(1) << 31)) return KVQ_ERR_INVALID_ARG;  // token indices are 32-bit on the device
   if (c->layout == KVQ_LAYOUT_ROWS_V2 && c->capacity % 128 != 0) return KVQ_ERR_INVALID_ARG;  // whole value blocks
@@ -70,6 +72,8 @@ kvq_status check_cache(const kvq_config* c, const kvq_cache* k) {
     if (p[i] == nullptr || !aligned(p[i], 16)) return KVQ_ERR_INVALID_ARG;
   }
   if (!aligned(k->seq_len_dev, 8)) return KVQ_ERR_INVALID_ARG;
+  if (c->outliers && (k->k_out == nullptr || k->v_out == nullptr || !aligned(k->k_out, 16) || !aligned(k->v_out, 16)))
+    return KVQ_ERR_INVALID_ARG;
   return KVQ_OK;
 }
 
@@ -99,6 +103,9 @@ QuantizeArgs quantize_args(const kvq_config* c, kvq_cache* k) {
   a.layout = c->layout;
   a.sink = c->sink;
   a.res_rows = a.ring + c->sink;
+  a.outliers = c->outliers;
+  a.k_out = static_cast<uint32_t*>(k->k_out);
+  a.v_out = static_cast<uint32_t*>(k->v_out);
   a.vwords = (c->layout == KVQ_LAYOUT_ROWS_V2 ? (c->capacity + 127) / 128 * 128 : c->capacity) * 4 * c->value_bits;
   return a;
 }
@@ -154,6 +161,15 @@ kvq_status kvq_cache_buffer_bytes(const kvq_config* cfg, size_t out_bytes[KVQ_NU
   if (s != KVQ_OK) return s;
   if (out_bytes == nullptr) return KVQ_ERR_INVALID_ARG;
   buffer_bytes(cfg, out_bytes);
+  return KVQ_OK;
+}
+
+kvq_status kvq_outlier_buffer_bytes(const kvq_config* cfg, size_t out_bytes[2]) {
+  const kvq_status s = check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (out_bytes == nullptr) return KVQ_ERR_INVALID_ARG;
+  const size_t n = cfg->outliers ? static_cast<size_t>(cfg->batch) * cfg->num_kv_heads * cfg->capacity * 4 : 0;
+  out_bytes[0] = out_bytes[1] = n;
   return KVQ_OK;
 }
 
@@ -240,7 +256,7 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
                   : cfg->layout == KVQ_LAYOUT_ROWS_V2
                       ? kvq::decode_tc_ctas_per_sm(cfg->group_size, cfg->num_q_heads / cfg->num_kv_heads)
                       : kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size,
-                                                cfg->num_q_heads / cfg->num_kv_heads);
+                                                cfg->num_q_heads / cfg->num_kv_heads, cfg->outliers);
   int nsplit = 1;
   const int L = plan_splits(cfg, cache->seq_len_host, sms * occ, &nsplit);
 
@@ -273,6 +289,9 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   a.ring = static_cast<int64_t>(cfg->residual) + cfg->group_size;
   a.sink = cfg->sink;
   a.res_rows = a.ring + cfg->sink;
+  a.outliers = cfg->outliers;
+  a.k_out = static_cast<const uint32_t*>(cache->k_out);
+  a.v_out = static_cast<const uint32_t*>(cache->v_out);
   a.layout = cfg->layout;
   a.split_len = L;
   a.nsplit = nsplit;

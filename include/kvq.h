@@ -62,7 +62,8 @@ typedef enum {
  *   residual R >= 0 (tokens kept in FP16 beyond the last full group; 0 <= R <= 4096);
  *   hadamard in {0, 1}; layout KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2; sink in {0, 1};
  *   rope_theta finite and >= 0; rope_theta > 0 needs hadamard = 0 (KVQ_ERR_INVALID_ARG) and layout
- *   KVQ_LAYOUT_ROWS_V2 (KVQ_ERR_UNSUPPORTED);
+ *   KVQ_LAYOUT_ROWS_V2 (KVQ_ERR_UNSUPPORTED); outliers in {0, 1}, outliers = 1 needs layout
+ *   KVQ_LAYOUT_TILE_V1 and rope_theta = 0 (KVQ_ERR_UNSUPPORTED);
  *   capacity >= 0, a multiple of G (maximum tokens per sequence); with layout ROWS_V2 also a
  *   multiple of 128 (value rows come in whole 128-token blocks). */
 typedef struct {
@@ -78,6 +79,7 @@ typedef struct {
   int32_t layout;
   int32_t sink;  /* 1: the first token of every sequence stays in fp16 (see below) */
   float rope_theta; /* > 0: keys are cached before RoPE and decode rotates them (see below); 0: off */
+  int32_t outliers; /* 1: each quantized token's largest key / value entry stays fp16 (see below) */
   int64_t capacity;
 } kvq_config;
 
@@ -113,6 +115,14 @@ typedef struct {
  * (already rotated at its own position by the caller). The decode workspace then also holds the
  * angle tables, built at the start of every call.
  *
+ * Dense-and-sparse outliers (outliers = 1; the KVQuant review, Method, keeps about 1% of the entries
+ * in an fp16 sparse store with per-vector thresholds): per quantized token and tensor, the entry of
+ * largest magnitude (ties: the lowest channel) is kept exactly. k_out / v_out hold one u32 per token
+ * and unit: bits 0..15 the channel (0xffff: none, e.g. the sink token), bits 16..31 the fp16 value.
+ * That entry stays out of its key group's (per channel) or value group's (per token) min / max and
+ * is coded 0; dequantization puts the fp16 value back. A key channel whose entries in a group are all
+ * outliers gets scale and zero 0. Sizes: kvq_outlier_buffer_bytes.
+ *
  * Tile v1: tile row k of a unit holds tokens 16k..16k+15. Within a tile, "lane" L (0..31) owns
  * words (w / 4) * 128 + 4L + (w % 4) for w in [0, 2*bits). Word w holds 16/bits code pairs; pair j
  * has its first code at bits [bits*j, bits*j + bits) and its second at bits [16 + bits*j, ...).
@@ -143,6 +153,8 @@ typedef struct {
   void* v_res;
   int64_t* seq_len_host;
   int64_t* seq_len_dev;
+  void* k_out;  /* outliers = 1 only: u32 [capacity] per unit, see below (NULL otherwise) */
+  void* v_out;
 } kvq_cache;
 
 enum {
@@ -160,6 +172,10 @@ enum {
 /* Byte size of each of the eight cache buffers for `cfg` (all units), in kvq_cache field order.
  * Returns KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED for a bad config or null pointers. */
 kvq_status kvq_cache_buffer_bytes(const kvq_config* cfg, size_t out_bytes[KVQ_NUM_BUFFERS]);
+
+/* Byte size of the two outlier buffers (k_out, v_out) for `cfg`: units * capacity * 4 each when
+ * outliers = 1, else 0. */
+kvq_status kvq_outlier_buffer_bytes(const kvq_config* cfg, size_t out_bytes[2]);
 
 /* Prefill: quantize whole prompts at once (KVQuant review, Limitations and Sparks: a prefill-side
  * kernel that compresses many keys and values in one pass).

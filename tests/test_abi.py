@@ -23,8 +23,8 @@ def _declared_symbols():
 def test_library_exports_every_declared_entry_point():
     names = _declared_symbols()
     assert names == ["kvq_append_token", "kvq_cache_buffer_bytes", "kvq_decode_attention",
-                     "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes", "kvq_quantize_prefill",
-                     "kvq_status_string"]
+                     "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes", "kvq_outlier_buffer_bytes",
+                     "kvq_quantize_prefill", "kvq_status_string"]
     lib = ctypes.CDLL(kvq.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -116,6 +116,46 @@ def test_rope_workspace_holds_the_angle_tables(cap):
     part = kvq.kvq_decode_workspace_bytes(base)
     tables = (-(-cap // 32) * 64 + 32 * 64) * 8
     assert kvq.kvq_decode_workspace_bytes(rope) == -(-part // 256) * 256 + tables
+
+
+@pytest.mark.parametrize("layout,theta,value,status", [
+    (1, 0.0, 1, kvq.KVQ_OK), (1, 0.0, 0, kvq.KVQ_OK),
+    (2, 0.0, 1, kvq.KVQ_ERR_UNSUPPORTED),        # the outlier path exists for tile v1 only
+    (2, 10000.0, 1, kvq.KVQ_ERR_UNSUPPORTED),    # and not with pre-RoPE keys
+    (1, 0.0, 2, kvq.KVQ_ERR_INVALID_ARG), (1, 0.0, -1, kvq.KVQ_ERR_INVALID_ARG),
+])
+def test_outlier_config_validation(layout, theta, value, status):
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024, layout=layout, rope_theta=theta, outliers=value)
+    sizes = (ctypes.c_size_t * 8)()
+    assert _status("kvq_cache_buffer_bytes", ctypes.byref(cfg), sizes) == status
+    out = (ctypes.c_size_t * 2)()
+    assert _status("kvq_outlier_buffer_bytes", ctypes.byref(cfg), out) == status
+
+
+@pytest.mark.parametrize("B,Hkv,cap", [(2, 2, 1024), (8, 32, 32768 + 1024), (1, 8, 1 << 20)])
+def test_outlier_buffer_bytes(B, Hkv, cap):
+    # one u32 (channel | fp16 value << 16) per (unit, token) for keys and for values; none when off
+    on = kvq.make_config(B, 4 * Hkv if Hkv <= 8 else Hkv, Hkv, 2, 2, 32, 128, 0, cap, outliers=1)
+    off = kvq.make_config(B, 4 * Hkv if Hkv <= 8 else Hkv, Hkv, 2, 2, 32, 128, 0, cap)
+    assert kvq.kvq_outlier_buffer_bytes(on) == [B * Hkv * cap * 4] * 2
+    assert kvq.kvq_outlier_buffer_bytes(off) == [0, 0]
+    assert kvq.kvq_cache_buffer_bytes(on) == kvq.kvq_cache_buffer_bytes(off)
+    assert _status("kvq_outlier_buffer_bytes", ctypes.byref(on), None) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_outlier_cache_needs_its_buffers():
+    # outliers = 1 with null outlier pointers is rejected on the host before any launch
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024, outliers=1)
+    c, host = _fake_cache(cfg, [0, 0])
+    k = ctypes.c_void_p(0x100000)
+    lens = np.array([64, 64], np.int64)
+    st = _lib.lib.kvq_quantize_prefill(ctypes.byref(cfg), ctypes.byref(c), k, k, 64 * 2 * 128, 2 * 128, 128,
+                                       lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+    c.k_out, c.v_out = 0x200000, 0x200008  # v_out not 16-byte aligned
+    st = _lib.lib.kvq_quantize_prefill(ctypes.byref(cfg), ctypes.byref(c), k, k, 64 * 2 * 128, 2 * 128, 128,
+                                       lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
 
 
 def _fake_cache(cfg, lens):
