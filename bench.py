@@ -43,9 +43,10 @@ METRIC = "decode-attn effective KV HBM GB/s (fraction of B200 peak); tokens/s"
 # ---------------------------------------------------------------------------------------------------
 # algorithmic bytes (what the method must move), per unit of work
 # ---------------------------------------------------------------------------------------------------
-def decode_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
+def decode_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0, outliers: int = 0) -> int:
     """Bytes one decode call must read/write: packed codes + key group scale/zero + value token
-    scale/zero for the quantized tokens, fp16 K/V for the window (and for the first token when the
+    scale/zero for the quantized tokens (and with the outliers on, one 4-byte key and one value
+    outlier word per quantized token), fp16 K/V for the window (and for the first token when the
     sink is on), q in and out."""
     G, R = w.group_size, w.residual
     total = 0
@@ -55,12 +56,15 @@ def decode_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
         per_unit = Q * 128 * (w.key_bits + w.value_bits) // 8 + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4
         if sink and Q > 0:
             per_unit += 128 * 4
+        if outliers:
+            per_unit += Q * 8
         total += w.num_kv_heads * per_unit
     return total + 2 * w.batch * w.num_q_heads * 128 * 2
 
 
-def prefill_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
-    """fp16 K and V read + codes, scales, zero-points and window (and the sink row) written."""
+def prefill_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0, outliers: int = 0) -> int:
+    """fp16 K and V read + codes, scales, zero-points and window (and the sink row, and the outlier
+    words) written."""
     G, R = w.group_size, w.residual
     total = 0
     for T in lens:
@@ -68,7 +72,7 @@ def prefill_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
         Q = max(T - R, 0) // G * G
         total += w.num_kv_heads * (T * 128 * 4 + Q * 128 * (w.key_bits + w.value_bits) // 8
                                    + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4
-                                   + (128 * 4 if sink and T > 0 else 0))
+                                   + (128 * 4 if sink and T > 0 else 0) + (Q * 8 if outliers else 0))
     return total
 
 
@@ -185,7 +189,7 @@ def measured_hbm_peak():
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------------------------------
 def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int = 1, sink: int = 0,
-                         rope: float = 0.0):
+                         rope: float = 0.0, outliers: int = 0):
     """Time the oracle's decode on a bounded sample of the workload: whole (sequence, KV head) units
     batched into one oracle problem (enough units to give every host core a query head), decoded
     repeatedly until about budget_s seconds have passed. Returns (GB/s of algorithmic decode bytes,
@@ -207,7 +211,7 @@ def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int
     if layout == 2:
         cap = -(-cap // 128) * 128
     ocfg = ref.Config(n, g, 1, w.key_bits, w.value_bits, w.group_size, w.residual, w.hadamard, cap,
-                      layout=layout, sink=sink, rope_theta=rope)
+                      layout=layout, sink=sink, rope_theta=rope, outliers=outliers)
     k = np.zeros((n, Tmax, 1, 128), np.float16)
     v = np.zeros_like(k)
     qs = np.zeros((n, g, 128), np.float16)
@@ -226,7 +230,7 @@ def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int
         ref.decode(ocfg, oc, qs, 1 / math.sqrt(128), threads=threads)
         spent += time.perf_counter() - t0
         calls += 1
-    per_call = decode_bytes(w.scaled(batch=n, num_q_heads=g, num_kv_heads=1), lens, sink)
+    per_call = decode_bytes(w.scaled(batch=n, num_q_heads=g, num_kv_heads=1), lens, sink, outliers)
     desc = f"{n} (sequence, KV head) units of {w.name} ({int(lens.sum())} tokens), decode x{calls}"
     return per_call * calls / spent / 1e9, threads, desc
 
@@ -237,7 +241,7 @@ def workload_config(w: inputs.Workload, args, step_bytes: int) -> dict:
             "num_kv_heads": w.num_kv_heads, "key_bits": w.key_bits, "value_bits": w.value_bits,
             "group_size": w.group_size, "residual": w.residual, "hadamard": w.hadamard,
             "ragged": bool(w.ragged_min), "parallelism": f"replicas{args.gpus}", "layout": args.layout,
-            "sink": args.sink, "rope_theta": args.rope, "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
+            "sink": args.sink, "rope_theta": args.rope, "outliers": args.outliers, "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
 
 
 def run_reference(args, w):
@@ -252,11 +256,12 @@ def run_reference(args, w):
     per_step = []
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
-        gbs, cores, sample = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink, rope=args.rope)
+        gbs, cores, sample = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink, rope=args.rope,
+                                                  outliers=args.outliers)
         if i >= args.warmup:
             per_step.append(gbs)
     value = statistics.mean(per_step)
-    step_bytes = decode_bytes(w, lens, args.sink)
+    step_bytes = decode_bytes(w, lens, args.sink, args.outliers)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_bytes / (value * 1e9) * 1e3, 3),
@@ -289,6 +294,8 @@ def main():
                     help="1: keep every sequence's first token in fp16 (attention sink)")
     ap.add_argument("--rope", type=float, default=0.0,
                     help="> 0: cache keys before RoPE with this theta and rotate them in decode (needs --layout 2)")
+    ap.add_argument("--outliers", type=int, default=0, choices=[0, 1],
+                    help="1: keep each quantized token's largest key / value entry in fp16 (needs --layout 1)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w0 = inputs.WORKLOADS[args.workload]
@@ -328,7 +335,8 @@ def main():
     if args.layout == 2:
         cap = -(-cap // 128) * 128  # rows v2 stores values in whole 128-token blocks
     cfg = kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size, w.residual,
-                          w.hadamard, cap, layout=args.layout, sink=args.sink, rope_theta=args.rope)
+                          w.hadamard, cap, layout=args.layout, sink=args.sink, rope_theta=args.rope,
+                          outliers=args.outliers)
     cache = kvq.Cache(cfg)
     stream = torch.cuda.current_stream()
 
@@ -342,7 +350,7 @@ def main():
         torch.cuda.synchronize()
         if i > 0:
             pre_ms.append(e0.elapsed_time(e1))
-    pre_bytes = prefill_bytes(w0, lens0, args.sink)
+    pre_bytes = prefill_bytes(w0, lens0, args.sink, args.outliers)
     del kd, vd
     torch.cuda.empty_cache()
 
@@ -390,7 +398,7 @@ def main():
     decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
     append_ms = [e[0].elapsed_time(e[1]) for e in evs]
     # bytes per step from the lengths each decode actually saw (append happens first)
-    step_bytes = [decode_bytes(w0, lens_before + i + 1, args.sink) for i in range(args.steps)]
+    step_bytes = [decode_bytes(w0, lens_before + i + 1, args.sink, args.outliers) for i in range(args.steps)]
     total_bytes = float(sum(step_bytes))
     tokens = w.batch * args.steps
 
@@ -424,7 +432,7 @@ def main():
         e1.record(stream)
         barrier()
         e2e_ms = e0.elapsed_time(e1)
-        e2e_bytes = float(sum(decode_bytes(w0, lens_e + i + 1, args.sink) for i in range(args.steps)))
+        e2e_bytes = float(sum(decode_bytes(w0, lens_e + i + 1, args.sink, args.outliers) for i in range(args.steps)))
         e2e_ms, e2e_bytes = reduce_over_ranks(dist, "cuda", e2e_ms, e2e_bytes)
         h2d = in_host[0].numel() * 2
         d2h = out_host.numel() * 2
@@ -479,7 +487,8 @@ def main():
         import oracle as ref
 
         ref.build()
-        gbs, cores, sample = oracle_decode_sample(w0, layout=args.layout, sink=args.sink, rope=args.rope)
+        gbs, cores, sample = oracle_decode_sample(w0, layout=args.layout, sink=args.sink, rope=args.rope,
+                                                  outliers=args.outliers)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     print(json.dumps(line), flush=True)
