@@ -67,3 +67,7 @@ def test_traffic_lookup_is_none_for_other_layouts_and_kernels():
     w = inputs.WORKLOADS["llama2_7b_mha"]
     assert bench.measured_traffic(w, 2, "decode") is None
     assert bench.measured_traffic(inputs.WORKLOADS["llama3_8b_gqa"], 1, "decode") is None
+    # the records were taken with the sink and RoPE off: other options get no traffic figure
+    assert bench.measured_traffic(w, 1, "decode", sink=1) is None
+    assert bench.measured_traffic(w, 1, "prefill", sink=1) is None
+    assert bench.measured_traffic(w, 2, "decode", rope=10000.0) is None
