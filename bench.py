@@ -151,12 +151,13 @@ def reduce_over_ranks(dist, device, ms: float, *sums: float):
     return out
 
 
-def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode", sink: int = 0, rope: float = 0.0):
+def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode", sink: int = 0, rope: float = 0.0,
+                     outliers: int = 0):
     """DRAM bytes per launch of the decode-split (kind "decode") or bulk-prefill (kind "prefill")
     kernel from the committed ncu counters (profiles/decode_traffic_counters.txt, JSON), scaled from
     the captured batch to this one by the units processed; None if there is no capture for this
-    workload, layout, kernel and options (sink, RoPE; a record without them was taken with them
-    off) or the kernel sources changed since it was taken."""
+    workload, layout, kernel and options (sink, RoPE, outliers; a record without them was taken with
+    them off) or the kernel sources changed since it was taken."""
     import hashlib
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "decode_traffic_counters.txt")
     try:
@@ -167,7 +168,7 @@ def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode", sink
     for e in entries.values():
         if e.get("workload") != w.name or e.get("layout") != layout or e.get("kind", "decode") != kind:
             continue
-        if e.get("sink", 0) != sink or e.get("rope_theta", 0.0) != rope:
+        if e.get("sink", 0) != sink or e.get("rope_theta", 0.0) != rope or e.get("outliers", 0) != outliers:
             continue
         h = hashlib.sha256()
         for f in e["kernel_sources"]:
@@ -471,14 +472,14 @@ def main():
         "decode_ms": round(mean_decode_ms, 4),
         "append_us": round(statistics.mean(append_ms) * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout, "decode", args.sink, args.rope), "peak_kind": peak_kind,
+                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout, "decode", args.sink, args.rope, args.outliers), "peak_kind": peak_kind,
                      "kernel": ("decode_rope_kernel" if args.rope > 0 else
                                 "decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
                      + " + decode_combine_kernel (one kvq_decode_attention call)"},
         "prefill": {"gbs": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9, 1),
                     "ms": round(statistics.mean(pre_ms), 3), "bytes": pre_bytes, "bound": "hbm", "peak": peak,
                     "frac": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9 / peak, 4),
-                    "traffic": measured_traffic(w0, args.layout, "prefill", args.sink, args.rope),
+                    "traffic": measured_traffic(w0, args.layout, "prefill", args.sink, args.rope, args.outliers),
                     "kernel": "prefill_block_kernel (one kvq_quantize_prefill call)"},
         # per step: append + length bump, then the decode split kernel + combine (+ the RoPE angle tables)
         "gpu_launches": (5 if args.rope > 0 else 4) * args.steps,
