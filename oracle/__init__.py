@@ -53,14 +53,15 @@ class _CConfig(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32), ("value_bits", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("residual", ctypes.c_int32), ("hadamard", ctypes.c_int32),
         ("layout", ctypes.c_int32), ("sink", ctypes.c_int32), ("rope_theta", ctypes.c_float),
-        ("outliers", ctypes.c_int32), ("capacity", ctypes.c_int64),
+        ("outliers", ctypes.c_int32), ("page_tokens", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+        ("capacity", ctypes.c_int64),
     ]
 
 
 class _CCache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero", "k_res", "v_res", "seq_len",
-                 "k_out_ch", "k_out_val", "v_out_ch", "v_out_val")]
+                 "k_out_ch", "k_out_val", "v_out_ch", "v_out_val", "page_table")]
 
 
 def _declare(L: ctypes.CDLL) -> None:
@@ -105,43 +106,61 @@ class Config:
     sink: int = 0    # 1: the first token stays in fp16 (an extra row after the ring)
     rope_theta: float = 0.0  # > 0: keys are cached before RoPE and decode applies it (0: off)
     outliers: int = 0  # 1: each quantized token's largest-magnitude key / value entry stays fp16
+    page_tokens: int = 0  # > 0: paged storage with pages of this many tokens (a multiple of 128); 0: contiguous
+    num_pages: int = 0    # pages in the pool (paged storage only)
 
     def c(self) -> _CConfig:
         return _CConfig(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.key_bits,
                         self.value_bits, self.group_size, self.residual, self.hadamard, self.layout, self.sink,
-                        self.rope_theta, self.outliers, self.capacity)
+                        self.rope_theta, self.outliers, self.page_tokens, self.num_pages, self.capacity)
 
 
 class Cache:
-    """Host buffers of the packed cache, laid out exactly as the product's device buffers."""
+    """Host buffers of the packed cache, laid out exactly as the product's device buffers.
 
-    def __init__(self, cfg: Config):
+    Contiguous storage: every per-token array has one slot of ``capacity`` tokens per unit, shape
+    [B][Hkv][...]. Paged storage (``cfg.page_tokens`` = P > 0, reading R13): one slot of P tokens per
+    physical page, shape [num_pages][...], and ``page_table`` [B][Hkv][capacity / P] (int32) names the
+    physical page of each logical page; by default unit u's page j is u * (capacity / P) + j."""
+
+    def __init__(self, cfg: Config, page_table: np.ndarray | None = None):
         B, H, cap, G = cfg.batch, cfg.num_kv_heads, cfg.capacity, cfg.group_size
         ring = cfg.residual + G + cfg.sink  # ring slots, then the first token's row when the sink is on
-        if cfg.layout == 2:
-            self.k_codes = np.zeros((B, H, cap, 4 * cfg.key_bits), np.uint32)
-            self.v_codes = np.zeros((B, H, (cap + 127) // 128, 128, 4 * cfg.value_bits), np.uint32)
+        if cfg.page_tokens:
+            lead, n = (cfg.num_pages,), cfg.page_tokens
+            per_unit = cap // cfg.page_tokens
+            if page_table is None:
+                page_table = np.arange(B * H * per_unit, dtype=np.int32).reshape(B, H, per_unit)
+            self.page_table = np.ascontiguousarray(page_table, np.int32)
+            assert self.page_table.shape == (B, H, per_unit)
         else:
-            self.k_codes = np.zeros((B, H, cap // 16, 64 * cfg.key_bits), np.uint32)
-            self.v_codes = np.zeros((B, H, cap // 16, 64 * cfg.value_bits), np.uint32)
-        self.k_scale = np.zeros((B, H, cap // G, 128), np.uint16)
-        self.k_zero = np.zeros((B, H, cap // G, 128), np.uint16)
-        self.v_scale = np.zeros((B, H, cap, 128 // G), np.uint16)
-        self.v_zero = np.zeros((B, H, cap, 128 // G), np.uint16)
+            lead, n = (B, H), cap
+            self.page_table = None
+        if cfg.layout == 2:
+            self.k_codes = np.zeros(lead + (n, 4 * cfg.key_bits), np.uint32)
+            self.v_codes = np.zeros(lead + ((n + 127) // 128, 128, 4 * cfg.value_bits), np.uint32)
+        else:
+            self.k_codes = np.zeros(lead + (n // 16, 64 * cfg.key_bits), np.uint32)
+            self.v_codes = np.zeros(lead + (n // 16, 64 * cfg.value_bits), np.uint32)
+        self.k_scale = np.zeros(lead + (n // G, 128), np.uint16)
+        self.k_zero = np.zeros(lead + (n // G, 128), np.uint16)
+        self.v_scale = np.zeros(lead + (n, 128 // G), np.uint16)
+        self.v_zero = np.zeros(lead + (n, 128 // G), np.uint16)
         self.k_res = np.zeros((B, H, ring, 128), np.uint16)
         self.v_res = np.zeros((B, H, ring, 128), np.uint16)
         self.seq_len = np.zeros((B,), np.int64)
         # sparse outliers (one per quantized token and tensor): channel (0xffff: none) and fp16 value
-        self.k_out_ch = np.full((B, H, cap), 0xFFFF, np.uint16)
-        self.k_out_val = np.zeros((B, H, cap), np.uint16)
-        self.v_out_ch = np.full((B, H, cap), 0xFFFF, np.uint16)
-        self.v_out_val = np.zeros((B, H, cap), np.uint16)
+        self.k_out_ch = np.full(lead + (n,), 0xFFFF, np.uint16)
+        self.k_out_val = np.zeros(lead + (n,), np.uint16)
+        self.v_out_ch = np.full(lead + (n,), 0xFFFF, np.uint16)
+        self.v_out_val = np.zeros(lead + (n,), np.uint16)
 
     def c(self) -> _CCache:
         return _CCache(*(a.ctypes.data for a in (self.k_codes, self.v_codes, self.k_scale, self.k_zero,
                                                  self.v_scale, self.v_zero, self.k_res, self.v_res,
                                                  self.seq_len, self.k_out_ch, self.k_out_val, self.v_out_ch,
-                                                 self.v_out_val)))
+                                                 self.v_out_val)),
+                       self.page_table.ctypes.data if self.page_table is not None else None)
 
 
 def _u16(a: np.ndarray) -> np.ndarray:

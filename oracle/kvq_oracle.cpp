@@ -53,6 +53,14 @@
 //      min/max of its key group (per channel) or value group (per token), and coded 0; dequantization
 //      puts the fp16 value back. A key channel whose entries in a group are all outliers gets scale
 //      and zero 0. The sink token (R10) has no outlier; the fp16 window needs none.
+//  R13 optional paged storage (page_tokens = P > 0; KVQuant review, Limitations, Future work and
+//      Sparks: blocked allocation instead of copying the previous tokens' data on every update).
+//      The quantized part of a unit is cut into logical pages of P tokens (P a multiple of 128, so
+//      a page holds whole 16-token tiles, whole 128-token value blocks of rows v2 and whole key
+//      groups). Logical page j of a unit lives in physical page page_table[unit][j] of a pool of
+//      num_pages pages; a page holds exactly what the contiguous layout holds for its P tokens
+//      (codes, key group scale / zero, value scale / zero, outliers), at the in-page token t mod P.
+//      The fp16 window and the sink row stay per unit. Paging changes addresses only, never values.
 //
 // Build: g++ -O2 -std=c++17 -ffp-contract=off -fno-fast-math -fPIC -shared (x86-64 SSE scalar fp32).
 
@@ -287,9 +295,14 @@ typedef struct {
   int32_t sink;        // 1: the first token stays in fp16 (reading R10)
   float rope_theta;    // > 0: keys are cached before RoPE, decode applies it (reading R11); 0: off
   int32_t outliers;    // 1: each quantized token's largest-magnitude key and value entry stay fp16 (R12)
-  int64_t capacity;
+  int32_t page_tokens; // > 0: paged storage with pages of this many tokens (reading R13); 0: contiguous
+  int32_t num_pages;   // pages in the pool (paged storage only)
+  int64_t capacity;    // tokens per sequence (paged: capacity / page_tokens logical pages per unit)
 } kvq_ref_config;
 
+// Contiguous storage: every per-token array below has one slot of capacity tokens per unit
+// ([B][Hkv][...]). Paged storage (R13): one slot of page_tokens tokens per physical page
+// ([num_pages][...]); the ring stays [B][Hkv][...].
 typedef struct {
   uint32_t* k_codes;  // [B][Hkv][Cap/16][64*key_bits]
   uint32_t* v_codes;  // [B][Hkv][Cap/16][64*value_bits]
@@ -304,6 +317,7 @@ typedef struct {
   uint16_t* k_out_val;  // [B][Hkv][Cap] its fp16 value
   uint16_t* v_out_ch;   // same for values
   uint16_t* v_out_val;
+  int32_t* page_table;  // [B][Hkv][Cap/page_tokens] physical page of each logical page (paged only)
 } kvq_ref_cache;
 
 enum { REF_OK = 0, REF_ERR_ARG = -1, REF_ERR_CAPACITY = -3 };
@@ -322,6 +336,8 @@ static int check_config(const kvq_ref_config* c) {
   if (!(c->rope_theta >= 0.0f) || !std::isfinite(c->rope_theta)) return REF_ERR_ARG;
   if (c->rope_theta > 0.0f && c->hadamard) return REF_ERR_ARG;
   if (c->outliers != 0 && c->outliers != 1) return REF_ERR_ARG;
+  if (c->page_tokens < 0 || c->num_pages < 0) return REF_ERR_ARG;
+  if (c->page_tokens > 0 && (c->page_tokens % 128 || c->capacity % c->page_tokens)) return REF_ERR_ARG;
   return REF_OK;
 }
 
@@ -352,22 +368,49 @@ static void value_pos(const kvq_ref_config* c, int64_t t, int ch, int64_t* word,
 static int key_param_index(const kvq_ref_config* c, int ch) { return c->layout == 2 ? ch : key_param_pos(ch); }
 
 struct Dims {
-  int64_t kw_tile, vw_tile, tiles, groups, ring, vpt;  // words per tile, tiles/unit, groups/unit, ring slots, value groups per token
-  int64_t kwords, vwords;                              // code words per unit
+  int64_t slot_tokens;                                 // tokens per storage slot: capacity (contiguous) or page_tokens (R13)
+  int64_t kw_tile, vw_tile, tiles, groups, ring, vpt;  // words per tile, tiles/slot, groups/slot, ring slots, value groups per token
+  int64_t kwords, vwords;                              // code words per slot
   int64_t res_rows;                                    // rows of k_res / v_res per unit: ring slots + the sink row
 };
 static Dims dims(const kvq_ref_config* c) {
   Dims d;
   d.kw_tile = 64 * c->key_bits;
   d.vw_tile = 64 * c->value_bits;
-  d.tiles = c->capacity / 16;
-  d.kwords = c->capacity * 4 * c->key_bits;
-  d.vwords = (c->layout == 2 ? (c->capacity + 127) / 128 * 128 : c->capacity) * 4 * c->value_bits;
-  d.groups = c->capacity / c->group_size;
+  d.slot_tokens = c->page_tokens > 0 ? c->page_tokens : c->capacity;
+  d.tiles = d.slot_tokens / 16;
+  d.kwords = d.slot_tokens * 4 * c->key_bits;
+  d.vwords = (c->layout == 2 ? (d.slot_tokens + 127) / 128 * 128 : d.slot_tokens) * 4 * c->value_bits;
+  d.groups = d.slot_tokens / c->group_size;
   d.ring = c->residual + c->group_size;
   d.res_rows = d.ring + c->sink;
   d.vpt = 128 / c->group_size;
   return d;
+}
+
+// Storage slot of token t of `unit` and the token's index within it (reading R13): the unit and t
+// for contiguous storage; the physical page of logical page t / P and t mod P for paged storage.
+static void locate(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t unit, int64_t t, int64_t* slot,
+                   int64_t* ts) {
+  if (c->page_tokens == 0) {
+    *slot = unit;
+    *ts = t;
+    return;
+  }
+  const int64_t pages_per_unit = c->capacity / c->page_tokens;
+  *slot = cache->page_table[unit * pages_per_unit + t / c->page_tokens];
+  *ts = t % c->page_tokens;
+}
+
+// Whether every logical page holding tokens [0, n) of `unit` maps to a page of the pool.
+static bool pages_valid(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t unit, int64_t n) {
+  if (c->page_tokens == 0) return true;
+  const int64_t pages_per_unit = c->capacity / c->page_tokens;
+  for (int64_t j = 0; j * c->page_tokens < n; ++j) {
+    const int32_t p = cache->page_table[unit * pages_per_unit + j];
+    if (p < 0 || p >= c->num_pages) return false;
+  }
+  return true;
 }
 
 // The channel of a token vector's largest-magnitude entry (reading R12): binary16 magnitudes order
@@ -389,11 +432,13 @@ static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, i
   const Dims d = dims(c);
   const int G = c->group_size;
   const int skip = (c->sink && t0 == 0) ? 1 : 0;  // tokens at the start of the span kept out
+  int64_t slot, ts0;  // where the span is stored (a group never crosses a page: P is a multiple of G)
+  locate(c, cache, unit, t0, &slot, &ts0);
   // Outliers (reading R12): each token's largest-magnitude key entry and value entry.
   std::vector<uint8_t> kout(static_cast<size_t>(G) * 128, 0), vout(static_cast<size_t>(G) * 128, 0);
   if (c->outliers) {
     for (int i = 0; i < G; ++i) {
-      const int64_t at = unit * c->capacity + t0 + i;
+      const int64_t at = slot * d.slot_tokens + ts0 + i;
       if (i < skip) {  // the sink token is fp16 as a whole
         cache->k_out_ch[at] = cache->v_out_ch[at] = 0xffffu;
         cache->k_out_val[at] = cache->v_out_val[at] = 0;
@@ -410,17 +455,17 @@ static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, i
   }
   // Keys: per channel over the G (or G - 1) tokens of the group, outliers left out.
   std::vector<uint8_t> kc(static_cast<size_t>(G) * 128, 0);
-  const int64_t g = t0 / G;
+  const int64_t g = ts0 / G;
   for (int ch = 0; ch < 128; ++ch) {
     GroupQ q = quantize_group(kt + skip * k_ld + ch, G - skip, static_cast<int>(k_ld), c->key_bits,
                               kc.data() + skip * 128 + ch, 128, kout.data() + skip * 128 + ch, 128);
     const int pos = key_param_index(c, ch);
-    cache->k_scale[(unit * d.groups + g) * 128 + pos] = q.scale;
-    cache->k_zero[(unit * d.groups + g) * 128 + pos] = q.zero;
+    cache->k_scale[(slot * d.groups + g) * 128 + pos] = q.scale;
+    cache->k_zero[(slot * d.groups + g) * 128 + pos] = q.zero;
   }
-  uint32_t* kbuf = cache->k_codes + unit * d.kwords;
+  uint32_t* kbuf = cache->k_codes + slot * d.kwords;
   for (int i = 0; i < G; ++i) {
-    const int64_t t = t0 + i;
+    const int64_t t = ts0 + i;
     for (int ch = 0; ch < 128; ++ch) {
       int64_t word;
       int bit;
@@ -432,7 +477,7 @@ static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, i
   // Values: per token over channel groups of G.
   std::vector<uint8_t> vc(128);
   for (int i = 0; i < G; ++i) {
-    const int64_t t = t0 + i;
+    const int64_t t = ts0 + i;
     for (int j = 0; j < d.vpt; ++j) {
       GroupQ q{0, 0};
       if (i < skip)
@@ -440,10 +485,10 @@ static void quantize_span(const kvq_ref_config* c, const kvq_ref_cache* cache, i
       else
         q = quantize_group(vt + i * v_ld + j * G, G, 1, c->value_bits, vc.data() + j * G, 1,
                            vout.data() + i * 128 + j * G, 1);
-      cache->v_scale[(unit * c->capacity + t) * d.vpt + j] = q.scale;
-      cache->v_zero[(unit * c->capacity + t) * d.vpt + j] = q.zero;
+      cache->v_scale[(slot * d.slot_tokens + t) * d.vpt + j] = q.scale;
+      cache->v_zero[(slot * d.slot_tokens + t) * d.vpt + j] = q.zero;
     }
-    uint32_t* vbuf = cache->v_codes + unit * d.vwords;
+    uint32_t* vbuf = cache->v_codes + slot * d.vwords;
     for (int ch = 0; ch < 128; ++ch) {
       int64_t word;
       int bit;
@@ -499,6 +544,9 @@ int kvq_ref_quantize_prefill(const kvq_ref_config* c, kvq_ref_cache* cache, cons
   for (int b = 0; b < c->batch; ++b)
     if (seq_lens[b] < 0 || seq_lens[b] > c->capacity) return REF_ERR_CAPACITY;
   const int64_t units = static_cast<int64_t>(c->batch) * c->num_kv_heads;
+  for (int64_t u = 0; u < units; ++u)
+    if (!pages_valid(c, cache, u, quantized_len(seq_lens[u / c->num_kv_heads], c->residual, c->group_size)))
+      return REF_ERR_ARG;
   auto work = [&](int64_t u0, int64_t step) {
     for (int64_t u = u0; u < units; u += step) {
       const int64_t b = u / c->num_kv_heads, h = u % c->num_kv_heads;
@@ -525,6 +573,11 @@ int kvq_ref_append_token(const kvq_ref_config* c, kvq_ref_cache* cache, const ui
   const int G = c->group_size;
   for (int b = 0; b < c->batch; ++b)
     if (cache->seq_len[b] + 1 > c->capacity) return REF_ERR_CAPACITY;
+  for (int b = 0; b < c->batch; ++b)
+    for (int h = 0; h < c->num_kv_heads; ++h)
+      if (!pages_valid(c, cache, static_cast<int64_t>(b) * c->num_kv_heads + h,
+                       quantized_len(cache->seq_len[b] + 1, c->residual, G)))
+        return REF_ERR_ARG;
   for (int b = 0; b < c->batch; ++b) {
     const int64_t t = cache->seq_len[b];
     const int64_t Q_old = quantized_len(t, c->residual, G);
@@ -570,21 +623,23 @@ static void key_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64_t
     for (int ch = 0; ch < 128; ++ch) out[ch] = half_to_float(r[ch]);
     return;
   }
-  const uint32_t* kbuf = cache->k_codes + unit * d.kwords;
-  const int64_t g = t / c->group_size;
+  int64_t slot, ts;  // where token t is stored (reading R13)
+  locate(c, cache, unit, t, &slot, &ts);
+  const uint32_t* kbuf = cache->k_codes + slot * d.kwords;
+  const int64_t g = ts / c->group_size;
   for (int ch = 0; ch < 128; ++ch) {
     int64_t word;
     int bit;
-    key_pos(c, t, ch, &word, &bit);
+    key_pos(c, ts, ch, &word, &bit);
     const uint32_t code = (kbuf[word] >> bit) & ((1u << c->key_bits) - 1u);
     const int pos = key_param_index(c, ch);
-    const double s = half_to_float(cache->k_scale[(unit * d.groups + g) * 128 + pos]);
-    const double z = half_to_float(cache->k_zero[(unit * d.groups + g) * 128 + pos]);
+    const double s = half_to_float(cache->k_scale[(slot * d.groups + g) * 128 + pos]);
+    const double z = half_to_float(cache->k_zero[(slot * d.groups + g) * 128 + pos]);
     out[ch] = static_cast<double>(code) * s + z;
   }
   if (c->outliers) {  // the token's fp16 outlier replaces its entry (reading R12)
-    const uint16_t ch = cache->k_out_ch[unit * c->capacity + t];
-    if (ch < 128) out[ch] = half_to_float(cache->k_out_val[unit * c->capacity + t]);
+    const uint16_t ch = cache->k_out_ch[slot * d.slot_tokens + ts];
+    if (ch < 128) out[ch] = half_to_float(cache->k_out_val[slot * d.slot_tokens + ts]);
   }
 }
 
@@ -596,20 +651,22 @@ static void value_row(const kvq_ref_config* c, const kvq_ref_cache* cache, int64
     for (int ch = 0; ch < 128; ++ch) out[ch] = half_to_float(r[ch]);
     return;
   }
-  const uint32_t* vbuf = cache->v_codes + unit * d.vwords;
+  int64_t slot, ts;  // where token t is stored (reading R13)
+  locate(c, cache, unit, t, &slot, &ts);
+  const uint32_t* vbuf = cache->v_codes + slot * d.vwords;
   for (int ch = 0; ch < 128; ++ch) {
     int64_t word;
     int bit;
-    value_pos(c, t, ch, &word, &bit);
+    value_pos(c, ts, ch, &word, &bit);
     const uint32_t code = (vbuf[word] >> bit) & ((1u << c->value_bits) - 1u);
     const int j = ch / c->group_size;
-    const double s = half_to_float(cache->v_scale[(unit * c->capacity + t) * d.vpt + j]);
-    const double z = half_to_float(cache->v_zero[(unit * c->capacity + t) * d.vpt + j]);
+    const double s = half_to_float(cache->v_scale[(slot * d.slot_tokens + ts) * d.vpt + j]);
+    const double z = half_to_float(cache->v_zero[(slot * d.slot_tokens + ts) * d.vpt + j]);
     out[ch] = static_cast<double>(code) * s + z;
   }
   if (c->outliers) {  // the token's fp16 outlier replaces its entry (reading R12)
-    const uint16_t ch = cache->v_out_ch[unit * c->capacity + t];
-    if (ch < 128) out[ch] = half_to_float(cache->v_out_val[unit * c->capacity + t]);
+    const uint16_t ch = cache->v_out_ch[slot * d.slot_tokens + ts];
+    if (ch < 128) out[ch] = half_to_float(cache->v_out_val[slot * d.slot_tokens + ts]);
   }
 }
 
@@ -666,6 +723,9 @@ int kvq_ref_decode(const kvq_ref_config* c, const kvq_ref_cache* cache, const ui
                    double* out, int nthreads) {
   int rc = check_config(c);
   if (rc) return rc;
+  for (int64_t u = 0; u < static_cast<int64_t>(c->batch) * c->num_kv_heads; ++u)
+    if (!pages_valid(c, cache, u, quantized_len(cache->seq_len[u / c->num_kv_heads], c->residual, c->group_size)))
+      return REF_ERR_ARG;
   const int64_t rows = static_cast<int64_t>(c->batch) * c->num_q_heads;
   auto work = [&](int64_t r0, int64_t step) {
     for (int64_t r = r0; r < rows; r += step)

@@ -73,9 +73,17 @@ MUTANTS = [
      "kc.data() + skip * 128 + ch, 128);",
      ["test_outliers_left_out_of_group_statistics"]),
     ("value_outlier_not_restored_in_decode",
-     "    if (ch < 128) out[ch] = half_to_float(cache->v_out_val[unit * c->capacity + t]);",
+     "    if (ch < 128) out[ch] = half_to_float(cache->v_out_val[slot * d.slot_tokens + ts]);",
      "    (void)ch;",
      ["test_outliers_dequantized_attention_equals_library_attention"]),
+    ("page_table_row_stride_dropped",
+     "  *slot = cache->page_table[unit * pages_per_unit + t / c->page_tokens];",
+     "  *slot = cache->page_table[unit + t / c->page_tokens];",
+     ["test_paged_shuffled_pool_gathers_to_the_contiguous_cache"]),
+    ("value_read_skips_the_page_table",
+     "  int64_t slot, ts;  // where token t is stored (reading R13)\n  locate(c, cache, unit, t, &slot, &ts);\n  const uint32_t* vbuf",
+     "  int64_t slot = unit, ts = t;\n  const uint32_t* vbuf",
+     ["test_paged_shuffled_pool_gathers_to_the_contiguous_cache"]),
     ("outlier_ties_to_the_highest_channel",
      "    if ((x[ch] & 0x7fffu) > (x[best] & 0x7fffu)) best = ch;",
      "    if ((x[ch] & 0x7fffu) >= (x[best] & 0x7fffu)) best = ch;",
@@ -113,6 +121,8 @@ def _run_pin(fn_name, mod):
         "test_rope_without_quantization_equals_library_attention_on_rotated_keys": [dict(theta=10000.0)],
         "test_outliers_left_out_of_group_statistics": [dict(layout=1)],
         "test_outliers_are_each_tokens_largest_entry_kept_in_fp16": [dict(layout=1)],
+        # all of the pool's table entries are valid pages here, so a wrong lookup stays in bounds
+        "test_paged_shuffled_pool_gathers_to_the_contiguous_cache": [dict(layout=1, outliers=0)],
     }.get(fn_name, [dict()])
     for kw in params:
         fn(mod, **kw)

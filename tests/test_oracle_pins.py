@@ -798,3 +798,158 @@ def test_outliers_streaming_equals_bulk(oracle_mod, layout):
         oracle_mod.append_token(cfg, stream, k[:, T0 + s], v[:, T0 + s])
     for name in ("k_codes", "k_scale", "k_zero", "v_scale", "v_zero", "k_out_ch", "k_out_val", "v_out_ch", "v_out_val"):
         assert np.array_equal(getattr(stream, name), getattr(bulk, name)), name
+
+
+# ---- R13: paged storage --------------------------------------------------------------------------
+# KVQuant review (Limitations, Future work, Sparks): blocked allocation instead of copying the
+# previous tokens' data on every update. Paging moves where a token's codes and parameters live, never
+# what they are: every pin below compares against the contiguous cache of the same inputs.
+
+_PAGED_ARRAYS = ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero", "k_out_ch", "k_out_val",
+                 "v_out_ch", "v_out_val")
+
+
+def _page_slice(cfg, name, j):
+    """Index range of logical page j along the token-derived axis of array `name` (contiguous layout)."""
+    P, G = cfg.page_tokens, cfg.group_size
+    per = {"k_scale": P // G, "k_zero": P // G}.get(name)
+    if per is None:
+        if name in ("k_codes", "v_codes") and cfg.layout == 1:
+            per = P // 16
+        elif name == "v_codes":  # rows v2: 128-token value blocks
+            per = P // 128
+        else:  # rows v2 key rows, value parameters, outliers: one entry per token
+            per = P
+    return slice(j * per, (j + 1) * per)
+
+
+def _paged_pair(oracle_mod, layout, outliers, sink, table_fn, lens, appends=0, seed=91):
+    B, Hkv, Hq, G, R, P, cap = 2, 2, 4, 32, 32, 128, 512
+    M = cap // P
+    extra = 3  # spare pool pages nobody uses
+    kw = dict(layout=layout, sink=sink)
+    contig = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=cap, **kw)
+    contig.outliers = outliers
+    paged = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=cap, **kw)
+    paged.outliers = outliers
+    paged.page_tokens, paged.num_pages = P, B * Hkv * M + extra
+    T = max(lens) + appends
+    k, v, q = _inputs(B, T, Hkv, Hq, seed)
+    table = table_fn(B, Hkv, M, paged.num_pages)
+    cc, pc = oracle_mod.Cache(contig), oracle_mod.Cache(paged, page_table=table)
+    for cfg, cache in ((contig, cc), (paged, pc)):
+        oracle_mod.quantize_prefill(cfg, cache, k[:, : max(lens)], v[:, : max(lens)], lens)
+        for s in range(appends):
+            t = max(lens) + s
+            oracle_mod.append_token(cfg, cache, k[:, t], v[:, t])
+    return contig, cc, paged, pc, q
+
+
+def _identity_table(B, H, M, n):
+    return np.arange(B * H * M, dtype=np.int32).reshape(B, H, M)
+
+
+def _shuffled_table(B, H, M, n):
+    perm = np.random.default_rng(7).permutation(n).astype(np.int32)
+    return perm[: B * H * M].reshape(B, H, M)
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+@pytest.mark.parametrize("outliers,sink", [(0, 0), (1, 1)])
+def test_paged_identity_table_is_the_contiguous_cache(oracle_mod, layout, outliers, sink):
+    # with unit u's page j at pool page u * M + j, the pool is the contiguous cache byte for byte:
+    # the layout repeats every P tokens, so paging is an address map and nothing else
+    contig, cc, paged, pc, q = _paged_pair(oracle_mod, layout, outliers, sink, _identity_table, [500, 300], appends=9)
+    for name in _PAGED_ARRAYS:
+        a, b = getattr(cc, name), getattr(pc, name)
+        used = a.reshape(-1).size
+        assert np.array_equal(b.reshape(-1)[:used], a.reshape(-1)), name
+    for name in ("k_res", "v_res", "seq_len"):
+        assert np.array_equal(getattr(cc, name), getattr(pc, name)), name
+    out_c = oracle_mod.decode(contig, cc, q, 1 / math.sqrt(128))
+    out_p = oracle_mod.decode(paged, pc, q, 1 / math.sqrt(128))
+    assert np.array_equal(out_c, out_p)
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+@pytest.mark.parametrize("outliers", [0, 1])
+def test_paged_shuffled_pool_gathers_to_the_contiguous_cache(oracle_mod, layout, outliers):
+    # pages scattered over a pool with spare pages: gathering each unit's pages through the table
+    # gives the contiguous arrays, the spare pages stay untouched, and decode is bit-identical
+    contig, cc, paged, pc, q = _paged_pair(oracle_mod, layout, outliers, 0, _shuffled_table, [500, 300], appends=12)
+    table = pc.page_table
+    used = set(table.reshape(-1).tolist())
+    for name in _PAGED_ARRAYS:
+        a, b = getattr(cc, name), getattr(pc, name)
+        for bb in range(table.shape[0]):
+            for h in range(table.shape[1]):
+                for j in range(table.shape[2]):
+                    np.testing.assert_array_equal(b[table[bb, h, j]], a[bb, h][_page_slice(paged, name, j)],
+                                                  err_msg=f"{name} unit {bb},{h} page {j}")
+        blank = 0xFFFF if name.endswith("_ch") else 0
+        for p in set(range(paged.num_pages)) - used:
+            assert (b[p] == blank).all(), f"{name}: spare page {p} was written"
+    out_c = oracle_mod.decode(contig, cc, q, 1 / math.sqrt(128))
+    out_p = oracle_mod.decode(paged, pc, q, 1 / math.sqrt(128))
+    assert np.array_equal(out_c, out_p)
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_paged_streaming_with_pages_allocated_on_demand(oracle_mod, layout):
+    # the caller hands out a page only when the quantized part first reaches it; streaming then
+    # equals a bulk prefill into the same pages, and a missing page is an argument error
+    B, Hkv, Hq, G, R, P, cap = 1, 2, 2, 32, 32, 128, 512
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=cap, layout=layout)
+    cfg.page_tokens, cfg.num_pages = P, 16
+    T0, n = 100, 300
+    k, v, q = _inputs(B, T0 + n, Hkv, Hq, 92)
+    table = np.full((B, Hkv, cap // P), -1, np.int32)
+    free = list(np.random.default_rng(3).permutation(cfg.num_pages))
+    stream = oracle_mod.Cache(cfg, page_table=table)
+
+    def need(T):  # allocate the pages the quantized part of length T reaches
+        Q = oracle_mod.quantized_len(T, R, G)
+        for h in range(Hkv):
+            for j in range(-(-Q // P)):
+                if stream.page_table[0, h, j] < 0:
+                    stream.page_table[0, h, j] = free.pop()
+
+    need(T0)
+    oracle_mod.quantize_prefill(cfg, stream, k[:, :T0], v[:, :T0], [T0])
+    for s in range(n):
+        t = T0 + s
+        if oracle_mod.quantized_len(t + 1, R, G) > oracle_mod.quantized_len(t, R, G) and \
+                (oracle_mod.quantized_len(t + 1, R, G) - 1) // P != (oracle_mod.quantized_len(t, R, G) - 1) // P:
+            with pytest.raises(ValueError):  # the flush reaches a page the caller has not handed out
+                oracle_mod.append_token(cfg, stream, k[:, t], v[:, t])
+            need(t + 1)
+        oracle_mod.append_token(cfg, stream, k[:, t], v[:, t])
+    bulk = oracle_mod.Cache(cfg, page_table=stream.page_table.copy())
+    oracle_mod.quantize_prefill(cfg, bulk, k, v, [T0 + n])
+    for name in _PAGED_ARRAYS + ("seq_len",):
+        assert np.array_equal(getattr(stream, name), getattr(bulk, name)), name
+    T, Q = T0 + n, oracle_mod.quantized_len(T0 + n, R, G)
+    live = [t % (R + G) for t in range(Q, T)]  # ring slots that hold window tokens
+    for name in ("k_res", "v_res"):
+        assert np.array_equal(getattr(stream, name)[:, :, live], getattr(bulk, name)[:, :, live]), name
+    assert np.array_equal(oracle_mod.decode(cfg, stream, q, 0.1), oracle_mod.decode(cfg, bulk, q, 0.1))
+
+
+def test_paged_config_and_table_validation(oracle_mod):
+    base = dict(B=1, Hq=2, Hkv=1, kb=2, vb=2, G=32, R=32, had=0, cap=512)
+    k, v, q = _inputs(1, 300, 1, 2, 93)
+    for P in (64, 96, 384):  # not a multiple of 128, or not dividing the capacity
+        cfg = _cfg(oracle_mod, **base)
+        cfg.page_tokens, cfg.num_pages = P, 8
+        with pytest.raises(ValueError):
+            oracle_mod.quantize_prefill(cfg, oracle_mod.Cache(cfg, page_table=np.zeros((1, 1, 512 // P), np.int32)),
+                                        k, v, [300])
+    cfg = _cfg(oracle_mod, **base)
+    cfg.page_tokens, cfg.num_pages = 128, 4
+    for bad in (-1, 4):  # a page the quantized part (256 tokens: pages 0 and 1) needs, outside the pool
+        table = np.array([[[0, bad, -1, -1]]], np.int32)
+        with pytest.raises(ValueError):
+            oracle_mod.quantize_prefill(cfg, oracle_mod.Cache(cfg, page_table=table), k, v, [300])
+    # pages past the quantized part may stay unassigned
+    oracle_mod.quantize_prefill(cfg, oracle_mod.Cache(cfg, page_table=np.array([[[2, 0, -1, -1]]], np.int32)),
+                                k, v, [300])
