@@ -39,14 +39,16 @@ class kvq_config(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32), ("value_bits", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("residual", ctypes.c_int32), ("hadamard", ctypes.c_int32),
         ("layout", ctypes.c_int32), ("sink", ctypes.c_int32), ("rope_theta", ctypes.c_float),
-        ("outliers", ctypes.c_int32), ("capacity", ctypes.c_int64),
+        ("outliers", ctypes.c_int32), ("page_tokens", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+        ("capacity", ctypes.c_int64),
     ]
 
 
 class kvq_cache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in BUFFER_NAMES] + [
         ("seq_len_host", ctypes.POINTER(ctypes.c_int64)), ("seq_len_dev", ctypes.c_void_p),
-        ("k_out", ctypes.c_void_p), ("v_out", ctypes.c_void_p)]
+        ("k_out", ctypes.c_void_p), ("v_out", ctypes.c_void_p),
+        ("page_table_host", ctypes.POINTER(ctypes.c_int32)), ("page_table_dev", ctypes.c_void_p)]
 
 
 def _load() -> ctypes.CDLL:
@@ -84,9 +86,9 @@ def kvq_status_string(status: int) -> str:
 def make_config(batch: int, num_q_heads: int, num_kv_heads: int, key_bits: int, value_bits: int, group_size: int,
                 residual: int, hadamard: int, capacity: int, head_dim: int = 128,
                 layout: int = KVQ_LAYOUT_TILE_V1, sink: int = 0, rope_theta: float = 0.0,
-                outliers: int = 0) -> kvq_config:
+                outliers: int = 0, page_tokens: int = 0, num_pages: int = 0) -> kvq_config:
     return kvq_config(batch, num_q_heads, num_kv_heads, head_dim, key_bits, value_bits, group_size, residual,
-                      hadamard, layout, sink, rope_theta, outliers, capacity)
+                      hadamard, layout, sink, rope_theta, outliers, page_tokens, num_pages, capacity)
 
 
 def _check(status: int, where: str) -> None:
@@ -113,9 +115,11 @@ def kvq_outlier_buffer_bytes(cfg: kvq_config) -> List[int]:
 
 class Cache:
     """Device buffers of the packed cache (allocated with torch) plus the host / device length mirrors,
-    and the two outlier buffers when the config has outliers = 1."""
+    the two outlier buffers when the config has outliers = 1, and with paged storage the page table
+    (``page_table_host``: numpy int32 [B][Hkv][capacity / page_tokens], by default unit u's page j at
+    pool page u * (capacity / page_tokens) + j; the caller may edit it in place before a call)."""
 
-    def __init__(self, cfg: kvq_config, device: str = "cuda"):
+    def __init__(self, cfg: kvq_config, device: str = "cuda", page_table: Optional[np.ndarray] = None):
         self.cfg = cfg
         sizes = kvq_cache_buffer_bytes(cfg)
         self.buffers = {n: torch.zeros(max(s, 16), dtype=torch.uint8, device=device) for n, s in zip(BUFFER_NAMES, sizes)}
@@ -127,11 +131,24 @@ class Cache:
                 self.sizes[n] = s
         self.seq_len_host = np.zeros(cfg.batch, np.int64)
         self.seq_len_dev = torch.zeros(cfg.batch, dtype=torch.int64, device=device)
+        self.page_table_host = None
+        self.page_table_dev = None
+        if cfg.page_tokens > 0:
+            per_unit = cfg.capacity // cfg.page_tokens
+            shape = (cfg.batch, cfg.num_kv_heads, per_unit)
+            if page_table is None:
+                page_table = np.arange(cfg.batch * cfg.num_kv_heads * per_unit, dtype=np.int32).reshape(shape)
+            self.page_table_host = np.ascontiguousarray(page_table, np.int32)
+            assert self.page_table_host.shape == shape
+            self.page_table_dev = torch.full((max(self.page_table_host.size, 4),), -1, dtype=torch.int32, device=device)
         self.c = kvq_cache(*(self.buffers[n].data_ptr() for n in BUFFER_NAMES),
                            self.seq_len_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
                            self.seq_len_dev.data_ptr(),
                            self.buffers["k_out"].data_ptr() if "k_out" in self.buffers else None,
-                           self.buffers["v_out"].data_ptr() if "v_out" in self.buffers else None)
+                           self.buffers["v_out"].data_ptr() if "v_out" in self.buffers else None,
+                           self.page_table_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+                           if self.page_table_host is not None else None,
+                           self.page_table_dev.data_ptr() if self.page_table_dev is not None else None)
 
     def view(self, name: str, dtype: torch.dtype) -> torch.Tensor:
         return self.buffers[name][: self.sizes[name]].view(dtype)

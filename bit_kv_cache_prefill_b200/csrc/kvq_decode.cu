@@ -294,19 +294,43 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   for (int m = 0; m < 8; ++m) bq[m][0] = bq[m][1] = 0u;
   float bias_col = 0.f;
 
-  const uint8_t* kc_ptr = reinterpret_cast<const uint8_t*>(a.k_codes + unit * a.tiles * (64 * KB)) +
-                          static_cast<int64_t>(first_token / kTile) * (256 * KB) + 16 * lane;
-  const uint8_t* vc_ptr = reinterpret_cast<const uint8_t*>(a.v_codes + unit * a.tiles * (64 * VB)) +
-                          static_cast<int64_t>(first_token / kTile) * (256 * VB) + 16 * lane;
-  const uint8_t* vs_ptr = reinterpret_cast<const uint8_t*>(a.v_scale + (unit * a.capacity + first_token) * VPT) + 16 * lane;
-  const uint8_t* vz_ptr = reinterpret_cast<const uint8_t*>(a.v_zero + (unit * a.capacity + first_token) * VPT) + 16 * lane;
-  const uint16_t* kp_src = (lane < 16 ? a.k_scale : a.k_zero) + unit * a.groups * kHeadDim + 8 * (lane & 15);
+  // Lane pointers of the step at token t: its storage slot (the unit, or with paged storage the pool
+  // page of its logical page) and in-slot token. A step never crosses a page (a page is a whole number
+  // of 128-token blocks), so with paged storage the pointers are re-based at every page start; the
+  // host has checked every table entry of the quantized part.
+  const uint8_t* kc_ptr = nullptr;
+  const uint8_t* vc_ptr = nullptr;
+  const uint8_t* vs_ptr = nullptr;
+  const uint8_t* vz_ptr = nullptr;
   const uint8_t* ko_ptr = nullptr;
   const uint8_t* vo_ptr = nullptr;
-  if constexpr (OUT) {
-    ko_ptr = reinterpret_cast<const uint8_t*>(a.k_out + unit * a.capacity + first_token) + 16 * lane;
-    vo_ptr = reinterpret_cast<const uint8_t*>(a.v_out + unit * a.capacity + first_token) + 16 * lane;
-  }
+  auto rebase = [&](int t) {
+    int64_t slot = unit, ts = t;
+    if (a.page_tokens > 0) {
+      slot = a.page_table[unit * a.pages_per_unit + t / a.page_tokens];
+      ts = t % a.page_tokens;
+    }
+    kc_ptr = reinterpret_cast<const uint8_t*>(a.k_codes + slot * a.tiles * (64 * KB)) + (ts / kTile) * (256 * KB) + 16 * lane;
+    vc_ptr = reinterpret_cast<const uint8_t*>(a.v_codes + slot * a.tiles * (64 * VB)) + (ts / kTile) * (256 * VB) + 16 * lane;
+    vs_ptr = reinterpret_cast<const uint8_t*>(a.v_scale + (slot * a.slot_tokens + ts) * VPT) + 16 * lane;
+    vz_ptr = reinterpret_cast<const uint8_t*>(a.v_zero + (slot * a.slot_tokens + ts) * VPT) + 16 * lane;
+    if constexpr (OUT) {
+      ko_ptr = reinterpret_cast<const uint8_t*>(a.k_out + slot * a.slot_tokens + ts) + 16 * lane;
+      vo_ptr = reinterpret_cast<const uint8_t*>(a.v_out + slot * a.slot_tokens + ts) + 16 * lane;
+    }
+  };
+  if (nst > 0) rebase(first_token);
+  // Key scale / zero row of key group g (g < q_groups) for this lane's 16-byte part.
+  const uint16_t* kp_base = (lane < 16 ? a.k_scale : a.k_zero) + 8 * (lane & 15);
+  auto kp_row = [&](int g) -> const uint16_t* {
+    int64_t slot = unit, gs = g;
+    if (a.page_tokens > 0) {
+      const int tg = g * G;
+      slot = a.page_table[unit * a.pages_per_unit + tg / a.page_tokens];
+      gs = (tg % a.page_tokens) / G;
+    }
+    return kp_base + (slot * a.groups + gs) * kHeadDim;
+  };
 
   // issue(i): step i of this warp into stage i % kStages (tracked by stage_in); the lane pointers
   // advance one step per call
@@ -314,6 +338,8 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(ring)) + 16 * lane;
   int stage_in = 0;
   auto issue = [&](int i) {
+    if (a.page_tokens > 0 && i > 0 && (first_token + i * kStepTokens) % a.page_tokens == 0)
+      rebase(first_token + i * kStepTokens);  // the step starts a new page
     const uint32_t st = ring_s + stage_in * S::kBytes;
     stage_in = stage_in == kStages - 1 ? 0 : stage_in + 1;
     cp_async16_at<S::oKC, 0>(st, kc_ptr);
@@ -344,7 +370,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
       for (int kg = 0; kg < KGB; ++kg) {
         const int g = blk * KGB + kg;
         const bool valid = g < q_groups;
-        cp_async16_zfill(kp + 512 * kg, kp_src + static_cast<int64_t>(valid ? g : 0) * kHeadDim, valid);
+        cp_async16_zfill(kp + 512 * kg, valid ? kp_row(g) : kp_base, valid);  // nothing is read when invalid
       }
     }
     kc_ptr += S::kKC;

@@ -130,9 +130,11 @@ constexpr int key_scratch_bytes() {
 // channel's min / max (as +inf for the min, -inf for the max), a channel whose entries in a group are
 // all outliers gets scale and zero 0, and after the parameters every outlier entry is overwritten with
 // its channel's zero, which codes to 0.
+// The block's tokens t0 .. t0 + nq - 1 are stored in slot `slot` from in-slot token ts0 on (the unit
+// and t0, or with paged storage the pool page and t0 mod page_tokens).
 template <int BITS, int LAYOUT, int G, bool OUT>
-__device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int nq, const uint16_t* rows, uint8_t* scratch,
-                          const uint8_t* och) {
+__device__ void key_block(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, int nq, const uint16_t* rows,
+                          uint8_t* scratch, const uint8_t* och) {
   constexpr int top = (1 << BITS) - 1;
   constexpr int P = 16 / BITS;  // code pairs per word
   const int NG = nq / G;
@@ -200,7 +202,7 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
       }
       const QuantParams p = all_out ? QuantParams{0.f, 0.f, 0, 0, true} : make_params(kmin, kmax, BITS);
       const int pos = LAYOUT == KVQ_LAYOUT_ROWS_V2 ? c : key_param_pos(c);
-      const int64_t pidx = (unit * a.groups + t0 / G + g) * kHeadDim + pos;
+      const int64_t pidx = (slot * a.groups + ts0 / G + g) * kHeadDim + pos;
       a.k_scale[pidx] = p.s16;
       a.k_zero[pidx] = p.z16;
       pz[g * 128 + c] = p.zf;
@@ -237,7 +239,7 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
       iv[i] = pinv[g * 128 + c0 + i];
       slow |= pcl[g * 128 + c0 + i] != 0;
     }
-    uint32_t* dst = a.k_codes + (unit * a.capacity + t0) * W + w;
+    uint32_t* dst = a.k_codes + (slot * a.slot_tokens + ts0) * W + w;
 #pragma unroll 2
     for (int it = 0; it < TPT; ++it) {
       const int t = tbase + STRIDE * it;
@@ -293,7 +295,7 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
     float zf[2 * NCP], iv[2 * NCP];
     bool slow = false;
     int gcur = -1;
-    uint32_t* dst = a.k_codes + (unit * a.tiles + t0 / kTile) * words + widx;
+    uint32_t* dst = a.k_codes + (slot * a.tiles + ts0 / kTile) * words + widx;
     for (int tl = tl0; tl < tl0 + ntl && tl * kTile < nq; ++tl) {
       const int g = (tl * kTile) / G;
       if (g != gcur) {
@@ -342,8 +344,8 @@ constexpr int val_scratch_bytes() {
 // With OUT, select_outliers has replaced each token's value outlier by its neighbour (so the min / max
 // leave it out); once the token's parameters are known the entry becomes its group's zero (code 0).
 template <int BITS, int LAYOUT, int G, bool OUT>
-__device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int nq, const uint16_t* rows, uint8_t* scratch,
-                            const uint8_t* och) {
+__device__ void value_block(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, int nq, const uint16_t* rows,
+                            uint8_t* scratch, const uint8_t* och) {
   constexpr int top = (1 << BITS) - 1;
   constexpr int P = 16 / BITS;
   constexpr int VPT = kHeadDim / G;
@@ -376,7 +378,7 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     QuantParams p = make_params(kmin, kmax, BITS);
     const bool sink_tok = a.sink && t0 + t == 0;  // the sink token: scale, zero and codes 0
     if (sink_tok) p = QuantParams{0.f, 0.f, 0, 0, true};
-    const int64_t pidx = (unit * a.capacity + t0 + t) * VPT + j;
+    const int64_t pidx = (slot * a.slot_tokens + ts0 + t) * VPT + j;
     a.v_scale[pidx] = p.s16;
     a.v_zero[pidx] = p.z16;
     prm[t * VPT + j] = make_float2(p.zf, p.inv);
@@ -426,7 +428,7 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     }
     __syncthreads();
     // 128 channel rows x nw words -> the block's rows (W words each), 16 bytes per thread-store
-    uint32_t* dst = a.v_codes + unit * a.vwords + (t0 / 128) * 128 * W;
+    uint32_t* dst = a.v_codes + slot * a.vwords + (ts0 / 128) * 128 * W;
     const int q4 = nw / 4;  // nw is a multiple of 4 when nq is a multiple of 16 * 4 / BITS ...
     if (q4 * 4 == nw) {
       for (int idx = tid; idx < 128 * q4; idx += kPThreads) {
@@ -456,7 +458,7 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     const int words = 64 * BITS;
     const int widx0 = (w >> 2) * 128 + 4 * L0 + (w & 3);  // lane L1 = L0 + 4: widx0 + 16
     const int ch0 = 16 * ((P * w) >> 2) + r0;              // channel of pair j: ch0 + 16 (j >> 2) + 8 (j & 1)
-    uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words + widx0;
+    uint32_t* dst = a.v_codes + (slot * a.tiles + ts0 / kTile) * words + widx0;
     for (int k = 0; k < TPT; ++k) {
       const int tl = 2 * (part + NPART * k) + half;
       if (tl * kTile >= nq) break;
@@ -542,16 +544,23 @@ __global__ void __launch_bounds__(kPThreads) prefill_block_kernel(QuantizeArgs a
     }
   }
   if (nq == 0) return;
+  // Storage slot of the block: the unit, or with paged storage the pool page of its logical page (a
+  // page is a whole number of 128-token blocks; the host has checked every entry that holds tokens).
+  int64_t slot = unit, ts0 = t0;
+  if (a.page_tokens > 0) {
+    slot = a.page_table[unit * a.pages_per_unit + t0 / a.page_tokens];
+    ts0 = t0 % a.page_tokens;
+  }
   uint8_t* och = scratch + scratch_bytes<BITS_K, BITS_V, LAYOUT, G>();
   if constexpr (OUT) {
-    select_outliers(rows, kRS, nq, (is_key ? a.k_out : a.v_out) + unit * a.capacity + t0, och, a.sink && t0 == 0,
-                    !is_key, kPThreads / 32);
+    select_outliers(rows, kRS, nq, (is_key ? a.k_out : a.v_out) + slot * a.slot_tokens + ts0, och,
+                    a.sink && t0 == 0, !is_key, kPThreads / 32);
     __syncthreads();
   }
   if (is_key)
-    key_block<BITS_K, LAYOUT, G, OUT>(a, unit, t0, nq, rows, scratch, och);
+    key_block<BITS_K, LAYOUT, G, OUT>(a, slot, ts0, t0, nq, rows, scratch, och);
   else
-    value_block<BITS_V, LAYOUT, G, OUT>(a, unit, t0, nq, rows, scratch, och);
+    value_block<BITS_V, LAYOUT, G, OUT>(a, slot, ts0, t0, nq, rows, scratch, och);
 }
 
 // Shared memory of one CTA: the rows, then the larger of the key and value scratch (and with OUT the

@@ -33,19 +33,21 @@ __device__ __forceinline__ uint32_t code_with(uint16_t x, float zf, float inv, i
   return __float_as_uint(__fadd_rn(v, 12582912.0f)) & 0xffu;
 }
 
-// Quantize G staged key rows (tokens t0 .. t0+G-1 of `unit`) and write key group t0/G.
+// Quantize G staged key rows (tokens t0 .. t0+G-1 of a unit, stored in slot `slot` from in-slot token
+// ts0 on: the unit and t0, or with paged storage the pool page and t0 mod page_tokens) and write their
+// key group.
 // All 256 threads work in every phase: min/max over token quarters for channel pairs, parameters per
 // channel, then one packed word per thread-iteration built straight from the fp16 rows.
 // With the outliers on, och[i] is row i's outlier channel: that entry stays out of its channel's
 // min / max, a channel whose entries are all outliers gets scale and zero 0, and the entry is then
 // overwritten with its channel's zero (code 0).
-__device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t t0, const uint16_t* rows,
+__device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, const uint16_t* rows,
                                     uint8_t* pbuf, const uint8_t* och) {
   const int G = a.G, bits = a.key_bits, top = (1 << bits) - 1;
   float2* prm = reinterpret_cast<float2*>(pbuf);                  // [128] (zf, inv)
   uint32_t* pmin = reinterpret_cast<uint32_t*>(pbuf + 128 * 8);   // [4][128]
   uint32_t* pmax = pmin + 4 * 128;                                // [4][128]
-  const int64_t g = t0 / G;
+  const int64_t g = ts0 / G;  // key group within the slot
   const bool sink0 = a.sink && t0 == 0;  // token 0 stays out of group 0 (min/max and codes)
   {
     const int cp = threadIdx.x & 63, tq = threadIdx.x >> 6;
@@ -77,7 +79,7 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
     // no entry outside the outliers: scale and zero 0
     const QuantParams p = kmin == 0xffffffffu ? QuantParams{0.f, 0.f, 0, 0, true} : make_params(kmin, kmax, bits);
     const int pos = a.layout == KVQ_LAYOUT_ROWS_V2 ? c : key_param_pos(c);  // rows v2: natural channel order
-    const int64_t pidx = (unit * a.groups + g) * kHeadDim + pos;
+    const int64_t pidx = (slot * a.groups + g) * kHeadDim + pos;
     a.k_scale[pidx] = p.s16;
     a.k_zero[pidx] = p.z16;
     prm[c] = make_float2(p.zf, p.inv);
@@ -96,7 +98,7 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
   if (a.layout == KVQ_LAYOUT_ROWS_V2) {
     // one row of 4*bits words per token: pair j = P*w + k holds channels 2j, 2j + 1
     const int wpt = 4 * bits;
-    uint32_t* dst2 = a.k_codes + (unit * a.capacity + t0) * wpt;
+    uint32_t* dst2 = a.k_codes + (slot * a.slot_tokens + ts0) * wpt;
     for (int idx = threadIdx.x; idx < G * wpt; idx += blockDim.x) {
       const int i = idx / wpt, w = idx % wpt;
       uint32_t word = 0;
@@ -111,7 +113,7 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
     }
     return;
   }
-  uint32_t* dst = a.k_codes + (unit * a.tiles + t0 / kTile) * words;
+  uint32_t* dst = a.k_codes + (slot * a.tiles + ts0 / kTile) * words;
   for (int idx = threadIdx.x; idx < (G / kTile) * words; idx += blockDim.x) {
     const int tile = idx / words, widx = idx % words;
     int lane, w;
@@ -132,7 +134,7 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
 // Quantize G staged value rows (per token, channel groups of G) and write their codes. With the
 // outliers on, each row's outlier entry has been replaced by its neighbour before (so the min / max
 // leave it out) and becomes its group's zero (code 0) once the parameters are known.
-__device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64_t t0, const uint16_t* rows,
+__device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, const uint16_t* rows,
                                       uint8_t* pbuf, const uint8_t* och) {
   const int G = a.G, bits = a.value_bits, top = (1 << bits) - 1;
   const int vpt = kHeadDim / G;
@@ -158,7 +160,7 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
     if (half == 0) {
       QuantParams p = make_params(kmin, kmax, bits);
       if (a.sink && t0 + i == 0) p = QuantParams{0.f, 0.f, 0, 0, true};  // the sink token: all zero
-      const int64_t pidx = (unit * a.capacity + t0 + i) * vpt + j;
+      const int64_t pidx = (slot * a.slot_tokens + ts0 + i) * vpt + j;
       a.v_scale[pidx] = p.s16;
       a.v_zero[pidx] = p.z16;
       prm[i * vpt + j] = make_float2(p.zf, p.inv);
@@ -171,9 +173,9 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
   if (a.layout == KVQ_LAYOUT_ROWS_V2) {
     // the chunk lies inside one 128-token block; channel c's row of that block gets G / (2P) words
     const int wpr = 4 * bits, wpc = G / (2 * P);
-    const int64_t block = t0 / 128;
-    const int ib = static_cast<int>(t0 % 128);
-    uint32_t* dst2 = a.v_codes + unit * a.vwords + block * 128 * wpr + (ib / 2) / P;
+    const int64_t block = ts0 / 128;
+    const int ib = static_cast<int>(ts0 % 128);
+    uint32_t* dst2 = a.v_codes + slot * a.vwords + block * 128 * wpr + (ib / 2) / P;
     for (int idx = threadIdx.x; idx < kHeadDim * wpc; idx += blockDim.x) {
       const int c = idx / wpc, w = idx % wpc;
       uint32_t word = 0;
@@ -187,7 +189,7 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
     }
     return;
   }
-  uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words;
+  uint32_t* dst = a.v_codes + (slot * a.tiles + ts0 / kTile) * words;
   for (int idx = threadIdx.x; idx < (G / kTile) * words; idx += blockDim.x) {
     const int tile = idx / words, widx = idx % words;
     int lane, w;
@@ -247,16 +249,23 @@ __global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint1
     reinterpret_cast<uint4*>(rows + i * kHeadDim)[part] = reinterpret_cast<const uint4*>(ring + slot * kHeadDim)[part];
   }
   __syncthreads();
+  // Storage slot of the group: the unit, or with paged storage the pool page of its logical page (a
+  // group never crosses a page; the host has checked the entry).
+  int64_t slot = unit, ts0 = Q_old;
+  if (a.page_tokens > 0) {
+    slot = a.page_table[unit * a.pages_per_unit + Q_old / a.page_tokens];
+    ts0 = Q_old % a.page_tokens;
+  }
   uint8_t* och = pbuf + kChunkParamBytes;
   if (a.outliers) {
-    select_outliers(rows, kHeadDim, G, (is_key ? a.k_out : a.v_out) + unit * a.capacity + Q_old, och,
+    select_outliers(rows, kHeadDim, G, (is_key ? a.k_out : a.v_out) + slot * a.slot_tokens + ts0, och,
                     a.sink && Q_old == 0, !is_key, blockDim.x / 32);
     __syncthreads();
   }
   if (is_key)
-    quantize_keys_chunk(a, unit, Q_old, rows, pbuf, och);
+    quantize_keys_chunk(a, slot, ts0, Q_old, rows, pbuf, och);
   else
-    quantize_values_chunk(a, unit, Q_old, rows, pbuf, och);
+    quantize_values_chunk(a, slot, ts0, Q_old, rows, pbuf, och);
 }
 
 __global__ void bump_lengths_kernel(int64_t* seq_len, int batch) {

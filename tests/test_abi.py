@@ -214,3 +214,74 @@ def test_decode_rejects_small_workspace_and_bad_scale():
     assert _status("kvq_decode_attention", *args, ctypes.c_float(float("nan")), 0x300000, need, None) == kvq.KVQ_ERR_INVALID_ARG
     assert _status("kvq_decode_attention", ctypes.byref(cfg), ctypes.byref(c), None, 0x200000, ctypes.c_float(0.1),
                    0x300000, need, None) == kvq.KVQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("P,pages,layout,theta,status", [
+    (128, 8, 1, 0.0, kvq.KVQ_OK), (512, 2, 1, 0.0, kvq.KVQ_OK), (1024, 1, 1, 0.0, kvq.KVQ_OK),
+    (64, 8, 1, 0.0, kvq.KVQ_ERR_INVALID_ARG),     # not a multiple of 128
+    (384, 8, 1, 0.0, kvq.KVQ_ERR_INVALID_ARG),    # does not divide the capacity
+    (128, 0, 1, 0.0, kvq.KVQ_ERR_INVALID_ARG),    # an empty pool
+    (-128, 8, 1, 0.0, kvq.KVQ_ERR_INVALID_ARG),
+    (128, 8, 2, 0.0, kvq.KVQ_ERR_UNSUPPORTED),    # paging exists for tile v1 only
+    (128, 8, 2, 10000.0, kvq.KVQ_ERR_UNSUPPORTED),
+])
+def test_paged_config_validation(P, pages, layout, theta, status):
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024, layout=layout, rope_theta=theta, page_tokens=P,
+                          num_pages=pages)
+    sizes = (ctypes.c_size_t * 8)()
+    assert _status("kvq_cache_buffer_bytes", ctypes.byref(cfg), sizes) == status
+
+
+@pytest.mark.parametrize("P,pages,outliers", [(128, 37, 0), (512, 5, 1), (256, 1000, 1)])
+def test_paged_buffer_bytes_are_pool_sized(P, pages, outliers):
+    # the six per-token buffers (and the outlier words) hold num_pages pages of P tokens; the fp16
+    # ring stays per unit
+    B, Hkv, G, R, cap = 3, 2, 32, 64, 2048
+    paged = kvq.make_config(B, 8, Hkv, 4, 2, G, R, 0, cap, outliers=outliers, page_tokens=P, num_pages=pages)
+    got = kvq.kvq_cache_buffer_bytes(paged)
+    want = [pages * P * 128 * 4 // 8, pages * P * 128 * 2 // 8, pages * (P // G) * 128 * 2,
+            pages * (P // G) * 128 * 2, pages * P * (128 // G) * 2, pages * P * (128 // G) * 2]
+    assert got[:6] == want
+    contiguous = kvq.make_config(B, 8, Hkv, 4, 2, G, R, 0, cap, outliers=outliers)
+    assert got[6:] == kvq.kvq_cache_buffer_bytes(contiguous)[6:]
+    assert kvq.kvq_outlier_buffer_bytes(paged) == ([pages * P * 4] * 2 if outliers else [0, 0])
+
+
+def _paged_fake_cache(cfg, lens, table):
+    c, host = _fake_cache(cfg, lens)
+    c.page_table_host = table.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    c.page_table_dev = 0xA0000
+    return c, host
+
+
+@pytest.mark.parametrize("bad", [-1, 4, 1 << 20])
+def test_paged_prefill_rejects_table_entries_outside_the_pool(bad):
+    # a page that would hold quantized tokens (T = 300, R = 32, G = 32: Q = 256, pages 0 and 1 of 128)
+    # must map into the pool; the call is refused on the host before anything is copied or launched
+    cfg = kvq.make_config(1, 2, 1, 2, 2, 32, 32, 0, 512, page_tokens=128, num_pages=4)
+    table = np.array([[[0, bad, -1, -1]]], np.int32)
+    c, _ = _paged_fake_cache(cfg, [0], table)
+    k = ctypes.c_void_p(0x100000)
+    lens = np.array([300], np.int64)
+    st = _lib.lib.kvq_quantize_prefill(ctypes.byref(cfg), ctypes.byref(c), k, k, 300 * 128, 128, 128,
+                                       lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_paged_append_and_decode_check_the_table():
+    # append: the flush that takes the quantized part into page 1 needs that page; decode: every page
+    # of the quantized part
+    cfg = kvq.make_config(1, 2, 1, 2, 2, 32, 32, 0, 512, page_tokens=128, num_pages=4)
+    table = np.array([[[2, -1, -1, -1]]], np.int32)
+    c, host = _paged_fake_cache(cfg, [159], table)  # Q = 96 -> 128 after this append: still page 0
+    kn = ctypes.c_void_p(0x100000)
+    host[0] = 191  # Q = 128 now; the append brings Q to 160, into page 1
+    assert _lib.lib.kvq_append_token(ctypes.byref(cfg), ctypes.byref(c), kn, kn, None) == kvq.KVQ_ERR_INVALID_ARG
+    host[0] = 200  # Q = 160: decode reads pages 0 and 1
+    ws = ctypes.c_void_p(0x200000)
+    st = _lib.lib.kvq_decode_attention(ctypes.byref(cfg), ctypes.byref(c), kn, kn, ctypes.c_float(0.1), ws,
+                                       1 << 30, None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+    c.page_table_host = None  # a paged cache without its table
+    host[0] = 0
+    assert _lib.lib.kvq_append_token(ctypes.byref(cfg), ctypes.byref(c), kn, kn, None) == kvq.KVQ_ERR_INVALID_ARG
