@@ -152,12 +152,12 @@ def reduce_over_ranks(dist, device, ms: float, *sums: float):
 
 
 def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode", sink: int = 0, rope: float = 0.0,
-                     outliers: int = 0):
+                     outliers: int = 0, page_tokens: int = 0):
     """DRAM bytes per launch of the decode-split (kind "decode") or bulk-prefill (kind "prefill")
     kernel from the committed ncu counters (profiles/decode_traffic_counters.txt, JSON), scaled from
     the captured batch to this one by the units processed; None if there is no capture for this
-    workload, layout, kernel and options (sink, RoPE, outliers; a record without them was taken with
-    them off) or the kernel sources changed since it was taken."""
+    workload, layout, kernel and options (sink, RoPE, outliers, pages; a record without them was taken
+    with them off) or the kernel sources changed since it was taken."""
     import hashlib
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "decode_traffic_counters.txt")
     try:
@@ -168,7 +168,8 @@ def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode", sink
     for e in entries.values():
         if e.get("workload") != w.name or e.get("layout") != layout or e.get("kind", "decode") != kind:
             continue
-        if e.get("sink", 0) != sink or e.get("rope_theta", 0.0) != rope or e.get("outliers", 0) != outliers:
+        if (e.get("sink", 0) != sink or e.get("rope_theta", 0.0) != rope or e.get("outliers", 0) != outliers
+                or e.get("page_tokens", 0) != page_tokens):
             continue
         h = hashlib.sha256()
         for f in e["kernel_sources"]:
@@ -245,7 +246,8 @@ def workload_config(w: inputs.Workload, args, step_bytes: int) -> dict:
             "num_kv_heads": w.num_kv_heads, "key_bits": w.key_bits, "value_bits": w.value_bits,
             "group_size": w.group_size, "residual": w.residual, "hadamard": w.hadamard,
             "ragged": bool(w.ragged_min), "parallelism": f"replicas{args.gpus}", "layout": args.layout,
-            "sink": args.sink, "rope_theta": args.rope, "outliers": args.outliers, "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
+            "sink": args.sink, "rope_theta": args.rope, "outliers": args.outliers,
+            "page_tokens": getattr(args, "page_tokens", 0), "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
 
 
 def run_reference(args, w):
@@ -298,6 +300,9 @@ def main():
                     help="1: keep every sequence's first token in fp16 (attention sink)")
     ap.add_argument("--rope", type=float, default=0.0,
                     help="> 0: cache keys before RoPE with this theta and rotate them in decode (needs --layout 2)")
+    ap.add_argument("--page-tokens", type=int, default=0,
+                    help="> 0: paged storage with pages of this many tokens (a multiple of 128; needs --layout 1); "
+                         "each unit's pages are consecutive pool pages")
     ap.add_argument("--outliers", type=int, default=0, choices=[0, 1],
                     help="1: keep each quantized token's largest key / value entry in fp16 (needs --layout 1)")
     args = ap.parse_args()
@@ -336,11 +341,14 @@ def main():
     kd, vd = k.cuda(), v.cuda()
     del k, v
     cap = w.capacity()
+    if args.page_tokens > 0:
+        cap = -(-cap // args.page_tokens) * args.page_tokens  # a whole number of pages
     if args.layout == 2:
         cap = -(-cap // 128) * 128  # rows v2 stores values in whole 128-token blocks
     cfg = kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size, w.residual,
                           w.hadamard, cap, layout=args.layout, sink=args.sink, rope_theta=args.rope,
-                          outliers=args.outliers)
+                          outliers=args.outliers, page_tokens=args.page_tokens,
+                          num_pages=w.batch * w.num_kv_heads * cap // max(args.page_tokens, 1) if args.page_tokens else 0)
     cache = kvq.Cache(cfg)
     stream = torch.cuda.current_stream()
 
@@ -472,14 +480,14 @@ def main():
         "decode_ms": round(mean_decode_ms, 4),
         "append_us": round(statistics.mean(append_ms) * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout, "decode", args.sink, args.rope, args.outliers), "peak_kind": peak_kind,
+                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout, "decode", args.sink, args.rope, args.outliers, args.page_tokens), "peak_kind": peak_kind,
                      "kernel": ("decode_rope_kernel" if args.rope > 0 else
                                 "decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
                      + " + decode_combine_kernel (one kvq_decode_attention call)"},
         "prefill": {"gbs": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9, 1),
                     "ms": round(statistics.mean(pre_ms), 3), "bytes": pre_bytes, "bound": "hbm", "peak": peak,
                     "frac": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9 / peak, 4),
-                    "traffic": measured_traffic(w0, args.layout, "prefill", args.sink, args.rope, args.outliers),
+                    "traffic": measured_traffic(w0, args.layout, "prefill", args.sink, args.rope, args.outliers, args.page_tokens),
                     "kernel": "prefill_block_kernel (one kvq_quantize_prefill call)"},
         # per step: append + length bump, then the decode split kernel + combine (+ the RoPE angle tables)
         "gpu_launches": (5 if args.rope > 0 else 4) * args.steps,
