@@ -10,8 +10,9 @@
 // Work split. The grid is (split, unit) with unit = (sequence, KV head). A CTA of 4 warps owns one
 // token range of split_len tokens; each warp owns a contiguous run of 16-token tiles of it (so a key
 // group's query fold is built once per group per warp) and round-robin the FP16 residual tokens.
-// Tiles stream through a per-warp 4-stage cp.async ring (codes, value scale/zero and, at a group
-// boundary, the group's key scale/zero) so about 4 tiles per warp are in flight.
+// Tiles stream through a per-warp 3-stage cp.async ring of steps of 1 or 2 tiles (codes, value
+// scale/zero and, at a key-block boundary, the block's key scale/zero), so up to 6 tiles per warp are
+// in flight.
 //
 // Arithmetic (per 16-token tile; scores in base-2 units, q already multiplied by sm_scale*log2 e):
 //   QK: s_t = 2^e * (sum_c code[t][c] * (q^[c] * sk[g][c]) + sum_c q^[c] * zk[g][c]), q^ = q * 2^-e.

@@ -285,3 +285,56 @@ def test_paged_append_and_decode_check_the_table():
     c.page_table_host = None  # a paged cache without its table
     host[0] = 0
     assert _lib.lib.kvq_append_token(ctypes.byref(cfg), ctypes.byref(c), kn, kn, None) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def _header_struct(name, path=os.path.join("include", "kvq.h")):
+    """Field (type, name) pairs of `typedef struct { ... } name;` in a C source, comments removed."""
+    text = open(os.path.join(ROOT, path)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    body = re.search(r"typedef struct \{([^{}]*)\}\s*" + name + r";", text).group(1)
+    fields = []
+    for decl in body.split(";"):  # "type name", "type* name" or "type a, b, c"
+        decl = decl.strip()
+        if decl:
+            base, rest = re.match(r"(\w+)\s*(.*)$", decl, flags=re.S).groups()
+            for d in rest.split(","):
+                d = d.strip()
+                name = d.lstrip("*").strip()
+                fields.append((base + "*" * (len(d) - len(d.lstrip("*"))), name))
+    return fields
+
+
+_CTYPE_OF = {"int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64, "float": ctypes.c_float}
+_SIZES = {"int32_t": 4, "float": 4, "int64_t": 8}
+
+
+def _oracle_structs():
+    import oracle
+    return [("kvq_ref_config", oracle._CConfig), ("kvq_ref_cache", oracle._CCache)]
+
+
+@pytest.mark.parametrize("name,binding,path", [
+    ("kvq_config", _lib.kvq_config, os.path.join("include", "kvq.h")),
+    ("kvq_cache", _lib.kvq_cache, os.path.join("include", "kvq.h")),
+    ("kvq_ref_config", "oracle", os.path.join("oracle", "kvq_oracle.cpp")),
+    ("kvq_ref_cache", "oracle", os.path.join("oracle", "kvq_oracle.cpp")),
+])
+def test_binding_structs_match_the_header(name, binding, path):
+    # the ctypes structs (library binding and oracle wrapper) must list the C struct's fields in the
+    # same order with the same types, and so have the same size: a drifted binding would pass every
+    # argument one field off
+    if binding == "oracle":
+        binding = dict(_oracle_structs())[name]
+    header = _header_struct(name, path)
+    assert [n for _, n in header] == [n for n, _ in binding._fields_]
+    for (ctype, fname), (_, btype) in zip(header, binding._fields_):
+        if ctype.endswith("*"):
+            assert btype is ctypes.c_void_p or issubclass(btype, ctypes._Pointer), fname
+        else:
+            assert btype is _CTYPE_OF[ctype], fname
+    off = 0
+    for ctype, _ in header:  # natural alignment, as the C compiler lays the struct out
+        sz = 8 if ctype.endswith("*") else _SIZES[ctype]
+        off = -(-off // sz) * sz + sz
+    assert ctypes.sizeof(binding) == -(-off // 8) * 8
