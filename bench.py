@@ -25,6 +25,7 @@ import subprocess
 import sys
 import threading
 import time
+from typing import List, NamedTuple, Optional
 
 import numpy as np
 import torch
@@ -78,6 +79,30 @@ def prefill_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0, outliers:
 
 def append_bytes(w: inputs.Workload) -> int:
     return 2 * w.batch * w.num_kv_heads * 128 * 2
+
+
+def flush_steps(w: inputs.Workload, lens_before: np.ndarray, steps: int) -> List[bool]:
+    """For each of `steps` appends starting from lengths lens_before: whether it flushes a group out
+    of the fp16 window in some sequence (its quantized length grows)."""
+    G, R = w.group_size, w.residual
+    q = lambda T: np.maximum(T - R, 0) // G * G  # noqa: E731
+    return [bool((q(lens_before + i + 1) > q(lens_before + i)).any()) for i in range(steps)]
+
+
+def kv_tokens(w: inputs.Workload, lens: np.ndarray) -> int:
+    """Cached (token, KV head) pairs one decode call scans."""
+    return int(np.asarray(lens, np.int64).sum()) * w.num_kv_heads
+
+
+def cpu_model() -> Optional[str]:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 # ---------------------------------------------------------------------------------------------------
@@ -193,12 +218,19 @@ def measured_hbm_peak():
 # ---------------------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------------------------------
+class OracleSample(NamedTuple):
+    gbs: float                          # algorithmic decode bytes / s, on `threads` threads
+    threads: int
+    sample: str                         # what was timed
+    single_thread_gbs: Optional[float]  # the same on one thread (when asked for)
+
+
 def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int = 1, sink: int = 0,
-                         rope: float = 0.0, outliers: int = 0):
+                         rope: float = 0.0, outliers: int = 0, single_thread_s: float = 0.0) -> OracleSample:
     """Time the oracle's decode on a bounded sample of the workload: whole (sequence, KV head) units
     batched into one oracle problem (enough units to give every host core a query head), decoded
-    repeatedly until about budget_s seconds have passed. Returns (GB/s of algorithmic decode bytes,
-    threads used, description of the sample)."""
+    repeatedly until about budget_s seconds have passed; with single_thread_s > 0, then on one thread
+    for about that long (at least one call)."""
     import oracle as ref
 
     cores = len(os.sched_getaffinity(0))
@@ -237,7 +269,17 @@ def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int
         calls += 1
     per_call = decode_bytes(w.scaled(batch=n, num_q_heads=g, num_kv_heads=1), lens, sink, outliers)
     desc = f"{n} (sequence, KV head) units of {w.name} ({int(lens.sum())} tokens), decode x{calls}"
-    return per_call * calls / spent / 1e9, threads, desc
+    single = None
+    if single_thread_s > 0:
+        st_calls, st_spent = 0, 0.0
+        while st_spent < single_thread_s or st_calls == 0:
+            t0 = time.perf_counter()
+            ref.decode(ocfg, oc, qs, 1 / math.sqrt(128), threads=1)
+            st_spent += time.perf_counter() - t0
+            st_calls += 1
+        single = per_call * st_calls / st_spent / 1e9
+        desc += f"; one thread: decode x{st_calls}"
+    return OracleSample(per_call * calls / spent / 1e9, threads, desc, single)
 
 
 def workload_config(w: inputs.Workload, args, step_bytes: int) -> dict:
@@ -262,10 +304,11 @@ def run_reference(args, w):
     per_step = []
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
-        gbs, cores, sample = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink, rope=args.rope,
-                                                  outliers=args.outliers)
+        res = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink, rope=args.rope,
+                                   outliers=args.outliers)
+        cores, sample = res.threads, res.sample
         if i >= args.warmup:
-            per_step.append(gbs)
+            per_step.append(res.gbs)
     value = statistics.mean(per_step)
     step_bytes = decode_bytes(w, lens, args.sink, args.outliers)
     line = {
@@ -273,7 +316,8 @@ def run_reference(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_bytes / (value * 1e9) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, args, step_bytes),
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -458,6 +502,10 @@ def main():
         return 0
 
     peak, peak_kind = measured_hbm_peak()
+    flush = flush_steps(w0, lens_before, args.steps)
+    app_flush = [a for a, f in zip(append_ms, flush) if f]
+    app_plain = [a for a, f in zip(append_ms, flush) if not f]
+    scanned = float(sum(kv_tokens(w0, lens_before + i + 1) for i in range(args.steps)))
     value = total_bytes / (total_ms * 1e-3) / 1e9
     mean_decode_ms = statistics.mean(decode_ms)
     achieved = statistics.mean(step_bytes) / (mean_decode_ms * 1e-3) / 1e9
@@ -479,12 +527,17 @@ def main():
         "frac_of_nominal_8tbs": round(value / NOMINAL_HBM_GBS, 4),
         "decode_ms": round(mean_decode_ms, 4),
         "append_us": round(statistics.mean(append_ms) * 1e3, 2),
+        # appends that flush a group out of the window in some sequence, and the others
+        "append_flush_us": round(statistics.mean(app_flush) * 1e3, 2) if app_flush else None,
+        "append_noflush_us": round(statistics.mean(app_plain) * 1e3, 2) if app_plain else None,
+        "kv_tokens_scanned_per_s": round(scanned / (sum(decode_ms) * 1e-3), 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout, "decode", args.sink, args.rope, args.outliers, args.page_tokens), "peak_kind": peak_kind,
                      "kernel": ("decode_rope_kernel" if args.rope > 0 else
                                 "decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
                      + " + decode_combine_kernel (one kvq_decode_attention call)"},
         "prefill": {"gbs": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9, 1),
+                    "elements_per_s": round(2 * 128 * kv_tokens(w0, lens0) / (statistics.mean(pre_ms) * 1e-3), 1),
                     "ms": round(statistics.mean(pre_ms), 3), "bytes": pre_bytes, "bound": "hbm", "peak": peak,
                     "frac": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9 / peak, 4),
                     "traffic": measured_traffic(w0, args.layout, "prefill", args.sink, args.rope, args.outliers, args.page_tokens),
@@ -499,10 +552,11 @@ def main():
         import oracle as ref
 
         ref.build()
-        gbs, cores, sample = oracle_decode_sample(w0, layout=args.layout, sink=args.sink, rope=args.rope,
-                                                  outliers=args.outliers)
-        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                                "sample": sample}
+        res = oracle_decode_sample(w0, layout=args.layout, sink=args.sink, rope=args.rope, outliers=args.outliers,
+                                   single_thread_s=3.0)
+        line["cpu_baseline"] = {"value": round(res.gbs, 4), "unit": "GB/s", "cores": res.threads, "kind": "oracle",
+                                "sample": res.sample, "single_thread_value": round(res.single_thread_gbs, 4),
+                                "cpu_model": cpu_model()}
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

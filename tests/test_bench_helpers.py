@@ -71,3 +71,21 @@ def test_traffic_lookup_is_none_for_other_layouts_and_kernels():
     assert bench.measured_traffic(w, 1, "decode", sink=1) is None
     assert bench.measured_traffic(w, 1, "prefill", sink=1) is None
     assert bench.measured_traffic(w, 2, "decode", rope=10000.0) is None
+
+
+def test_flush_steps_and_scanned_tokens():
+    # G = 32, R = 128: from T = 160 (Q = 32) the append that makes T = 192 flushes (Q 32 -> 64), then
+    # every 32nd append; with ragged lengths any sequence's flush counts
+    w = inputs.WORKLOADS["llama2_7b_mha"].scaled(batch=2)
+    flags = bench.flush_steps(w, np.array([160, 160]), 70)
+    assert [i for i, f in enumerate(flags) if f] == [31, 63]
+    flags = bench.flush_steps(w, np.array([160, 170]), 40)
+    assert [i for i, f in enumerate(flags) if f] == [21, 31]
+    assert not any(bench.flush_steps(w, np.array([10, 20]), 100))  # still inside the window (T < R + G)
+    assert bench.kv_tokens(w, np.array([100, 200])) == 300 * w.num_kv_heads
+
+
+def test_oracle_sample_reports_one_thread_time():
+    res = bench.oracle_decode_sample(inputs.WORKLOADS["tiny"], budget_s=0.05, single_thread_s=0.01)
+    assert res.gbs > 0 and res.threads >= 1 and res.single_thread_gbs > 0 and "one thread" in res.sample
+    assert bench.oracle_decode_sample(inputs.WORKLOADS["tiny"], budget_s=0.01).single_thread_gbs is None
