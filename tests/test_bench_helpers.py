@@ -88,4 +88,23 @@ def test_flush_steps_and_scanned_tokens():
 def test_oracle_sample_reports_one_thread_time():
     res = bench.oracle_decode_sample(inputs.WORKLOADS["tiny"], budget_s=0.05, single_thread_s=0.01)
     assert res.gbs > 0 and res.threads >= 1 and res.single_thread_gbs > 0 and "one thread" in res.sample
+    assert res.prefill_gbs > 0
     assert bench.oracle_decode_sample(inputs.WORKLOADS["tiny"], budget_s=0.01).single_thread_gbs is None
+
+
+def test_reference_arm_prints_one_line(capsys, monkeypatch):
+    # --impl reference on the tiny workload: the oracle timed on the host, one JSON line with the
+    # fields the line needs (the same metric and config keys as the GPU arm); each sample is cut short
+    import sys
+    real = bench.oracle_decode_sample
+    monkeypatch.setattr(bench, "oracle_decode_sample", lambda *a, **k: real(*a, **{**k, "budget_s": 0.05}))
+    argv = sys.argv
+    sys.argv = ["bench.py", "--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"]
+    try:
+        assert bench.main() == 0
+    finally:
+        sys.argv = argv
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["prefill_value"] > 0
+    assert line["config"]["workload"] == "tiny" and line["e2e"]["h2d_bytes_per_step"] == 0
