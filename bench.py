@@ -94,6 +94,26 @@ def kv_tokens(w: inputs.Workload, lens: np.ndarray) -> int:
     return int(np.asarray(lens, np.int64).sum()) * w.num_kv_heads
 
 
+def input_digest(*arrays) -> str:
+    """SHA-256 of the arrays' bytes in order (C-contiguous numpy arrays): names the exact synthetic
+    inputs a run used."""
+    import hashlib
+    h = hashlib.sha256()
+    for a in arrays:
+        h.update(memoryview(np.ascontiguousarray(a)))
+    return h.hexdigest()
+
+
+def append_summary(ms: List[float], flush: List[bool]) -> Optional[dict]:
+    """Mean µs of a run of appends, overall and split by whether the append flushed a group."""
+    if not ms:
+        return None
+    fl = [m for m, f in zip(ms, flush) if f]
+    pl = [m for m, f in zip(ms, flush) if not f]
+    us = lambda xs: round(statistics.mean(xs) * 1e3, 2) if xs else None  # noqa: E731
+    return {"n": len(ms), "mean_us": us(ms), "flush_us": us(fl), "n_flush": len(fl), "noflush_us": us(pl)}
+
+
 def cpu_model() -> Optional[str]:
     try:
         with open("/proc/cpuinfo") as f:
@@ -386,6 +406,7 @@ def main():
     w = w0.scaled(appends=n_app)
     lens0 = w0.seq_lens()
     k, v, _ = inputs.full_kv(w0)  # CPU, seeded
+    digest = input_digest(k.numpy(), v.numpy(), inputs.query(w0).numpy())
     kd, vd = k.cuda(), v.cuda()
     del k, v
     cap = w.capacity()
@@ -414,11 +435,17 @@ def main():
     del kd, vd
     torch.cuda.empty_cache()
 
-    # the workload's own streaming appends (e.g. 256 new tokens per sequence) before decode
-    for s in range(w0.appends):
-        kn, vn = inputs.append_tokens(w0, s)
-        kvq.kvq_append_token(cfg, cache, kn.cuda(), vn.cuda())
+    # the workload's own streaming appends (e.g. 256 new tokens per sequence) before decode, each
+    # timed with CUDA events on the stream (its inputs already on the device)
+    wl_app = [tuple(t.cuda() for t in inputs.append_tokens(w0, s)) for s in range(w0.appends)]
+    wl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in wl_app]
+    for (kn, vn), (ea, eb) in zip(wl_app, wl_ev):
+        ea.record(stream)
+        kvq.kvq_append_token(cfg, cache, kn, vn)
+        eb.record(stream)
     torch.cuda.synchronize()
+    wl_app_ms = [ea.elapsed_time(eb) for ea, eb in wl_ev]
+    del wl_app
 
     q = inputs.query(w0).cuda()
     out = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float16, device="cuda")
@@ -549,6 +576,9 @@ def main():
         # per step: append + length bump, then the decode split kernel + combine (+ the RoPE angle tables)
         "gpu_launches": (5 if args.rope > 0 else 4) * args.steps,
         "clocks": clocks.summary(),
+        "input_sha256": digest,  # prefill K, V (fp16 [B][T][Hkv][128], zero past each length) and q
+        # the workload's own appends before the timed steps (e.g. 256 per sequence), one event pair each
+        "workload_appends": append_summary(wl_app_ms, flush_steps(w0, lens0, len(wl_app_ms))),
     }
     if e2e is not None:
         line["e2e"] = e2e

@@ -108,3 +108,20 @@ def test_reference_arm_prints_one_line(capsys, monkeypatch):
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["prefill_value"] > 0
     assert line["config"]["workload"] == "tiny" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_input_digest_names_the_inputs():
+    w = inputs.WORKLOADS["tiny"]
+    k, v, _ = inputs.full_kv(w)
+    d1 = bench.input_digest(k.numpy(), v.numpy(), inputs.query(w).numpy())
+    k2, v2, _ = inputs.full_kv(w)  # the same seeds give the same bytes
+    assert bench.input_digest(k2.numpy(), v2.numpy(), inputs.query(w).numpy()) == d1
+    v2[0, 0, 0, 0] += 1
+    assert bench.input_digest(k2.numpy(), v2.numpy(), inputs.query(w).numpy()) != d1
+
+
+def test_append_summary():
+    assert bench.append_summary([], []) is None
+    got = bench.append_summary([0.004, 0.010, 0.006], [False, True, False])
+    assert got == {"n": 3, "mean_us": 6.67, "flush_us": 10.0, "n_flush": 1, "noflush_us": 5.0}
+    assert bench.append_summary([0.004], [False])["flush_us"] is None
