@@ -42,7 +42,7 @@ extern "C" {
 typedef enum {
   KVQ_OK = 0,
   KVQ_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned pointer, inconsistent config */
-  KVQ_ERR_UNSUPPORTED = -2, /* a configuration this build does not implement (e.g. head_dim != 128) */
+  KVQ_ERR_UNSUPPORTED = -2, /* a configuration the library does not implement (e.g. head_dim != 128) */
   KVQ_ERR_CAPACITY = -3,    /* a sequence would exceed config.capacity tokens */
   KVQ_ERR_WORKSPACE = -4,   /* workspace missing or smaller than kvq_decode_workspace_bytes */
   KVQ_ERR_CUDA = -5         /* a kernel launch or copy failed */
