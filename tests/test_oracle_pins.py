@@ -714,6 +714,26 @@ def test_outliers_are_each_tokens_largest_entry_kept_in_fp16(oracle_mod, layout)
     assert cache.k_out_ch[0, 1, 17] == 40 and cache.v_out_ch[0, 0, 20] == 3
 
 
+def test_outliers_are_chosen_on_the_rotated_keys(oracle_mod):
+    # with the Hadamard option the cache holds rotated keys (reading R2), so a key's outlier is the
+    # largest entry of the rotated fp16 key: rotate each input key with the pinned fp32 transform,
+    # round to fp16, and take the first largest magnitude; values are not rotated
+    B, T, Hkv, Hq, G, R = 1, 200, 1, 2, 32, 32
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 1, cap=224)
+    cfg.outliers = 1
+    k, v, q = _inputs(B, T, Hkv, Hq, 85)
+    cache = oracle_mod.Cache(cfg)
+    oracle_mod.quantize_prefill(cfg, cache, k, v, [T])
+    Q = (T - R) // G * G
+    rot = np.stack([oracle_mod.f32_to_f16(oracle_mod.wht128_f32(oracle_mod.f16_to_f32(k[0, t, 0]))) for t in range(Q)])
+    want = (rot & 0x7FFF).argmax(axis=1)
+    assert np.array_equal(cache.k_out_ch[0, 0, :Q], want)
+    assert np.array_equal(cache.k_out_val[0, 0, :Q], rot[np.arange(Q), want])
+    raw = (k[0, :Q, 0].view(np.uint16) & 0x7FFF).argmax(axis=1)
+    assert not np.array_equal(want, raw)  # the rotation moves the outliers (channels 5 and 77 are spread)
+    assert np.array_equal(cache.v_out_ch[0, 0, :Q], (v[0, :Q, 0].view(np.uint16) & 0x7FFF).argmax(axis=1))
+
+
 @pytest.mark.parametrize("layout", [1, 2])
 def test_outliers_left_out_of_group_statistics(oracle_mod, layout):
     # every key group's per-channel min / max and every value group's per-token min / max run over
@@ -894,12 +914,15 @@ def test_paged_shuffled_pool_gathers_to_the_contiguous_cache(oracle_mod, layout,
     assert np.array_equal(out_c, out_p)
 
 
+@pytest.mark.parametrize("outliers,sink", [(0, 0), (1, 1)])
 @pytest.mark.parametrize("layout", [1, 2])
-def test_paged_streaming_with_pages_allocated_on_demand(oracle_mod, layout):
+def test_paged_streaming_with_pages_allocated_on_demand(oracle_mod, layout, outliers, sink):
     # the caller hands out a page only when the quantized part first reaches it; streaming then
-    # equals a bulk prefill into the same pages, and a missing page is an argument error
+    # equals a bulk prefill into the same pages (outlier words and the sink row included), and a
+    # missing page is an argument error
     B, Hkv, Hq, G, R, P, cap = 1, 2, 2, 32, 32, 128, 512
-    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=cap, layout=layout)
+    cfg = _cfg(oracle_mod, B, Hq, Hkv, 2, 2, G, R, 0, cap=cap, layout=layout, sink=sink)
+    cfg.outliers = outliers
     cfg.page_tokens, cfg.num_pages = P, 16
     T0, n = 100, 300
     k, v, q = _inputs(B, T0 + n, Hkv, Hq, 92)
@@ -930,6 +953,8 @@ def test_paged_streaming_with_pages_allocated_on_demand(oracle_mod, layout):
         assert np.array_equal(getattr(stream, name), getattr(bulk, name)), name
     T, Q = T0 + n, oracle_mod.quantized_len(T0 + n, R, G)
     live = [t % (R + G) for t in range(Q, T)]  # ring slots that hold window tokens
+    if sink:
+        live.append(R + G)  # the first token's fp16 row
     for name in ("k_res", "v_res"):
         assert np.array_equal(getattr(stream, name)[:, :, live], getattr(bulk, name)[:, :, live]), name
     assert np.array_equal(oracle_mod.decode(cfg, stream, q, 0.1), oracle_mod.decode(cfg, bulk, q, 0.1))
