@@ -85,18 +85,21 @@ def host_cuda(monkeypatch):
     return calls, w
 
 
-def test_gpu_arm_host_logic_prints_a_complete_line(host_cuda, capsys, monkeypatch):
+@pytest.mark.parametrize("opts,launches", [([], 4), (["--layout", "2", "--sink", "1"], 4),
+                                           (["--layout", "2", "--rope", "10000"], 5)],
+                         ids=["tile_v1", "rows_v2_sink", "rows_v2_rope"])
+def test_gpu_arm_host_logic_prints_a_complete_line(host_cuda, capsys, monkeypatch, opts, launches):
     calls, w = host_cuda
     steps, warmup = 4, 3
     monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "hostpath", "--steps", str(steps),
-                                      "--warmup", str(warmup), "--prefill-iters", "2"])
+                                      "--warmup", str(warmup), "--prefill-iters", "2"] + opts)
     assert bench.main() == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "cpu_baseline", "e2e",
                 "gpu_launches", "clocks", "prefill", "input_sha256", "workload_appends"):
         assert key in line, key
-    assert line["metric"] == bench.METRIC and line["steps"] == steps and line["gpu_launches"] == 4 * steps
+    assert line["metric"] == bench.METRIC and line["steps"] == steps and line["gpu_launches"] == launches * steps
     assert set(line["roofline"]) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
     assert set(line["cpu_baseline"]) >= {"value", "unit", "cores", "kind", "sample"}
     assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
@@ -106,7 +109,7 @@ def test_gpu_arm_host_logic_prints_a_complete_line(host_cuda, capsys, monkeypatc
     assert line["workload_appends"]["n"] == 40
     # bytes per timed step from the lengths each decode saw: prefill 300 + 40 appends + warm-up
     lens = np.full(w.batch, 300 + 40 + warmup, np.int64)
-    want = sum(bench.decode_bytes(w, lens + i + 1) for i in range(steps))
+    want = sum(bench.decode_bytes(w, lens + i + 1, sink=1 if "--sink" in opts else 0) for i in range(steps))
     assert line["value"] == pytest.approx(want / (line["ms_per_step"] * steps * 1e-3) / 1e9, rel=1e-3)
     k, v, _ = inputs.full_kv(w)
     assert line["input_sha256"] == bench.input_digest(k.numpy(), v.numpy(), inputs.query(w).numpy())
