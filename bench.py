@@ -44,9 +44,10 @@ METRIC = "decode-attn effective KV HBM GB/s (fraction of B200 peak); tokens/s"
 # ---------------------------------------------------------------------------------------------------
 # algorithmic bytes (what the method must move), per unit of work
 # ---------------------------------------------------------------------------------------------------
-def decode_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
+def decode_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0, outliers: int = 0) -> int:
     """Bytes one decode call must read/write: packed codes + key group scale/zero + value token
-    scale/zero for the quantized tokens, fp16 K/V for the window (and for the first token when the
+    scale/zero for the quantized tokens (and with the outliers on, one 4-byte key and one value
+    outlier word per quantized token), fp16 K/V for the window (and for the first token when the
     sink is on), q in and out."""
     G, R = w.group_size, w.residual
     total = 0
@@ -56,12 +57,15 @@ def decode_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
         per_unit = Q * 128 * (w.key_bits + w.value_bits) // 8 + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4
         if sink and Q > 0:
             per_unit += 128 * 4
+        if outliers:
+            per_unit += Q * 8
         total += w.num_kv_heads * per_unit
     return total + 2 * w.batch * w.num_q_heads * 128 * 2
 
 
-def prefill_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
-    """fp16 K and V read + codes, scales, zero-points and window (and the sink row) written."""
+def prefill_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0, outliers: int = 0) -> int:
+    """fp16 K and V read + codes, scales, zero-points and window (and the sink row, and the outlier
+    words) written."""
     G, R = w.group_size, w.residual
     total = 0
     for T in lens:
@@ -69,7 +73,7 @@ def prefill_bytes(w: inputs.Workload, lens: np.ndarray, sink: int = 0) -> int:
         Q = max(T - R, 0) // G * G
         total += w.num_kv_heads * (T * 128 * 4 + Q * 128 * (w.key_bits + w.value_bits) // 8
                                    + (Q // G) * 128 * 4 + Q * (128 // G) * 4 + (T - Q) * 128 * 4
-                                   + (128 * 4 if sink and T > 0 else 0))
+                                   + (128 * 4 if sink and T > 0 else 0) + (Q * 8 if outliers else 0))
     return total
 
 
@@ -192,12 +196,13 @@ def reduce_over_ranks(dist, device, ms: float, *sums: float):
     return out
 
 
-def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode", sink: int = 0, rope: float = 0.0):
+def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode", sink: int = 0, rope: float = 0.0,
+                     outliers: int = 0, page_tokens: int = 0):
     """DRAM bytes per launch of the decode-split (kind "decode") or bulk-prefill (kind "prefill")
     kernel from the committed ncu counters (profiles/decode_traffic_counters.txt, JSON), scaled from
     the captured batch to this one by the units processed; None if there is no capture for this
-    workload, layout, kernel and options (sink, RoPE; a record without them was taken with them
-    off) or the kernel sources changed since it was taken."""
+    workload, layout, kernel and options (sink, RoPE, outliers, pages; a record without them was taken
+    with them off) or the kernel sources changed since it was taken."""
     import hashlib
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "decode_traffic_counters.txt")
     try:
@@ -208,7 +213,8 @@ def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode", sink
     for e in entries.values():
         if e.get("workload") != w.name or e.get("layout") != layout or e.get("kind", "decode") != kind:
             continue
-        if e.get("sink", 0) != sink or e.get("rope_theta", 0.0) != rope:
+        if (e.get("sink", 0) != sink or e.get("rope_theta", 0.0) != rope or e.get("outliers", 0) != outliers
+                or e.get("page_tokens", 0) != page_tokens):
             continue
         h = hashlib.sha256()
         for f in e["kernel_sources"]:
@@ -241,7 +247,7 @@ class OracleSample(NamedTuple):
 
 
 def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int = 1, sink: int = 0,
-                         rope: float = 0.0, single_thread_s: float = 0.0) -> OracleSample:
+                         rope: float = 0.0, outliers: int = 0, single_thread_s: float = 0.0) -> OracleSample:
     """Time the oracle's decode on a bounded sample of the workload: whole (sequence, KV head) units
     batched into one oracle problem (enough units to give every host core a query head), decoded
     repeatedly until about budget_s seconds have passed; with single_thread_s > 0, then on one thread
@@ -263,7 +269,7 @@ def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int
     if layout == 2:
         cap = -(-cap // 128) * 128
     ocfg = ref.Config(n, g, 1, w.key_bits, w.value_bits, w.group_size, w.residual, w.hadamard, cap,
-                      layout=layout, sink=sink, rope_theta=rope)
+                      layout=layout, sink=sink, rope_theta=rope, outliers=outliers)
     k = np.zeros((n, Tmax, 1, 128), np.float16)
     v = np.zeros_like(k)
     qs = np.zeros((n, g, 128), np.float16)
@@ -284,7 +290,7 @@ def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int
         ref.decode(ocfg, oc, qs, 1 / math.sqrt(128), threads=threads)
         spent += time.perf_counter() - t0
         calls += 1
-    per_call = decode_bytes(w.scaled(batch=n, num_q_heads=g, num_kv_heads=1), lens, sink)
+    per_call = decode_bytes(w.scaled(batch=n, num_q_heads=g, num_kv_heads=1), lens, sink, outliers)
     desc = f"{n} (sequence, KV head) units of {w.name} ({int(lens.sum())} tokens), decode x{calls}"
     single = None
     if single_thread_s > 0:
@@ -306,7 +312,8 @@ def workload_config(w: inputs.Workload, args, step_bytes: int) -> dict:
             "num_kv_heads": w.num_kv_heads, "key_bits": w.key_bits, "value_bits": w.value_bits,
             "group_size": w.group_size, "residual": w.residual, "hadamard": w.hadamard,
             "ragged": bool(w.ragged_min), "parallelism": f"replicas{args.gpus}", "layout": args.layout,
-            "sink": args.sink, "rope_theta": args.rope, "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
+            "sink": args.sink, "rope_theta": args.rope, "outliers": args.outliers,
+            "page_tokens": getattr(args, "page_tokens", 0), "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
 
 
 def run_reference(args, w):
@@ -321,12 +328,13 @@ def run_reference(args, w):
     per_step = []
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
-        res = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink, rope=args.rope)
+        res = oracle_decode_sample(w, budget_s=budget, layout=args.layout, sink=args.sink, rope=args.rope,
+                                   outliers=args.outliers)
         cores, sample, pre_gbs = res.threads, res.sample, res.prefill_gbs
         if i >= args.warmup:
             per_step.append(res.gbs)
     value = statistics.mean(per_step)
-    step_bytes = decode_bytes(w, lens, args.sink)
+    step_bytes = decode_bytes(w, lens, args.sink, args.outliers)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_bytes / (value * 1e9) * 1e3, 3),
@@ -360,6 +368,11 @@ def main():
                     help="1: keep every sequence's first token in fp16 (attention sink)")
     ap.add_argument("--rope", type=float, default=0.0,
                     help="> 0: cache keys before RoPE with this theta and rotate them in decode (needs --layout 2)")
+    ap.add_argument("--page-tokens", type=int, default=0,
+                    help="> 0: paged storage with pages of this many tokens (a multiple of 128; needs --layout 1); "
+                         "each unit's pages are consecutive pool pages")
+    ap.add_argument("--outliers", type=int, default=0, choices=[0, 1],
+                    help="1: keep each quantized token's largest key / value entry in fp16 (needs --layout 1)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w0 = inputs.WORKLOADS[args.workload]
@@ -397,10 +410,14 @@ def main():
     kd, vd = k.cuda(), v.cuda()
     del k, v
     cap = w.capacity()
+    if args.page_tokens > 0:
+        cap = -(-cap // args.page_tokens) * args.page_tokens  # a whole number of pages
     if args.layout == 2:
         cap = -(-cap // 128) * 128  # rows v2 stores values in whole 128-token blocks
     cfg = kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size, w.residual,
-                          w.hadamard, cap, layout=args.layout, sink=args.sink, rope_theta=args.rope)
+                          w.hadamard, cap, layout=args.layout, sink=args.sink, rope_theta=args.rope,
+                          outliers=args.outliers, page_tokens=args.page_tokens,
+                          num_pages=w.batch * w.num_kv_heads * cap // max(args.page_tokens, 1) if args.page_tokens else 0)
     cache = kvq.Cache(cfg)
     stream = torch.cuda.current_stream()
 
@@ -414,7 +431,7 @@ def main():
         torch.cuda.synchronize()
         if i > 0:
             pre_ms.append(e0.elapsed_time(e1))
-    pre_bytes = prefill_bytes(w0, lens0, args.sink)
+    pre_bytes = prefill_bytes(w0, lens0, args.sink, args.outliers)
     del kd, vd
     torch.cuda.empty_cache()
 
@@ -468,7 +485,7 @@ def main():
     decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
     append_ms = [e[0].elapsed_time(e[1]) for e in evs]
     # bytes per step from the lengths each decode actually saw (append happens first)
-    step_bytes = [decode_bytes(w0, lens_before + i + 1, args.sink) for i in range(args.steps)]
+    step_bytes = [decode_bytes(w0, lens_before + i + 1, args.sink, args.outliers) for i in range(args.steps)]
     total_bytes = float(sum(step_bytes))
     tokens = w.batch * args.steps
 
@@ -502,7 +519,7 @@ def main():
         e1.record(stream)
         barrier()
         e2e_ms = e0.elapsed_time(e1)
-        e2e_bytes = float(sum(decode_bytes(w0, lens_e + i + 1, args.sink) for i in range(args.steps)))
+        e2e_bytes = float(sum(decode_bytes(w0, lens_e + i + 1, args.sink, args.outliers) for i in range(args.steps)))
         e2e_ms, e2e_bytes = reduce_over_ranks(dist, "cuda", e2e_ms, e2e_bytes)
         h2d = in_host[0].numel() * 2
         d2h = out_host.numel() * 2
@@ -546,7 +563,7 @@ def main():
         "append_noflush_us": round(statistics.mean(app_plain) * 1e3, 2) if app_plain else None,
         "kv_tokens_scanned_per_s": round(scanned / (sum(decode_ms) * 1e-3), 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout, "decode", args.sink, args.rope), "peak_kind": peak_kind,
+                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout, "decode", args.sink, args.rope, args.outliers, args.page_tokens), "peak_kind": peak_kind,
                      "kernel": ("decode_rope_kernel" if args.rope > 0 else
                                 "decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
                      + " + decode_combine_kernel (one kvq_decode_attention call)"},
@@ -554,7 +571,7 @@ def main():
                     "elements_per_s": round(2 * 128 * kv_tokens(w0, lens0) / (statistics.mean(pre_ms) * 1e-3), 1),
                     "ms": round(statistics.mean(pre_ms), 3), "bytes": pre_bytes, "bound": "hbm", "peak": peak,
                     "frac": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9 / peak, 4),
-                    "traffic": measured_traffic(w0, args.layout, "prefill", args.sink, args.rope),
+                    "traffic": measured_traffic(w0, args.layout, "prefill", args.sink, args.rope, args.outliers, args.page_tokens),
                     "kernel": "prefill_block_kernel (one kvq_quantize_prefill call)"},
         # per step: append + length bump, then the decode split kernel + combine (+ the RoPE angle tables)
         "gpu_launches": (5 if args.rope > 0 else 4) * args.steps,
@@ -569,7 +586,8 @@ def main():
         import oracle as ref
 
         ref.build()
-        res = oracle_decode_sample(w0, layout=args.layout, sink=args.sink, rope=args.rope, single_thread_s=3.0)
+        res = oracle_decode_sample(w0, layout=args.layout, sink=args.sink, rope=args.rope, outliers=args.outliers,
+                                   single_thread_s=3.0)
         line["cpu_baseline"] = {"value": round(res.gbs, 4), "unit": "GB/s", "cores": res.threads, "kind": "oracle",
                                 "sample": res.sample, "single_thread_value": round(res.single_thread_gbs, 4),
                                 "prefill_value": round(res.prefill_gbs, 4), "cpu_model": cpu_model()}

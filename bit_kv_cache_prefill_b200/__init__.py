@@ -10,7 +10,7 @@ _BINDING_NAMES = {
     "KVQ_ERR_UNSUPPORTED", "KVQ_ERR_WORKSPACE", "KVQ_OK", "LIB_PATH", "kvq_append_token", "kvq_cache",
     "kvq_cache_buffer_bytes", "kvq_config", "kvq_decode_attention", "kvq_decode_workspace_bytes",
     "kvq_quantize_prefill", "kvq_status_string", "make_config", "kvq_decode_attention_noalloc",
-    "STATIC_SCRATCH_BYTES", "KVQ_LAYOUT_TILE_V1", "KVQ_LAYOUT_ROWS_V2",
+    "STATIC_SCRATCH_BYTES", "KVQ_LAYOUT_TILE_V1", "KVQ_LAYOUT_ROWS_V2", "kvq_outlier_buffer_bytes",
 }
 
 

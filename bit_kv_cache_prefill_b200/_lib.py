@@ -39,13 +39,16 @@ class kvq_config(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32), ("value_bits", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("residual", ctypes.c_int32), ("hadamard", ctypes.c_int32),
         ("layout", ctypes.c_int32), ("sink", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+        ("outliers", ctypes.c_int32), ("page_tokens", ctypes.c_int32), ("num_pages", ctypes.c_int32),
         ("capacity", ctypes.c_int64),
     ]
 
 
 class kvq_cache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in BUFFER_NAMES] + [
-        ("seq_len_host", ctypes.POINTER(ctypes.c_int64)), ("seq_len_dev", ctypes.c_void_p)]
+        ("seq_len_host", ctypes.POINTER(ctypes.c_int64)), ("seq_len_dev", ctypes.c_void_p),
+        ("k_out", ctypes.c_void_p), ("v_out", ctypes.c_void_p),
+        ("page_table_host", ctypes.POINTER(ctypes.c_int32)), ("page_table_dev", ctypes.c_void_p)]
 
 
 def _load() -> ctypes.CDLL:
@@ -56,6 +59,8 @@ def _load() -> ctypes.CDLL:
                        ctypes.c_int)
     L.kvq_cache_buffer_bytes.argtypes = [C, ctypes.POINTER(ctypes.c_size_t)]
     L.kvq_cache_buffer_bytes.restype = S
+    L.kvq_outlier_buffer_bytes.argtypes = [C, ctypes.POINTER(ctypes.c_size_t)]
+    L.kvq_outlier_buffer_bytes.restype = S
     L.kvq_quantize_prefill.argtypes = [C, K, P, P, I64, I64, I64, ctypes.POINTER(ctypes.c_int64), P]
     L.kvq_quantize_prefill.restype = S
     L.kvq_append_token.argtypes = [C, K, P, P, P]
@@ -80,9 +85,10 @@ def kvq_status_string(status: int) -> str:
 
 def make_config(batch: int, num_q_heads: int, num_kv_heads: int, key_bits: int, value_bits: int, group_size: int,
                 residual: int, hadamard: int, capacity: int, head_dim: int = 128,
-                layout: int = KVQ_LAYOUT_TILE_V1, sink: int = 0, rope_theta: float = 0.0) -> kvq_config:
+                layout: int = KVQ_LAYOUT_TILE_V1, sink: int = 0, rope_theta: float = 0.0,
+                outliers: int = 0, page_tokens: int = 0, num_pages: int = 0) -> kvq_config:
     return kvq_config(batch, num_q_heads, num_kv_heads, head_dim, key_bits, value_bits, group_size, residual,
-                      hadamard, layout, sink, rope_theta, capacity)
+                      hadamard, layout, sink, rope_theta, outliers, page_tokens, num_pages, capacity)
 
 
 def _check(status: int, where: str) -> None:
@@ -101,19 +107,48 @@ def kvq_cache_buffer_bytes(cfg: kvq_config) -> List[int]:
     return [int(x) for x in out]
 
 
-class Cache:
-    """Device buffers of the packed cache (allocated with torch) plus the host / device length mirrors."""
+def kvq_outlier_buffer_bytes(cfg: kvq_config) -> List[int]:
+    out = (ctypes.c_size_t * 2)()
+    _check(lib.kvq_outlier_buffer_bytes(ctypes.byref(cfg), out), "kvq_outlier_buffer_bytes")
+    return [int(x) for x in out]
 
-    def __init__(self, cfg: kvq_config, device: str = "cuda"):
+
+class Cache:
+    """Device buffers of the packed cache (allocated with torch) plus the host / device length mirrors,
+    the two outlier buffers when the config has outliers = 1, and with paged storage the page table
+    (``page_table_host``: numpy int32 [B][Hkv][capacity / page_tokens], by default unit u's page j at
+    pool page u * (capacity / page_tokens) + j; the caller may edit it in place before a call)."""
+
+    def __init__(self, cfg: kvq_config, device: str = "cuda", page_table: Optional[np.ndarray] = None):
         self.cfg = cfg
         sizes = kvq_cache_buffer_bytes(cfg)
         self.buffers = {n: torch.zeros(max(s, 16), dtype=torch.uint8, device=device) for n, s in zip(BUFFER_NAMES, sizes)}
         self.sizes = dict(zip(BUFFER_NAMES, sizes))
+        out_sizes = kvq_outlier_buffer_bytes(cfg)
+        for n, s in zip(("k_out", "v_out"), out_sizes):
+            if s:
+                self.buffers[n] = torch.zeros(s, dtype=torch.uint8, device=device)
+                self.sizes[n] = s
         self.seq_len_host = np.zeros(cfg.batch, np.int64)
         self.seq_len_dev = torch.zeros(cfg.batch, dtype=torch.int64, device=device)
+        self.page_table_host = None
+        self.page_table_dev = None
+        if cfg.page_tokens > 0:
+            per_unit = cfg.capacity // cfg.page_tokens
+            shape = (cfg.batch, cfg.num_kv_heads, per_unit)
+            if page_table is None:
+                page_table = np.arange(cfg.batch * cfg.num_kv_heads * per_unit, dtype=np.int32).reshape(shape)
+            self.page_table_host = np.ascontiguousarray(page_table, np.int32)
+            assert self.page_table_host.shape == shape
+            self.page_table_dev = torch.full((max(self.page_table_host.size, 4),), -1, dtype=torch.int32, device=device)
         self.c = kvq_cache(*(self.buffers[n].data_ptr() for n in BUFFER_NAMES),
                            self.seq_len_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
-                           self.seq_len_dev.data_ptr())
+                           self.seq_len_dev.data_ptr(),
+                           self.buffers["k_out"].data_ptr() if "k_out" in self.buffers else None,
+                           self.buffers["v_out"].data_ptr() if "v_out" in self.buffers else None,
+                           self.page_table_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+                           if self.page_table_host is not None else None,
+                           self.page_table_dev.data_ptr() if self.page_table_dev is not None else None)
 
     def view(self, name: str, dtype: torch.dtype) -> torch.Tensor:
         return self.buffers[name][: self.sizes[name]].view(dtype)

@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <vector>
 
 #include "kvq.h"
 #include "kvq_common.cuh"
@@ -38,6 +39,13 @@ kvq_status check_config(const kvq_config* c) {
   if (!(c->rope_theta >= 0.f) || !std::isfinite(c->rope_theta)) return KVQ_ERR_INVALID_ARG;
   if (c->rope_theta > 0.f && c->hadamard) return KVQ_ERR_INVALID_ARG;                 // the two exclude each other
   if (c->rope_theta > 0.f && c->layout != KVQ_LAYOUT_ROWS_V2) return KVQ_ERR_UNSUPPORTED;  // token-row keys only
+  if (c->outliers != 0 && c->outliers != 1) return KVQ_ERR_INVALID_ARG;
+  if (c->outliers && (c->layout != KVQ_LAYOUT_TILE_V1 || c->rope_theta > 0.f)) return KVQ_ERR_UNSUPPORTED;
+  if (c->page_tokens < 0) return KVQ_ERR_INVALID_ARG;
+  if (c->page_tokens > 0) {
+    if (c->page_tokens % 128 != 0 || c->capacity % c->page_tokens != 0 || c->num_pages < 1) return KVQ_ERR_INVALID_ARG;
+    if (c->layout != KVQ_LAYOUT_TILE_V1 || c->rope_theta > 0.f) return KVQ_ERR_UNSUPPORTED;
+  }
   if (c->capacity < 0 || c->capacity % G != 0) return KVQ_ERR_INVALID_ARG;
   if (c->capacity >= (int64_t(1) << 31)) return KVQ_ERR_INVALID_ARG;  // token indices are 32-bit on the device
   if (c->layout == KVQ_LAYOUT_ROWS_V2 && c->capacity % 128 != 0) return KVQ_ERR_INVALID_ARG;  // whole value blocks
@@ -45,16 +53,24 @@ kvq_status check_config(const kvq_config* c) {
   return KVQ_OK;
 }
 
+// Storage slots of the per-token buffers and tokens per slot: one slot of capacity tokens per unit,
+// or (paged) one slot of page_tokens tokens per pool page.
+size_t storage_slots(const kvq_config* c) {
+  return c->page_tokens > 0 ? static_cast<size_t>(c->num_pages) : static_cast<size_t>(c->batch) * c->num_kv_heads;
+}
+int64_t slot_tokens(const kvq_config* c) { return c->page_tokens > 0 ? c->page_tokens : c->capacity; }
+
 void buffer_bytes(const kvq_config* c, size_t out[KVQ_NUM_BUFFERS]) {
   const size_t units = static_cast<size_t>(c->batch) * c->num_kv_heads;
-  const size_t cap = static_cast<size_t>(c->capacity);
+  const size_t slots = storage_slots(c);
+  const size_t cap = static_cast<size_t>(slot_tokens(c));
   const size_t G = static_cast<size_t>(c->group_size);
-  out[KVQ_BUF_K_CODES] = units * (cap / 16) * 64 * c->key_bits * 4;
+  out[KVQ_BUF_K_CODES] = slots * (cap / 16) * 64 * c->key_bits * 4;
   const size_t vcap = c->layout == KVQ_LAYOUT_ROWS_V2 ? (cap + 127) / 128 * 128 : cap;
-  out[KVQ_BUF_V_CODES] = units * (vcap / 16) * 64 * c->value_bits * 4;
-  out[KVQ_BUF_K_SCALE] = units * (cap / G) * 128 * 2;
+  out[KVQ_BUF_V_CODES] = slots * (vcap / 16) * 64 * c->value_bits * 4;
+  out[KVQ_BUF_K_SCALE] = slots * (cap / G) * 128 * 2;
   out[KVQ_BUF_K_ZERO] = out[KVQ_BUF_K_SCALE];
-  out[KVQ_BUF_V_SCALE] = units * cap * (128 / G) * 2;
+  out[KVQ_BUF_V_SCALE] = slots * cap * (128 / G) * 2;
   out[KVQ_BUF_V_ZERO] = out[KVQ_BUF_V_SCALE];
   out[KVQ_BUF_K_RES] = units * (static_cast<size_t>(c->residual) + G + c->sink) * 128 * 2;
   out[KVQ_BUF_V_RES] = out[KVQ_BUF_K_RES];
@@ -70,7 +86,36 @@ kvq_status check_cache(const kvq_config* c, const kvq_cache* k) {
     if (p[i] == nullptr || !aligned(p[i], 16)) return KVQ_ERR_INVALID_ARG;
   }
   if (!aligned(k->seq_len_dev, 8)) return KVQ_ERR_INVALID_ARG;
+  if (c->outliers && (k->k_out == nullptr || k->v_out == nullptr || !aligned(k->k_out, 16) || !aligned(k->v_out, 16)))
+    return KVQ_ERR_INVALID_ARG;
+  if (c->page_tokens > 0 && (k->page_table_host == nullptr || k->page_table_dev == nullptr || !aligned(k->page_table_dev, 16)))
+    return KVQ_ERR_INVALID_ARG;
   return KVQ_OK;
+}
+
+int64_t pages_per_unit(const kvq_config* c) { return c->page_tokens > 0 ? c->capacity / c->page_tokens : 0; }
+
+// Paged storage: every page that holds quantized tokens of a sequence of lens[b] tokens must map to a
+// page of the pool (the kernels read exactly those table entries).
+kvq_status check_pages(const kvq_config* c, const kvq_cache* k, const int64_t* lens) {
+  if (c->page_tokens <= 0) return KVQ_OK;
+  const int64_t M = pages_per_unit(c);
+  for (int b = 0; b < c->batch; ++b) {
+    const int64_t Q = kvq::quantized_len(lens[b], c->residual, c->group_size);
+    const int64_t used = (Q + c->page_tokens - 1) / c->page_tokens;
+    for (int h = 0; h < c->num_kv_heads; ++h) {
+      const int32_t* row = k->page_table_host + (static_cast<int64_t>(b) * c->num_kv_heads + h) * M;
+      for (int64_t j = 0; j < used; ++j)
+        if (row[j] < 0 || row[j] >= c->num_pages) return KVQ_ERR_INVALID_ARG;
+    }
+  }
+  return KVQ_OK;
+}
+
+// Copy the whole page table to its device mirror on the stream.
+cudaError_t upload_pages(const kvq_config* c, const kvq_cache* k, cudaStream_t stream) {
+  const size_t bytes = static_cast<size_t>(c->batch) * c->num_kv_heads * pages_per_unit(c) * sizeof(int32_t);
+  return cudaMemcpyAsync(k->page_table_dev, k->page_table_host, bytes, cudaMemcpyHostToDevice, stream);
 }
 
 QuantizeArgs quantize_args(const kvq_config* c, kvq_cache* k) {
@@ -93,13 +138,20 @@ QuantizeArgs quantize_args(const kvq_config* c, kvq_cache* k) {
   a.value_bits = c->value_bits;
   a.hadamard = c->hadamard;
   a.capacity = c->capacity;
-  a.tiles = c->capacity / kvq::kTile;
-  a.groups = c->capacity / c->group_size;
+  a.slot_tokens = slot_tokens(c);
+  a.tiles = a.slot_tokens / kvq::kTile;
+  a.groups = a.slot_tokens / c->group_size;
   a.ring = static_cast<int64_t>(c->residual) + c->group_size;
   a.layout = c->layout;
+  a.page_tokens = c->page_tokens;
+  a.pages_per_unit = pages_per_unit(c);
+  a.page_table = k->page_table_dev;
   a.sink = c->sink;
   a.res_rows = a.ring + c->sink;
-  a.vwords = (c->layout == KVQ_LAYOUT_ROWS_V2 ? (c->capacity + 127) / 128 * 128 : c->capacity) * 4 * c->value_bits;
+  a.outliers = c->outliers;
+  a.k_out = static_cast<uint32_t*>(k->k_out);
+  a.v_out = static_cast<uint32_t*>(k->v_out);
+  a.vwords = (c->layout == KVQ_LAYOUT_ROWS_V2 ? (a.slot_tokens + 127) / 128 * 128 : a.slot_tokens) * 4 * c->value_bits;
   return a;
 }
 
@@ -157,6 +209,15 @@ kvq_status kvq_cache_buffer_bytes(const kvq_config* cfg, size_t out_bytes[KVQ_NU
   return KVQ_OK;
 }
 
+kvq_status kvq_outlier_buffer_bytes(const kvq_config* cfg, size_t out_bytes[2]) {
+  const kvq_status s = check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (out_bytes == nullptr) return KVQ_ERR_INVALID_ARG;
+  const size_t n = cfg->outliers ? storage_slots(cfg) * static_cast<size_t>(slot_tokens(cfg)) * 4 : 0;
+  out_bytes[0] = out_bytes[1] = n;
+  return KVQ_OK;
+}
+
 kvq_status kvq_quantize_prefill(const kvq_config* cfg, kvq_cache* cache, const void* k, const void* v, int64_t stride_b,
                                 int64_t stride_t, int64_t stride_h, const int64_t* seq_lens, void* cuda_stream) {
   kvq_status s = check_config(cfg);
@@ -172,11 +233,13 @@ kvq_status kvq_quantize_prefill(const kvq_config* cfg, kvq_cache* cache, const v
     if (k == nullptr || v == nullptr || !aligned(k, 16) || !aligned(v, 16)) return KVQ_ERR_INVALID_ARG;
     if (stride_b < 0 || stride_t < 0 || stride_h < 0 || stride_b % 8 || stride_t % 8 || stride_h % 8) return KVQ_ERR_INVALID_ARG;
   }
+  if ((s = check_pages(cfg, cache, seq_lens)) != KVQ_OK) return s;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   std::memcpy(cache->seq_len_host, seq_lens, sizeof(int64_t) * cfg->batch);
   cudaError_t e = cudaMemcpyAsync(cache->seq_len_dev, cache->seq_len_host, sizeof(int64_t) * cfg->batch,
                                   cudaMemcpyHostToDevice, stream);
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cfg->page_tokens > 0 && upload_pages(cfg, cache, stream) != cudaSuccess) return KVQ_ERR_CUDA;
   QuantizeArgs a = quantize_args(cfg, cache);
   a.k = static_cast<const uint16_t*>(k);
   a.v = static_cast<const uint16_t*>(v);
@@ -194,6 +257,20 @@ kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache, const void*
   if (k_new == nullptr || v_new == nullptr || !aligned(k_new, 16) || !aligned(v_new, 16)) return KVQ_ERR_INVALID_ARG;
   for (int b = 0; b < cfg->batch; ++b)
     if (cache->seq_len_host[b] < 0 || cache->seq_len_host[b] + 1 > cfg->capacity) return KVQ_ERR_CAPACITY;
+  if (cfg->page_tokens > 0) {
+    // The flush of this append may enter a new page: check the table for the new lengths and, if
+    // some unit's quantized part reaches a page it did not reach before, refresh the device mirror.
+    std::vector<int64_t> next(cache->seq_len_host, cache->seq_len_host + cfg->batch);
+    bool enters = false;
+    for (int b = 0; b < cfg->batch; ++b) {
+      const int64_t q0 = kvq::quantized_len(next[b], cfg->residual, cfg->group_size);
+      const int64_t q1 = kvq::quantized_len(next[b] + 1, cfg->residual, cfg->group_size);
+      enters |= (q1 + cfg->page_tokens - 1) / cfg->page_tokens > (q0 + cfg->page_tokens - 1) / cfg->page_tokens;
+      next[b] += 1;
+    }
+    if ((s = check_pages(cfg, cache, next.data())) != KVQ_OK) return s;
+    if (enters && upload_pages(cfg, cache, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return KVQ_ERR_CUDA;
+  }
   QuantizeArgs a = quantize_args(cfg, cache);
   const kvq_status r = cuda_status(kvq::launch_append(a, static_cast<const uint16_t*>(k_new),
                                                       static_cast<const uint16_t*>(v_new),
@@ -227,6 +304,7 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return KVQ_ERR_WORKSPACE;
   for (int b = 0; b < cfg->batch; ++b)
     if (cache->seq_len_host[b] < 0 || cache->seq_len_host[b] > cfg->capacity) return KVQ_ERR_INVALID_ARG;
+  if ((s = check_pages(cfg, cache, cache->seq_len_host)) != KVQ_OK) return s;
 
   static kvq::DeviceMemo sm_count;
   const int sms = sm_count.get([] {
@@ -240,7 +318,7 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
                   : cfg->layout == KVQ_LAYOUT_ROWS_V2
                       ? kvq::decode_tc_ctas_per_sm(cfg->group_size, cfg->num_q_heads / cfg->num_kv_heads)
                       : kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size,
-                                                cfg->num_q_heads / cfg->num_kv_heads);
+                                                cfg->num_q_heads / cfg->num_kv_heads, cfg->outliers);
   int nsplit = 1;
   const int L = plan_splits(cfg, cache->seq_len_host, sms * occ, &nsplit);
 
@@ -268,11 +346,18 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   a.value_bits = cfg->value_bits;
   a.hadamard = cfg->hadamard;
   a.capacity = cfg->capacity;
-  a.tiles = cfg->capacity / kvq::kTile;
-  a.groups = cfg->capacity / cfg->group_size;
+  a.slot_tokens = slot_tokens(cfg);
+  a.tiles = a.slot_tokens / kvq::kTile;
+  a.groups = a.slot_tokens / cfg->group_size;
+  a.page_tokens = cfg->page_tokens;
+  a.pages_per_unit = pages_per_unit(cfg);
+  a.page_table = cache->page_table_dev;
   a.ring = static_cast<int64_t>(cfg->residual) + cfg->group_size;
   a.sink = cfg->sink;
   a.res_rows = a.ring + cfg->sink;
+  a.outliers = cfg->outliers;
+  a.k_out = static_cast<const uint32_t*>(cache->k_out);
+  a.v_out = static_cast<const uint32_t*>(cache->v_out);
   a.layout = cfg->layout;
   a.split_len = L;
   a.nsplit = nsplit;

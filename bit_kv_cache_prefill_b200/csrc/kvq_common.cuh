@@ -86,6 +86,38 @@ __device__ __forceinline__ int key_param_pos(int c) {
   return 32 * qd + 4 * m + 2 * hh + e;
 }
 
+// --- dense-and-sparse outliers ------------------------------------------------------------------------
+// KVQuant review, Method: a small share of the entries stays in fp16, chosen per vector. For each of
+// the n staged rows (stride `stride` halves), the entry of largest magnitude, ties to the lowest
+// channel: fp16 magnitudes order like the integers of their low 15 bits, so the wanted entry has the
+// largest (|x| bits << 7) | (127 - channel). One warp per row (nwarps warps take part); the lane holding
+// the entry records its channel in och[i] (0xff: none, which is row 0 when `sink_first`) and the word
+// channel | fp16 value << 16 in out[i] (0xffff: none). With `replace` the entry is then overwritten
+// with its neighbour ch ^ 1, which lies in the same value group (G is even), so that group's min / max
+// become those of its other entries.
+__device__ __forceinline__ void select_outliers(uint16_t* rows, int stride, int n, uint32_t* out, uint8_t* och,
+                                                bool sink_first, bool replace, int nwarps) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = warp; i < n; i += nwarps) {
+    const uint2 x = *reinterpret_cast<const uint2*>(rows + i * stride + 4 * lane);
+    const uint32_t h[4] = {x.x & 0xffffu, x.x >> 16, x.y & 0xffffu, x.y >> 16};
+    uint32_t key = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) key = max(key, ((h[e] & 0x7fffu) << 7) | (127u - (4 * lane + e)));
+    key = __reduce_max_sync(0xffffffffu, key);
+    const int ch = 127 - static_cast<int>(key & 127u);
+    if (lane == (ch >> 2)) {
+      const bool none = sink_first && i == 0;
+      const int e = ch & 3;
+      const uint32_t val = e == 0 ? h[0] : e == 1 ? h[1] : e == 2 ? h[2] : h[3];
+      const uint32_t nbr = e == 0 ? h[1] : e == 1 ? h[0] : e == 2 ? h[3] : h[2];
+      och[i] = none ? 0xffu : static_cast<uint8_t>(ch);
+      out[i] = none ? 0xffffu : (static_cast<uint32_t>(ch) | (val << 16));
+      if (replace && !none) rows[i * stride + ch] = static_cast<uint16_t>(nbr);
+    }
+  }
+}
+
 // --- 128-point Walsh-Hadamard rotation ----------------------------------------------------------------
 // Sylvester-ordered butterflies with strides 1, 2, ..., 64 (pair (i, i+h) -> (a+b, a-b)) in fp32,
 // then one multiply by fp32(1/sqrt(128)) (bit pattern 0x3DB504F3). The framework page (In practice)

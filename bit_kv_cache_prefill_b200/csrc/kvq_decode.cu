@@ -77,8 +77,8 @@ __device__ __forceinline__ void cp_async_wait() {
 // so a new block's parameters may land in the slot of the block two back only once that block's
 // first step has been consumed: with kBlockSteps >= 2 this holds for two slots (a partial first
 // block plus a full block lie in between); one-step blocks use four slots (three blocks lie in
-// between).
-template <int KB, int VB, int VPT, int KGB, int TS>
+// between). With OUT a stage also holds the key and value outlier words of the step's tokens.
+template <int KB, int VB, int VPT, int KGB, int TS, bool OUT>
 struct Stage {
   static constexpr int kKC = 256 * KB * TS;  // key codes of the step's tiles
   static constexpr int kVC = 256 * VB * TS;  // value codes
@@ -87,7 +87,10 @@ struct Stage {
   static constexpr int oVC = oKC + kKC;
   static constexpr int oVS = oVC + kVC;
   static constexpr int oVZ = oVS + kVS;
-  static constexpr int kBytes = oVZ + kVS;
+  static constexpr int kKO = OUT ? 64 * TS : 0;  // key (or value) outlier words of the step's tokens
+  static constexpr int oKO = oVZ + kVS;
+  static constexpr int oVO = oKO + kKO;
+  static constexpr int kBytes = oVO + kKO;
   static constexpr int kKP = 512 * KGB;  // key scale[128] + zero[128] per group of the block
   static constexpr int kBlockSteps = (128 / VPT) * KGB / (16 * TS);
   static constexpr int kKPSlots = kBlockSteps >= 2 ? 2 : 4;
@@ -105,21 +108,28 @@ constexpr int kCmO = 4;    // offset of o[] within a shared-memory partial
 constexpr int kSmemEpilogue = kDecodeWarps * 4 * kCm * 4 + kDecodeWarps * 4 * 8 * 4;
 static_assert(kSmemFixed % 16 == 0, "stage ring must start 16-byte aligned");
 
-template <int KB, int VB, int VPT, int GQ>
+template <int KB, int VB, int VPT, int GQ, bool OUT>
 struct Shape {
   static constexpr int KGB = 4 / GQ;                     // key groups per QK B block
   static constexpr int VGB = 4 / GQ;                     // value groups per PV n-block
   static constexpr int NBV = (VPT + VGB - 1) / VGB;      // PV n-blocks
   static constexpr int G = 128 / VPT;
   static constexpr int TS = G >= 32 ? 2 : 1;             // tiles per step
-  using S = Stage<KB, VB, VPT, KGB, TS>;
+  using S = Stage<KB, VB, VPT, KGB, TS, OUT>;
 };
 
-template <int KB, int VB, int VPT, int GQ>
-constexpr int decode_smem_bytes() {
-  using S = typename Shape<KB, VB, VPT, GQ>::S;
+// With OUT, the per-warp outlier corrections of the value sum [W][4][128] f32 follow the ring /
+// epilogue area (they live through both).
+constexpr int kSmemCorr = kDecodeWarps * 4 * 128 * 4;
+template <int KB, int VB, int VPT, int GQ, bool OUT>
+constexpr int decode_corr_offset() {
+  using S = typename Shape<KB, VB, VPT, GQ, OUT>::S;
   constexpr int ring = kDecodeWarps * S::kWarpBytes;
   return kSmemFixed + (ring > kSmemEpilogue ? ring : kSmemEpilogue);
+}
+template <int KB, int VB, int VPT, int GQ, bool OUT>
+constexpr int decode_smem_bytes() {
+  return decode_corr_offset<KB, VB, VPT, GQ, OUT>() + (OUT ? kSmemCorr : 0);
 }
 
 // cp.async of 16 bytes that writes zeros (and reads nothing) when `valid` is false.
@@ -170,9 +180,15 @@ __device__ __forceinline__ void tile_scores(const uint8_t* kc, int lane, const u
 // With GQ = 4 every column is a (head, part) of one group; with GQ = 1 one B fragment covers 4 key
 // groups (QK) or 4 value groups (PV), so the per-group B rebuild is shared by 4 groups.
 // A lane (r, qd) of a D fragment holds columns 2qd, 2qd + 1, i.e. (group offset qd / GQ, head qd % GQ).
-template <int KB, int VB, int VPT, int GQ>
+//
+// OUT: dense-and-sparse outliers (KVQuant review, Method). Each quantized token's key and value keep
+// one fp16 entry (channel, value); its code is 0, so the packed path dequantizes it to the group's
+// zero. The score of the token gets q~[ch] * (k_out - zk[g][ch]) added before the softmax, and the
+// value sum gets p * (v_out - zv[t][ch / G]) at channel ch, gathered per warp in shared memory
+// (rescaled with the running max like the accumulators) and added to the warp partial at the end.
+template <int KB, int VB, int VPT, int GQ, bool OUT>
 __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a) {
-  using SH = Shape<KB, VB, VPT, GQ>;
+  using SH = Shape<KB, VB, VPT, GQ, OUT>;
   using S = typename SH::S;
   constexpr int KGB = SH::KGB, VGB = SH::VGB, NBV = SH::NBV, G = SH::G, TS = SH::TS;
   constexpr int kBlockTokens = G * KGB;
@@ -197,6 +213,12 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   const int end = min(start + L, T);
   const int Q = static_cast<int>(quantized_len(T, a.R, G));
   const int qend = min(end, Q);
+  float* corr = reinterpret_cast<float*>(smem + decode_corr_offset<KB, VB, VPT, GQ, OUT>()) + warp * 4 * kHeadDim;
+  if constexpr (OUT) {
+#pragma unroll
+    for (int h = 0; h < 4; ++h) *reinterpret_cast<float4*>(corr + h * kHeadDim + 4 * lane) = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncwarp();
+  }
 
   // ---- query: optional Hadamard rotation, scale to base-2 logits, per-head power-of-two exponent.
   {
@@ -273,13 +295,43 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   for (int m = 0; m < 8; ++m) bq[m][0] = bq[m][1] = 0u;
   float bias_col = 0.f;
 
-  const uint8_t* kc_ptr = reinterpret_cast<const uint8_t*>(a.k_codes + unit * a.tiles * (64 * KB)) +
-                          static_cast<int64_t>(first_token / kTile) * (256 * KB) + 16 * lane;
-  const uint8_t* vc_ptr = reinterpret_cast<const uint8_t*>(a.v_codes + unit * a.tiles * (64 * VB)) +
-                          static_cast<int64_t>(first_token / kTile) * (256 * VB) + 16 * lane;
-  const uint8_t* vs_ptr = reinterpret_cast<const uint8_t*>(a.v_scale + (unit * a.capacity + first_token) * VPT) + 16 * lane;
-  const uint8_t* vz_ptr = reinterpret_cast<const uint8_t*>(a.v_zero + (unit * a.capacity + first_token) * VPT) + 16 * lane;
-  const uint16_t* kp_src = (lane < 16 ? a.k_scale : a.k_zero) + unit * a.groups * kHeadDim + 8 * (lane & 15);
+  // Lane pointers of the step at token t: its storage slot (the unit, or with paged storage the pool
+  // page of its logical page) and in-slot token. A step never crosses a page (a page is a whole number
+  // of 128-token blocks), so with paged storage the pointers are re-based at every page start; the
+  // host has checked every table entry of the quantized part.
+  const uint8_t* kc_ptr = nullptr;
+  const uint8_t* vc_ptr = nullptr;
+  const uint8_t* vs_ptr = nullptr;
+  const uint8_t* vz_ptr = nullptr;
+  const uint8_t* ko_ptr = nullptr;
+  const uint8_t* vo_ptr = nullptr;
+  auto rebase = [&](int t) {
+    int64_t slot = unit, ts = t;
+    if (a.page_tokens > 0) {
+      slot = a.page_table[unit * a.pages_per_unit + t / a.page_tokens];
+      ts = t % a.page_tokens;
+    }
+    kc_ptr = reinterpret_cast<const uint8_t*>(a.k_codes + slot * a.tiles * (64 * KB)) + (ts / kTile) * (256 * KB) + 16 * lane;
+    vc_ptr = reinterpret_cast<const uint8_t*>(a.v_codes + slot * a.tiles * (64 * VB)) + (ts / kTile) * (256 * VB) + 16 * lane;
+    vs_ptr = reinterpret_cast<const uint8_t*>(a.v_scale + (slot * a.slot_tokens + ts) * VPT) + 16 * lane;
+    vz_ptr = reinterpret_cast<const uint8_t*>(a.v_zero + (slot * a.slot_tokens + ts) * VPT) + 16 * lane;
+    if constexpr (OUT) {
+      ko_ptr = reinterpret_cast<const uint8_t*>(a.k_out + slot * a.slot_tokens + ts) + 16 * lane;
+      vo_ptr = reinterpret_cast<const uint8_t*>(a.v_out + slot * a.slot_tokens + ts) + 16 * lane;
+    }
+  };
+  if (nst > 0) rebase(first_token);
+  // Key scale / zero row of key group g (g < q_groups) for this lane's 16-byte part.
+  const uint16_t* kp_base = (lane < 16 ? a.k_scale : a.k_zero) + 8 * (lane & 15);
+  auto kp_row = [&](int g) -> const uint16_t* {
+    int64_t slot = unit, gs = g;
+    if (a.page_tokens > 0) {
+      const int tg = g * G;
+      slot = a.page_table[unit * a.pages_per_unit + tg / a.page_tokens];
+      gs = (tg % a.page_tokens) / G;
+    }
+    return kp_base + (slot * a.groups + gs) * kHeadDim;
+  };
 
   // issue(i): step i of this warp into stage i % kStages (tracked by stage_in); the lane pointers
   // advance one step per call
@@ -287,6 +339,8 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(ring)) + 16 * lane;
   int stage_in = 0;
   auto issue = [&](int i) {
+    if (a.page_tokens > 0 && i > 0 && (first_token + i * kStepTokens) % a.page_tokens == 0)
+      rebase(first_token + i * kStepTokens);  // the step starts a new page
     const uint32_t st = ring_s + stage_in * S::kBytes;
     stage_in = stage_in == kStages - 1 ? 0 : stage_in + 1;
     cp_async16_at<S::oKC, 0>(st, kc_ptr);
@@ -301,6 +355,14 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
       cp_async16_at<S::oVS, 0>(st, vs_ptr);
       cp_async16_at<S::oVZ, 0>(st, vz_ptr);
     }
+    if constexpr (OUT) {
+      if (lane < S::kKO / 16) {
+        cp_async16_at<S::oKO, 0>(st, ko_ptr);
+        cp_async16_at<S::oVO, 0>(st, vo_ptr);
+      }
+      ko_ptr += S::kKO;
+      vo_ptr += S::kKO;
+    }
     const int t = first_token + i * kStepTokens;
     if (i == 0 || (t % kBlockTokens) == 0) {
       const int blk = t / kBlockTokens;
@@ -309,7 +371,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
       for (int kg = 0; kg < KGB; ++kg) {
         const int g = blk * KGB + kg;
         const bool valid = g < q_groups;
-        cp_async16_zfill(kp + 512 * kg, kp_src + static_cast<int64_t>(valid ? g : 0) * kHeadDim, valid);
+        cp_async16_zfill(kp + 512 * kg, valid ? kp_row(g) : kp_base, valid);  // nothing is read when invalid
       }
     }
     kc_ptr += S::kKC;
@@ -395,6 +457,21 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
         s[u][1] = __shfl_sync(kFull, s[u][1], src);
       }
     }
+    if constexpr (OUT) {  // key outliers: q~[ch] * (k_out - zk[g][ch]) for this lane's tokens and head h_d
+      const uint32_t* kos = reinterpret_cast<const uint32_t*>(st + S::oKO);
+      const uint16_t* kz = reinterpret_cast<const uint16_t*>(kp_ring + ((t / kBlockTokens) % S::kKPSlots) * S::kKP +
+                                                             512 * ((t / G) % KGB) + 256);
+      const float* qh = sq + h_d * kHeadDim;
+#pragma unroll
+      for (int u = 0; u < TS; ++u)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t ko = kos[16 * u + r + 8 * e];
+          const uint32_t ch = ko & 0xffffu;
+          if (ch < 128u)
+            s[u][e] = fmaf(qh[ch], h2f(static_cast<uint16_t>(ko >> 16)) - h2f(kz[key_param_pos(static_cast<int>(ch))]), s[u][e]);
+        }
+    }
     if (a.sink && t == 0 && r == 0) s[0][0] = -CUDART_INF_F;  // the sink token is read from its fp16 row
 
     // -- online softmax for head h_d over the step
@@ -426,8 +503,39 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
       const float az = __shfl_sync(kFull, alpha, col_head);  // lane col_head has h_d == col_head
 #pragma unroll
       for (int j = 0; j < NBV; ++j) zacc[j] *= az;
+      if constexpr (OUT) {
+#pragma unroll
+        for (int h = 0; h < GQ; ++h) {
+          const float ah = __shfl_sync(kFull, alpha, h);  // lane h has h_d == h
+          float4* c4 = reinterpret_cast<float4*>(corr + h * kHeadDim + 4 * lane);
+          float4 v = *c4;
+          v.x *= ah;
+          v.y *= ah;
+          v.z *= ah;
+          v.w *= ah;
+          *c4 = v;
+        }
+      }
     }
     m_run = m_new;
+    if constexpr (OUT) {  // value outliers: p * (v_out - zv[t][ch / G]) at channel ch, one lane per (token, head)
+      __syncwarp();
+      if (qd < GQ) {
+        const uint32_t* vos = reinterpret_cast<const uint32_t*>(st + S::oVO);
+        const uint16_t* vz = reinterpret_cast<const uint16_t*>(st + S::oVZ);
+#pragma unroll
+        for (int u = 0; u < TS; ++u)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int tk = 16 * u + r + 8 * e;
+            const uint32_t vo = vos[tk];
+            const uint32_t ch = vo & 0xffffu;
+            if (ch < 128u)
+              atomicAdd(corr + h_d * kHeadDim + ch,
+                        p[u][e] * (h2f(static_cast<uint16_t>(vo >> 16)) - h2f(vz[tk * VPT + ch / G])));
+          }
+      }
+    }
 
     // -- P.V per tile: B = p * sv (hi/lo) of head col_head for tokens 2qd, 2qd+1, 2qd+8, 2qd+9 and
     //    the value group of this lane's column in each n-block; A = centered value codes
@@ -538,7 +646,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   __syncwarp();
   for (int idx = lane; idx < gq * kHeadDim; idx += 32) {
     const int h = idx >> 7, c = idx & 127;
-    cw[h * kCm + kCmO + c] += zb[(warp * 4 + h) * 8 + c / G];
+    cw[h * kCm + kCmO + c] += zb[(warp * 4 + h) * 8 + c / G] + (OUT ? corr[h * kHeadDim + c] : 0.f);
   }
   __syncwarp();
 
@@ -676,28 +784,28 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a)
   out[c] = __half_as_ushort(__float2half_rn(acc / l));
 }
 
-template <int KB, int VB, int VPT, int GQ>
+template <int KB, int VB, int VPT, int GQ, bool OUT>
 cudaError_t launch_split(const DecodeArgs& a, cudaStream_t stream) {
-  constexpr int smem = decode_smem_bytes<KB, VB, VPT, GQ>();
+  constexpr int smem = decode_smem_bytes<KB, VB, VPT, GQ, OUT>();
   static DeviceMemo attr;
   const int ok = attr.get([] {
-    return cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1 : -1;
+    return cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1 : -1;
   });
   if (ok < 0) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads));
-  decode_split_kernel<KB, VB, VPT, GQ><<<grid, 32 * kDecodeWarps, smem, stream>>>(a);
+  decode_split_kernel<KB, VB, VPT, GQ, OUT><<<grid, 32 * kDecodeWarps, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <int KB, int VB, int VPT, int GQ>
+template <int KB, int VB, int VPT, int GQ, bool OUT>
 int occupancy() {
   static DeviceMemo memo;
   return memo.get([] {
-    constexpr int smem = decode_smem_bytes<KB, VB, VPT, GQ>();
-    if (cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    constexpr int smem = decode_smem_bytes<KB, VB, VPT, GQ, OUT>();
+    if (cudaFuncSetAttribute(decode_split_kernel<KB, VB, VPT, GQ, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<KB, VB, VPT, GQ>, 32 * kDecodeWarps, smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<KB, VB, VPT, GQ, OUT>, 32 * kDecodeWarps, smem) != cudaSuccess)
       return 1;
     return n > 0 ? n : 1;
   });
@@ -706,22 +814,32 @@ int occupancy() {
 // GQ template: the smallest of 1, 2, 4 that holds the query heads of one KV head.
 inline int gq_class(int gqa) { return gqa <= 1 ? 1 : (gqa <= 2 ? 2 : 4); }
 
-template <int KB, int VB, int VPT>
-cudaError_t dispatch_gq(const DecodeArgs& a, cudaStream_t s) {
+template <int KB, int VB, int VPT, bool OUT>
+cudaError_t dispatch_gq_out(const DecodeArgs& a, cudaStream_t s) {
   switch (gq_class(a.gqa)) {
-    case 1: return launch_split<KB, VB, VPT, 1>(a, s);
-    case 2: return launch_split<KB, VB, VPT, 2>(a, s);
-    default: return launch_split<KB, VB, VPT, 4>(a, s);
+    case 1: return launch_split<KB, VB, VPT, 1, OUT>(a, s);
+    case 2: return launch_split<KB, VB, VPT, 2, OUT>(a, s);
+    default: return launch_split<KB, VB, VPT, 4, OUT>(a, s);
   }
 }
 
 template <int KB, int VB, int VPT>
-int occupancy_gq(int gqa) {
+cudaError_t dispatch_gq(const DecodeArgs& a, cudaStream_t s) {
+  return a.outliers ? dispatch_gq_out<KB, VB, VPT, true>(a, s) : dispatch_gq_out<KB, VB, VPT, false>(a, s);
+}
+
+template <int KB, int VB, int VPT, bool OUT>
+int occupancy_gq_out(int gqa) {
   switch (gq_class(gqa)) {
-    case 1: return occupancy<KB, VB, VPT, 1>();
-    case 2: return occupancy<KB, VB, VPT, 2>();
-    default: return occupancy<KB, VB, VPT, 4>();
+    case 1: return occupancy<KB, VB, VPT, 1, OUT>();
+    case 2: return occupancy<KB, VB, VPT, 2, OUT>();
+    default: return occupancy<KB, VB, VPT, 4, OUT>();
   }
+}
+
+template <int KB, int VB, int VPT>
+int occupancy_gq(int gqa, int outliers) {
+  return outliers ? occupancy_gq_out<KB, VB, VPT, true>(gqa) : occupancy_gq_out<KB, VB, VPT, false>(gqa);
 }
 
 template <int KB, int VB>
@@ -735,12 +853,12 @@ cudaError_t dispatch_vpt(const DecodeArgs& a, cudaStream_t s) {
 }
 
 template <int KB, int VB>
-int occupancy_vpt(int G, int gqa) {
+int occupancy_vpt(int G, int gqa, int outliers) {
   switch (G) {
-    case 128: return occupancy_gq<KB, VB, 1>(gqa);
-    case 64: return occupancy_gq<KB, VB, 2>(gqa);
-    case 32: return occupancy_gq<KB, VB, 4>(gqa);
-    default: return occupancy_gq<KB, VB, 8>(gqa);
+    case 128: return occupancy_gq<KB, VB, 1>(gqa, outliers);
+    case 64: return occupancy_gq<KB, VB, 2>(gqa, outliers);
+    case 32: return occupancy_gq<KB, VB, 4>(gqa, outliers);
+    default: return occupancy_gq<KB, VB, 8>(gqa, outliers);
   }
 }
 
@@ -761,9 +879,9 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa) {
-  if (key_bits == 2) return value_bits == 2 ? occupancy_vpt<2, 2>(G, gqa) : occupancy_vpt<2, 4>(G, gqa);
-  return value_bits == 2 ? occupancy_vpt<4, 2>(G, gqa) : occupancy_vpt<4, 4>(G, gqa);
+int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa, int outliers) {
+  if (key_bits == 2) return value_bits == 2 ? occupancy_vpt<2, 2>(G, gqa, outliers) : occupancy_vpt<2, 4>(G, gqa, outliers);
+  return value_bits == 2 ? occupancy_vpt<4, 2>(G, gqa, outliers) : occupancy_vpt<4, 4>(G, gqa, outliers);
 }
 
 }  // namespace kvq

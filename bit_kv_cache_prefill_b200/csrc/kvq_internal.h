@@ -27,6 +27,16 @@ struct QuantizeArgs {
   int64_t vwords;                         // value code words per unit
   int sink;                               // 1: token 0 stays in fp16 in ring row R+G
   int64_t res_rows;                       // rows of k_res / v_res per unit: R + G + sink
+  int outliers;                           // 1: each quantized token's largest entry stays fp16
+  uint32_t* k_out;                        // [slots][slot_tokens]: channel | fp16 value << 16 (0xffff: none)
+  uint32_t* v_out;
+  // Storage slots: one per unit (contiguous) or one per pool page (paged). tiles, groups and vwords
+  // above count per slot; token t of a unit lives in slot page_table[unit][t / page_tokens] at
+  // t mod page_tokens (paged), else in slot `unit` at t.
+  int64_t slot_tokens;                    // capacity, or page_tokens when paged
+  int page_tokens;                        // 0: contiguous
+  int64_t pages_per_unit;                 // capacity / page_tokens
+  const int32_t* page_table;              // device [units][pages_per_unit]
 };
 
 struct DecodeArgs {
@@ -46,6 +56,13 @@ struct DecodeArgs {
   int64_t capacity, tiles, groups, ring;
   int sink;          // 1: token 0 is read from ring row R+G (fp16) and masked in the quantized part
   int64_t res_rows;  // rows of k_res / v_res per unit: R + G + sink
+  int outliers;             // 1: add each quantized token's fp16 key / value outlier (tile v1 only)
+  const uint32_t* k_out;    // [slots][slot_tokens]: channel | fp16 value << 16 (0xffff: none)
+  const uint32_t* v_out;
+  int64_t slot_tokens;      // storage slot extent (tiles, groups count per slot): capacity, or page_tokens
+  int page_tokens;          // 0: contiguous; else token t of a unit lives in slot page_table[unit][t / page_tokens]
+  int64_t pages_per_unit;
+  const int32_t* page_table;  // device [units][pages_per_unit]
   int layout;     // KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2
   int split_len;  // tokens per split (multiple of 64; rows v2: multiple of 128)
   int nsplit;     // splits per unit in the grid
@@ -62,7 +79,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // rows
 cudaError_t launch_decode_rope(const DecodeArgs& a, cudaStream_t stream);  // pre-RoPE keys: tables + split kernel
 int decode_rope_ctas_per_sm();
 int64_t rope_table_floats(int64_t capacity);  // floats of the two RoPE tables in the workspace
-int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);  // tile-v1 kernel
+int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa, int outliers);  // tile-v1 kernel
 int decode_tc_ctas_per_sm(int G, int gqa);                              // rows-v2 kernel (1 or 2)
 
 // Per-device memo of a small non-negative value (a function attribute already set, an occupancy, an

@@ -126,8 +126,15 @@ constexpr int key_scratch_bytes() {
   return 2 * NGM * 4 * 64 * 4 + 2 * NGM * 128 * 4 + NGM * 128;
 }
 
-template <int BITS, int LAYOUT, int G>
-__device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int nq, const uint16_t* rows, uint8_t* scratch) {
+// With OUT, och[t] is token t's key outlier channel (0xff: none): that entry stays out of its
+// channel's min / max (as +inf for the min, -inf for the max), a channel whose entries in a group are
+// all outliers gets scale and zero 0, and after the parameters every outlier entry is overwritten with
+// its channel's zero, which codes to 0.
+// The block's tokens t0 .. t0 + nq - 1 are stored in slot `slot` from in-slot token ts0 on (the unit
+// and t0, or with paged storage the pool page and t0 mod page_tokens).
+template <int BITS, int LAYOUT, int G, bool OUT>
+__device__ void key_block(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, int nq, const uint16_t* rows,
+                          uint8_t* scratch, const uint8_t* och) {
   constexpr int top = (1 << BITS) - 1;
   constexpr int P = 16 / BITS;  // code pairs per word
   const int NG = nq / G;
@@ -149,8 +156,20 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
       const uint16_t* src = rows + (g * G + q * ql) * kRS + 2 * cp;
       for (int i = (sink0 && g == 0 && q == 0) ? 1 : 0; i < ql; ++i) {
         const uint32_t x = *reinterpret_cast<const uint32_t*>(src + i * kRS);
-        mn = hmin2u(mn, x);
-        mx = hmax2u(mx, x);
+        if constexpr (OUT) {
+          const int o = och[g * G + q * ql + i];
+          uint32_t xmn = x, xmx = x;
+          if ((o >> 1) == cp) {
+            const uint32_t hm = (o & 1) ? 0xffff0000u : 0x0000ffffu;
+            xmn = (x & ~hm) | (kPosInf2 & hm);
+            xmx = (x & ~hm) | (kNegInf2 & hm);
+          }
+          mn = hmin2u(mn, xmn);
+          mx = hmax2u(mx, xmx);
+        } else {
+          mn = hmin2u(mn, x);
+          mx = hmax2u(mx, x);
+        }
       }
       pmn[(g * 4 + q) * 64 + cp] = mn;
       pmx[(g * 4 + q) * 64 + cp] = mx;
@@ -168,19 +187,22 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
         mx2 = hmax2u(mx2, pmx[(g * 4 + q) * 64 + (c >> 1)]);
       }
       const uint32_t hmn = (mn2 >> sh) & 0xffffu, hmx = (mx2 >> sh) & 0xffffu;
+      // min +inf with max -inf: no entry outside the outliers (finite inputs)
+      const bool all_out = OUT && hmn == 0x7C00u && hmx == 0xFC00u;
       uint32_t kmin = order_key(hmn), kmax = order_key(hmx);
-      if (is_zero_h(hmn) || is_zero_h(hmx)) {  // a signed zero: redo with the total order (-0 < +0)
+      if (!all_out && (is_zero_h(hmn) || is_zero_h(hmx))) {  // a signed zero: redo with the total order (-0 < +0)
         kmin = 0xffffu;
         kmax = 0u;
         for (int t = g * G + ((sink0 && g == 0) ? 1 : 0); t < (g + 1) * G; ++t) {
+          if (OUT && och[t] == c) continue;
           const uint32_t k = order_key(rows[t * kRS + c]);
           kmin = min(kmin, k);
           kmax = max(kmax, k);
         }
       }
-      const QuantParams p = make_params(kmin, kmax, BITS);
+      const QuantParams p = all_out ? QuantParams{0.f, 0.f, 0, 0, true} : make_params(kmin, kmax, BITS);
       const int pos = LAYOUT == KVQ_LAYOUT_ROWS_V2 ? c : key_param_pos(c);
-      const int64_t pidx = (unit * a.groups + t0 / G + g) * kHeadDim + pos;
+      const int64_t pidx = (slot * a.groups + ts0 / G + g) * kHeadDim + pos;
       a.k_scale[pidx] = p.s16;
       a.k_zero[pidx] = p.z16;
       pz[g * 128 + c] = p.zf;
@@ -191,6 +213,13 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
     }
   }
   __syncthreads();
+  if constexpr (OUT) {  // outlier entries -> their channel's zero (f32(zero) converts back exactly)
+    for (int t = tid; t < nq; t += kPThreads) {
+      const int o = och[t];
+      if (o != 0xff) const_cast<uint16_t*>(rows)[t * kRS + o] = __half_as_ushort(__float2half_rn(pz[(t / G) * 128 + o]));
+    }
+    __syncthreads();
+  }
 
   if constexpr (LAYOUT == KVQ_LAYOUT_ROWS_V2) {
     // word w of token t holds channels [2P w, 2P w + 2P): pair k -> channels 2(Pw + k), +1 at bits
@@ -210,7 +239,7 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
       iv[i] = pinv[g * 128 + c0 + i];
       slow |= pcl[g * 128 + c0 + i] != 0;
     }
-    uint32_t* dst = a.k_codes + (unit * a.capacity + t0) * W + w;
+    uint32_t* dst = a.k_codes + (slot * a.slot_tokens + ts0) * W + w;
 #pragma unroll 2
     for (int it = 0; it < TPT; ++it) {
       const int t = tbase + STRIDE * it;
@@ -266,7 +295,7 @@ __device__ void key_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int n
     float zf[2 * NCP], iv[2 * NCP];
     bool slow = false;
     int gcur = -1;
-    uint32_t* dst = a.k_codes + (unit * a.tiles + t0 / kTile) * words + widx;
+    uint32_t* dst = a.k_codes + (slot * a.tiles + ts0 / kTile) * words + widx;
     for (int tl = tl0; tl < tl0 + ntl && tl * kTile < nq; ++tl) {
       const int g = (tl * kTile) / G;
       if (g != gcur) {
@@ -312,8 +341,11 @@ constexpr int val_scratch_bytes() {
   return kPB * VPT * 8 + kPB * VPT + (LAYOUT == KVQ_LAYOUT_ROWS_V2 ? kHeadDim * 4 * BITS * 4 : 0);
 }
 
-template <int BITS, int LAYOUT, int G>
-__device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int nq, const uint16_t* rows, uint8_t* scratch) {
+// With OUT, select_outliers has replaced each token's value outlier by its neighbour (so the min / max
+// leave it out); once the token's parameters are known the entry becomes its group's zero (code 0).
+template <int BITS, int LAYOUT, int G, bool OUT>
+__device__ void value_block(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, int nq, const uint16_t* rows,
+                            uint8_t* scratch, const uint8_t* och) {
   constexpr int top = (1 << BITS) - 1;
   constexpr int P = 16 / BITS;
   constexpr int VPT = kHeadDim / G;
@@ -346,11 +378,15 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     QuantParams p = make_params(kmin, kmax, BITS);
     const bool sink_tok = a.sink && t0 + t == 0;  // the sink token: scale, zero and codes 0
     if (sink_tok) p = QuantParams{0.f, 0.f, 0, 0, true};
-    const int64_t pidx = (unit * a.capacity + t0 + t) * VPT + j;
+    const int64_t pidx = (slot * a.slot_tokens + ts0 + t) * VPT + j;
     a.v_scale[pidx] = p.s16;
     a.v_zero[pidx] = p.z16;
     prm[t * VPT + j] = make_float2(p.zf, p.inv);
     pcl[t * VPT + j] = !sink_tok && needs_clamp(p, kmax, top) ? 1 : 0;
+    if constexpr (OUT) {
+      const int o = och[t];
+      if (o != 0xff && o / G == j) const_cast<uint16_t*>(rows)[t * kRS + o] = p.z16;
+    }
   }
   __syncthreads();
 
@@ -392,7 +428,7 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     }
     __syncthreads();
     // 128 channel rows x nw words -> the block's rows (W words each), 16 bytes per thread-store
-    uint32_t* dst = a.v_codes + unit * a.vwords + (t0 / 128) * 128 * W;
+    uint32_t* dst = a.v_codes + slot * a.vwords + (ts0 / 128) * 128 * W;
     const int q4 = nw / 4;  // nw is a multiple of 4 when nq is a multiple of 16 * 4 / BITS ...
     if (q4 * 4 == nw) {
       for (int idx = tid; idx < 128 * q4; idx += kPThreads) {
@@ -422,7 +458,7 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
     const int words = 64 * BITS;
     const int widx0 = (w >> 2) * 128 + 4 * L0 + (w & 3);  // lane L1 = L0 + 4: widx0 + 16
     const int ch0 = 16 * ((P * w) >> 2) + r0;              // channel of pair j: ch0 + 16 (j >> 2) + 8 (j & 1)
-    uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words + widx0;
+    uint32_t* dst = a.v_codes + (slot * a.tiles + ts0 / kTile) * words + widx0;
     for (int k = 0; k < TPT; ++k) {
       const int tl = 2 * (part + NPART * k) + half;
       if (tl * kTile >= nq) break;
@@ -459,8 +495,15 @@ __device__ void value_block(const QuantizeArgs& a, int64_t unit, int64_t t0, int
   }
 }
 
-// G (16, 32, 64 or 128) is a template parameter so that every division by it is a shift.
-template <int BITS_K, int BITS_V, int LAYOUT, int G>
+template <int BK, int BV, int LAYOUT, int G>
+constexpr int scratch_bytes() {
+  constexpr int ks = key_scratch_bytes<G>(), vs = val_scratch_bytes<G, LAYOUT, BV>();
+  return ks > vs ? ks : vs;
+}
+
+// G (16, 32, 64 or 128) is a template parameter so that every division by it is a shift. OUT: the
+// dense-and-sparse outliers are on (och[128] follows the scratch).
+template <int BITS_K, int BITS_V, int LAYOUT, int G, bool OUT>
 __global__ void __launch_bounds__(kPThreads) prefill_block_kernel(QuantizeArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
@@ -501,40 +544,60 @@ __global__ void __launch_bounds__(kPThreads) prefill_block_kernel(QuantizeArgs a
     }
   }
   if (nq == 0) return;
+  // Storage slot of the block: the unit, or with paged storage the pool page of its logical page (a
+  // page is a whole number of 128-token blocks; the host has checked every entry that holds tokens).
+  int64_t slot = unit, ts0 = t0;
+  if (a.page_tokens > 0) {
+    slot = a.page_table[unit * a.pages_per_unit + t0 / a.page_tokens];
+    ts0 = t0 % a.page_tokens;
+  }
+  uint8_t* och = scratch + scratch_bytes<BITS_K, BITS_V, LAYOUT, G>();
+  if constexpr (OUT) {
+    select_outliers(rows, kRS, nq, (is_key ? a.k_out : a.v_out) + slot * a.slot_tokens + ts0, och,
+                    a.sink && t0 == 0, !is_key, kPThreads / 32);
+    __syncthreads();
+  }
   if (is_key)
-    key_block<BITS_K, LAYOUT, G>(a, unit, t0, nq, rows, scratch);
+    key_block<BITS_K, LAYOUT, G, OUT>(a, slot, ts0, t0, nq, rows, scratch, och);
   else
-    value_block<BITS_V, LAYOUT, G>(a, unit, t0, nq, rows, scratch);
+    value_block<BITS_V, LAYOUT, G, OUT>(a, slot, ts0, t0, nq, rows, scratch, och);
 }
 
-// Shared memory of one CTA: the rows, then the larger of the key and value scratch. With G >= 32 it
-// fits four CTAs per SM.
-template <int BK, int BV, int LAYOUT, int G>
+// Shared memory of one CTA: the rows, then the larger of the key and value scratch (and with OUT the
+// outlier channels). With G >= 32 it fits four CTAs per SM.
+template <int BK, int BV, int LAYOUT, int G, bool OUT>
 constexpr int prefill_smem_bytes() {
-  constexpr int ks = key_scratch_bytes<G>(), vs = val_scratch_bytes<G, LAYOUT, BV>();
-  return kPB * kRS * 2 + (ks > vs ? ks : vs);
+  return kPB * kRS * 2 + scratch_bytes<BK, BV, LAYOUT, G>() + (OUT ? kPB : 0);
 }
 
-template <int BK, int BV, int LAYOUT, int G>
+template <int BK, int BV, int LAYOUT, int G, bool OUT>
 cudaError_t launch_block(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
   static DeviceMemo attr;
   const int ok = attr.get([] {
-    return cudaFuncSetAttribute(prefill_block_kernel<BK, BV, LAYOUT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                prefill_smem_bytes<BK, BV, LAYOUT, G>()) == cudaSuccess ? 1 : -1;
+    return cudaFuncSetAttribute(prefill_block_kernel<BK, BV, LAYOUT, G, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                prefill_smem_bytes<BK, BV, LAYOUT, G, OUT>()) == cudaSuccess ? 1 : -1;
   });
   if (ok < 0) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>((max_len + kPB - 1) / kPB), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads), 2);
-  prefill_block_kernel<BK, BV, LAYOUT, G><<<grid, kPThreads, prefill_smem_bytes<BK, BV, LAYOUT, G>(), stream>>>(a);
+  prefill_block_kernel<BK, BV, LAYOUT, G, OUT><<<grid, kPThreads, prefill_smem_bytes<BK, BV, LAYOUT, G, OUT>(), stream>>>(a);
   return cudaGetLastError();
+}
+
+// The outlier instances exist for tile v1 only (the configuration check rejects the others).
+template <int BK, int BV, int LAYOUT, int G>
+cudaError_t launch_out(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
+  if constexpr (LAYOUT == KVQ_LAYOUT_TILE_V1)
+    if (a.outliers) return launch_block<BK, BV, LAYOUT, G, true>(a, max_len, stream);
+  return launch_block<BK, BV, LAYOUT, G, false>(a, max_len, stream);
 }
 
 template <int BK, int BV, int LAYOUT>
 cudaError_t launch_group(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream) {
   switch (a.G) {
-    case 16: return launch_block<BK, BV, LAYOUT, 16>(a, max_len, stream);
-    case 32: return launch_block<BK, BV, LAYOUT, 32>(a, max_len, stream);
-    case 64: return launch_block<BK, BV, LAYOUT, 64>(a, max_len, stream);
-    case 128: return launch_block<BK, BV, LAYOUT, 128>(a, max_len, stream);
+    case 16: return launch_out<BK, BV, LAYOUT, 16>(a, max_len, stream);
+    case 32: return launch_out<BK, BV, LAYOUT, 32>(a, max_len, stream);
+    case 64: return launch_out<BK, BV, LAYOUT, 64>(a, max_len, stream);
+    case 128: return launch_out<BK, BV, LAYOUT, 128>(a, max_len, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -18,8 +18,10 @@ namespace kvq {
 
 // Shared memory of one chunk: fp16 rows [G][128], then per-chunk parameters: keys use (f32(zero),
 // 1/f32(scale)) per channel [128] plus per-quarter min/max keys [4][128] x 2; values use
-// (f32(zero), 1/f32(scale)) per (token, channel group) [G][128/G] = 128 entries.
-static size_t chunk_smem_bytes(int G) { return static_cast<size_t>(G) * kHeadDim * 2 + 128 * 8 + 2 * 4 * 128 * 4; }
+// (f32(zero), 1/f32(scale)) per (token, channel group) [G][128/G] = 128 entries. Then the outlier
+// channel of each row [G] u8 (0xff: none).
+constexpr int kChunkParamBytes = 128 * 8 + 2 * 4 * 128 * 4;
+static size_t chunk_smem_bytes(int G) { return static_cast<size_t>(G) * kHeadDim * 2 + kChunkParamBytes + 128; }
 
 // Code of x on the grid (zf, inv): rint_even((f32(x) - zf) * inv) clamped to [0, 2^bits - 1].
 // inv == 0 encodes a zero scale and yields code 0 (x - zf is finite). v = (x - zf) * inv is >= 0
@@ -31,16 +33,21 @@ __device__ __forceinline__ uint32_t code_with(uint16_t x, float zf, float inv, i
   return __float_as_uint(__fadd_rn(v, 12582912.0f)) & 0xffu;
 }
 
-// Quantize G staged key rows (tokens t0 .. t0+G-1 of `unit`) and write key group t0/G.
+// Quantize G staged key rows (tokens t0 .. t0+G-1 of a unit, stored in slot `slot` from in-slot token
+// ts0 on: the unit and t0, or with paged storage the pool page and t0 mod page_tokens) and write their
+// key group.
 // All 256 threads work in every phase: min/max over token quarters for channel pairs, parameters per
 // channel, then one packed word per thread-iteration built straight from the fp16 rows.
-__device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t t0, const uint16_t* rows,
-                                    uint8_t* pbuf) {
+// With the outliers on, och[i] is row i's outlier channel: that entry stays out of its channel's
+// min / max, a channel whose entries are all outliers gets scale and zero 0, and the entry is then
+// overwritten with its channel's zero (code 0).
+__device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, const uint16_t* rows,
+                                    uint8_t* pbuf, const uint8_t* och) {
   const int G = a.G, bits = a.key_bits, top = (1 << bits) - 1;
   float2* prm = reinterpret_cast<float2*>(pbuf);                  // [128] (zf, inv)
   uint32_t* pmin = reinterpret_cast<uint32_t*>(pbuf + 128 * 8);   // [4][128]
   uint32_t* pmax = pmin + 4 * 128;                                // [4][128]
-  const int64_t g = t0 / G;
+  const int64_t g = ts0 / G;  // key group within the slot
   const bool sink0 = a.sink && t0 == 0;  // token 0 stays out of group 0 (min/max and codes)
   {
     const int cp = threadIdx.x & 63, tq = threadIdx.x >> 6;
@@ -49,10 +56,15 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
     for (int i = tq * n + ((sink0 && tq == 0) ? 1 : 0); i < (tq + 1) * n; ++i) {
       const uint32_t w = *reinterpret_cast<const uint32_t*>(rows + i * kHeadDim + 2 * cp);
       const uint32_t k0 = order_key(w & 0xffffu), k1 = order_key(w >> 16);
-      mn0 = min(mn0, k0);
-      mx0 = max(mx0, k0);
-      mn1 = min(mn1, k1);
-      mx1 = max(mx1, k1);
+      const int o = a.outliers ? och[i] : 0xff;
+      if (o != 2 * cp) {
+        mn0 = min(mn0, k0);
+        mx0 = max(mx0, k0);
+      }
+      if (o != 2 * cp + 1) {
+        mn1 = min(mn1, k1);
+        mx1 = max(mx1, k1);
+      }
     }
     pmin[tq * 128 + 2 * cp] = mn0;
     pmin[tq * 128 + 2 * cp + 1] = mn1;
@@ -64,21 +76,29 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
     const int c = threadIdx.x;
     const uint32_t kmin = min(min(pmin[c], pmin[128 + c]), min(pmin[256 + c], pmin[384 + c]));
     const uint32_t kmax = max(max(pmax[c], pmax[128 + c]), max(pmax[256 + c], pmax[384 + c]));
-    const QuantParams p = make_params(kmin, kmax, bits);
+    // no entry outside the outliers: scale and zero 0
+    const QuantParams p = kmin == 0xffffffffu ? QuantParams{0.f, 0.f, 0, 0, true} : make_params(kmin, kmax, bits);
     const int pos = a.layout == KVQ_LAYOUT_ROWS_V2 ? c : key_param_pos(c);  // rows v2: natural channel order
-    const int64_t pidx = (unit * a.groups + g) * kHeadDim + pos;
+    const int64_t pidx = (slot * a.groups + g) * kHeadDim + pos;
     a.k_scale[pidx] = p.s16;
     a.k_zero[pidx] = p.z16;
     prm[c] = make_float2(p.zf, p.inv);
     if (sink0) const_cast<uint16_t*>(rows)[c] = p.z16;  // codes to 0: x - zf = 0
   }
   __syncthreads();
+  if (a.outliers) {  // outlier entries -> their channel's zero (f32(zero) converts back exactly)
+    if (threadIdx.x < G && och[threadIdx.x] != 0xff) {
+      const int o = och[threadIdx.x];
+      const_cast<uint16_t*>(rows)[threadIdx.x * kHeadDim + o] = __half_as_ushort(__float2half_rn(prm[o].x));
+    }
+    __syncthreads();
+  }
   const int words = 64 * bits;
   const int P = 16 / bits;
   if (a.layout == KVQ_LAYOUT_ROWS_V2) {
     // one row of 4*bits words per token: pair j = P*w + k holds channels 2j, 2j + 1
     const int wpt = 4 * bits;
-    uint32_t* dst2 = a.k_codes + (unit * a.capacity + t0) * wpt;
+    uint32_t* dst2 = a.k_codes + (slot * a.slot_tokens + ts0) * wpt;
     for (int idx = threadIdx.x; idx < G * wpt; idx += blockDim.x) {
       const int i = idx / wpt, w = idx % wpt;
       uint32_t word = 0;
@@ -93,7 +113,7 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
     }
     return;
   }
-  uint32_t* dst = a.k_codes + (unit * a.tiles + t0 / kTile) * words;
+  uint32_t* dst = a.k_codes + (slot * a.tiles + ts0 / kTile) * words;
   for (int idx = threadIdx.x; idx < (G / kTile) * words; idx += blockDim.x) {
     const int tile = idx / words, widx = idx % words;
     int lane, w;
@@ -111,9 +131,11 @@ __device__ void quantize_keys_chunk(const QuantizeArgs& a, int64_t unit, int64_t
   }
 }
 
-// Quantize G staged value rows (per token, channel groups of G) and write their codes.
-__device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64_t t0, const uint16_t* rows,
-                                      uint8_t* pbuf) {
+// Quantize G staged value rows (per token, channel groups of G) and write their codes. With the
+// outliers on, each row's outlier entry has been replaced by its neighbour before (so the min / max
+// leave it out) and becomes its group's zero (code 0) once the parameters are known.
+__device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, const uint16_t* rows,
+                                      uint8_t* pbuf, const uint8_t* och) {
   const int G = a.G, bits = a.value_bits, top = (1 << bits) - 1;
   const int vpt = kHeadDim / G;
   float2* prm = reinterpret_cast<float2*>(pbuf);  // [G][vpt] (zf, inv)
@@ -138,10 +160,11 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
     if (half == 0) {
       QuantParams p = make_params(kmin, kmax, bits);
       if (a.sink && t0 + i == 0) p = QuantParams{0.f, 0.f, 0, 0, true};  // the sink token: all zero
-      const int64_t pidx = (unit * a.capacity + t0 + i) * vpt + j;
+      const int64_t pidx = (slot * a.slot_tokens + ts0 + i) * vpt + j;
       a.v_scale[pidx] = p.s16;
       a.v_zero[pidx] = p.z16;
       prm[i * vpt + j] = make_float2(p.zf, p.inv);
+      if (a.outliers && och[i] != 0xff && och[i] / G == j) const_cast<uint16_t*>(rows)[i * kHeadDim + och[i]] = p.z16;
     }
   }
   __syncthreads();
@@ -150,9 +173,9 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
   if (a.layout == KVQ_LAYOUT_ROWS_V2) {
     // the chunk lies inside one 128-token block; channel c's row of that block gets G / (2P) words
     const int wpr = 4 * bits, wpc = G / (2 * P);
-    const int64_t block = t0 / 128;
-    const int ib = static_cast<int>(t0 % 128);
-    uint32_t* dst2 = a.v_codes + unit * a.vwords + block * 128 * wpr + (ib / 2) / P;
+    const int64_t block = ts0 / 128;
+    const int ib = static_cast<int>(ts0 % 128);
+    uint32_t* dst2 = a.v_codes + slot * a.vwords + block * 128 * wpr + (ib / 2) / P;
     for (int idx = threadIdx.x; idx < kHeadDim * wpc; idx += blockDim.x) {
       const int c = idx / wpc, w = idx % wpc;
       uint32_t word = 0;
@@ -166,7 +189,7 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t unit, int64
     }
     return;
   }
-  uint32_t* dst = a.v_codes + (unit * a.tiles + t0 / kTile) * words;
+  uint32_t* dst = a.v_codes + (slot * a.tiles + ts0 / kTile) * words;
   for (int idx = threadIdx.x; idx < (G / kTile) * words; idx += blockDim.x) {
     const int tile = idx / words, widx = idx % words;
     int lane, w;
@@ -226,10 +249,23 @@ __global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint1
     reinterpret_cast<uint4*>(rows + i * kHeadDim)[part] = reinterpret_cast<const uint4*>(ring + slot * kHeadDim)[part];
   }
   __syncthreads();
+  // Storage slot of the group: the unit, or with paged storage the pool page of its logical page (a
+  // group never crosses a page; the host has checked the entry).
+  int64_t slot = unit, ts0 = Q_old;
+  if (a.page_tokens > 0) {
+    slot = a.page_table[unit * a.pages_per_unit + Q_old / a.page_tokens];
+    ts0 = Q_old % a.page_tokens;
+  }
+  uint8_t* och = pbuf + kChunkParamBytes;
+  if (a.outliers) {
+    select_outliers(rows, kHeadDim, G, (is_key ? a.k_out : a.v_out) + slot * a.slot_tokens + ts0, och,
+                    a.sink && Q_old == 0, !is_key, blockDim.x / 32);
+    __syncthreads();
+  }
   if (is_key)
-    quantize_keys_chunk(a, unit, Q_old, rows, pbuf);
+    quantize_keys_chunk(a, slot, ts0, Q_old, rows, pbuf, och);
   else
-    quantize_values_chunk(a, unit, Q_old, rows, pbuf);
+    quantize_values_chunk(a, slot, ts0, Q_old, rows, pbuf, och);
 }
 
 __global__ void bump_lengths_kernel(int64_t* seq_len, int batch) {

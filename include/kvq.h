@@ -62,9 +62,12 @@ typedef enum {
  *   residual R >= 0 (tokens kept in FP16 beyond the last full group; 0 <= R <= 4096);
  *   hadamard in {0, 1}; layout KVQ_LAYOUT_TILE_V1 or KVQ_LAYOUT_ROWS_V2; sink in {0, 1};
  *   rope_theta finite and >= 0; rope_theta > 0 needs hadamard = 0 (KVQ_ERR_INVALID_ARG) and layout
- *   KVQ_LAYOUT_ROWS_V2 (KVQ_ERR_UNSUPPORTED);
+ *   KVQ_LAYOUT_ROWS_V2 (KVQ_ERR_UNSUPPORTED); outliers in {0, 1}, outliers = 1 needs layout
+ *   KVQ_LAYOUT_TILE_V1 and rope_theta = 0 (KVQ_ERR_UNSUPPORTED);
  *   capacity >= 0, a multiple of G (maximum tokens per sequence); with layout ROWS_V2 also a
- *   multiple of 128 (value rows come in whole 128-token blocks). */
+ *   multiple of 128 (value rows come in whole 128-token blocks);
+ *   page_tokens 0 (contiguous) or a positive multiple of 128 that divides capacity, with
+ *   num_pages >= 1; paging needs layout KVQ_LAYOUT_TILE_V1 and rope_theta = 0 (KVQ_ERR_UNSUPPORTED). */
 typedef struct {
   int32_t batch;
   int32_t num_q_heads;
@@ -78,6 +81,9 @@ typedef struct {
   int32_t layout;
   int32_t sink;  /* 1: the first token of every sequence stays in fp16 (see below) */
   float rope_theta; /* > 0: keys are cached before RoPE and decode rotates them (see below); 0: off */
+  int32_t outliers; /* 1: each quantized token's largest key / value entry stays fp16 (see below) */
+  int32_t page_tokens; /* > 0: paged storage, pages of this many tokens (see below); 0: contiguous */
+  int32_t num_pages;   /* pages in the pool (paged storage only) */
   int64_t capacity;
 } kvq_config;
 
@@ -113,6 +119,28 @@ typedef struct {
  * (already rotated at its own position by the caller). The decode workspace then also holds the
  * angle tables, built at the start of every call.
  *
+ * Dense-and-sparse outliers (outliers = 1; the KVQuant review, Method, keeps about 1% of the entries
+ * in an fp16 sparse store with per-vector thresholds): per quantized token and tensor, the entry of
+ * largest magnitude (ties: the lowest channel) is kept exactly. k_out / v_out hold one u32 per token
+ * and unit: bits 0..15 the channel (0xffff: none, e.g. the sink token), bits 16..31 the fp16 value.
+ * That entry stays out of its key group's (per channel) or value group's (per token) min / max and
+ * is coded 0; dequantization puts the fp16 value back. A key channel whose entries in a group are all
+ * outliers gets scale and zero 0. Sizes: kvq_outlier_buffer_bytes.
+ *
+ * Paged storage (page_tokens = P > 0; the KVQuant review, Limitations, Future work and Sparks, names
+ * blocked allocation as the fix for copying earlier tokens' data on every update): the quantized part
+ * of a unit is cut into logical pages of P tokens. Logical page j of unit u lives in pool page
+ * page_table[u][j] (int32 [units][capacity / P]). k_codes, v_codes, k_scale, k_zero, v_scale, v_zero,
+ * k_out and v_out then hold num_pages pages instead of one slot per unit: each page holds what the
+ * per-unit layout above holds for P tokens (read "P" for "capacity"), at the in-page token t mod P;
+ * k_res and v_res stay per unit. The library reads the entries of the pages that hold quantized
+ * tokens, j < ceil(Q / P), and rejects (KVQ_ERR_INVALID_ARG) such an entry outside [0, num_pages);
+ * other entries may hold anything (e.g. -1, not yet handed out). Distinct (unit, page) pairs must get
+ * distinct pool pages, and an entry must not change while its page holds tokens.
+ * page_table_host is the caller's table in host memory; page_table_dev is its device mirror (caller-
+ * allocated, same shape), written by the library on the stream: the whole table is copied on every
+ * prefill and on every append in which some unit's quantized part enters a new page.
+ *
  * Tile v1: tile row k of a unit holds tokens 16k..16k+15. Within a tile, "lane" L (0..31) owns
  * words (w / 4) * 128 + 4L + (w % 4) for w in [0, 2*bits). Word w holds 16/bits code pairs; pair j
  * has its first code at bits [bits*j, bits*j + bits) and its second at bits [16 + bits*j, ...).
@@ -143,6 +171,10 @@ typedef struct {
   void* v_res;
   int64_t* seq_len_host;
   int64_t* seq_len_dev;
+  void* k_out;  /* outliers = 1 only: u32 [capacity] per unit, see below (NULL otherwise) */
+  void* v_out;
+  int32_t* page_table_host; /* page_tokens > 0 only: int32 [units][capacity / page_tokens], see above */
+  int32_t* page_table_dev;  /* its device mirror, written by the library */
 } kvq_cache;
 
 enum {
@@ -157,9 +189,14 @@ enum {
   KVQ_NUM_BUFFERS = 8
 };
 
-/* Byte size of each of the eight cache buffers for `cfg` (all units), in kvq_cache field order.
+/* Byte size of each of the eight cache buffers for `cfg` (all units, or the whole pool of num_pages
+ * pages for the first six with paged storage), in kvq_cache field order.
  * Returns KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED for a bad config or null pointers. */
 kvq_status kvq_cache_buffer_bytes(const kvq_config* cfg, size_t out_bytes[KVQ_NUM_BUFFERS]);
+
+/* Byte size of the two outlier buffers (k_out, v_out) for `cfg`: units * capacity * 4 each (paged:
+ * num_pages * page_tokens * 4) when outliers = 1, else 0. */
+kvq_status kvq_outlier_buffer_bytes(const kvq_config* cfg, size_t out_bytes[2]);
 
 /* Prefill: quantize whole prompts at once (KVQuant review, Limitations and Sparks: a prefill-side
  * kernel that compresses many keys and values in one pass).

@@ -22,17 +22,18 @@ def capacity(w: inputs.Workload, layout: int) -> int:
 
 
 def oracle_config(oracle, w: inputs.Workload, batch=None, hq=None, hkv=None, layout: int = 1, sink: int = 0,
-                  rope: float = 0.0):
+                  rope: float = 0.0, outliers: int = 0):
     return oracle.Config(batch or w.batch, hq or w.num_q_heads, hkv or w.num_kv_heads, w.key_bits, w.value_bits,
                          w.group_size, w.residual, w.hadamard, capacity(w, layout), layout=layout, sink=sink,
-                         rope_theta=rope)
+                         rope_theta=rope, outliers=outliers)
 
 
-def gpu_config(w: inputs.Workload, layout: int = 1, sink: int = 0, rope: float = 0.0):
+def gpu_config(w: inputs.Workload, layout: int = 1, sink: int = 0, rope: float = 0.0, outliers: int = 0):
     import bit_kv_cache_prefill_b200 as kvq
 
     return kvq.make_config(w.batch, w.num_q_heads, w.num_kv_heads, w.key_bits, w.value_bits, w.group_size,
-                           w.residual, w.hadamard, capacity(w, layout), layout=layout, sink=sink, rope_theta=rope)
+                           w.residual, w.hadamard, capacity(w, layout), layout=layout, sink=sink, rope_theta=rope,
+                           outliers=outliers)
 
 
 @dataclass
@@ -43,15 +44,16 @@ class GpuRun:
     lens: np.ndarray
     layout: int = 1
     sink: int = 0
+    outliers: int = 0
 
 
 def run_gpu(w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
             appends: int = 0, sm_scale: Optional[float] = None, layout: int = 1, decode: bool = True,
-            sink: int = 0, rope: float = 0.0) -> GpuRun:
+            sink: int = 0, rope: float = 0.0, outliers: int = 0) -> GpuRun:
     """Prefill (k, v on the device), `appends` streaming appends, one decode (unless decode=False)."""
     import bit_kv_cache_prefill_b200 as kvq
 
-    cfg = gpu_config(w, layout, sink, rope)
+    cfg = gpu_config(w, layout, sink, rope, outliers)
     cache = kvq.Cache(cfg)
     kvq.kvq_quantize_prefill(cfg, cache, k, v, lens)
     for step in range(appends):
@@ -62,7 +64,7 @@ def run_gpu(w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarr
         ws = torch.empty(kvq.kvq_decode_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
         kvq.kvq_decode_attention(cfg, cache, q.cuda(), out, sm_scale or 1 / math.sqrt(128), ws)
     torch.cuda.synchronize()
-    return GpuRun(cfg, cache, out, lens + appends, layout, sink)
+    return GpuRun(cfg, cache, out, lens + appends, layout, sink, outliers)
 
 
 def code_shapes(w: inputs.Workload, layout: int):
@@ -78,7 +80,13 @@ def gpu_views(w: inputs.Workload, run: GpuRun) -> Dict[str, np.ndarray]:
     ring = w.residual + G + run.sink  # ring slots, then the sink row
     c = run.cache
     ks, vs = code_shapes(w, run.layout)
-    return {
+    extra = {}
+    if run.outliers:  # u32 per (unit, token): channel | fp16 value << 16
+        for n in ("k_out", "v_out"):
+            words = c.view(n, torch.int32).cpu().numpy().view(np.uint32).reshape(B, H, cap)
+            extra[n + "_ch"] = (words & 0xFFFF).astype(np.uint16)
+            extra[n + "_val"] = (words >> 16).astype(np.uint16)
+    return extra | {
         "k_codes": c.view("k_codes", torch.int32).cpu().numpy().view(np.uint32).reshape(ks),
         "v_codes": c.view("v_codes", torch.int32).cpu().numpy().view(np.uint32).reshape(vs),
         "k_scale": c.view("k_scale", torch.int16).cpu().numpy().view(np.uint16).reshape(B, H, cap // G, 128),
@@ -91,10 +99,13 @@ def gpu_views(w: inputs.Workload, run: GpuRun) -> Dict[str, np.ndarray]:
 
 
 def compare_unit_cache(w: inputs.Workload, gv: Dict[str, np.ndarray], b: int, h: int, oc, ob: int, oh: int, T: int,
-                       layout: int = 1, sink: int = 0) -> None:
+                       layout: int = 1, sink: int = 0, outliers: int = 0) -> None:
     """Bit-exact comparison of everything that is defined for one unit of length T."""
     G, R = w.group_size, w.residual
     Q = max(T - R, 0) // G * G
+    if outliers:  # the (channel, fp16 value) of every quantized token's key and value outlier
+        for key in ("k_out_ch", "k_out_val", "v_out_ch", "v_out_val"):
+            np.testing.assert_array_equal(gv[key][b, h, :Q], getattr(oc, key)[ob, oh, :Q], err_msg=f"{key} unit {b},{h}")
     ring = R + G
     if layout == 2:
         np.testing.assert_array_equal(gv["k_codes"][b, h, :Q], oc.k_codes[ob, oh, :Q], err_msg=f"k_codes unit {b},{h}")
@@ -132,8 +143,8 @@ def check_attention(gpu_out: np.ndarray, ref: np.ndarray, what: str) -> Tuple[fl
 
 def oracle_full(oracle, w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
                 appends: int = 0, sm_scale: Optional[float] = None, threads: int = 8, layout: int = 1, sink: int = 0,
-                rope: float = 0.0):
-    ocfg = oracle_config(oracle, w, layout=layout, sink=sink, rope=rope)
+                rope: float = 0.0, outliers: int = 0):
+    ocfg = oracle_config(oracle, w, layout=layout, sink=sink, rope=rope, outliers=outliers)
     oc = oracle.Cache(ocfg)
     oracle.quantize_prefill(ocfg, oc, k.numpy(), v.numpy(), lens, threads=threads)
     for step in range(appends):

@@ -23,8 +23,8 @@ def _declared_symbols():
 def test_library_exports_every_declared_entry_point():
     names = _declared_symbols()
     assert names == ["kvq_append_token", "kvq_cache_buffer_bytes", "kvq_decode_attention",
-                     "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes", "kvq_quantize_prefill",
-                     "kvq_status_string"]
+                     "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes", "kvq_outlier_buffer_bytes",
+                     "kvq_quantize_prefill", "kvq_status_string"]
     lib = ctypes.CDLL(kvq.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -118,6 +118,46 @@ def test_rope_workspace_holds_the_angle_tables(cap):
     assert kvq.kvq_decode_workspace_bytes(rope) == -(-part // 256) * 256 + tables
 
 
+@pytest.mark.parametrize("layout,theta,value,status", [
+    (1, 0.0, 1, kvq.KVQ_OK), (1, 0.0, 0, kvq.KVQ_OK),
+    (2, 0.0, 1, kvq.KVQ_ERR_UNSUPPORTED),        # the outlier path exists for tile v1 only
+    (2, 10000.0, 1, kvq.KVQ_ERR_UNSUPPORTED),    # and not with pre-RoPE keys
+    (1, 0.0, 2, kvq.KVQ_ERR_INVALID_ARG), (1, 0.0, -1, kvq.KVQ_ERR_INVALID_ARG),
+])
+def test_outlier_config_validation(layout, theta, value, status):
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024, layout=layout, rope_theta=theta, outliers=value)
+    sizes = (ctypes.c_size_t * 8)()
+    assert _status("kvq_cache_buffer_bytes", ctypes.byref(cfg), sizes) == status
+    out = (ctypes.c_size_t * 2)()
+    assert _status("kvq_outlier_buffer_bytes", ctypes.byref(cfg), out) == status
+
+
+@pytest.mark.parametrize("B,Hkv,cap", [(2, 2, 1024), (8, 32, 32768 + 1024), (1, 8, 1 << 20)])
+def test_outlier_buffer_bytes(B, Hkv, cap):
+    # one u32 (channel | fp16 value << 16) per (unit, token) for keys and for values; none when off
+    on = kvq.make_config(B, 4 * Hkv if Hkv <= 8 else Hkv, Hkv, 2, 2, 32, 128, 0, cap, outliers=1)
+    off = kvq.make_config(B, 4 * Hkv if Hkv <= 8 else Hkv, Hkv, 2, 2, 32, 128, 0, cap)
+    assert kvq.kvq_outlier_buffer_bytes(on) == [B * Hkv * cap * 4] * 2
+    assert kvq.kvq_outlier_buffer_bytes(off) == [0, 0]
+    assert kvq.kvq_cache_buffer_bytes(on) == kvq.kvq_cache_buffer_bytes(off)
+    assert _status("kvq_outlier_buffer_bytes", ctypes.byref(on), None) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_outlier_cache_needs_its_buffers():
+    # outliers = 1 with null outlier pointers is rejected on the host before any launch
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024, outliers=1)
+    c, host = _fake_cache(cfg, [0, 0])
+    k = ctypes.c_void_p(0x100000)
+    lens = np.array([64, 64], np.int64)
+    st = _lib.lib.kvq_quantize_prefill(ctypes.byref(cfg), ctypes.byref(c), k, k, 64 * 2 * 128, 2 * 128, 128,
+                                       lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+    c.k_out, c.v_out = 0x200000, 0x200008  # v_out not 16-byte aligned
+    st = _lib.lib.kvq_quantize_prefill(ctypes.byref(cfg), ctypes.byref(c), k, k, 64 * 2 * 128, 2 * 128, 128,
+                                       lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+
+
 def _fake_cache(cfg, lens):
     # Non-null, 16-byte aligned placeholder addresses: every call below is rejected on the host before
     # any of them could be used.
@@ -174,6 +214,77 @@ def test_decode_rejects_small_workspace_and_bad_scale():
     assert _status("kvq_decode_attention", *args, ctypes.c_float(float("nan")), 0x300000, need, None) == kvq.KVQ_ERR_INVALID_ARG
     assert _status("kvq_decode_attention", ctypes.byref(cfg), ctypes.byref(c), None, 0x200000, ctypes.c_float(0.1),
                    0x300000, need, None) == kvq.KVQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("P,pages,layout,theta,status", [
+    (128, 8, 1, 0.0, kvq.KVQ_OK), (512, 2, 1, 0.0, kvq.KVQ_OK), (1024, 1, 1, 0.0, kvq.KVQ_OK),
+    (64, 8, 1, 0.0, kvq.KVQ_ERR_INVALID_ARG),     # not a multiple of 128
+    (384, 8, 1, 0.0, kvq.KVQ_ERR_INVALID_ARG),    # does not divide the capacity
+    (128, 0, 1, 0.0, kvq.KVQ_ERR_INVALID_ARG),    # an empty pool
+    (-128, 8, 1, 0.0, kvq.KVQ_ERR_INVALID_ARG),
+    (128, 8, 2, 0.0, kvq.KVQ_ERR_UNSUPPORTED),    # paging exists for tile v1 only
+    (128, 8, 2, 10000.0, kvq.KVQ_ERR_UNSUPPORTED),
+])
+def test_paged_config_validation(P, pages, layout, theta, status):
+    cfg = kvq.make_config(2, 8, 2, 2, 2, 32, 32, 0, 1024, layout=layout, rope_theta=theta, page_tokens=P,
+                          num_pages=pages)
+    sizes = (ctypes.c_size_t * 8)()
+    assert _status("kvq_cache_buffer_bytes", ctypes.byref(cfg), sizes) == status
+
+
+@pytest.mark.parametrize("P,pages,outliers", [(128, 37, 0), (512, 5, 1), (256, 1000, 1)])
+def test_paged_buffer_bytes_are_pool_sized(P, pages, outliers):
+    # the six per-token buffers (and the outlier words) hold num_pages pages of P tokens; the fp16
+    # ring stays per unit
+    B, Hkv, G, R, cap = 3, 2, 32, 64, 2048
+    paged = kvq.make_config(B, 8, Hkv, 4, 2, G, R, 0, cap, outliers=outliers, page_tokens=P, num_pages=pages)
+    got = kvq.kvq_cache_buffer_bytes(paged)
+    want = [pages * P * 128 * 4 // 8, pages * P * 128 * 2 // 8, pages * (P // G) * 128 * 2,
+            pages * (P // G) * 128 * 2, pages * P * (128 // G) * 2, pages * P * (128 // G) * 2]
+    assert got[:6] == want
+    contiguous = kvq.make_config(B, 8, Hkv, 4, 2, G, R, 0, cap, outliers=outliers)
+    assert got[6:] == kvq.kvq_cache_buffer_bytes(contiguous)[6:]
+    assert kvq.kvq_outlier_buffer_bytes(paged) == ([pages * P * 4] * 2 if outliers else [0, 0])
+
+
+def _paged_fake_cache(cfg, lens, table):
+    c, host = _fake_cache(cfg, lens)
+    c.page_table_host = table.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    c.page_table_dev = 0xA0000
+    return c, host
+
+
+@pytest.mark.parametrize("bad", [-1, 4, 1 << 20])
+def test_paged_prefill_rejects_table_entries_outside_the_pool(bad):
+    # a page that would hold quantized tokens (T = 300, R = 32, G = 32: Q = 256, pages 0 and 1 of 128)
+    # must map into the pool; the call is refused on the host before anything is copied or launched
+    cfg = kvq.make_config(1, 2, 1, 2, 2, 32, 32, 0, 512, page_tokens=128, num_pages=4)
+    table = np.array([[[0, bad, -1, -1]]], np.int32)
+    c, _ = _paged_fake_cache(cfg, [0], table)
+    k = ctypes.c_void_p(0x100000)
+    lens = np.array([300], np.int64)
+    st = _lib.lib.kvq_quantize_prefill(ctypes.byref(cfg), ctypes.byref(c), k, k, 300 * 128, 128, 128,
+                                       lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_paged_append_and_decode_check_the_table():
+    # append: the flush that takes the quantized part into page 1 needs that page; decode: every page
+    # of the quantized part
+    cfg = kvq.make_config(1, 2, 1, 2, 2, 32, 32, 0, 512, page_tokens=128, num_pages=4)
+    table = np.array([[[2, -1, -1, -1]]], np.int32)
+    c, host = _paged_fake_cache(cfg, [159], table)  # Q = 96 -> 128 after this append: still page 0
+    kn = ctypes.c_void_p(0x100000)
+    host[0] = 191  # Q = 128 now; the append brings Q to 160, into page 1
+    assert _lib.lib.kvq_append_token(ctypes.byref(cfg), ctypes.byref(c), kn, kn, None) == kvq.KVQ_ERR_INVALID_ARG
+    host[0] = 200  # Q = 160: decode reads pages 0 and 1
+    ws = ctypes.c_void_p(0x200000)
+    st = _lib.lib.kvq_decode_attention(ctypes.byref(cfg), ctypes.byref(c), kn, kn, ctypes.c_float(0.1), ws,
+                                       1 << 30, None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+    c.page_table_host = None  # a paged cache without its table
+    host[0] = 0
+    assert _lib.lib.kvq_append_token(ctypes.byref(cfg), ctypes.byref(c), kn, kn, None) == kvq.KVQ_ERR_INVALID_ARG
 
 
 def _header_struct(name, path=os.path.join("include", "kvq.h")):

@@ -21,6 +21,9 @@ def test_decode_bytes_closed_form():
     # the sink adds the first token's fp16 key and value row once a group is quantized
     assert bench.decode_bytes(w, np.full(8, T), sink=1) == want + 8 * 32 * 512
     assert bench.decode_bytes(w, np.full(8, 100), sink=1) == bench.decode_bytes(w, np.full(8, 100))
+    # outliers: a 4-byte key and a 4-byte value word per quantized token
+    Q = (T - w.residual) // w.group_size * w.group_size
+    assert bench.decode_bytes(w, np.full(8, T), outliers=1) == want + 8 * w.num_kv_heads * Q * 8
 
 
 def test_prefill_bytes_closed_form():

@@ -86,8 +86,9 @@ def host_cuda(monkeypatch):
 
 
 @pytest.mark.parametrize("opts,launches", [([], 4), (["--layout", "2", "--sink", "1"], 4),
-                                           (["--layout", "2", "--rope", "10000"], 5)],
-                         ids=["tile_v1", "rows_v2_sink", "rows_v2_rope"])
+                                           (["--layout", "2", "--rope", "10000"], 5),
+                                           (["--outliers", "1"], 4), (["--page-tokens", "128", "--outliers", "1"], 4)],
+                         ids=["tile_v1", "rows_v2_sink", "rows_v2_rope", "outliers", "paged_outliers"])
 def test_gpu_arm_host_logic_prints_a_complete_line(host_cuda, capsys, monkeypatch, opts, launches):
     calls, w = host_cuda
     steps, warmup = 4, 3
@@ -109,7 +110,8 @@ def test_gpu_arm_host_logic_prints_a_complete_line(host_cuda, capsys, monkeypatc
     assert line["workload_appends"]["n"] == 40
     # bytes per timed step from the lengths each decode saw: prefill 300 + 40 appends + warm-up
     lens = np.full(w.batch, 300 + 40 + warmup, np.int64)
-    want = sum(bench.decode_bytes(w, lens + i + 1, sink=1 if "--sink" in opts else 0) for i in range(steps))
+    want = sum(bench.decode_bytes(w, lens + i + 1, sink=1 if "--sink" in opts else 0,
+                                  outliers=1 if "--outliers" in opts else 0) for i in range(steps))
     assert line["value"] == pytest.approx(want / (line["ms_per_step"] * steps * 1e-3) / 1e9, rel=1e-3)
     k, v, _ = inputs.full_kv(w)
     assert line["input_sha256"] == bench.input_digest(k.numpy(), v.numpy(), inputs.query(w).numpy())
