@@ -236,9 +236,11 @@ kvq_status kvq_quantize_prefill(const kvq_config* cfg, kvq_cache* cache, const v
   if ((s = check_pages(cfg, cache, seq_lens)) != KVQ_OK) return s;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   std::memcpy(cache->seq_len_host, seq_lens, sizeof(int64_t) * cfg->batch);
-  cudaError_t e = cudaMemcpyAsync(cache->seq_len_dev, cache->seq_len_host, sizeof(int64_t) * cfg->batch,
-                                  cudaMemcpyHostToDevice, stream);
-  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  // The lengths reach the device by value (kernel arguments), never by a queued copy of host memory
+  // that a later call rewrites.
+  if (kvq::launch_set_lengths(static_cast<int64_t*>(cache->seq_len_dev), cache->seq_len_host, cfg->batch, stream) !=
+      cudaSuccess)
+    return KVQ_ERR_CUDA;
   if (cfg->page_tokens > 0 && upload_pages(cfg, cache, stream) != cudaSuccess) return KVQ_ERR_CUDA;
   QuantizeArgs a = quantize_args(cfg, cache);
   a.k = static_cast<const uint16_t*>(k);
@@ -272,7 +274,7 @@ kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache, const void*
     if (enters && upload_pages(cfg, cache, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return KVQ_ERR_CUDA;
   }
   QuantizeArgs a = quantize_args(cfg, cache);
-  const kvq_status r = cuda_status(kvq::launch_append(a, static_cast<const uint16_t*>(k_new),
+  const kvq_status r = cuda_status(kvq::launch_append(a, cache->seq_len_host, static_cast<const uint16_t*>(k_new),
                                                       static_cast<const uint16_t*>(v_new),
                                                       static_cast<cudaStream_t>(cuda_stream)));
   if (r == KVQ_OK)

@@ -72,8 +72,24 @@ struct DecodeArgs {
   float2* rope_off;   // workspace: (cos, sin)(j w_i), [32][64]
 };
 
+// Sequence lengths of up to kLenChunk consecutive sequences [base, base + n), passed to a kernel by
+// value. The host never hands the device a pointer to its length array: a queued copy from caller
+// memory that the library rewrites on the next call could otherwise read the later value.
+constexpr int kLenChunk = 256;
+struct LenChunk {
+  int64_t base;
+  int32_t n;
+  int32_t pad;
+  int64_t len[kLenChunk];
+};
+
+// Write lens[0 .. batch) into the device mirror (one small launch per kLenChunk sequences).
+cudaError_t launch_set_lengths(int64_t* seq_len_dev, const int64_t* lens, int batch, cudaStream_t stream);
 cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream);
-cudaError_t launch_append(const QuantizeArgs& a, const uint16_t* k_new, const uint16_t* v_new, cudaStream_t stream);
+// Append one token to every sequence; old_lens[b] is sequence b's length before the append (the host
+// mirror). The launch also writes the new lengths into the device mirror.
+cudaError_t launch_append(const QuantizeArgs& a, const int64_t* old_lens, const uint16_t* k_new, const uint16_t* v_new,
+                          cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);     // split + combine, either layout
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // rows-v2 split kernel only
 cudaError_t launch_decode_rope(const DecodeArgs& a, cudaStream_t stream);  // pre-RoPE keys: tables + split kernel

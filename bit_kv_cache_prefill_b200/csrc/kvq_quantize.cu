@@ -207,16 +207,18 @@ __device__ void quantize_values_chunk(const QuantizeArgs& a, int64_t slot, int64
   }
 }
 
-// Append one token to every (sequence, KV head) and flush a full group out of the window.
-// Lengths are read from the device mirror and not modified here (bump_lengths_kernel follows).
-__global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint16_t* __restrict__ k_new,
+// Append one token to every (sequence, KV head) of the chunk's sequences and flush a full group out
+// of the window. Each CTA takes its sequence's old length from the by-value chunk, so no CTA reads
+// the device mirror, and the key CTA of KV head 0 stores the new length there: one launch per chunk.
+__global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const LenChunk lens, const uint16_t* __restrict__ k_new,
                                                      const uint16_t* __restrict__ v_new) {
   extern __shared__ __align__(16) uint8_t smem[];
-  const int64_t unit = blockIdx.x;
+  const int64_t unit = lens.base * a.num_kv_heads + blockIdx.x;
   const bool is_key = blockIdx.y == 0;
   const int64_t b = unit / a.num_kv_heads;
   const int G = a.G;
-  const int64_t t = a.seq_len[b];
+  const int64_t t = lens.len[blockIdx.x / a.num_kv_heads];
+  if (is_key && threadIdx.x == 0 && blockIdx.x % a.num_kv_heads == 0) a.seq_len[b] = t + 1;
   const int64_t Q_old = quantized_len(t, a.R, G);
   const int64_t Q_new = quantized_len(t + 1, a.R, G);
   uint16_t* rows = reinterpret_cast<uint16_t*>(smem);
@@ -268,24 +270,45 @@ __global__ void __launch_bounds__(256) append_kernel(QuantizeArgs a, const uint1
     quantize_values_chunk(a, slot, ts0, Q_old, rows, pbuf, och);
 }
 
-__global__ void bump_lengths_kernel(int64_t* seq_len, int batch) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < batch) seq_len[b] += 1;
+__global__ void set_lengths_kernel(int64_t* seq_len, const LenChunk lens) {
+  const int i = threadIdx.x;
+  if (i < lens.n) seq_len[lens.base + i] = lens.len[i];
 }
 
 // ---- host launchers ---------------------------------------------------------------------------------
-cudaError_t launch_append(const QuantizeArgs& a, const uint16_t* k_new, const uint16_t* v_new, cudaStream_t stream) {
+static LenChunk make_chunk(const int64_t* lens, int batch, int base) {
+  LenChunk c;
+  c.base = base;
+  c.n = batch - base < kLenChunk ? batch - base : kLenChunk;
+  c.pad = 0;
+  for (int i = 0; i < kLenChunk; ++i) c.len[i] = i < c.n ? lens[base + i] : 0;
+  return c;
+}
+
+cudaError_t launch_set_lengths(int64_t* seq_len_dev, const int64_t* lens, int batch, cudaStream_t stream) {
+  for (int base = 0; base < batch; base += kLenChunk) {
+    set_lengths_kernel<<<1, kLenChunk, 0, stream>>>(seq_len_dev, make_chunk(lens, batch, base));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_append(const QuantizeArgs& a, const int64_t* old_lens, const uint16_t* k_new, const uint16_t* v_new,
+                          cudaStream_t stream) {
   const size_t smem = chunk_smem_bytes(a.G);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads), 2);
-  append_kernel<<<grid, 256, smem, stream>>>(a, k_new, v_new);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  bump_lengths_kernel<<<(a.batch + 255) / 256, 256, 0, stream>>>(a.seq_len, a.batch);
-  return cudaGetLastError();
+  for (int base = 0; base < a.batch; base += kLenChunk) {
+    const LenChunk c = make_chunk(old_lens, a.batch, base);
+    const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(c.n) * a.num_kv_heads), 2);
+    append_kernel<<<grid, 256, smem, stream>>>(a, c, k_new, v_new);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace kvq

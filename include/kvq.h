@@ -139,7 +139,10 @@ typedef struct {
  * distinct pool pages, and an entry must not change while its page holds tokens.
  * page_table_host is the caller's table in host memory; page_table_dev is its device mirror (caller-
  * allocated, same shape), written by the library on the stream: the whole table is copied on every
- * prefill and on every append in which some unit's quantized part enters a new page.
+ * prefill and on every append in which some unit's quantized part enters a new page. That copy is an
+ * asynchronous host-to-device copy: if page_table_host is pinned, the caller must not change it
+ * until the stream has passed the call (from pageable memory the copy is staged before the call
+ * returns).
  *
  * Tile v1: tile row k of a unit holds tokens 16k..16k+15. Within a tile, "lane" L (0..31) owns
  * words (w / 4) * 128 + 4L + (w % 4) for w in [0, 2*bits). Word w holds 16/bits code pairs; pair j
@@ -157,8 +160,12 @@ typedef struct {
  *   values: token t lies in block t/128 at i = t%128; channel c's row of that block holds token
  *           pair j = i/2 in word j/P as pair j%P (token 2j first).
  *
- * seq_len_host: int64 [batch] in host memory, read and updated by the library.
- * seq_len_dev:  int64 [batch] in device memory, the device mirror, updated on the stream.
+ * seq_len_host: int64 [batch] in host memory, read and updated by the library on the calling thread.
+ *               The library never queues a copy from it: lengths reach the device as kernel
+ *               arguments, so the array may be pageable or pinned and is free to change as soon
+ *               as a call returns.
+ * seq_len_dev:  int64 [batch] in device memory, the device mirror, written by kernels on the stream
+ *               (prefill, and each append for the new lengths).
  */
 typedef struct {
   void* k_codes;

@@ -130,13 +130,26 @@ def compare_unit_cache(w: inputs.Workload, gv: Dict[str, np.ndarray], b: int, h:
             np.testing.assert_array_equal(gv[key][b, h, ring], getattr(oc, key)[ob, oh, ring], err_msg=f"{key} sink row {b},{h}")
 
 
+def fp16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of binary16 values at |x| (2^-24 in the subnormal range)."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -14)))
+    return 2.0 ** (e - 10)
+
+
 def check_attention(gpu_out: np.ndarray, ref: np.ndarray, what: str) -> Tuple[float, float]:
+    """Max-abs and relative-L2 error of the fp16 output against the fp64 oracle. The absolute bound is
+    MAX_ABS_TOL where fp16 can hold it, i.e. for |out| < 4; a larger output element (a planted value
+    outlier of hundreds) is held to one fp16 spacing at its magnitude, since rounding the output to
+    fp16 alone moves it by up to half of one."""
     gpu = gpu_out.astype(np.float64)
     err = np.abs(gpu - ref)
     max_abs = float(err.max()) if err.size else 0.0
     denom = float(np.linalg.norm(ref))
     rel = float(np.linalg.norm(gpu - ref) / denom) if denom > 0 else float(np.linalg.norm(gpu))
-    assert max_abs <= MAX_ABS_TOL, f"{what}: max abs error {max_abs:.3e} > {MAX_ABS_TOL}"
+    tol = np.maximum(MAX_ABS_TOL, fp16_ulp(ref))
+    if err.size and not (err <= tol).all():
+        i = int(np.argmax(err - tol))
+        raise AssertionError(f"{what}: max abs error {err.flat[i]:.3e} > {tol.flat[i]:.3e} at |out| = {abs(ref.flat[i]):.3g}")
     assert rel <= REL_L2_TOL, f"{what}: relative L2 error {rel:.3e} > {REL_L2_TOL}"
     return max_abs, rel
 
