@@ -89,6 +89,24 @@ def flush_steps(w: inputs.Workload, lens_before: np.ndarray, steps: int) -> List
     return [bool((q(lens_before + i + 1) > q(lens_before + i)).any()) for i in range(steps)]
 
 
+def align_pad(w: inputs.Workload, lens: np.ndarray, steps: int) -> int:
+    """Appends to make before `steps` timed appends from lengths `lens` so that the first append that
+    flushes a group (in the longest sequence) is timed step steps // 2 (0 if it would already fall
+    inside the timed steps without padding before that point)."""
+    G, R = w.group_size, w.residual
+    T = int(np.max(lens))
+    # append i (0-based) makes the length T + i + 1; it flushes when (T + i + 1 - R) is a positive multiple of G
+    first = next(i for i in range(G) if T + i + 1 - R > 0 and (T + i + 1 - R) % G == 0)
+    want = min(steps // 2, G - 1)
+    return (first - want) % G
+
+
+def align_appends(w: inputs.Workload, lens: np.ndarray, steps: int):
+    """The padding appends of align_pad (seeded tokens after the workload's own)."""
+    n = align_pad(w, lens, steps)
+    return [inputs.append_tokens(w, 10_000 + s) for s in range(n)]
+
+
 def kv_tokens(w: inputs.Workload, lens: np.ndarray) -> int:
     """Cached (token, KV head) pairs one decode call scans."""
     return int(np.asarray(lens, np.int64).sum()) * w.num_kv_heads
@@ -306,8 +324,10 @@ def oracle_decode_sample(w: inputs.Workload, budget_s: float = 15.0, layout: int
     return OracleSample(per_call * calls / spent / 1e9, threads, desc, single, pre / t_pre / 1e9)
 
 
-def workload_config(w: inputs.Workload, args, step_bytes: int) -> dict:
-    """The JSON line's config, the same for both arms."""
+def workload_config(w: inputs.Workload, args) -> dict:
+    """The JSON line's config, the same for both arms (a function of the workload and the options only:
+    the read size quoted is that of a decode at the workload's lengths after its own appends)."""
+    step_bytes = decode_bytes(w, w.seq_lens() + w.appends, args.sink, args.outliers)
     return {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "num_q_heads": w.num_q_heads,
             "num_kv_heads": w.num_kv_heads, "key_bits": w.key_bits, "value_bits": w.value_bits,
             "group_size": w.group_size, "residual": w.residual, "hadamard": w.hadamard,
@@ -339,7 +359,7 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_bytes / (value * 1e9) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, args, step_bytes),
+        "config": workload_config(w, args),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
                          "prefill_value": round(pre_gbs, 4), "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -356,7 +376,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="llama2_7b_mha", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--workload", default="llama3_8b_gqa", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--prefill-iters", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -402,7 +422,7 @@ def main():
         torch.cuda.synchronize()
 
     # capacity for the prefill plus every appended token of this run
-    n_app = w0.appends + args.warmup + args.steps + (1 if not args.no_e2e else 0) * (args.steps + args.warmup)
+    n_app = w0.appends + args.warmup + args.steps + w0.group_size + (1 if not args.no_e2e else 0) * (args.steps + args.warmup)
     w = w0.scaled(appends=n_app)
     lens0 = w0.seq_lens()
     k, v, _ = inputs.full_kv(w0)  # CPU, seeded
@@ -467,6 +487,10 @@ def main():
 
     for i in range(args.warmup):
         step(i)
+    # untimed appends (at most G - 1) so that the first group flush after warm-up falls in the middle of
+    # the timed steps: the timed region then holds the flush cost of one step in G
+    for kn, vn in align_appends(w0, cache.seq_len_host, args.steps):
+        kvq.kvq_append_token(cfg, cache, kn.cuda(), vn.cuda())
     barrier()
     lens_before = cache.seq_len_host.copy()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -553,7 +577,7 @@ def main():
         "vs_baseline": None,
         "dtype": "u2/u4 codes, fp16 in/out, fp32 accumulate",
         "data": "synthetic",
-        "config": workload_config(w0, args, step_bytes[0]),
+        "config": workload_config(w0, args),
         "tokens_per_s": round(tokens / (total_ms * 1e-3), 1),
         "frac_of_nominal_8tbs": round(value / NOMINAL_HBM_GBS, 4),
         "decode_ms": round(mean_decode_ms, 4),
@@ -573,8 +597,9 @@ def main():
                     "frac": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9 / peak, 4),
                     "traffic": measured_traffic(w0, args.layout, "prefill", args.sink, args.rope, args.outliers, args.page_tokens),
                     "kernel": "prefill_block_kernel (one kvq_quantize_prefill call)"},
-        # per step: append + length bump, then the decode split kernel + combine (+ the RoPE angle tables)
-        "gpu_launches": (5 if args.rope > 0 else 4) * args.steps,
+        # per step: append (one launch per 256 sequences), then the decode split kernel + combine (+ the
+        # RoPE angle tables)
+        "gpu_launches": (-(-w.batch // 256) + (3 if args.rope > 0 else 2)) * args.steps,
         "clocks": clocks.summary(),
         "input_sha256": digest,  # prefill K, V (fp16 [B][T][Hkv][128], zero past each length) and q
         # the workload's own appends before the timed steps (e.g. 256 per sequence), one event pair each

@@ -85,9 +85,9 @@ def host_cuda(monkeypatch):
     return calls, w
 
 
-@pytest.mark.parametrize("opts,launches", [([], 4), (["--layout", "2", "--sink", "1"], 4),
-                                           (["--layout", "2", "--rope", "10000"], 5),
-                                           (["--outliers", "1"], 4), (["--page-tokens", "128", "--outliers", "1"], 4)],
+@pytest.mark.parametrize("opts,launches", [([], 3), (["--layout", "2", "--sink", "1"], 3),
+                                           (["--layout", "2", "--rope", "10000"], 4),
+                                           (["--outliers", "1"], 3), (["--page-tokens", "128", "--outliers", "1"], 3)],
                          ids=["tile_v1", "rows_v2_sink", "rows_v2_rope", "outliers", "paged_outliers"])
 def test_gpu_arm_host_logic_prints_a_complete_line(host_cuda, capsys, monkeypatch, opts, launches):
     calls, w = host_cuda
@@ -104,12 +104,15 @@ def test_gpu_arm_host_logic_prints_a_complete_line(host_cuda, capsys, monkeypatc
     assert set(line["roofline"]) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
     assert set(line["cpu_baseline"]) >= {"value", "unit", "cores", "kind", "sample"}
     assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
-    # the workload's 40 appends, the warm-up steps, the timed steps, then the end-to-end steps
-    assert calls["prefill"] == 3 and calls["append"] == 40 + warmup + 2 * steps
+    # the workload's 40 appends, the warm-up steps, the padding that puts a group flush inside the
+    # timed steps, the timed steps, then the end-to-end steps
+    pad = bench.align_pad(w, np.full(w.batch, 300 + 40 + warmup, np.int64), steps)
+    assert calls["prefill"] == 3 and calls["append"] == 40 + warmup + pad + 2 * steps
     assert calls["decode"] == warmup + 2 * steps
     assert line["workload_appends"]["n"] == 40
-    # bytes per timed step from the lengths each decode saw: prefill 300 + 40 appends + warm-up
-    lens = np.full(w.batch, 300 + 40 + warmup, np.int64)
+    assert line["append_flush_us"] is not None  # a flush fell inside the timed steps
+    # bytes per timed step from the lengths each decode saw: prefill 300 + 40 appends + warm-up + padding
+    lens = np.full(w.batch, 300 + 40 + warmup + pad, np.int64)
     want = sum(bench.decode_bytes(w, lens + i + 1, sink=1 if "--sink" in opts else 0,
                                   outliers=1 if "--outliers" in opts else 0) for i in range(steps))
     assert line["value"] == pytest.approx(want / (line["ms_per_step"] * steps * 1e-3) / 1e9, rel=1e-3)
