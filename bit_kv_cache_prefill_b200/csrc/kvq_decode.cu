@@ -10,9 +10,9 @@
 // Work split. The grid is (split, unit) with unit = (sequence, KV head). A CTA of 4 warps owns one
 // token range of split_len tokens; each warp owns a contiguous run of 16-token tiles of it (so a key
 // group's query fold is built once per group per warp) and round-robin the FP16 residual tokens.
-// Tiles stream through a per-warp 3-stage cp.async ring of steps of 1 or 2 tiles (codes, value
-// scale/zero and, at a key-block boundary, the block's key scale/zero), so up to 6 tiles per warp are
-// in flight.
+// Tiles stream through a per-warp cp.async ring (codes, value scale/zero and, at a key-block
+// boundary, the block's key scale/zero): 3 stages of steps of 1 or 2 tiles, or 2 stages of 4-tile
+// steps for 2-bit caches with G >= 64, so up to 6 or 8 tiles per warp are in flight.
 //
 // Arithmetic (per 16-token tile; scores in base-2 units, q already multiplied by sm_scale*log2 e):
 //   QK: s_t = 2^e * (sum_c code[t][c] * (q^[c] * sk[g][c]) + sum_c q^[c] * zk[g][c]), q^ = q * 2^-e.
@@ -47,7 +47,6 @@
 namespace kvq {
 namespace {
 
-constexpr int kStages = 3;  // pipeline stages per warp (each one step of 1 or 2 tiles)
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -73,13 +72,17 @@ __device__ __forceinline__ void cp_async_wait() {
 // Per-warp pipeline: a ring of kStages stages, each holding one step of TS 16-token tiles (codes
 // and value scale/zero), plus a ring of KP slots holding the key scale and zero of the KGB key groups
 // of one key block. A key block spans kBlockSteps steps; its parameters are read only when the
-// block's first step is consumed. Step j is issued at the top of iteration j - (kStages - 1) = j - 2,
-// so a new block's parameters may land in the slot of the block two back only once that block's
-// first step has been consumed: with kBlockSteps >= 2 this holds for two slots (a partial first
-// block plus a full block lie in between); one-step blocks use four slots (three blocks lie in
-// between). With OUT a stage also holds the key and value outlier words of the step's tokens.
+// block's first step is consumed. Step j is issued at the top of iteration j - (kStages - 1) (j - 2,
+// or j - 1 with two stages), so a new block's parameters may land in the slot of the block two back
+// only once that block's first step has been consumed: with kBlockSteps >= 2 this holds for two
+// slots (a partial first block plus a full block lie in between); one-step blocks use four slots
+// (three blocks lie in between). With OUT a stage also holds the key and value outlier words of the
+// step's tokens.
 template <int KB, int VB, int VPT, int KGB, int TS, bool OUT>
 struct Stage {
+  // 3 stages of steps of 1 or 2 tiles, or 2 stages of 4-tile steps (the same 8 tiles in flight in less
+  // shared memory, so that 4 CTAs still fit an SM)
+  static constexpr int kStages = TS >= 4 ? 2 : 3;
   static constexpr int kKC = 256 * KB * TS;  // key codes of the step's tiles
   static constexpr int kVC = 256 * VB * TS;  // value codes
   static constexpr int kVS = 32 * VPT * TS;  // value scale (or zero) of the step's tokens
@@ -114,7 +117,9 @@ struct Shape {
   static constexpr int VGB = 4 / GQ;                     // value groups per PV n-block
   static constexpr int NBV = (VPT + VGB - 1) / VGB;      // PV n-blocks
   static constexpr int G = 128 / VPT;
-  static constexpr int TS = G >= 32 ? 2 : 1;             // tiles per step
+  // tiles per step: 4 for 2-bit keys and values with G >= 64 (a step never spans two key groups),
+  // which halves the per-step pipeline and softmax bookkeeping per tile
+  static constexpr int TS = (KB == 2 && VB == 2 && G >= 64) ? 4 : (G >= 32 ? 2 : 1);
   using S = Stage<KB, VB, VPT, KGB, TS, OUT>;
 };
 
@@ -279,6 +284,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   const int sb = min(nsteps, per * warp);
   const int nst = min(nsteps, per * (warp + 1)) - sb;
   uint8_t* ring = rings + warp * S::kWarpBytes;
+  constexpr int kStages = S::kStages;
   uint8_t* kp_ring = ring + kStages * S::kBytes;
   const int first_token = start + sb * kStepTokens;
   const int q_groups = Q / G;

@@ -7,6 +7,7 @@ the FP16 window, R = 0, flush boundaries); the model-shaped workloads run at ful
 oracle checking sampled (sequence, KV head) units.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -150,41 +151,30 @@ def test_sm_scale_and_single_token(oracle_mod, layout):
     H.check_attention(run2.out.cpu().numpy(), ref2, "sm_scale 0.02")
 
 
-# ---- model-shaped workloads at full size; the oracle checks sampled units -------------------------
+# ---- model-shaped workloads at full size, in the launch configuration the bench uses: the oracle
+#      runs the whole workload (multi-threaded) and every unit's cache and every output is compared
 FULL = ["tiny", "llama2_7b_mha", "llama3_8b_gqa", "mistral_7b_ragged", "million_token"]
-
-
-def _sample_units(w, lens):
-    B, Hkv = w.batch, w.num_kv_heads
-    picks = {(0, 0), (B - 1, Hkv - 1), (B // 2, Hkv // 2)}
-    if w.ragged_min:
-        picks |= {(int(np.argmax(lens)), 0), (int(np.argmin(lens)), Hkv - 1)}
-    if w.seq_len >= 1 << 20:
-        picks = {(0, Hkv - 1)}
-    return sorted(picks)
 
 
 @pytest.mark.parametrize("layout", LAYOUTS, ids=["tile_v1", "rows_v2"])
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_workload_sampled(oracle_mod, name, layout):
+def test_full_size_workload_every_unit(oracle_mod, name, layout):
     w = inputs.WORKLOADS[name]
     k, v, lens = inputs.full_kv(w)
     q = inputs.query(w)
     run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, appends=w.appends, layout=layout)
-    del k, v
     gv = H.gpu_views(w, run)
     out = run.out.cpu().numpy()
-    refs, gots = [], []
-    for b, h in _sample_units(w, lens):
-        oc, ref = H.oracle_unit(oracle_mod, w, b, h, int(lens[b]), q, appends=w.appends, layout=layout)
-        H.compare_unit_cache(w, gv, b, h, oc, 0, 0, int(lens[b]) + w.appends, layout=layout)
-        got = out[b, h * w.gqa:(h + 1) * w.gqa]
-        H.check_attention(got, ref, f"{name} unit ({b},{h})")
-        refs.append(ref)
-        gots.append(got)
-    H.check_attention(np.concatenate(gots), np.concatenate(refs), f"{name} sampled units")
-    # every output is finite and the lengths advanced by the appends
-    assert np.isfinite(out.astype(np.float32)).all()
+    threads = len(os.sched_getaffinity(0))
+    oc, ref = H.oracle_full(oracle_mod, w, k, v, lens, q, appends=w.appends, layout=layout, threads=threads)
+    del k, v
+    units = 0
+    for b in range(w.batch):
+        for h in range(w.num_kv_heads):
+            H.compare_unit_cache(w, gv, b, h, oc, b, h, int(lens[b]) + w.appends, layout=layout)
+            units += 1
+    assert units == w.batch * w.num_kv_heads
+    H.check_attention(out, ref, f"{name}, all {w.batch * w.num_q_heads} query heads")
     assert np.array_equal(run.cache.seq_len_host, lens + w.appends)
 
 
