@@ -239,8 +239,13 @@ def measured_traffic(w: inputs.Workload, layout: int, kind: str = "decode", sink
             h.update(open(os.path.join(root, f), "rb").read())
         if h.hexdigest() != e["sources_sha256"]:
             return None
-        units = w.batch * w.num_kv_heads
-        return int(round((e["dram_read_bytes"] + e["dram_write_bytes"]) * units / e["capture_units"]))
+        # traffic grows with the units processed; a capture at a reduced prefill length records its
+        # (token, KV head) pairs, and then scales by those instead
+        if "capture_tokens" in e:
+            scale = float(np.sum(w.seq_lens())) * w.num_kv_heads / e["capture_tokens"]
+        else:
+            scale = w.batch * w.num_kv_heads / e["capture_units"]
+        return int(round((e["dram_read_bytes"] + e["dram_write_bytes"]) * scale))
     return None
 
 
@@ -382,6 +387,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling captures)")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override the workload's prefill length (profiling captures of single-sequence workloads)")
     ap.add_argument("--layout", type=int, default=1, choices=[1, 2],
                     help="packed layout: 1 = tile v1 (mma.sync decode), 2 = rows v2 (tcgen05 decode)")
     ap.add_argument("--sink", type=int, default=0, choices=[0, 1],
@@ -398,6 +405,8 @@ def main():
     w0 = inputs.WORKLOADS[args.workload]
     if args.batch > 0:
         w0 = w0.scaled(batch=args.batch)
+    if args.seq_len > 0:
+        w0 = w0.scaled(seq_len=args.seq_len, ragged_min=min(w0.ragged_min, args.seq_len))
 
     if args.impl == "reference":
         return run_reference(args, w0)

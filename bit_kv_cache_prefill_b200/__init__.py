@@ -11,6 +11,7 @@ _BINDING_NAMES = {
     "kvq_cache_buffer_bytes", "kvq_config", "kvq_decode_attention", "kvq_decode_workspace_bytes",
     "kvq_quantize_prefill", "kvq_status_string", "make_config", "kvq_decode_attention_noalloc",
     "STATIC_SCRATCH_BYTES", "KVQ_LAYOUT_TILE_V1", "KVQ_LAYOUT_ROWS_V2", "kvq_outlier_buffer_bytes",
+    "KVQ_ERR_TIMEOUT", "kvq_decode_status",
 }
 
 

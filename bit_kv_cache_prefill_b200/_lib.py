@@ -22,6 +22,7 @@ KVQ_ERR_UNSUPPORTED = -2
 KVQ_ERR_CAPACITY = -3
 KVQ_ERR_WORKSPACE = -4
 KVQ_ERR_CUDA = -5
+KVQ_ERR_TIMEOUT = -6
 KVQ_LAYOUT_TILE_V1 = 1
 KVQ_LAYOUT_ROWS_V2 = 2
 BUFFER_NAMES = ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero", "k_res", "v_res")
@@ -71,6 +72,8 @@ def _load() -> ctypes.CDLL:
     L.kvq_decode_attention.restype = S
     L.kvq_decode_attention_noalloc.argtypes = [C, K, P, P, ctypes.c_float, P]
     L.kvq_decode_attention_noalloc.restype = S
+    L.kvq_decode_status.argtypes = [C, P, P]
+    L.kvq_decode_status.restype = S
     L.kvq_status_string.argtypes = [S]
     L.kvq_status_string.restype = ctypes.c_char_p
     return L
@@ -199,3 +202,12 @@ def kvq_decode_attention_noalloc(cfg: kvq_config, cache: Cache, q: torch.Tensor,
     assert q.is_contiguous() and out.is_contiguous()
     _check(lib.kvq_decode_attention_noalloc(ctypes.byref(cfg), ctypes.byref(cache.c), q.data_ptr(), out.data_ptr(),
                                             float(sm_scale), _stream_ptr(stream)), "kvq_decode_attention_noalloc")
+
+
+def kvq_decode_status(cfg: kvq_config, workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Status of the last decode that used ``workspace``: KVQ_OK or KVQ_ERR_TIMEOUT (other errors raise).
+    Synchronises the stream."""
+    st = lib.kvq_decode_status(ctypes.byref(cfg), workspace.data_ptr(), _stream_ptr(stream))
+    if st not in (KVQ_OK, KVQ_ERR_TIMEOUT):
+        raise KvqError(st, "kvq_decode_status")
+    return st

@@ -155,6 +155,26 @@ QuantizeArgs quantize_args(const kvq_config* c, kvq_cache* k) {
   return a;
 }
 
+int64_t max_splits(const kvq_config* c);
+
+// Decode workspace: split partials, then (pre-RoPE keys) the angle tables, then one status record per
+// (sequence, query head); each part starts 256-byte aligned.
+struct WorkspaceLayout {
+  size_t rope, status, total;
+};
+WorkspaceLayout workspace_layout(const kvq_config* c) {
+  const int64_t units = static_cast<int64_t>(c->batch) * c->num_kv_heads;
+  const int64_t g = c->num_q_heads / c->num_kv_heads;
+  const size_t part = static_cast<size_t>(units * max_splits(c) * g * kvq::kPartFloats) * sizeof(float);
+  WorkspaceLayout w;
+  w.rope = (part + 255) / 256 * 256;
+  size_t end = part;
+  if (c->rope_theta > 0.f) end = w.rope + static_cast<size_t>(kvq::rope_table_floats(c->capacity)) * 4;
+  w.status = (end + 255) / 256 * 256;
+  w.total = w.status + static_cast<size_t>(c->batch) * c->num_q_heads * 4;
+  return w;
+}
+
 int64_t max_splits(const kvq_config* c) {
   const int64_t units = static_cast<int64_t>(c->batch) * c->num_kv_heads;
   return std::max<int64_t>(1, (2 * kTargetCtas + units - 1) / units);
@@ -286,12 +306,28 @@ kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, size_t* bytes) {
   const kvq_status s = check_config(cfg);
   if (s != KVQ_OK) return s;
   if (bytes == nullptr) return KVQ_ERR_INVALID_ARG;
-  const int64_t units = static_cast<int64_t>(cfg->batch) * cfg->num_kv_heads;
-  const int64_t g = cfg->num_q_heads / cfg->num_kv_heads;
-  size_t part = static_cast<size_t>(units * max_splits(cfg) * g * kvq::kPartFloats) * sizeof(float);
-  if (cfg->rope_theta > 0.f) part = (part + 255) / 256 * 256 + static_cast<size_t>(kvq::rope_table_floats(cfg->capacity)) * 4;
-  *bytes = part;
+  *bytes = workspace_layout(cfg).total;
   return KVQ_OK;
+}
+
+kvq_status kvq_decode_status(const kvq_config* cfg, const void* workspace, void* cuda_stream) {
+  const kvq_status s = check_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (workspace == nullptr || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
+  const WorkspaceLayout w = workspace_layout(cfg);
+  const uint32_t* rec = reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(workspace) + w.status);
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  const int64_t n = static_cast<int64_t>(cfg->batch) * cfg->num_q_heads;
+  uint32_t buf[1024];  // the records, a chunk at a time (no host allocation)
+  bool gave_up = false;
+  for (int64_t i = 0; i < n; i += 1024) {
+    const int64_t m = std::min<int64_t>(1024, n - i);
+    if (cudaMemcpyAsync(buf, rec + i, static_cast<size_t>(m) * 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return KVQ_ERR_CUDA;
+    for (int64_t j = 0; j < m; ++j) gave_up |= buf[j] != 0;
+  }
+  return gave_up ? KVQ_ERR_TIMEOUT : KVQ_OK;
 }
 
 kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, const void* q, void* out, float sm_scale,
@@ -364,11 +400,11 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   a.split_len = L;
   a.nsplit = nsplit;
   a.qscale = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  const WorkspaceLayout wl = workspace_layout(cfg);
+  a.status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + wl.status);
   if (cfg->rope_theta > 0.f) {
-    const size_t part = static_cast<size_t>(static_cast<int64_t>(cfg->batch) * cfg->num_kv_heads * max_splits(cfg) *
-                                            a.gqa * kvq::kPartFloats) * sizeof(float);
     a.rope_theta = cfg->rope_theta;
-    a.rope_base = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + (part + 255) / 256 * 256);
+    a.rope_base = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + wl.rope);
     a.rope_off = a.rope_base + (cfg->capacity + 31) / 32 * 64;
   }
   return cuda_status(kvq::launch_decode(a, static_cast<cudaStream_t>(cuda_stream)));
@@ -382,6 +418,7 @@ const char* kvq_status_string(kvq_status status) {
     case KVQ_ERR_CAPACITY: return "sequence would exceed the cache capacity";
     case KVQ_ERR_WORKSPACE: return "decode workspace missing, misaligned or too small";
     case KVQ_ERR_CUDA: return "CUDA launch or copy failed";
+    case KVQ_ERR_TIMEOUT: return "a decode kernel gave up a bounded wait (its outputs are NaN)";
   }
   return "unknown status";
 }

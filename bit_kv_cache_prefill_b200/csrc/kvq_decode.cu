@@ -773,6 +773,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a)
   uint16_t* out = a.out + row * kHeadDim;
   if (T <= 0) {
     out[c] = 0;
+    if (c == 0) a.status[row] = 0u;
     return;
   }
   const int ns = static_cast<int>((T + a.split_len - 1) / a.split_len);
@@ -788,6 +789,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a)
     acc = fmaf(f, p[2 + c], acc);
   }
   out[c] = __half_as_ushort(__float2half_rn(acc / l));
+  // l is NaN only where a split kernel gave up a bounded wait and wrote a NaN partial (finite inputs)
+  if (c == 0) a.status[row] = l != l ? 1u : 0u;
 }
 
 template <int KB, int VB, int VPT, int GQ, bool OUT>

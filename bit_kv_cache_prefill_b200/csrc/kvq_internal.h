@@ -52,6 +52,7 @@ struct DecodeArgs {
   const uint16_t* q;       // fp16 [batch][Hq][128]
   uint16_t* out;           // fp16 [batch][Hq][128]
   float* part;             // split partials [units][nsplit][g][2 + 128]
+  uint32_t* status;        // [batch][Hq]: 1 where the output is NaN from a bounded wait that gave up
   int batch, num_q_heads, num_kv_heads, gqa, G, R, key_bits, value_bits, hadamard;
   int64_t capacity, tiles, groups, ring;
   int sink;          // 1: token 0 is read from ring row R+G (fp16) and masked in the quantized part

@@ -45,7 +45,8 @@ typedef enum {
   KVQ_ERR_UNSUPPORTED = -2, /* a configuration the library does not implement (e.g. head_dim != 128) */
   KVQ_ERR_CAPACITY = -3,    /* a sequence would exceed config.capacity tokens */
   KVQ_ERR_WORKSPACE = -4,   /* workspace missing or smaller than kvq_decode_workspace_bytes */
-  KVQ_ERR_CUDA = -5         /* a kernel launch or copy failed */
+  KVQ_ERR_CUDA = -5,        /* a kernel launch or copy failed */
+  KVQ_ERR_TIMEOUT = -6      /* kvq_decode_status: a decode kernel gave up a bounded wait (outputs NaN) */
 } kvq_status;
 
 /* Packed layouts (see kvq_cache below): "tile v1" feeds warp-level mma fragments, "rows v2" feeds
@@ -265,6 +266,19 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
 #define KVQ_STATIC_SCRATCH_BYTES (16u << 20)
 kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache* cache, const void* q, void* out,
                                         float sm_scale, void* cuda_stream);
+
+/* Outcome of the last decode call that used `workspace` for `cfg`. The source pages have no
+ * counterpart to this entry point; it reports a failure that the asynchronous decode call itself
+ * cannot. The rows-v2 (tcgen05) decode kernel waits on its own copies and tensor-core products with
+ * bounded waits (about 2 s); a CTA that gives up writes NaN partials instead of hanging, and the
+ * split combine then records, per (sequence, query head), whether its output came out NaN that way.
+ * Every decode call rewrites those records (they sit at the end of the workspace, within
+ * kvq_decode_workspace_bytes), so nothing needs clearing.
+ * This call copies the records to the host on `cuda_stream` and synchronises that stream: call it
+ * on the stream of the decode (or after it), before the workspace is reused.
+ * Returns KVQ_OK, KVQ_ERR_TIMEOUT if some output of that decode is NaN from a give-up, or
+ * KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED / KVQ_ERR_CUDA. */
+kvq_status kvq_decode_status(const kvq_config* cfg, const void* workspace, void* cuda_stream);
 
 /* Static description of a status code. */
 const char* kvq_status_string(kvq_status status);

@@ -23,8 +23,8 @@ def _declared_symbols():
 def test_library_exports_every_declared_entry_point():
     names = _declared_symbols()
     assert names == ["kvq_append_token", "kvq_cache_buffer_bytes", "kvq_decode_attention",
-                     "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes", "kvq_outlier_buffer_bytes",
-                     "kvq_quantize_prefill", "kvq_status_string"]
+                     "kvq_decode_attention_noalloc", "kvq_decode_status", "kvq_decode_workspace_bytes",
+                     "kvq_outlier_buffer_bytes", "kvq_quantize_prefill", "kvq_status_string"]
     lib = ctypes.CDLL(kvq.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -32,7 +32,7 @@ def test_library_exports_every_declared_entry_point():
 
 
 def test_status_strings():
-    for s in (0, -1, -2, -3, -4, -5):
+    for s in (0, -1, -2, -3, -4, -5, -6):
         assert kvq.kvq_status_string(s) and kvq.kvq_status_string(s) != "unknown status"
     assert kvq.kvq_status_string(7) == "unknown status"
 
@@ -113,9 +113,10 @@ def test_rope_workspace_holds_the_angle_tables(cap):
     base = kvq.make_config(1, 32, 8, 2, 2, 128, 128, 0, cap, layout=kvq.KVQ_LAYOUT_ROWS_V2)
     rope = kvq.make_config(1, 32, 8, 2, 2, 128, 128, 0, cap, layout=kvq.KVQ_LAYOUT_ROWS_V2, rope_theta=10000.0)
     assert kvq.kvq_cache_buffer_bytes(rope) == kvq.kvq_cache_buffer_bytes(base)
-    part = kvq.kvq_decode_workspace_bytes(base)
+    records = 1 * 32 * 4  # one u32 status record per (sequence, query head) closes the workspace
+    part = kvq.kvq_decode_workspace_bytes(base) - records  # partials, 256-byte aligned end
     tables = (-(-cap // 32) * 64 + 32 * 64) * 8
-    assert kvq.kvq_decode_workspace_bytes(rope) == -(-part // 256) * 256 + tables
+    assert kvq.kvq_decode_workspace_bytes(rope) == -(-(part + tables) // 256) * 256 + records
 
 
 @pytest.mark.parametrize("layout,theta,value,status", [
@@ -338,3 +339,20 @@ def test_binding_structs_match_the_header(name, binding, path):
         sz = 8 if ctype.endswith("*") else _SIZES[ctype]
         off = -(-off // sz) * sz + sz
     assert ctypes.sizeof(binding) == -(-off // 8) * 8
+
+
+def test_decode_workspace_ends_with_one_status_record_per_query_head():
+    """The workspace bound covers the split partials, the RoPE tables (pre-RoPE keys) and, 256-byte
+    aligned at the end, one u32 status record per (sequence, query head)."""
+    for B, Hq, Hkv, rope, layout in [(8, 32, 32, 0.0, 1), (16, 32, 8, 0.0, 1), (3, 8, 2, 10000.0, 2)]:
+        cfg = kvq.make_config(B, Hq, Hkv, 2, 2, 32, 32, 0, 4096, layout=layout, rope_theta=rope)
+        n = kvq.kvq_decode_workspace_bytes(cfg)
+        assert (n - B * Hq * 4) % 256 == 0 and n > B * Hq * 4
+
+
+def test_decode_status_rejects_bad_arguments():
+    cfg = kvq.make_config(2, 4, 2, 2, 2, 32, 32, 0, 1024)
+    assert _lib.lib.kvq_decode_status(ctypes.byref(cfg), None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert _lib.lib.kvq_decode_status(ctypes.byref(cfg), ctypes.c_void_p(0x1001), None) == kvq.KVQ_ERR_INVALID_ARG
+    bad = kvq.make_config(2, 4, 2, 3, 2, 32, 32, 0, 1024)
+    assert _lib.lib.kvq_decode_status(ctypes.byref(bad), ctypes.c_void_p(0x1000), None) == kvq.KVQ_ERR_INVALID_ARG

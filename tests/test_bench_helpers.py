@@ -44,32 +44,37 @@ def _sources_hash(root, files):
 
 
 def test_traffic_counters_are_used_only_while_their_sources_match():
-    # every committed counter names its kernel sources and their hash; a record is used only while
-    # the hash matches (else roofline.traffic is null), and it scales by the units processed
+    # every committed counter names its workload, kernel sources and their hash; a record is used only
+    # while the hash matches (else the traffic is null), and it scales by the units processed (or, for a
+    # capture at a reduced length, by the (token, KV head) pairs)
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     entries = json.load(open(os.path.join(root, "profiles", "decode_traffic_counters.txt")))
     assert {"decode", "prefill"} <= {e.get("kind", "decode") for e in entries.values()}
-    w = inputs.WORKLOADS["llama2_7b_mha"]
-    algorithmic = {"decode": bench.decode_bytes(w, w.seq_lens()), "prefill": bench.prefill_bytes(w, w.seq_lens())}
     for e in entries.values():
         kind = e.get("kind", "decode")
+        w = inputs.WORKLOADS[e["workload"]]
         got = bench.measured_traffic(w, e["layout"], kind)
         if _sources_hash(root, e["kernel_sources"]) != e["sources_sha256"]:
             assert got is None  # the kernel changed since the capture
             continue
-        units = w.batch * w.num_kv_heads
-        assert got == round((e["dram_read_bytes"] + e["dram_write_bytes"]) * units / e["capture_units"])
-        # the captured DRAM bytes stay within a few percent of the algorithmic bytes
-        assert 0.95 < got / algorithmic[kind] < 1.06
+        if "capture_tokens" in e:
+            scale = float(np.sum(w.seq_lens())) * w.num_kv_heads / e["capture_tokens"]
+        else:
+            scale = w.batch * w.num_kv_heads / e["capture_units"]
+        assert got == round((e["dram_read_bytes"] + e["dram_write_bytes"]) * scale)
+        # the captured DRAM bytes stay within a few percent of the algorithmic bytes of the workload
+        lens = w.seq_lens()
+        algorithmic = bench.decode_bytes(w, lens + w.appends) if kind == "decode" else bench.prefill_bytes(w, lens)
+        assert 0.95 < got / algorithmic < 1.06, (e["workload"], kind, got / algorithmic)
 
 
 def test_traffic_lookup_is_none_for_other_layouts_and_kernels():
     w = inputs.WORKLOADS["llama2_7b_mha"]
     assert bench.measured_traffic(w, 2, "decode") is None
-    assert bench.measured_traffic(inputs.WORKLOADS["llama3_8b_gqa"], 1, "decode") is None
+    assert bench.measured_traffic(inputs.WORKLOADS["tiny"], 1, "decode") is None
     # the records were taken with the sink and RoPE off: other options get no traffic figure
     assert bench.measured_traffic(w, 1, "decode", sink=1) is None
-    assert bench.measured_traffic(w, 1, "prefill", sink=1) is None
+    assert bench.measured_traffic(inputs.WORKLOADS["llama3_8b_gqa"], 1, "prefill", sink=1) is None
     assert bench.measured_traffic(w, 2, "decode", rope=10000.0) is None
 
 

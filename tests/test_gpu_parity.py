@@ -232,3 +232,24 @@ def test_signed_zero_groups_bit_exact(oracle_mod, layout, G):
         kz = gv["k_zero"][0, :, : (T - w.residual) // G]
         assert np.all(kz[:, :, 48:56] == 0x8000) and np.all(kz[:, :, 56:64] == 0x0000)
     H.check_attention(run.out.cpu().numpy(), ref, f"signed zeros G={G}")
+
+
+@pytest.mark.parametrize("layout", LAYOUTS, ids=["tile_v1", "rows_v2"])
+def test_decode_status_is_ok_after_a_decode_that_finishes(layout):
+    """kvq_decode_status reads the per-(sequence, query head) records the split combine writes at the
+    end of the workspace: all clear after a decode whose kernels never gave up a wait (including a
+    sequence of length 0)."""
+    import bit_kv_cache_prefill_b200 as kvq
+
+    name, w, lens = SMALL[2]
+    w = _lens_workload(w, lens)
+    lens = np.array(lens, np.int64)
+    k, v = _inputs_for(w, lens)
+    cfg = H.gpu_config(w, layout)
+    cache = kvq.Cache(cfg)
+    kvq.kvq_quantize_prefill(cfg, cache, k.cuda(), v.cuda(), lens)
+    ws = torch.full((kvq.kvq_decode_workspace_bytes(cfg),), 0xFF, dtype=torch.uint8, device="cuda")  # stale bits
+    out = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float16, device="cuda")
+    kvq.kvq_decode_attention(cfg, cache, inputs.query(w).cuda(), out, 1 / math.sqrt(128), ws)
+    assert kvq.kvq_decode_status(cfg, ws) == kvq.KVQ_OK
+    assert torch.isfinite(out.float()).all()

@@ -22,20 +22,32 @@ import _harness as H
 pytestmark = pytest.mark.gpu
 
 
-def _prepared(w: inputs.Workload):
+def _prepared(w: inputs.Workload, layout: int = 1, sink: int = 0, rope: float = 0.0):
     k, v, lens = inputs.full_kv(w)
-    cfg = H.gpu_config(w)
+    cfg = H.gpu_config(w, layout=layout, sink=sink, rope=rope)
     cache = kvq.Cache(cfg)
     kvq.kvq_quantize_prefill(cfg, cache, k.cuda(), v.cuda(), lens)
     return cfg, cache
 
 
-def test_noalloc_decode_matches_workspace_decode_on_two_calls():
-    w1 = inputs.Workload("na1", 4, 16, 4, 2, 2, 32, 64, 0, 3000, seed=41, ragged_min=700)
-    w2 = inputs.Workload("na2", 2, 8, 8, 4, 2, 64, 32, 1, 5000, seed=42)
+# (workload, layout, sink, rope_theta): tile v1 (mma.sync decode); rows v2 (tcgen05 decode, its own
+# split length); rows v2 with pre-RoPE keys (the RoPE angle tables share the scratch, behind the
+# split partials)
+CASES = {
+    "tile_v1": [(inputs.Workload("na1", 4, 16, 4, 2, 2, 32, 64, 0, 3000, seed=41, ragged_min=700), 1, 0, 0.0),
+                (inputs.Workload("na2", 2, 8, 8, 4, 2, 64, 32, 1, 5000, seed=42), 1, 0, 0.0)],
+    "rows_v2": [(inputs.Workload("na3", 3, 8, 2, 2, 2, 32, 32, 0, 2500, seed=43), 2, 1, 0.0),
+                (inputs.Workload("na4", 2, 4, 4, 2, 2, 128, 128, 0, 4000, seed=44), 2, 0, 0.0)],
+    "rope": [(inputs.Workload("na5", 2, 8, 2, 2, 2, 64, 64, 0, 3000, seed=45), 2, 1, 10000.0),
+             (inputs.Workload("na6", 3, 4, 4, 2, 2, 32, 32, 0, 2000, seed=46, ragged_min=500), 2, 0, 500000.0)],
+}
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_noalloc_decode_matches_workspace_decode_on_two_calls(case):
     runs = []
-    for w in (w1, w2):
-        cfg, cache = _prepared(w)
+    for w, layout, sink, rope in CASES[case]:
+        cfg, cache = _prepared(w, layout, sink, rope)
         q = inputs.query(w).cuda()
         ws = torch.empty(kvq.kvq_decode_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
         ref = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float16, device="cuda")
