@@ -144,10 +144,45 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
   const int jv = c0 / G;      // their value group
   int kp_group = -1;          // first key group staged in wkp
 
+  // Codes of step i (this lane's key row and its channels' value words), loaded one step ahead so that
+  // the global loads of the next step overlap this step's arithmetic.
+  constexpr int NWV = kRStep / (2 * VP);  // value words per step per channel
+  uint32_t kw_next[KW], vw_next[4][NWV];
+  auto load_codes = [&](int ii) {
+    const int tn = start + (sb + ii) * kRStep;
+    const int tl = tn + lane;
+    const uint4* src = reinterpret_cast<const uint4*>(a.k_codes + (unit * a.capacity + (tl < qend ? tl : 0)) * KW);
+#pragma unroll
+    for (int v = 0; v < KW / 4; ++v) {
+      const uint4 x = src[v];
+      kw_next[4 * v] = x.x;
+      kw_next[4 * v + 1] = x.y;
+      kw_next[4 * v + 2] = x.z;
+      kw_next[4 * v + 3] = x.w;
+    }
+    const int64_t blk = tn / 128;
+    const int wv0 = ((tn & 127) >> 1) / VP;  // first value word of the step
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t* row = a.v_codes + (unit * a.capacity + blk * 128 + c0 + e) * VW + wv0;
+#pragma unroll
+      for (int k = 0; k < NWV; ++k) vw_next[e][k] = row[k];
+    }
+  };
+  if (nst > 0) load_codes(0);
+
   for (int i = 0; i < nst; ++i) {
     const int t0 = start + (sb + i) * kRStep;
     const int t = t0 + lane;
     const bool valid = t < qend && !(a.sink && t == 0);
+    uint32_t kw[KW], vw[4][NWV];
+#pragma unroll
+    for (int k = 0; k < KW; ++k) kw[k] = kw_next[k];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+      for (int k = 0; k < NWV; ++k) vw[e][k] = vw_next[e][k];
+    if (i + 1 < nst) load_codes(i + 1);
     // key scale / zero of the step's groups: wkp[g][half][p] = (s, z) of channels 2p, 2p + 1
     // (half 0) or 64 + 2p, 65 + 2p (half 1), fp16 scales pre-multiplied by 2^(24 - (bit & 7)) of
     // their code position (code_pair reads a code at bit & 7) so that the subnormal code times the
@@ -205,16 +240,6 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
 #pragma unroll
     for (int h = 0; h < GQ; ++h) s[h] = 0.f;
     {
-      uint32_t kw[KW];
-      const uint4* src = reinterpret_cast<const uint4*>(a.k_codes + (unit * a.capacity + (valid ? t : 0)) * KW);
-#pragma unroll
-      for (int v = 0; v < KW / 4; ++v) {
-        const uint4 x = src[v];
-        kw[4 * v] = x.x;
-        kw[4 * v + 1] = x.y;
-        kw[4 * v + 2] = x.z;
-        kw[4 * v + 3] = x.w;
-      }
       const int gl = G >= kRStep ? 0 : lane / G;  // this token's group among the staged ones
       const float4* oj = soff + lane * kOffStride;
 #pragma unroll
@@ -264,16 +289,6 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
 
     // -- PV: lane = channels c0 .. c0 + 3; token pairs of the channel rows of this 128-token block
     {
-      const int64_t blk = t0 / 128;
-      const int wv0 = ((t0 & 127) >> 1) / VP;  // first value word of the step
-      constexpr int NWV = kRStep / (2 * VP);   // value words per step per channel
-      uint32_t vw[4][NWV];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t* row = a.v_codes + (unit * a.capacity + blk * 128 + c0 + e) * VW + wv0;
-#pragma unroll
-        for (int k = 0; k < NWV; ++k) vw[e][k] = row[k];
-      }
 #pragma unroll
       for (int jp = 0; jp < kRStep / 2; ++jp) {  // token pair (2 jp, 2 jp + 1) of the step
         const int k = jp / VP, slot = jp % VP;
@@ -462,19 +477,46 @@ cudaError_t launch_decode_rope(const DecodeArgs& a, cudaStream_t stream) {
   return a.value_bits == 2 ? rope_g<4, 2>(a, stream) : rope_g<4, 4>(a, stream);
 }
 
-int decode_rope_ctas_per_sm() {
+namespace {
+// CTAs per SM of the instance a launch uses (its registers and shared memory depend on the
+// template arguments, GQ above all).
+template <int KB, int VB, int G, int GQ>
+int rope_occupancy() {
   static DeviceMemo occ;
   return occ.get([] {
-    using SM = RopeSmem<4>;
-    if (cudaFuncSetAttribute(decode_rope_kernel<2, 2, 32, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) !=
+    using SM = RopeSmem<GQ>;
+    if (cudaFuncSetAttribute(decode_rope_kernel<KB, VB, G, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) !=
         cudaSuccess)
       return 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rope_kernel<2, 2, 32, 4>, kRW * 32, SM::kBytes) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rope_kernel<KB, VB, G, GQ>, kRW * 32, SM::kBytes) !=
         cudaSuccess)
       return 1;
     return n > 0 ? n : 1;
   });
+}
+template <int KB, int VB, int G>
+int rope_occ_gq(int gqa) {
+  switch (gqa) {
+    case 1: return rope_occupancy<KB, VB, G, 1>();
+    case 2: return rope_occupancy<KB, VB, G, 2>();
+    default: return rope_occupancy<KB, VB, G, 4>();
+  }
+}
+template <int KB, int VB>
+int rope_occ_g(int G, int gqa) {
+  switch (G) {
+    case 16: return rope_occ_gq<KB, VB, 16>(gqa);
+    case 32: return rope_occ_gq<KB, VB, 32>(gqa);
+    case 64: return rope_occ_gq<KB, VB, 64>(gqa);
+    default: return rope_occ_gq<KB, VB, 128>(gqa);
+  }
+}
+}  // namespace
+
+int decode_rope_ctas_per_sm(int key_bits, int value_bits, int G, int gqa) {
+  if (key_bits == 2) return value_bits == 2 ? rope_occ_g<2, 2>(G, gqa) : rope_occ_g<2, 4>(G, gqa);
+  return value_bits == 2 ? rope_occ_g<4, 2>(G, gqa) : rope_occ_g<4, 4>(G, gqa);
 }
 
 }  // namespace kvq

@@ -94,7 +94,7 @@ cudaError_t launch_append(const QuantizeArgs& a, const int64_t* old_lens, const 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);     // split + combine, either layout
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // rows-v2 split kernel only
 cudaError_t launch_decode_rope(const DecodeArgs& a, cudaStream_t stream);  // pre-RoPE keys: tables + split kernel
-int decode_rope_ctas_per_sm();
+int decode_rope_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);  // pre-RoPE kernel
 int64_t rope_table_floats(int64_t capacity);  // floats of the two RoPE tables in the workspace
 int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa, int outliers);  // tile-v1 kernel
 int decode_tc_ctas_per_sm(int G, int gqa);                              // rows-v2 kernel (1 or 2)
