@@ -338,7 +338,7 @@ def workload_config(w: inputs.Workload, args) -> dict:
             "group_size": w.group_size, "residual": w.residual, "hadamard": w.hadamard,
             "ragged": bool(w.ragged_min), "parallelism": f"replicas{args.gpus}", "layout": args.layout,
             "sink": args.sink, "rope_theta": args.rope, "outliers": args.outliers,
-            "page_tokens": getattr(args, "page_tokens", 0), "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
+            "page_tokens": getattr(args, "page_tokens", 0), "cuda_cores": getattr(args, "cuda_cores", 0), "l2": f"inputs larger than L2 ({step_bytes / 2**20:.0f} MiB read per decode > 126 MiB)"}
 
 
 def run_reference(args, w):
@@ -398,6 +398,9 @@ def main():
     ap.add_argument("--page-tokens", type=int, default=0,
                     help="> 0: paged storage with pages of this many tokens (a multiple of 128; needs --layout 1); "
                          "each unit's pages are consecutive pool pages")
+    ap.add_argument("--cuda-cores", type=int, default=0, choices=[0, 1],
+                    help="1: decode with the CUDA-core control kernel instead of the tensor-core one (needs --layout 2, "
+                         "no RoPE, no Hadamard rotation); for measuring the tensor-core gain")
     ap.add_argument("--outliers", type=int, default=0, choices=[0, 1],
                     help="1: keep each quantized token's largest key / value entry in fp16 (needs --layout 1)")
     args = ap.parse_args()
@@ -413,6 +416,10 @@ def main():
 
     import bit_kv_cache_prefill_b200 as kvq
 
+    if args.cuda_cores:
+        if args.layout != 2 or args.rope > 0 or w0.hadamard:
+            raise SystemExit("--cuda-cores 1 needs --layout 2, no RoPE and a workload without the Hadamard rotation")
+        os.environ["KVQ_DECODE_CUDA_CORES"] = "1"  # read by the library at each decode call
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -598,6 +605,7 @@ def main():
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": measured_traffic(w0, args.layout, "decode", args.sink, args.rope, args.outliers, args.page_tokens), "peak_kind": peak_kind,
                      "kernel": ("decode_rope_kernel" if args.rope > 0 else
+                                "decode_rope_kernel without rotations (CUDA-core control)" if args.cuda_cores else
                                 "decode_split_kernel" if args.layout == 1 else "decode_tc_kernel")
                      + " + decode_combine_kernel (one kvq_decode_attention call)"},
         "prefill": {"gbs": round(pre_bytes / (statistics.mean(pre_ms) * 1e-3) / 1e9, 1),

@@ -352,8 +352,10 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
     return n;
   });
   if (sms <= 0) return KVQ_ERR_CUDA;
-  const int occ = cfg->rope_theta > 0.f ? kvq::decode_rope_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size,
-                                                                       cfg->num_q_heads / cfg->num_kv_heads)
+  const int gqa = cfg->num_q_heads / cfg->num_kv_heads;
+  const int occ = cfg->rope_theta > 0.f ? kvq::decode_rope_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size, gqa)
+                  : kvq::cuda_core_control_requested(cfg->layout, cfg->rope_theta, cfg->hadamard)
+                      ? kvq::decode_cuda_cores_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size, gqa)
                   : cfg->layout == KVQ_LAYOUT_ROWS_V2
                       ? kvq::decode_tc_ctas_per_sm(cfg->group_size, cfg->num_q_heads / cfg->num_kv_heads)
                       : kvq::decode_ctas_per_sm(cfg->key_bits, cfg->value_bits, cfg->group_size,

@@ -40,6 +40,8 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <cstdlib>
+
 #include "kvq_common.cuh"
 #include "kvq_decode_common.cuh"
 #include "kvq_internal.h"
@@ -873,10 +875,18 @@ int occupancy_vpt(int G, int gqa, int outliers) {
 
 }  // namespace
 
+bool cuda_core_control_requested(int layout, float rope_theta, int hadamard) {
+  if (layout != KVQ_LAYOUT_ROWS_V2 || rope_theta > 0.f || hadamard) return false;
+  const char* v = std::getenv("KVQ_DECODE_CUDA_CORES");
+  return v != nullptr && v[0] == '1';
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e;
   if (a.rope_theta > 0.f)
     e = launch_decode_rope(a, stream);
+  else if (cuda_core_control_requested(a.layout, a.rope_theta, a.hadamard))
+    e = launch_decode_cuda_cores(a, stream);
   else if (a.layout == KVQ_LAYOUT_ROWS_V2)
     e = launch_decode_tc(a, stream);
   else if (a.key_bits == 2)

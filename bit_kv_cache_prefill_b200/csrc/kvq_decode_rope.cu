@@ -82,7 +82,10 @@ __device__ __forceinline__ float2 code_pair(uint32_t word, int slot) {  // slot:
   return sub2f((o >= 8 ? word >> 8 : word) & (m | (m << 16)));
 }
 
-template <int KB, int VB, int G, int GQ>
+// ROT = false: the same kernel with every rotation left out (keys used as cached, no angle tables): a
+// CUDA-core decode of the rows-v2 cache, kept as the control against which the tensor-core kernels'
+// gain is measured (selected with KVQ_DECODE_CUDA_CORES=1, see launch_decode_cuda_cores).
+template <int KB, int VB, int G, int GQ, bool ROT = true>
 __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs a, const float2* __restrict__ rbase,
                                                                const float2* __restrict__ roff) {
   using SM = RopeSmem<GQ>;
@@ -119,10 +122,12 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
     const int h = idx >> 7, c = idx & 127;
     sq[idx] = h < gq ? h2f(a.q[(b * a.num_q_heads + static_cast<int64_t>(kvh) * gq + h) * kHeadDim + c]) * a.qscale : 0.f;
   }
-  for (int idx = threadIdx.x; idx < kRStep * 32; idx += kRW * 32) {
-    const int j = idx >> 5, p = idx & 31;
-    const float2 c0 = roff[j * 64 + 2 * p], c1 = roff[j * 64 + 2 * p + 1];
-    soff[j * kOffStride + p] = make_float4(c0.x, c0.y, c1.x, c1.y);
+  if constexpr (ROT) {
+    for (int idx = threadIdx.x; idx < kRStep * 32; idx += kRW * 32) {
+      const int j = idx >> 5, p = idx & 31;
+      const float2 c0 = roff[j * 64 + 2 * p], c1 = roff[j * 64 + 2 * p + 1];
+      soff[j * kOffStride + p] = make_float4(c0.x, c0.y, c1.x, c1.y);
+    }
   }
   __syncthreads();
 
@@ -221,7 +226,13 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       wvz[jj * VPT + g] = ok ? h2f(a.v_zero[pidx]) : 0.f;
     }
     // the query turned back to the step start: R_-t0 q, pair (i, i + 64) by -t0 w_i
-    {
+    if constexpr (!ROT) {
+#pragma unroll
+      for (int h = 0; h < GQ; ++h) {
+        const float* qh = sq + h * kHeadDim;
+        wq[h * 32 + lane] = make_float4(qh[2 * lane], qh[2 * lane + 1], qh[64 + 2 * lane], qh[65 + 2 * lane]);
+      }
+    } else {
       const float2* bt = rbase + static_cast<int64_t>(t0 / kRStep) * 64;
       const float2 cs0 = bt[2 * lane], cs1 = bt[2 * lane + 1];  // pairs 2 lane, 2 lane + 1
 #pragma unroll
@@ -252,10 +263,15 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
         const float x0 = fmaf(lo.x, kl.x, kl.y), x1 = fmaf(lo.y, kl.z, kl.w);
         const float y0 = fmaf(hi.x, kh.x, kh.y), y1 = fmaf(hi.y, kh.z, kh.w);
         // R_j on pairs (c, c + 64) and (c + 1, c + 65)
-        const float4 csn = oj[p];
-        const float cs0 = csn.x, sn0 = csn.y, cs1 = csn.z, sn1 = csn.w;
-        const float r0 = fmaf(x0, cs0, -y0 * sn0), u0 = fmaf(x0, sn0, y0 * cs0);
-        const float r1 = fmaf(x1, cs1, -y1 * sn1), u1 = fmaf(x1, sn1, y1 * cs1);
+        float r0 = x0, u0 = y0, r1 = x1, u1 = y1;
+        if constexpr (ROT) {
+          const float4 csn = oj[p];
+          const float cs0 = csn.x, sn0 = csn.y, cs1 = csn.z, sn1 = csn.w;
+          r0 = fmaf(x0, cs0, -y0 * sn0);
+          u0 = fmaf(x0, sn0, y0 * cs0);
+          r1 = fmaf(x1, cs1, -y1 * sn1);
+          u1 = fmaf(x1, sn1, y1 * cs1);
+        }
 #pragma unroll
         for (int h = 0; h < GQ; ++h) {
           const float4 qv = wq[h * 32 + p];
@@ -351,9 +367,10 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       const uint16_t* vr = vres + static_cast<int64_t>(slot) * kHeadDim;
       const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(kr + 2 * lane));
       const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(kr + 64 + 2 * lane));
+      float r[4] = {lo.x, lo.y, hi.x, hi.y};
+      if constexpr (ROT) {
       const float2* bt = rbase + static_cast<int64_t>(pos / kRStep) * 64;
       const int j = pos % kRStep;
-      float r[4];
       const float4 oj = soff[j * kOffStride + lane];  // in-step (cos, sin) of pairs 2 lane, 2 lane + 1
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -365,6 +382,7 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
         const float x = e ? lo.y : lo.x, y = e ? hi.y : hi.x;
         r[e] = fmaf(x, cs, -y * sn);      // channel i
         r[2 + e] = fmaf(x, sn, y * cs);   // channel i + 64
+      }
       }
       const float2 v_lo = __half22float2(*reinterpret_cast<const __half2*>(vr + 2 * lane));
       const float2 v_hi = __half22float2(*reinterpret_cast<const __half2*>(vr + 64 + 2 * lane));
@@ -425,38 +443,38 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
   }
 }
 
-template <int KB, int VB, int G, int GQ>
+template <int KB, int VB, int G, int GQ, bool ROT>
 cudaError_t launch_rope_kernel(const DecodeArgs& a, cudaStream_t stream) {
   using SM = RopeSmem<GQ>;
   static DeviceMemo attr;
   const int ok = attr.get([] {
-    return cudaFuncSetAttribute(decode_rope_kernel<KB, VB, G, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(decode_rope_kernel<KB, VB, G, GQ, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 SM::kBytes) == cudaSuccess ? 1 : -1;
   });
   if (ok < 0) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.num_kv_heads));
-  decode_rope_kernel<KB, VB, G, GQ><<<grid, kRW * 32, SM::kBytes, stream>>>(a, a.rope_base, a.rope_off);
+  decode_rope_kernel<KB, VB, G, GQ, ROT><<<grid, kRW * 32, SM::kBytes, stream>>>(a, a.rope_base, a.rope_off);
   return cudaGetLastError();
 }
 
-template <int KB, int VB, int G>
+template <int KB, int VB, int G, bool ROT>
 cudaError_t rope_gq(const DecodeArgs& a, cudaStream_t stream) {
   switch (a.gqa) {
-    case 1: return launch_rope_kernel<KB, VB, G, 1>(a, stream);
-    case 2: return launch_rope_kernel<KB, VB, G, 2>(a, stream);
+    case 1: return launch_rope_kernel<KB, VB, G, 1, ROT>(a, stream);
+    case 2: return launch_rope_kernel<KB, VB, G, 2, ROT>(a, stream);
     case 3:
-    case 4: return launch_rope_kernel<KB, VB, G, 4>(a, stream);
+    case 4: return launch_rope_kernel<KB, VB, G, 4, ROT>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
 
-template <int KB, int VB>
+template <int KB, int VB, bool ROT>
 cudaError_t rope_g(const DecodeArgs& a, cudaStream_t stream) {
   switch (a.G) {
-    case 16: return rope_gq<KB, VB, 16>(a, stream);
-    case 32: return rope_gq<KB, VB, 32>(a, stream);
-    case 64: return rope_gq<KB, VB, 64>(a, stream);
-    case 128: return rope_gq<KB, VB, 128>(a, stream);
+    case 16: return rope_gq<KB, VB, 16, ROT>(a, stream);
+    case 32: return rope_gq<KB, VB, 32, ROT>(a, stream);
+    case 64: return rope_gq<KB, VB, 64, ROT>(a, stream);
+    case 128: return rope_gq<KB, VB, 128, ROT>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -473,50 +491,62 @@ cudaError_t launch_decode_rope(const DecodeArgs& a, cudaStream_t stream) {
   rope_table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(a.rope_base, a.rope_off, nbase, a.rope_theta);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (a.key_bits == 2) return a.value_bits == 2 ? rope_g<2, 2>(a, stream) : rope_g<2, 4>(a, stream);
-  return a.value_bits == 2 ? rope_g<4, 2>(a, stream) : rope_g<4, 4>(a, stream);
+  if (a.key_bits == 2) return a.value_bits == 2 ? rope_g<2, 2, true>(a, stream) : rope_g<2, 4, true>(a, stream);
+  return a.value_bits == 2 ? rope_g<4, 2, true>(a, stream) : rope_g<4, 4, true>(a, stream);
+}
+
+cudaError_t launch_decode_cuda_cores(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.key_bits == 2) return a.value_bits == 2 ? rope_g<2, 2, false>(a, stream) : rope_g<2, 4, false>(a, stream);
+  return a.value_bits == 2 ? rope_g<4, 2, false>(a, stream) : rope_g<4, 4, false>(a, stream);
 }
 
 namespace {
 // CTAs per SM of the instance a launch uses (its registers and shared memory depend on the
 // template arguments, GQ above all).
-template <int KB, int VB, int G, int GQ>
+template <int KB, int VB, int G, int GQ, bool ROT>
 int rope_occupancy() {
   static DeviceMemo occ;
   return occ.get([] {
     using SM = RopeSmem<GQ>;
-    if (cudaFuncSetAttribute(decode_rope_kernel<KB, VB, G, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(decode_rope_kernel<KB, VB, G, GQ, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SM::kBytes) != cudaSuccess)
       return 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rope_kernel<KB, VB, G, GQ>, kRW * 32, SM::kBytes) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rope_kernel<KB, VB, G, GQ, ROT>, kRW * 32, SM::kBytes) !=
         cudaSuccess)
       return 1;
     return n > 0 ? n : 1;
   });
 }
-template <int KB, int VB, int G>
+template <int KB, int VB, int G, bool ROT>
 int rope_occ_gq(int gqa) {
   switch (gqa) {
-    case 1: return rope_occupancy<KB, VB, G, 1>();
-    case 2: return rope_occupancy<KB, VB, G, 2>();
-    default: return rope_occupancy<KB, VB, G, 4>();
+    case 1: return rope_occupancy<KB, VB, G, 1, ROT>();
+    case 2: return rope_occupancy<KB, VB, G, 2, ROT>();
+    default: return rope_occupancy<KB, VB, G, 4, ROT>();
   }
 }
-template <int KB, int VB>
+template <int KB, int VB, bool ROT>
 int rope_occ_g(int G, int gqa) {
   switch (G) {
-    case 16: return rope_occ_gq<KB, VB, 16>(gqa);
-    case 32: return rope_occ_gq<KB, VB, 32>(gqa);
-    case 64: return rope_occ_gq<KB, VB, 64>(gqa);
-    default: return rope_occ_gq<KB, VB, 128>(gqa);
+    case 16: return rope_occ_gq<KB, VB, 16, ROT>(gqa);
+    case 32: return rope_occ_gq<KB, VB, 32, ROT>(gqa);
+    case 64: return rope_occ_gq<KB, VB, 64, ROT>(gqa);
+    default: return rope_occ_gq<KB, VB, 128, ROT>(gqa);
   }
+}
+template <bool ROT>
+int rope_occ(int key_bits, int value_bits, int G, int gqa) {
+  if (key_bits == 2) return value_bits == 2 ? rope_occ_g<2, 2, ROT>(G, gqa) : rope_occ_g<2, 4, ROT>(G, gqa);
+  return value_bits == 2 ? rope_occ_g<4, 2, ROT>(G, gqa) : rope_occ_g<4, 4, ROT>(G, gqa);
 }
 }  // namespace
 
 int decode_rope_ctas_per_sm(int key_bits, int value_bits, int G, int gqa) {
-  if (key_bits == 2) return value_bits == 2 ? rope_occ_g<2, 2>(G, gqa) : rope_occ_g<2, 4>(G, gqa);
-  return value_bits == 2 ? rope_occ_g<4, 2>(G, gqa) : rope_occ_g<4, 4>(G, gqa);
+  return rope_occ<true>(key_bits, value_bits, G, gqa);
+}
+int decode_cuda_cores_ctas_per_sm(int key_bits, int value_bits, int G, int gqa) {
+  return rope_occ<false>(key_bits, value_bits, G, gqa);
 }
 
 }  // namespace kvq

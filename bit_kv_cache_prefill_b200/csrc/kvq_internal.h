@@ -95,6 +95,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);     // spli
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // rows-v2 split kernel only
 cudaError_t launch_decode_rope(const DecodeArgs& a, cudaStream_t stream);  // pre-RoPE keys: tables + split kernel
 int decode_rope_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);  // pre-RoPE kernel
+// The CUDA-core control: the pre-RoPE kernel without its rotations, on a rows-v2 cache without
+// rotations (rope_theta = 0, hadamard = 0), for measuring the tensor-core kernels' gain. It runs in
+// place of the tcgen05 kernel when the environment sets KVQ_DECODE_CUDA_CORES=1.
+cudaError_t launch_decode_cuda_cores(const DecodeArgs& a, cudaStream_t stream);
+int decode_cuda_cores_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);
+bool cuda_core_control_requested(int layout, float rope_theta, int hadamard);
 int64_t rope_table_floats(int64_t capacity);  // floats of the two RoPE tables in the workspace
 int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa, int outliers);  // tile-v1 kernel
 int decode_tc_ctas_per_sm(int G, int gqa);                              // rows-v2 kernel (1 or 2)

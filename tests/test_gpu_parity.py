@@ -253,3 +253,18 @@ def test_decode_status_is_ok_after_a_decode_that_finishes(layout):
     kvq.kvq_decode_attention(cfg, cache, inputs.query(w).cuda(), out, 1 / math.sqrt(128), ws)
     assert kvq.kvq_decode_status(cfg, ws) == kvq.KVQ_OK
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("sink", [0, 1], ids=["nosink", "sink"])
+@pytest.mark.parametrize("name,w,lens", [c for c in SMALL if not c[1].hadamard][:6], ids=lambda x: x if isinstance(x, str) else "")
+def test_cuda_core_control_matches_the_oracle(oracle_mod, monkeypatch, name, w, lens, sink):
+    """KVQ_DECODE_CUDA_CORES=1 runs the CUDA-core control decode (the pre-RoPE kernel without its
+    rotations) on a rows-v2 cache in place of the tcgen05 kernel: same outputs within tolerance."""
+    monkeypatch.setenv("KVQ_DECODE_CUDA_CORES", "1")
+    w = _lens_workload(w, lens).scaled(appends=3)
+    lens = np.array(lens, np.int64)
+    k, v = _inputs_for(w, lens)
+    q = inputs.query(w)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, appends=3, layout=2, sink=sink)
+    _, ref = H.oracle_full(oracle_mod, w, k, v, lens, q, appends=3, layout=2, sink=sink)
+    H.check_attention(run.out.cpu().numpy(), ref, f"CUDA-core control {name}")
