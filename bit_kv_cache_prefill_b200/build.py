@@ -39,14 +39,26 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    """Compile every source to an object in parallel (one nvcc per file), then link libkvq.so."""
     if not (force or ptxas_verbose or _stale()):
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp]
+    import concurrent.futures
+    import tempfile
+
+    common = [_nvcc(), *[f for f in NVCC_FLAGS if f != "-shared"], "-I", INCLUDE, "-I", CSRC]
     if ptxas_verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES]
-    subprocess.check_call(cmd)
+        common += ["-Xptxas", "-v"]
+    with tempfile.TemporaryDirectory(prefix="kvq_build_") as objdir:
+        objs = [os.path.join(objdir, os.path.splitext(s)[0] + ".o") for s in SOURCES]
+
+        def compile_one(i: int) -> None:
+            subprocess.check_call([*common, "-c", os.path.join(CSRC, SOURCES[i]), "-o", objs[i]])
+
+        workers = max(1, min(len(SOURCES), os.cpu_count() or 1))
+        with concurrent.futures.ThreadPoolExecutor(workers) as pool:
+            list(pool.map(compile_one, range(len(SOURCES))))  # re-raises the first failure
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs])
     os.replace(tmp, LIB)
     return LIB
 

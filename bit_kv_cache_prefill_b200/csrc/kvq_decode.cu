@@ -98,20 +98,26 @@ struct Stage {
   static constexpr int kBytes = oVO + kKO;
   static constexpr int kKP = 512 * KGB;  // key scale[128] + zero[128] per group of the block
   static constexpr int kBlockSteps = (128 / VPT) * KGB / (16 * TS);
-  static constexpr int kKPSlots = kBlockSteps >= 2 ? 2 : 4;
+  // one-step blocks: with two stages the next block's parameters land while the current one is read
+  // (two slots); with three, two later blocks may be in flight (four slots, a power of two)
+  static constexpr int kKPSlots = kBlockSteps >= 2 ? 2 : (kStages == 2 ? 2 : 4);
   static constexpr int kWarpBytes = kStages * kBytes + kKPSlots * kKP;
 };
 
-// Shared memory: q~ [4][128] f32 (base-2 logit units), q^ = q~ * 2^-e [4][128] f32, exponents [4]
-// i32 (16 B), then the per-warp rings. After the main loops the ring area holds the warp partials
-// [W][4][130] f32 and the zero-point sums [W][4][8] f32.
-constexpr int kSmemQ = 2 * 4 * 128 * 4;
-constexpr int kSmemE = 16;
-constexpr int kSmemFixed = kSmemQ + kSmemE;
+// Shared memory: q~ [GQ][128] f32 (base-2 logit units), q^ = q~ * 2^-e [GQ][128] f32, then the
+// per-warp rings (GQ: the query heads per KV head the instance serves, 1, 2 or 4). The per-head
+// exponents [4] i32 sit at the start of the ring area until every warp has read them (a CTA barrier
+// separates that from the first copy into the rings). After the main loops the ring area holds the
+// warp partials [W][4][130] f32 and the zero-point sums [W][4][8] f32.
+template <int GQ>
+constexpr int smem_q() { return 2 * GQ * 128 * 4; }
+template <int GQ>
+constexpr int smem_fixed() { return smem_q<GQ>(); }
 constexpr int kCm = 132;   // shared-memory partial stride (floats): m, l, 2 pad, o[128] 16-byte aligned
 constexpr int kCmO = 4;    // offset of o[] within a shared-memory partial
 constexpr int kSmemEpilogue = kDecodeWarps * 4 * kCm * 4 + kDecodeWarps * 4 * 8 * 4;
-static_assert(kSmemFixed % 16 == 0, "stage ring must start 16-byte aligned");
+static_assert(smem_fixed<1>() % 16 == 0 && smem_fixed<2>() % 16 == 0 && smem_fixed<4>() % 16 == 0,
+              "stage ring must start 16-byte aligned");
 
 template <int KB, int VB, int VPT, int GQ, bool OUT>
 struct Shape {
@@ -125,18 +131,19 @@ struct Shape {
   using S = Stage<KB, VB, VPT, KGB, TS, OUT>;
 };
 
-// With OUT, the per-warp outlier corrections of the value sum [W][4][128] f32 follow the ring /
+// With OUT, the per-warp outlier corrections of the value sum [W][GQ][128] f32 follow the ring /
 // epilogue area (they live through both).
-constexpr int kSmemCorr = kDecodeWarps * 4 * 128 * 4;
+template <int GQ>
+constexpr int smem_corr() { return kDecodeWarps * GQ * 128 * 4; }
 template <int KB, int VB, int VPT, int GQ, bool OUT>
 constexpr int decode_corr_offset() {
   using S = typename Shape<KB, VB, VPT, GQ, OUT>::S;
   constexpr int ring = kDecodeWarps * S::kWarpBytes;
-  return kSmemFixed + (ring > kSmemEpilogue ? ring : kSmemEpilogue);
+  return smem_fixed<GQ>() + (ring > kSmemEpilogue ? ring : kSmemEpilogue);
 }
 template <int KB, int VB, int VPT, int GQ, bool OUT>
 constexpr int decode_smem_bytes() {
-  return decode_corr_offset<KB, VB, VPT, GQ, OUT>() + (OUT ? kSmemCorr : 0);
+  return decode_corr_offset<KB, VB, VPT, GQ, OUT>() + (OUT ? smem_corr<GQ>() : 0);
 }
 
 // cp.async of 16 bytes that writes zeros (and reads nothing) when `valid` is false.
@@ -202,8 +209,8 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   constexpr int kStepTokens = 16 * TS;
   extern __shared__ __align__(16) uint8_t smem[];
   float* sq = reinterpret_cast<float*>(smem);
-  int* se = reinterpret_cast<int*>(smem + kSmemQ);
-  uint8_t* rings = smem + kSmemFixed;
+  uint8_t* rings = smem + smem_fixed<GQ>();
+  int* se = reinterpret_cast<int*>(rings);  // until the barrier after the exponents are read
   float* cm = reinterpret_cast<float*>(rings);        // epilogue: [W][4][kCm] (m, l, -, -, o[128])
   float* zb = cm + kDecodeWarps * 4 * kCm;            // epilogue: [W][4][8]
 
@@ -220,10 +227,10 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   const int end = min(start + L, T);
   const int Q = static_cast<int>(quantized_len(T, a.R, G));
   const int qend = min(end, Q);
-  float* corr = reinterpret_cast<float*>(smem + decode_corr_offset<KB, VB, VPT, GQ, OUT>()) + warp * 4 * kHeadDim;
+  float* corr = reinterpret_cast<float*>(smem + decode_corr_offset<KB, VB, VPT, GQ, OUT>()) + warp * GQ * kHeadDim;
   if constexpr (OUT) {
 #pragma unroll
-    for (int h = 0; h < 4; ++h) *reinterpret_cast<float4*>(corr + h * kHeadDim + 4 * lane) = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int h = 0; h < GQ; ++h) *reinterpret_cast<float4*>(corr + h * kHeadDim + 4 * lane) = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncwarp();
   }
 
@@ -262,10 +269,12 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, d));
     const int e = mx > 0.f ? ((__float_as_int(mx) >> 23) & 0xff) - 126 : 0;
-    *reinterpret_cast<float4*>(sq + warp * kHeadDim + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
-    const float inv = pow2i(-e);
-    *reinterpret_cast<float4*>(sq + 4 * kHeadDim + warp * kHeadDim + 4 * lane) =
-        make_float4(x[0] * inv, x[1] * inv, x[2] * inv, x[3] * inv);
+    if (warp < GQ) {  // the instance holds GQ heads (gq <= GQ; the heads past gq get zeros)
+      *reinterpret_cast<float4*>(sq + warp * kHeadDim + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
+      const float inv = pow2i(-e);
+      *reinterpret_cast<float4*>(sq + GQ * kHeadDim + warp * kHeadDim + 4 * lane) =
+          make_float4(x[0] * inv, x[1] * inv, x[2] * inv, x[3] * inv);
+    }
     if (lane == 0) se[warp] = e;
   }
   __syncthreads();
@@ -277,8 +286,9 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   const bool lo_half = (r & 1) != 0;
   // D-fragment role: this lane's head for the softmax.
   const int h_d = qd % GQ;
-  const float* qn_row = sq + 4 * kHeadDim + col_head * kHeadDim + 2 * qd;  // q^ of head col_head
+  const float* qn_row = sq + GQ * kHeadDim + col_head * kHeadDim + 2 * qd;  // q^ of head col_head
   const float p2e_d = pow2i(se[h_d]);
+  __syncthreads();  // every warp has its exponent: the ring area may be written
 
   // ---- this warp's quantized steps (contiguous)
   const int nsteps = qend > start ? (qend - start) / kStepTokens : 0;
@@ -313,12 +323,14 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   const uint8_t* vz_ptr = nullptr;
   const uint8_t* ko_ptr = nullptr;
   const uint8_t* vo_ptr = nullptr;
+  int64_t page_slot = unit;  // storage slot of the page of the steps being issued
   auto rebase = [&](int t) {
     int64_t slot = unit, ts = t;
     if (a.page_tokens > 0) {
       slot = a.page_table[unit * a.pages_per_unit + t / a.page_tokens];
       ts = t % a.page_tokens;
     }
+    page_slot = slot;
     kc_ptr = reinterpret_cast<const uint8_t*>(a.k_codes + slot * a.tiles * (64 * KB)) + (ts / kTile) * (256 * KB) + 16 * lane;
     vc_ptr = reinterpret_cast<const uint8_t*>(a.v_codes + slot * a.tiles * (64 * VB)) + (ts / kTile) * (256 * VB) + 16 * lane;
     vs_ptr = reinterpret_cast<const uint8_t*>(a.v_scale + (slot * a.slot_tokens + ts) * VPT) + 16 * lane;
@@ -331,12 +343,13 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   if (nst > 0) rebase(first_token);
   // Key scale / zero row of key group g (g < q_groups) for this lane's 16-byte part.
   const uint16_t* kp_base = (lane < 16 ? a.k_scale : a.k_zero) + 8 * (lane & 15);
+  // A key block (at most 128 tokens) never crosses a page, so its groups live in the page of the
+  // step that issues them (rebased just before): no second table lookup.
   auto kp_row = [&](int g) -> const uint16_t* {
     int64_t slot = unit, gs = g;
     if (a.page_tokens > 0) {
-      const int tg = g * G;
-      slot = a.page_table[unit * a.pages_per_unit + tg / a.page_tokens];
-      gs = (tg % a.page_tokens) / G;
+      slot = page_slot;
+      gs = ((g * G) % a.page_tokens) / G;
     }
     return kp_base + (slot * a.groups + gs) * kHeadDim;
   };
