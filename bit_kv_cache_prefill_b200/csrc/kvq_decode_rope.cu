@@ -63,7 +63,8 @@ struct RopeSmem {
   static constexpr int wKP = wQ + GQ * 32 * 16;
   static constexpr int wVS = wKP + 2 * 2 * 32 * 16;
   static constexpr int wVZ = wVS + kRStep * 8 * 4;
-  static constexpr int kWarpBytes = wVZ + kRStep * 8 * 4;
+  static constexpr int wP = wVZ + kRStep * 8 * 4;  // tensor-core P.V: p of the step's tokens [32][GQ] f32
+  static constexpr int kWarpBytes = wP + kRStep * GQ * 4;
   static constexpr int kLoop = oWarp + kRW * kWarpBytes;
   static constexpr int kEpi = oWarp + kRW * GQ * kRPart * 4;  // warp partials reuse the per-warp areas
   static constexpr int kBytes = kLoop > kEpi ? kLoop : kEpi;
@@ -75,6 +76,24 @@ struct RopeSmem {
 __device__ __forceinline__ float2 sub2f(uint32_t x) {
   return __half22float2(*reinterpret_cast<const __half2*>(&x));
 }
+__device__ __forceinline__ void mma16816_rope(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Centered 2-bit value codes of one token pair of a rows-v2 value word (channel row), as the fp16
+// subnormal pair (2c - 3) 2^-24 of the pair's two tokens. x is the word moved so that the pair's codes
+// sit at bits 1..2 (even token) and 17..18 (odd token), i.e. the codes doubled; the odd integer 2c - 3
+// comes from one exact subnormal subtraction. Pair slot k sits at bits 2k and 16 + 2k of the word:
+// slots 0..3 are read from (word << 1) >> 2k, slots 4..7 from word >> (2k - 1), so that no code bit
+// is shifted out.
+__device__ __forceinline__ uint32_t vpair_centered(uint32_t x) {
+  return hsub2(x & 0x00060006u, 0x00030003u);
+}
+
 template <int BITS>
 __device__ __forceinline__ float2 code_pair(uint32_t word, int slot) {  // slot: compile-time after unrolling
   const int o = BITS * slot;
@@ -90,6 +109,12 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
                                                                const float2* __restrict__ roff) {
   using SM = RopeSmem<GQ>;
   constexpr int VPT = kHeadDim / G;
+  // P.V on the tensor cores (mma.sync, channels on M, tokens on K) for 2-bit values with the
+  // rotations on; the CUDA-core control (ROT = false) and 4-bit values keep the CUDA-core P.V.
+  constexpr bool TCPV = ROT && VB == 2;
+  constexpr int VGB = 4 / GQ, NBV = (VPT + VGB - 1) / VGB;  // value groups per n-block, n-blocks
+  static_assert(GQ == 1 || GQ == 2 || GQ == 4, "an n-block holds 4 / GQ value groups of GQ heads");
+  static_assert(G >= 16, "a 16-channel m-tile lies in one value group");
   constexpr int KW = 4 * KB;       // key words per token
   constexpr int KP = 16 / KB;      // code pairs per key word
   constexpr int VW = 4 * VB;       // value words per channel row of a 128-token block
@@ -145,6 +170,17 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
     zacc[h] = 0.f;
     o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0.f;
   }
+  // TCPV roles (the m16n8k16 fragments): lane (r, qd); B column n = r holds (value group offset
+  // col_off, head col_head, hi / lo part); D columns 2qd, 2qd + 1 belong to head h_d.
+  const int qd = lane & 3, r = lane >> 2;
+  const int col_off = r / (2 * GQ), col_head = (r >> 1) % GQ, h_d = qd % GQ;
+  const bool lo_half = (r & 1) != 0;
+  float O[8][4], zt[NBV];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) O[m][0] = O[m][1] = O[m][2] = O[m][3] = 0.f;
+#pragma unroll
+  for (int j = 0; j < NBV; ++j) zt[j] = 0.f;
+  float* wp = reinterpret_cast<float*>(wsm + SM::wP);  // TCPV: p of the step's tokens [32][GQ]
   const int c0 = 4 * lane;    // PV: this lane's channels c0 .. c0 + 3
   const int jv = c0 / G;      // their value group
   int kp_group = -1;          // first key group staged in wkp
@@ -165,13 +201,15 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       kw_next[4 * v + 2] = x.z;
       kw_next[4 * v + 3] = x.w;
     }
-    const int64_t blk = tn / 128;
-    const int wv0 = ((tn & 127) >> 1) / VP;  // first value word of the step
+    if constexpr (!TCPV) {
+      const int64_t blk = tn / 128;
+      const int wv0 = ((tn & 127) >> 1) / VP;  // first value word of the step
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t* row = a.v_codes + (unit * a.capacity + blk * 128 + c0 + e) * VW + wv0;
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t* row = a.v_codes + (unit * a.capacity + blk * 128 + c0 + e) * VW + wv0;
 #pragma unroll
-      for (int k = 0; k < NWV; ++k) vw_next[e][k] = row[k];
+        for (int k = 0; k < NWV; ++k) vw_next[e][k] = row[k];
+      }
     }
   };
   if (nst > 0) load_codes(0);
@@ -222,8 +260,14 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       const bool ok = tt < qend;
       const int64_t pidx = (unit * a.capacity + (ok ? tt : 0)) * VPT + g;
       const int slot = ((tt & 127) >> 1) % VP;
-      wvs[jj * VPT + g] = ok ? h2f(a.v_scale[pidx]) * pow2i(24 - ((VB * slot) & 7)) : 0.f;
-      wvz[jj * VPT + g] = ok ? h2f(a.v_zero[pidx]) : 0.f;
+      if constexpr (TCPV) {  // the scale and the group midpoint zero + 1.5 scale (centered codes)
+        const float sv = ok ? h2f(a.v_scale[pidx]) : 0.f;
+        wvs[jj * VPT + g] = sv;
+        wvz[jj * VPT + g] = ok ? fmaf(1.5f, sv, h2f(a.v_zero[pidx])) : 0.f;
+      } else {
+        wvs[jj * VPT + g] = ok ? h2f(a.v_scale[pidx]) * pow2i(24 - ((VB * slot) & 7)) : 0.f;
+        wvz[jj * VPT + g] = ok ? h2f(a.v_zero[pidx]) : 0.f;
+      }
     }
     // the query turned back to the step start: R_-t0 q, pair (i, i + 64) by -t0 w_i
     if constexpr (!ROT) {
@@ -283,8 +327,18 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       }
     }
 
+    // TCPV: the step's two value words (16 tokens each) of channels 16m + r and 16m + r + 8, loaded
+    // here so that the softmax covers part of their latency
+    uint2 vt[8][2];
+    if constexpr (TCPV) {
+      const uint32_t* vrow = a.v_codes + (unit * a.capacity + (t0 / 128) * 128 + r) * VW + ((t0 & 127) >> 1) / VP;
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) vt[m][u] = *reinterpret_cast<const uint2*>(vrow + (16 * m + 8 * u) * VW);
+    }
     // -- online softmax per head over the step
-    float p[GQ];
+    float p[GQ], alph[GQ];
 #pragma unroll
     for (int h = 0; h < GQ; ++h) {
       const float sh = valid && h < gq ? s[h] : -CUDART_INF_F;
@@ -293,18 +347,85 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kAll, mx, d));
       const float m_new = fmaxf(m_run[h], mx);
       const float alpha = m_new == -CUDART_INF_F ? 1.f : fast_exp2(m_run[h] - m_new);
+      alph[h] = alpha;
       p[h] = sh == -CUDART_INF_F ? 0.f : fast_exp2(sh - m_new);
       l_run[h] = fmaf(l_run[h], alpha, p[h]);
-      zacc[h] *= alpha;
-      o[h][0] *= alpha;
-      o[h][1] *= alpha;
-      o[h][2] *= alpha;
-      o[h][3] *= alpha;
+      if constexpr (!TCPV) {
+        zacc[h] *= alpha;
+        o[h][0] *= alpha;
+        o[h][1] *= alpha;
+        o[h][2] *= alpha;
+        o[h][3] *= alpha;
+      }
       m_run[h] = m_new;
     }
+    if constexpr (TCPV) {
+      // rescale the fragments of head h_d (D) and of col_head (the midpoint sums) when a maximum moved
+      bool moved = false;
+#pragma unroll
+      for (int h = 0; h < GQ; ++h) moved |= alph[h] != 1.f;  // warp-uniform
+      if (moved) {
+        float ad = alph[0], ac = alph[0];
+#pragma unroll
+        for (int h = 1; h < GQ; ++h) {
+          ad = h_d == h ? alph[h] : ad;
+          ac = col_head == h ? alph[h] : ac;
+        }
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          O[m][0] *= ad;
+          O[m][1] *= ad;
+          O[m][2] *= ad;
+          O[m][3] *= ad;
+        }
+#pragma unroll
+        for (int j = 0; j < NBV; ++j) zt[j] *= ac;
+      }
+    }
 
+    if constexpr (TCPV) {
+      // -- PV on the tensor cores. p of the step's tokens goes through shared memory to the B
+      //    fragments: B = p * sv of head col_head, value group nb * VGB + col_off, for tokens 2qd,
+      //    2qd + 1 (b0) and 2qd + 8, 2qd + 9 (b1) of each 16-token k-block, as hi / lo fp16 parts (the
+      //    hi lane of a column makes both parts of its two tokens and passes the lo lane its part, and
+      //    the other way round); A = the centered value codes (channels on M).
+#pragma unroll
+      for (int h = 0; h < GQ; ++h) wp[lane * GQ + h] = p[h];
+      __syncwarp();
+      const int sh_lo = 2 * qd, sh_hi = 7 + 2 * qd;  // pairs qd (from word << 1) and 4 + qd (from word)
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb) {
+        const int tb = 16 * kb + 2 * qd + (lo_half ? 8 : 0);  // this lane's first token in the step
+        const float pe = wp[tb * GQ + col_head], po = wp[(tb + 1) * GQ + col_head];
+        uint32_t bp[NBV][2];
+#pragma unroll
+        for (int nb = 0; nb < NBV; ++nb) {
+          const int j = nb * VGB + col_off;
+          uint32_t hpk = 0u, lpk = 0u;
+          if (VPT % VGB == 0 || j < VPT) {
+            const float se = wvs[tb * VPT + j], so = wvs[(tb + 1) * VPT + j];
+            const float xe = pe * se, xo = po * so;
+            const float he = __uint_as_float(__float_as_uint(xe) & 0xFFFFE000u);
+            const float ho = __uint_as_float(__float_as_uint(xo) & 0xFFFFE000u);
+            hpk = pack_h2(he, ho);
+            lpk = pack_h2(__fsub_rn(xe, he), __fsub_rn(xo, ho));
+            zt[nb] = fmaf(pe, wvz[tb * VPT + j], fmaf(po, wvz[(tb + 1) * VPT + j], zt[nb]));
+          }
+          const uint32_t recv = __shfl_xor_sync(kAll, lo_half ? hpk : lpk, 4);
+          bp[nb][0] = lo_half ? recv : hpk;
+          bp[nb][1] = lo_half ? lpk : recv;
+        }
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const uint32_t wl = kb ? vt[m][0].y : vt[m][0].x;  // channel 16m + r
+          const uint32_t wh = kb ? vt[m][1].y : vt[m][1].x;  // channel 16m + r + 8
+          const int nb = ((16 * m) / G) / VGB;
+          mma16816_rope(O[m], vpair_centered((wl << 1) >> sh_lo), vpair_centered((wh << 1) >> sh_lo),
+                        vpair_centered(wl >> sh_hi), vpair_centered(wh >> sh_hi), bp[nb][0], bp[nb][1]);
+        }
+      }
+    } else {
     // -- PV: lane = channels c0 .. c0 + 3; token pairs of the channel rows of this 128-token block
-    {
 #pragma unroll
       for (int jp = 0; jp < kRStep / 2; ++jp) {  // token pair (2 jp, 2 jp + 1) of the step
         const int k = jp / VP, slot = jp % VP;
@@ -347,8 +468,31 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       ph[0] = m_run[h];
       ph[1] = l;
     }
-    *reinterpret_cast<float4*>(ph + 4 + c0) =
-        make_float4(o[h][0] + zacc[h], o[h][1] + zacc[h], o[h][2] + zacc[h], o[h][3] + zacc[h]);
+    if constexpr (!TCPV)
+      *reinterpret_cast<float4*>(ph + 4 + c0) =
+          make_float4(o[h][0] + zacc[h], o[h][1] + zacc[h], o[h][2] + zacc[h], o[h][3] + zacc[h]);
+  }
+  if constexpr (TCPV) {
+    // midpoint sums over the 8 lanes of a column pair (lanes 8 cp .. 8 cp + 7, pair cp = off GQ + head);
+    // channel rows 16m + r and 16m + r + 8 of head h_d come from the column pair of their value group
+    // jm = 16m / G, held by the lanes with qd / GQ = jm mod VGB; the centered codes carry 2^-24 and
+    // the factor 1/2 of (2c - 3) / 2, hence 2^23
+#pragma unroll
+    for (int j = 0; j < NBV; ++j) {
+      zt[j] += __shfl_xor_sync(kAll, zt[j], 1);
+      zt[j] += __shfl_xor_sync(kAll, zt[j], 2);
+      zt[j] += __shfl_xor_sync(kAll, zt[j], 4);
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int jm = (16 * m) / G;
+      const float z = __shfl_sync(kAll, zt[jm / VGB], 8 * ((jm % VGB) * GQ + h_d));
+      if (qd / GQ == jm % VGB) {
+        float* ph = cw + h_d * kRPart + 4 + 16 * m + r;
+        ph[0] = fmaf(O[m][0] + O[m][1], 0x1p23f, z);
+        ph[8] = fmaf(O[m][2] + O[m][3], 0x1p23f, z);
+      }
+    }
   }
   __syncwarp();
 

@@ -27,6 +27,12 @@ CASES = [
     ("k2v4_g16_r5_gqa3", W("r4", 2, 6, 2, 2, 4, 16, 5, 0, 401, seed=74), [401, 1], 1000000.0, 0),
     ("k4v4_g128_r0_gqa2", W("r5", 1, 4, 2, 4, 4, 128, 0, 0, 3000, seed=75), [3000], 10000.0, 1),
     ("all_in_window", W("r6", 2, 4, 1, 2, 2, 32, 256, 0, 200, seed=76), [200, 256], 10000.0, 0),
+    # 2-bit values (P.V on the tensor cores) at every group size and head ratio: n-blocks of 4, 2 and 1
+    # value groups, channel tiles of one group (G = 16) up to one group per 8 tiles (G = 128)
+    ("k2v2_g16_r16_gqa2", W("r7", 2, 4, 2, 2, 2, 16, 16, 0, 700, seed=77), [700, 129], 10000.0, 0),
+    ("k2v2_g128_r64_mha", W("r8", 1, 2, 2, 2, 2, 128, 64, 0, 1500, seed=78), [1500], 10000.0, 1),
+    ("k4v2_g64_r32_gqa2", W("r9", 2, 4, 2, 4, 2, 64, 32, 0, 1100, seed=79), [1100, 97], 500000.0, 0),
+    ("k2v2_g16_r0_mha_ragged", W("r10", 3, 2, 2, 2, 2, 16, 0, 0, 333, seed=80), [333, 31, 65], 10000.0, 1),
 ]
 
 
