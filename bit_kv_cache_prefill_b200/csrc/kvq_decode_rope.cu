@@ -54,7 +54,7 @@ __global__ void rope_table_kernel(float2* base, float2* off, int nbase, float th
 template <int GQ>
 struct RopeSmem {
   static constexpr int oQ = 0;                                  // q~ [GQ][128] f32 (base-2 logits)
-  static constexpr int oOff = oQ + GQ * 128 * 4;                // (cos, sin) (j w_i), pairs 2p, 2p + 1: [32][33] float4
+  static constexpr int oOff = oQ + GQ * 128 * 4;                // (cos, cos, sin, sin) (j w_i), pairs 2p, 2p + 1: [32][33] float4
   static constexpr int oWarp = oOff + kRStep * kOffStride * 16;  // per-warp areas
   // per warp: turned query [GQ][64] float4 (q_i, q_{i+1}, q_{i+64}, q_{i+65}) for even i -> [GQ][32]
   // float4; key scale / zero of up to two groups [2][32] float4 x 2 (low / high channel pairs);
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
     for (int idx = threadIdx.x; idx < kRStep * 32; idx += kRW * 32) {
       const int j = idx >> 5, p = idx & 31;
       const float2 c0 = roff[j * 64 + 2 * p], c1 = roff[j * 64 + 2 * p + 1];
-      soff[j * kOffStride + p] = make_float4(c0.x, c0.y, c1.x, c1.y);
+      soff[j * kOffStride + p] = make_float4(c0.x, c1.x, c0.y, c1.y);
     }
   }
   __syncthreads();
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
 #pragma unroll
       for (int k = 0; k < NWV; ++k) vw[e][k] = vw_next[e][k];
     if (i + 1 < nst) load_codes(i + 1);
-    // key scale / zero of the step's groups: wkp[g][half][p] = (s, z) of channels 2p, 2p + 1
+    // key scale / zero of the step's groups: wkp[g][half][p] = (s, s, z, z) of channels 2p, 2p + 1
     // (half 0) or 64 + 2p, 65 + 2p (half 1), fp16 scales pre-multiplied by 2^(24 - (bit & 7)) of
     // their code position (code_pair reads a code at bit & 7) so that the subnormal code times the
     // scale is code * s
@@ -246,8 +246,8 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
           const int slot = (c % (2 * KP)) / 2;
           const float sc = pow2i(24 - ((KB * slot) & 7));
           wkp[(gg * 2 + hf) * 32 + lane] = make_float4(h2f(static_cast<uint16_t>(sv & 0xffffu)) * sc,
-                                                       h2f(static_cast<uint16_t>(zv & 0xffffu)),
                                                        h2f(static_cast<uint16_t>(sv >> 16)) * sc,
+                                                       h2f(static_cast<uint16_t>(zv & 0xffffu)),
                                                        h2f(static_cast<uint16_t>(zv >> 16)));
         }
       }
@@ -291,10 +291,13 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
     __syncwarp();
 
     // -- QK: lane = token t, offset j = lane from the step start
+    // Packed fp32 (f32x2) arithmetic on the channel pairs (c, c + 1) and (c + 64, c + 65): half the
+    // instructions of the scalar form for the same operations.
     float s[GQ];
-#pragma unroll
-    for (int h = 0; h < GQ; ++h) s[h] = 0.f;
     {
+      float2 s2[GQ];
+#pragma unroll
+      for (int h = 0; h < GQ; ++h) s2[h] = make_float2(0.f, 0.f);
       const int gl = G >= kRStep ? 0 : lane / G;  // this token's group among the staged ones
       const float4* oj = soff + lane * kOffStride;
 #pragma unroll
@@ -302,29 +305,27 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
         const int c = 2 * p, w = c / (2 * KP), slot = (c % (2 * KP)) / 2;
         const float2 lo = code_pair<KB>(kw[w], slot);           // codes of c, c + 1
         const float2 hi = code_pair<KB>(kw[w + KW / 2], slot);  // codes of c + 64, c + 65
-        const float4 kl = wkp[(gl * 2 + 0) * 32 + p];
+        const float4 kl = wkp[(gl * 2 + 0) * 32 + p];           // (s_c, s_c+1, z_c, z_c+1)
         const float4 kh = wkp[(gl * 2 + 1) * 32 + p];
-        const float x0 = fmaf(lo.x, kl.x, kl.y), x1 = fmaf(lo.y, kl.z, kl.w);
-        const float y0 = fmaf(hi.x, kh.x, kh.y), y1 = fmaf(hi.y, kh.z, kh.w);
-        // R_j on pairs (c, c + 64) and (c + 1, c + 65)
-        float r0 = x0, u0 = y0, r1 = x1, u1 = y1;
+        const float2 x = __ffma2_rn(lo, make_float2(kl.x, kl.y), make_float2(kl.z, kl.w));  // k_c, k_c+1
+        const float2 y = __ffma2_rn(hi, make_float2(kh.x, kh.y), make_float2(kh.z, kh.w));  // k_c+64, k_c+65
+        // R_j on pairs (c, c + 64) and (c + 1, c + 65): r = x cos - y sin, u = x sin + y cos
+        float2 r = x, u = y;
         if constexpr (ROT) {
-          const float4 csn = oj[p];
-          const float cs0 = csn.x, sn0 = csn.y, cs1 = csn.z, sn1 = csn.w;
-          r0 = fmaf(x0, cs0, -y0 * sn0);
-          u0 = fmaf(x0, sn0, y0 * cs0);
-          r1 = fmaf(x1, cs1, -y1 * sn1);
-          u1 = fmaf(x1, sn1, y1 * cs1);
+          const float4 csn = oj[p];  // (cos_c, cos_c+1, sin_c, sin_c+1)
+          const float2 cs = make_float2(csn.x, csn.y), sn = make_float2(csn.z, csn.w);
+          r = __ffma2_rn(make_float2(-y.x, -y.y), sn, __fmul2_rn(x, cs));
+          u = __ffma2_rn(x, sn, __fmul2_rn(y, cs));
         }
 #pragma unroll
         for (int h = 0; h < GQ; ++h) {
           const float4 qv = wq[h * 32 + p];
-          s[h] = fmaf(qv.x, r0, s[h]);
-          s[h] = fmaf(qv.y, r1, s[h]);
-          s[h] = fmaf(qv.z, u0, s[h]);
-          s[h] = fmaf(qv.w, u1, s[h]);
+          s2[h] = __ffma2_rn(make_float2(qv.x, qv.y), r, s2[h]);
+          s2[h] = __ffma2_rn(make_float2(qv.z, qv.w), u, s2[h]);
         }
       }
+#pragma unroll
+      for (int h = 0; h < GQ; ++h) s[h] = s2[h].x + s2[h].y;
     }
 
     // TCPV: the step's two value words (16 tokens each) of channels 16m + r and 16m + r + 8, loaded
@@ -520,7 +521,7 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       for (int e = 0; e < 2; ++e) {
         const int i = 2 * lane + e;
         const float2 cb = bt[i];
-        const float co = e ? oj.z : oj.x, so = e ? oj.w : oj.y;
+        const float co = e ? oj.y : oj.x, so = e ? oj.w : oj.z;
         const float cs = fmaf(cb.x, co, -cb.y * so);
         const float sn = fmaf(cb.y, co, cb.x * so);
         const float x = e ? lo.y : lo.x, y = e ? hi.y : hi.x;
