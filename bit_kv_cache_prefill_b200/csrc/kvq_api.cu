@@ -268,7 +268,7 @@ kvq_status kvq_quantize_prefill(const kvq_config* cfg, kvq_cache* cache, const v
   a.stride_b = stride_b;
   a.stride_t = stride_t;
   a.stride_h = stride_h;
-  return cuda_status(kvq::launch_prefill(a, tmax, stream));
+  return cuda_status(kvq::launch_prefill(a, cache->seq_len_host, stream));
 }
 
 kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache, const void* k_new, const void* v_new,

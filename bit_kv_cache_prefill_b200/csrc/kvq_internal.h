@@ -84,9 +84,18 @@ struct LenChunk {
   int64_t len[kLenChunk];
 };
 
+// The 128-token blocks of up to kLenChunk consecutive sequences [b0, b0 + n), numbered in sequence
+// order: sequence b0 + i owns blocks cum[i] .. cum[i + 1] - 1. Passed by value to a prefill launch
+// whose grid enumerates only the blocks that exist (ragged batches); n = 0 selects the plain grid.
+struct BlockMap {
+  int32_t b0;
+  int32_t n;
+  int32_t cum[kLenChunk + 1];
+};
+
 // Write lens[0 .. batch) into the device mirror (one small launch per kLenChunk sequences).
 cudaError_t launch_set_lengths(int64_t* seq_len_dev, const int64_t* lens, int batch, cudaStream_t stream);
-cudaError_t launch_prefill(const QuantizeArgs& a, int64_t max_len, cudaStream_t stream);
+cudaError_t launch_prefill(const QuantizeArgs& a, const int64_t* lens, cudaStream_t stream);  // lens: host [batch]
 // Append one token to every sequence; old_lens[b] is sequence b's length before the append (the host
 // mirror). The launch also writes the new lengths into the device mirror.
 cudaError_t launch_append(const QuantizeArgs& a, const int64_t* old_lens, const uint16_t* k_new, const uint16_t* v_new,

@@ -83,6 +83,29 @@ def test_more_sequences_than_one_length_chunk(oracle_mod):
         H.compare_unit_cache(w, gv, b, 0, oc, b, 0, int(lens[b]) + appends)
 
 
+@pytest.mark.parametrize("layout", [1, 2])
+def test_compact_prefill_grid_over_chunks(oracle_mod, layout):
+    """A ragged batch of 300 sequences (0 to 768 tokens, half of the plain grid past the sequences' ends):
+    on the tile layout the prefill launches only the blocks that exist, 256 sequences per launch (the
+    rows layout keeps the plain grid), and every unit's codes, parameters and ring match the oracle bit
+    for bit; the decode over them matches too."""
+
+    w = inputs.Workload("compact", 300, 4, 2, 2, 2, 32, 32, 0, 768, seed=73)
+    lens = (np.arange(300, dtype=np.int64) * 97) % 701
+    lens[::37] = 0
+    lens[5] = 768  # the longest sequence sets the plain grid's width
+    assert 4 * (300 * 6 - int(np.sum((lens + 127) // 128))) > 300 * 6  # the compact grid is chosen
+    k, v = _inputs(w, lens)
+    q = inputs.query(w)
+    run = H.run_gpu(w, k.cuda(), v.cuda(), lens, q, layout=layout)
+    oc, ref = H.oracle_full(oracle_mod, w, k, v, lens, q, layout=layout)
+    gv = H.gpu_views(w, run)
+    for b in range(w.batch):
+        for h in range(w.num_kv_heads):
+            H.compare_unit_cache(w, gv, b, h, oc, b, h, int(lens[b]), layout=layout)
+    H.check_attention(run.out.cpu().numpy(), ref, f"compact grid, layout {layout}")
+
+
 def _inputs(w, lens):
     k = torch.zeros(w.batch, int(lens.max()), w.num_kv_heads, 128, dtype=torch.float16)
     v = torch.zeros_like(k)
