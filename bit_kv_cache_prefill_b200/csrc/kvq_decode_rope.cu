@@ -50,25 +50,45 @@ __global__ void rope_table_kernel(float2* base, float2* off, int nbase, float th
   }
 }
 
-// Shared memory layout (bytes).
-template <int GQ>
+// Shared memory layout (bytes). TC: the tensor-core P.V instance, which also stages the next
+// step's value words, value scale / zero and key scale / zero with cp.async.
+template <int GQ, int G, bool TC>
 struct RopeSmem {
+  static constexpr int VPT = kHeadDim / G;
+  static constexpr int NG = G >= kRStep ? 1 : kRStep / G;       // key groups per step
   static constexpr int oQ = 0;                                  // q~ [GQ][128] f32 (base-2 logits)
   static constexpr int oOff = oQ + GQ * 128 * 4;                // (cos, cos, sin, sin) (j w_i), pairs 2p, 2p + 1: [32][33] float4
   static constexpr int oWarp = oOff + kRStep * kOffStride * 16;  // per-warp areas
   // per warp: turned query [GQ][64] float4 (q_i, q_{i+1}, q_{i+64}, q_{i+65}) for even i -> [GQ][32]
-  // float4; key scale / zero of up to two groups [2][32] float4 x 2 (low / high channel pairs);
-  // value scale (pre-scaled) / zero of the step's tokens [32][8] f32 x 2
+  // float4; key scale / zero of the step's groups [NG][2][32] float4 (low / high channel pairs);
+  // value scale / zero (f32) of the step's tokens [32][VPT] x 2
   static constexpr int wQ = 0;
   static constexpr int wKP = wQ + GQ * 32 * 16;
-  static constexpr int wVS = wKP + 2 * 2 * 32 * 16;
-  static constexpr int wVZ = wVS + kRStep * 8 * 4;
-  static constexpr int wP = wVZ + kRStep * 8 * 4;  // tensor-core P.V: p of the step's tokens [32][GQ] f32
-  static constexpr int kWarpBytes = wP + kRStep * GQ * 4;
+  static constexpr int wVS = wKP + NG * 2 * 32 * 16;
+  static constexpr int wVZ = wVS + kRStep * VPT * 4;
+  static constexpr int wP = wVZ + kRStep * VPT * 4;                      // p of the step's tokens [32][GQ] f32
+  static constexpr int wVC = wP + (TC ? kRStep * GQ * 4 : 0);            // value words [2 stages][128 rows] x 8 bytes
+  static constexpr int kVR = 2 * kRStep * VPT * 2;                       // fp16 value scale | zero of one step
+  static constexpr int wVR = wVC + (TC ? 2 * 128 * 8 : 0);               // [2 stages][kVR]
+  static constexpr int wKR = wVR + (TC ? 2 * kVR : 0);                   // fp16 key scale | zero: [2][NG][512]
+  static constexpr int kWarpBytes = wKR + (TC ? 2 * NG * 512 : 0);
   static constexpr int kLoop = oWarp + kRW * kWarpBytes;
   static constexpr int kEpi = oWarp + kRW * GQ * kRPart * 4;  // warp partials reuse the per-warp areas
   static constexpr int kBytes = kLoop > kEpi ? kLoop : kEpi;
+  static_assert(wVC % 16 == 0 && wVR % 16 == 0 && wKR % 16 == 0 && kWarpBytes % 16 == 0, "cp.async alignment");
 };
+
+__device__ __forceinline__ void rope_cp8(uint32_t saddr, const void* g) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(saddr), "l"(g));
+}
+__device__ __forceinline__ void rope_cp16(uint32_t saddr, const void* g) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(saddr), "l"(g));
+}
+__device__ __forceinline__ void rope_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void rope_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
 
 // Two codes of a word as the fp16 subnormals code * 2^(bit - 24), converted to fp32. Only bits 0..9
 // of a half are mantissa, so a code at bit offset o >= 8 of its half is first shifted down by 8:
@@ -105,13 +125,13 @@ __device__ __forceinline__ float2 code_pair(uint32_t word, int slot) {  // slot:
 // CUDA-core decode of the rows-v2 cache, kept as the control against which the tensor-core kernels'
 // gain is measured (selected with KVQ_DECODE_CUDA_CORES=1, see launch_decode_cuda_cores).
 template <int KB, int VB, int G, int GQ, bool ROT = true>
-__global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs a, const float2* __restrict__ rbase,
+__global__ void __launch_bounds__(kRW * 32, (ROT && VB == 2) ? (GQ == 4 ? 4 : 5) : 1) decode_rope_kernel(const DecodeArgs a, const float2* __restrict__ rbase,
                                                                const float2* __restrict__ roff) {
-  using SM = RopeSmem<GQ>;
-  constexpr int VPT = kHeadDim / G;
   // P.V on the tensor cores (mma.sync, channels on M, tokens on K) for 2-bit values with the
   // rotations on; the CUDA-core control (ROT = false) and 4-bit values keep the CUDA-core P.V.
   constexpr bool TCPV = ROT && VB == 2;
+  using SM = RopeSmem<GQ, G, TCPV>;
+  constexpr int VPT = kHeadDim / G;
   constexpr int VGB = 4 / GQ, NBV = (VPT + VGB - 1) / VGB;  // value groups per n-block, n-blocks
   static_assert(GQ == 1 || GQ == 2 || GQ == 4, "an n-block holds 4 / GQ value groups of GQ heads");
   static_assert(G >= 16, "a 16-channel m-tile lies in one value group");
@@ -213,6 +233,36 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
     }
   };
   if (nst > 0) load_codes(0);
+  // TCPV: the step's value words (channel rows 0..127, the two words of its 32 tokens), fp16 value
+  // scale / zero and, when the step starts a key group, the fp16 key scale / zero of its groups, copied
+  // with cp.async into stage ii & 1 one step ahead
+  const uint32_t wsm_s = static_cast<uint32_t>(__cvta_generic_to_shared(wsm));
+  auto stage_copy = [&](int ii) {
+    const int tn = start + (sb + ii) * kRStep;
+    const int stg = ii & 1;
+    const uint32_t* vsrc = a.v_codes + (unit * a.capacity + (tn / 128) * 128 + lane) * VW + ((tn & 127) >> 1) / VP;
+    const uint32_t vdst = wsm_s + SM::wVC + stg * 1024 + 8 * lane;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rope_cp8(vdst + 256 * k, vsrc + 32 * k * VW);  // rows lane + 32 k
+    if (lane < 4 * VPT) {  // 64 VPT bytes of scales and as many of zeros: 16 bytes per lane
+      const int64_t pb = (unit * a.capacity + tn) * VPT;
+      const uint32_t rdst = wsm_s + SM::wVR + stg * SM::kVR + 16 * lane;
+      rope_cp16(rdst, reinterpret_cast<const uint8_t*>(a.v_scale + pb) + 16 * lane);
+      rope_cp16(rdst + SM::kVR / 2, reinterpret_cast<const uint8_t*>(a.v_zero + pb) + 16 * lane);
+    }
+    if (ii == 0 || tn / G != (tn - kRStep) / G) {  // lanes 0..15: scales, 16..31: zeros of a group
+#pragma unroll
+      for (int gg = 0; gg < SM::NG; ++gg) {
+        const uint16_t* src =
+            (lane < 16 ? a.k_scale : a.k_zero) + (unit * a.groups + tn / G + gg) * kHeadDim + 8 * (lane & 15);
+        rope_cp16(wsm_s + SM::wKR + (stg * SM::NG + gg) * 512 + 16 * lane, src);
+      }
+    }
+    rope_commit();
+  };
+  if constexpr (TCPV) {
+    if (nst > 0) stage_copy(0);
+  }
 
   for (int i = 0; i < nst; ++i) {
     const int t0 = start + (sb + i) * kRStep;
@@ -226,6 +276,12 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
 #pragma unroll
       for (int k = 0; k < NWV; ++k) vw[e][k] = vw_next[e][k];
     if (i + 1 < nst) load_codes(i + 1);
+    if constexpr (TCPV) {  // the next step's copies in flight, this step's landed (every lane's)
+      if (i + 1 < nst) stage_copy(i + 1);
+      else rope_commit();
+      rope_wait<1>();
+      __syncwarp();
+    }
     // key scale / zero of the step's groups: wkp[g][half][p] = (s, s, z, z) of channels 2p, 2p + 1
     // (half 0) or 64 + 2p, 65 + 2p (half 1), fp16 scales pre-multiplied by 2^(24 - (bit & 7)) of
     // their code position (code_pair reads a code at bit & 7) so that the subnormal code times the
@@ -240,8 +296,15 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           const int c = 64 * hf + 2 * lane;
-          const uint32_t sv = *reinterpret_cast<const uint32_t*>(a.k_scale + gidx + c);
-          const uint32_t zv = *reinterpret_cast<const uint32_t*>(a.k_zero + gidx + c);
+          uint32_t sv, zv;
+          if constexpr (TCPV) {  // staged by cp.async
+            const uint8_t* kr = wsm + SM::wKR + ((i & 1) * SM::NG + gg) * 512;
+            sv = *reinterpret_cast<const uint32_t*>(kr + 2 * c);
+            zv = *reinterpret_cast<const uint32_t*>(kr + 256 + 2 * c);
+          } else {
+            sv = *reinterpret_cast<const uint32_t*>(a.k_scale + gidx + c);
+            zv = *reinterpret_cast<const uint32_t*>(a.k_zero + gidx + c);
+          }
           // channel c sits in key word c / (2 KP) at pair slot (c % (2 KP)) / 2, bit KB * slot
           const int slot = (c % (2 * KP)) / 2;
           const float sc = pow2i(24 - ((KB * slot) & 7));
@@ -261,9 +324,10 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       const int64_t pidx = (unit * a.capacity + (ok ? tt : 0)) * VPT + g;
       const int slot = ((tt & 127) >> 1) % VP;
       if constexpr (TCPV) {  // the scale and the group midpoint zero + 1.5 scale (centered codes)
-        const float sv = ok ? h2f(a.v_scale[pidx]) : 0.f;
+        const uint16_t* vr = reinterpret_cast<const uint16_t*>(wsm + SM::wVR + (i & 1) * SM::kVR);
+        const float sv = ok ? h2f(vr[idx]) : 0.f;
         wvs[jj * VPT + g] = sv;
-        wvz[jj * VPT + g] = ok ? fmaf(1.5f, sv, h2f(a.v_zero[pidx])) : 0.f;
+        wvz[jj * VPT + g] = ok ? fmaf(1.5f, sv, h2f(vr[kRStep * VPT + idx])) : 0.f;
       } else {
         wvs[jj * VPT + g] = ok ? h2f(a.v_scale[pidx]) * pow2i(24 - ((VB * slot) & 7)) : 0.f;
         wvz[jj * VPT + g] = ok ? h2f(a.v_zero[pidx]) : 0.f;
@@ -328,16 +392,6 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       for (int h = 0; h < GQ; ++h) s[h] = s2[h].x + s2[h].y;
     }
 
-    // TCPV: the step's two value words (16 tokens each) of channels 16m + r and 16m + r + 8, loaded
-    // here so that the softmax covers part of their latency
-    uint2 vt[8][2];
-    if constexpr (TCPV) {
-      const uint32_t* vrow = a.v_codes + (unit * a.capacity + (t0 / 128) * 128 + r) * VW + ((t0 & 127) >> 1) / VP;
-#pragma unroll
-      for (int m = 0; m < 8; ++m)
-#pragma unroll
-        for (int u = 0; u < 2; ++u) vt[m][u] = *reinterpret_cast<const uint2*>(vrow + (16 * m + 8 * u) * VW);
-    }
     // -- online softmax per head over the step
     float p[GQ], alph[GQ];
 #pragma unroll
@@ -394,11 +448,11 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
       for (int h = 0; h < GQ; ++h) wp[lane * GQ + h] = p[h];
       __syncwarp();
       const int sh_lo = 2 * qd, sh_hi = 7 + 2 * qd;  // pairs qd (from word << 1) and 4 + qd (from word)
+      uint32_t bp[2][NBV][2];
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb) {
         const int tb = 16 * kb + 2 * qd + (lo_half ? 8 : 0);  // this lane's first token in the step
         const float pe = wp[tb * GQ + col_head], po = wp[(tb + 1) * GQ + col_head];
-        uint32_t bp[NBV][2];
 #pragma unroll
         for (int nb = 0; nb < NBV; ++nb) {
           const int j = nb * VGB + col_off;
@@ -413,17 +467,21 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
             zt[nb] = fmaf(pe, wvz[tb * VPT + j], fmaf(po, wvz[(tb + 1) * VPT + j], zt[nb]));
           }
           const uint32_t recv = __shfl_xor_sync(kAll, lo_half ? hpk : lpk, 4);
-          bp[nb][0] = lo_half ? recv : hpk;
-          bp[nb][1] = lo_half ? lpk : recv;
+          bp[kb][nb][0] = lo_half ? recv : hpk;
+          bp[kb][nb][1] = lo_half ? lpk : recv;
         }
+      }
+      // A: the staged value words of channel rows 16m + r and 16m + r + 8 (word x: tokens 0..15 of
+      // the step, k-block 0; word y: tokens 16..31, k-block 1)
+      const uint2* vc = reinterpret_cast<const uint2*>(wsm + SM::wVC + (i & 1) * 1024);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const uint32_t wl = kb ? vt[m][0].y : vt[m][0].x;  // channel 16m + r
-          const uint32_t wh = kb ? vt[m][1].y : vt[m][1].x;  // channel 16m + r + 8
-          const int nb = ((16 * m) / G) / VGB;
-          mma16816_rope(O[m], vpair_centered((wl << 1) >> sh_lo), vpair_centered((wh << 1) >> sh_lo),
-                        vpair_centered(wl >> sh_hi), vpair_centered(wh >> sh_hi), bp[nb][0], bp[nb][1]);
-        }
+      for (int m = 0; m < 8; ++m) {
+        const uint2 wl = vc[16 * m + r], wh = vc[16 * m + 8 + r];
+        const int nb = ((16 * m) / G) / VGB;
+        mma16816_rope(O[m], vpair_centered((wl.x << 1) >> sh_lo), vpair_centered((wh.x << 1) >> sh_lo),
+                      vpair_centered(wl.x >> sh_hi), vpair_centered(wh.x >> sh_hi), bp[0][nb][0], bp[0][nb][1]);
+        mma16816_rope(O[m], vpair_centered((wl.y << 1) >> sh_lo), vpair_centered((wh.y << 1) >> sh_lo),
+                      vpair_centered(wl.y >> sh_hi), vpair_centered(wh.y >> sh_hi), bp[1][nb][0], bp[1][nb][1]);
       }
     } else {
     // -- PV: lane = channels c0 .. c0 + 3; token pairs of the channel rows of this 128-token block
@@ -457,6 +515,7 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
   }
 
   // ---- warp partials -> shared memory (l summed over lanes; the zero-point term per value group)
+  if constexpr (TCPV) rope_wait<0>();  // no copy in flight into the per-warp areas
   __syncthreads();  // the per-warp areas become the partials
   float* cw = reinterpret_cast<float*>(smem + SM::oWarp) + warp * GQ * kRPart;
 #pragma unroll
@@ -590,7 +649,7 @@ __global__ void __launch_bounds__(kRW * 32) decode_rope_kernel(const DecodeArgs 
 
 template <int KB, int VB, int G, int GQ, bool ROT>
 cudaError_t launch_rope_kernel(const DecodeArgs& a, cudaStream_t stream) {
-  using SM = RopeSmem<GQ>;
+  using SM = RopeSmem<GQ, G, ROT && VB == 2>;
   static DeviceMemo attr;
   const int ok = attr.get([] {
     return cudaFuncSetAttribute(decode_rope_kernel<KB, VB, G, GQ, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -652,7 +711,7 @@ template <int KB, int VB, int G, int GQ, bool ROT>
 int rope_occupancy() {
   static DeviceMemo occ;
   return occ.get([] {
-    using SM = RopeSmem<GQ>;
+    using SM = RopeSmem<GQ, G, ROT && VB == 2>;
     if (cudaFuncSetAttribute(decode_rope_kernel<KB, VB, G, GQ, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SM::kBytes) != cudaSuccess)
       return 1;
