@@ -405,6 +405,7 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
   a.qscale = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
   const WorkspaceLayout wl = workspace_layout(cfg);
   a.status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + wl.status);
+  a.stall_test = kvq::stall_test_requested() ? 1 : 0;
   if (cfg->rope_theta > 0.f) {
     a.rope_theta = cfg->rope_theta;
     a.rope_base = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + wl.rope);

@@ -894,6 +894,11 @@ bool cuda_core_control_requested(int layout, float rope_theta, int hadamard) {
   return v != nullptr && v[0] == '1';
 }
 
+bool stall_test_requested() {
+  const char* v = std::getenv("KVQ_TEST_STALL_TC");
+  return v != nullptr && v[0] == '1';
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e;
   if (a.rope_theta > 0.f)

@@ -314,7 +314,9 @@ __global__ void __launch_bounds__(kThreads, TcPlan<KB, VB, VPT, GQ>::kCtasPerSm)
   const int end = min(start + L, T);
   const int Q = static_cast<int>(quantized_len(T, a.R, G));
   const int qend = min(end, Q);
-  const int nsteps = qend > start ? (qend - start + kStep - 1) / kStep : 0;
+  // a.stall_test: no quantized step is issued (nothing lands in shared memory, no MMA runs), and one
+  // thread waits below on a barrier phase that nothing completes
+  const int nsteps = qend > start && !a.stall_test ? (qend - start + kStep - 1) / kStep : 0;
 
   // Bulk copies of step j into stage j % S (one thread).
   const uint8_t* kc_base = reinterpret_cast<const uint8_t*>(a.k_codes) + (unit * a.capacity + start) * (16 * KB);
@@ -792,6 +794,7 @@ __global__ void __launch_bounds__(kThreads, TcPlan<KB, VB, VPT, GQ>::kCtasPerSm)
       }
     }
   }
+  if (a.stall_test && tid == 0) mbar_wait(&bars[P::kBarPV], 0, sflag);  // gives up after about 2 s
   const bool gave_up = __syncthreads_or(*sflag != 0);
 
   // ---- CTA partial: merge the quantized partial and the 8 window partials -> workspace

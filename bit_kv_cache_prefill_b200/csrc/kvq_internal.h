@@ -71,6 +71,8 @@ struct DecodeArgs {
   float rope_theta;  // > 0: keys are cached before RoPE; decode rotates them (rows v2 only)
   float2* rope_base;  // workspace: (cos, sin)(32 s w_i), [ceil(capacity / 32)][64]
   float2* rope_off;   // workspace: (cos, sin)(j w_i), [32][64]
+  int stall_test;     // 1: the tcgen05 kernel runs no quantized step and waits on a barrier that nothing
+                      // completes, so its bounded wait gives up (a test of the give-up path; KVQ_TEST_STALL_TC=1)
 };
 
 // Sequence lengths of up to kLenChunk consecutive sequences [base, base + n), passed to a kernel by
@@ -110,6 +112,8 @@ int decode_rope_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);  // p
 cudaError_t launch_decode_cuda_cores(const DecodeArgs& a, cudaStream_t stream);
 int decode_cuda_cores_ctas_per_sm(int key_bits, int value_bits, int G, int gqa);
 bool cuda_core_control_requested(int layout, float rope_theta, int hadamard);
+// KVQ_TEST_STALL_TC=1: the tcgen05 decode gives up a bounded wait on purpose (no copy or MMA in flight).
+bool stall_test_requested();
 int64_t rope_table_floats(int64_t capacity);  // floats of the two RoPE tables in the workspace
 int decode_ctas_per_sm(int key_bits, int value_bits, int G, int gqa, int outliers);  // tile-v1 kernel
 int decode_tc_ctas_per_sm(int G, int gqa);                              // rows-v2 kernel (1 or 2)

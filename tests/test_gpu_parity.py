@@ -255,6 +255,33 @@ def test_decode_status_is_ok_after_a_decode_that_finishes(layout):
     assert torch.isfinite(out.float()).all()
 
 
+def test_tcgen05_bounded_wait_gives_up_and_reports(oracle_mod, monkeypatch):
+    """KVQ_TEST_STALL_TC=1 makes one thread of every tcgen05 decode CTA wait on a barrier phase that
+    nothing completes, with no copy and no MMA in flight (the CTA issues no quantized step): the bounded
+    wait gives up after about 2 s, the outputs are NaN and kvq_decode_status reports KVQ_ERR_TIMEOUT.
+    The next decode on the same context and workspace is correct and reports KVQ_OK."""
+    import bit_kv_cache_prefill_b200 as kvq
+
+    w = inputs.Workload("stall", 1, 4, 1, 2, 2, 32, 32, 0, 640, seed=91)
+    lens = np.array([640], np.int64)
+    k, v = _inputs_for(w, lens)
+    q = inputs.query(w)
+    cfg = H.gpu_config(w, 2)
+    cache = kvq.Cache(cfg)
+    kvq.kvq_quantize_prefill(cfg, cache, k.cuda(), v.cuda(), lens)
+    ws = torch.zeros(kvq.kvq_decode_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+    out = torch.empty(w.batch, w.num_q_heads, 128, dtype=torch.float16, device="cuda")
+    monkeypatch.setenv("KVQ_TEST_STALL_TC", "1")
+    kvq.kvq_decode_attention(cfg, cache, q.cuda(), out, 1 / math.sqrt(128), ws)
+    assert kvq.kvq_decode_status(cfg, ws) == kvq.KVQ_ERR_TIMEOUT
+    assert torch.isnan(out.float()).all()
+    monkeypatch.delenv("KVQ_TEST_STALL_TC")
+    kvq.kvq_decode_attention(cfg, cache, q.cuda(), out, 1 / math.sqrt(128), ws)
+    assert kvq.kvq_decode_status(cfg, ws) == kvq.KVQ_OK
+    _, ref = H.oracle_full(oracle_mod, w, k, v, lens, q, layout=2)
+    H.check_attention(out.cpu().numpy(), ref, "decode after a give-up")
+
+
 @pytest.mark.parametrize("sink", [0, 1], ids=["nosink", "sink"])
 @pytest.mark.parametrize("name,w,lens", [c for c in SMALL if not c[1].hadamard][:6], ids=lambda x: x if isinstance(x, str) else "")
 def test_cuda_core_control_matches_the_oracle(oracle_mod, monkeypatch, name, w, lens, sink):
