@@ -273,7 +273,9 @@ kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache* 
  * bounded waits (about 2 s); a CTA that gives up writes NaN partials instead of hanging, and the
  * split combine then records, per (sequence, query head), whether its output came out NaN that way.
  * Every decode call rewrites those records (they sit at the end of the workspace, within
- * kvq_decode_workspace_bytes), so nothing needs clearing.
+ * kvq_decode_workspace_bytes), so nothing needs clearing. With KVQ_TEST_STALL_TC=1 in the process
+ * environment, the rows-v2 decode (no RoPE) issues no quantized step and waits on a barrier that
+ * nothing completes, so that it gives up on purpose: a test hook for this path, off by default.
  * This call copies the records to the host on `cuda_stream` and synchronises that stream: call it
  * on the stream of the decode (or after it), before the workspace is reused.
  * Returns KVQ_OK, KVQ_ERR_TIMEOUT if some output of that decode is NaN from a give-up, or
