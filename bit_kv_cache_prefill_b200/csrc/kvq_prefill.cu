@@ -132,9 +132,12 @@ constexpr int key_scratch_bytes() {
 // its channel's zero, which codes to 0.
 // The block's tokens t0 .. t0 + nq - 1 are stored in slot `slot` from in-slot token ts0 on (the unit
 // and t0, or with paged storage the pool page and t0 mod page_tokens).
-template <int BITS, int LAYOUT, int G, bool OUT>
-__device__ void key_block(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, int nq, const uint16_t* rows,
+// NQ = kPB: a whole block of quantized tokens (every trip count fixed at compile time); NQ = 0: nq of
+// them.
+template <int BITS, int LAYOUT, int G, bool OUT, int NQ>
+__device__ void key_block(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, int nq_arg, const uint16_t* rows,
                           uint8_t* scratch, const uint8_t* och) {
+  const int nq = NQ ? NQ : nq_arg;
   constexpr int top = (1 << BITS) - 1;
   constexpr int P = 16 / BITS;  // code pairs per word
   const int NG = nq / G;
@@ -343,9 +346,10 @@ constexpr int val_scratch_bytes() {
 
 // With OUT, select_outliers has replaced each token's value outlier by its neighbour (so the min / max
 // leave it out); once the token's parameters are known the entry becomes its group's zero (code 0).
-template <int BITS, int LAYOUT, int G, bool OUT>
-__device__ void value_block(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, int nq, const uint16_t* rows,
+template <int BITS, int LAYOUT, int G, bool OUT, int NQ>
+__device__ void value_block(const QuantizeArgs& a, int64_t slot, int64_t ts0, int64_t t0, int nq_arg, const uint16_t* rows,
                             uint8_t* scratch, const uint8_t* och) {
+  const int nq = NQ ? NQ : nq_arg;  // NQ = kPB: a whole block (trip counts fixed at compile time)
   constexpr int top = (1 << BITS) - 1;
   constexpr int P = 16 / BITS;
   constexpr int VPT = kHeadDim / G;
@@ -574,10 +578,21 @@ __global__ void __launch_bounds__(kPThreads) prefill_block_kernel(QuantizeArgs a
                     a.sink && t0 == 0, !is_key, kPThreads / 32);
     __syncthreads();
   }
+  // whole blocks of the tile layout take the instance with fixed trip counts (on the rows layout it
+  // needs more registers than five CTAs per SM allow)
+  if constexpr (LAYOUT == KVQ_LAYOUT_TILE_V1) {
+    if (nq == kPB) {
+      if (is_key)
+        key_block<BITS_K, LAYOUT, G, OUT, kPB>(a, slot, ts0, t0, nq, rows, scratch, och);
+      else
+        value_block<BITS_V, LAYOUT, G, OUT, kPB>(a, slot, ts0, t0, nq, rows, scratch, och);
+      return;
+    }
+  }
   if (is_key)
-    key_block<BITS_K, LAYOUT, G, OUT>(a, slot, ts0, t0, nq, rows, scratch, och);
+    key_block<BITS_K, LAYOUT, G, OUT, 0>(a, slot, ts0, t0, nq, rows, scratch, och);
   else
-    value_block<BITS_V, LAYOUT, G, OUT>(a, slot, ts0, t0, nq, rows, scratch, och);
+    value_block<BITS_V, LAYOUT, G, OUT, 0>(a, slot, ts0, t0, nq, rows, scratch, och);
 }
 
 // Shared memory of one CTA: the rows, then the larger of the key and value scratch (and with OUT the
