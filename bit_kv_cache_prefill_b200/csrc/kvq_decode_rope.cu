@@ -1,4 +1,5 @@
-// kvq_decode_rope.cu — split-K decode attention over pre-RoPE keys (rows-v2 layout), on CUDA cores.
+// kvq_decode_rope.cu — split-K decode attention over pre-RoPE keys (rows-v2 layout): QK on CUDA
+// cores, P.V on the tensor cores (2-bit values).
 //
 // Keys can be cached before RoPE and rotated only after dequantization (KVQuant review, Method and
 // Key idea: RoPE mixes channel pairs and smears the key outlier channels, so the quantizer runs
@@ -6,15 +7,20 @@
 // turned pair by pair, channels (i, i + 64), by the angle t * theta^(-i/64); the query arrives already
 // rotated at its own position.
 //
-// A rotation per token defeats the shared-B tensor-core formulation of the other decode kernels (the
-// effective query would change with every key row), so this path computes on CUDA cores:
+// A rotation per token defeats the shared-B tensor-core formulation of QK in the other decode kernels
+// (the effective query would change with every key row), so QK runs on CUDA cores:
 //   * QK, lane = token. <q, R_t k> = <R_-t0 q, R_j k> with t = t0 + j and t0 the warp step's first
 //     token (a multiple of 32): the query is turned once per step to R_-t0 q (cooperatively, into
 //     shared memory) and each lane turns its dequantized key by its in-step offset j only, from a
-//     padded shared table of (cos, sin) (j w_i) for two channel pairs per 16-byte entry.
-//   * PV, lane = 4 channels. o = sum_t (p_t sv_t) c_t + sum_t p_t zv_t per value group.
+//     padded shared table of (cos, sin) (j w_i) for two channel pairs per 16-byte entry. The
+//     dequantization, rotation and dot products run in packed f32x2 arithmetic.
 //   * Codes are read as fp16 subnormals (one AND per code pair, the position's power of two folded
 //     into the staged scales), as in the tile-v1 kernel.
+//   * P.V is untouched by the rotation: with 2-bit values it is an mma.sync (channels on M, tokens on
+//     K, A = the centered value codes, B = p * sv as hi / lo fp16 per value group and head), and the
+//     next step's value words and value / key parameters are staged with cp.async. With 4-bit values
+//     (and in the CUDA-core control instance, ROT = false) P.V runs on CUDA cores, lane = 4 channels:
+//     o = sum_t (p_t sv_t) c_t + sum_t p_t zv_t per value group.
 // The angle tables are built once per call in fp64 (cos / sin of 32 s w_i and of j w_i) into the
 // decode workspace behind the split partials; partials have the layout the split-combine kernel
 // reads.
