@@ -131,7 +131,7 @@ __device__ __forceinline__ float2 code_pair(uint32_t word, int slot) {  // slot:
 // CUDA-core decode of the rows-v2 cache, kept as the control against which the tensor-core kernels'
 // gain is measured (selected with KVQ_DECODE_CUDA_CORES=1, see launch_decode_cuda_cores).
 template <int KB, int VB, int G, int GQ, bool ROT = true>
-__global__ void __launch_bounds__(kRW * 32, (ROT && VB == 2) ? (GQ == 4 ? 4 : 5) : 1) decode_rope_kernel(const DecodeArgs a, const float2* __restrict__ rbase,
+__global__ void __launch_bounds__(kRW * 32, (ROT && VB == 2) ? ((GQ == 4 || (KB == 4 && GQ == 2)) ? 4 : 5) : 1) decode_rope_kernel(const DecodeArgs a, const float2* __restrict__ rbase,
                                                                const float2* __restrict__ roff) {
   // P.V on the tensor cores (mma.sync, channels on M, tokens on K) for 2-bit values with the
   // rotations on; the CUDA-core control (ROT = false) and 4-bit values keep the CUDA-core P.V.
