@@ -122,7 +122,11 @@ static_assert(smem_fixed<1>() % 16 == 0 && smem_fixed<2>() % 16 == 0 && smem_fix
 template <int KB, int VB, int VPT, int GQ, bool OUT>
 struct Shape {
   static constexpr int KGB = 4 / GQ;                     // key groups per QK B block
-  static constexpr int VGB = 4 / GQ;                     // value groups per PV n-block
+  // P.V B operand: with every column of an n-block in use (VPT a multiple of 8 / GQ), one fp16 column
+  // per (value group, head), 8 / GQ value groups per n-block (PV1); else hi / lo fp16 column pairs,
+  // 4 / GQ value groups per n-block
+  static constexpr bool PV1 = VPT % (8 / GQ) == 0;
+  static constexpr int VGB = PV1 ? 8 / GQ : 4 / GQ;      // value groups per PV n-block
   static constexpr int NBV = (VPT + VGB - 1) / VGB;      // PV n-blocks
   static constexpr int G = 128 / VPT;
   // tiles per step: 4 for 2-bit keys and values with G >= 64 (a step never spans two key groups),
@@ -205,6 +209,7 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   using SH = Shape<KB, VB, VPT, GQ, OUT>;
   using S = typename SH::S;
   constexpr int KGB = SH::KGB, VGB = SH::VGB, NBV = SH::NBV, G = SH::G, TS = SH::TS;
+  constexpr bool PV1 = SH::PV1;
   constexpr int kBlockTokens = G * KGB;
   constexpr int kStepTokens = 16 * TS;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -284,6 +289,10 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   const int col_off = r / (2 * GQ);
   const int col_head = (r >> 1) % GQ;
   const bool lo_half = (r & 1) != 0;
+  // P.V B-fragment role (column n = r): value group offset and head (PV1: one column each; else the
+  // QK roles, hi / lo pairs)
+  const int pv_off = PV1 ? r / GQ : col_off;
+  const int pv_head = PV1 ? r % GQ : col_head;
   // D-fragment role: this lane's head for the softmax.
   const int h_d = qd % GQ;
   const float* qn_row = sq + GQ * kHeadDim + col_head * kHeadDim + 2 * qd;  // q^ of head col_head
@@ -514,14 +523,26 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
     }
     l_run = fmaf(l_run, alpha, lsum);
     if (__any_sync(kFull, alpha != 1.f)) {
+      if constexpr (PV1) {  // D columns 2qd, 2qd + 1: heads (2qd) % GQ and (2qd + 1) % GQ
+        const float a0 = __shfl_sync(kFull, alpha, (2 * qd) % GQ);  // lane h has h_d == h
+        const float a1 = __shfl_sync(kFull, alpha, (2 * qd + 1) % GQ);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        O[m][0] *= alpha;
-        O[m][1] *= alpha;
-        O[m][2] *= alpha;
-        O[m][3] *= alpha;
+        for (int m = 0; m < 8; ++m) {
+          O[m][0] *= a0;
+          O[m][1] *= a1;
+          O[m][2] *= a0;
+          O[m][3] *= a1;
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          O[m][0] *= alpha;
+          O[m][1] *= alpha;
+          O[m][2] *= alpha;
+          O[m][3] *= alpha;
+        }
       }
-      const float az = __shfl_sync(kFull, alpha, col_head);  // lane col_head has h_d == col_head
+      const float az = __shfl_sync(kFull, alpha, pv_head);  // lane pv_head has h_d == pv_head
 #pragma unroll
       for (int j = 0; j < NBV; ++j) zacc[j] *= az;
       if constexpr (OUT) {
@@ -560,42 +581,67 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
 
     // -- P.V per tile: B = p * sv (hi/lo) of head col_head for tokens 2qd, 2qd+1, 2qd+8, 2qd+9 and
     //    the value group of this lane's column in each n-block; A = centered value codes
-    const int la = 8 * qd + col_head;
+    const int la = 8 * qd + pv_head;
     constexpr float kCbar = VB == 2 ? 1.5f : 7.5f;
 #pragma unroll
     for (int u = 0; u < TS; ++u) {
       const float pa = __shfl_sync(kFull, p[u][0], la), pb = __shfl_sync(kFull, p[u][0], la + 4);
       const float pc = __shfl_sync(kFull, p[u][1], la), pd = __shfl_sync(kFull, p[u][1], la + 4);
-      // The hi lane of a column (r even) takes tokens 2qd, 2qd + 1 (the lower K half of the B
-      // fragment), the lo lane (r odd) tokens 2qd + 8, 2qd + 9; each makes both parts of its products
-      // and passes the partner lane (L ^ 4) the part that lane needs.
       // 2-bit: tokens 2qd + 8, + 9 (the upper K half) carry 2^-4 against the subnormal codes
       constexpr float kTf = VB == 2 ? 0.0625f : 1.f;
-      const float pe = lo_half ? pc : pa, po = lo_half ? pd : pb;  // probabilities of this lane's tokens
-      const float pes = lo_half ? pc * kTf : pa, pos = lo_half ? pd * kTf : pb;
       const uint16_t* vsh = reinterpret_cast<const uint16_t*>(st + S::oVS) + u * 16 * VPT;
       const uint16_t* vzh = reinterpret_cast<const uint16_t*>(st + S::oVZ) + u * 16 * VPT;
       uint32_t bp[NBV][2];
+      if constexpr (PV1) {
+        // one fp16 column per (value group, head): this lane makes all four products of its column,
+        // tokens 2qd, 2qd + 1 (b0) and 2qd + 8, 2qd + 9 (b1). The products keep fp16's 11 significant
+        // bits: a relative error of at most 2^-12 per term of the output sum, far inside the output
+        // tolerance (QK keeps hi / lo, where an error is exponentiated).
+        const float pcs = pc * kTf, pds = pd * kTf;
 #pragma unroll
-      for (int nb = 0; nb < NBV; ++nb) {
-        const int j = nb * VGB + col_off;
-        uint32_t hpk = 0u, lpk = 0u;  // both parts of this lane's two products (0 past the groups)
-        if (VPT % VGB == 0 || j < VPT) {
-          const int te = 2 * qd * VPT + j + (lo_half ? 8 * VPT : 0);  // this lane's first token
-          const float se = h2f(vsh[te]), so = h2f(vsh[te + VPT]);
-          const float ze = h2f(vzh[te]), zo = h2f(vzh[te + VPT]);
-          const float xe = pes * se, xo = pos * so;
-          const float he = split_part(xe, false), ho = split_part(xo, false);
-          hpk = pack_h2(he, ho);
-          lpk = pack_h2(__fsub_rn(xe, he), __fsub_rn(xo, ho));
+        for (int nb = 0; nb < NBV; ++nb) {
+          const int j = nb * VGB + pv_off;  // < VPT: every column is in use
+          const int te = 2 * qd * VPT + j;
+          const float s0 = h2f(vsh[te]), s1 = h2f(vsh[te + VPT]);
+          const float s8 = h2f(vsh[te + 8 * VPT]), s9 = h2f(vsh[te + 9 * VPT]);
+          const float z0 = h2f(vzh[te]), z1 = h2f(vzh[te + VPT]);
+          const float z8 = h2f(vzh[te + 8 * VPT]), z9 = h2f(vzh[te + 9 * VPT]);
+          bp[nb][0] = pack_h2(pa * s0, pb * s1);
+          bp[nb][1] = pack_h2(pcs * s8, pds * s9);
           float z = zacc[nb];
-          z = fmaf(pe, fmaf(kCbar, se, ze), z);
-          z = fmaf(po, fmaf(kCbar, so, zo), z);
+          z = fmaf(pa, fmaf(kCbar, s0, z0), z);
+          z = fmaf(pb, fmaf(kCbar, s1, z1), z);
+          z = fmaf(pc, fmaf(kCbar, s8, z8), z);
+          z = fmaf(pd, fmaf(kCbar, s9, z9), z);
           zacc[nb] = z;
         }
-        const uint32_t recv = __shfl_xor_sync(kFull, lo_half ? hpk : lpk, 4);
-        bp[nb][0] = lo_half ? recv : hpk;  // tokens 2qd, 2qd + 1: hi part here (hi lane), lo part from it
-        bp[nb][1] = lo_half ? lpk : recv;  // tokens 2qd + 8, + 9: lo part here (lo lane), hi part from it
+      } else {
+        // The hi lane of a column (r even) takes tokens 2qd, 2qd + 1 (the lower K half of the B
+        // fragment), the lo lane (r odd) tokens 2qd + 8, 2qd + 9; each makes both parts of its products
+        // and passes the partner lane (L ^ 4) the part that lane needs.
+        const float pe = lo_half ? pc : pa, po = lo_half ? pd : pb;  // probabilities of this lane's tokens
+        const float pes = lo_half ? pc * kTf : pa, pos = lo_half ? pd * kTf : pb;
+#pragma unroll
+        for (int nb = 0; nb < NBV; ++nb) {
+          const int j = nb * VGB + col_off;
+          uint32_t hpk = 0u, lpk = 0u;  // both parts of this lane's two products (0 past the groups)
+          if (VPT % VGB == 0 || j < VPT) {
+            const int te = 2 * qd * VPT + j + (lo_half ? 8 * VPT : 0);  // this lane's first token
+            const float se = h2f(vsh[te]), so = h2f(vsh[te + VPT]);
+            const float ze = h2f(vzh[te]), zo = h2f(vzh[te + VPT]);
+            const float xe = pes * se, xo = pos * so;
+            const float he = split_part(xe, false), ho = split_part(xo, false);
+            hpk = pack_h2(he, ho);
+            lpk = pack_h2(__fsub_rn(xe, he), __fsub_rn(xo, ho));
+            float z = zacc[nb];
+            z = fmaf(pe, fmaf(kCbar, se, ze), z);
+            z = fmaf(po, fmaf(kCbar, so, zo), z);
+            zacc[nb] = z;
+          }
+          const uint32_t recv = __shfl_xor_sync(kFull, lo_half ? hpk : lpk, 4);
+          bp[nb][0] = lo_half ? recv : hpk;  // tokens 2qd, 2qd + 1: hi part here (hi lane), lo part from it
+          bp[nb][1] = lo_half ? lpk : recv;  // tokens 2qd + 8, + 9: lo part here (lo lane), hi part from it
+        }
       }
       // m-block m (channels 16m .. 16m+15) lies in value group (16m) / G, held by n-block group / VGB
       const uint8_t* vc = st + S::oVC + u * 256 * VB;
@@ -635,33 +681,47 @@ __global__ void __launch_bounds__(128, 4) decode_split_kernel(const DecodeArgs a
   l_run += __shfl_xor_sync(kFull, l_run, 16);
 #pragma unroll
   for (int j = 0; j < NBV; ++j) {
-    zacc[j] += __shfl_xor_sync(kFull, zacc[j], 4);  // the hi and lo lanes' tokens
+    if constexpr (!PV1) zacc[j] += __shfl_xor_sync(kFull, zacc[j], 4);  // the hi and lo lanes' tokens
     zacc[j] += __shfl_xor_sync(kFull, zacc[j], 1);
     zacc[j] += __shfl_xor_sync(kFull, zacc[j], 2);
   }
   float* cw = cm + warp * 4 * kCm;
-  if (h_d < gq) {
+  // row scales of the subnormal centered codes (2 (c - cbar) 2^-24 on row r)
+  constexpr float kORowLo = 8388608.0f, kORowHi = VB == 2 ? 2097152.0f : 524288.0f;  // 2^23, 2^21 / 2^19
+  if constexpr (PV1) {
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int jm = (16 * m) / G;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {  // D column 2qd + e: value group offset (2qd + e) / GQ, head (2qd + e) % GQ
+        const int he = (2 * qd + e) % GQ;
+        if ((2 * qd + e) / GQ == jm % VGB && he < gq) {
+          float* o = cw + he * kCm + kCmO;
+          o[16 * m + r] = O[m][e] * kORowLo;
+          o[16 * m + r + 8] = O[m][2 + e] * kORowHi;
+        }
+      }
+    }
+  } else if (h_d < gq) {
     float* o = cw + h_d * kCm + kCmO;
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       const int jm = (16 * m) / G;
       if (qd / GQ == jm % VGB) {  // this lane owns the columns of m-block m's value group
-        // row scales of the subnormal centered codes (2 (c - cbar) 2^-24 on row r)
-        constexpr float kORowLo = 8388608.0f, kORowHi = VB == 2 ? 2097152.0f : 524288.0f;  // 2^23, 2^21 / 2^19
         o[16 * m + r] = (O[m][0] + O[m][1]) * kORowLo;
         o[16 * m + r + 8] = (O[m][2] + O[m][3]) * kORowHi;
       }
     }
-    if (r == 0 && qd < GQ) {
-      cw[h_d * kCm] = m_run;
-      cw[h_d * kCm + 1] = l_run;
-    }
   }
-  if (qd == 0 && !lo_half && col_head < gq) {
+  if (h_d < gq && r == 0 && qd < GQ) {
+    cw[h_d * kCm] = m_run;
+    cw[h_d * kCm + 1] = l_run;
+  }
+  if (qd == 0 && (PV1 || !lo_half) && pv_head < gq) {
 #pragma unroll
     for (int nb = 0; nb < NBV; ++nb) {
-      const int j = nb * VGB + col_off;
-      if (j < VPT) zb[(warp * 4 + col_head) * 8 + j] = zacc[nb];
+      const int j = nb * VGB + pv_off;
+      if (j < VPT) zb[(warp * 4 + pv_head) * 8 + j] = zacc[nb];
     }
   }
   __syncwarp();
