@@ -37,7 +37,7 @@ def gpu_config(w: inputs.Workload, layout: int = 1, sink: int = 0, rope: float =
 
 
 @dataclass
-class GpuRun:
+class DeviceRun:
     cfg: object
     cache: object
     out: torch.Tensor  # fp16 [B][Hq][128] on the device
@@ -49,7 +49,7 @@ class GpuRun:
 
 def run_gpu(w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarray, q: torch.Tensor,
             appends: int = 0, sm_scale: Optional[float] = None, layout: int = 1, decode: bool = True,
-            sink: int = 0, rope: float = 0.0, outliers: int = 0) -> GpuRun:
+            sink: int = 0, rope: float = 0.0, outliers: int = 0) -> DeviceRun:
     """Prefill (k, v on the device), `appends` streaming appends, one decode (unless decode=False)."""
     import bit_kv_cache_prefill_b200 as kvq
 
@@ -64,7 +64,7 @@ def run_gpu(w: inputs.Workload, k: torch.Tensor, v: torch.Tensor, lens: np.ndarr
         ws = torch.empty(kvq.kvq_decode_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
         kvq.kvq_decode_attention(cfg, cache, q.cuda(), out, sm_scale or 1 / math.sqrt(128), ws)
     torch.cuda.synchronize()
-    return GpuRun(cfg, cache, out, lens + appends, layout, sink, outliers)
+    return DeviceRun(cfg, cache, out, lens + appends, layout, sink, outliers)
 
 
 def code_shapes(w: inputs.Workload, layout: int):
@@ -74,7 +74,7 @@ def code_shapes(w: inputs.Workload, layout: int):
     return (B, H, cap // 16, 64 * w.key_bits), (B, H, cap // 16, 64 * w.value_bits)
 
 
-def gpu_views(w: inputs.Workload, run: GpuRun) -> Dict[str, np.ndarray]:
+def gpu_views(w: inputs.Workload, run: DeviceRun) -> Dict[str, np.ndarray]:
     """GPU cache buffers as numpy arrays with the oracle's shapes."""
     B, H, cap, G = w.batch, w.num_kv_heads, capacity(w, run.layout), w.group_size
     ring = w.residual + G + run.sink  # ring slots, then the sink row

@@ -51,7 +51,7 @@ def test_pinned_host_lengths_prefill_then_appends(oracle_mod, appends):
     assert (cache.seq_len_host == lens + appends).all()
     assert (cache.seq_len_dev.cpu().numpy() == lens + appends).all()
     oc, ref = H.oracle_full(oracle_mod, w.scaled(appends=appends), k, v, lens, q, appends=appends)
-    run = H.GpuRun(cfg, cache, out, lens + appends)
+    run = H.DeviceRun(cfg, cache, out, lens + appends)
     gv = H.gpu_views(w.scaled(appends=appends), run)
     for b in range(w.batch):
         for h in range(w.num_kv_heads):
@@ -77,7 +77,7 @@ def test_more_sequences_than_one_length_chunk(oracle_mod):
     torch.cuda.synchronize()
     assert (cache.seq_len_dev.cpu().numpy() == lens + appends).all()
     oc, _ = H.oracle_full(oracle_mod, w.scaled(appends=appends), k, v, lens, inputs.query(w), appends=appends)
-    run = H.GpuRun(cfg, cache, torch.empty(0), lens + appends)
+    run = H.DeviceRun(cfg, cache, torch.empty(0), lens + appends)
     gv = H.gpu_views(w.scaled(appends=appends), run)
     for b in range(w.batch):
         H.compare_unit_cache(w, gv, b, 0, oc, b, 0, int(lens[b]) + appends)
